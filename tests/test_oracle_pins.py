@@ -1,0 +1,416 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each check relies on something the pages or mathematics fix: exact integer
+arithmetic, a brute-force loop written independently on tiny inputs, textbook
+values of the normal distribution, closed forms (prefix mean, identity
+weights), and central finite differences for every backward.  The last group
+plants plausible mistakes in a copy of the oracle and shows that some pin
+fails for each of them.
+
+Partition identities come from "图解Transformer并行计算：从矩阵乘法切分到
+Megatron架构设计" (§1.1 row split = sum of partials, §1.2 column split =
+concatenation, §2.1 GeLU per column shard, §2.2 and §3.2 mirror rule), and
+the split-then-gather round trip and divisibility errors from "5.1 Tensor并行
+与算子拆分" §1.1.
+"""
+import math
+import os
+import types
+
+import numpy as np
+import pytest
+
+from oracle import tp_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _int_mat(shape, seed, lo=-3, hi=3):
+    return _rng(seed).integers(lo, hi + 1, size=shape).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Independent brute-force routines (pure Python loops, math module only)
+# ---------------------------------------------------------------------------
+
+def bf_matmul_int(X, W):
+    """Exact integer product with Python ints."""
+    M, K = len(X), len(X[0])
+    N = len(W[0])
+    return [[sum(int(X[i][k]) * int(W[k][j]) for k in range(K)) for j in range(N)]
+            for i in range(M)]
+
+
+def bf_phi_cdf(x):
+    return 0.5 * math.erfc(-x / math.sqrt(2.0))
+
+
+def bf_mlp(X, A, bA, B, bB):
+    """Loop MLP: Z[r][c] = sum_j GeLU(sum_k X[r][k] A[k][j] + bA[j]) B[j][c] + bB[c]."""
+    M, h = X.shape
+    f = A.shape[1]
+    Z = np.zeros((M, B.shape[1]))
+    for r in range(M):
+        Hrow = []
+        for j in range(f):
+            y = bA[j]
+            for k in range(h):
+                y += X[r, k] * A[k, j]
+            Hrow.append(y * bf_phi_cdf(y))
+        for c in range(B.shape[1]):
+            z = bB[c]
+            for j in range(f):
+                z += Hrow[j] * B[j, c]
+            Z[r, c] = z
+    return Z
+
+
+def bf_attention(Xb, Wqkv, Wo, heads, causal):
+    """Loop multi-head attention for one sequence, indexing [Wq | Wk | Wv] by hand."""
+    s, h = Xb.shape
+    d = h // heads
+    qkv = [[sum(Xb[r, k] * Wqkv[k, c] for k in range(h)) for c in range(3 * h)]
+           for r in range(s)]
+    Ocat = [[0.0] * h for _ in range(s)]
+    lse = [[0.0] * s for _ in range(heads)]
+    for j in range(heads):
+        for r in range(s):
+            scores = []
+            for c in range(s):
+                if causal and c > r:
+                    continue
+                dot = sum(qkv[r][j * d + e] * qkv[c][h + j * d + e] for e in range(d))
+                scores.append((c, dot / math.sqrt(d)))
+            mx = max(v for _, v in scores)
+            w = [(c, math.exp(v - mx)) for c, v in scores]
+            den = sum(v for _, v in w)
+            lse[j][r] = mx + math.log(den)
+            for e in range(d):
+                Ocat[r][j * d + e] = sum(p * qkv[c][2 * h + j * d + e] for c, p in w) / den
+    Z = [[sum(Ocat[r][k] * Wo[k, c] for k in range(h)) for c in range(h)] for r in range(s)]
+    return np.array(Z), np.array(Ocat), np.array(lse)
+
+
+# ---------------------------------------------------------------------------
+# Pin checks, written as functions of an oracle module so that the planted-
+# mistake tests can run them against a broken copy.
+# ---------------------------------------------------------------------------
+
+def check_gelu_table(o):
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "normal_cdf_pdf.txt"))
+            if l.strip() and not l.startswith("#")]
+    for x, cdf, pdf in ((float(a), float(b), float(c)) for a, b, c in rows):
+        assert abs(float(o.gelu(np.array([x]))[0]) - x * cdf) <= 1e-15 * max(1.0, abs(x))
+        assert abs(float(o.gelu_prime(np.array([x]))[0]) - (cdf + x * pdf)) <= 2e-15
+
+
+def check_linear_exact(o):
+    X, W = _int_mat((7, 24), 1), _int_mat((24, 16), 2)
+    b = _int_mat((16,), 3)
+    ref = np.array(bf_matmul_int(X.tolist(), W.tolist()), dtype=np.float64) + b
+    assert np.array_equal(o.linear(X, W, b), ref)
+    for t in (1, 2, 4, 8):
+        assert np.array_equal(o.linear_col_parallel(X, W, b, t), ref)
+        assert np.array_equal(o.linear_row_parallel(X, W, b, t), ref)
+    Ws = _int_mat((24, 24), 4)  # square weight: a transposed operand would go unnoticed otherwise
+    ref = np.array(bf_matmul_int(X.tolist(), Ws.tolist()), dtype=np.float64)
+    assert np.array_equal(o.linear(X, Ws), ref)
+
+
+def check_mlp_bruteforce(o):
+    r = _rng(11)
+    X = r.standard_normal((3, 4))
+    A, B = r.standard_normal((4, 8)) * 0.5, r.standard_normal((8, 4)) * 0.5
+    bA, bB = r.standard_normal(8) * 0.1, r.standard_normal(4) * 0.1
+    ref = bf_mlp(X, A, bA, B, bB)
+    got = o.mlp_fwd(X, A, bA, B, bB)["Z"]
+    assert np.max(np.abs(got - ref)) < 1e-13
+    for t in (1, 2, 4):
+        assert np.max(np.abs(o.mlp_fwd_parallel(X, A, bA, B, bB, t)["Z"] - ref)) < 1e-13
+
+
+def _fd_grad(fun, P, eps=1e-6):
+    g = np.zeros_like(P)
+    it = np.nditer(P, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        old = P[i]
+        P[i] = old + eps
+        up = fun()
+        P[i] = old - eps
+        dn = fun()
+        P[i] = old
+        g[i] = (up - dn) / (2 * eps)
+    return g
+
+
+def check_mlp_bwd_fd(o):
+    r = _rng(12)
+    X = r.standard_normal((3, 4))
+    A, B = r.standard_normal((4, 8)) * 0.7, r.standard_normal((8, 4)) * 0.7
+    bA, bB = r.standard_normal(8) * 0.1, r.standard_normal(4) * 0.1
+    G = r.standard_normal((3, 4))  # L = <G, Z>, so dZ = G
+    loss = lambda: float(np.sum(G * o.mlp_fwd(X, A, bA, B, bB)["Z"]))
+    g = o.mlp_bwd(X, A, bA, B, G)
+    for name, P in (("dX", X), ("dA", A), ("dbA", bA), ("dB", B), ("dbB", bB)):
+        fd = _fd_grad(loss, P)
+        assert np.max(np.abs(g[name] - fd)) < 1e-7, name
+    for t in (1, 2, 4):
+        gp = o.mlp_bwd_parallel(X, A, bA, B, G, t)
+        for name in ("dX", "dA", "dbA", "dB", "dbB"):
+            assert np.max(np.abs(gp[name] - g[name])) < 1e-12, (name, t)
+
+
+def check_attention_bruteforce(o):
+    r = _rng(13)
+    b, s, h, heads = 2, 4, 8, 2
+    X = r.standard_normal((b * s, h))
+    Wqkv, Wo = r.standard_normal((h, 3 * h)) * 0.5, r.standard_normal((h, h)) * 0.5
+    for causal in (True, False):
+        got = o.attn_fwd(X, Wqkv, Wo, b, s, heads, causal)
+        for bi in range(b):
+            Z, Ocat, lse = bf_attention(X[bi * s:(bi + 1) * s], Wqkv, Wo, heads, causal)
+            assert np.max(np.abs(got["Z"][bi * s:(bi + 1) * s] - Z)) < 1e-12
+            assert np.max(np.abs(got["O"][bi * s:(bi + 1) * s] - Ocat)) < 1e-12
+            assert np.max(np.abs(got["LSE"][bi] - lse)) < 1e-12
+        for t in (1, 2):
+            gp = o.attn_fwd_parallel(X, Wqkv, Wo, b, s, heads, t, causal)
+            assert np.max(np.abs(gp["Z"] - got["Z"])) < 1e-12
+
+
+def check_attention_closed_forms(o):
+    r = _rng(14)
+    s, d = 9, 8
+    V = r.standard_normal((s, d))
+    K = r.standard_normal((s, d))
+    # Q = 0: every unmasked score is 0, so row r of O is the mean of V[0..r].
+    Oq0, P, lse = o.attention_core(np.zeros((s, d)), K, V, causal=True)
+    prefix_mean = np.cumsum(V, axis=0) / np.arange(1, s + 1)[:, None]
+    assert np.max(np.abs(Oq0 - prefix_mean)) < 1e-14
+    assert np.allclose(lse, np.log(np.arange(1, s + 1)), rtol=0, atol=1e-14)
+    # Row 0 sees only key 0, so O[0] = V[0] exactly; rows of P sum to 1; masked part is 0.
+    Q = r.standard_normal((s, d))
+    Oc, P, _ = o.attention_core(Q, K, V, causal=True)
+    assert np.array_equal(Oc[0], V[0])
+    assert np.max(np.abs(P.sum(axis=1) - 1.0)) < 1e-15
+    assert np.all(np.triu(P, 1) == 0.0)
+
+
+def check_attention_bwd_fd(o):
+    r = _rng(15)
+    b, s, h, heads = 2, 4, 8, 2
+    X = r.standard_normal((b * s, h))
+    Wqkv, Wo = r.standard_normal((h, 3 * h)) * 0.5, r.standard_normal((h, h)) * 0.5
+    G = r.standard_normal((b * s, h))
+    loss = lambda: float(np.sum(G * o.attn_fwd(X, Wqkv, Wo, b, s, heads, True)["Z"]))
+    g = o.attn_bwd(X, Wqkv, Wo, G, b, s, heads, True)
+    for name, P in (("dX", X), ("dWqkv", Wqkv), ("dWo", Wo)):
+        fd = _fd_grad(loss, P)
+        assert np.max(np.abs(g[name] - fd)) < 1e-7, name
+    for t in (1, 2):
+        gp = o.attn_bwd_parallel(X, Wqkv, Wo, G, b, s, heads, t, True)
+        for name in ("dX", "dWqkv", "dWo"):
+            assert np.max(np.abs(gp[name] - g[name])) < 1e-12, (name, t)
+
+
+PINS = [check_gelu_table, check_linear_exact, check_mlp_bruteforce, check_mlp_bwd_fd,
+        check_attention_bruteforce, check_attention_closed_forms, check_attention_bwd_fd]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
+def test_oracle_pin(pin):
+    pin(O)
+
+
+# ---------------------------------------------------------------------------
+# Slicing and partition identities (bit-exact)
+# ---------------------------------------------------------------------------
+
+def test_split_gather_roundtrip_and_contiguity():
+    W = _rng(20).standard_normal((32, 48))
+    for t in (1, 2, 4, 8):
+        cs, rs = O.split_cols(W, t), O.split_rows(W, t)
+        assert np.array_equal(np.concatenate(cs, axis=1), W)
+        assert np.array_equal(np.concatenate(rs, axis=0), W)
+        for i in range(t):
+            assert np.array_equal(cs[i], W[:, i * 48 // t:(i + 1) * 48 // t])
+            assert np.array_equal(rs[i], W[i * 32 // t:(i + 1) * 32 // t])
+
+
+def test_split_rejects_non_divisible():
+    W = np.zeros((12, 10))
+    with pytest.raises(ValueError):
+        O.split_cols(W, 4)
+    with pytest.raises(ValueError):
+        O.split_rows(W, 5)
+    with pytest.raises(ValueError):
+        O.group_columns(64, 6, 4, 0)
+
+
+def test_row_partials_sum_exactly_on_integers():
+    X, W = _int_mat((16, 64), 21), _int_mat((64, 24), 22)
+    ref = np.array(bf_matmul_int(X.tolist(), W.tolist()), dtype=np.float64)
+    for t in (1, 2, 4, 8):
+        Z, parts = O.linear_row_parallel(X, W, None, t, return_partials=True)
+        assert np.array_equal(Z, ref)
+        for i, p in enumerate(parts):
+            k = 64 // t
+            sub = np.array(bf_matmul_int(X[:, i * k:(i + 1) * k].tolist(),
+                                         W[i * k:(i + 1) * k].tolist()), dtype=np.float64)
+            assert np.array_equal(p, sub)
+
+
+def test_gelu_per_shard_equals_gelu_on_full():
+    X, A = _int_mat((8, 16), 23), _int_mat((16, 32), 24) / 4.0  # exact dyadic values
+    full = O.mlp_fwd(X, A, None, np.zeros((32, 16)), None)
+    for t in (1, 2, 4, 8):
+        par = O.mlp_fwd_parallel(X, A, None, np.zeros((32, 16)), None, t)
+        assert np.array_equal(par["Y"], full["Y"])
+        assert np.array_equal(par["H"], full["H"])
+
+
+def test_gelu_identities():
+    x = np.linspace(-6, 6, 1001)
+    assert np.max(np.abs(O.gelu(x) - O.gelu(-x) - x)) < 1e-14
+    assert np.max(np.abs(O.gelu_prime(x) + O.gelu_prime(-x) - 1.0)) < 1e-14
+    assert O.gelu(np.array([0.0]))[0] == 0.0
+    assert abs(O.gelu(np.array([10.0]))[0] - 10.0) < 1e-20 * 10 + 1e-15
+    fd = (O.gelu(x + 1e-6) - O.gelu(x - 1e-6)) / 2e-6
+    assert np.max(np.abs(fd - O.gelu_prime(x))) < 1e-8
+
+
+def test_mlp_identity_weights_closed_form():
+    X = _rng(25).standard_normal((5, 6))
+    I = np.eye(6)
+    assert np.max(np.abs(O.mlp_fwd(X, I, None, I, None)["Z"] - X * np.vectorize(bf_phi_cdf)(X))) < 1e-15
+
+
+def test_cross_t_agreement_mlp_and_attention():
+    r = _rng(26)
+    X = r.standard_normal((8, 16))
+    A, B = r.standard_normal((16, 64)) * 0.3, r.standard_normal((64, 16)) * 0.3
+    bA, bB = r.standard_normal(64) * 0.1, r.standard_normal(16) * 0.1
+    ref = O.mlp_fwd(X, A, bA, B, bB)["Z"]
+    for t in (1, 2, 4, 8):
+        assert np.max(np.abs(O.mlp_fwd_parallel(X, A, bA, B, bB, t)["Z"] - ref)) < 1e-13
+    Xa = r.standard_normal((2 * 5, 16))
+    Wqkv, Wo = r.standard_normal((16, 48)) * 0.3, r.standard_normal((16, 16)) * 0.3
+    ref = O.attn_fwd(Xa, Wqkv, Wo, 2, 5, 8)["Z"]
+    for t in (1, 2, 4, 8):
+        assert np.max(np.abs(O.attn_fwd_parallel(Xa, Wqkv, Wo, 2, 5, 8, t)["Z"] - ref)) < 1e-13
+
+
+def test_group_columns_layout():
+    h, heads, t = 16, 4, 2  # d = 4, two heads per group
+    g1 = O.group_columns(h, heads, t, 1)
+    assert g1.tolist() == [8, 9, 10, 11, 12, 13, 14, 15,
+                           24, 25, 26, 27, 28, 29, 30, 31,
+                           40, 41, 42, 43, 44, 45, 46, 47]
+
+
+def test_error_measures():
+    ref = np.array([1.0, -4.0, 2.0])
+    got = np.array([1.5, -4.0, 2.0])
+    assert O.max_rel_error(got, ref) == 0.5 / 4.0
+    assert abs(O.normwise_error(got, ref) - 0.5 / math.sqrt(21.0)) < 1e-16
+
+
+# ---------------------------------------------------------------------------
+# Planted mistakes: each broken copy of the oracle must fail at least one pin
+# ---------------------------------------------------------------------------
+
+def _mutant(**overrides):
+    m = types.ModuleType("oracle_mutant")
+    m.__dict__.update({k: getattr(O, k) for k in dir(O) if not k.startswith("__")})
+    m.__dict__.update(overrides)
+    # Re-bind the module-level functions so they see the overrides.
+    for name in O.__all__:
+        if name in overrides:
+            continue
+        fn = getattr(O, name)
+        if callable(fn) and hasattr(fn, "__code__"):
+            m.__dict__[name] = types.FunctionType(fn.__code__, m.__dict__, fn.__name__,
+                                                  fn.__defaults__, fn.__closure__)
+    return m
+
+
+def _tanh_gelu(x):
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1 + np.tanh(math.sqrt(2 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def _bwd_without_gelu_prime(X, A, bA, B, dZ, Y=None):
+    X, A, B, dZ = (np.asarray(v, dtype=np.float64) for v in (X, A, B, dZ))
+    Y = X @ A + (bA if bA is not None else 0.0)
+    H = O.gelu(Y)
+    dY = dZ @ B.T  # mistake: the GeLU' factor is dropped
+    return {"dX": dY @ A.T, "dA": X.T @ dY, "dbA": dY.sum(0), "dB": H.T @ dZ,
+            "dbB": dZ.sum(0), "dY": dY}
+
+
+def _core_no_scale(Q, K, V, causal=True):
+    Q, K, V = (np.asarray(v, dtype=np.float64) for v in (Q, K, V))
+    S = Q @ K.T  # mistake: no 1/sqrt(d)
+    if causal:
+        S = np.where(np.arange(S.shape[1])[None, :] > np.arange(S.shape[0])[:, None], -np.inf, S)
+    m = S.max(1, keepdims=True)
+    E = np.exp(S - m)
+    return (E / E.sum(1, keepdims=True)) @ V, E / E.sum(1, keepdims=True), (m + np.log(E.sum(1, keepdims=True)))[:, 0]
+
+
+def _core_mask_off_by_one(Q, K, V, causal=True):
+    Q, K, V = (np.asarray(v, dtype=np.float64) for v in (Q, K, V))
+    S = Q @ K.T / math.sqrt(Q.shape[1])
+    if causal:  # mistake: also hides the diagonal key except on row 0
+        r, c = np.arange(S.shape[0])[:, None], np.arange(S.shape[1])[None, :]
+        S = np.where((c >= r) & (r > 0), -np.inf, S)
+    m = S.max(1, keepdims=True)
+    E = np.exp(S - m)
+    return (E / E.sum(1, keepdims=True)) @ V, E / E.sum(1, keepdims=True), (m + np.log(E.sum(1, keepdims=True)))[:, 0]
+
+
+def _row_parallel_bias_per_shard(X, W, bias, t, return_partials=False):
+    Xs, Ws = O.split_cols(X, t), O.split_rows(W, t)
+    parts = [Xi @ Wi + (bias if bias is not None else 0.0) for Xi, Wi in zip(Xs, Ws)]
+    Z = sum(parts[1:], parts[0].copy())
+    return (Z, parts) if return_partials else Z
+
+
+def _transposed_linear(X, W, bias=None):
+    X, W = np.asarray(X, dtype=np.float64), np.asarray(W, dtype=np.float64)
+    Y = X @ (W.T if W.shape[0] == W.shape[1] else W)  # mistake only visible for square W
+    return Y + (bias if bias is not None else 0.0)
+
+
+def _head_columns_swapped(h, heads, j):
+    d = h // heads
+    base = np.arange(j * d, (j + 1) * d)
+    other = np.arange((heads - 1 - j) * d, (heads - j) * d)
+    return {"q": base, "k": h + other, "v": 2 * h + base}  # mistake: k of the mirrored head
+
+
+MUTANTS = {
+    "wrong head columns": dict(head_columns=_head_columns_swapped),
+    "tanh GeLU": dict(gelu=_tanh_gelu),
+    "GeLU' dropped": dict(mlp_bwd=_bwd_without_gelu_prime),
+    "no 1/sqrt(d)": dict(attention_core=_core_no_scale),
+    "mask off by one": dict(attention_core=_core_mask_off_by_one),
+    "row bias per shard": dict(linear_row_parallel=_row_parallel_bias_per_shard),
+    "transposed square weight": dict(linear=_transposed_linear),
+}
+
+
+@pytest.mark.parametrize("name", list(MUTANTS))
+def test_planted_mistake_is_caught(name):
+    m = _mutant(**MUTANTS[name])
+    failures = 0
+    for pin in PINS:
+        try:
+            pin(m)
+        except AssertionError:
+            failures += 1
+    assert failures >= 1, f"no pin caught the planted mistake '{name}'"
