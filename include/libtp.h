@@ -1,0 +1,194 @@
+/*
+ * libtp — the Megatron-style partitioned Transformer layer on one B200.
+ *
+ * The layer is split into t *logical* shards that all live on one GPU.  What
+ * the pages do with an AllReduce across GPUs (the sum of row-shard partials)
+ * happens here inside the kernel: the partial products of every shard are
+ * accumulated in tensor memory, shard after shard, and never written to HBM.
+ *
+ * Sources (page title, then section):
+ *   [P3] "图解Transformer并行计算：从矩阵乘法切分到Megatron架构设计"
+ *        §1.1 row split, §1.2 column split, §2.1/§2.2 MLP, §3.1/§3.2 attention.
+ *   [P2] PyTorch tensor-parallel tutorial (page title "企业官网建设流程全解析"),
+ *        §2.2 ParallelAttention, §3.2 ColumnParallelLinear, §3.3 the block.
+ *   [P4] "5.1 Tensor并行与算子拆分" §1.1 tensor_parallel_split (divisibility).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every tensor is row-major and dense; a [rows, cols] tensor has leading
+ *   dimension cols.  Weights are stored [in, out] ([P3] §1: W is [h, h']).
+ * - Every pointer is a DEVICE pointer owned by the caller; the library keeps
+ *   no reference after the call returns and allocates no device memory.
+ *   Scratch space comes from the caller's workspace `ws` of `ws_bytes`
+ *   bytes, sized with tp_workspace_size().
+ * - Each call validates its arguments on the host, synchronously, before any
+ *   launch, and then enqueues its kernels on `stream` (a cudaStream_t; NULL is
+ *   the legacy default stream) and returns without waiting.
+ * - Alignment: every pointer must be 16-byte aligned and every row length
+ *   (number of columns) a multiple of 8 elements, otherwise TP_ERR_ALIGN.
+ * - Shard i of a column split owns columns [i*n/t, (i+1)*n/t); shard i of a
+ *   row split owns rows [i*k/t, (i+1)*k/t) ([P4] §1.1: contiguous, equal
+ *   shards; a size that t does not divide is an error, TP_ERR_SHAPE).
+ *   t must be in [1, 64].
+ * - bf16 work multiplies in bf16 and accumulates in fp32 on the tensor cores
+ *   (tcgen05); outputs are rounded to the output type round-to-nearest-even.
+ *   fp32 work runs on the CUDA cores in fp32.
+ * - No C++ exception crosses this interface.  A non-TP_OK status leaves a
+ *   message for tp_last_error().  TP_ERR_CUDA reports a launch error.  Errors
+ *   that kernels detect while running (a bounded wait that expired) are
+ *   recorded in a device status word, read by tp_device_status().
+ */
+#ifndef LIBTP_H_
+#define LIBTP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tp_status {
+  TP_OK = 0,
+  TP_ERR_NULL = 1,         /* a required pointer is NULL                         */
+  TP_ERR_SHAPE = 2,        /* a size <= 0, or t / heads does not divide a size   */
+  TP_ERR_ALIGN = 3,        /* pointer not 16B aligned or row length % 8 != 0     */
+  TP_ERR_DTYPE = 4,        /* unknown dtype or a disallowed dtype combination    */
+  TP_ERR_UNSUPPORTED = 5,  /* valid request outside what is implemented          */
+  TP_ERR_CUDA = 6,         /* CUDA runtime error (launch or query)               */
+  TP_ERR_KERNEL = 7,       /* a kernel recorded an error in the status word      */
+  TP_ERR_WORKSPACE = 8     /* ws is NULL or smaller than tp_workspace_size()     */
+} tp_status;
+
+typedef enum tp_dtype { TP_F32 = 0, TP_BF16 = 1 } tp_dtype;
+
+typedef enum tp_op {
+  TP_OP_MLP_FWD = 0,
+  TP_OP_MLP_BWD = 1,
+  TP_OP_ATTN_FWD = 2,
+  TP_OP_ATTN_BWD = 3
+} tp_op;
+
+/*
+ * Column-parallel linear ([P3] §1.2; [P2] §3.2 ColumnParallelLinear):
+ * W = [W_0 | ... | W_{t-1}] split on its output columns, X whole,
+ * Y_i = X @ W_i + bias_i, Y = concat_i Y_i (the All-Gather is the layout:
+ * shard i's tiles write columns [i*N/t, (i+1)*N/t) of Y).
+ *   X    [M, K]  dtype          W [K, N] dtype          bias [N] dtype or NULL
+ *   Y    shard <  0: [M, N] out_dtype, every shard
+ *        shard >= 0: [M, N/t] out_dtype, shard `shard` only (its columns)
+ *   dtype TP_BF16 allows out_dtype TP_BF16 or TP_F32; dtype TP_F32 needs TP_F32.
+ * Errors: NULL X/W/Y; M, K, N <= 0; N % t; shard >= t; alignment; dtypes.
+ */
+tp_status tp_linear_col(const void* X, const void* W, const void* bias, void* Y,
+                        int64_t M, int64_t K, int64_t N, int t, int shard,
+                        tp_dtype dtype, tp_dtype out_dtype, void* stream);
+
+/*
+ * Row-parallel linear ([P3] §1.1): W = [W_0; ...; W_{t-1}] split on its
+ * input rows, X split on its last dimension (the library slices the full X
+ * itself), Z = sum_i X_i @ W_i + bias.  The partials are summed in the
+ * accumulator, shard 0 first; none is written to memory.  The bias is added
+ * once, after the sum.
+ *   X [M, K] dtype; W [K, N] dtype; bias [N] dtype or NULL; Z [M, N] out_dtype.
+ *   shard >= 0: Z receives the partial X_shard @ W_shard alone (the bias is
+ *   added to shard 0's partial only, so that the t partials sum to the full
+ *   result); use out_dtype TP_F32 to keep partials unrounded.
+ * Errors: as tp_linear_col, with K % t instead of N % t.
+ */
+tp_status tp_linear_row(const void* X, const void* W, const void* bias, void* Z,
+                        int64_t M, int64_t K, int64_t N, int t, int shard,
+                        tp_dtype dtype, tp_dtype out_dtype, void* stream);
+
+/*
+ * Partitioned MLP forward ([P3] §2.1 steps 1-3, §2.2 MLP_forward_TP):
+ *   shard i: Y_i = X @ A_i + bA_i;  H_i = GeLU(Y_i)  (exact erf GeLU, [P2] §3.3);
+ *   Z = sum_i H_i @ B_i + bB   (A split by columns, B by rows, f = 4h typically).
+ *   X [M, h]; A [h, f]; bA [f] or NULL; B [f, h]; bB [h] or NULL; Z [M, h];
+ *   Ysave [M, f] or NULL: receives the pre-activation Y for the backward.
+ *   All tensors in `dtype`.  H lives in the workspace.
+ * Errors: NULL X/A/B/Z/ws; f % t; alignment; TP_ERR_WORKSPACE.
+ */
+tp_status tp_mlp_fwd(const void* X, const void* A, const void* bA, const void* B,
+                     const void* bB, void* Z, void* Ysave, int64_t M, int64_t h,
+                     int64_t f, int t, tp_dtype dtype, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/*
+ * Partitioned MLP backward, the pages' mirror rule ([P3] §2.2):
+ *   dY_i = (dZ @ B_i^T) * GeLU'(Y_i);  dB_i = H_i^T @ dZ;  dA_i = X^T @ dY_i
+ *   (weight gradients per shard, no exchange);  dX = sum_i dY_i @ A_i^T (the
+ *   partials summed in the accumulator);  dbA = colsum(dY);  dbB = colsum(dZ).
+ *   Ysave: the forward's pre-activation, or NULL to recompute it from X, A, bA.
+ *   Outputs dX [M, h], dA [h, f], dB [f, h] in `dtype`; dbA [f], dbB [h] in
+ *   `dtype`, each computed only when its pointer is not NULL.
+ * Errors: NULL X/A/B/dZ/dX/dA/dB/ws; f % t; alignment; TP_ERR_WORKSPACE.
+ */
+tp_status tp_mlp_bwd(const void* X, const void* A, const void* bA, const void* B,
+                     const void* Ysave, const void* dZ, void* dX, void* dA, void* dbA,
+                     void* dB, void* dbB, int64_t M, int64_t h, int64_t f, int t,
+                     tp_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Head-wise partitioned attention forward ([P3] §3.1, §3.2 forward steps 1-3;
+ * [P2] §2.2 ParallelAttention):
+ *   Wqkv = [Wq | Wk | Wv] ([h, 3h]); head j owns columns [j*d, (j+1)*d) of
+ *   each block, d = h/heads; head group g owns heads [g*heads/t, (g+1)*heads/t)
+ *   and so three column ranges of Wqkv.  QKV_g = X @ Wqkv_g;  per head
+ *   O_j = softmax(Q_j K_j^T / sqrt(d) + mask) V_j with the causal mask hiding
+ *   key c from query r when c > r ([P4] masked_fill(mask == 0, -inf));
+ *   Z = sum_g O_g @ Wo_g with Wo split by rows (no concatenation before Wo).
+ *   X [M = b*s, h]; Wqkv [h, 3h]; Wo [h, h]; Z [M, h]; all bf16.
+ *   QKVsave [M, 3h] bf16 or NULL; Osave [M, h] bf16 or NULL (heads in column
+ *   order); LSEsave [b, heads, s] fp32 or NULL: natural-log softmax
+ *   denominators of the scaled, masked scores.
+ *   d must be 128.  dtype must be TP_BF16 (else TP_ERR_UNSUPPORTED).
+ * Errors: NULL X/Wqkv/Wo/Z/ws; heads % t; h % heads; s < 1; TP_ERR_WORKSPACE.
+ */
+tp_status tp_attn_fwd(const void* X, const void* Wqkv, const void* Wo, void* Z,
+                      void* QKVsave, void* Osave, void* LSEsave, int64_t b, int64_t s,
+                      int64_t h, int heads, int t, int causal, tp_dtype dtype, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/*
+ * Head-wise attention backward ([P3] §3.2 backward steps 1-3):
+ *   dO_g = dZ @ Wo_g^T;  dWo_g = O_g^T @ dZ;  per head the softmax backward
+ *   gives dQ, dK, dV;  dWqkv_g = X^T @ dQKV_g;  dX = sum_g dQKV_g @ Wqkv_g^T
+ *   with the group partials summed in the accumulator, group 0 first.
+ *   Osave, LSEsave: from tp_attn_fwd (required).  QKVsave: from tp_attn_fwd,
+ *   or NULL to recompute QKV = X @ Wqkv.  Outputs dX [M, h], dWqkv [h, 3h],
+ *   dWo [h, h], all bf16.
+ * Errors: as tp_attn_fwd, plus NULL Osave/LSEsave/dZ/dX/dWqkv/dWo.
+ */
+tp_status tp_attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* QKVsave,
+                      const void* Osave, const void* LSEsave, const void* dZ, void* dX,
+                      void* dWqkv, void* dWo, int64_t b, int64_t s, int64_t h, int heads,
+                      int t, int causal, tp_dtype dtype, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/*
+ * Workspace bytes that `op` needs for these sizes (M = b*s tokens; f is
+ * ignored by the attention ops, heads by the MLP ops).  Returns 0 for
+ * invalid arguments.  The size covers the worst case (recomputed Y / QKV).
+ */
+size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, int t,
+                         tp_dtype dtype);
+
+/* Message for the last non-TP_OK status returned on this host thread. */
+const char* tp_last_error(void);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device status word of the
+ * current device.  TP_OK, TP_ERR_KERNEL (a kernel gave up a bounded wait;
+ * the message names where) or TP_ERR_CUDA.
+ */
+tp_status tp_device_status(void* stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int tp_version(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* LIBTP_H_ */

@@ -1,0 +1,165 @@
+"""Python binding of libtp: argument marshalling only.
+
+Each function has the name of the C entry point it calls (see
+include/libtp.h), takes torch CUDA tensors (PyTorch supplies device memory
+and streams; nothing is computed here), derives the sizes from their shapes,
+passes raw device pointers, and raises TPError on a non-OK status.  There is
+no fallback: if libtp.so is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtp.so")
+
+TP_OK, TP_ERR_NULL, TP_ERR_SHAPE, TP_ERR_ALIGN, TP_ERR_DTYPE = 0, 1, 2, 3, 4
+TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_KERNEL, TP_ERR_WORKSPACE = 5, 6, 7, 8
+TP_F32, TP_BF16 = 0, 1
+TP_OP_MLP_FWD, TP_OP_MLP_BWD, TP_OP_ATTN_FWD, TP_OP_ATTN_BWD = 0, 1, 2, 3
+
+EXPORTS = ("tp_linear_col", "tp_linear_row", "tp_mlp_fwd", "tp_mlp_bwd", "tp_attn_fwd",
+           "tp_attn_bwd", "tp_workspace_size", "tp_last_error", "tp_device_status",
+           "tp_version")
+
+
+class TPError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"libtp status {status}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Loads libtp.so once and declares its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built: run "
+                           "`python -m megatron_tensor_transformer_logical_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    L.tp_linear_col.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, vp]
+    L.tp_linear_row.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, vp]
+    L.tp_mlp_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, sz, vp]
+    L.tp_mlp_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32,
+                             i32, vp, sz, vp]
+    L.tp_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32,
+                              vp, sz, vp]
+    L.tp_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32,
+                              i32, i32, vp, sz, vp]
+    L.tp_workspace_size.argtypes = [i32, i64, i64, i64, i32, i32, i32]
+    L.tp_workspace_size.restype = sz
+    L.tp_last_error.argtypes = []
+    L.tp_last_error.restype = ctypes.c_char_p
+    L.tp_device_status.argtypes = [vp]
+    L.tp_version.argtypes = []
+    for name in EXPORTS:
+        if name not in ("tp_workspace_size", "tp_last_error"):
+            getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("libtp takes dense row-major (contiguous) tensors")
+    return t.data_ptr()
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return TP_BF16
+    if t.dtype == torch.float32:
+        return TP_F32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _check(status: int) -> None:
+    if status != TP_OK:
+        raise TPError(status, load().tp_last_error().decode(errors="replace"))
+
+
+def tp_linear_col(X, W, bias, Y, t: int, shard: int = -1, stream=None) -> None:
+    M, K = X.shape
+    N = W.shape[1]
+    _check(load().tp_linear_col(_ptr(X), _ptr(W), _ptr(bias), _ptr(Y), M, K, N, t, shard,
+                                _dtype(X), _dtype(Y), _stream(stream)))
+
+
+def tp_linear_row(X, W, bias, Z, t: int, shard: int = -1, stream=None) -> None:
+    M, K = X.shape
+    N = W.shape[1]
+    _check(load().tp_linear_row(_ptr(X), _ptr(W), _ptr(bias), _ptr(Z), M, K, N, t, shard,
+                                _dtype(X), _dtype(Z), _stream(stream)))
+
+
+def tp_workspace_size(op: int, M: int, h: int, f: int, heads: int, t: int, dtype: int) -> int:
+    return int(load().tp_workspace_size(op, M, h, f, heads, t, dtype))
+
+
+def tp_mlp_fwd(X, A, bA, B, bB, Z, Ysave, t: int, ws, stream=None) -> None:
+    M, h = X.shape
+    f = A.shape[1]
+    _check(load().tp_mlp_fwd(_ptr(X), _ptr(A), _ptr(bA), _ptr(B), _ptr(bB), _ptr(Z),
+                             _ptr(Ysave), M, h, f, t, _dtype(X), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def tp_mlp_bwd(X, A, bA, B, Ysave, dZ, dX, dA, dbA, dB, dbB, t: int, ws, stream=None) -> None:
+    M, h = X.shape
+    f = A.shape[1]
+    _check(load().tp_mlp_bwd(_ptr(X), _ptr(A), _ptr(bA), _ptr(B), _ptr(Ysave), _ptr(dZ),
+                             _ptr(dX), _ptr(dA), _ptr(dbA), _ptr(dB), _ptr(dbB), M, h, f, t,
+                             _dtype(X), _ptr(ws), ws.numel() * ws.element_size(),
+                             _stream(stream)))
+
+
+def tp_attn_fwd(X, Wqkv, Wo, Z, QKVsave, Osave, LSEsave, b: int, s: int, heads: int, t: int,
+                causal: bool, ws, stream=None) -> None:
+    h = X.shape[1]
+    _check(load().tp_attn_fwd(_ptr(X), _ptr(Wqkv), _ptr(Wo), _ptr(Z), _ptr(QKVsave),
+                              _ptr(Osave), _ptr(LSEsave), b, s, h, heads, t, int(causal),
+                              _dtype(X), _ptr(ws), ws.numel() * ws.element_size(),
+                              _stream(stream)))
+
+
+def tp_attn_bwd(X, Wqkv, Wo, QKVsave, Osave, LSEsave, dZ, dX, dWqkv, dWo, b: int, s: int,
+                heads: int, t: int, causal: bool, ws, stream=None) -> None:
+    h = X.shape[1]
+    _check(load().tp_attn_bwd(_ptr(X), _ptr(Wqkv), _ptr(Wo), _ptr(QKVsave), _ptr(Osave),
+                              _ptr(LSEsave), _ptr(dZ), _ptr(dX), _ptr(dWqkv), _ptr(dWo), b, s,
+                              h, heads, t, int(causal), _dtype(X), _ptr(ws),
+                              ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def tp_device_status(stream=None) -> None:
+    _check(load().tp_device_status(_stream(stream)))
+
+
+def tp_version() -> int:
+    return int(load().tp_version())
+
+
+def workspace(op: int, M: int, h: int, f: int, heads: int, t: int, dtype: int,
+              device="cuda") -> torch.Tensor:
+    """A byte tensor of tp_workspace_size() bytes on `device`."""
+    n = tp_workspace_size(op, M, h, f, heads, t, dtype)
+    if n == 0:
+        raise TPError(TP_ERR_SHAPE, "invalid sizes for the workspace query")
+    return torch.empty(n, dtype=torch.uint8, device=device)

@@ -1,0 +1,563 @@
+// libtp C entry points: host-side validation, the shard planner (how each
+// partitioned operation of the pages maps onto kernel launches), workspace
+// carving and the device status word.  Nothing here computes on the host.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <exception>
+#include <mutex>
+#include <string>
+
+#include "../../include/libtp.h"
+#include "ptx_sm100.cuh"
+#include "tp_internal.h"
+
+namespace tp {
+
+namespace {
+thread_local std::string g_last_error;
+constexpr int kMaxDevices = 64;
+}  // namespace
+
+// Device status word: kernels that give up a bounded wait record a code here.
+__device__ int g_tp_status_word;
+
+tp_status fail(tp_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+tp_status cuda_fail(cudaError_t e, const char* where) {
+  g_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+  return TP_ERR_CUDA;
+}
+
+int* device_status_ptr() {
+  static int* ptrs[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_tp_status_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+int sm_count() {
+  static int counts[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
+namespace {
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t esize(tp_dtype d) { return d == TP_F32 ? 4 : 2; }
+
+// Bump allocator over the caller's workspace.
+struct Carve {
+  char* base;
+  size_t cap, off = 0;
+  Carve(void* b, size_t c) : base(static_cast<char*>(b)), cap(c) {}
+  void* take(size_t bytes) {
+    off = align_up(off, 256);
+    void* p = base + off;
+    off += bytes;
+    return p;
+  }
+};
+
+tp_status check_dtype(tp_dtype d) {
+  if (d != TP_F32 && d != TP_BF16) return fail(TP_ERR_DTYPE, "unknown dtype");
+  return TP_OK;
+}
+
+tp_status check_t(int t) {
+  if (t < 1 || t > 64) return fail(TP_ERR_SHAPE, "shard count t must be in [1, 64]");
+  return TP_OK;
+}
+
+tp_status check_ptrs_aligned(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (p != nullptr && !aligned16(p)) return fail(TP_ERR_ALIGN, "pointer not 16-byte aligned");
+  return TP_OK;
+}
+
+tp_status check_rows(std::initializer_list<int64_t> lens) {
+  for (int64_t n : lens)
+    if (n % 8 != 0) return fail(TP_ERR_ALIGN, "row length not a multiple of 8 elements");
+  return TP_OK;
+}
+
+inline tp_status run(const Gemm& g, bool f32, cudaStream_t s) {
+  return f32 ? launch_gemm_f32(g, s) : launch_gemm_bf16(g, s);
+}
+
+#define TP_TRY(expr)                   \
+  do {                                 \
+    tp_status _st = (expr);            \
+    if (_st != TP_OK) return _st;      \
+  } while (0)
+
+// ------------------------------------------------------------------ linear
+
+tp_status linear_common(const void* X, const void* W, const void* bias, void* Y, int64_t M,
+                        int64_t K, int64_t N, int t, int shard, tp_dtype dtype,
+                        tp_dtype out_dtype, bool col, cudaStream_t stream) {
+  if (X == nullptr || W == nullptr || Y == nullptr) return fail(TP_ERR_NULL, "X, W and Y are required");
+  TP_TRY(check_dtype(dtype));
+  TP_TRY(check_dtype(out_dtype));
+  if (dtype == TP_F32 && out_dtype != TP_F32)
+    return fail(TP_ERR_DTYPE, "fp32 inputs need an fp32 output");
+  if (M <= 0 || K <= 0 || N <= 0) return fail(TP_ERR_SHAPE, "M, K and N must be positive");
+  TP_TRY(check_t(t));
+  if (shard >= t) return fail(TP_ERR_SHAPE, "shard must be < t");
+  const int64_t split = col ? N : K;
+  if (split % t != 0)
+    return fail(TP_ERR_SHAPE, col ? "N must be divisible by t (column split)"
+                                  : "K must be divisible by t (row split)");
+  TP_TRY(check_ptrs_aligned({X, W, bias, Y}));
+  TP_TRY(check_rows({K, N}));
+  const int64_t part = split / t;
+  if (shard >= 0) TP_TRY(check_rows({part}));
+
+  const bool f32 = dtype == TP_F32;
+  const size_t es = esize(dtype);
+  Gemm g;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.a = {X, K, true};
+  g.b = {W, N, false};
+  g.epi = kEpiStore;
+  g.out = Y;
+  g.ldo = N;
+  g.out_f32 = out_dtype == TP_F32;
+  g.bias = bias;
+  if (col) {
+    if (shard < 0) {
+      g.n_shard = part;  // tiles of shard i cover columns [i*N/t, (i+1)*N/t) only
+    } else {
+      g.N = part;
+      g.b.ptr = static_cast<const char*>(W) + shard * part * es;
+      if (bias) g.bias = static_cast<const char*>(bias) + shard * part * es;
+      g.ldo = part;
+    }
+  } else if (shard >= 0) {
+    // Partial of row shard `shard`: X[:, K_i] @ W[K_i, :]; bias on shard 0 only.
+    g.K = part;
+    g.a.ptr = static_cast<const char*>(X) + shard * part * es;
+    g.b.ptr = static_cast<const char*>(W) + shard * part * N * es;
+    if (shard != 0) g.bias = nullptr;
+  }
+  return run(g, f32, stream);
+}
+
+// --------------------------------------------------------------------- MLP
+
+size_t mlp_fwd_ws(int64_t M, int64_t f, tp_dtype d) { return align_up(M * f * esize(d), 256) + 256; }
+
+size_t mlp_bwd_ws(int64_t M, int64_t h, int64_t f, tp_dtype d) {
+  const size_t mf = align_up(M * f * esize(d), 256);
+  size_t cs = colsum_scratch_bytes(M, f);
+  const size_t cs2 = colsum_scratch_bytes(M, h);
+  if (cs2 > cs) cs = cs2;
+  return 3 * mf + align_up(cs, 256) + 1024;
+}
+
+tp_status mlp_fwd(const void* X, const void* A, const void* bA, const void* B, const void* bB,
+                  void* Z, void* Ysave, int64_t M, int64_t h, int64_t f, int t, tp_dtype dtype,
+                  void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!X || !A || !B || !Z) return fail(TP_ERR_NULL, "X, A, B and Z are required");
+  TP_TRY(check_dtype(dtype));
+  if (M <= 0 || h <= 0 || f <= 0) return fail(TP_ERR_SHAPE, "M, h and f must be positive");
+  TP_TRY(check_t(t));
+  if (f % t != 0) return fail(TP_ERR_SHAPE, "f must be divisible by t");
+  TP_TRY(check_ptrs_aligned({X, A, bA, B, bB, Z, Ysave, ws}));
+  TP_TRY(check_rows({h, f}));
+  if (ws == nullptr || ws_bytes < mlp_fwd_ws(M, f, dtype))
+    return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
+  const bool f32 = dtype == TP_F32;
+  Carve c(ws, ws_bytes);
+  void* H = c.take(M * f * esize(dtype));
+
+  // Column-split first linear with GeLU per shard ([P3] §2.1 steps 1-2).
+  Gemm g1;
+  g1.M = M; g1.N = f; g1.K = h;
+  g1.a = {X, h, true};
+  g1.b = {A, f, false};
+  g1.epi = kEpiBiasGelu;
+  g1.out = H; g1.ldo = f; g1.out_f32 = f32;
+  g1.bias = bA;
+  g1.out2 = Ysave; g1.ldo2 = f;
+  g1.n_shard = f / t;
+  TP_TRY(run(g1, f32, stream));
+
+  // Row-split second linear; the t partials are summed in the accumulator
+  // (K walks shard 0's rows of B first) and bB is added once.
+  Gemm g2;
+  g2.M = M; g2.N = h; g2.K = f;
+  g2.a = {H, f, true};
+  g2.b = {B, h, false};
+  g2.epi = kEpiStore;
+  g2.out = Z; g2.ldo = h; g2.out_f32 = f32;
+  g2.bias = bB;
+  return run(g2, f32, stream);
+}
+
+tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, const void* Ysave,
+                  const void* dZ, void* dX, void* dA, void* dbA, void* dB, void* dbB, int64_t M,
+                  int64_t h, int64_t f, int t, tp_dtype dtype, void* ws, size_t ws_bytes,
+                  cudaStream_t stream) {
+  if (!X || !A || !B || !dZ || !dX || !dA || !dB)
+    return fail(TP_ERR_NULL, "X, A, B, dZ, dX, dA and dB are required");
+  TP_TRY(check_dtype(dtype));
+  if (M <= 0 || h <= 0 || f <= 0) return fail(TP_ERR_SHAPE, "M, h and f must be positive");
+  TP_TRY(check_t(t));
+  if (f % t != 0) return fail(TP_ERR_SHAPE, "f must be divisible by t");
+  TP_TRY(check_ptrs_aligned({X, A, bA, B, Ysave, dZ, dX, dA, dbA, dB, dbB, ws}));
+  TP_TRY(check_rows({h, f}));
+  if (ws == nullptr || ws_bytes < mlp_bwd_ws(M, h, f, dtype))
+    return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
+  const bool f32 = dtype == TP_F32;
+  const size_t es = esize(dtype);
+  Carve c(ws, ws_bytes);
+  void* dY = c.take(M * f * es);
+  void* H = c.take(M * f * es);
+  void* Yrec = c.take(M * f * es);
+  size_t cs = colsum_scratch_bytes(M, f);
+  if (colsum_scratch_bytes(M, h) > cs) cs = colsum_scratch_bytes(M, h);
+  void* scratch = c.take(cs);
+
+  const void* Y = Ysave;
+  if (Y == nullptr) {
+    // Recompute the pre-activation (and H from it, as in the forward).
+    Gemm gr;
+    gr.M = M; gr.N = f; gr.K = h;
+    gr.a = {X, h, true};
+    gr.b = {A, f, false};
+    gr.epi = kEpiBiasGelu;
+    gr.out = H; gr.ldo = f; gr.out_f32 = f32;
+    gr.bias = bA;
+    gr.out2 = Yrec; gr.ldo2 = f;
+    gr.n_shard = f / t;
+    TP_TRY(run(gr, f32, stream));
+    Y = Yrec;
+  }
+
+  // dY_i = (dZ @ B_i^T) * GeLU'(Y_i) per column shard; H_i = GeLU(Y_i) too.
+  Gemm g3;
+  g3.M = M; g3.N = f; g3.K = h;
+  g3.a = {dZ, h, true};
+  g3.b = {B, h, true};  // B [f, h] read as B^T: n = f index, K contiguous
+  g3.epi = kEpiDGelu;
+  g3.aux = Y; g3.ldaux = f;
+  g3.out = dY; g3.ldo = f; g3.out_f32 = f32;
+  g3.out2 = (Ysave != nullptr) ? H : nullptr; g3.ldo2 = f;
+  g3.n_shard = f / t;
+  TP_TRY(run(g3, f32, stream));
+
+  // dB_i = H_i^T @ dZ: shard i's rows of dB, no exchange.
+  Gemm g4;
+  g4.M = f; g4.N = h; g4.K = M;
+  g4.a = {H, f, false};
+  g4.b = {dZ, h, false};
+  g4.epi = kEpiStore;
+  g4.out = dB; g4.ldo = h; g4.out_f32 = f32;
+  TP_TRY(run(g4, f32, stream));
+
+  // dA_i = X^T @ dY_i: shard i's columns of dA, no exchange.
+  Gemm g5;
+  g5.M = h; g5.N = f; g5.K = M;
+  g5.a = {X, h, false};
+  g5.b = {dY, f, false};
+  g5.epi = kEpiStore;
+  g5.out = dA; g5.ldo = f; g5.out_f32 = f32;
+  g5.n_shard = f / t;
+  TP_TRY(run(g5, f32, stream));
+
+  // dX = sum_i dY_i @ A_i^T: shard partials summed in the accumulator.
+  Gemm g6;
+  g6.M = M; g6.N = h; g6.K = f;
+  g6.a = {dY, f, true};
+  g6.b = {A, f, true};  // A [h, f] read as A^T: n = h index, K contiguous
+  g6.epi = kEpiStore;
+  g6.out = dX; g6.ldo = h; g6.out_f32 = f32;
+  TP_TRY(run(g6, f32, stream));
+
+  if (dbA) TP_TRY(launch_colsum(dY, M, f, f32, dbA, scratch, stream));
+  if (dbB) TP_TRY(launch_colsum(dZ, M, h, f32, dbB, scratch, stream));
+  return TP_OK;
+}
+
+// --------------------------------------------------------------- attention
+
+size_t attn_fwd_ws(int64_t M, int64_t h, int heads) {
+  return align_up(M * 3 * h * 2, 256) + align_up(M * h * 2, 256) +
+         align_up(static_cast<size_t>(M) * heads * 4, 256) + 1024;
+}
+
+size_t attn_bwd_ws(int64_t M, int64_t h, int heads) {
+  AttnShape sh;
+  sh.b = 1; sh.s = M; sh.h = h; sh.heads = heads;
+  return 2 * align_up(M * 3 * h * 2, 256) + align_up(M * h * 2, 256) +
+         align_up(attn_core_bwd_scratch_bytes(sh), 256) + 1024;
+}
+
+tp_status attn_check(const void* X, const void* Wqkv, const void* Wo, int64_t b, int64_t s,
+                     int64_t h, int heads, int t, tp_dtype dtype) {
+  if (!X || !Wqkv || !Wo) return fail(TP_ERR_NULL, "X, Wqkv and Wo are required");
+  TP_TRY(check_dtype(dtype));
+  if (dtype != TP_BF16) return fail(TP_ERR_UNSUPPORTED, "attention is implemented for bf16 only");
+  if (b <= 0 || s <= 0 || h <= 0 || heads <= 0)
+    return fail(TP_ERR_SHAPE, "b, s, h and heads must be positive");
+  TP_TRY(check_t(t));
+  if (h % heads != 0) return fail(TP_ERR_SHAPE, "h must be divisible by heads");
+  if (heads % t != 0) return fail(TP_ERR_SHAPE, "heads must be divisible by t");
+  if (h / heads != 128) return fail(TP_ERR_UNSUPPORTED, "head dimension must be 128");
+  if (b * s > (1ll << 31) - 256) return fail(TP_ERR_SHAPE, "too many tokens");
+  TP_TRY(check_rows({h}));
+  return TP_OK;
+}
+
+tp_status attn_fwd(const void* X, const void* Wqkv, const void* Wo, void* Z, void* QKVsave,
+                   void* Osave, void* LSEsave, int64_t b, int64_t s, int64_t h, int heads, int t,
+                   int causal, tp_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  TP_TRY(attn_check(X, Wqkv, Wo, b, s, h, heads, t, dtype));
+  if (!Z) return fail(TP_ERR_NULL, "Z is required");
+  TP_TRY(check_ptrs_aligned({X, Wqkv, Wo, Z, QKVsave, Osave, LSEsave, ws}));
+  const int64_t M = b * s;
+  if (ws == nullptr || ws_bytes < attn_fwd_ws(M, h, heads))
+    return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
+  Carve c(ws, ws_bytes);
+  void* QKVw = c.take(M * 3 * h * 2);
+  void* Ow = c.take(M * h * 2);
+  void* LSEw = c.take(static_cast<size_t>(M) * heads * 4);
+  void* QKV = QKVsave ? QKVsave : QKVw;
+  void* O = Osave ? Osave : Ow;
+  float* LSE = static_cast<float*>(LSEsave ? LSEsave : LSEw);
+
+  // QKV_g = X @ Wqkv_g: column tiles aligned to the head groups' ranges.
+  Gemm gq;
+  gq.M = M; gq.N = 3 * h; gq.K = h;
+  gq.a = {X, h, true};
+  gq.b = {Wqkv, 3 * h, false};
+  gq.out = QKV; gq.ldo = 3 * h;
+  gq.n_shard = h / t;
+  TP_TRY(launch_gemm_bf16(gq, stream));
+
+  AttnShape sh;
+  sh.b = b; sh.s = s; sh.h = h; sh.heads = heads; sh.causal = causal ? 1 : 0;
+  TP_TRY(launch_attn_core_fwd(sh, QKV, O, LSE, stream));
+
+  // Z = sum_g O_g @ Wo_g: group partials summed in the accumulator.
+  Gemm go;
+  go.M = M; go.N = h; go.K = h;
+  go.a = {O, h, true};
+  go.b = {Wo, h, false};
+  go.out = Z; go.ldo = h;
+  return launch_gemm_bf16(go, stream);
+}
+
+tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* QKVsave,
+                   const void* Osave, const void* LSEsave, const void* dZ, void* dX, void* dWqkv,
+                   void* dWo, int64_t b, int64_t s, int64_t h, int heads, int t, int causal,
+                   tp_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  TP_TRY(attn_check(X, Wqkv, Wo, b, s, h, heads, t, dtype));
+  if (!Osave || !LSEsave || !dZ || !dX || !dWqkv || !dWo)
+    return fail(TP_ERR_NULL, "Osave, LSEsave, dZ, dX, dWqkv and dWo are required");
+  TP_TRY(check_ptrs_aligned({X, Wqkv, Wo, QKVsave, Osave, LSEsave, dZ, dX, dWqkv, dWo, ws}));
+  const int64_t M = b * s;
+  if (ws == nullptr || ws_bytes < attn_bwd_ws(M, h, heads))
+    return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
+  Carve c(ws, ws_bytes);
+  void* QKVw = c.take(M * 3 * h * 2);
+  void* dO = c.take(M * h * 2);
+  void* dQKV = c.take(M * 3 * h * 2);
+  AttnShape sh;
+  sh.b = b; sh.s = s; sh.h = h; sh.heads = heads; sh.causal = causal ? 1 : 0;
+  void* scratch = c.take(attn_core_bwd_scratch_bytes(sh));
+
+  const void* QKV = QKVsave;
+  if (QKV == nullptr) {
+    Gemm gq;
+    gq.M = M; gq.N = 3 * h; gq.K = h;
+    gq.a = {X, h, true};
+    gq.b = {Wqkv, 3 * h, false};
+    gq.out = QKVw; gq.ldo = 3 * h;
+    gq.n_shard = h / t;
+    TP_TRY(launch_gemm_bf16(gq, stream));
+    QKV = QKVw;
+  }
+
+  // dO_g = dZ @ Wo_g^T: group g's columns of dO.
+  Gemm g1;
+  g1.M = M; g1.N = h; g1.K = h;
+  g1.a = {dZ, h, true};
+  g1.b = {Wo, h, true};
+  g1.out = dO; g1.ldo = h;
+  g1.n_shard = h / t;
+  TP_TRY(launch_gemm_bf16(g1, stream));
+
+  // dWo_g = O_g^T @ dZ: group g's rows of dWo, no exchange.
+  Gemm g2;
+  g2.M = h; g2.N = h; g2.K = M;
+  g2.a = {Osave, h, false};
+  g2.b = {dZ, h, false};
+  g2.out = dWo; g2.ldo = h;
+  TP_TRY(launch_gemm_bf16(g2, stream));
+
+  TP_TRY(launch_attn_core_bwd(sh, QKV, Osave, static_cast<const float*>(LSEsave), dO, dQKV,
+                              scratch, stream));
+
+  // dWqkv_g = X^T @ dQKV_g: group g's three column ranges, no exchange.
+  Gemm g3;
+  g3.M = h; g3.N = 3 * h; g3.K = M;
+  g3.a = {X, h, false};
+  g3.b = {dQKV, 3 * h, false};
+  g3.out = dWqkv; g3.ldo = 3 * h;
+  g3.n_shard = h / t;
+  TP_TRY(launch_gemm_bf16(g3, stream));
+
+  // dX = sum_g dQKV_g @ Wqkv_g^T: the K loop visits group 0's q, k and v
+  // ranges, then group 1's, ..., all into one accumulator.
+  Gemm g4;
+  g4.M = M; g4.N = h; g4.K = 3 * h;
+  g4.a = {dQKV, 3 * h, true};
+  g4.b = {Wqkv, 3 * h, true};
+  g4.out = dX; g4.ldo = h;
+  const int64_t width = h / t;
+  if (width % 64 == 0) {
+    g4.korder.range_blocks = static_cast<int>(width / 64);
+    g4.korder.t = t;
+    g4.korder.width = static_cast<int>(width);
+    g4.korder.h = static_cast<int>(h);
+  }
+  return launch_gemm_bf16(g4, stream);
+}
+
+}  // namespace
+}  // namespace tp
+
+using namespace tp;
+
+#define TP_GUARD(body)                                              \
+  try {                                                             \
+    body                                                            \
+  } catch (const std::exception& e) {                               \
+    return fail(TP_ERR_UNSUPPORTED, std::string("internal: ") + e.what()); \
+  } catch (...) {                                                   \
+    return fail(TP_ERR_UNSUPPORTED, "internal error");              \
+  }
+
+extern "C" {
+
+tp_status tp_linear_col(const void* X, const void* W, const void* bias, void* Y, int64_t M,
+                        int64_t K, int64_t N, int t, int shard, tp_dtype dtype,
+                        tp_dtype out_dtype, void* stream) {
+  TP_GUARD(return linear_common(X, W, bias, Y, M, K, N, t, shard, dtype, out_dtype, true,
+                                static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_linear_row(const void* X, const void* W, const void* bias, void* Z, int64_t M,
+                        int64_t K, int64_t N, int t, int shard, tp_dtype dtype,
+                        tp_dtype out_dtype, void* stream) {
+  TP_GUARD(return linear_common(X, W, bias, Z, M, K, N, t, shard, dtype, out_dtype, false,
+                                static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_mlp_fwd(const void* X, const void* A, const void* bA, const void* B, const void* bB,
+                     void* Z, void* Ysave, int64_t M, int64_t h, int64_t f, int t, tp_dtype dtype,
+                     void* ws, size_t ws_bytes, void* stream) {
+  TP_GUARD(return mlp_fwd(X, A, bA, B, bB, Z, Ysave, M, h, f, t, dtype, ws, ws_bytes,
+                          static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_mlp_bwd(const void* X, const void* A, const void* bA, const void* B,
+                     const void* Ysave, const void* dZ, void* dX, void* dA, void* dbA, void* dB,
+                     void* dbB, int64_t M, int64_t h, int64_t f, int t, tp_dtype dtype, void* ws,
+                     size_t ws_bytes, void* stream) {
+  TP_GUARD(return mlp_bwd(X, A, bA, B, Ysave, dZ, dX, dA, dbA, dB, dbB, M, h, f, t, dtype, ws,
+                          ws_bytes, static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_attn_fwd(const void* X, const void* Wqkv, const void* Wo, void* Z, void* QKVsave,
+                      void* Osave, void* LSEsave, int64_t b, int64_t s, int64_t h, int heads,
+                      int t, int causal, tp_dtype dtype, void* ws, size_t ws_bytes,
+                      void* stream) {
+  TP_GUARD(return attn_fwd(X, Wqkv, Wo, Z, QKVsave, Osave, LSEsave, b, s, h, heads, t, causal,
+                           dtype, ws, ws_bytes, static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* QKVsave,
+                      const void* Osave, const void* LSEsave, const void* dZ, void* dX,
+                      void* dWqkv, void* dWo, int64_t b, int64_t s, int64_t h, int heads, int t,
+                      int causal, tp_dtype dtype, void* ws, size_t ws_bytes, void* stream) {
+  TP_GUARD(return attn_bwd(X, Wqkv, Wo, QKVsave, Osave, LSEsave, dZ, dX, dWqkv, dWo, b, s, h,
+                           heads, t, causal, dtype, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream));)
+}
+
+size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, int t,
+                         tp_dtype dtype) {
+  try {
+    if (M <= 0 || h <= 0 || t < 1 || (dtype != TP_F32 && dtype != TP_BF16)) return 0;
+    switch (op) {
+      case TP_OP_MLP_FWD: return f > 0 ? mlp_fwd_ws(M, f, dtype) : 0;
+      case TP_OP_MLP_BWD: return f > 0 ? mlp_bwd_ws(M, h, f, dtype) : 0;
+      case TP_OP_ATTN_FWD: return heads > 0 ? attn_fwd_ws(M, h, heads) : 0;
+      case TP_OP_ATTN_BWD: return heads > 0 ? attn_bwd_ws(M, h, heads) : 0;
+    }
+  } catch (...) {
+  }
+  return 0;
+}
+
+const char* tp_last_error(void) { return g_last_error.c_str(); }
+
+tp_status tp_device_status(void* stream) {
+  try {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int* p = device_status_ptr();
+    if (p == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
+    int v = 0;
+    e = cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    if (v != 0) {
+      const int zero = 0;
+      cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
+      char buf[128];
+      const char* who = v == kStatusProducerTimeout   ? "GEMM TMA producer"
+                        : v == kStatusMmaTimeout      ? "GEMM MMA issuer"
+                        : v == kStatusEpilogueTimeout ? "GEMM epilogue"
+                        : v == kStatusAttnTimeout     ? "attention kernel"
+                                                      : "unknown";
+      std::snprintf(buf, sizeof(buf), "kernel gave up a bounded wait (code 0x%x, %s)", v, who);
+      return fail(TP_ERR_KERNEL, buf);
+    }
+    return TP_OK;
+  } catch (...) {
+    return fail(TP_ERR_UNSUPPORTED, "internal error");
+  }
+}
+
+int tp_version(void) { return 100; }
+
+}  // extern "C"

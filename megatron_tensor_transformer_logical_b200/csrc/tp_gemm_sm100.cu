@@ -1,0 +1,525 @@
+// tcgen05 GEMM for sm_100a: D[M,N] = sum_k A(m,k) B(k,n), bf16 inputs,
+// fp32 accumulation in tensor memory, fused epilogue, bf16 or fp32 output.
+//
+// This one kernel carries every contraction of the partitioned layer:
+// * column-split linears ("图解Transformer并行计算" §1.2, §2.1 step 1): the
+//   column tiles are laid out shard by shard, so no tile straddles two
+//   shards, and each shard's tiles write its own column slice of the output;
+//   the concatenation (the pages' All-Gather) is the output layout itself.
+// * row-split linears (same page, §1.1, §2.1 step 3): the K loop walks the
+//   shards' K ranges in order and every partial product lands in the same
+//   tensor-memory accumulator, so the sum of partials (the pages' AllReduce)
+//   costs no memory traffic and no extra pass.
+// * the backward mirror (same page, §2.2, §3.2): dgrad GEMMs read the weight
+//   K-major (B^T without a transpose in memory), wgrad GEMMs read both
+//   operands MN-major (X^T, H^T likewise).
+//
+// Structure (one CTA per SM, persistent over output tiles of 128 x BN):
+//   warp 0      one thread issues TMA loads of A/B K-blocks (64 deep) into a
+//               ring of shared-memory stages (128-byte swizzle);
+//   warp 1      allocates tensor memory; one thread issues tcgen05.mma
+//               (128 x BN x 16 each) into one of two accumulator buffers;
+//   warps 4-11  epilogue: tcgen05.ld the accumulator (warp w reads lanes
+//               32*(w%4)..+31, i.e. one output row per thread), apply
+//               bias / GeLU / GeLU' in fp32 and store; the other buffer is
+//               being filled meanwhile.
+// Every wait is bounded (see mbar_wait): on expiry the kernel records an
+// error code in the device status word and unwinds.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <mutex>
+
+#include "ptx_sm100.cuh"
+#include "tp_internal.h"
+
+namespace tp {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 384;
+constexpr int kEpiWarps = 8;
+constexpr int kFirstEpiWarp = 4;
+
+template <int BN>
+struct Cfg {
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kBarBytes;
+};
+
+struct Args {
+  int M, N, K;
+  int m_tiles, n_tiles, k_blocks, group_m;
+  int n_shard, n_tiles_per_shard;
+  int kr_range_blocks, kr_t, kr_width, kr_h;
+  void* out;
+  long long ldo;
+  const void* bias;
+  __nv_bfloat16* out2;
+  long long ldo2;
+  const __nv_bfloat16* aux;
+  long long ldaux;
+  int* status;
+};
+
+struct TileCoord {
+  int m0, n0, n_end;
+};
+
+// Grouped raster: bands of group_m row tiles; inside a band the row tile
+// varies fastest, so the CTAs running at one time share B tiles and the
+// band's A rows stay in L2.
+template <int BN>
+__device__ __forceinline__ TileCoord tile_coord(int tile, const Args& a) {
+  const int band = a.group_m * a.n_tiles;
+  const int g = tile / band;
+  const int first_m = g * a.group_m;
+  const int gm = min(a.m_tiles - first_m, a.group_m);
+  const int local = tile - g * band;
+  const int mt = first_m + local % gm;
+  const int nt = local / gm;
+  TileCoord c;
+  c.m0 = mt * BM;
+  if (a.n_shard > 0) {
+    const int sh = nt / a.n_tiles_per_shard;
+    const int j = nt - sh * a.n_tiles_per_shard;
+    c.n0 = sh * a.n_shard + j * BN;
+    c.n_end = min(c.n0 + BN, (sh + 1) * a.n_shard);
+  } else {
+    c.n0 = nt * BN;
+    c.n_end = min(c.n0 + BN, a.N);
+  }
+  return c;
+}
+
+// K coordinate (in elements) of K-block kb.
+__device__ __forceinline__ int k_coord(int kb, const Args& a) {
+  if (a.kr_range_blocks == 0) return kb * BK;
+  const int r = kb / a.kr_range_blocks;   // range index in visiting order
+  const int within = kb - r * a.kr_range_blocks;
+  const int g = r / 3, which = r - 3 * (r / 3);
+  return which * a.kr_h + g * a.kr_width + within * BK;
+}
+
+__device__ __forceinline__ float gelu_f(float x) {
+  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
+
+__device__ __forceinline__ float gelu_prime_f(float x) {
+  return 0.5f * (1.0f + erff(x * 0.70710678118654752f)) +
+         x * 0.39894228040143268f * expf(-0.5f * x * x);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(p[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  uint4 u;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&t);
+  }
+  return u;
+}
+
+// Applies the epilogue to 32 consecutive columns of one row and stores them.
+// col_end is a multiple of 8, so each group of 8 columns is all in or all out.
+template <int EPI, bool OUT_F32, bool BIAS_F32>
+__device__ __forceinline__ void epilogue_row32(float (&v)[32], int row, int col0, int col_end,
+                                               const Args& a) {
+  if (row >= a.M) return;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const int col = col0 + 8 * g;
+    if (col + 8 > col_end) continue;
+    float* x = v + 8 * g;
+    if (EPI != kEpiDGelu && a.bias != nullptr) {
+      float bb[8];
+      if (BIAS_F32) {
+        const float4* bp = reinterpret_cast<const float4*>(static_cast<const float*>(a.bias) + col);
+        const float4 b0 = bp[0], b1 = bp[1];
+        bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
+        bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+      } else {
+        unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.bias) + col),
+                bb);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] += bb[i];
+    }
+    if (EPI == kEpiBiasGelu) {
+      if (a.out2 != nullptr)
+        *reinterpret_cast<uint4*>(a.out2 + (long long)row * a.ldo2 + col) = pack8(x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = gelu_f(x[i]);
+    } else if (EPI == kEpiDGelu) {
+      float y[8];
+      unpack8(*reinterpret_cast<const uint4*>(a.aux + (long long)row * a.ldaux + col), y);
+      if (a.out2 != nullptr) {
+        float hh[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hh[i] = gelu_f(y[i]);
+        *reinterpret_cast<uint4*>(a.out2 + (long long)row * a.ldo2 + col) = pack8(hh);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] *= gelu_prime_f(y[i]);
+    }
+    if (OUT_F32) {
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + (long long)row * a.ldo + col);
+      o[0] = make_float4(x[0], x[1], x[2], x[3]);
+      o[1] = make_float4(x[4], x[5], x[6], x[7]);
+    } else {
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (long long)row * a.ldo + col) =
+          pack8(x);
+    }
+  }
+}
+
+template <int BN, bool A_KMAJ, bool B_KMAJ, int EPI, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmB, const Args args) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::kStages * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], kEpiWarps);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = args.m_tiles * args.n_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const TileCoord tc = tile_coord<BN>(tile, args);
+        for (int kb = 0; kb < args.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, args.status, kStatusProducerTimeout)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes);
+          const int kc = k_coord(kb, args);
+          uint8_t* a_dst = sA + stage * C::kABytes;
+          uint8_t* b_dst = sB + stage * C::kBBytes;
+          if (A_KMAJ) {
+            tma_load_2d(a_dst, &tmA, &full[stage], kc, tc.m0);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_2d(a_dst + c * (BK * 128), &tmA, &full[stage], tc.m0 + 64 * c, kc);
+          }
+          if (B_KMAJ) {
+            tma_load_2d(b_dst, &tmB, &full[stage], kc, tc.n0);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(b_dst + c * (BK * 128), &tmB, &full[stage], tc.n0 + 64 * c, kc);
+          }
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, !A_KMAJ, !B_KMAJ);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.status, kStatusMmaTimeout)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < args.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, args.status, kStatusMmaTimeout)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = A_KMAJ ? sw128_desc(a0 + k * 32, 16, 1024)
+                                       : sw128_desc(a0 + k * 2048, BK * 128, 1024);
+            const uint64_t bd = B_KMAJ ? sw128_desc(b0 + k * 32, 16, 1024)
+                                       : sw128_desc(b0 + k * 2048, BK * 128, 1024);
+            umma_bf16(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp >= kFirstEpiWarp) {
+    // -------------------------------------------------------- epilogue
+    const int ew = warp - kFirstEpiWarp;
+    const int quarter = warp & 3;  // tensor-memory lanes this warp may read
+    const int half = ew >> 2;      // which half of the tile's columns
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const TileCoord tc = tile_coord<BN>(tile, args);
+      if (!mbar_wait(&tfull[acc], acc_phase, args.status, kStatusEpilogueTimeout)) break;
+      tc_fence_after();
+      const int row = tc.m0 + quarter * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < BN / 2; c += 32) {
+        const int cl = half * (BN / 2) + c;
+        if (tc.n0 + cl >= tc.n_end) break;  // warp-uniform
+        float v[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                      static_cast<uint32_t>(acc * BN + cl),
+                  v);
+        epilogue_row32<EPI, OUT_F32, false>(v, row, tc.n0 + cl, tc.n_end, args);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map of a row-major bf16 matrix with `inner` columns (contiguous),
+// `outer` rows, leading dimension `ld`; boxes of box_inner x box_outer with
+// the 128-byte swizzle; out-of-range elements read as zero.
+bool make_map(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, int64_t ld,
+              int box_inner, int box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct Plan {
+  int bn;
+  int m_tiles, n_tiles, n_tiles_per_shard;
+};
+
+Plan plan_for(const Gemm& g, int bn) {
+  Plan p;
+  p.bn = bn;
+  p.m_tiles = static_cast<int>((g.M + BM - 1) / BM);
+  if (g.n_shard > 0) {
+    p.n_tiles_per_shard = static_cast<int>((g.n_shard + bn - 1) / bn);
+    p.n_tiles = static_cast<int>(g.N / g.n_shard) * p.n_tiles_per_shard;
+  } else {
+    p.n_tiles_per_shard = 0;
+    p.n_tiles = static_cast<int>((g.N + bn - 1) / bn);
+  }
+  return p;
+}
+
+// Picks the column tile: 256 wide unless the 128-wide grid fills the SMs in
+// markedly fewer waves (128-wide tiles run at ~85% of the 256-wide rate).
+int choose_bn(const Gemm& g) {
+  if (const char* e = std::getenv("TP_GEMM_BN")) {
+    const int v = std::atoi(e);
+    if (v == 128 || v == 256) return v;
+  }
+  const int sms = sm_count();
+  const Plan p256 = plan_for(g, 256), p128 = plan_for(g, 128);
+  const double w256 = std::ceil(double(p256.m_tiles) * p256.n_tiles / sms);
+  const double w128 = std::ceil(double(p128.m_tiles) * p128.n_tiles / sms);
+  return (w128 * 0.5 / 0.85 < w256 * 0.98) ? 128 : 256;
+}
+
+template <int BN, bool AK, bool BKM, int EPI, bool F32>
+tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
+  using C = Cfg<BN>;
+  CUtensorMap ta, tb;
+  const bool ok_a = AK ? make_map(&ta, g.a.ptr, g.K, g.M, g.a.ld, BK, BM)
+                       : make_map(&ta, g.a.ptr, g.M, g.K, g.a.ld, 64, BK);
+  const bool ok_b = BKM ? make_map(&tb, g.b.ptr, g.K, g.N, g.b.ld, BK, BN)
+                        : make_map(&tb, g.b.ptr, g.N, g.K, g.b.ld, 64, BK);
+  if (!ok_a || !ok_b) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+
+  const Plan p = plan_for(g, BN);
+  Args a;
+  a.M = static_cast<int>(g.M);
+  a.N = static_cast<int>(g.N);
+  a.K = static_cast<int>(g.K);
+  a.m_tiles = p.m_tiles;
+  a.n_tiles = p.n_tiles;
+  a.k_blocks = static_cast<int>((g.K + BK - 1) / BK);
+  a.group_m = 16;
+  a.n_shard = static_cast<int>(g.n_shard);
+  a.n_tiles_per_shard = p.n_tiles_per_shard;
+  a.kr_range_blocks = g.korder.range_blocks;
+  a.kr_t = g.korder.t;
+  a.kr_width = g.korder.width;
+  a.kr_h = g.korder.h;
+  a.out = g.out;
+  a.ldo = g.ldo;
+  a.bias = g.bias;
+  a.out2 = static_cast<__nv_bfloat16*>(g.out2);
+  a.ldo2 = g.ldo2;
+  a.aux = static_cast<const __nv_bfloat16*>(g.aux);
+  a.ldaux = g.ldaux;
+  a.status = device_status_ptr();
+  if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
+
+  auto kern = gemm_bf16_tcgen05<BN, AK, BKM, EPI, F32>;
+  static int configured_mask = 0;  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(configured_mask & (1 << (dev & 31)))) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
+    configured_mask |= 1 << (dev & 31);
+  }
+  const long long tiles = static_cast<long long>(p.m_tiles) * p.n_tiles;
+  if (tiles == 0) return TP_OK;
+  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(ta, tb, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "gemm_bf16_tcgen05 launch");
+  return TP_OK;
+}
+
+template <int BN>
+tp_status dispatch(const Gemm& g, cudaStream_t s) {
+  const bool ak = g.a.k_major, bk = g.b.k_major;
+  if (g.epi == kEpiBiasGelu) {
+    if (ak && !bk && !g.out_f32) return launch_impl<BN, true, false, kEpiBiasGelu, false>(g, s);
+  } else if (g.epi == kEpiDGelu) {
+    if (ak && bk && !g.out_f32) return launch_impl<BN, true, true, kEpiDGelu, false>(g, s);
+  } else {
+    if (ak && !bk) {
+      return g.out_f32 ? launch_impl<BN, true, false, kEpiStore, true>(g, s)
+                       : launch_impl<BN, true, false, kEpiStore, false>(g, s);
+    }
+    if (ak && bk) {
+      return g.out_f32 ? launch_impl<BN, true, true, kEpiStore, true>(g, s)
+                       : launch_impl<BN, true, true, kEpiStore, false>(g, s);
+    }
+    if (!ak && !bk) {
+      return g.out_f32 ? launch_impl<BN, false, false, kEpiStore, true>(g, s)
+                       : launch_impl<BN, false, false, kEpiStore, false>(g, s);
+    }
+  }
+  return fail(TP_ERR_UNSUPPORTED, "gemm: operand layout / epilogue combination not built");
+}
+
+}  // namespace
+
+tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream) {
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return TP_OK;
+  if (g.M > (1ll << 31) - BM || g.N > (1ll << 31) - 256 || g.K > (1ll << 31) - BK)
+    return fail(TP_ERR_SHAPE, "gemm: dimension too large");
+  if (g.a.ld % 8 != 0 || g.b.ld % 8 != 0 || g.ldo % 8 != 0 ||
+      (g.out2 != nullptr && g.ldo2 % 8 != 0) || (g.aux != nullptr && g.ldaux % 8 != 0))
+    return fail(TP_ERR_ALIGN, "gemm: leading dimensions must be multiples of 8 elements");
+  if (g.korder.range_blocks > 0 &&
+      (g.korder.width % BK != 0 || g.korder.h % 8 != 0 ||
+       static_cast<int64_t>(g.korder.t) * 3 * g.korder.width != g.K))
+    return fail(TP_ERR_SHAPE, "gemm: inconsistent shard K order");
+  Gemm gg = g;
+  // A shard-aligned column tile starts at shard * n_shard; the TMA x
+  // coordinate must be a multiple of 8 elements (16 bytes) and the epilogue
+  // stores whole groups of 8 columns, so other shard widths tile plainly
+  // (every column is still computed by the same K loop).
+  if (gg.n_shard > 0 && (gg.n_shard % 8 != 0 || gg.N % gg.n_shard != 0)) gg.n_shard = 0;
+  return choose_bn(gg) == 128 ? dispatch<128>(gg, stream) : dispatch<256>(gg, stream);
+}
+
+}  // namespace tp

@@ -1,0 +1,94 @@
+// Host-side interface between libtp's C entry points and its kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/libtp.h"
+
+namespace tp {
+
+// Records a message for tp_last_error() and returns the status.
+tp_status fail(tp_status st, const std::string& msg);
+tp_status cuda_fail(cudaError_t e, const char* where);
+
+// Device status word of the current device (kernels record bounded-wait
+// expiry there); resolved once per device with cudaGetSymbolAddress.
+int* device_status_ptr();
+int sm_count();
+
+// Epilogue applied to each fp32 accumulator value before it is stored.
+enum Epi : int {
+  kEpiStore = 0,     // out = acc (+ bias[col])
+  kEpiBiasGelu = 1,  // v = acc + bias[col]; out = GeLU(v); out2 = v (if out2)
+  kEpiDGelu = 2,     // y = aux[row,col]; out = acc * GeLU'(y); out2 = GeLU(y) (if out2)
+};
+
+// One operand of D[M,N] = sum_k A(m,k) B(k,n) stored as a row-major matrix.
+// k_major: A stored [M, K] / B stored [N, K] (K contiguous).
+// otherwise: A stored [K, M] / B stored [K, N] (M or N contiguous).
+struct Operand {
+  const void* ptr = nullptr;
+  int64_t ld = 0;  // leading dimension (elements) of the stored matrix
+  bool k_major = true;
+};
+
+// K-block visiting order for a reduction whose shards are not one contiguous
+// K range.  With range_blocks > 0, the K extent is t shards of 3 ranges of
+// `width` columns each (the q, k and v columns of one head group); shard g's
+// ranges start at 0*h + g*width, 1*h + g*width, 2*h + g*width.  The K loop
+// visits shard 0's three ranges, then shard 1's, and so on.
+struct KOrder {
+  int range_blocks = 0;  // 64-column blocks per range (0: natural order)
+  int t = 1;
+  int width = 0;
+  int h = 0;
+};
+
+struct Gemm {
+  int64_t M = 0, N = 0, K = 0;
+  Operand a, b;
+  int epi = kEpiStore;
+  void* out = nullptr;
+  int64_t ldo = 0;
+  bool out_f32 = false;
+  const void* bias = nullptr;  // [N] bf16 / f32 (same type as inputs)
+  void* out2 = nullptr;        // second output (bf16), ldo2
+  int64_t ldo2 = 0;
+  const void* aux = nullptr;   // auxiliary input (bf16), ldaux
+  int64_t ldaux = 0;
+  int64_t n_shard = 0;         // columns per shard: column tiles never straddle shards
+  KOrder korder;
+};
+
+// bf16 x bf16 -> fp32 accumulate on tcgen05; out bf16 or fp32.
+tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream);
+// fp32 SIMT path (exact fp32 products and sums).
+tp_status launch_gemm_f32(const Gemm& g, cudaStream_t stream);
+
+// Column sums: out[c] = sum_r in[r, c] for in [rows, cols] (bf16 or f32),
+// written in the same type.  `scratch` holds `colsum_scratch_bytes` bytes.
+size_t colsum_scratch_bytes(int64_t rows, int64_t cols);
+tp_status launch_colsum(const void* in, int64_t rows, int64_t cols, bool f32, void* out,
+                        void* scratch, cudaStream_t stream);
+
+// Attention core (per head causal softmax attention), bf16 with d = 128.
+struct AttnShape {
+  int64_t b = 0, s = 0, h = 0;
+  int heads = 0;
+  int causal = 1;
+};
+// Q, K, V are column blocks of QKV [M, 3h]; O [M, h]; LSE [b, heads, s] fp32.
+tp_status launch_attn_core_fwd(const AttnShape& sh, const void* QKV, void* O, float* LSE,
+                               cudaStream_t stream);
+// dO [M, h]; writes dQKV [M, 3h] (bf16).  `scratch` holds
+// attn_core_bwd_scratch_bytes bytes (fp32 dQ accumulator and row terms).
+size_t attn_core_bwd_scratch_bytes(const AttnShape& sh);
+tp_status launch_attn_core_bwd(const AttnShape& sh, const void* QKV, const void* O,
+                               const float* LSE, const void* dO, void* dQKV, void* scratch,
+                               cudaStream_t stream);
+
+}  // namespace tp

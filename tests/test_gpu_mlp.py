@@ -1,0 +1,123 @@
+"""GPU parity of the partitioned MLP forward and backward against the oracle.
+
+Forward ("图解Transformer并行计算" §2.1): Y_i = X @ A_i + bA_i, H_i = GeLU(Y_i)
+per column shard, Z = sum_i H_i @ B_i + bB.  Backward (same page, §2.2):
+weight gradients per shard, dX = sum of the shards' partials.
+"""
+import numpy as np
+import pytest
+import torch
+
+from megatron_tensor_transformer_logical_b200 import binding as L
+from megatron_tensor_transformer_logical_b200.inputs import WORKLOADS, Workload, make_mlp_inputs
+from oracle import tp_oracle as O
+from tests.parity import check, cuda, need_gpu, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    need_gpu()
+    yield
+    L.tp_device_status()
+
+
+def gpu_mlp(inp, t, save_y=True, dtype=torch.bfloat16):
+    d = {k: cuda(v) for k, v in inp.items()}
+    X, A, B = d["X"], d["A"], d["B"]
+    M, h = X.shape
+    f = A.shape[1]
+    tpd = L.TP_F32 if dtype == torch.float32 else L.TP_BF16
+    Z = torch.empty(M, h, dtype=dtype, device="cuda")
+    Y = torch.empty(M, f, dtype=dtype, device="cuda") if save_y else None
+    ws = L.workspace(L.TP_OP_MLP_FWD, M, h, f, 0, t, tpd)
+    L.tp_mlp_fwd(X, A, d["bA"], B, d["bB"], Z, Y, t, ws)
+    out = {"Z": Z, "Y": Y}
+    g = {k: torch.empty_like(v) for k, v in (("dX", X), ("dA", A), ("dB", B))}
+    g["dbA"] = torch.empty(f, dtype=dtype, device="cuda")
+    g["dbB"] = torch.empty(h, dtype=dtype, device="cuda")
+    wsb = L.workspace(L.TP_OP_MLP_BWD, M, h, f, 0, t, tpd)
+    L.tp_mlp_bwd(X, A, d["bA"], B, Y, d["dZ"], g["dX"], g["dA"], g["dbA"], g["dB"], g["dbB"], t,
+                 wsb)
+    torch.cuda.synchronize()
+    out.update(g)
+    return out
+
+
+def compare_full(out, inp, dtype):
+    fw = O.mlp_fwd(inp["X"], inp["A"], inp["bA"], inp["B"], inp["bB"])
+    bw = O.mlp_bwd(inp["X"], inp["A"], inp["bA"], inp["B"], inp["dZ"])
+    check(out["Z"], fw["Z"], "Z", dtype)
+    if out["Y"] is not None:
+        check(out["Y"], fw["Y"], "Ysave", dtype)
+    for k in ("dX", "dA", "dB", "dbA", "dbB"):
+        check(out[k], bw[k], k, dtype)
+
+
+def test_mlp_config1_fp32():
+    wl = WORKLOADS[1]
+    inp = make_mlp_inputs(wl)
+    out = gpu_mlp(inp, wl.t, dtype=torch.float32)
+    compare_full(out, inp, "f32")
+
+
+@pytest.mark.parametrize("save_y", [True, False], ids=["Ysave", "recompute"])
+def test_mlp_ragged_bf16(save_y):
+    # 200 rows (two row tiles, ragged), h=136, f=544: ragged column and K tails.
+    wl = Workload(90, "ragged", b=1, s=200, h=136, f=544, t=4, w_std=0.05, bias_std=0.05)
+    inp = make_mlp_inputs(wl)
+    out = gpu_mlp(inp, wl.t, save_y=save_y)
+    compare_full(out, inp, "bf16")
+
+
+@pytest.mark.parametrize("t", [1, 2, 8])
+def test_mlp_fp32_shard_counts(t):
+    wl = Workload(91, "fp32 sweep", b=3, s=40, h=64, f=256, t=t, dtype="f32", bias_std=0.02)
+    inp = make_mlp_inputs(wl)
+    compare_full(gpu_mlp(inp, t, dtype=torch.float32), inp, "f32")
+
+
+def test_mlp_config2_bf16():
+    wl = WORKLOADS[2]
+    inp = make_mlp_inputs(wl)
+    out = gpu_mlp(inp, wl.t)
+    compare_full(out, inp, "bf16")
+
+
+def test_mlp_cross_t_agreement_bf16():
+    """t = 1/2/4/8 agree: column tiles never straddle shards, the K order is fixed."""
+    wl = Workload(92, "cross-t", b=2, s=256, h=256, f=1024, t=1, w_std=0.05, bias_std=0.05)
+    inp = make_mlp_inputs(wl)
+    outs = [gpu_mlp(inp, t) for t in (1, 2, 4, 8)]
+    for o in outs[1:]:
+        for k in ("Z", "dX", "dA", "dB"):
+            assert torch.equal(o[k], outs[0][k]), k
+
+
+def test_mlp_config5_sampled():
+    """The 175B-shaped MLP (h=12288, f=49152, t=8) at full size, sampled.
+
+    Rows of Z and dX depend only on the same rows of X and dZ; column j of
+    dA, entry j of dbA and row j of dB depend only on hidden unit j.  So the
+    oracle on sampled rows / hidden units is an exact reference.
+    """
+    wl = WORKLOADS[5]
+    inp = make_mlp_inputs(wl)
+    out = gpu_mlp(inp, wl.t)
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.r_[0, wl.M - 1, rng.integers(0, wl.M, 6)])
+    units = np.unique(np.r_[0, wl.f - 1, wl.f // wl.t, rng.integers(0, wl.f, 13)])
+    X64, dZ64 = to64(inp["X"]), to64(inp["dZ"])
+    A64, B64 = to64(inp["A"]), to64(inp["B"])
+    fw = O.mlp_fwd(X64[rows], A64, None, B64, None)
+    check(out["Z"][torch.as_tensor(rows, device="cuda")], fw["Z"], "Z rows", "bf16")
+    check(out["Y"][torch.as_tensor(rows, device="cuda")], fw["Y"], "Y rows", "bf16")
+    bw_rows = O.mlp_bwd(X64[rows], A64, None, B64, dZ64[rows])
+    check(out["dX"][torch.as_tensor(rows, device="cuda")], bw_rows["dX"], "dX rows", "bf16")
+    bw_units = O.mlp_bwd(X64, A64[:, units], None, B64[units], dZ64)
+    u = torch.as_tensor(units, device="cuda")
+    check(out["dA"][:, u], bw_units["dA"], "dA cols", "bf16")
+    check(out["dbA"][u], bw_units["dbA"], "dbA", "bf16")
+    check(out["dB"][u], bw_units["dB"], "dB rows", "bf16")
+    check(out["dbB"], bw_units["dbB"], "dbB", "bf16")
