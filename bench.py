@@ -1,0 +1,458 @@
+#!/usr/bin/env python
+"""Throughput of the partitioned Transformer layer on B200 (libtp).
+
+One step = the whole hot path over one batch of synthetic input: head-wise
+attention forward + backward and the partitioned MLP forward + backward
+(tp_attn_fwd, tp_attn_bwd, tp_mlp_fwd, tp_mlp_bwd) on the 175B-shaped layer
+(b=1, s=2048, h=12288, f=49152, 96 heads of 128, t=8 logical shards, bf16
+with fp32 accumulation, weights ~ N(0, 0.006^2), random-init, synthetic data).
+
+Prints one JSON line (rank 0).  `value` is algorithmic TFLOP/s of the whole
+job (2*M*N*K per GEMM; causal attention counts the unmasked half; backward
+core = 2.5x forward core), timed on the device with CUDA events over exactly
+`--steps` steps after `--warmup` steps, max over ranks.  The weights (2.7 GB
+per step) are larger than L2, so every step streams them from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libtp|reference]
+
+--impl reference times the CPU oracle (the reference arm of this build) on
+the host cores on a bounded sample of the same workload.  Under torchrun,
+each rank runs an independent replica (the layer does not shard across GPUs
+here: replicas only); rank 0 prints.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from megatron_tensor_transformer_logical_b200.inputs import WORKLOADS  # noqa: E402
+
+METRIC = "partitioned MLP+attn fwd+bwd TFLOP/s and tokens/s, % of B200 BF16 peak"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+# --------------------------------------------------------------- FLOP model
+def layer_flops(b, s, h, f, heads, causal=True):
+    M = b * s
+    d = h // heads
+    g = lambda m, n, k: 2.0 * m * n * k
+    pairs = 0.5 * s * s if causal else float(s * s)
+    core = 4.0 * d * pairs * b * heads
+    mlp_f = g(M, f, h) + g(M, h, f)
+    mlp_b = 2 * mlp_f
+    att_f = g(M, 3 * h, h) + core + g(M, h, h)
+    att_b = g(M, h, h) + g(h, h, M) + 2.5 * core + g(h, 3 * h, M) + g(M, h, 3 * h)
+    return {"mlp_fwd": mlp_f, "mlp_bwd": mlp_b, "attn_fwd": att_f, "attn_bwd": att_b,
+            "total": mlp_f + mlp_b + att_f + att_b}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_source_hash():
+    p = os.path.join(ROOT, "megatron_tensor_transformer_logical_b200", "csrc", "tp_gemm_sm100.cu")
+    with open(p, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def traffic_per_launch():
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current kernel source; otherwise None."""
+    p = os.path.join(ROOT, "profiles", "gemm_tcgen05_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    if d.get("source_sha256_16") != gemm_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ clock sampling
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(suffix=".csv")
+        self.proc = None
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def mark(self):
+        return time.time()
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+                except (ValueError, IndexError):
+                    continue
+        os.unlink(self.path)
+        inside = [r for r in rows if t0 - 0.15 <= r[0] <= t1 + 0.15] or rows
+        if not inside:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside)}
+
+
+# ------------------------------------------------------------- libtp arm
+class LayerStep:
+    """Device buffers and the four libtp calls of one layer step."""
+
+    def __init__(self, wl, dev):
+        from megatron_tensor_transformer_logical_b200 import binding as L
+        from megatron_tensor_transformer_logical_b200.inputs import make_attn_inputs, make_mlp_inputs
+        self.L = L
+        self.wl = wl
+        mi = make_mlp_inputs(wl)
+        ai = make_attn_inputs(wl)
+        bf = torch.bfloat16
+        M, h, f = wl.M, wl.h, wl.f
+        self.X = mi["X"].to(dev)
+        self.dZ = mi["dZ"].to(dev)
+        self.A, self.B = mi["A"].to(dev), mi["B"].to(dev)
+        self.Wqkv, self.Wo = ai["Wqkv"].to(dev), ai["Wo"].to(dev)
+        e = lambda *s, dt=bf: torch.empty(*s, dtype=dt, device=dev)
+        self.Zm, self.Y = e(M, h), e(M, f)
+        self.dXm, self.dA, self.dB = e(M, h), e(h, f), e(f, h)
+        self.Za, self.QKV, self.O = e(M, h), e(M, 3 * h), e(M, h)
+        self.LSE = e(wl.b, wl.heads, wl.s, dt=torch.float32)
+        self.dXa, self.dWqkv, self.dWo = e(M, h), e(h, 3 * h), e(h, h)
+        self.ws = {op: L.workspace(op, M, h, f, wl.heads, wl.t, L.TP_BF16, device=dev)
+                   for op in (L.TP_OP_MLP_FWD, L.TP_OP_MLP_BWD, L.TP_OP_ATTN_FWD,
+                              L.TP_OP_ATTN_BWD)}
+
+    def attn(self):
+        L, wl = self.L, self.wl
+        L.tp_attn_fwd(self.X, self.Wqkv, self.Wo, self.Za, self.QKV, self.O, self.LSE, wl.b, wl.s,
+                      wl.heads, wl.t, True, self.ws[L.TP_OP_ATTN_FWD])
+        L.tp_attn_bwd(self.X, self.Wqkv, self.Wo, self.QKV, self.O, self.LSE, self.dZ, self.dXa,
+                      self.dWqkv, self.dWo, wl.b, wl.s, wl.heads, wl.t, True,
+                      self.ws[L.TP_OP_ATTN_BWD])
+
+    def mlp(self):
+        L, wl = self.L, self.wl
+        L.tp_mlp_fwd(self.X, self.A, None, self.B, None, self.Zm, self.Y, wl.t,
+                     self.ws[L.TP_OP_MLP_FWD])
+        L.tp_mlp_bwd(self.X, self.A, None, self.B, self.Y, self.dZ, self.dXm, self.dA, None,
+                     self.dB, None, wl.t, self.ws[L.TP_OP_MLP_BWD])
+
+    def step(self):
+        self.attn()
+        self.mlp()
+
+    def outputs(self):
+        return (self.Za, self.Zm, self.dXa, self.dXm)
+
+
+def timed(fn, steps, stream):
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        fn()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    return ev0.elapsed_time(ev1)
+
+
+def run_libtp(args, rank, world, local_rank, dist):
+    from megatron_tensor_transformer_logical_b200 import binding as L
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    st = LayerStep(wl, dev)
+    stream = torch.cuda.current_stream()
+    fl = layer_flops(wl.b, wl.s, wl.h, wl.f, wl.heads)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local_rank])
+
+    for _ in range(args.warmup):
+        st.step()
+    torch.cuda.synchronize()
+    L.tp_device_status()
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0.0)
+    barrier()
+    L.tp_profile_enable(True)
+    n0 = L.tp_launch_count()
+    t0 = time.time()
+    ms = timed(st.step, args.steps, stream)
+    t1 = time.time()
+    launches = L.tp_launch_count() - n0
+    prof = {name: L.tp_profile_read(k) for k, name in L.KIND_NAMES.items()}
+    L.tp_profile_enable(False)
+    barrier()
+    clocks = sampler.stop(t0, t1) if sampler else None
+    L.tp_device_status()
+
+    # MLP fwd+bwd alone (the benchmark spec's target), same protocol.
+    for _ in range(2):
+        st.mlp()
+    barrier()
+    mlp_ms = timed(st.mlp, args.steps, stream)
+    barrier()
+
+    # End to end through the public API: per step, the step's inputs (X, dZ)
+    # copied from pinned host memory and its results (Z and dX of both
+    # sublayers) read back into pinned host memory, inside the timed region.
+    e2e_ms = None
+    h2d = d2h = 0
+    if not args.no_e2e:
+        hX = torch.empty_like(st.X, device="cpu").pin_memory()
+        hdZ = torch.empty_like(st.dZ, device="cpu").pin_memory()
+        hX.copy_(st.X.cpu())
+        hdZ.copy_(st.dZ.cpu())
+        houts = [torch.empty_like(o, device="cpu").pin_memory() for o in st.outputs()]
+
+        def e2e_step():
+            st.X.copy_(hX, non_blocking=True)
+            st.dZ.copy_(hdZ, non_blocking=True)
+            st.step()
+            for ho, o in zip(houts, st.outputs()):
+                ho.copy_(o, non_blocking=True)
+
+        h2d = sum(t.numel() * t.element_size() for t in (hX, hdZ))
+        d2h = sum(t.numel() * t.element_size() for t in houts)
+        e2e_step()
+        barrier()
+        e2e_ms = timed(e2e_step, args.steps, stream)
+        barrier()
+    L.tp_device_status()
+
+    def maxall(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    ms, mlp_ms = maxall(ms), maxall(mlp_ms)
+    e2e_ms = maxall(e2e_ms) if e2e_ms is not None else None
+    if rank != 0:
+        return None
+
+    per_step = ms / args.steps
+    tflops = world * fl["total"] / (per_step * 1e-3) / 1e12
+    tokens = world * wl.M / (per_step * 1e-3)
+    peaks, peak_src = load_peaks()
+    g = prof["gemm_tcgen05"]
+    achieved = g["flops"] / (g["total_ms"] * 1e-3) / 1e12 if g["total_ms"] > 0 else 0.0
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    traffic = traffic_per_launch()
+    mlp_tflops = world * (fl["mlp_fwd"] + fl["mlp_bwd"]) / (mlp_ms / args.steps * 1e-3) / 1e12
+    kernels = {}
+    for name, p in prof.items():
+        if p["launches"]:
+            kernels[name] = {"launches_per_step": p["launches"] / args.steps,
+                             "ms_per_step": p["total_ms"] / args.steps,
+                             "share": p["total_ms"] / ms,
+                             "tflops": p["flops"] / (p["total_ms"] * 1e-3) / 1e12}
+    out = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,0.006^2) random-init weights)",
+        "config": {"workload": f"{wl.name}: attention + MLP fwd+bwd", "b": wl.b, "s": wl.s,
+                   "h": wl.h, "f": wl.f, "heads": wl.heads, "head_dim": wl.h // wl.heads,
+                   "t": wl.t, "causal": True, "global_batch_tokens": world * wl.M,
+                   "parallelism": f"replicas{world} (t={wl.t} logical shards per GPU)",
+                   "l2": "no flush: weights (2.7 GB per step) exceed the 126 MB L2"},
+        "tokens_per_s": round(tokens, 1),
+        "frac_of_nominal_bf16_peak": round(tflops / world / NOMINAL_BF16_TFLOPS, 4),
+        "mlp_fwd_bwd": {"tflops": round(mlp_tflops, 2), "ms_per_step": round(mlp_ms / args.steps, 4),
+                        "frac_of_nominal_2250": round(mlp_tflops / world / NOMINAL_BF16_TFLOPS, 4),
+                        "frac_of_measured_sustained": round(mlp_tflops / world / peak, 4)},
+        "roofline": {"bound": "tensor", "kernel": "gemm_bf16_tcgen05",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "traffic": traffic,
+                     "algorithmic_bytes_per_launch": (g["bytes"] / g["launches"]) if g["launches"] else None,
+                     "flops_per_launch": (g["flops"] / g["launches"]) if g["launches"] else None},
+        "kernels": kernels,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if e2e_ms is not None:
+        out["e2e"] = {"value": round(world * fl["total"] / (e2e_ms / args.steps * 1e-3) / 1e12, 2),
+                      "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "ms_per_step": round(e2e_ms / args.steps, 4)}
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, seconds_hint=args.cpu_sample_tokens)
+    return out
+
+
+# ----------------------------------------------------- the oracle (CPU) arm
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:  # noqa: BLE001
+        return os.cpu_count()
+
+
+def oracle_layer_sample(wl, tokens: int, mi=None, ai=None):
+    """Returns (fn, flops): one oracle pass (attention and MLP, forward and
+    backward) over the first `tokens` tokens of the workload, full width."""
+    import numpy as np  # noqa: F401
+
+    from megatron_tensor_transformer_logical_b200.inputs import make_attn_inputs, make_mlp_inputs
+    from oracle import tp_oracle as O
+    mi = mi or make_mlp_inputs(wl)
+    ai = ai or make_attn_inputs(wl)
+    f64 = lambda t: t.float().numpy().astype("float64")
+    X, dZ = f64(mi["X"][:tokens]), f64(mi["dZ"][:tokens])
+    A, B = f64(mi["A"]), f64(mi["B"])
+    Wqkv, Wo = f64(ai["Wqkv"]), f64(ai["Wo"])
+
+    def fn():
+        O.attn_fwd(X, Wqkv, Wo, 1, tokens, wl.heads)
+        O.attn_bwd(X, Wqkv, Wo, dZ, 1, tokens, wl.heads)
+        O.mlp_fwd(X, A, None, B, None)
+        O.mlp_bwd(X, A, None, B, dZ)
+
+    return fn, layer_flops(1, tokens, wl.h, wl.f, wl.heads)["total"]
+
+
+def cpu_baseline(wl, seconds_hint=512):
+    tokens = int(seconds_hint)
+    fn, flops = oracle_layer_sample(wl, tokens)
+    t0 = time.perf_counter()
+    fn()
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"first {tokens} of {wl.M} tokens of the same layer (full h, f, heads), "
+                      f"attention + MLP fwd+bwd in fp64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl = WORKLOADS[args.workload]
+    tokens = args.ref_sample_tokens
+    fn, flops = oracle_layer_sample(wl, tokens)
+    for _ in range(args.warmup):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fn()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = flops / dt / 1e12
+    cores = _blas_threads()
+    sample = f"first {tokens} of {wl.M} tokens per step (full h, f, heads), fp64 numpy oracle"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: attention + MLP fwd+bwd", "b": wl.b, "s": wl.s,
+                   "h": wl.h, "f": wl.f, "heads": wl.heads, "t": wl.t,
+                   "sample_tokens": tokens},
+        "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["libtp", "reference"], default="libtp")
+    ap.add_argument("--workload", type=int, default=5, choices=[5])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=384)
+    ap.add_argument("--ref-sample-tokens", type=int, default=64)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "libtp":
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+        if args.impl == "libtp":
+            torch.cuda.set_device(local_rank)
+            tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                     device_id=torch.device("cuda", local_rank))
+            dist = tdist
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+    else:
+        out = run_libtp(args, rank, world, local_rank, dist)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

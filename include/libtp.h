@@ -174,6 +174,38 @@ tp_status tp_attn_bwd(const void* X, const void* Wqkv, const void* Wo, const voi
 size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, int t,
                          tp_dtype dtype);
 
+/*
+ * Launch profiling (tracing).  While enabled, every kernel that libtp
+ * launches is bracketed by a pair of CUDA events recorded on the launching
+ * stream, tagged with its kind and its algorithmic work (2*M*N*K FLOPs for a
+ * contraction; unmasked score pairs for attention; bytes read + written for
+ * the memory-bound helpers).  tp_profile_read() waits for the recorded
+ * events and returns the totals of one kind.  Independently of profiling,
+ * tp_launch_count() counts every launch libtp has made since it was loaded.
+ */
+typedef enum tp_kernel_kind {
+  TP_KIND_GEMM_TCGEN05 = 0,  /* bf16 tensor-core GEMM (all linear layers)   */
+  TP_KIND_GEMM_SIMT = 1,     /* fp32 CUDA-core GEMM                          */
+  TP_KIND_ATTN_FWD = 2,      /* attention core forward                       */
+  TP_KIND_ATTN_BWD = 3,      /* attention core backward (all its kernels)    */
+  TP_KIND_REDUCE = 4,        /* column sums, row terms                       */
+  TP_KIND_COUNT = 5
+} tp_kernel_kind;
+
+typedef struct tp_profile_stats {
+  int64_t launches;   /* launches of this kind while profiling was on */
+  double total_ms;    /* sum of their event-timed durations           */
+  double flops;       /* sum of their algorithmic FLOPs                */
+  double bytes;       /* sum of their algorithmic HBM bytes            */
+} tp_profile_stats;
+
+/* Turns launch profiling on (1) or off (0); turning it on clears the totals. */
+tp_status tp_profile_enable(int on);
+/* Synchronizes on the recorded events and fills *out for `kind`. */
+tp_status tp_profile_read(tp_kernel_kind kind, tp_profile_stats* out);
+/* Kernels launched by libtp since the library was loaded. */
+int64_t tp_launch_count(void);
+
 /* Message for the last non-TP_OK status returned on this host thread. */
 const char* tp_last_error(void);
 

@@ -22,9 +22,18 @@ TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_KERNEL, TP_ERR_WORKSPACE = 5, 6, 7, 8
 TP_F32, TP_BF16 = 0, 1
 TP_OP_MLP_FWD, TP_OP_MLP_BWD, TP_OP_ATTN_FWD, TP_OP_ATTN_BWD = 0, 1, 2, 3
 
+TP_KIND_GEMM_TCGEN05, TP_KIND_GEMM_SIMT, TP_KIND_ATTN_FWD, TP_KIND_ATTN_BWD, TP_KIND_REDUCE = range(5)
+KIND_NAMES = {TP_KIND_GEMM_TCGEN05: "gemm_tcgen05", TP_KIND_GEMM_SIMT: "gemm_simt",
+              TP_KIND_ATTN_FWD: "attn_fwd", TP_KIND_ATTN_BWD: "attn_bwd", TP_KIND_REDUCE: "reduce"}
+
 EXPORTS = ("tp_linear_col", "tp_linear_row", "tp_mlp_fwd", "tp_mlp_bwd", "tp_attn_fwd",
            "tp_attn_bwd", "tp_workspace_size", "tp_last_error", "tp_device_status",
-           "tp_version")
+           "tp_version", "tp_profile_enable", "tp_profile_read", "tp_launch_count")
+
+
+class ProfileStats(ctypes.Structure):
+    _fields_ = [("launches", ctypes.c_int64), ("total_ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
 class TPError(RuntimeError):
@@ -61,9 +70,13 @@ def load() -> ctypes.CDLL:
     L.tp_last_error.restype = ctypes.c_char_p
     L.tp_device_status.argtypes = [vp]
     L.tp_version.argtypes = []
+    L.tp_profile_enable.argtypes = [i32]
+    L.tp_profile_read.argtypes = [i32, ctypes.POINTER(ProfileStats)]
+    L.tp_launch_count.argtypes = []
     for name in EXPORTS:
-        if name not in ("tp_workspace_size", "tp_last_error"):
+        if name not in ("tp_workspace_size", "tp_last_error", "tp_launch_count"):
             getattr(L, name).restype = ctypes.c_int
+    L.tp_launch_count.restype = ctypes.c_int64
     _lib = L
     return L
 
@@ -154,6 +167,20 @@ def tp_device_status(stream=None) -> None:
 
 def tp_version() -> int:
     return int(load().tp_version())
+
+
+def tp_profile_enable(on: bool) -> None:
+    _check(load().tp_profile_enable(1 if on else 0))
+
+
+def tp_profile_read(kind: int) -> dict:
+    st = ProfileStats()
+    _check(load().tp_profile_read(kind, ctypes.byref(st)))
+    return {"launches": st.launches, "total_ms": st.total_ms, "flops": st.flops, "bytes": st.bytes}
+
+
+def tp_launch_count() -> int:
+    return int(load().tp_launch_count())
 
 
 def workspace(op: int, M: int, h: int, f: int, heads: int, t: int, dtype: int,

@@ -7,8 +7,10 @@
 #include <cstdio>
 #include <cstring>
 #include <exception>
+#include <atomic>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/libtp.h"
 #include "ptx_sm100.cuh"
@@ -59,6 +61,46 @@ int sm_count() {
     counts[dev] = n;
   }
   return counts[dev];
+}
+
+
+// ------------------------------------------------------------ launch profiling
+namespace {
+struct ProfRecord {
+  cudaEvent_t start = nullptr, stop = nullptr;
+  tp_kernel_kind kind = TP_KIND_GEMM_TCGEN05;
+  double flops = 0, bytes = 0;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof;  // events are created once and reused
+size_t g_prof_used = 0;
+std::atomic<int64_t> g_launches{0};
+}  // namespace
+
+LaunchScope::LaunchScope(tp_kernel_kind kind, double flops, double bytes, cudaStream_t stream)
+    : stream_(stream) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  if (!g_prof_on) return;
+  if (g_prof_used == g_prof.size()) {
+    ProfRecord r;
+    if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess)
+      return;
+    g_prof.push_back(r);
+  }
+  ProfRecord& r = g_prof[g_prof_used];
+  r.kind = kind;
+  r.flops = flops;
+  r.bytes = bytes;
+  if (cudaEventRecord(r.start, stream) != cudaSuccess) return;
+  slot_ = static_cast<int>(g_prof_used++);
+}
+
+LaunchScope::~LaunchScope() {
+  if (slot_ < 0) return;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  cudaEventRecord(g_prof[slot_].stop, stream_);
 }
 
 namespace {
@@ -557,6 +599,45 @@ tp_status tp_device_status(void* stream) {
     return fail(TP_ERR_UNSUPPORTED, "internal error");
   }
 }
+
+tp_status tp_profile_enable(int on) {
+  try {
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    g_prof_on = on != 0;
+    if (g_prof_on) g_prof_used = 0;
+    return TP_OK;
+  } catch (...) {
+    return fail(TP_ERR_UNSUPPORTED, "internal error");
+  }
+}
+
+tp_status tp_profile_read(tp_kernel_kind kind, tp_profile_stats* out) {
+  try {
+    if (out == nullptr) return fail(TP_ERR_NULL, "out is required");
+    if (kind < 0 || kind >= TP_KIND_COUNT) return fail(TP_ERR_SHAPE, "unknown kernel kind");
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    tp_profile_stats st{0, 0.0, 0.0, 0.0};
+    for (size_t i = 0; i < g_prof_used; ++i) {
+      const ProfRecord& r = g_prof[i];
+      if (r.kind != kind) continue;
+      cudaError_t e = cudaEventSynchronize(r.stop);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+      float ms = 0.0f;
+      e = cudaEventElapsedTime(&ms, r.start, r.stop);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+      st.launches += 1;
+      st.total_ms += ms;
+      st.flops += r.flops;
+      st.bytes += r.bytes;
+    }
+    *out = st;
+    return TP_OK;
+  } catch (...) {
+    return fail(TP_ERR_UNSUPPORTED, "internal error");
+  }
+}
+
+int64_t tp_launch_count(void) { return g_launches.load(); }
 
 int tp_version(void) { return 100; }
 

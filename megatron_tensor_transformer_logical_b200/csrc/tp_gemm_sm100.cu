@@ -470,7 +470,15 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   const long long tiles = static_cast<long long>(p.m_tiles) * p.n_tiles;
   if (tiles == 0) return TP_OK;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(ta, tb, a);
+  const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
+  const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
+                       (F32 ? 4.0 : 2.0) * double(g.M) * g.N +
+                       (g.out2 ? 2.0 * double(g.M) * g.N : 0.0) +
+                       (g.aux ? 2.0 * double(g.M) * g.N : 0.0);
+  {
+    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream);
+    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(ta, tb, a);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm_bf16_tcgen05 launch");
   return TP_OK;

@@ -20,6 +20,20 @@ tp_status cuda_fail(cudaError_t e, const char* where);
 int* device_status_ptr();
 int sm_count();
 
+// Brackets one kernel launch: counts it and, while profiling is enabled,
+// records a start/stop event pair on `stream` with its kind and work.
+class LaunchScope {
+ public:
+  LaunchScope(tp_kernel_kind kind, double flops, double bytes, cudaStream_t stream);
+  ~LaunchScope();
+  LaunchScope(const LaunchScope&) = delete;
+  LaunchScope& operator=(const LaunchScope&) = delete;
+
+ private:
+  int slot_ = -1;
+  cudaStream_t stream_;
+};
+
 // Epilogue applied to each fp32 accumulator value before it is stored.
 enum Epi : int {
   kEpiStore = 0,     // out = acc (+ bias[col])

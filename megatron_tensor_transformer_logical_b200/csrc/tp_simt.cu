@@ -136,10 +136,14 @@ tp_status launch_gemm_f32(const Gemm& g, cudaStream_t stream) {
   a.aux = static_cast<const float*>(g.aux);
   a.ldaux = g.ldaux;
   dim3 grid(static_cast<unsigned>((g.N + TN - 1) / TN), static_cast<unsigned>((g.M + TM - 1) / TM));
-  switch (g.epi) {
-    case kEpiBiasGelu: gemm_f32_simt<kEpiBiasGelu><<<grid, 256, 0, stream>>>(a); break;
-    case kEpiDGelu: gemm_f32_simt<kEpiDGelu><<<grid, 256, 0, stream>>>(a); break;
-    default: gemm_f32_simt<kEpiStore><<<grid, 256, 0, stream>>>(a); break;
+  {
+    LaunchScope scope(TP_KIND_GEMM_SIMT, 2.0 * double(g.M) * g.N * g.K,
+                      4.0 * (double(g.M) * g.K + double(g.K) * g.N + double(g.M) * g.N), stream);
+    switch (g.epi) {
+      case kEpiBiasGelu: gemm_f32_simt<kEpiBiasGelu><<<grid, 256, 0, stream>>>(a); break;
+      case kEpiDGelu: gemm_f32_simt<kEpiDGelu><<<grid, 256, 0, stream>>>(a); break;
+      default: gemm_f32_simt<kEpiStore><<<grid, 256, 0, stream>>>(a); break;
+    }
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm_f32_simt launch");

@@ -64,6 +64,9 @@ tp_status launch_colsum(const void* in, int64_t rows, int64_t cols, bool f32, vo
   dim3 g1(static_cast<unsigned>((cols + 255) / 256), static_cast<unsigned>(chunks));
   dim3 g2(static_cast<unsigned>((cols + 255) / 256));
   float* part = static_cast<float*>(scratch);
+  const double es = f32 ? 4.0 : 2.0;
+  LaunchScope s1(TP_KIND_REDUCE, double(rows) * cols, es * rows * cols + 4.0 * chunks * cols,
+                 stream);
   if (f32) {
     colsum_partial<true><<<g1, 256, 0, stream>>>(in, rows, cols, rpc, part);
     colsum_final<true><<<g2, 256, 0, stream>>>(part, chunks, cols, out);

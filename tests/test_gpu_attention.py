@@ -1,0 +1,149 @@
+"""GPU parity of head-wise partitioned attention, forward and backward.
+
+"图解Transformer并行计算" §3.2: Wqkv split by columns in head groups, each
+group runs its heads' softmax(Q K^T / sqrt(d)) V, Wo split by rows and the
+group partials summed; backward mirrors it (dWqkv, dWo per group, dX summed).
+"""
+import numpy as np
+import pytest
+import torch
+
+from megatron_tensor_transformer_logical_b200 import binding as L
+from megatron_tensor_transformer_logical_b200.inputs import WORKLOADS, Workload, make_attn_inputs
+from oracle import tp_oracle as O
+from tests.parity import check, cuda, need_gpu, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    need_gpu()
+    yield
+    L.tp_device_status()
+
+
+def gpu_attn(inp, wl, causal=True, save_qkv=True, t=None):
+    t = wl.t if t is None else t
+    d = {k: cuda(v) for k, v in inp.items()}
+    M, h = wl.M, wl.h
+    Z = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
+    QKV = torch.empty(M, 3 * h, dtype=torch.bfloat16, device="cuda") if save_qkv else None
+    Os = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
+    LSE = torch.empty(wl.b, wl.heads, wl.s, dtype=torch.float32, device="cuda")
+    L.tp_attn_fwd(d["X"], d["Wqkv"], d["Wo"], Z, QKV, Os, LSE, wl.b, wl.s, wl.heads, t, causal,
+                  L.workspace(L.TP_OP_ATTN_FWD, M, h, 0, wl.heads, t, L.TP_BF16))
+    dX, dWqkv, dWo = (torch.empty_like(d[k]) for k in ("X", "Wqkv", "Wo"))
+    L.tp_attn_bwd(d["X"], d["Wqkv"], d["Wo"], QKV, Os, LSE, d["dZ"], dX, dWqkv, dWo, wl.b, wl.s,
+                  wl.heads, t, causal,
+                  L.workspace(L.TP_OP_ATTN_BWD, M, h, 0, wl.heads, t, L.TP_BF16))
+    torch.cuda.synchronize()
+    return {"Z": Z, "QKV": QKV, "O": Os, "LSE": LSE, "dX": dX, "dWqkv": dWqkv, "dWo": dWo}
+
+
+def compare_full(out, inp, wl, causal):
+    fw = O.attn_fwd(inp["X"], inp["Wqkv"], inp["Wo"], wl.b, wl.s, wl.heads, causal)
+    bw = O.attn_bwd(inp["X"], inp["Wqkv"], inp["Wo"], inp["dZ"], wl.b, wl.s, wl.heads, causal)
+    for k in ("Z", "O"):
+        check(out[k], fw[k], k, "bf16")
+    if out["QKV"] is not None:
+        check(out["QKV"], fw["QKV"], "QKV", "bf16")
+    assert np.max(np.abs(to64(out["LSE"]) - fw["LSE"])) < 2e-2
+    for k in ("dX", "dWqkv", "dWo"):
+        check(out[k], bw[k], k, "bf16")
+
+
+@pytest.mark.parametrize("causal", [True, False], ids=["causal", "full"])
+@pytest.mark.parametrize("save_qkv", [True, False], ids=["QKVsave", "recompute"])
+def test_attention_small_ragged(causal, save_qkv):
+    # s = 200: four 64-row query blocks (the last ragged), seven 32-row blocks.
+    wl = Workload(80, "attn ragged", b=2, s=200, h=512, heads=4, t=2, w_std=0.05)
+    inp = make_attn_inputs(wl)
+    compare_full(gpu_attn(inp, wl, causal, save_qkv), inp, wl, causal)
+
+
+def test_attention_single_token_and_short():
+    # s = 1 (a row that sees only itself: O = V) and s = 3.
+    for s in (1, 3):
+        wl = Workload(81, "attn short", b=3, s=s, h=256, heads=2, t=2, w_std=0.05)
+        inp = make_attn_inputs(wl)
+        out = gpu_attn(inp, wl)
+        compare_full(out, inp, wl, True)
+        if s == 1:
+            qkv = to64(out["QKV"])
+            assert np.allclose(to64(out["O"]), qkv[:, 2 * wl.h:], rtol=1e-2, atol=1e-2)
+
+
+def test_attention_group_count_sweep():
+    """t = 1, 2, 4: forward results and the per-group weight gradients agree
+    bitwise (grouping only moves tile boundaries); dX agrees within tolerance
+    (its K loop visits the groups' ranges in group order)."""
+    wl = Workload(82, "attn t sweep", b=2, s=256, h=512, heads=4, t=1, w_std=0.05)
+    inp = make_attn_inputs(wl)
+    outs = {t: gpu_attn(inp, wl, t=t) for t in (1, 2, 4)}
+    for t in (2, 4):
+        for k in ("Z", "QKV", "O", "LSE", "dWqkv", "dWo"):
+            assert torch.equal(outs[t][k], outs[1][k]), (t, k)
+        check(outs[t]["dX"], to64(outs[1]["dX"]), f"dX t={t} vs t=1", "bf16")
+    compare_full(outs[4], inp, wl, True)
+
+
+def _head_slice(W, h, heads, j):
+    c = O.head_columns(h, heads, j)
+    return np.concatenate([c["q"], c["k"], c["v"]])
+
+
+def test_attention_config4_full_size():
+    """Config 4 (b=4, s=2048, h=4096, 32 heads, t=8) at full size.
+
+    Rows of one batch element depend on that element alone, so the oracle on
+    batch element 3 is exact for those rows; dWqkv columns and dWo rows of one
+    head depend on that head alone, so a one-head oracle is exact for them.
+    """
+    wl = WORKLOADS[4]
+    inp = make_attn_inputs(wl)
+    out = gpu_attn(inp, wl)
+    X, Wqkv, Wo, dZ = (to64(inp[k]) for k in ("X", "Wqkv", "Wo", "dZ"))
+    bi = 3
+    rows = slice(bi * wl.s, (bi + 1) * wl.s)
+    fw = O.attn_fwd(X[rows], Wqkv, Wo, 1, wl.s, wl.heads)
+    bw = O.attn_bwd(X[rows], Wqkv, Wo, dZ[rows], 1, wl.s, wl.heads)
+    check(out["Z"][rows], fw["Z"], "Z (batch 3)", "bf16")
+    check(out["O"][rows], fw["O"], "O (batch 3)", "bf16")
+    assert np.max(np.abs(to64(out["LSE"][bi]) - fw["LSE"][0])) < 2e-2
+    check(out["dX"][rows], bw["dX"], "dX (batch 3)", "bf16")
+    for j in (0, 13, 31):  # heads in groups 0, 3 and 7
+        cols = _head_slice(Wqkv, wl.h, wl.heads, j)
+        d = wl.h // wl.heads
+        w_rows = slice(j * d, (j + 1) * d)
+        bj = O.attn_bwd(X, Wqkv[:, cols], Wo[w_rows], dZ, wl.b, wl.s, 1)
+        c = torch.as_tensor(cols, device="cuda")
+        check(out["dWqkv"][:, c], bj["dWqkv"], f"dWqkv head {j}", "bf16")
+        check(out["dWo"][w_rows], bj["dWo"], f"dWo head {j}", "bf16")
+
+
+def test_attention_config5_sampled():
+    """Config 5 attention (s=2048, h=12288, 96 heads, t=8).
+
+    With the causal mask, rows 0..255 depend only on rows 0..255, so the
+    oracle on the first 256 tokens is exact for them; per-head quantities
+    (O columns, LSE, dWqkv columns, dWo rows) come from a one-head oracle.
+    """
+    wl = WORKLOADS[5]
+    inp = make_attn_inputs(wl)
+    out = gpu_attn(inp, wl)
+    X, Wqkv, Wo, dZ = (to64(inp[k]) for k in ("X", "Wqkv", "Wo", "dZ"))
+    r = 256
+    fw = O.attn_fwd(X[:r], Wqkv, Wo, 1, r, wl.heads)
+    check(out["Z"][:r], fw["Z"], "Z rows < 256", "bf16")
+    d = wl.h // wl.heads
+    for j in (0, 50, 95):
+        cols = _head_slice(Wqkv, wl.h, wl.heads, j)
+        w_rows = slice(j * d, (j + 1) * d)
+        fj = O.attn_fwd(X, Wqkv[:, cols], Wo[w_rows], 1, wl.s, 1)
+        check(out["O"][:, j * d:(j + 1) * d], fj["O"], f"O head {j}", "bf16")
+        assert np.max(np.abs(to64(out["LSE"][0, j]) - fj["LSE"][0, 0])) < 2e-2
+        bj = O.attn_bwd(X, Wqkv[:, cols], Wo[w_rows], dZ, 1, wl.s, 1)
+        c = torch.as_tensor(cols, device="cuda")
+        check(out["dWqkv"][:, c], bj["dWqkv"], f"dWqkv head {j}", "bf16")
+        check(out["dWo"][w_rows], bj["dWo"], f"dWo head {j}", "bf16")
