@@ -161,7 +161,7 @@ class LayerStep:
         e = lambda *s, dt=bf: torch.empty(*s, dtype=dt, device=dev)
         self.Zm, self.Y = e(M, h), e(M, f)
         self.dXm, self.dA, self.dB = e(M, h), e(h, f), e(f, h)
-        self.Za, self.QKV, self.O = e(M, h), e(M, 3 * h), e(M, h)
+        self.Za, self.QKV, self.O = e(M, h), e(M, 3 * h, dt=torch.float16), e(M, h)
         self.LSE = e(wl.b, wl.heads, wl.s, dt=torch.float32)
         self.dXa, self.dWqkv, self.dWo = e(M, h), e(h, 3 * h), e(h, h)
         self.ws = {op: L.workspace(op, M, h, f, wl.heads, wl.t, L.TP_BF16, device=dev)

@@ -139,9 +139,14 @@ tp_status tp_mlp_bwd(const void* X, const void* A, const void* bA, const void* B
  *   key c from query r when c > r ([P4] masked_fill(mask == 0, -inf));
  *   Z = sum_g O_g @ Wo_g with Wo split by rows (no concatenation before Wo).
  *   X [M = b*s, h]; Wqkv [h, 3h]; Wo [h, h]; Z [M, h]; all bf16.
- *   QKVsave [M, 3h] bf16 or NULL; Osave [M, h] bf16 or NULL (heads in column
+ *   QKVsave [M, 3h] fp16 or NULL; Osave [M, h] bf16 or NULL (heads in column
  *   order); LSEsave [b, heads, s] fp32 or NULL: natural-log softmax
  *   denominators of the scaled, masked scores.
+ *   Precision: the linears multiply bf16 with fp32 accumulation; the
+ *   attention core takes Q, K, V (and, in the backward, dO) as fp16, which
+ *   the QKV (dO) GEMM writes, and rounds P and dS to fp16 for its products
+ *   (fp32 accumulation).  A QKV or dO value beyond the fp16 range is
+ *   saturated and reported by tp_device_status() as TP_ERR_KERNEL.
  *   d must be 128.  dtype must be TP_BF16 (else TP_ERR_UNSUPPORTED).
  * Errors: NULL X/Wqkv/Wo/Z/ws; heads % t; h % heads; s < 1; TP_ERR_WORKSPACE.
  */
@@ -155,8 +160,8 @@ tp_status tp_attn_fwd(const void* X, const void* Wqkv, const void* Wo, void* Z,
  *   dO_g = dZ @ Wo_g^T;  dWo_g = O_g^T @ dZ;  per head the softmax backward
  *   gives dQ, dK, dV;  dWqkv_g = X^T @ dQKV_g;  dX = sum_g dQKV_g @ Wqkv_g^T
  *   with the group partials summed in the accumulator, group 0 first.
- *   Osave, LSEsave: from tp_attn_fwd (required).  QKVsave: from tp_attn_fwd,
- *   or NULL to recompute QKV = X @ Wqkv.  Outputs dX [M, h], dWqkv [h, 3h],
+ *   Osave, LSEsave: from tp_attn_fwd (required).  QKVsave (fp16): from
+ *   tp_attn_fwd, or NULL to recompute QKV = X @ Wqkv.  Outputs dX [M, h], dWqkv [h, 3h],
  *   dWo [h, h], all bf16.
  * Errors: as tp_attn_fwd, plus NULL Osave/LSEsave/dZ/dX/dWqkv/dWo.
  */
@@ -211,8 +216,9 @@ const char* tp_last_error(void);
 
 /*
  * Synchronizes `stream`, then reads and clears the device status word of the
- * current device.  TP_OK, TP_ERR_KERNEL (a kernel gave up a bounded wait;
- * the message names where) or TP_ERR_CUDA.
+ * current device.  TP_OK, TP_ERR_KERNEL (a kernel gave up a bounded wait, or
+ * an fp16 attention intermediate was saturated; the message says which) or
+ * TP_ERR_CUDA.
  */
 tp_status tp_device_status(void* stream);
 

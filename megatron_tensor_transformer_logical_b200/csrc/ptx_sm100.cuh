@@ -15,6 +15,7 @@ enum : int {
   kStatusMmaTimeout = 0x102,
   kStatusEpilogueTimeout = 0x103,
   kStatusAttnTimeout = 0x104,
+  kStatusF16Range = 0x201,  // a value outside the fp16 range was saturated
 };
 
 // A wait that has not completed after this long is treated as a hang: the

@@ -399,7 +399,7 @@ tp_status attn_fwd(const void* X, const void* Wqkv, const void* Wo, void* Z, voi
   gq.M = M; gq.N = 3 * h; gq.K = h;
   gq.a = {X, h, true};
   gq.b = {Wqkv, 3 * h, false};
-  gq.out = QKV; gq.ldo = 3 * h;
+  gq.out = QKV; gq.ldo = 3 * h; gq.out_f16 = true;  // the attention core reads fp16
   gq.n_shard = h / t;
   TP_TRY(launch_gemm_bf16(gq, stream));
 
@@ -441,7 +441,7 @@ tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* 
     gq.M = M; gq.N = 3 * h; gq.K = h;
     gq.a = {X, h, true};
     gq.b = {Wqkv, 3 * h, false};
-    gq.out = QKVw; gq.ldo = 3 * h;
+    gq.out = QKVw; gq.ldo = 3 * h; gq.out_f16 = true;
     gq.n_shard = h / t;
     TP_TRY(launch_gemm_bf16(gq, stream));
     QKV = QKVw;
@@ -452,7 +452,7 @@ tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* 
   g1.M = M; g1.N = h; g1.K = h;
   g1.a = {dZ, h, true};
   g1.b = {Wo, h, true};
-  g1.out = dO; g1.ldo = h;
+  g1.out = dO; g1.ldo = h; g1.out_f16 = true;  // the attention core reads fp16
   g1.n_shard = h / t;
   TP_TRY(launch_gemm_bf16(g1, stream));
 
@@ -591,7 +591,12 @@ tp_status tp_device_status(void* stream) {
                         : v == kStatusEpilogueTimeout ? "GEMM epilogue"
                         : v == kStatusAttnTimeout     ? "attention kernel"
                                                       : "unknown";
-      std::snprintf(buf, sizeof(buf), "kernel gave up a bounded wait (code 0x%x, %s)", v, who);
+      if (v == kStatusF16Range)
+        std::snprintf(buf, sizeof(buf),
+                      "an fp16 attention intermediate (QKV or dO) exceeded the fp16 range and "
+                      "was saturated (code 0x%x)", v);
+      else
+        std::snprintf(buf, sizeof(buf), "kernel gave up a bounded wait (code 0x%x, %s)", v, who);
       return fail(TP_ERR_KERNEL, buf);
     }
     return TP_OK;

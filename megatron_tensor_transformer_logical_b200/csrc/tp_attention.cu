@@ -13,8 +13,11 @@
 // Forward: one CTA per (64 query rows, batch, head); 4 warps x 16 rows;
 // keys in blocks of 64 through a double-buffered cp.async pipeline; online
 // softmax (row max / sum in registers, quad shuffles); P stays in registers
-// as the A operand of P V.  Tensor-core work uses mma.sync m16n8k16 (bf16 in,
-// fp32 accumulate).
+// as the A operand of P V.  Tensor-core work uses mma.sync m16n8k16 with fp16
+// operands and fp32 accumulation: Q, K, V, dO arrive in fp16 (written so by
+// the GEMMs that produce them) and P, dS are rounded to fp16 for the
+// products.  fp16 keeps three more mantissa bits than bf16, which halves the
+// backward's rounding error; O and dQKV are written in bf16 for the linears.
 //
 // Backward, without atomics: D = rowsum(dO * O) per row and head; one kernel
 // per key block accumulates dK and dV over the query blocks that see it;
@@ -22,6 +25,7 @@
 //   P = exp(S*scale - LSE); dV = P^T dO; dP = dO V^T; dS = P * (dP - D);
 //   dQ = scale * dS K; dK = scale * dS^T Q.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -37,9 +41,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.69314718055994531f;
 
 struct AttnArgs {
-  const __nv_bfloat16* qkv;  // [M, 3h]
-  const __nv_bfloat16* o;    // [M, h]
-  const __nv_bfloat16* dout; // [M, h]
+  const __half* qkv;         // [M, 3h] fp16
+  const __nv_bfloat16* o;    // [M, h] bf16
+  const __half* dout;        // [M, h] fp16
   const float* lse;          // [b, heads, s]
   const float* dsum;         // [b, heads, s]: rowsum(dO * O)
   __nv_bfloat16* out;        // O (fwd) or dQKV (bwd)
@@ -86,7 +90,7 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
       "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -94,6 +98,11 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 t = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&t);
 }
 
@@ -125,7 +134,7 @@ __device__ __forceinline__ void ldb_kn(uint32_t tile, int k0, int n0, int lane, 
 // matrix with leading dimension ld (elements) and column offset col into a
 // swizzled tile; rows at or beyond row_end are zero-filled.
 template <int ROWS, int THREADS>
-__device__ __forceinline__ void load_tile(uint32_t tile, const __nv_bfloat16* base, long long ld,
+__device__ __forceinline__ void load_tile(uint32_t tile, const __half* base, long long ld,
                                           int g0, int row_end, int col) {
   constexpr int CHUNKS = ROWS * 16;
 #pragma unroll
@@ -133,7 +142,7 @@ __device__ __forceinline__ void load_tile(uint32_t tile, const __nv_bfloat16* ba
     const int r = i >> 4, c = i & 15;
     const int gr = g0 + r;
     const bool ok = gr < row_end;
-    const __nv_bfloat16* src = base + static_cast<long long>(ok ? gr : 0) * ld + col + c * 8;
+    const __half* src = base + static_cast<long long>(ok ? gr : 0) * ld + col + c * 8;
     cp_async16(tile + swz(r, c), src, ok);
   }
 }
@@ -154,7 +163,7 @@ __global__ void __launch_bounds__(FWD_THREADS) attn_fwd_kernel(const AttnArgs a)
   const int head = blockIdx.y % a.heads, bi = blockIdx.y / a.heads;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long ld = 3LL * a.h;
-  const __nv_bfloat16* base = a.qkv + static_cast<long long>(bi) * a.s * ld;
+  const __half* base = a.qkv + static_cast<long long>(bi) * a.s * ld;
   const int q0 = qb * FWD_BM;
   const int n_kb = a.causal ? (min(q0 + FWD_BM, a.s) + FWD_BN - 1) / FWD_BN
                             : (a.s + FWD_BN - 1) / FWD_BN;
@@ -254,10 +263,10 @@ __global__ void __launch_bounds__(FWD_THREADS) attn_fwd_kernel(const AttnArgs a)
     // O += P V: P (16 x 64) from registers as four k16 A fragments.
 #pragma unroll
     for (int kk = 0; kk < FWD_BN / 16; ++kk) {
-      const uint32_t a0 = pack_bf16(sc[2 * kk][0], sc[2 * kk][1]);
-      const uint32_t a1 = pack_bf16(sc[2 * kk][2], sc[2 * kk][3]);
-      const uint32_t a2 = pack_bf16(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
-      const uint32_t a3 = pack_bf16(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+      const uint32_t a0 = pack_f16(sc[2 * kk][0], sc[2 * kk][1]);
+      const uint32_t a1 = pack_f16(sc[2 * kk][2], sc[2 * kk][3]);
+      const uint32_t a2 = pack_f16(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+      const uint32_t a3 = pack_f16(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
 #pragma unroll
       for (int n = 0; n < 16; n += 2) {
         uint32_t bf[4];
@@ -302,11 +311,11 @@ __global__ void attn_bwd_dsum_kernel(const AttnArgs a, float* dsum, long long M)
   const uint2 ov = *reinterpret_cast<const uint2*>(a.o + off);
   const uint2 dv = *reinterpret_cast<const uint2*>(a.dout + off);
   const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-  const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+  const __half2* d2 = reinterpret_cast<const __half2*>(&dv);
   float acc = 0.0f;
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const float2 x = __bfloat1622float2(o2[i]), y = __bfloat1622float2(d2[i]);
+    const float2 x = __bfloat1622float2(o2[i]), y = __half22float2(d2[i]);
     acc += x.x * y.x + x.y * y.y;
   }
 #pragma unroll
@@ -335,8 +344,8 @@ __global__ void __launch_bounds__(DQ_THREADS) attn_bwd_dq_kernel(const AttnArgs 
   const int head = blockIdx.y % a.heads, bi = blockIdx.y / a.heads;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long ld = 3LL * a.h;
-  const __nv_bfloat16* base = a.qkv + static_cast<long long>(bi) * a.s * ld;
-  const __nv_bfloat16* dbase = a.dout + static_cast<long long>(bi) * a.s * a.h;
+  const __half* base = a.qkv + static_cast<long long>(bi) * a.s * ld;
+  const __half* dbase = a.dout + static_cast<long long>(bi) * a.s * a.h;
   const int q0 = qb * DQ_BM;
   const int n_kb = a.causal ? (min(q0 + DQ_BM, a.s) + DQ_BN - 1) / DQ_BN
                             : (a.s + DQ_BN - 1) / DQ_BN;
@@ -411,10 +420,10 @@ __global__ void __launch_bounds__(DQ_THREADS) attn_bwd_dq_kernel(const AttnArgs 
     // dQ += dS K (K stored [key][d]: k = key rows, n = d contiguous).
 #pragma unroll
     for (int kk = 0; kk < DQ_BN / 16; ++kk) {
-      const uint32_t a0 = pack_bf16(sc[2 * kk][0], sc[2 * kk][1]);
-      const uint32_t a1 = pack_bf16(sc[2 * kk][2], sc[2 * kk][3]);
-      const uint32_t a2 = pack_bf16(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
-      const uint32_t a3 = pack_bf16(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+      const uint32_t a0 = pack_f16(sc[2 * kk][0], sc[2 * kk][1]);
+      const uint32_t a1 = pack_f16(sc[2 * kk][2], sc[2 * kk][3]);
+      const uint32_t a2 = pack_f16(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+      const uint32_t a3 = pack_f16(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
 #pragma unroll
       for (int n = 0; n < 16; n += 2) {
         uint32_t bf[4];
@@ -460,8 +469,8 @@ __global__ void __launch_bounds__(KV_THREADS) attn_bwd_dkdv_kernel(const AttnArg
   const int head = blockIdx.y % a.heads, bi = blockIdx.y / a.heads;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long ld = 3LL * a.h;
-  const __nv_bfloat16* base = a.qkv + static_cast<long long>(bi) * a.s * ld;
-  const __nv_bfloat16* dbase = a.dout + static_cast<long long>(bi) * a.s * a.h;
+  const __half* base = a.qkv + static_cast<long long>(bi) * a.s * ld;
+  const __half* dbase = a.dout + static_cast<long long>(bi) * a.s * a.h;
   const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.s;
   const int k0 = kb * KV_BN;
   const int qb_first = a.causal ? k0 / KV_BM : 0;
@@ -542,14 +551,14 @@ __global__ void __launch_bounds__(KV_THREADS) attn_bwd_dkdv_kernel(const AttnArg
     // dV += P^T dO and dK += dS^T Q (dO, Q stored [query][d]: k = query rows).
 #pragma unroll
     for (int kk = 0; kk < KV_BM / 16; ++kk) {
-      const uint32_t p0 = pack_bf16(st[2 * kk][0], st[2 * kk][1]);
-      const uint32_t p1 = pack_bf16(st[2 * kk][2], st[2 * kk][3]);
-      const uint32_t p2 = pack_bf16(st[2 * kk + 1][0], st[2 * kk + 1][1]);
-      const uint32_t p3 = pack_bf16(st[2 * kk + 1][2], st[2 * kk + 1][3]);
-      const uint32_t s0 = pack_bf16(dpt[2 * kk][0], dpt[2 * kk][1]);
-      const uint32_t s1 = pack_bf16(dpt[2 * kk][2], dpt[2 * kk][3]);
-      const uint32_t s2 = pack_bf16(dpt[2 * kk + 1][0], dpt[2 * kk + 1][1]);
-      const uint32_t s3 = pack_bf16(dpt[2 * kk + 1][2], dpt[2 * kk + 1][3]);
+      const uint32_t p0 = pack_f16(st[2 * kk][0], st[2 * kk][1]);
+      const uint32_t p1 = pack_f16(st[2 * kk][2], st[2 * kk][3]);
+      const uint32_t p2 = pack_f16(st[2 * kk + 1][0], st[2 * kk + 1][1]);
+      const uint32_t p3 = pack_f16(st[2 * kk + 1][2], st[2 * kk + 1][3]);
+      const uint32_t s0 = pack_f16(dpt[2 * kk][0], dpt[2 * kk][1]);
+      const uint32_t s1 = pack_f16(dpt[2 * kk][2], dpt[2 * kk][3]);
+      const uint32_t s2 = pack_f16(dpt[2 * kk + 1][0], dpt[2 * kk + 1][1]);
+      const uint32_t s3 = pack_f16(dpt[2 * kk + 1][2], dpt[2 * kk + 1][3]);
 #pragma unroll
       for (int n = 0; n < 16; n += 2) {
         uint32_t bd[4], bq[4];
@@ -609,7 +618,7 @@ tp_status launch_attn_core_fwd(const AttnShape& sh, const void* QKV, void* O, fl
   if (sh.h / sh.heads != D) return fail(TP_ERR_UNSUPPORTED, "attention: head dimension must be 128");
   if (sh.b * sh.heads > 65535) return fail(TP_ERR_SHAPE, "attention: b * heads too large");
   AttnArgs a = base_args(sh);
-  a.qkv = static_cast<const __nv_bfloat16*>(QKV);
+  a.qkv = static_cast<const __half*>(QKV);
   a.out = static_cast<__nv_bfloat16*>(O);
   a.lse_out = LSE;
   cudaError_t e = set_smem(attn_fwd_kernel, FWD_SMEM);
@@ -635,9 +644,9 @@ tp_status launch_attn_core_bwd(const AttnShape& sh, const void* QKV, const void*
   if (sh.h / sh.heads != D) return fail(TP_ERR_UNSUPPORTED, "attention: head dimension must be 128");
   if (sh.b * sh.heads > 65535) return fail(TP_ERR_SHAPE, "attention: b * heads too large");
   AttnArgs a = base_args(sh);
-  a.qkv = static_cast<const __nv_bfloat16*>(QKV);
+  a.qkv = static_cast<const __half*>(QKV);
   a.o = static_cast<const __nv_bfloat16*>(O);
-  a.dout = static_cast<const __nv_bfloat16*>(dO);
+  a.dout = static_cast<const __half*>(dO);
   a.lse = LSE;
   float* dsum = static_cast<float*>(scratch);
   a.dsum = dsum;

@@ -28,6 +28,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -129,6 +130,31 @@ __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
   }
 }
 
+// Output element types of the epilogue.
+enum Out : int { kOutBF16 = 0, kOutF32 = 1, kOutF16 = 2 };
+
+constexpr float kF16Max = 65504.0f;
+
+// Eight fp32 values to fp16, saturated to the finite range; returns whether
+// any finite value had to be clamped.
+__device__ __forceinline__ uint4 pack8_f16(float* f, bool& clamped) {
+  uint4 u;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (fabsf(f[i]) > kF16Max) {
+      clamped = true;
+      f[i] = copysignf(kF16Max, f[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 t = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&t);
+  }
+  return u;
+}
+
 __device__ __forceinline__ uint4 pack8(const float* f) {
   uint4 u;
   uint32_t* w = reinterpret_cast<uint32_t*>(&u);
@@ -142,10 +168,11 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
 
 // Applies the epilogue to 32 consecutive columns of one row and stores them.
 // col_end is a multiple of 8, so each group of 8 columns is all in or all out.
-template <int EPI, bool OUT_F32, bool BIAS_F32>
+template <int EPI, int OUT, bool BIAS_F32>
 __device__ __forceinline__ void epilogue_row32(float (&v)[32], int row, int col0, int col_end,
                                                const Args& a) {
   if (row >= a.M) return;
+  bool clamped = false;
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     const int col = col0 + 8 * g;
@@ -182,18 +209,22 @@ __device__ __forceinline__ void epilogue_row32(float (&v)[32], int row, int col0
 #pragma unroll
       for (int i = 0; i < 8; ++i) x[i] *= gelu_prime_f(y[i]);
     }
-    if (OUT_F32) {
+    if (OUT == kOutF32) {
       float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + (long long)row * a.ldo + col);
       o[0] = make_float4(x[0], x[1], x[2], x[3]);
       o[1] = make_float4(x[4], x[5], x[6], x[7]);
+    } else if (OUT == kOutF16) {
+      *reinterpret_cast<uint4*>(static_cast<__half*>(a.out) + (long long)row * a.ldo + col) =
+          pack8_f16(x, clamped);
     } else {
       *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (long long)row * a.ldo + col) =
           pack8(x);
     }
   }
+  if (OUT == kOutF16 && clamped) atomicCAS(a.status, 0, kStatusF16Range);
 }
 
-template <int BN, bool A_KMAJ, bool B_KMAJ, int EPI, bool OUT_F32>
+template <int BN, bool A_KMAJ, bool B_KMAJ, int EPI, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, const Args args) {
@@ -338,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                       static_cast<uint32_t>(acc * BN + cl),
                   v);
-        epilogue_row32<EPI, OUT_F32, false>(v, row, tc.n0 + cl, tc.n_end, args);
+        epilogue_row32<EPI, OUT, false>(v, row, tc.n0 + cl, tc.n_end, args);
       }
       tc_fence_before();
       __syncwarp();
@@ -422,7 +453,7 @@ int choose_bn(const Gemm& g) {
   return (w128 * 0.5 / 0.85 < w256 * 0.98) ? 128 : 256;
 }
 
-template <int BN, bool AK, bool BKM, int EPI, bool F32>
+template <int BN, bool AK, bool BKM, int EPI, int OUT>
 tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   using C = Cfg<BN>;
   CUtensorMap ta, tb;
@@ -457,7 +488,7 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   a.status = device_status_ptr();
   if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
 
-  auto kern = gemm_bf16_tcgen05<BN, AK, BKM, EPI, F32>;
+  auto kern = gemm_bf16_tcgen05<BN, AK, BKM, EPI, OUT>;
   static int configured_mask = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -472,7 +503,7 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
   const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
-                       (F32 ? 4.0 : 2.0) * double(g.M) * g.N +
+                       (OUT == kOutF32 ? 4.0 : 2.0) * double(g.M) * g.N +
                        (g.out2 ? 2.0 * double(g.M) * g.N : 0.0) +
                        (g.aux ? 2.0 * double(g.M) * g.N : 0.0);
   {
@@ -484,25 +515,27 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   return TP_OK;
 }
 
+template <int BN, bool AK, bool BKM, int EPI>
+tp_status by_out(const Gemm& g, cudaStream_t s) {
+  if (g.out_f32) return launch_impl<BN, AK, BKM, EPI, kOutF32>(g, s);
+  if (g.out_f16) return launch_impl<BN, AK, BKM, EPI, kOutF16>(g, s);
+  return launch_impl<BN, AK, BKM, EPI, kOutBF16>(g, s);
+}
+
 template <int BN>
 tp_status dispatch(const Gemm& g, cudaStream_t s) {
   const bool ak = g.a.k_major, bk = g.b.k_major;
+  const bool plain_out = !g.out_f32 && !g.out_f16;
   if (g.epi == kEpiBiasGelu) {
-    if (ak && !bk && !g.out_f32) return launch_impl<BN, true, false, kEpiBiasGelu, false>(g, s);
+    if (ak && !bk && plain_out) return launch_impl<BN, true, false, kEpiBiasGelu, kOutBF16>(g, s);
   } else if (g.epi == kEpiDGelu) {
-    if (ak && bk && !g.out_f32) return launch_impl<BN, true, true, kEpiDGelu, false>(g, s);
+    if (ak && bk && plain_out) return launch_impl<BN, true, true, kEpiDGelu, kOutBF16>(g, s);
   } else {
-    if (ak && !bk) {
-      return g.out_f32 ? launch_impl<BN, true, false, kEpiStore, true>(g, s)
-                       : launch_impl<BN, true, false, kEpiStore, false>(g, s);
-    }
-    if (ak && bk) {
-      return g.out_f32 ? launch_impl<BN, true, true, kEpiStore, true>(g, s)
-                       : launch_impl<BN, true, true, kEpiStore, false>(g, s);
-    }
-    if (!ak && !bk) {
-      return g.out_f32 ? launch_impl<BN, false, false, kEpiStore, true>(g, s)
-                       : launch_impl<BN, false, false, kEpiStore, false>(g, s);
+    if (ak && !bk) return by_out<BN, true, false, kEpiStore>(g, s);
+    if (ak && bk) return by_out<BN, true, true, kEpiStore>(g, s);
+    if (!ak && !bk && !g.out_f16) {
+      return g.out_f32 ? launch_impl<BN, false, false, kEpiStore, kOutF32>(g, s)
+                       : launch_impl<BN, false, false, kEpiStore, kOutBF16>(g, s);
     }
   }
   return fail(TP_ERR_UNSUPPORTED, "gemm: operand layout / epilogue combination not built");

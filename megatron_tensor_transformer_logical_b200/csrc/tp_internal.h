@@ -69,6 +69,7 @@ struct Gemm {
   void* out = nullptr;
   int64_t ldo = 0;
   bool out_f32 = false;
+  bool out_f16 = false;        // fp16 output (saturating; range errors are flagged)
   const void* bias = nullptr;  // [N] bf16 / f32 (same type as inputs)
   void* out2 = nullptr;        // second output (bf16), ldo2
   int64_t ldo2 = 0;
@@ -78,7 +79,7 @@ struct Gemm {
   KOrder korder;
 };
 
-// bf16 x bf16 -> fp32 accumulate on tcgen05; out bf16 or fp32.
+// bf16 x bf16 -> fp32 accumulate on tcgen05; out bf16, fp16 or fp32.
 tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream);
 // fp32 SIMT path (exact fp32 products and sums).
 tp_status launch_gemm_f32(const Gemm& g, cudaStream_t stream);

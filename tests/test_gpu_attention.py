@@ -28,7 +28,7 @@ def gpu_attn(inp, wl, causal=True, save_qkv=True, t=None):
     d = {k: cuda(v) for k, v in inp.items()}
     M, h = wl.M, wl.h
     Z = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
-    QKV = torch.empty(M, 3 * h, dtype=torch.bfloat16, device="cuda") if save_qkv else None
+    QKV = torch.empty(M, 3 * h, dtype=torch.float16, device="cuda") if save_qkv else None
     Os = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
     LSE = torch.empty(wl.b, wl.heads, wl.s, dtype=torch.float32, device="cuda")
     L.tp_attn_fwd(d["X"], d["Wqkv"], d["Wo"], Z, QKV, Os, LSE, wl.b, wl.s, wl.heads, t, causal,
@@ -147,3 +147,22 @@ def test_attention_config5_sampled():
         c = torch.as_tensor(cols, device="cuda")
         check(out["dWqkv"][:, c], bj["dWqkv"], f"dWqkv head {j}", "bf16")
         check(out["dWo"][w_rows], bj["dWo"], f"dWo head {j}", "bf16")
+
+
+def test_fp16_range_overflow_is_reported():
+    """QKV beyond the fp16 range is saturated and reported as TP_ERR_KERNEL."""
+    wl = Workload(83, "attn overflow", b=1, s=64, h=256, heads=2, t=1, w_std=0.05)
+    inp = make_attn_inputs(wl)
+    inp["X"] = torch.full_like(inp["X"], 256.0)
+    inp["Wqkv"] = torch.full_like(inp["Wqkv"], 2.0)  # every QKV entry = 256 * 2 * 256
+    d = {k: cuda(v) for k, v in inp.items()}
+    M, h = wl.M, wl.h
+    Z = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
+    QKV = torch.empty(M, 3 * h, dtype=torch.float16, device="cuda")
+    L.tp_attn_fwd(d["X"], d["Wqkv"], d["Wo"], Z, QKV, None, None, wl.b, wl.s, wl.heads, 1, True,
+                  L.workspace(L.TP_OP_ATTN_FWD, M, h, 0, wl.heads, 1, L.TP_BF16))
+    with pytest.raises(L.TPError) as e:
+        L.tp_device_status()
+    assert e.value.status == L.TP_ERR_KERNEL and "fp16" in str(e.value)
+    assert torch.isfinite(QKV.float()).all() and QKV.float().max().item() == 65504.0
+    L.tp_device_status()  # the word was cleared
