@@ -310,12 +310,18 @@ def attention_core_bwd(Q, K, V, dO, causal: bool = True):
     return dQ, dK, dV
 
 
-def _attn_dims(X, h: int, heads: int, b: int, s: int):
-    if h % heads != 0:
+def _attn_dims(X, Wqkv, heads: int, b: int, s: int):
+    """Returns (hi, d): the attention width hi = Wqkv columns / 3 (h for the
+    whole layer; a head group's or one head's width for a slice of Wqkv) and
+    the head dimension d = hi / heads."""
+    if Wqkv.shape[1] % 3 != 0:
+        raise ValueError("Wqkv must have 3 * width columns")
+    hi = Wqkv.shape[1] // 3
+    if hi % heads != 0:
         raise ValueError("hidden size must be divisible by the number of heads")
-    if X.shape != (b * s, h):
-        raise ValueError(f"X must be [b*s, h] = [{b * s}, {h}], got {X.shape}")
-    return h // heads
+    if X.shape != (b * s, Wqkv.shape[0]):
+        raise ValueError(f"X must be [b*s, h] = [{b * s}, {Wqkv.shape[0]}], got {X.shape}")
+    return hi, hi // heads
 
 
 def attn_fwd(X, Wqkv, Wo, b: int, s: int, heads: int, causal: bool = True):
@@ -323,11 +329,12 @@ def attn_fwd(X, Wqkv, Wo, b: int, s: int, heads: int, causal: bool = True):
 
     QKV = X @ Wqkv; per batch element and head j, O_j = attention_core of
     (Q_j, K_j, V_j); the heads are concatenated in column order to O [M, h];
-    Z = O @ Wo.  Returns QKV, O, LSE [b, heads, s] and Z.
+    Z = O @ Wo.  Returns QKV, O, LSE [b, heads, s] and Z.  Given the column
+    slice of Wqkv of some heads and the matching rows of Wo (as one head
+    group holds them, [P3] §3.2), it computes exactly those heads.
     """
     X, Wqkv, Wo = _f64(X), _f64(Wqkv), _f64(Wo)
-    h = X.shape[1]
-    d = _attn_dims(X, h, heads, b, s)
+    h, d = _attn_dims(X, Wqkv, heads, b, s)
     QKV = X @ Wqkv
     O = np.zeros((b * s, h))
     LSE = np.zeros((b, heads, s))
@@ -350,8 +357,7 @@ def attn_fwd_parallel(X, Wqkv, Wo, b: int, s: int, heads: int, t: int, causal: b
     Wo that match its heads; Z = sum_g Z_g.
     """
     X, Wqkv, Wo = _f64(X), _f64(Wqkv), _f64(Wo)
-    h = X.shape[1]
-    d = _attn_dims(X, h, heads, b, s)
+    h, d = _attn_dims(X, Wqkv, heads, b, s)
     hg = _check_divisible(heads, t, "heads")
     Zs = []
     for g in range(t):
@@ -381,8 +387,7 @@ def attn_bwd(X, Wqkv, Wo, dZ, b: int, s: int, heads: int, causal: bool = True):
     dWqkv = X^T @ dQKV; dX = dQKV @ Wqkv^T.
     """
     X, Wqkv, Wo, dZ = _f64(X), _f64(Wqkv), _f64(Wo), _f64(dZ)
-    h = X.shape[1]
-    d = _attn_dims(X, h, heads, b, s)
+    h, d = _attn_dims(X, Wqkv, heads, b, s)
     fw = attn_fwd(X, Wqkv, Wo, b, s, heads, causal)
     QKV, O = fw["QKV"], fw["O"]
     dO = dZ @ Wo.T
@@ -409,8 +414,7 @@ def attn_bwd_parallel(X, Wqkv, Wo, dZ, b: int, s: int, heads: int, t: int,
     a partial dX_g = dQKV_g @ Wqkv_g^T; dX = sum_g dX_g.
     """
     X, Wqkv, Wo, dZ = _f64(X), _f64(Wqkv), _f64(Wo), _f64(dZ)
-    h = X.shape[1]
-    d = _attn_dims(X, h, heads, b, s)
+    h, d = _attn_dims(X, Wqkv, heads, b, s)
     hg = _check_divisible(heads, t, "heads")
     w = hg * d
     dWqkv = np.zeros_like(Wqkv)

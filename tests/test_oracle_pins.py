@@ -414,3 +414,26 @@ def test_planted_mistake_is_caught(name):
         except AssertionError:
             failures += 1
     assert failures >= 1, f"no pin caught the planted mistake '{name}'"
+
+
+def test_head_slice_equals_the_heads_columns():
+    """[P3] §3.2: a head group computes its heads from its own column slice of
+    Wq, Wk, Wv and row slice of Wo; the slice gives exactly those heads' O,
+    LSE, dWqkv columns and dWo rows of the whole layer."""
+    r = _rng(30)
+    b, s, h, heads = 2, 5, 16, 4
+    X = r.standard_normal((b * s, h))
+    Wqkv, Wo = r.standard_normal((h, 3 * h)) * 0.4, r.standard_normal((h, h)) * 0.4
+    dZ = r.standard_normal((b * s, h))
+    full = O.attn_fwd(X, Wqkv, Wo, b, s, heads)
+    gfull = O.attn_bwd(X, Wqkv, Wo, dZ, b, s, heads)
+    d = h // heads
+    for j in range(heads):
+        c = O.head_columns(h, heads, j)
+        cols = np.concatenate([c["q"], c["k"], c["v"]])
+        one = O.attn_fwd(X, Wqkv[:, cols], Wo[j * d:(j + 1) * d], b, s, 1)
+        assert np.max(np.abs(one["O"] - full["O"][:, j * d:(j + 1) * d])) < 1e-13
+        assert np.max(np.abs(one["LSE"][:, 0] - full["LSE"][:, j])) < 1e-13
+        g = O.attn_bwd(X, Wqkv[:, cols], Wo[j * d:(j + 1) * d], dZ, b, s, 1)
+        assert np.max(np.abs(g["dWqkv"] - gfull["dWqkv"][:, cols])) < 1e-12
+        assert np.max(np.abs(g["dWo"] - gfull["dWo"][j * d:(j + 1) * d])) < 1e-12
