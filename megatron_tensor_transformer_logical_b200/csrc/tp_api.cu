@@ -78,9 +78,10 @@ size_t g_prof_used = 0;
 std::atomic<int64_t> g_launches{0};
 }  // namespace
 
-LaunchScope::LaunchScope(tp_kernel_kind kind, double flops, double bytes, cudaStream_t stream)
+LaunchScope::LaunchScope(tp_kernel_kind kind, double flops, double bytes, cudaStream_t stream,
+                         int kernels)
     : stream_(stream) {
-  g_launches.fetch_add(1, std::memory_order_relaxed);
+  g_launches.fetch_add(kernels, std::memory_order_relaxed);
   std::lock_guard<std::mutex> lock(g_prof_mu);
   if (!g_prof_on) return;
   if (g_prof_used == g_prof.size()) {

@@ -653,7 +653,8 @@ tp_status launch_attn_core_bwd(const AttnShape& sh, const void* QKV, const void*
   a.out = static_cast<__nv_bfloat16*>(dQKV);
   const long long M = sh.b * sh.s;
   const long long warps = M * sh.heads;
-  LaunchScope scope(TP_KIND_ATTN_BWD, 2.5 * core_flops(sh), 2.0 * double(M) * 8 * sh.h, stream);
+  LaunchScope scope(TP_KIND_ATTN_BWD, 2.5 * core_flops(sh), 2.0 * double(M) * 8 * sh.h, stream,
+                    3);
   attn_bwd_dsum_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, stream>>>(a, dsum, M);
   cudaError_t e = set_smem(attn_bwd_dq_kernel, DQ_SMEM);
   if (e == cudaSuccess) e = set_smem(attn_bwd_dkdv_kernel, KV_SMEM);

@@ -24,7 +24,9 @@ int sm_count();
 // records a start/stop event pair on `stream` with its kind and work.
 class LaunchScope {
  public:
-  LaunchScope(tp_kernel_kind kind, double flops, double bytes, cudaStream_t stream);
+  // `kernels`: how many kernels the bracketed region launches.
+  LaunchScope(tp_kernel_kind kind, double flops, double bytes, cudaStream_t stream,
+              int kernels = 1);
   ~LaunchScope();
   LaunchScope(const LaunchScope&) = delete;
   LaunchScope& operator=(const LaunchScope&) = delete;

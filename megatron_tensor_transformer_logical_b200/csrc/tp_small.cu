@@ -66,7 +66,7 @@ tp_status launch_colsum(const void* in, int64_t rows, int64_t cols, bool f32, vo
   float* part = static_cast<float*>(scratch);
   const double es = f32 ? 4.0 : 2.0;
   LaunchScope s1(TP_KIND_REDUCE, double(rows) * cols, es * rows * cols + 4.0 * chunks * cols,
-                 stream);
+                 stream, 2);
   if (f32) {
     colsum_partial<true><<<g1, 256, 0, stream>>>(in, rows, cols, rpc, part);
     colsum_final<true><<<g2, 256, 0, stream>>>(part, chunks, cols, out);

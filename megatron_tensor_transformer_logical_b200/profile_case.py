@@ -1,0 +1,94 @@
+"""Runs one libtp operation at a chosen shape a few times, for profilers.
+
+    python -m megatron_tensor_transformer_logical_b200.profile_case CASE [--iters N]
+
+Cases (175B-shaped layer unless noted; bf16, t = 8):
+  mlp_g1      tp_linear_col  X[2048,12288] @ A[12288,49152]      (column split)
+  mlp_g2      tp_linear_row  H[2048,49152] @ B[49152,12288]      (row split, sum in TMEM)
+  mlp_fwd     tp_mlp_fwd     (two GEMMs)
+  mlp_bwd     tp_mlp_bwd     (dgrad+GeLU', two wgrads, dgrad)
+  attn_fwd    tp_attn_fwd    (QKV GEMM, attention core, Wo GEMM)
+  attn_bwd    tp_attn_bwd
+  small_gemm  tp_linear_col  X[1024,4096] @ W[4096,8192] (a quick case)
+
+Inputs are seeded N(0,1) / N(0, 0.006^2) tensors made on the device; nothing
+is checked here (the tests do that).  Prints the mean device time per call.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import binding as L
+
+
+def _t(shape, std, dtype=torch.bfloat16, seed=0):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    return (torch.randn(*shape, generator=g, device="cuda") * std).to(dtype)
+
+
+def make_case(name: str):
+    M, h, f, heads, t = 2048, 12288, 49152, 96, 8
+    bf = torch.bfloat16
+    if name == "small_gemm":
+        X, W = _t((1024, 4096), 1.0), _t((4096, 8192), 0.02, seed=1)
+        Y = torch.empty(1024, 8192, dtype=bf, device="cuda")
+        return lambda: L.tp_linear_col(X, W, None, Y, t)
+    if name == "mlp_g1":
+        X, A = _t((M, h), 1.0), _t((h, f), 0.006, seed=1)
+        Y = torch.empty(M, f, dtype=bf, device="cuda")
+        return lambda: L.tp_linear_col(X, A, None, Y, t)
+    if name == "mlp_g2":
+        H, B = _t((M, f), 0.5), _t((f, h), 0.006, seed=1)
+        Z = torch.empty(M, h, dtype=bf, device="cuda")
+        return lambda: L.tp_linear_row(H, B, None, Z, t)
+    if name in ("mlp_fwd", "mlp_bwd"):
+        X, A, B = _t((M, h), 1.0), _t((h, f), 0.006, seed=1), _t((f, h), 0.006, seed=2)
+        dZ = _t((M, h), 1.0, seed=3)
+        Z, Y = torch.empty(M, h, dtype=bf, device="cuda"), torch.empty(M, f, dtype=bf, device="cuda")
+        wsf = L.workspace(L.TP_OP_MLP_FWD, M, h, f, 0, t, L.TP_BF16)
+        L.tp_mlp_fwd(X, A, None, B, None, Z, Y, t, wsf)
+        if name == "mlp_fwd":
+            return lambda: L.tp_mlp_fwd(X, A, None, B, None, Z, Y, t, wsf)
+        dX, dA, dB = torch.empty_like(X), torch.empty_like(A), torch.empty_like(B)
+        wsb = L.workspace(L.TP_OP_MLP_BWD, M, h, f, 0, t, L.TP_BF16)
+        return lambda: L.tp_mlp_bwd(X, A, None, B, Y, dZ, dX, dA, None, dB, None, t, wsb)
+    if name in ("attn_fwd", "attn_bwd"):
+        X, Wqkv, Wo = _t((M, h), 1.0), _t((h, 3 * h), 0.006, seed=1), _t((h, h), 0.006, seed=2)
+        dZ = _t((M, h), 1.0, seed=3)
+        Z = torch.empty(M, h, dtype=bf, device="cuda")
+        QKV = torch.empty(M, 3 * h, dtype=torch.float16, device="cuda")
+        O = torch.empty(M, h, dtype=bf, device="cuda")
+        LSE = torch.empty(1, heads, M, dtype=torch.float32, device="cuda")
+        wsf = L.workspace(L.TP_OP_ATTN_FWD, M, h, 0, heads, t, L.TP_BF16)
+        fwd = lambda: L.tp_attn_fwd(X, Wqkv, Wo, Z, QKV, O, LSE, 1, M, heads, t, True, wsf)
+        fwd()
+        if name == "attn_fwd":
+            return fwd
+        dX, dWqkv, dWo = torch.empty_like(X), torch.empty_like(Wqkv), torch.empty_like(Wo)
+        wsb = L.workspace(L.TP_OP_ATTN_BWD, M, h, 0, heads, t, L.TP_BF16)
+        return lambda: L.tp_attn_bwd(X, Wqkv, Wo, QKV, O, LSE, dZ, dX, dWqkv, dWo, 1, M, heads, t,
+                                     True, wsb)
+    raise SystemExit(f"unknown case {name}")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case")
+    ap.add_argument("--iters", type=int, default=3)
+    a = ap.parse_args()
+    fn = make_case(a.case)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    L.tp_device_status()
+    print(f"{a.case}: {e0.elapsed_time(e1) / a.iters:.3f} ms per call")
+
+
+if __name__ == "__main__":
+    main()
