@@ -115,6 +115,31 @@ tp_status tp_mlp_fwd(const void* X, const void* A, const void* bA, const void* B
                      void* stream);
 
 /*
+ * tp_mlp_fwd without a workspace, for callers that cannot allocate device
+ * memory (a host that owns all device memory and forbids allocation on its
+ * inference path, a latency-critical loop that cannot afford cudaMalloc's
+ * synchronisation, a plugin interface that passes only inputs and outputs).
+ * The source pages have no counterpart: this is a deployment variant.
+ *   Same arguments, arithmetic and kernels as tp_mlp_fwd; the intermediate
+ *   H [M, f] lives in a fixed 64 MiB (67108864-byte) array compiled into
+ *   libtp, which every GPU that loads the library holds until the process
+ *   exits.  M * f * element size must not exceed 64 MiB (H alone; so
+ *   M * f <= 33554432 for bf16, 16777216 for fp32), otherwise TP_ERR_SHAPE
+ *   with a message saying so.  Allocates nothing and calls no allocator.
+ *   The first call on each device looks up the array's device address with
+ *   cudaGetSymbolAddress (that device must be current); make that first call
+ *   before any stream capture.  Every call shares the one array and it keeps
+ *   the previous call's contents; nothing in it needs to start at zero (H is
+ *   fully written before it is read).  Calls whose executions overlap on the
+ *   GPU (on different streams, or on several host threads) race on it.
+ * Errors: those of tp_mlp_fwd (without TP_ERR_WORKSPACE), plus TP_ERR_SHAPE
+ * for sizes beyond the array and TP_ERR_CUDA if the lookup fails.
+ */
+tp_status tp_mlp_fwd_noalloc(const void* X, const void* A, const void* bA, const void* B,
+                             const void* bB, void* Z, void* Ysave, int64_t M, int64_t h,
+                             int64_t f, int t, tp_dtype dtype, void* stream);
+
+/*
  * Partitioned MLP backward, the pages' mirror rule ([P3] §2.2):
  *   dY_i = (dZ @ B_i^T) * GeLU'(Y_i);  dB_i = H_i^T @ dZ;  dA_i = X^T @ dY_i
  *   (weight gradients per shard, no exchange);  dX = sum_i dY_i @ A_i^T (the

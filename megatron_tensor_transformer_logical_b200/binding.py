@@ -28,7 +28,8 @@ KIND_NAMES = {TP_KIND_GEMM_TCGEN05: "gemm_tcgen05", TP_KIND_GEMM_SIMT: "gemm_sim
 
 EXPORTS = ("tp_linear_col", "tp_linear_row", "tp_mlp_fwd", "tp_mlp_bwd", "tp_attn_fwd",
            "tp_attn_bwd", "tp_workspace_size", "tp_last_error", "tp_device_status",
-           "tp_version", "tp_profile_enable", "tp_profile_read", "tp_launch_count")
+           "tp_version", "tp_profile_enable", "tp_profile_read", "tp_launch_count",
+           "tp_mlp_fwd_noalloc")
 
 
 class ProfileStats(ctypes.Structure):
@@ -58,6 +59,7 @@ def load() -> ctypes.CDLL:
     L.tp_linear_col.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, vp]
     L.tp_linear_row.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, vp]
     L.tp_mlp_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, sz, vp]
+    L.tp_mlp_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp]
     L.tp_mlp_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32,
                              i32, vp, sz, vp]
     L.tp_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32,
@@ -132,6 +134,15 @@ def tp_mlp_fwd(X, A, bA, B, bB, Z, Ysave, t: int, ws, stream=None) -> None:
     _check(load().tp_mlp_fwd(_ptr(X), _ptr(A), _ptr(bA), _ptr(B), _ptr(bB), _ptr(Z),
                              _ptr(Ysave), M, h, f, t, _dtype(X), _ptr(ws),
                              ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def tp_mlp_fwd_noalloc(X, A, bA, B, bB, Z, Ysave, t: int, stream=None) -> None:
+    """tp_mlp_fwd with its intermediate in libtp's fixed 64 MiB device array:
+    for callers that cannot allocate a workspace (see include/libtp.h)."""
+    M, h = X.shape
+    f = A.shape[1]
+    _check(load().tp_mlp_fwd_noalloc(_ptr(X), _ptr(A), _ptr(bA), _ptr(B), _ptr(bB), _ptr(Z),
+                                     _ptr(Ysave), M, h, f, t, _dtype(X), _stream(stream)))
 
 
 def tp_mlp_bwd(X, A, bA, B, Ysave, dZ, dX, dA, dbA, dB, dbB, t: int, ws, stream=None) -> None:
