@@ -33,6 +33,7 @@
 
 #include <cmath>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "ptx_sm100.cuh"
@@ -381,10 +382,221 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  __syncwarp();  // lane 0 of the producer / MMA warps rejoins its warp
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+
+// ------------------------------------------------------- two-SM (CTA pair)
+// The same GEMM on 256 x 256 output tiles computed by a pair of CTAs on two
+// SMs with tcgen05.mma.cta_group::2: each CTA loads 128 rows of the A tile
+// and 128 columns of the B tile (a plain TMA load into its own shared memory,
+// counted on the even CTA's barrier); one thread of the even CTA issues the
+// 256 x 256 x 16 MMAs; each CTA's tensor memory receives its 128 output rows.
+// Per SM this halves the B bytes pulled from L2 per FLOP.
+constexpr int kPairStages = 6;
+constexpr int kPairABytes = 128 * BK * 2;  // 16 KB: this CTA's half of A
+constexpr int kPairBBytes = 128 * BK * 2;  // 16 KB: this CTA's half of B
+constexpr int kPairSmemBytes = 1024 + kPairStages * (kPairABytes + kPairBBytes) + 256;
+constexpr int kPairTM = 256, kPairTN = 256;
+
+__device__ __forceinline__ TileCoord tile_coord_pair(int tile, const Args& a) {
+  const int band = a.group_m * a.n_tiles;
+  const int g = tile / band;
+  const int first_m = g * a.group_m;
+  const int gm = min(a.m_tiles - first_m, a.group_m);
+  const int local = tile - g * band;
+  const int mt = first_m + local % gm;
+  const int nt = local / gm;
+  TileCoord c;
+  c.m0 = mt * kPairTM;
+  if (a.n_shard > 0) {
+    const int sh = nt / a.n_tiles_per_shard;
+    const int j = nt - sh * a.n_tiles_per_shard;
+    c.n0 = sh * a.n_shard + j * kPairTN;
+    c.n_end = min(c.n0 + kPairTN, (sh + 1) * a.n_shard);
+  } else {
+    c.n0 = nt * kPairTN;
+    c.n_end = min(c.n0 + kPairTN, a.N);
+  }
+  return c;
+}
+
+template <bool A_KMAJ, bool B_KMAJ, int EPI, int OUT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmA,
+                           const __grid_constant__ CUtensorMap tmB, const Args args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kPairStages * kPairABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPairStages * kPairBBytes);
+  uint64_t* empty = full + kPairStages;
+  uint64_t* tfull = empty + kPairStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs, 1: its peer
+  const uint32_t peer = rank ^ 1u;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 2 * kEpiWarps);  // both CTAs' epilogue warps
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers initialised and tensor memory allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = args.m_tiles * args.n_tiles;
+  const int cluster_id = static_cast<int>(blockIdx.x >> 1);
+  const int num_clusters = static_cast<int>(gridDim.x >> 1);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+        const TileCoord tc = tile_coord_pair(tile, args);
+        const int am0 = tc.m0 + 128 * static_cast<int>(rank);
+        const int bn0 = tc.n0 + 128 * static_cast<int>(rank);
+        for (int kb = 0; kb < args.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, args.status, kStatusProducerTimeout)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (kPairABytes + kPairBBytes));
+          const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+          const int kc = k_coord(kb, args);
+          uint8_t* a_dst = sA + stage * kPairABytes;
+          uint8_t* b_dst = sB + stage * kPairBBytes;
+          if (A_KMAJ) {
+            tma_load_2d_pair(a_dst, &tmA, bar, kc, am0);
+          } else {
+            tma_load_2d_pair(a_dst, &tmA, bar, am0, kc);
+            tma_load_2d_pair(a_dst + BK * 128, &tmA, bar, am0 + 64, kc);
+          }
+          if (B_KMAJ) {
+            tma_load_2d_pair(b_dst, &tmB, bar, kc, bn0);
+          } else {
+            tma_load_2d_pair(b_dst, &tmB, bar, bn0, kc);
+            tma_load_2d_pair(b_dst + BK * 128, &tmB, bar, bn0 + 64, kc);
+          }
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------- MMA issuer (even CTA only)
+      constexpr uint32_t kIdesc = idesc_bf16_f32(kPairTM, kPairTN, !A_KMAJ, !B_KMAJ);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.status, kStatusMmaTimeout)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kPairTN);
+        for (int kb = 0; kb < args.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, args.status, kStatusMmaTimeout)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * kPairABytes);
+          const uint32_t b0 = smem_u32(sB + stage * kPairBBytes);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = A_KMAJ ? sw128_desc(a0 + k * 32, 16, 1024)
+                                       : sw128_desc(a0 + k * 2048, BK * 128, 1024);
+            const uint64_t bd = B_KMAJ ? sw128_desc(b0 + k * 32, 16, 1024)
+                                       : sw128_desc(b0 + k * 2048, BK * 128, 1024);
+            umma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          // Free the stage in both CTAs once these MMAs have read it.
+          umma_commit_pair(mapa_shared(smem_u32(&empty[stage]), 0));
+          umma_commit_pair(mapa_shared(smem_u32(&empty[stage]), 1));
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(mapa_shared(smem_u32(&tfull[acc]), 0));
+        umma_commit_pair(mapa_shared(smem_u32(&tfull[acc]), 1));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp >= kFirstEpiWarp) {
+    // ------------------------------------------------ epilogue (both CTAs)
+    const int ew = warp - kFirstEpiWarp;
+    const int quarter = warp & 3;
+    const int half = ew >> 2;
+    const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0),
+                                       mapa_shared(smem_u32(&tempty[1]), 0)};
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cluster_id; tile < num_tiles; tile += num_clusters) {
+      const TileCoord tc = tile_coord_pair(tile, args);
+      if (!mbar_wait(&tfull[acc], acc_phase, args.status, kStatusEpilogueTimeout)) break;
+      tc_fence_after();
+      const int row = tc.m0 + 128 * static_cast<int>(rank) + quarter * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < kPairTN / 2; c += 32) {
+        const int cl = half * (kPairTN / 2) + c;
+        if (tc.n0 + cl >= tc.n_end) break;  // warp-uniform
+        float v[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                      static_cast<uint32_t>(acc * kPairTN + cl),
+                  v);
+        epilogue_row32<EPI, OUT, false>(v, row, tc.n0 + cl, tc.n_end, args);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  (void)peer;
+
+  __syncwarp();  // lane 0 of the producer / MMA warps rejoins its warp
+  tc_fence_before();
+  cluster_sync();  // no CTA frees tensor memory while its pair may still use it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
 }
 
 // ------------------------------------------------------------------ host side
@@ -441,11 +653,18 @@ Plan plan_for(const Gemm& g, int bn) {
 
 // Picks the column tile: 256 wide unless the 128-wide grid fills the SMs in
 // markedly fewer waves (128-wide tiles run at ~85% of the 256-wide rate).
+// Tile override for tests and tuning: TP_GEMM_TILE = 128 | 256 | pair.
+int tile_override() {
+  const char* e = std::getenv("TP_GEMM_TILE");
+  if (e == nullptr) return 0;
+  if (std::strcmp(e, "pair") == 0) return 512;
+  const int v = std::atoi(e);
+  return (v == 128 || v == 256) ? v : 0;
+}
+
 int choose_bn(const Gemm& g) {
-  if (const char* e = std::getenv("TP_GEMM_BN")) {
-    const int v = std::atoi(e);
-    if (v == 128 || v == 256) return v;
-  }
+  const int ov = tile_override();
+  if (ov == 128 || ov == 256) return ov;
   const int sms = sm_count();
   const Plan p256 = plan_for(g, 256), p128 = plan_for(g, 128);
   const double w256 = std::ceil(double(p256.m_tiles) * p256.n_tiles / sms);
@@ -541,6 +760,115 @@ tp_status dispatch(const Gemm& g, cudaStream_t s) {
   return fail(TP_ERR_UNSUPPORTED, "gemm: operand layout / epilogue combination not built");
 }
 
+
+template <bool AK, bool BKM, int EPI, int OUT>
+tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  const bool ok_a = AK ? make_map(&ta, g.a.ptr, g.K, g.M, g.a.ld, BK, 128)
+                       : make_map(&ta, g.a.ptr, g.M, g.K, g.a.ld, 64, BK);
+  const bool ok_b = BKM ? make_map(&tb, g.b.ptr, g.K, g.N, g.b.ld, BK, 128)
+                        : make_map(&tb, g.b.ptr, g.N, g.K, g.b.ld, 64, BK);
+  if (!ok_a || !ok_b) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  const Plan p = plan_for(g, kPairTN);
+  Args a;
+  a.M = static_cast<int>(g.M);
+  a.N = static_cast<int>(g.N);
+  a.K = static_cast<int>(g.K);
+  a.m_tiles = static_cast<int>((g.M + kPairTM - 1) / kPairTM);
+  a.n_tiles = p.n_tiles;
+  a.k_blocks = static_cast<int>((g.K + BK - 1) / BK);
+  a.group_m = 8;
+  a.n_shard = static_cast<int>(g.n_shard);
+  a.n_tiles_per_shard = p.n_tiles_per_shard;
+  a.kr_range_blocks = g.korder.range_blocks;
+  a.kr_t = g.korder.t;
+  a.kr_width = g.korder.width;
+  a.kr_h = g.korder.h;
+  a.out = g.out;
+  a.ldo = g.ldo;
+  a.bias = g.bias;
+  a.out2 = static_cast<__nv_bfloat16*>(g.out2);
+  a.ldo2 = g.ldo2;
+  a.aux = static_cast<const __nv_bfloat16*>(g.aux);
+  a.ldaux = g.ldaux;
+  a.status = device_status_ptr();
+  if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
+
+  auto kern = gemm_bf16_tcgen05_pair<AK, BKM, EPI, OUT>;
+  static int configured_mask = 0;
+  static int max_clusters[32] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(configured_mask & (1 << (dev & 31)))) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = sm_count() / 2;
+    }
+    max_clusters[dev & 31] = n;
+    configured_mask |= 1 << (dev & 31);
+  }
+  const long long tiles = static_cast<long long>(a.m_tiles) * a.n_tiles;
+  if (tiles == 0) return TP_OK;
+  const int mc = max_clusters[dev & 31];
+  const int clusters = static_cast<int>(tiles < mc ? tiles : mc);
+  const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
+  const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
+                       (OUT == kOutF32 ? 4.0 : 2.0) * double(g.M) * g.N +
+                       (g.out2 ? 2.0 * double(g.M) * g.N : 0.0) +
+                       (g.aux ? 2.0 * double(g.M) * g.N : 0.0);
+  {
+    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream);
+    kern<<<2 * clusters, kThreads, kPairSmemBytes, stream>>>(ta, tb, a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "gemm_bf16_tcgen05_pair launch");
+  return TP_OK;
+}
+
+template <bool AK, bool BKM, int EPI>
+tp_status pair_by_out(const Gemm& g, cudaStream_t s) {
+  if (g.out_f32) return launch_pair<AK, BKM, EPI, kOutF32>(g, s);
+  if (g.out_f16) return launch_pair<AK, BKM, EPI, kOutF16>(g, s);
+  return launch_pair<AK, BKM, EPI, kOutBF16>(g, s);
+}
+
+tp_status dispatch_pair(const Gemm& g, cudaStream_t s) {
+  const bool ak = g.a.k_major, bk = g.b.k_major;
+  const bool plain_out = !g.out_f32 && !g.out_f16;
+  if (g.epi == kEpiBiasGelu) {
+    if (ak && !bk && plain_out) return launch_pair<true, false, kEpiBiasGelu, kOutBF16>(g, s);
+  } else if (g.epi == kEpiDGelu) {
+    if (ak && bk && plain_out) return launch_pair<true, true, kEpiDGelu, kOutBF16>(g, s);
+  } else {
+    if (ak && !bk) return pair_by_out<true, false, kEpiStore>(g, s);
+    if (ak && bk) return pair_by_out<true, true, kEpiStore>(g, s);
+    if (!ak && !bk && !g.out_f16) {
+      return g.out_f32 ? launch_pair<false, false, kEpiStore, kOutF32>(g, s)
+                       : launch_pair<false, false, kEpiStore, kOutBF16>(g, s);
+    }
+  }
+  return fail(TP_ERR_UNSUPPORTED, "gemm: operand layout / epilogue combination not built");
+}
+
+// The pair kernel wherever its 256 x 256 tiles fill at least one wave of
+// SM pairs; the single-SM kernel for smaller problems.
+bool use_pair(const Gemm& g) {
+  const int ov = tile_override();
+  if (ov == 512) return true;
+  if (ov != 0) return false;
+  const Plan p = plan_for(g, kPairTN);
+  const long long tiles = ((g.M + kPairTM - 1) / kPairTM) * static_cast<long long>(p.n_tiles);
+  return tiles >= sm_count() / 2;
+}
+
 }  // namespace
 
 tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream) {
@@ -560,6 +888,7 @@ tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream) {
   // stores whole groups of 8 columns, so other shard widths tile plainly
   // (every column is still computed by the same K loop).
   if (gg.n_shard > 0 && (gg.n_shard % 8 != 0 || gg.N % gg.n_shard != 0)) gg.n_shard = 0;
+  if (use_pair(gg)) return dispatch_pair(gg, stream);
   return choose_bn(gg) == 128 ? dispatch<128>(gg, stream) : dispatch<256>(gg, stream);
 }
 

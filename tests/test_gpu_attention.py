@@ -53,9 +53,12 @@ def compare_full(out, inp, wl, causal):
         check(out[k], bw[k], k, "bf16")
 
 
+@pytest.mark.parametrize("tile", ["auto", "pair"])
 @pytest.mark.parametrize("causal", [True, False], ids=["causal", "full"])
 @pytest.mark.parametrize("save_qkv", [True, False], ids=["QKVsave", "recompute"])
-def test_attention_small_ragged(causal, save_qkv):
+def test_attention_small_ragged(monkeypatch, causal, save_qkv, tile):
+    if tile != "auto":
+        monkeypatch.setenv("TP_GEMM_TILE", tile)
     # s = 200: four 64-row query blocks (the last ragged), seven 32-row blocks.
     wl = Workload(80, "attn ragged", b=2, s=200, h=512, heads=4, t=2, w_std=0.05)
     inp = make_attn_inputs(wl)

@@ -37,17 +37,19 @@ def run(mode, X, W, b, t, shard=-1, out_dtype=torch.bfloat16):
     return Y
 
 
-# M spans 3 row tiles with a ragged tail, N 3 column tiles of 256 (ragged),
-# K 5 blocks of 64; every K/t and N/t is a multiple of 8.
+# M spans 3 row tiles of 128 (2 pair tiles of 256) with a ragged tail, N 3
+# column tiles of 256 (ragged), K 5 blocks of 64; every K/t and N/t is a
+# multiple of 8.  TP_GEMM_TILE forces the 128- or 256-wide single-SM tile or
+# the 256 x 256 two-SM tile.
 SMALL = (300, 320, 576)
 
 
-@pytest.mark.parametrize("bn", ["128", "256"])
+@pytest.mark.parametrize("tile", ["128", "256", "pair"])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
 @pytest.mark.parametrize("t", [1, 2, 4, 8])
 @pytest.mark.parametrize("mode", ["col", "row"])
-def test_linear_random_small(monkeypatch, mode, t, out_dtype, bn):
-    monkeypatch.setenv("TP_GEMM_BN", bn)
+def test_linear_random_small(monkeypatch, mode, t, out_dtype, tile):
+    monkeypatch.setenv("TP_GEMM_TILE", tile)
     M, K, N = SMALL
     X, W = normal_tensor((M, K), 1.0, 1), normal_tensor((K, N), 0.05, 2)
     b = normal_tensor((N,), 0.1, 3)
@@ -59,11 +61,11 @@ def test_linear_random_small(monkeypatch, mode, t, out_dtype, bn):
         check(Y, ref, f"{mode} t={t}", "bf16")
 
 
-@pytest.mark.parametrize("bn", ["128", "256"])
+@pytest.mark.parametrize("tile", ["128", "256", "pair"])
 @pytest.mark.parametrize("t", [1, 2, 4, 8])
 @pytest.mark.parametrize("mode", ["col", "row"])
-def test_linear_integer_bit_exact(monkeypatch, mode, t, bn):
-    monkeypatch.setenv("TP_GEMM_BN", bn)
+def test_linear_integer_bit_exact(monkeypatch, mode, t, tile):
+    monkeypatch.setenv("TP_GEMM_TILE", tile)
     M, K, N = SMALL
     X, W = integer_tensor((M, K), -3, 3, 4), integer_tensor((K, N), -3, 3, 5)
     b = integer_tensor((N,), -8, 8, 6)
@@ -71,8 +73,10 @@ def test_linear_integer_bit_exact(monkeypatch, mode, t, bn):
     assert np.array_equal(to64(Y), O.linear(X, W, b))
 
 
+@pytest.mark.parametrize("tile", ["256", "pair"])
 @pytest.mark.parametrize("t", [2, 4, 8])
-def test_column_shard_slices_bit_exact(t):
+def test_column_shard_slices_bit_exact(monkeypatch, t, tile):
+    monkeypatch.setenv("TP_GEMM_TILE", tile)
     M, K, N = SMALL
     X, W = cuda(normal_tensor((M, K), 1.0, 7)), cuda(normal_tensor((K, N), 0.05, 8))
     b = cuda(normal_tensor((N,), 0.1, 9))
@@ -84,8 +88,10 @@ def test_column_shard_slices_bit_exact(t):
             assert torch.equal(part, full[:, i * w:(i + 1) * w]), (t, i)
 
 
+@pytest.mark.parametrize("tile", ["256", "pair"])
 @pytest.mark.parametrize("t", [2, 4, 8])
-def test_row_shard_partials_sum_to_full(t):
+def test_row_shard_partials_sum_to_full(monkeypatch, t, tile):
+    monkeypatch.setenv("TP_GEMM_TILE", tile)
     M, K, N = SMALL
     X, W = integer_tensor((M, K), -3, 3, 10), integer_tensor((K, N), -3, 3, 11)
     b = integer_tensor((N,), -8, 8, 12)

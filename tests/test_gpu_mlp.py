@@ -62,8 +62,11 @@ def test_mlp_config1_fp32():
     compare_full(out, inp, "f32")
 
 
+@pytest.mark.parametrize("tile", ["auto", "256", "pair"])
 @pytest.mark.parametrize("save_y", [True, False], ids=["Ysave", "recompute"])
-def test_mlp_ragged_bf16(save_y):
+def test_mlp_ragged_bf16(monkeypatch, save_y, tile):
+    if tile != "auto":
+        monkeypatch.setenv("TP_GEMM_TILE", tile)
     # 200 rows (two row tiles, ragged), h=136, f=544: ragged column and K tails.
     wl = Workload(90, "ragged", b=1, s=200, h=136, f=544, t=4, w_std=0.05, bias_std=0.05)
     inp = make_mlp_inputs(wl)
