@@ -231,6 +231,7 @@ def run_libtp(args, rank, world, local_rank, dist):
     t1 = time.time()
     launches = L.tp_launch_count() - n0
     prof = {name: L.tp_profile_read(k) for k, name in L.KIND_NAMES.items()}
+    records = L.tp_profile_records()
     L.tp_profile_enable(False)
     barrier()
     clocks = sampler.stop(t0, t1) if sampler else None
@@ -291,6 +292,18 @@ def run_libtp(args, rank, world, local_rank, dist):
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     traffic = traffic_per_launch()
     mlp_tflops = world * (fl["mlp_fwd"] + fl["mlp_bwd"]) / (mlp_ms / args.steps * 1e-3) / 1e12
+    gemms = {}
+    for r in records:
+        if r["kind"] != "gemm_tcgen05":
+            continue
+        key = f'{r["m"]}x{r["n"]}x{r["k"]}'
+        g_ = gemms.setdefault(key, {"tile": r["tile"], "ms": 0.0, "flops": 0.0, "n": 0})
+        g_["ms"] += r["ms"]
+        g_["flops"] += r["flops"]
+        g_["n"] += 1
+    gemm_shapes = {k: {"tile": v["tile"], "ms_per_launch": round(v["ms"] / v["n"], 4),
+                       "tflops": round(v["flops"] / (v["ms"] * 1e-3) / 1e12, 1)}
+                   for k, v in gemms.items()}
     kernels = {}
     for name, p in prof.items():
         if p["launches"]:
@@ -329,6 +342,7 @@ def run_libtp(args, rank, world, local_rank, dist):
                      "algorithmic_bytes_per_launch": (g["bytes"] / g["launches"]) if g["launches"] else None,
                      "flops_per_launch": (g["flops"] / g["launches"]) if g["launches"] else None},
         "kernels": kernels,
+        "gemm_shapes": gemm_shapes,
         "gpu_launches": launches,
         "clocks": clocks,
     }

@@ -236,6 +236,21 @@ tp_status tp_profile_read(tp_kernel_kind kind, tp_profile_stats* out);
 /* Kernels launched by libtp since the library was loaded. */
 int64_t tp_launch_count(void);
 
+/* One traced launch (or launch group) recorded while profiling was on. */
+typedef struct tp_launch_record {
+  int kind;            /* tp_kernel_kind                                        */
+  int tile;            /* GEMM tile: 128/192/256 columns on one SM, 512 = 256x256 */
+                       /* on an SM pair; 0 for other kernels                    */
+  int64_t m, n, k;     /* GEMM problem size (0 for other kernels)               */
+  double ms;           /* event-timed duration                                  */
+  double flops, bytes; /* algorithmic work                                      */
+} tp_launch_record;
+
+/* Records taken since profiling was last turned on. */
+int64_t tp_profile_count(void);
+/* Synchronizes on record `index`'s events and fills *out. */
+tp_status tp_profile_record(int64_t index, tp_launch_record* out);
+
 /* Message for the last non-TP_OK status returned on this host thread. */
 const char* tp_last_error(void);
 

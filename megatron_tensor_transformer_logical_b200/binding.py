@@ -29,7 +29,13 @@ KIND_NAMES = {TP_KIND_GEMM_TCGEN05: "gemm_tcgen05", TP_KIND_GEMM_SIMT: "gemm_sim
 EXPORTS = ("tp_linear_col", "tp_linear_row", "tp_mlp_fwd", "tp_mlp_bwd", "tp_attn_fwd",
            "tp_attn_bwd", "tp_workspace_size", "tp_last_error", "tp_device_status",
            "tp_version", "tp_profile_enable", "tp_profile_read", "tp_launch_count",
-           "tp_mlp_fwd_noalloc")
+           "tp_mlp_fwd_noalloc", "tp_profile_count", "tp_profile_record")
+
+
+class LaunchRecord(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("tile", ctypes.c_int), ("m", ctypes.c_int64),
+                ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
 class ProfileStats(ctypes.Structure):
@@ -75,8 +81,12 @@ def load() -> ctypes.CDLL:
     L.tp_profile_enable.argtypes = [i32]
     L.tp_profile_read.argtypes = [i32, ctypes.POINTER(ProfileStats)]
     L.tp_launch_count.argtypes = []
+    L.tp_profile_count.argtypes = []
+    L.tp_profile_count.restype = ctypes.c_int64
+    L.tp_profile_record.argtypes = [ctypes.c_int64, ctypes.POINTER(LaunchRecord)]
     for name in EXPORTS:
-        if name not in ("tp_workspace_size", "tp_last_error", "tp_launch_count"):
+        if name not in ("tp_workspace_size", "tp_last_error", "tp_launch_count",
+                        "tp_profile_count"):
             getattr(L, name).restype = ctypes.c_int
     L.tp_launch_count.restype = ctypes.c_int64
     _lib = L
@@ -192,6 +202,18 @@ def tp_profile_read(kind: int) -> dict:
 
 def tp_launch_count() -> int:
     return int(load().tp_launch_count())
+
+
+def tp_profile_records() -> list:
+    """Every launch recorded since profiling was turned on, as dicts."""
+    L = load()
+    out = []
+    for i in range(int(L.tp_profile_count())):
+        r = LaunchRecord()
+        _check(L.tp_profile_record(i, ctypes.byref(r)))
+        out.append({"kind": KIND_NAMES.get(r.kind, str(r.kind)), "tile": r.tile, "m": r.m,
+                    "n": r.n, "k": r.k, "ms": r.ms, "flops": r.flops, "bytes": r.bytes})
+    return out
 
 
 def workspace(op: int, M: int, h: int, f: int, heads: int, t: int, dtype: int,

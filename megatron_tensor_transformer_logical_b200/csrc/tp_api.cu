@@ -70,6 +70,8 @@ struct ProfRecord {
   cudaEvent_t start = nullptr, stop = nullptr;
   tp_kernel_kind kind = TP_KIND_GEMM_TCGEN05;
   double flops = 0, bytes = 0;
+  int tile = 0;
+  int64_t m = 0, n = 0, k = 0;
 };
 std::mutex g_prof_mu;
 bool g_prof_on = false;
@@ -79,7 +81,7 @@ std::atomic<int64_t> g_launches{0};
 }  // namespace
 
 LaunchScope::LaunchScope(tp_kernel_kind kind, double flops, double bytes, cudaStream_t stream,
-                         int kernels)
+                         int kernels, int tile, int64_t m, int64_t n, int64_t k)
     : stream_(stream) {
   g_launches.fetch_add(kernels, std::memory_order_relaxed);
   std::lock_guard<std::mutex> lock(g_prof_mu);
@@ -94,6 +96,10 @@ LaunchScope::LaunchScope(tp_kernel_kind kind, double flops, double bytes, cudaSt
   r.kind = kind;
   r.flops = flops;
   r.bytes = bytes;
+  r.tile = tile;
+  r.m = m;
+  r.n = n;
+  r.k = k;
   if (cudaEventRecord(r.start, stream) != cudaSuccess) return;
   slot_ = static_cast<int>(g_prof_used++);
 }
@@ -644,6 +650,37 @@ tp_status tp_profile_read(tp_kernel_kind kind, tp_profile_stats* out) {
 }
 
 int64_t tp_launch_count(void) { return g_launches.load(); }
+
+int64_t tp_profile_count(void) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  return static_cast<int64_t>(g_prof_used);
+}
+
+tp_status tp_profile_record(int64_t index, tp_launch_record* out) {
+  try {
+    if (out == nullptr) return fail(TP_ERR_NULL, "out is required");
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    if (index < 0 || static_cast<size_t>(index) >= g_prof_used)
+      return fail(TP_ERR_SHAPE, "no such launch record");
+    const ProfRecord& r = g_prof[static_cast<size_t>(index)];
+    cudaError_t e = cudaEventSynchronize(r.stop);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+    float ms = 0.0f;
+    e = cudaEventElapsedTime(&ms, r.start, r.stop);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+    out->kind = r.kind;
+    out->tile = r.tile;
+    out->m = r.m;
+    out->n = r.n;
+    out->k = r.k;
+    out->ms = ms;
+    out->flops = r.flops;
+    out->bytes = r.bytes;
+    return TP_OK;
+  } catch (...) {
+    return fail(TP_ERR_UNSUPPORTED, "internal error");
+  }
+}
 
 int tp_version(void) { return 100; }
 

@@ -50,10 +50,10 @@ constexpr int kFirstEpiWarp = 4;
 
 template <int BN>
 struct Cfg {
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kStages = (BN == 256) ? 4 : (BN == 192 ? 5 : 6);
   static constexpr int kABytes = BM * BK * 2;
   static constexpr int kBBytes = BN * BK * 2;
-  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kTmemCols = (2 * BN > 256) ? 512 : 256;  // a power of two
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kBarBytes;
 };
@@ -651,25 +651,41 @@ Plan plan_for(const Gemm& g, int bn) {
   return p;
 }
 
-// Picks the column tile: 256 wide unless the 128-wide grid fills the SMs in
-// markedly fewer waves (128-wide tiles run at ~85% of the 256-wide rate).
 // Tile override for tests and tuning: TP_GEMM_TILE = 128 | 256 | pair.
 int tile_override() {
   const char* e = std::getenv("TP_GEMM_TILE");
   if (e == nullptr) return 0;
   if (std::strcmp(e, "pair") == 0) return 512;
   const int v = std::atoi(e);
-  return (v == 128 || v == 256) ? v : 0;
+  return (v == 128 || v == 192 || v == 256) ? v : 0;
 }
 
-int choose_bn(const Gemm& g) {
+// Tile kind: 128, 192 or 256 columns on one SM, or 512 = 256 x 256 on an SM
+// pair.  Picks the least estimated time, ceil(tiles / slots) x work per tile
+// / relative rate; the rates (per-clock throughput of each tile kind
+// relative to the 256-wide single-SM tile) were measured on the 175B-shaped
+// layer's GEMMs.  Narrower tiles win where they fill the last wave better.
+int choose_tile(const Gemm& g) {
   const int ov = tile_override();
-  if (ov == 128 || ov == 256) return ov;
-  const int sms = sm_count();
-  const Plan p256 = plan_for(g, 256), p128 = plan_for(g, 128);
-  const double w256 = std::ceil(double(p256.m_tiles) * p256.n_tiles / sms);
-  const double w128 = std::ceil(double(p128.m_tiles) * p128.n_tiles / sms);
-  return (w128 * 0.5 / 0.85 < w256 * 0.98) ? 128 : 256;
+  if (ov != 0) return ov;
+  const double sms = sm_count();
+  double best = 1e300;
+  int kind = 256;
+  const int widths[3] = {256, 192, 128};
+  const double rate[3] = {1.0, 0.985, 0.88};
+  for (int i = 0; i < 3; ++i) {
+    const Plan p = plan_for(g, widths[i]);
+    const double t = std::ceil(double(p.m_tiles) * p.n_tiles / sms) * 128.0 * widths[i] / rate[i];
+    if (t < best * 0.999) {
+      best = t;
+      kind = widths[i];
+    }
+  }
+  const Plan pp = plan_for(g, kPairTN);
+  const double pair_tiles = double((g.M + kPairTM - 1) / kPairTM) * pp.n_tiles;
+  const double tp = std::ceil(pair_tiles / std::floor(sms / 2)) * 256.0 * 256.0 / 2.0 / 1.0;
+  if (tp < best * 0.999) kind = 512;
+  return kind;
 }
 
 template <int BN, bool AK, bool BKM, int EPI, int OUT>
@@ -726,7 +742,7 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
                        (g.out2 ? 2.0 * double(g.M) * g.N : 0.0) +
                        (g.aux ? 2.0 * double(g.M) * g.N : 0.0);
   {
-    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream);
+    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, 1, BN, g.M, g.N, g.K);
     kern<<<grid, kThreads, C::kSmemBytes, stream>>>(ta, tb, a);
   }
   cudaError_t e = cudaGetLastError();
@@ -825,7 +841,7 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
                        (g.out2 ? 2.0 * double(g.M) * g.N : 0.0) +
                        (g.aux ? 2.0 * double(g.M) * g.N : 0.0);
   {
-    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream);
+    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, 1, 512, g.M, g.N, g.K);
     kern<<<2 * clusters, kThreads, kPairSmemBytes, stream>>>(ta, tb, a);
   }
   cudaError_t e = cudaGetLastError();
@@ -858,17 +874,6 @@ tp_status dispatch_pair(const Gemm& g, cudaStream_t s) {
   return fail(TP_ERR_UNSUPPORTED, "gemm: operand layout / epilogue combination not built");
 }
 
-// The pair kernel wherever its 256 x 256 tiles fill at least one wave of
-// SM pairs; the single-SM kernel for smaller problems.
-bool use_pair(const Gemm& g) {
-  const int ov = tile_override();
-  if (ov == 512) return true;
-  if (ov != 0) return false;
-  const Plan p = plan_for(g, kPairTN);
-  const long long tiles = ((g.M + kPairTM - 1) / kPairTM) * static_cast<long long>(p.n_tiles);
-  return tiles >= sm_count() / 2;
-}
-
 }  // namespace
 
 tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream) {
@@ -888,8 +893,12 @@ tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream) {
   // stores whole groups of 8 columns, so other shard widths tile plainly
   // (every column is still computed by the same K loop).
   if (gg.n_shard > 0 && (gg.n_shard % 8 != 0 || gg.N % gg.n_shard != 0)) gg.n_shard = 0;
-  if (use_pair(gg)) return dispatch_pair(gg, stream);
-  return choose_bn(gg) == 128 ? dispatch<128>(gg, stream) : dispatch<256>(gg, stream);
+  switch (choose_tile(gg)) {
+    case 512: return dispatch_pair(gg, stream);
+    case 128: return dispatch<128>(gg, stream);
+    case 192: return dispatch<192>(gg, stream);
+    default: return dispatch<256>(gg, stream);
+  }
 }
 
 }  // namespace tp

@@ -25,8 +25,9 @@ int sm_count();
 class LaunchScope {
  public:
   // `kernels`: how many kernels the bracketed region launches.
+  // `tile`, m, n, k describe a GEMM launch for the per-launch trace.
   LaunchScope(tp_kernel_kind kind, double flops, double bytes, cudaStream_t stream,
-              int kernels = 1);
+              int kernels = 1, int tile = 0, int64_t m = 0, int64_t n = 0, int64_t k = 0);
   ~LaunchScope();
   LaunchScope(const LaunchScope&) = delete;
   LaunchScope& operator=(const LaunchScope&) = delete;

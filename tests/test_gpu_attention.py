@@ -53,7 +53,7 @@ def compare_full(out, inp, wl, causal):
         check(out[k], bw[k], k, "bf16")
 
 
-@pytest.mark.parametrize("tile", ["auto", "pair"])
+@pytest.mark.parametrize("tile", ["auto", "192", "pair"])
 @pytest.mark.parametrize("causal", [True, False], ids=["causal", "full"])
 @pytest.mark.parametrize("save_qkv", [True, False], ids=["QKVsave", "recompute"])
 def test_attention_small_ragged(monkeypatch, causal, save_qkv, tile):

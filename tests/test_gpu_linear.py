@@ -39,12 +39,12 @@ def run(mode, X, W, b, t, shard=-1, out_dtype=torch.bfloat16):
 
 # M spans 3 row tiles of 128 (2 pair tiles of 256) with a ragged tail, N 3
 # column tiles of 256 (ragged), K 5 blocks of 64; every K/t and N/t is a
-# multiple of 8.  TP_GEMM_TILE forces the 128- or 256-wide single-SM tile or
+# multiple of 8.  TP_GEMM_TILE forces the 128-, 192- or 256-wide single-SM tile or
 # the 256 x 256 two-SM tile.
 SMALL = (300, 320, 576)
 
 
-@pytest.mark.parametrize("tile", ["128", "256", "pair"])
+@pytest.mark.parametrize("tile", ["128", "192", "256", "pair"])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
 @pytest.mark.parametrize("t", [1, 2, 4, 8])
 @pytest.mark.parametrize("mode", ["col", "row"])
@@ -61,7 +61,7 @@ def test_linear_random_small(monkeypatch, mode, t, out_dtype, tile):
         check(Y, ref, f"{mode} t={t}", "bf16")
 
 
-@pytest.mark.parametrize("tile", ["128", "256", "pair"])
+@pytest.mark.parametrize("tile", ["128", "192", "256", "pair"])
 @pytest.mark.parametrize("t", [1, 2, 4, 8])
 @pytest.mark.parametrize("mode", ["col", "row"])
 def test_linear_integer_bit_exact(monkeypatch, mode, t, tile):
@@ -73,7 +73,7 @@ def test_linear_integer_bit_exact(monkeypatch, mode, t, tile):
     assert np.array_equal(to64(Y), O.linear(X, W, b))
 
 
-@pytest.mark.parametrize("tile", ["256", "pair"])
+@pytest.mark.parametrize("tile", ["192", "256", "pair"])
 @pytest.mark.parametrize("t", [2, 4, 8])
 def test_column_shard_slices_bit_exact(monkeypatch, t, tile):
     monkeypatch.setenv("TP_GEMM_TILE", tile)

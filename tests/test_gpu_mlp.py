@@ -62,7 +62,7 @@ def test_mlp_config1_fp32():
     compare_full(out, inp, "f32")
 
 
-@pytest.mark.parametrize("tile", ["auto", "256", "pair"])
+@pytest.mark.parametrize("tile", ["auto", "192", "256", "pair"])
 @pytest.mark.parametrize("save_y", [True, False], ids=["Ysave", "recompute"])
 def test_mlp_ragged_bf16(monkeypatch, save_y, tile):
     if tile != "auto":
