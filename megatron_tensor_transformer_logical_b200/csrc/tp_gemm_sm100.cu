@@ -662,9 +662,12 @@ int tile_override() {
 
 // Tile kind: 128, 192 or 256 columns on one SM, or 512 = 256 x 256 on an SM
 // pair.  Picks the least estimated time, ceil(tiles / slots) x work per tile
-// / relative rate; the rates (per-clock throughput of each tile kind
-// relative to the 256-wide single-SM tile) were measured on the 175B-shaped
-// layer's GEMMs.  Narrower tiles win where they fill the last wave better.
+// / relative rate.  The rates are per-clock throughputs relative to the
+// 256-wide single-SM tile, measured on the 175B-shaped layer's twelve GEMMs
+// under the sustained power cap: with A K-major and B MN-major (the forward
+// linears) the single-SM tile is ~5% faster than the pair; with B K-major
+// (dgrads) or both operands MN-major (wgrads) the pair is 4-10% faster; the
+// 192- and 128-wide tiles only pay where they fill the last wave far better.
 int choose_tile(const Gemm& g) {
   const int ov = tile_override();
   if (ov != 0) return ov;
@@ -672,7 +675,7 @@ int choose_tile(const Gemm& g) {
   double best = 1e300;
   int kind = 256;
   const int widths[3] = {256, 192, 128};
-  const double rate[3] = {1.0, 0.985, 0.88};
+  const double rate[3] = {1.0, 0.8, 0.8};
   for (int i = 0; i < 3; ++i) {
     const Plan p = plan_for(g, widths[i]);
     const double t = std::ceil(double(p.m_tiles) * p.n_tiles / sms) * 128.0 * widths[i] / rate[i];
@@ -681,9 +684,10 @@ int choose_tile(const Gemm& g) {
       kind = widths[i];
     }
   }
+  const double pair_rate = (g.a.k_major && !g.b.k_major) ? 0.95 : 1.07;
   const Plan pp = plan_for(g, kPairTN);
   const double pair_tiles = double((g.M + kPairTM - 1) / kPairTM) * pp.n_tiles;
-  const double tp = std::ceil(pair_tiles / std::floor(sms / 2)) * 256.0 * 256.0 / 2.0 / 1.0;
+  const double tp = std::ceil(pair_tiles / std::floor(sms / 2)) * 256.0 * 256.0 / 2.0 / pair_rate;
   if (tp < best * 0.999) kind = 512;
   return kind;
 }
