@@ -10,14 +10,12 @@
 // d = 128.  O [M, h] holds head j at columns j*d.  LSE [b, heads, s] is the
 // natural log of each row's softmax denominator.
 //
-// Forward: one CTA per (64 query rows, batch, head); 4 warps x 16 rows;
-// keys in blocks of 64 through a double-buffered cp.async pipeline; online
-// softmax (row max / sum in registers, quad shuffles); P stays in registers
-// as the A operand of P V.  Tensor-core work uses mma.sync m16n8k16 with fp16
-// operands and fp32 accumulation: Q, K, V, dO arrive in fp16 (written so by
-// the GEMMs that produce them) and P, dS are rounded to fp16 for the
-// products.  fp16 keeps three more mantissa bits than bf16, which halves the
-// backward's rounding error; O and dQKV are written in bf16 for the linears.
+// The forward runs on tcgen05 (tp_attention_sm100.cu).  The backward kernels
+// here use mma.sync m16n8k16 with fp16 operands and fp32 accumulation: Q, K,
+// V, dO arrive in fp16 (written so by the GEMMs that produce them) and P, dS
+// are rounded to fp16 for the products.  fp16 keeps three more mantissa bits
+// than bf16, which halves the backward's rounding error; dQKV is written in
+// bf16 for the linears.
 //
 // Backward, without atomics: D = rowsum(dO * O) per row and head; one kernel
 // per key block accumulates dK and dV over the query blocks that see it;
@@ -38,7 +36,6 @@ namespace {
 constexpr int D = 128;            // head dimension
 constexpr int ROW_BYTES = D * 2;  // 256 bytes per row of a [rows][128] bf16 tile
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.69314718055994531f;
 
 struct AttnArgs {
   const __half* qkv;         // [M, 3h] fp16
@@ -144,157 +141,6 @@ __device__ __forceinline__ void load_tile(uint32_t tile, const __half* base, lon
     const bool ok = gr < row_end;
     const __half* src = base + static_cast<long long>(ok ? gr : 0) * ld + col + c * 8;
     cp_async16(tile + swz(r, c), src, ok);
-  }
-}
-
-// ------------------------------------------------------------------ forward
-constexpr int FWD_BM = 64, FWD_BN = 64, FWD_THREADS = 128;
-constexpr int FWD_SMEM = (FWD_BM + 4 * FWD_BN) * ROW_BYTES;  // Q + 2 x (K, V)
-
-__global__ void __launch_bounds__(FWD_THREADS) attn_fwd_kernel(const AttnArgs a) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  const uint32_t sQ = saddr(sm);
-  const uint32_t sK[2] = {sQ + FWD_BM * ROW_BYTES, sQ + (FWD_BM + 2 * FWD_BN) * ROW_BYTES};
-  const uint32_t sV[2] = {sQ + (FWD_BM + FWD_BN) * ROW_BYTES,
-                          sQ + (FWD_BM + 3 * FWD_BN) * ROW_BYTES};
-
-  const int nqb = (a.s + FWD_BM - 1) / FWD_BM;
-  const int qb = nqb - 1 - static_cast<int>(blockIdx.x);  // longest rows first
-  const int head = blockIdx.y % a.heads, bi = blockIdx.y / a.heads;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long ld = 3LL * a.h;
-  const __half* base = a.qkv + static_cast<long long>(bi) * a.s * ld;
-  const int q0 = qb * FWD_BM;
-  const int n_kb = a.causal ? (min(q0 + FWD_BM, a.s) + FWD_BN - 1) / FWD_BN
-                            : (a.s + FWD_BN - 1) / FWD_BN;
-
-  load_tile<FWD_BM, FWD_THREADS>(sQ, base, ld, q0, a.s, head * D);
-  load_tile<FWD_BN, FWD_THREADS>(sK[0], base, ld, 0, a.s, a.h + head * D);
-  load_tile<FWD_BN, FWD_THREADS>(sV[0], base, ld, 0, a.s, 2 * a.h + head * D);
-  cp_commit();
-
-  float o[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-  float m_r[2] = {-INFINITY, -INFINITY};
-  float l_r[2] = {0.0f, 0.0f};
-  const int g = lane >> 2, tq = lane & 3;
-  const int row_a = q0 + warp * 16 + g;  // rows of c0/c1; c2/c3 at row_a + 8
-
-  for (int kb = 0; kb < n_kb; ++kb) {
-    const int buf = kb & 1;
-    if (kb + 1 < n_kb) {
-      load_tile<FWD_BN, FWD_THREADS>(sK[buf ^ 1], base, ld, (kb + 1) * FWD_BN, a.s,
-                                     a.h + head * D);
-      load_tile<FWD_BN, FWD_THREADS>(sV[buf ^ 1], base, ld, (kb + 1) * FWD_BN, a.s,
-                                     2 * a.h + head * D);
-      cp_commit();
-      cp_wait<1>();
-    } else {
-      cp_wait<0>();
-    }
-    __syncthreads();
-
-    // S = Q K^T for this warp's 16 rows x 64 keys.
-    float sc[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.0f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t af[4];
-      lda(sQ, warp * 16, kk, lane, af);
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) {
-        uint32_t bf[4];
-        ldb_nk(sK[buf], j * 8, kk, lane, bf);
-        mma16816(sc[j], af[0], af[1], af[2], af[3], bf[0], bf[1]);
-        mma16816(sc[j + 1], af[0], af[1], af[2], af[3], bf[2], bf[3]);
-      }
-    }
-    // Scale into the log2 domain, mask, and update the running max / sum.
-    const int k0 = kb * FWD_BN;
-    float mx[2] = {m_r[0], m_r[1]};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = k0 + j * 8 + 2 * tq + (e & 1);
-        const int row = row_a + ((e >> 1) << 3);
-        float v = sc[j][e] * a.scale_log2;
-        if (col >= a.s || (a.causal && col > row)) v = -INFINITY;
-        sc[j][e] = v;
-        mx[e >> 1] = fmaxf(mx[e >> 1], v);
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-    }
-    float corr[2], rs[2] = {0.0f, 0.0f};
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      corr[r] = (m_r[r] == -INFINITY) ? 0.0f : exp2f(m_r[r] - mx[r]);
-      m_r[r] = mx[r];
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float mm = m_r[e >> 1];
-        const float p = (mm == -INFINITY) ? 0.0f : exp2f(sc[j][e] - mm);
-        sc[j][e] = p;
-        rs[e >> 1] += p;
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 1);
-      rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 2);
-      l_r[r] = l_r[r] * corr[r] + rs[r];
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      o[i][0] *= corr[0];
-      o[i][1] *= corr[0];
-      o[i][2] *= corr[1];
-      o[i][3] *= corr[1];
-    }
-    // O += P V: P (16 x 64) from registers as four k16 A fragments.
-#pragma unroll
-    for (int kk = 0; kk < FWD_BN / 16; ++kk) {
-      const uint32_t a0 = pack_f16(sc[2 * kk][0], sc[2 * kk][1]);
-      const uint32_t a1 = pack_f16(sc[2 * kk][2], sc[2 * kk][3]);
-      const uint32_t a2 = pack_f16(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
-      const uint32_t a3 = pack_f16(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
-#pragma unroll
-      for (int n = 0; n < 16; n += 2) {
-        uint32_t bf[4];
-        ldb_kn(sV[buf], kk * 16, n * 8, lane, bf);
-        mma16816(o[n], a0, a1, a2, a3, bf[0], bf[1]);
-        mma16816(o[n + 1], a0, a1, a2, a3, bf[2], bf[3]);
-      }
-    }
-    __syncthreads();  // the buffer is refilled next iteration
-  }
-
-  // Normalise, store O and the natural-log LSE.
-  const float inv[2] = {l_r[0] > 0.0f ? 1.0f / l_r[0] : 0.0f, l_r[1] > 0.0f ? 1.0f / l_r[1] : 0.0f};
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int row = row_a + 8 * r;
-    if (row >= a.s) continue;
-    __nv_bfloat16* orow = a.out + (static_cast<long long>(bi) * a.s + row) * a.h + head * D;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      const int col = n * 8 + 2 * tq;
-      *reinterpret_cast<uint32_t*>(orow + col) =
-          pack_bf16(o[n][2 * r] * inv[r], o[n][2 * r + 1] * inv[r]);
-    }
-    if (tq == 0) {
-      a.lse_out[(static_cast<long long>(bi) * a.heads + head) * a.s + row] =
-          (m_r[r] + log2f(l_r[r])) * kLn2;
-    }
   }
 }
 
@@ -615,23 +461,7 @@ AttnArgs base_args(const AttnShape& sh) {
 
 tp_status launch_attn_core_fwd(const AttnShape& sh, const void* QKV, void* O, float* LSE,
                                cudaStream_t stream) {
-  if (sh.h / sh.heads != D) return fail(TP_ERR_UNSUPPORTED, "attention: head dimension must be 128");
-  if (sh.b * sh.heads > 65535) return fail(TP_ERR_SHAPE, "attention: b * heads too large");
-  AttnArgs a = base_args(sh);
-  a.qkv = static_cast<const __half*>(QKV);
-  a.out = static_cast<__nv_bfloat16*>(O);
-  a.lse_out = LSE;
-  cudaError_t e = set_smem(attn_fwd_kernel, FWD_SMEM);
-  if (e != cudaSuccess) return cuda_fail(e, "attention fwd smem attribute");
-  dim3 grid(static_cast<unsigned>((sh.s + FWD_BM - 1) / FWD_BM),
-            static_cast<unsigned>(sh.b * sh.heads));
-  {
-    LaunchScope scope(TP_KIND_ATTN_FWD, core_flops(sh), 2.0 * double(sh.b * sh.s) * 4 * sh.h, stream);
-    attn_fwd_kernel<<<grid, FWD_THREADS, FWD_SMEM, stream>>>(a);
-  }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "attention fwd launch");
-  return TP_OK;
+  return launch_attn_core_fwd_tc(sh, QKV, O, LSE, stream);
 }
 
 size_t attn_core_bwd_scratch_bytes(const AttnShape& sh) {
