@@ -199,27 +199,33 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     uint8_t* prow = sP + (r >> 3) * 1024 + (r & 7) * 128;  // row r in the SW128 layout
+    // Keys [0, limit) are visible to this row (causal: up to the row itself).
+    const int limit = a.causal ? min(a.s, qrow + 1) : a.s;
     for (int j = 0; j < n_kb; ++j) {
       const int st = j & 1;
       if (!(ok = mbar_wait(&s_full[st], static_cast<uint32_t>(j >> 1) & 1u, a.status,
                            kStatusAttnTimeout)))
         break;
       tc_fence_after();
-      const int k0 = j * kBN;
-      const bool edge = (a.causal && j == qb) || (k0 + kBN > a.s);
-      // pass 1: row max of this block
-      float mx = m_run;
+      const int vis = limit - j * kBN;  // visible keys of this block: [0, vis)
+      // pass 1: row max of the raw scores (the scale is positive, so the max
+      // of the scaled scores is the scaled max)
+      float mraw = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kBN; c += 32) {
         float v[32];
         tmem_ld32(tS[st] + lane_off + c, v);
+        if (vis < c + 32) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = k0 + c + i;
-          const bool masked = edge && (key >= a.s || (a.causal && key > qrow));
-          mx = fmaxf(mx, masked ? -INFINITY : v[i] * a.scale_log2);
+          for (int i = 0; i < 32; ++i) v[i] = (c + i < vis) ? v[i] : -INFINITY;
         }
+#pragma unroll
+        for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) v[i] = fmaxf(v[i], v[i + w]);
+        mraw = fmaxf(mraw, v[0]);
       }
+      const float mx = fmaxf(m_run, mraw * a.scale_log2);
       const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - mx);
       m_run = mx;
       // fold in O_{j-1} (scaled at m_{j-1}) and rescale to m_j
@@ -236,25 +242,28 @@ __global__ void __launch_bounds__(kThreadsA, 1)
           for (int i = 0; i < 32; ++i) o[c + i] = (o[c + i] + v[i]) * alpha;
         }
       }
-      // pass 2: P = 2^(s - m), row sum, fp16 into the P tile
+      // pass 2: P = 2^(s * scale - m), row sum, fp16 into the P tile
       float rs = 0.0f;
 #pragma unroll
       for (int c = 0; c < kBN; c += 32) {
         float v[32];
         tmem_ld32(tS[st] + lane_off + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = exp2f(fmaf(v[i], a.scale_log2, -mx));
+        if (vis < c + 32) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = (c + i < vis) ? v[i] : 0.0f;
+        }
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int key = k0 + c + i;
-          const bool m0 = edge && (key >= a.s || (a.causal && key > qrow));
-          const bool m1 = edge && (key + 1 >= a.s || (a.causal && key + 1 > qrow));
-          const float p0 = m0 ? 0.0f : exp2f(v[i] * a.scale_log2 - mx);
-          const float p1 = m1 ? 0.0f : exp2f(v[i + 1] * a.scale_log2 - mx);
-          rs += p0 + p1;
-          pk[i >> 1] = pack_half2(p0, p1);
-        }
+        for (int i = 0; i < 16; ++i) pk[i] = pack_half2(v[2 * i], v[2 * i + 1]);
+#pragma unroll
+        for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) v[i] += v[i + w];
+        rs += v[0];
         // 32 keys = 64 bytes = four 16-byte chunks of the row's 128-byte line
-        // in the 64-key half c / 64; chunk index is swizzled by (row & 7).
+        // in the 64-key half c / 64; the chunk index is swizzled by (row & 7).
         uint8_t* line = prow + (c >> 6) * kHalf;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
