@@ -316,6 +316,466 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+
+// ------------------------------------------------------------------ backward
+// Two kernels, no atomics (deterministic), both on tcgen05 with the same
+// warp roles as the forward; P and dS are recomputed from the saved LSE:
+//   P = 2^(S * scale_log2 - LSE * log2e),  dS = P * (dP - D),  D = rowsum(dO * O).
+// dQ kernel  (per 128 query rows, 64-key blocks):
+//   S = Q K^T, dP = dO V^T (TMEM, two buffers) -> dS (fp16, shared memory)
+//   -> dQ += dS K (TMEM); dQ is scaled by 1/sqrt(d) at the end.
+// dK/dV kernel (per 128 keys, 64-query blocks):
+//   S^T = K Q^T, dP^T = V dO^T (TMEM, two buffers) -> P^T, dS^T (shared memory)
+//   -> dV += P^T dO, dK += dS^T Q (TMEM); dK is scaled by 1/sqrt(d) at the end.
+constexpr int kB64 = 64;
+constexpr int kTile64 = 64 * 128 * 2;   // [64 rows x 128] fp16: 16 KB (two 8 KB halves)
+constexpr int kHalf64 = kTile64 / 2;
+constexpr int kTile128x64 = 128 * 64 * 2;  // [128 rows x 64] fp16: 16 KB (one SW128 atom wide)
+
+struct BwdArgs {
+  int s, h, heads, causal;
+  float scale_log2, scale;
+  const float* lse;   // [b, heads, s]
+  const float* dsum;  // [b, heads, s]
+  __nv_bfloat16* dqkv;  // [M, 3h]
+  int* status;
+};
+
+// Q (128 rows, once), dO (128 rows, once), then K_j, V_j (64 rows) in two stages.
+// Shared memory: Q 32K | dO 32K | KV[2] (K 16K + V 16K) | dS[2] 16K each.
+constexpr int kSmemDQ = 1024 + 2 * kTile + 2 * (2 * kTile64) + 2 * kTile128x64 + 256;
+
+__global__ void __launch_bounds__(kThreadsA, 1)
+    attn_bwd_dq_tcgen05(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
+                        const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sdO = smem + kTile;
+  uint8_t* sKV = smem + 2 * kTile;                 // stage st: K at +0, V at +kTile64
+  uint8_t* sdS = sKV + 2 * (2 * kTile64);           // [2] x 16 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sdS + 2 * kTile128x64);
+  uint64_t* qd_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* ds_full = bars + 7;   // [2]
+  uint64_t* ds_free = bars + 9;   // [2]
+  uint64_t* dq_done = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (a.s + kBM - 1) / kBM;
+  const int qb = nqb - 1 - static_cast<int>(blockIdx.x);
+  const int head = blockIdx.y % a.heads, bi = blockIdx.y / a.heads;
+  const int q0 = qb * kBM;
+  const int nkb_all = (a.s + kB64 - 1) / kB64;
+  const int n_kb = a.causal ? min(2 * qb + 2, nkb_all) : nkb_all;
+  const int row0 = bi * a.s;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qd_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&ds_full[i], 4);
+      mbar_init(&ds_free[i], 1);
+    }
+    mbar_init(dq_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem, tmem + 64};
+  const uint32_t tP[2] = {tmem + 128, tmem + 192};
+  const uint32_t tQ = tmem + 256;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmKV);
+      tma_prefetch_desc(&tmdO);
+      mbar_arrive_expect_tx(qd_full, 2 * kTile);
+      tma_load_2d(sQ, &tmQ, qd_full, head * kD, row0 + q0);
+      tma_load_2d(sQ + kHalf, &tmQ, qd_full, head * kD + 64, row0 + q0);
+      tma_load_2d(sdO, &tmdO, qd_full, head * kD, row0 + q0);
+      tma_load_2d(sdO + kHalf, &tmdO, qd_full, head * kD + 64, row0 + q0);
+      for (int j = 0; j < n_kb && ok; ++j) {
+        const int st = j & 1;
+        if (!(ok = mbar_wait(&kv_empty[st], ((static_cast<uint32_t>(j) >> 1) & 1u) ^ 1u, a.status,
+                             kStatusAttnTimeout)))
+          break;
+        mbar_arrive_expect_tx(&kv_full[st], 2 * kTile64);
+        uint8_t* k_dst = sKV + st * (2 * kTile64);
+        const int krow = row0 + j * kB64;
+        tma_load_2d(k_dst, &tmKV, &kv_full[st], a.h + head * kD, krow);
+        tma_load_2d(k_dst + kHalf64, &tmKV, &kv_full[st], a.h + head * kD + 64, krow);
+        tma_load_2d(k_dst + kTile64, &tmKV, &kv_full[st], 2 * a.h + head * kD, krow);
+        tma_load_2d(k_dst + kTile64 + kHalf64, &tmKV, &kv_full[st], 2 * a.h + head * kD + 64, krow);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t kIdSP = idesc_f16_f32(128, 64, false, false);  // Q K^T, dO V^T
+      constexpr uint32_t kIdQ = idesc_f16_f32(128, 128, false, true);   // dS K
+      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sdO);
+      bool ok = mbar_wait(qd_full, 0, a.status, kStatusAttnTimeout);
+      auto issue_sp = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!mbar_wait(&kv_full[st], (static_cast<uint32_t>(j) >> 1) & 1u, a.status,
+                       kStatusAttnTimeout))
+          return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sKV + st * (2 * kTile64));
+        const uint32_t v_addr = k_addr + kTile64;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t a_off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          const uint32_t b_off = (kk >> 2) * kHalf64 + (kk & 3) * 32;
+          umma_bf16(tS[st], sw128_desc(q_addr + a_off, 16, 1024),
+                    sw128_desc(k_addr + b_off, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
+          umma_bf16(tP[st], sw128_desc(do_addr + a_off, 16, 1024),
+                    sw128_desc(v_addr + b_off, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[st]);
+        return true;
+      };
+      if (ok) ok = issue_sp(0);
+      for (int j = 0; j < n_kb && ok; ++j) {
+        if (j + 1 < n_kb && !(ok = issue_sp(j + 1))) break;
+        const int st = j & 1;
+        if (!(ok = mbar_wait(&ds_full[st], (static_cast<uint32_t>(j) >> 1) & 1u, a.status,
+                             kStatusAttnTimeout)))
+          break;
+        tc_fence_after();
+        const uint32_t ds_addr = smem_u32(sdS + st * kTile128x64);
+        const uint32_t k_addr = smem_u32(sKV + st * (2 * kTile64));
+#pragma unroll
+        for (int kk = 0; kk < kB64 / 16; ++kk) {
+          umma_bf16(tQ, sw128_desc(ds_addr + kk * 32, 16, 1024),
+                    sw128_desc(k_addr + kk * 2048, kHalf64, 1024), kIdQ, (j | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit(&kv_empty[st]);
+        umma_commit(&ds_free[st]);
+      }
+      if (ok) umma_commit(dq_done);
+    }
+  } else if (warp >= 4) {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int qrow = q0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.s;
+    const int qc = min(qrow, a.s - 1);
+    const float lse2 = a.lse[stat + qc] * kLog2eA;
+    const float dd = a.dsum[stat + qc];
+    const int limit = a.causal ? min(a.s, qrow + 1) : a.s;
+    bool ok = true;
+    for (int j = 0; j < n_kb && ok; ++j) {
+      const int st = j & 1;
+      if (!(ok = mbar_wait(&s_full[st], (static_cast<uint32_t>(j) >> 1) & 1u, a.status,
+                           kStatusAttnTimeout)))
+        break;
+      if (j >= 2 && !(ok = mbar_wait(&ds_free[st], ((static_cast<uint32_t>(j) >> 1) - 1u) & 1u,
+                                     a.status, kStatusAttnTimeout)))
+        break;
+      tc_fence_after();
+      const int vis = limit - j * kB64;
+      uint8_t* row = sdS + st * kTile128x64 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+      for (int c = 0; c < kB64; c += 32) {
+        float sv[32], pv[32];
+        tmem_ld32(tS[st] + lane_off + c, sv);
+        tmem_ld32(tP[st] + lane_off + c, pv);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float p0 = exp2f(fmaf(sv[i], a.scale_log2, -lse2));
+          float p1 = exp2f(fmaf(sv[i + 1], a.scale_log2, -lse2));
+          p0 = (c + i < vis) ? p0 : 0.0f;
+          p1 = (c + i + 1 < vis) ? p1 : 0.0f;
+          pk[i >> 1] = pack_half2(p0 * (pv[i] - dd), p1 * (pv[i + 1] - dd));
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = (c >> 3) + q;
+          *reinterpret_cast<uint4*>(row + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ds_full[st]);
+    }
+    if (ok && mbar_wait(dq_done, 0, a.status, kStatusAttnTimeout)) {
+      tc_fence_after();
+      __nv_bfloat16* out = a.dqkv + static_cast<long long>(row0 + qrow) * (3LL * a.h) + head * kD;
+#pragma unroll
+      for (int c = 0; c < kD; c += 32) {
+        float v[32];
+        tmem_ld32(tQ + lane_off + c, v);
+        if (qrow < a.s) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 u;
+            uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 t = __floats2bfloat162_rn(v[8 * q + 2 * e] * a.scale,
+                                                       v[8 * q + 2 * e + 1] * a.scale);
+              w[e] = *reinterpret_cast<uint32_t*>(&t);
+            }
+            *reinterpret_cast<uint4*>(out + c + 8 * q) = u;
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// K, V (128 rows, once), then Q_i, dO_i (64 rows) in two stages; P^T and dS^T
+// tiles [128 keys x 64 queries] in two stages.
+// Shared memory: K 32K | V 32K | QdO[2] (Q 16K + dO 16K) | PdS[2] (P^T 16K + dS^T 16K).
+constexpr int kSmemKV = 1024 + 2 * kTile + 2 * (2 * kTile64) + 2 * (2 * kTile128x64) + 256;
+
+__global__ void __launch_bounds__(kThreadsA, 1)
+    attn_bwd_dkdv_tcgen05(const __grid_constant__ CUtensorMap tmKV128,
+                          const __grid_constant__ CUtensorMap tmQ64,
+                          const __grid_constant__ CUtensorMap tmdO64, const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + kTile;
+  uint8_t* sQdO = smem + 2 * kTile;                     // stage st: Q at +0, dO at +kTile64
+  uint8_t* sPdS = sQdO + 2 * (2 * kTile64);             // stage st: P^T at +0, dS^T at +16K
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sPdS + 2 * (2 * kTile128x64));
+  uint64_t* kv_full = bars + 0;
+  uint64_t* qd_full = bars + 1;   // [2]
+  uint64_t* qd_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* p_full = bars + 7;    // [2]
+  uint64_t* p_free = bars + 9;    // [2]
+  uint64_t* acc_done = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kb = static_cast<int>(blockIdx.x);  // early keys see the most queries: first
+  const int head = blockIdx.y % a.heads, bi = blockIdx.y / a.heads;
+  const int k0 = kb * kBN;
+  const int nqb_all = (a.s + kB64 - 1) / kB64;
+  const int i0 = a.causal ? (k0 / kB64) : 0;
+  const int n_qb = nqb_all - i0;
+  const int row0 = bi * a.s;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qd_full[i], 1);
+      mbar_init(&qd_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&p_free[i], 1);
+    }
+    mbar_init(acc_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem, tmem + 64};
+  const uint32_t tP[2] = {tmem + 128, tmem + 192};
+  const uint32_t tdV = tmem + 256, tdK = tmem + 384;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      tma_prefetch_desc(&tmKV128);
+      tma_prefetch_desc(&tmQ64);
+      tma_prefetch_desc(&tmdO64);
+      mbar_arrive_expect_tx(kv_full, 2 * kTile);
+      tma_load_2d(sK, &tmKV128, kv_full, a.h + head * kD, row0 + k0);
+      tma_load_2d(sK + kHalf, &tmKV128, kv_full, a.h + head * kD + 64, row0 + k0);
+      tma_load_2d(sV, &tmKV128, kv_full, 2 * a.h + head * kD, row0 + k0);
+      tma_load_2d(sV + kHalf, &tmKV128, kv_full, 2 * a.h + head * kD + 64, row0 + k0);
+      for (int it = 0; it < n_qb && ok; ++it) {
+        const int st = it & 1;
+        if (!(ok = mbar_wait(&qd_empty[st], ((static_cast<uint32_t>(it) >> 1) & 1u) ^ 1u,
+                             a.status, kStatusAttnTimeout)))
+          break;
+        mbar_arrive_expect_tx(&qd_full[st], 2 * kTile64);
+        uint8_t* dst = sQdO + st * (2 * kTile64);
+        const int qrow = row0 + (i0 + it) * kB64;
+        tma_load_2d(dst, &tmQ64, &qd_full[st], head * kD, qrow);
+        tma_load_2d(dst + kHalf64, &tmQ64, &qd_full[st], head * kD + 64, qrow);
+        tma_load_2d(dst + kTile64, &tmdO64, &qd_full[st], head * kD, qrow);
+        tma_load_2d(dst + kTile64 + kHalf64, &tmdO64, &qd_full[st], head * kD + 64, qrow);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t kIdSP = idesc_f16_f32(128, 64, false, false);  // K Q^T, V dO^T
+      constexpr uint32_t kIdAcc = idesc_f16_f32(128, 128, false, true);  // P^T dO, dS^T Q
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      bool ok = mbar_wait(kv_full, 0, a.status, kStatusAttnTimeout);
+      auto issue_sp = [&](int it) -> bool {
+        const int st = it & 1;
+        if (!mbar_wait(&qd_full[st], (static_cast<uint32_t>(it) >> 1) & 1u, a.status,
+                       kStatusAttnTimeout))
+          return false;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sQdO + st * (2 * kTile64));
+        const uint32_t do_addr = q_addr + kTile64;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t a_off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          const uint32_t b_off = (kk >> 2) * kHalf64 + (kk & 3) * 32;
+          umma_bf16(tS[st], sw128_desc(k_addr + a_off, 16, 1024),
+                    sw128_desc(q_addr + b_off, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
+          umma_bf16(tP[st], sw128_desc(v_addr + a_off, 16, 1024),
+                    sw128_desc(do_addr + b_off, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[st]);
+        return true;
+      };
+      if (ok && n_qb > 0) ok = issue_sp(0);
+      for (int it = 0; it < n_qb && ok; ++it) {
+        if (it + 1 < n_qb && !(ok = issue_sp(it + 1))) break;
+        const int st = it & 1;
+        if (!(ok = mbar_wait(&p_full[st], (static_cast<uint32_t>(it) >> 1) & 1u, a.status,
+                             kStatusAttnTimeout)))
+          break;
+        tc_fence_after();
+        const uint32_t pt_addr = smem_u32(sPdS + st * (2 * kTile128x64));
+        const uint32_t dst_addr = pt_addr + kTile128x64;
+        const uint32_t q_addr = smem_u32(sQdO + st * (2 * kTile64));
+        const uint32_t do_addr = q_addr + kTile64;
+#pragma unroll
+        for (int kk = 0; kk < kB64 / 16; ++kk) {
+          const uint32_t acc = (it | kk) != 0 ? 1u : 0u;
+          umma_bf16(tdV, sw128_desc(pt_addr + kk * 32, 16, 1024),
+                    sw128_desc(do_addr + kk * 2048, kHalf64, 1024), kIdAcc, acc);
+          umma_bf16(tdK, sw128_desc(dst_addr + kk * 32, 16, 1024),
+                    sw128_desc(q_addr + kk * 2048, kHalf64, 1024), kIdAcc, acc);
+        }
+        umma_commit(&qd_empty[st]);
+        umma_commit(&p_free[st]);
+      }
+      if (ok) umma_commit(acc_done);
+    }
+  } else if (warp >= 4) {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int key = k0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.s;
+    bool ok = true;
+    for (int it = 0; it < n_qb && ok; ++it) {
+      const int st = it & 1;
+      if (!(ok = mbar_wait(&s_full[st], (static_cast<uint32_t>(it) >> 1) & 1u, a.status,
+                           kStatusAttnTimeout)))
+        break;
+      if (it >= 2 && !(ok = mbar_wait(&p_free[st], ((static_cast<uint32_t>(it) >> 1) - 1u) & 1u,
+                                      a.status, kStatusAttnTimeout)))
+        break;
+      tc_fence_after();
+      const int q0 = (i0 + it) * kB64;
+      // query q = q0 + c is visible to this key when key <= q (causal) and q < s
+      const int first = a.causal ? max(key - q0, 0) : 0;  // first visible column
+      const int last = min(a.s - q0, kB64);                // one past the last
+      const bool key_ok = key < a.s;
+      uint8_t* prow = sPdS + st * (2 * kTile128x64) + (r >> 3) * 1024 + (r & 7) * 128;
+      uint8_t* drow = prow + kTile128x64;
+#pragma unroll
+      for (int c = 0; c < kB64; c += 32) {
+        float sv[32], pv[32];
+        tmem_ld32(tS[st] + lane_off + c, sv);
+        tmem_ld32(tP[st] + lane_off + c, pv);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int qa = min(q0 + c + i, a.s - 1), qb2 = min(q0 + c + i + 1, a.s - 1);
+          const float l0 = a.lse[stat + qa] * kLog2eA, l1 = a.lse[stat + qb2] * kLog2eA;
+          const float d0 = a.dsum[stat + qa], d1 = a.dsum[stat + qb2];
+          float p0 = exp2f(fmaf(sv[i], a.scale_log2, -l0));
+          float p1 = exp2f(fmaf(sv[i + 1], a.scale_log2, -l1));
+          const bool v0 = key_ok && (c + i >= first) && (c + i < last);
+          const bool v1 = key_ok && (c + i + 1 >= first) && (c + i + 1 < last);
+          p0 = v0 ? p0 : 0.0f;
+          p1 = v1 ? p1 : 0.0f;
+          pk[i >> 1] = pack_half2(p0, p1);
+          dk[i >> 1] = pack_half2(p0 * (pv[i] - d0), p1 * (pv[i + 1] - d1));
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int off = ((((c >> 3) + q) ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(prow + off) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          *reinterpret_cast<uint4*>(drow + off) =
+              make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[st]);
+    }
+    if (ok && n_qb > 0 && mbar_wait(acc_done, 0, a.status, kStatusAttnTimeout)) {
+      tc_fence_after();
+      __nv_bfloat16* out = a.dqkv + static_cast<long long>(row0 + key) * (3LL * a.h);
+#pragma unroll
+      for (int c = 0; c < kD; c += 32) {
+        float vk[32], vv[32];
+        tmem_ld32(tdK + lane_off + c, vk);
+        tmem_ld32(tdV + lane_off + c, vv);
+        if (key < a.s) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 uk, uv;
+            uint32_t* wk = reinterpret_cast<uint32_t*>(&uk);
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&uv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 8 * q + 2 * e;
+              __nv_bfloat162 tk = __floats2bfloat162_rn(vk[i] * a.scale, vk[i + 1] * a.scale);
+              __nv_bfloat162 tv = __floats2bfloat162_rn(vv[i], vv[i + 1]);
+              wk[e] = *reinterpret_cast<uint32_t*>(&tk);
+              wv[e] = *reinterpret_cast<uint32_t*>(&tv);
+            }
+            *reinterpret_cast<uint4*>(out + a.h + head * kD + c + 8 * q) = uk;
+            *reinterpret_cast<uint4*>(out + 2 * a.h + head * kD + c + 8 * q) = uv;
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn_attn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -368,6 +828,58 @@ tp_status launch_attn_core_fwd_tc(const AttnShape& sh, const void* QKV, void* O,
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention fwd (tcgen05) launch");
+  return TP_OK;
+}
+
+namespace {
+bool make_map_f16(CUtensorMap* m, const void* ptr, int64_t cols, int64_t rows, int box_rows) {
+  auto fn = encode_fn_attn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+// D = rowsum(dO * O) must already be in `dsum`.
+tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const void* dO,
+                                  const float* LSE, const float* dsum, void* dQKV,
+                                  cudaStream_t stream) {
+  if (sh.h / sh.heads != kD) return fail(TP_ERR_UNSUPPORTED, "attention: head dimension must be 128");
+  if (sh.b * sh.heads > 65535) return fail(TP_ERR_SHAPE, "attention: b * heads too large");
+  const int64_t M = sh.b * sh.s;
+  CUtensorMap qkv128, qkv64, do128, do64;
+  if (!make_map_f16(&qkv128, QKV, 3 * sh.h, M, 128) || !make_map_f16(&qkv64, QKV, 3 * sh.h, M, 64) ||
+      !make_map_f16(&do128, dO, sh.h, M, 128) || !make_map_f16(&do64, dO, sh.h, M, 64))
+    return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled failed (attention backward)");
+  BwdArgs a;
+  a.s = static_cast<int>(sh.s);
+  a.h = static_cast<int>(sh.h);
+  a.heads = sh.heads;
+  a.causal = sh.causal;
+  a.scale = 1.0f / std::sqrt(static_cast<float>(kD));
+  a.scale_log2 = a.scale * kLog2eA;
+  a.lse = LSE;
+  a.dsum = dsum;
+  a.dqkv = static_cast<__nv_bfloat16*>(dQKV);
+  a.status = device_status_ptr();
+  if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_tcgen05,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDQ);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_bwd_dkdv_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemKV);
+  if (e != cudaSuccess) return cuda_fail(e, "attention bwd smem attribute");
+  dim3 gq(static_cast<unsigned>((sh.s + kBM - 1) / kBM), static_cast<unsigned>(sh.b * sh.heads));
+  dim3 gk(static_cast<unsigned>((sh.s + kBN - 1) / kBN), static_cast<unsigned>(sh.b * sh.heads));
+  attn_bwd_dq_tcgen05<<<gq, kThreadsA, kSmemDQ, stream>>>(qkv128, qkv64, do128, a);
+  attn_bwd_dkdv_tcgen05<<<gk, kThreadsA, kSmemKV, stream>>>(qkv128, qkv64, do64, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attention bwd (tcgen05) launch");
   return TP_OK;
 }
 

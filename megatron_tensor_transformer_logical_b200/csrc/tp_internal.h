@@ -105,6 +105,10 @@ tp_status launch_attn_core_fwd(const AttnShape& sh, const void* QKV, void* O, fl
 // The tcgen05 / TMEM forward that launch_attn_core_fwd runs.
 tp_status launch_attn_core_fwd_tc(const AttnShape& sh, const void* QKV, void* O, float* LSE,
                                   cudaStream_t stream);
+// The tcgen05 dQ and dK/dV kernels; D = rowsum(dO * O) must be in `dsum`.
+tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const void* dO,
+                                  const float* LSE, const float* dsum, void* dQKV,
+                                  cudaStream_t stream);
 // dO [M, h]; writes dQKV [M, 3h] (bf16).  `scratch` holds
 // attn_core_bwd_scratch_bytes bytes (fp32 dQ accumulator and row terms).
 size_t attn_core_bwd_scratch_bytes(const AttnShape& sh);
