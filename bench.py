@@ -176,11 +176,15 @@ class LayerStep:
                       self.dWqkv, self.dWo, wl.b, wl.s, wl.heads, wl.t, True,
                       self.ws[L.TP_OP_ATTN_BWD])
 
-    def mlp(self):
+    def mlp(self, save_y=True):
+        """MLP forward + backward.  save_y: keep the pre-activation Y from the
+        forward for the backward (default); otherwise the backward recomputes
+        it with one more GEMM (the activation-recompute policy)."""
         L, wl = self.L, self.wl
-        L.tp_mlp_fwd(self.X, self.A, None, self.B, None, self.Zm, self.Y, wl.t,
+        Y = self.Y if save_y else None
+        L.tp_mlp_fwd(self.X, self.A, None, self.B, None, self.Zm, Y, wl.t,
                      self.ws[L.TP_OP_MLP_FWD])
-        L.tp_mlp_bwd(self.X, self.A, None, self.B, self.Y, self.dZ, self.dXm, self.dA, None,
+        L.tp_mlp_bwd(self.X, self.A, None, self.B, Y, self.dZ, self.dXm, self.dA, None,
                      self.dB, None, wl.t, self.ws[L.TP_OP_MLP_BWD])
 
     def step(self):
@@ -243,6 +247,12 @@ def run_libtp(args, rank, world, local_rank, dist):
     barrier()
     mlp_ms = timed(st.mlp, args.steps, stream)
     barrier()
+    # Activation policy: recompute Y in the backward instead of keeping it.
+    for _ in range(2):
+        st.mlp(save_y=False)
+    barrier()
+    mlp_rec_ms = timed(lambda: st.mlp(save_y=False), args.steps, stream)
+    barrier()
 
     # End to end through the public API: per step, the step's inputs (X, dZ)
     # copied from pinned host memory and its results (Z and dX of both
@@ -278,7 +288,7 @@ def run_libtp(args, rank, world, local_rank, dist):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    ms, mlp_ms = maxall(ms), maxall(mlp_ms)
+    ms, mlp_ms, mlp_rec_ms = maxall(ms), maxall(mlp_ms), maxall(mlp_rec_ms)
     e2e_ms = maxall(e2e_ms) if e2e_ms is not None else None
     if rank != 0:
         return None
@@ -334,6 +344,12 @@ def run_libtp(args, rank, world, local_rank, dist):
         "mlp_fwd_bwd": {"tflops": round(mlp_tflops, 2), "ms_per_step": round(mlp_ms / args.steps, 4),
                         "frac_of_nominal_2250": round(mlp_tflops / world / NOMINAL_BF16_TFLOPS, 4),
                         "frac_of_measured_sustained": round(mlp_tflops / world / peak, 4)},
+        "activation_policy": {
+            "save_y": {"mlp_ms_per_step": round(mlp_ms / args.steps, 4),
+                       "bytes_kept_fwd_to_bwd": wl.M * wl.f * 2},
+            "recompute_y": {"mlp_ms_per_step": round(mlp_rec_ms / args.steps, 4),
+                            "bytes_kept_fwd_to_bwd": 0,
+                            "extra_flops": 2.0 * wl.M * wl.h * wl.f}},
         "roofline": {"bound": "tensor", "kernel": "gemm_bf16_tcgen05",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4),

@@ -28,7 +28,8 @@ Sources (page title, then section):
   - §3.2 Wq, Wk, Wv split by columns in head groups, ``W_o`` split by rows,
     ``Z = sum_g O_g @ Wo_g``; backward mirrors it.
 * [P2] the PyTorch tensor-parallel tutorial (page title "企业官网建设流程全解析"):
-  §3.3 uses ``nn.GELU()`` between the two linears (the exact erf form).
+  §3.3 uses ``nn.GELU()`` between the two linears (the exact erf form) and
+  builds the block as x + attention(LayerNorm(x)), then x + mlp(LayerNorm(x)).
 * [P4] "5.1 Tensor并行与算子拆分": ``tensor_parallel_split`` raises on a
   dimension that the partition count does not divide; the attention listing
   uses ``masked_fill(mask == 0, -inf)`` and ``1/sqrt(d_k)`` scaling.
@@ -62,7 +63,8 @@ __all__ = [
     "linear_col_parallel", "linear_row_parallel", "mlp_fwd", "mlp_fwd_parallel",
     "mlp_bwd", "mlp_bwd_parallel", "head_columns", "group_columns",
     "attention_core", "attention_core_bwd", "attn_fwd", "attn_fwd_parallel",
-    "attn_bwd", "attn_bwd_parallel", "max_rel_error", "normwise_error",
+    "attn_bwd", "attn_bwd_parallel", "layernorm_fwd", "layernorm_bwd", "block_fwd",
+    "block_bwd", "max_rel_error", "normwise_error",
 ]
 
 _SQRT2 = math.sqrt(2.0)
@@ -444,6 +446,68 @@ def attn_bwd_parallel(X, Wqkv, Wo, dZ, b: int, s: int, heads: int, t: int,
     for p in dXs[1:]:
         dX = dX + p
     return {"dX": dX, "dWqkv": dWqkv, "dWo": dWo, "dX_partials": dXs}
+
+
+# ---------------------------------------------------------------------------
+# LayerNorm and the Transformer block ([P2] §3.3 ParallelTransformerBlock:
+# x = x + attention(norm1(x)); x = x + mlp(norm2(x)), norm = nn.LayerNorm)
+# ---------------------------------------------------------------------------
+
+def layernorm_fwd(X, gamma=None, beta=None, eps: float = 1e-5):
+    """Row-wise LayerNorm: Y = (X - mean) / sqrt(var + eps) * gamma + beta,
+    mean and (biased) variance over the last dimension.  Returns Y, mean and
+    rstd = 1 / sqrt(var + eps) per row."""
+    X = _f64(X)
+    mean = X.mean(axis=-1)
+    var = ((X - mean[:, None]) ** 2).mean(axis=-1)
+    rstd = 1.0 / np.sqrt(var + eps)
+    Y = (X - mean[:, None]) * rstd[:, None]
+    if gamma is not None:
+        Y = Y * _f64(gamma)
+    if beta is not None:
+        Y = Y + _f64(beta)
+    return {"Y": Y, "mean": mean, "rstd": rstd}
+
+
+def layernorm_bwd(X, gamma, dY, eps: float = 1e-5):
+    """Backward of layernorm_fwd by the chain rule, with xhat = (X - mean) * rstd
+    and g = dY * gamma: dX = rstd * (g - mean(g) - xhat * mean(g * xhat)),
+    dgamma = sum over rows of dY * xhat, dbeta = sum over rows of dY."""
+    X, dY = _f64(X), _f64(dY)
+    f = layernorm_fwd(X, None, None, eps)
+    xhat = (X - f["mean"][:, None]) * f["rstd"][:, None]
+    g = dY * (_f64(gamma) if gamma is not None else 1.0)
+    dX = f["rstd"][:, None] * (g - g.mean(axis=-1, keepdims=True)
+                               - xhat * (g * xhat).mean(axis=-1, keepdims=True))
+    return {"dX": dX, "dgamma": (dY * xhat).sum(axis=0), "dbeta": dY.sum(axis=0)}
+
+
+def block_fwd(X, w, b: int, s: int, heads: int, eps: float = 1e-5, causal: bool = True):
+    """One Transformer block: X1 = X + Attn(LN1(X)); X2 = X1 + MLP(LN2(X1)).
+    `w` holds ln1_g, ln1_b, Wqkv, Wo, ln2_g, ln2_b, A, bA, B, bB."""
+    X = _f64(X)
+    n1 = layernorm_fwd(X, w["ln1_g"], w["ln1_b"], eps)
+    at = attn_fwd(n1["Y"], w["Wqkv"], w["Wo"], b, s, heads, causal)
+    X1 = X + at["Z"]
+    n2 = layernorm_fwd(X1, w["ln2_g"], w["ln2_b"], eps)
+    ml = mlp_fwd(n2["Y"], w["A"], w.get("bA"), w["B"], w.get("bB"))
+    return {"X1": X1, "X2": X1 + ml["Z"], "Xn1": n1["Y"], "Xn2": n2["Y"]}
+
+
+def block_bwd(X, w, dX2, b: int, s: int, heads: int, eps: float = 1e-5, causal: bool = True):
+    """Backward of block_fwd: the residual paths pass the gradient through,
+    the sublayers add theirs: dX1 = dX2 + LN2'(MLP'(dX2)); dX = dX1 + LN1'(Attn'(dX1))."""
+    X, dX2 = _f64(X), _f64(dX2)
+    fw = block_fwd(X, w, b, s, heads, eps, causal)
+    mb = mlp_bwd(fw["Xn2"], w["A"], w.get("bA"), w["B"], dX2)
+    l2 = layernorm_bwd(fw["X1"], w["ln2_g"], mb["dX"], eps)
+    dX1 = dX2 + l2["dX"]
+    ab = attn_bwd(fw["Xn1"], w["Wqkv"], w["Wo"], dX1, b, s, heads, causal)
+    l1 = layernorm_bwd(X, w["ln1_g"], ab["dX"], eps)
+    return {"dX": dX1 + l1["dX"], "dX1": dX1,
+            "dln1_g": l1["dgamma"], "dln1_b": l1["dbeta"], "dWqkv": ab["dWqkv"], "dWo": ab["dWo"],
+            "dln2_g": l2["dgamma"], "dln2_b": l2["dbeta"], "dA": mb["dA"], "dbA": mb["dbA"],
+            "dB": mb["dB"], "dbB": mb["dbB"]}
 
 
 # ---------------------------------------------------------------------------

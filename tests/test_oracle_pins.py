@@ -437,3 +437,86 @@ def test_head_slice_equals_the_heads_columns():
         g = O.attn_bwd(X, Wqkv[:, cols], Wo[j * d:(j + 1) * d], dZ, b, s, 1)
         assert np.max(np.abs(g["dWqkv"] - gfull["dWqkv"][:, cols])) < 1e-12
         assert np.max(np.abs(g["dWo"] - gfull["dWo"][j * d:(j + 1) * d])) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# LayerNorm and the block ([P2] §3.3)
+# ---------------------------------------------------------------------------
+
+def bf_layernorm_row(x, g, b, eps):
+    n = len(x)
+    mu = sum(x) / n
+    var = sum((v - mu) ** 2 for v in x) / n
+    return [(v - mu) / math.sqrt(var + eps) * gi + bi for v, gi, bi in zip(x, g, b)]
+
+
+def check_layernorm(o):
+    r = _rng(40)
+    X = r.standard_normal((5, 12)) * 3 + 1.5
+    g, b = r.standard_normal(12), r.standard_normal(12)
+    out = o.layernorm_fwd(X, g, b, 1e-5)
+    for i in range(5):
+        ref = bf_layernorm_row(list(X[i]), list(g), list(b), 1e-5)
+        assert np.max(np.abs(out["Y"][i] - ref)) < 1e-12
+    plain = o.layernorm_fwd(X, None, None, 0.0)["Y"]  # closed form: zero mean, unit variance
+    assert np.max(np.abs(plain.mean(axis=1))) < 1e-14
+    assert np.max(np.abs((plain ** 2).mean(axis=1) - 1.0)) < 1e-13
+    G = r.standard_normal((5, 12))
+    loss = lambda: float(np.sum(G * o.layernorm_fwd(X, g, b, 1e-5)["Y"]))
+    bw = o.layernorm_bwd(X, g, G, 1e-5)
+    for name, P in (("dX", X), ("dgamma", g), ("dbeta", b)):
+        assert np.max(np.abs(bw[name] - _fd_grad(loss, P))) < 1e-7, name
+
+
+def _tiny_block(seed):
+    r = _rng(seed)
+    h, f = 8, 16
+    w = {"ln1_g": 1 + 0.1 * r.standard_normal(h), "ln1_b": 0.1 * r.standard_normal(h),
+         "Wqkv": r.standard_normal((h, 3 * h)) * 0.4, "Wo": r.standard_normal((h, h)) * 0.4,
+         "ln2_g": 1 + 0.1 * r.standard_normal(h), "ln2_b": 0.1 * r.standard_normal(h),
+         "A": r.standard_normal((h, f)) * 0.4, "bA": 0.1 * r.standard_normal(f),
+         "B": r.standard_normal((f, h)) * 0.4, "bB": 0.1 * r.standard_normal(h)}
+    return w, r.standard_normal((2 * 3, h)), r.standard_normal((2 * 3, h))
+
+
+def check_block_bwd_fd(o):
+    w, X, G = _tiny_block(41)
+    loss = lambda: float(np.sum(G * o.block_fwd(X, w, 2, 3, 2)["X2"]))
+    bw = o.block_bwd(X, w, G, 2, 3, 2)
+    assert np.max(np.abs(bw["dX"] - _fd_grad(loss, X))) < 1e-6
+    for name, key in (("dln1_g", "ln1_g"), ("dWqkv", "Wqkv"), ("dWo", "Wo"), ("dln2_b", "ln2_b"),
+                      ("dA", "A"), ("dbB", "bB")):
+        assert np.max(np.abs(bw[name] - _fd_grad(loss, w[key]))) < 1e-6, name
+
+
+PINS += [check_layernorm, check_block_bwd_fd]
+
+
+@pytest.mark.parametrize("pin", [check_layernorm, check_block_bwd_fd], ids=lambda p: p.__name__)
+def test_block_pins(pin):
+    pin(O)
+
+
+def test_block_residual_identity():
+    """With zero Wo and zero B the sublayers add nothing: X2 = X1 = X."""
+    w, X, _ = _tiny_block(42)
+    w["Wo"] = np.zeros_like(w["Wo"])
+    w["B"], w["bB"] = np.zeros_like(w["B"]), np.zeros_like(w["bB"])
+    out = O.block_fwd(X, w, 2, 3, 2)
+    assert np.array_equal(out["X1"], X) and np.array_equal(out["X2"], X)
+
+
+def _ln_no_centering(X, gamma=None, beta=None, eps=1e-5):
+    X = np.asarray(X, dtype=np.float64)
+    rstd = 1.0 / np.sqrt((X ** 2).mean(axis=-1) + eps)  # mistake: RMS norm, no mean removed
+    Y = X * rstd[:, None] * (gamma if gamma is not None else 1.0) + (beta if beta is not None else 0.0)
+    return {"Y": Y, "mean": X.mean(axis=-1), "rstd": rstd}
+
+
+MUTANTS["LayerNorm without centering"] = dict(layernorm_fwd=_ln_no_centering)
+
+
+def test_planted_layernorm_mistake_is_caught():
+    m = _mutant(layernorm_fwd=_ln_no_centering)
+    with pytest.raises(AssertionError):
+        check_layernorm(m)
