@@ -66,7 +66,10 @@ typedef enum tp_op {
   TP_OP_MLP_FWD = 0,
   TP_OP_MLP_BWD = 1,
   TP_OP_ATTN_FWD = 2,
-  TP_OP_ATTN_BWD = 3
+  TP_OP_ATTN_BWD = 3,
+  TP_OP_LN_BWD = 4,
+  TP_OP_BLOCK_FWD = 5,
+  TP_OP_BLOCK_BWD = 6
 } tp_op;
 
 /*
@@ -197,9 +200,103 @@ tp_status tp_attn_bwd(const void* X, const void* Wqkv, const void* Wo, const voi
                       void* stream);
 
 /*
+ * LayerNorm over the last dimension, as nn.LayerNorm in the tutorial's block
+ * ([P2] §3.3): Y = (X - mean) * rstd * gamma + beta per row, with mean and
+ * the biased variance over the row, rstd = 1 / sqrt(var + eps); statistics
+ * in fp32.  Replicated across the logical shards (not partitioned).
+ *   X, Y [M, h] dtype; gamma, beta [h] dtype or NULL (1 and 0); mean, rstd
+ *   [M] fp32 or NULL (saved for the backward).  h % 8 == 0, h <= 16384.
+ * Errors: NULL X/Y; M, h <= 0; alignment; h > 16384 is TP_ERR_UNSUPPORTED.
+ */
+tp_status tp_layernorm_fwd(const void* X, const void* gamma, const void* beta, void* Y,
+                           float* mean, float* rstd, int64_t M, int64_t h, float eps,
+                           tp_dtype dtype, void* stream);
+
+/*
+ * LayerNorm backward: with xhat = (X - mean) * rstd and g = dY * gamma,
+ *   dX = rstd * (g - rowmean(g) - xhat * rowmean(g * xhat)) (+ dR if not NULL:
+ *   the gradient of a residual path that joins here), dgamma = colsum(dY * xhat),
+ *   dbeta = colsum(dY) (each only if its pointer is not NULL).
+ *   mean, rstd: from tp_layernorm_fwd (required).  ws: tp_workspace_size(TP_OP_LN_BWD).
+ */
+tp_status tp_layernorm_bwd(const void* X, const void* gamma, const float* mean,
+                           const float* rstd, const void* dY, const void* dR, void* dX,
+                           void* dgamma, void* dbeta, int64_t M, int64_t h, tp_dtype dtype,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Weights of one Transformer block (bf16; biases and LayerNorm affines may be NULL). */
+typedef struct tp_block_weights {
+  const void* ln1_g;
+  const void* ln1_b;
+  const void* Wqkv; /* [h, 3h] */
+  const void* Wo;   /* [h, h]  */
+  const void* ln2_g;
+  const void* ln2_b;
+  const void* A;    /* [h, f]  */
+  const void* bA;   /* [f]     */
+  const void* B;    /* [f, h]  */
+  const void* bB;   /* [h]     */
+} tp_block_weights;
+
+/* Activations the block forward keeps for its backward (all required). */
+typedef struct tp_block_saves {
+  void* Xn1;    /* [M, h] bf16: LN1(X)                 */
+  float* mean1; /* [M]                                  */
+  float* rstd1; /* [M]                                  */
+  void* QKV;    /* [M, 3h] fp16                         */
+  void* O;      /* [M, h] bf16                          */
+  float* LSE;   /* [b, heads, s]                        */
+  void* X1;     /* [M, h] bf16: X + Attn(LN1(X))        */
+  void* Xn2;    /* [M, h] bf16: LN2(X1)                 */
+  float* mean2; /* [M]                                  */
+  float* rstd2; /* [M]                                  */
+  void* Y;      /* [M, f] bf16: MLP pre-activation      */
+} tp_block_saves;
+
+/* Weight gradients of one block (bf16; the bias / affine ones may be NULL). */
+typedef struct tp_block_grads {
+  void* dln1_g;
+  void* dln1_b;
+  void* dWqkv;
+  void* dWo;
+  void* dln2_g;
+  void* dln2_b;
+  void* dA;
+  void* dbA;
+  void* dB;
+  void* dbB;
+} tp_block_grads;
+
+/*
+ * One Transformer block, the tutorial's ParallelTransformerBlock.forward
+ * ([P2] §3.3):  X1 = X + Attn(LN1(X));  X2 = X1 + MLP(LN2(X1)),
+ * with the attention and the MLP partitioned exactly as tp_attn_fwd and
+ * tp_mlp_fwd (t logical shards, causal attention) and each residual addition
+ * fused into the epilogue of the row-split GEMM that ends its sublayer.
+ *   X, X2 [M = b*s, h] bf16; weights, saves as above; eps for both norms.
+ *   ws: tp_workspace_size(TP_OP_BLOCK_FWD, M, h, f, heads, t, TP_BF16).
+ * Errors: those of the parts; a NULL save is TP_ERR_NULL; dtype must be bf16.
+ */
+tp_status tp_block_fwd(const void* X, const tp_block_weights* w, void* X2, tp_block_saves* saves,
+                       int64_t b, int64_t s, int64_t h, int64_t f, int heads, int t, float eps,
+                       tp_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Backward of tp_block_fwd (the mirror rule for each sublayer, residual paths
+ * passing the gradient through):  dX1 = dX2 + LN2'(MLP'(dX2));
+ * dX = dX1 + LN1'(Attn'(dX1)).  Writes dX [M, h] and every gradient in g.
+ *   ws: tp_workspace_size(TP_OP_BLOCK_BWD, M, h, f, heads, t, TP_BF16).
+ */
+tp_status tp_block_bwd(const void* X, const tp_block_weights* w, const tp_block_saves* saves,
+                       const void* dX2, void* dX, const tp_block_grads* g, int64_t b, int64_t s,
+                       int64_t h, int64_t f, int heads, int t, float eps, tp_dtype dtype,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Workspace bytes that `op` needs for these sizes (M = b*s tokens; f is
- * ignored by the attention ops, heads by the MLP ops).  Returns 0 for
- * invalid arguments.  The size covers the worst case (recomputed Y / QKV).
+ * ignored by the attention and LayerNorm ops, heads by the MLP and LayerNorm
+ * ops).  Returns 0 for invalid arguments.  The size covers the worst case
+ * (recomputed Y / QKV).
  */
 size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, int t,
                          tp_dtype dtype);

@@ -21,6 +21,7 @@ TP_OK, TP_ERR_NULL, TP_ERR_SHAPE, TP_ERR_ALIGN, TP_ERR_DTYPE = 0, 1, 2, 3, 4
 TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_KERNEL, TP_ERR_WORKSPACE = 5, 6, 7, 8
 TP_F32, TP_BF16 = 0, 1
 TP_OP_MLP_FWD, TP_OP_MLP_BWD, TP_OP_ATTN_FWD, TP_OP_ATTN_BWD = 0, 1, 2, 3
+TP_OP_LN_BWD, TP_OP_BLOCK_FWD, TP_OP_BLOCK_BWD = 4, 5, 6
 
 TP_KIND_GEMM_TCGEN05, TP_KIND_GEMM_SIMT, TP_KIND_ATTN_FWD, TP_KIND_ATTN_BWD, TP_KIND_REDUCE = range(5)
 KIND_NAMES = {TP_KIND_GEMM_TCGEN05: "gemm_tcgen05", TP_KIND_GEMM_SIMT: "gemm_simt",
@@ -29,7 +30,24 @@ KIND_NAMES = {TP_KIND_GEMM_TCGEN05: "gemm_tcgen05", TP_KIND_GEMM_SIMT: "gemm_sim
 EXPORTS = ("tp_linear_col", "tp_linear_row", "tp_mlp_fwd", "tp_mlp_bwd", "tp_attn_fwd",
            "tp_attn_bwd", "tp_workspace_size", "tp_last_error", "tp_device_status",
            "tp_version", "tp_profile_enable", "tp_profile_read", "tp_launch_count",
-           "tp_mlp_fwd_noalloc", "tp_profile_count", "tp_profile_record")
+           "tp_mlp_fwd_noalloc", "tp_profile_count", "tp_profile_record", "tp_layernorm_fwd",
+           "tp_layernorm_bwd", "tp_block_fwd", "tp_block_bwd")
+
+_W_FIELDS = ("ln1_g", "ln1_b", "Wqkv", "Wo", "ln2_g", "ln2_b", "A", "bA", "B", "bB")
+_S_FIELDS = ("Xn1", "mean1", "rstd1", "QKV", "O", "LSE", "X1", "Xn2", "mean2", "rstd2", "Y")
+_G_FIELDS = ("dln1_g", "dln1_b", "dWqkv", "dWo", "dln2_g", "dln2_b", "dA", "dbA", "dB", "dbB")
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _W_FIELDS]
+
+
+class BlockSaves(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _S_FIELDS]
+
+
+class BlockGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _G_FIELDS]
 
 
 class LaunchRecord(ctypes.Structure):
@@ -72,6 +90,14 @@ def load() -> ctypes.CDLL:
                               vp, sz, vp]
     L.tp_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32,
                               i32, i32, vp, sz, vp]
+    f32 = ctypes.c_float
+    L.tp_layernorm_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, f32, i32, vp]
+    L.tp_layernorm_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i32, vp, sz, vp]
+    L.tp_block_fwd.argtypes = [vp, ctypes.POINTER(BlockWeights), vp, ctypes.POINTER(BlockSaves),
+                               i64, i64, i64, i64, i32, i32, f32, i32, vp, sz, vp]
+    L.tp_block_bwd.argtypes = [vp, ctypes.POINTER(BlockWeights), ctypes.POINTER(BlockSaves), vp,
+                               vp, ctypes.POINTER(BlockGrads), i64, i64, i64, i64, i32, i32, f32,
+                               i32, vp, sz, vp]
     L.tp_workspace_size.argtypes = [i32, i64, i64, i64, i32, i32, i32]
     L.tp_workspace_size.restype = sz
     L.tp_last_error.argtypes = []
@@ -180,6 +206,43 @@ def tp_attn_bwd(X, Wqkv, Wo, QKVsave, Osave, LSEsave, dZ, dX, dWqkv, dWo, b: int
                               _ptr(LSEsave), _ptr(dZ), _ptr(dX), _ptr(dWqkv), _ptr(dWo), b, s,
                               h, heads, t, int(causal), _dtype(X), _ptr(ws),
                               ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def tp_layernorm_fwd(X, gamma, beta, Y, mean, rstd, eps: float = 1e-5, stream=None) -> None:
+    M, h = X.shape
+    _check(load().tp_layernorm_fwd(_ptr(X), _ptr(gamma), _ptr(beta), _ptr(Y), _ptr(mean),
+                                   _ptr(rstd), M, h, eps, _dtype(X), _stream(stream)))
+
+
+def tp_layernorm_bwd(X, gamma, mean, rstd, dY, dR, dX, dgamma, dbeta, ws, stream=None) -> None:
+    M, h = X.shape
+    _check(load().tp_layernorm_bwd(_ptr(X), _ptr(gamma), _ptr(mean), _ptr(rstd), _ptr(dY),
+                                   _ptr(dR), _ptr(dX), _ptr(dgamma), _ptr(dbeta), M, h, _dtype(X),
+                                   _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def _struct(cls, fields, d):
+    return cls(*[_ptr(d.get(n)) for n in fields])
+
+
+def tp_block_fwd(X, w: dict, X2, saves: dict, b: int, s: int, f: int, heads: int, t: int,
+                 eps: float, ws, stream=None) -> None:
+    """w: dict of the tp_block_weights fields; saves: dict of tp_block_saves fields."""
+    h = X.shape[1]
+    W, S = _struct(BlockWeights, _W_FIELDS, w), _struct(BlockSaves, _S_FIELDS, saves)
+    _check(load().tp_block_fwd(_ptr(X), ctypes.byref(W), _ptr(X2), ctypes.byref(S), b, s, h, f,
+                               heads, t, eps, _dtype(X), _ptr(ws), ws.numel() * ws.element_size(),
+                               _stream(stream)))
+
+
+def tp_block_bwd(X, w: dict, saves: dict, dX2, dX, grads: dict, b: int, s: int, f: int,
+                 heads: int, t: int, eps: float, ws, stream=None) -> None:
+    h = X.shape[1]
+    W, S = _struct(BlockWeights, _W_FIELDS, w), _struct(BlockSaves, _S_FIELDS, saves)
+    G = _struct(BlockGrads, _G_FIELDS, grads)
+    _check(load().tp_block_bwd(_ptr(X), ctypes.byref(W), ctypes.byref(S), _ptr(dX2), _ptr(dX),
+                               ctypes.byref(G), b, s, h, f, heads, t, eps, _dtype(X), _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def tp_device_status(stream=None) -> None:

@@ -231,7 +231,7 @@ size_t mlp_bwd_ws(int64_t M, int64_t h, int64_t f, tp_dtype d) {
 
 tp_status mlp_fwd(const void* X, const void* A, const void* bA, const void* B, const void* bB,
                   void* Z, void* Ysave, int64_t M, int64_t h, int64_t f, int t, tp_dtype dtype,
-                  void* ws, size_t ws_bytes, cudaStream_t stream) {
+                  void* ws, size_t ws_bytes, cudaStream_t stream, const void* residual = nullptr) {
   if (!X || !A || !B || !Z) return fail(TP_ERR_NULL, "X, A, B and Z are required");
   TP_TRY(check_dtype(dtype));
   if (M <= 0 || h <= 0 || f <= 0) return fail(TP_ERR_SHAPE, "M, h and f must be positive");
@@ -263,7 +263,8 @@ tp_status mlp_fwd(const void* X, const void* A, const void* bA, const void* B, c
   g2.M = M; g2.N = h; g2.K = f;
   g2.a = {H, f, true};
   g2.b = {B, h, false};
-  g2.epi = kEpiStore;
+  g2.epi = residual ? kEpiResidual : kEpiStore;  // Z = residual + MLP(X) when given
+  g2.aux = residual; g2.ldaux = h;
   g2.out = Z; g2.ldo = h; g2.out_f32 = f32;
   g2.bias = bB;
   return run(g2, f32, stream);
@@ -386,7 +387,8 @@ tp_status attn_check(const void* X, const void* Wqkv, const void* Wo, int64_t b,
 
 tp_status attn_fwd(const void* X, const void* Wqkv, const void* Wo, void* Z, void* QKVsave,
                    void* Osave, void* LSEsave, int64_t b, int64_t s, int64_t h, int heads, int t,
-                   int causal, tp_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                   int causal, tp_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream,
+                   const void* residual = nullptr) {
   TP_TRY(attn_check(X, Wqkv, Wo, b, s, h, heads, t, dtype));
   if (!Z) return fail(TP_ERR_NULL, "Z is required");
   TP_TRY(check_ptrs_aligned({X, Wqkv, Wo, Z, QKVsave, Osave, LSEsave, ws}));
@@ -420,6 +422,8 @@ tp_status attn_fwd(const void* X, const void* Wqkv, const void* Wo, void* Z, voi
   go.a = {O, h, true};
   go.b = {Wo, h, false};
   go.out = Z; go.ldo = h;
+  go.epi = residual ? kEpiResidual : kEpiStore;  // Z = residual + Attn(X) when given
+  go.aux = residual; go.ldaux = h;
   return launch_gemm_bf16(go, stream);
 }
 
@@ -500,6 +504,105 @@ tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* 
   return launch_gemm_bf16(g4, stream);
 }
 
+// -------------------------------------------------------------- LayerNorm
+
+tp_status ln_check(const void* X, const void* Y, int64_t M, int64_t h, tp_dtype dtype) {
+  if (!X || !Y) return fail(TP_ERR_NULL, "X and Y are required");
+  TP_TRY(check_dtype(dtype));
+  if (M <= 0 || h <= 0) return fail(TP_ERR_SHAPE, "M and h must be positive");
+  TP_TRY(check_rows({h}));
+  if (h > layernorm_max_h()) return fail(TP_ERR_UNSUPPORTED, "layernorm: h must be at most 16384");
+  return TP_OK;
+}
+
+size_t ln_bwd_ws(int64_t M, int64_t h) { return align_up(layernorm_bwd_scratch_bytes(M, h), 256) + 256; }
+
+// ------------------------------------------------------------------- block
+
+size_t block_fwd_ws(int64_t M, int64_t h, int64_t f, int heads) {
+  const size_t a = attn_fwd_ws(M, h, heads), m = mlp_fwd_ws(M, f, TP_BF16);
+  return a > m ? a : m;
+}
+
+size_t block_bwd_ws(int64_t M, int64_t h, int64_t f, int heads) {
+  size_t inner = mlp_bwd_ws(M, h, f, TP_BF16);
+  if (attn_bwd_ws(M, h, heads) > inner) inner = attn_bwd_ws(M, h, heads);
+  if (ln_bwd_ws(M, h) > inner) inner = ln_bwd_ws(M, h);
+  return 3 * align_up(M * h * 2, 256) + inner + 1024;
+}
+
+tp_status block_check(const void* X, const tp_block_weights* w, int64_t b, int64_t s, int64_t h,
+                      int64_t f, int heads, int t, tp_dtype dtype) {
+  if (!X || !w) return fail(TP_ERR_NULL, "X and the weights are required");
+  if (!w->Wqkv || !w->Wo || !w->A || !w->B) return fail(TP_ERR_NULL, "Wqkv, Wo, A and B are required");
+  TP_TRY(attn_check(X, w->Wqkv, w->Wo, b, s, h, heads, t, dtype));
+  if (f <= 0 || f % t != 0) return fail(TP_ERR_SHAPE, "f must be positive and divisible by t");
+  TP_TRY(check_rows({f}));
+  if (h > layernorm_max_h()) return fail(TP_ERR_UNSUPPORTED, "layernorm: h must be at most 16384");
+  TP_TRY(check_ptrs_aligned({X, w->ln1_g, w->ln1_b, w->Wqkv, w->Wo, w->ln2_g, w->ln2_b, w->A,
+                             w->bA, w->B, w->bB}));
+  return TP_OK;
+}
+
+tp_status block_fwd(const void* X, const tp_block_weights* w, void* X2, tp_block_saves* sv,
+                    int64_t b, int64_t s, int64_t h, int64_t f, int heads, int t, float eps,
+                    tp_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  TP_TRY(block_check(X, w, b, s, h, f, heads, t, dtype));
+  if (!X2 || !sv) return fail(TP_ERR_NULL, "X2 and the saves are required");
+  if (!sv->Xn1 || !sv->mean1 || !sv->rstd1 || !sv->QKV || !sv->O || !sv->LSE || !sv->X1 ||
+      !sv->Xn2 || !sv->mean2 || !sv->rstd2 || !sv->Y)
+    return fail(TP_ERR_NULL, "every tp_block_saves pointer is required");
+  TP_TRY(check_ptrs_aligned({X2, sv->Xn1, sv->QKV, sv->O, sv->LSE, sv->X1, sv->Xn2, sv->Y, ws}));
+  const int64_t M = b * s;
+  if (ws == nullptr || ws_bytes < block_fwd_ws(M, h, f, heads))
+    return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
+  // X1 = X + Attn(LN1(X))
+  TP_TRY(launch_layernorm_fwd(X, w->ln1_g, w->ln1_b, sv->Xn1, sv->mean1, sv->rstd1, M, h, eps,
+                              false, stream));
+  TP_TRY(attn_fwd(sv->Xn1, w->Wqkv, w->Wo, sv->X1, sv->QKV, sv->O, sv->LSE, b, s, h, heads, t, 1,
+                  dtype, ws, ws_bytes, stream, X));
+  // X2 = X1 + MLP(LN2(X1))
+  TP_TRY(launch_layernorm_fwd(sv->X1, w->ln2_g, w->ln2_b, sv->Xn2, sv->mean2, sv->rstd2, M, h,
+                              eps, false, stream));
+  return mlp_fwd(sv->Xn2, w->A, w->bA, w->B, w->bB, X2, sv->Y, M, h, f, t, dtype, ws, ws_bytes,
+                 stream, sv->X1);
+}
+
+tp_status block_bwd(const void* X, const tp_block_weights* w, const tp_block_saves* sv,
+                    const void* dX2, void* dX, const tp_block_grads* g, int64_t b, int64_t s,
+                    int64_t h, int64_t f, int heads, int t, float eps, tp_dtype dtype, void* ws,
+                    size_t ws_bytes, cudaStream_t stream) {
+  (void)eps;
+  TP_TRY(block_check(X, w, b, s, h, f, heads, t, dtype));
+  if (!sv || !dX2 || !dX || !g) return fail(TP_ERR_NULL, "saves, dX2, dX and the grads are required");
+  if (!sv->Xn1 || !sv->mean1 || !sv->rstd1 || !sv->QKV || !sv->O || !sv->LSE || !sv->X1 ||
+      !sv->Xn2 || !sv->mean2 || !sv->rstd2 || !sv->Y)
+    return fail(TP_ERR_NULL, "every tp_block_saves pointer is required");
+  if (!g->dWqkv || !g->dWo || !g->dA || !g->dB)
+    return fail(TP_ERR_NULL, "dWqkv, dWo, dA and dB are required");
+  TP_TRY(check_ptrs_aligned({dX2, dX, g->dln1_g, g->dln1_b, g->dWqkv, g->dWo, g->dln2_g, g->dln2_b,
+                             g->dA, g->dbA, g->dB, g->dbB, ws}));
+  const int64_t M = b * s;
+  if (ws == nullptr || ws_bytes < block_bwd_ws(M, h, f, heads))
+    return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
+  Carve c(ws, ws_bytes);
+  void* dXn2 = c.take(M * h * 2);
+  void* dX1 = c.take(M * h * 2);
+  void* dXn1 = c.take(M * h * 2);
+  void* inner = c.take(0);
+  const size_t inner_bytes = ws_bytes - (static_cast<char*>(inner) - static_cast<char*>(ws));
+  // MLP sublayer, then LN2 with the residual path's gradient joining: dX1.
+  TP_TRY(mlp_bwd(sv->Xn2, w->A, w->bA, w->B, sv->Y, dX2, dXn2, g->dA, g->dbA, g->dB, g->dbB, M, h,
+                 f, t, dtype, inner, inner_bytes, stream));
+  TP_TRY(launch_layernorm_bwd(sv->X1, w->ln2_g, sv->mean2, sv->rstd2, dXn2, dX2, dX1, g->dln2_g,
+                              g->dln2_b, M, h, false, inner, stream));
+  // Attention sublayer, then LN1 with the residual gradient: dX.
+  TP_TRY(attn_bwd(sv->Xn1, w->Wqkv, w->Wo, sv->QKV, sv->O, sv->LSE, dX1, dXn1, g->dWqkv, g->dWo, b,
+                  s, h, heads, t, 1, dtype, inner, inner_bytes, stream));
+  return launch_layernorm_bwd(X, w->ln1_g, sv->mean1, sv->rstd1, dXn1, dX1, dX, g->dln1_g,
+                              g->dln1_b, M, h, false, inner, stream);
+}
+
 }  // namespace
 }  // namespace tp
 
@@ -562,6 +665,43 @@ tp_status tp_attn_bwd(const void* X, const void* Wqkv, const void* Wo, const voi
                            static_cast<cudaStream_t>(stream));)
 }
 
+tp_status tp_layernorm_fwd(const void* X, const void* gamma, const void* beta, void* Y,
+                           float* mean, float* rstd, int64_t M, int64_t h, float eps,
+                           tp_dtype dtype, void* stream) {
+  TP_GUARD(TP_TRY(ln_check(X, Y, M, h, dtype));
+           TP_TRY(check_ptrs_aligned({X, gamma, beta, Y, mean, rstd}));
+           return launch_layernorm_fwd(X, gamma, beta, Y, mean, rstd, M, h, eps, dtype == TP_F32,
+                                       static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_layernorm_bwd(const void* X, const void* gamma, const float* mean,
+                           const float* rstd, const void* dY, const void* dR, void* dX,
+                           void* dgamma, void* dbeta, int64_t M, int64_t h, tp_dtype dtype,
+                           void* ws, size_t ws_bytes, void* stream) {
+  TP_GUARD(TP_TRY(ln_check(X, dX, M, h, dtype));
+           if (!mean || !rstd || !dY) return fail(TP_ERR_NULL, "mean, rstd and dY are required");
+           TP_TRY(check_ptrs_aligned({X, gamma, dY, dR, dX, dgamma, dbeta, ws}));
+           if (ws == nullptr || ws_bytes < ln_bwd_ws(M, h))
+             return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
+           return launch_layernorm_bwd(X, gamma, mean, rstd, dY, dR, dX, dgamma, dbeta, M, h,
+                                       dtype == TP_F32, ws, static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_block_fwd(const void* X, const tp_block_weights* w, void* X2, tp_block_saves* saves,
+                       int64_t b, int64_t s, int64_t h, int64_t f, int heads, int t, float eps,
+                       tp_dtype dtype, void* ws, size_t ws_bytes, void* stream) {
+  TP_GUARD(return block_fwd(X, w, X2, saves, b, s, h, f, heads, t, eps, dtype, ws, ws_bytes,
+                            static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_block_bwd(const void* X, const tp_block_weights* w, const tp_block_saves* saves,
+                       const void* dX2, void* dX, const tp_block_grads* g, int64_t b, int64_t s,
+                       int64_t h, int64_t f, int heads, int t, float eps, tp_dtype dtype,
+                       void* ws, size_t ws_bytes, void* stream) {
+  TP_GUARD(return block_bwd(X, w, saves, dX2, dX, g, b, s, h, f, heads, t, eps, dtype, ws,
+                            ws_bytes, static_cast<cudaStream_t>(stream));)
+}
+
 size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, int t,
                          tp_dtype dtype) {
   try {
@@ -571,6 +711,9 @@ size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, i
       case TP_OP_MLP_BWD: return f > 0 ? mlp_bwd_ws(M, h, f, dtype) : 0;
       case TP_OP_ATTN_FWD: return heads > 0 ? attn_fwd_ws(M, h, heads) : 0;
       case TP_OP_ATTN_BWD: return heads > 0 ? attn_bwd_ws(M, h, heads) : 0;
+      case TP_OP_LN_BWD: return ln_bwd_ws(M, h);
+      case TP_OP_BLOCK_FWD: return (heads > 0 && f > 0) ? block_fwd_ws(M, h, f, heads) : 0;
+      case TP_OP_BLOCK_BWD: return (heads > 0 && f > 0) ? block_bwd_ws(M, h, f, heads) : 0;
     }
   } catch (...) {
   }

@@ -193,6 +193,12 @@ __device__ __forceinline__ void epilogue_row32(float (&v)[32], int row, int col0
 #pragma unroll
       for (int i = 0; i < 8; ++i) x[i] += bb[i];
     }
+    if (EPI == kEpiResidual) {
+      float rr[8];
+      unpack8(*reinterpret_cast<const uint4*>(a.aux + (long long)row * a.ldaux + col), rr);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] += rr[i];
+    }
     if (EPI == kEpiBiasGelu) {
       if (a.out2 != nullptr)
         *reinterpret_cast<uint4*>(a.out2 + (long long)row * a.ldo2 + col) = pack8(x);
@@ -767,6 +773,8 @@ tp_status dispatch(const Gemm& g, cudaStream_t s) {
   const bool plain_out = !g.out_f32 && !g.out_f16;
   if (g.epi == kEpiBiasGelu) {
     if (ak && !bk && plain_out) return launch_impl<BN, true, false, kEpiBiasGelu, kOutBF16>(g, s);
+  } else if (g.epi == kEpiResidual) {
+    if (ak && !bk && plain_out) return launch_impl<BN, true, false, kEpiResidual, kOutBF16>(g, s);
   } else if (g.epi == kEpiDGelu) {
     if (ak && bk && plain_out) return launch_impl<BN, true, true, kEpiDGelu, kOutBF16>(g, s);
   } else {
@@ -865,6 +873,8 @@ tp_status dispatch_pair(const Gemm& g, cudaStream_t s) {
   const bool plain_out = !g.out_f32 && !g.out_f16;
   if (g.epi == kEpiBiasGelu) {
     if (ak && !bk && plain_out) return launch_pair<true, false, kEpiBiasGelu, kOutBF16>(g, s);
+  } else if (g.epi == kEpiResidual) {
+    if (ak && !bk && plain_out) return launch_pair<true, false, kEpiResidual, kOutBF16>(g, s);
   } else if (g.epi == kEpiDGelu) {
     if (ak && bk && plain_out) return launch_pair<true, true, kEpiDGelu, kOutBF16>(g, s);
   } else {

@@ -42,6 +42,7 @@ enum Epi : int {
   kEpiStore = 0,     // out = acc (+ bias[col])
   kEpiBiasGelu = 1,  // v = acc + bias[col]; out = GeLU(v); out2 = v (if out2)
   kEpiDGelu = 2,     // y = aux[row,col]; out = acc * GeLU'(y); out2 = GeLU(y) (if out2)
+  kEpiResidual = 3,  // out = acc (+ bias[col]) + aux[row,col]: a residual addition
 };
 
 // One operand of D[M,N] = sum_k A(m,k) B(k,n) stored as a row-major matrix.
@@ -92,6 +93,17 @@ tp_status launch_gemm_f32(const Gemm& g, cudaStream_t stream);
 size_t colsum_scratch_bytes(int64_t rows, int64_t cols);
 tp_status launch_colsum(const void* in, int64_t rows, int64_t cols, bool f32, void* out,
                         void* scratch, cudaStream_t stream);
+
+// LayerNorm over rows of [M, h] (h % 8 == 0, h <= layernorm_max_h()).
+int64_t layernorm_max_h();
+tp_status launch_layernorm_fwd(const void* X, const void* gamma, const void* beta, void* Y,
+                               float* mean, float* rstd, int64_t M, int64_t h, float eps,
+                               bool f32, cudaStream_t stream);
+size_t layernorm_bwd_scratch_bytes(int64_t M, int64_t h);
+tp_status launch_layernorm_bwd(const void* X, const void* gamma, const float* mean,
+                               const float* rstd, const void* dY, const void* dR, void* dX,
+                               void* dgamma, void* dbeta, int64_t M, int64_t h, bool f32,
+                               void* scratch, cudaStream_t stream);
 
 // Attention core (per head causal softmax attention), bf16 with d = 128.
 struct AttnShape {

@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(256) gemm_f32_simt(const ArgsF32 a) {
       if (c >= a.N) continue;
       float x = acc[i][j];
       if (EPI != kEpiDGelu && a.bias != nullptr) x += a.bias[c];
+      if (EPI == kEpiResidual) x += a.aux[(long long)r * a.ldaux + c];
       if (EPI == kEpiBiasGelu) {
         if (a.out2 != nullptr) a.out2[(long long)r * a.ldo2 + c] = x;
         x = gelu32(x);
@@ -142,6 +143,7 @@ tp_status launch_gemm_f32(const Gemm& g, cudaStream_t stream) {
     switch (g.epi) {
       case kEpiBiasGelu: gemm_f32_simt<kEpiBiasGelu><<<grid, 256, 0, stream>>>(a); break;
       case kEpiDGelu: gemm_f32_simt<kEpiDGelu><<<grid, 256, 0, stream>>>(a); break;
+      case kEpiResidual: gemm_f32_simt<kEpiResidual><<<grid, 256, 0, stream>>>(a); break;
       default: gemm_f32_simt<kEpiStore><<<grid, 256, 0, stream>>>(a); break;
     }
   }

@@ -134,3 +134,23 @@ def test_workspace_sizes(lib):
     assert ws(L.TP_OP_ATTN_BWD, M, h, 0, 96, 8, L.TP_BF16) >= M * 7 * h * 2
     assert ws(L.TP_OP_MLP_FWD, 0, h, f, 0, 8, L.TP_BF16) == 0
     assert ws(L.TP_OP_ATTN_FWD, M, h, 0, 0, 8, L.TP_BF16) == 0
+
+
+def test_layernorm_and_block_validation(lib):
+    import ctypes as C
+    big = 1 << 40
+    assert lib.tp_layernorm_fwd(None, None, None, P[1], None, None, 4, 64, 1e-5, L.TP_BF16, None) == L.TP_ERR_NULL
+    assert lib.tp_layernorm_fwd(P[0], None, None, P[1], None, None, 4, 60, 1e-5, L.TP_BF16, None) == L.TP_ERR_ALIGN
+    assert lib.tp_layernorm_fwd(P[0], None, None, P[1], None, None, 4, 16392, 1e-5, L.TP_BF16, None) == L.TP_ERR_UNSUPPORTED
+    assert lib.tp_layernorm_bwd(P[0], None, None, P[2], P[3], None, P[4], None, None, 4, 64, L.TP_BF16, P[9], big, None) == L.TP_ERR_NULL
+    assert lib.tp_layernorm_bwd(P[0], None, P[1], P[2], P[3], None, P[4], None, None, 4, 64, L.TP_BF16, None, 0, None) == L.TP_ERR_WORKSPACE
+    W = L.BlockWeights(*([None] * 10))
+    S = L.BlockSaves(*([P[5]] * 11))
+    assert lib.tp_block_fwd(P[0], C.byref(W), P[1], C.byref(S), 1, 64, 512, 2048, 4, 2, 1e-5, L.TP_BF16, P[9], big, None) == L.TP_ERR_NULL
+    W = L.BlockWeights(None, None, P[2], P[3], None, None, P[4], None, P[6], None)
+    assert lib.tp_block_fwd(P[0], C.byref(W), P[1], C.byref(S), 1, 64, 512, 2044, 4, 2, 1e-5, L.TP_BF16, P[9], big, None) == L.TP_ERR_SHAPE
+    S0 = L.BlockSaves(*([P[5]] * 10 + [None]))
+    assert lib.tp_block_fwd(P[0], C.byref(W), P[1], C.byref(S0), 1, 64, 512, 2048, 4, 2, 1e-5, L.TP_BF16, P[9], big, None) == L.TP_ERR_NULL
+    assert lib.tp_block_fwd(P[0], C.byref(W), P[1], C.byref(S), 1, 64, 512, 2048, 4, 2, 1e-5, L.TP_F32, P[9], big, None) == L.TP_ERR_UNSUPPORTED
+    assert lib.tp_workspace_size(L.TP_OP_BLOCK_BWD, 2048, 12288, 49152, 96, 8, L.TP_BF16) > 3 * 2048 * 12288 * 2
+    assert lib.tp_workspace_size(L.TP_OP_LN_BWD, 2048, 12288, 0, 0, 1, L.TP_BF16) >= 2 * 296 * 12288 * 4
