@@ -148,7 +148,7 @@ def test_layernorm_and_block_validation(lib):
     S = L.BlockSaves(*([P[5]] * 11))
     assert lib.tp_block_fwd(P[0], C.byref(W), P[1], C.byref(S), 1, 64, 512, 2048, 4, 2, 1e-5, L.TP_BF16, P[9], big, None) == L.TP_ERR_NULL
     W = L.BlockWeights(None, None, P[2], P[3], None, None, P[4], None, P[6], None)
-    assert lib.tp_block_fwd(P[0], C.byref(W), P[1], C.byref(S), 1, 64, 512, 2044, 4, 2, 1e-5, L.TP_BF16, P[9], big, None) == L.TP_ERR_SHAPE
+    assert lib.tp_block_fwd(P[0], C.byref(W), P[1], C.byref(S), 1, 64, 512, 2047, 4, 2, 1e-5, L.TP_BF16, P[9], big, None) == L.TP_ERR_SHAPE
     S0 = L.BlockSaves(*([P[5]] * 10 + [None]))
     assert lib.tp_block_fwd(P[0], C.byref(W), P[1], C.byref(S0), 1, 64, 512, 2048, 4, 2, 1e-5, L.TP_BF16, P[9], big, None) == L.TP_ERR_NULL
     assert lib.tp_block_fwd(P[0], C.byref(W), P[1], C.byref(S), 1, 64, 512, 2048, 4, 2, 1e-5, L.TP_F32, P[9], big, None) == L.TP_ERR_UNSUPPORTED
