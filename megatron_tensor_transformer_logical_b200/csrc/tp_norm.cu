@@ -72,7 +72,7 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   __syncthreads();
   float t = lane < kLnThreads / 32 ? red[lane] : 0.0f;
 #pragma unroll
-  for (int s = 8; s > 0; s >>= 1) t += __shfl_xor_sync(0xffffffffu, t, s);
+  for (int s = 16; s > 0; s >>= 1) t += __shfl_xor_sync(0xffffffffu, t, s);  // every lane: the sum
   return t;
 }
 
