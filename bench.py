@@ -191,6 +191,32 @@ class LayerStep:
         self.attn()
         self.mlp()
 
+    def make_block(self, dev):
+        """Buffers of the full Transformer block (LayerNorm + residual around
+        the same attention and MLP weights)."""
+        L, wl = self.L, self.wl
+        M, h, f = wl.M, wl.h, wl.f
+        bf, f32 = torch.bfloat16, torch.float32
+        e = lambda *sh, dt=bf: torch.empty(*sh, dtype=dt, device=dev)
+        ones, zeros = torch.ones(h, dtype=bf, device=dev), torch.zeros(h, dtype=bf, device=dev)
+        self.bw = {"ln1_g": ones, "ln1_b": zeros, "Wqkv": self.Wqkv, "Wo": self.Wo,
+                   "ln2_g": ones, "ln2_b": zeros, "A": self.A, "B": self.B}
+        self.bsv = {"Xn1": e(M, h), "mean1": e(M, dt=f32), "rstd1": e(M, dt=f32),
+                    "QKV": self.QKV, "O": self.O, "LSE": self.LSE, "X1": e(M, h), "Xn2": e(M, h),
+                    "mean2": e(M, dt=f32), "rstd2": e(M, dt=f32), "Y": self.Y}
+        self.bg = {"dln1_g": e(h), "dln1_b": e(h), "dWqkv": self.dWqkv, "dWo": self.dWo,
+                   "dln2_g": e(h), "dln2_b": e(h), "dA": self.dA, "dB": self.dB}
+        self.bX2, self.bdX = e(M, h), e(M, h)
+        self.bws_f = L.workspace(L.TP_OP_BLOCK_FWD, M, h, f, wl.heads, wl.t, L.TP_BF16, device=dev)
+        self.bws_b = L.workspace(L.TP_OP_BLOCK_BWD, M, h, f, wl.heads, wl.t, L.TP_BF16, device=dev)
+
+    def block(self):
+        L, wl = self.L, self.wl
+        L.tp_block_fwd(self.X, self.bw, self.bX2, self.bsv, wl.b, wl.s, wl.f, wl.heads, wl.t, 1e-5,
+                       self.bws_f)
+        L.tp_block_bwd(self.X, self.bw, self.bsv, self.dZ, self.bdX, self.bg, wl.b, wl.s, wl.f,
+                       wl.heads, wl.t, 1e-5, self.bws_b)
+
     def outputs(self):
         return (self.Za, self.Zm, self.dXa, self.dXm)
 
@@ -253,6 +279,13 @@ def run_libtp(args, rank, world, local_rank, dist):
     barrier()
     mlp_rec_ms = timed(lambda: st.mlp(save_y=False), args.steps, stream)
     barrier()
+    # The full Transformer block: LayerNorm and residual around both sublayers.
+    st.make_block(dev)
+    for _ in range(2):
+        st.block()
+    barrier()
+    block_ms = timed(st.block, args.steps, stream)
+    barrier()
 
     # End to end through the public API: per step, the step's inputs (X, dZ)
     # copied from pinned host memory and its results (Z and dX of both
@@ -289,6 +322,7 @@ def run_libtp(args, rank, world, local_rank, dist):
         return float(t.item())
 
     ms, mlp_ms, mlp_rec_ms = maxall(ms), maxall(mlp_ms), maxall(mlp_rec_ms)
+    block_ms = maxall(block_ms)
     e2e_ms = maxall(e2e_ms) if e2e_ms is not None else None
     if rank != 0:
         return None
@@ -344,6 +378,11 @@ def run_libtp(args, rank, world, local_rank, dist):
         "mlp_fwd_bwd": {"tflops": round(mlp_tflops, 2), "ms_per_step": round(mlp_ms / args.steps, 4),
                         "frac_of_nominal_2250": round(mlp_tflops / world / NOMINAL_BF16_TFLOPS, 4),
                         "frac_of_measured_sustained": round(mlp_tflops / world / peak, 4)},
+        "block_fwd_bwd": {
+            "what": "LN1 -> attention -> +residual -> LN2 -> MLP -> +residual, forward and backward",
+            "ms_per_step": round(block_ms / args.steps, 4),
+            "tflops": round(world * fl["total"] / (block_ms / args.steps * 1e-3) / 1e12, 2),
+            "overhead_vs_layer_step": round(block_ms / ms - 1.0, 4)},
         "activation_policy": {
             "save_y": {"mlp_ms_per_step": round(mlp_ms / args.steps, 4),
                        "bytes_kept_fwd_to_bwd": wl.M * wl.f * 2},
