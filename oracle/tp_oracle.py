@@ -64,7 +64,8 @@ __all__ = [
     "mlp_bwd", "mlp_bwd_parallel", "head_columns", "group_columns",
     "attention_core", "attention_core_bwd", "attn_fwd", "attn_fwd_parallel",
     "attn_bwd", "attn_bwd_parallel", "layernorm_fwd", "layernorm_bwd", "block_fwd",
-    "block_bwd", "max_rel_error", "normwise_error",
+    "block_bwd", "vocab_embed_fwd", "vocab_embed_fwd_parallel", "vocab_embed_bwd",
+    "vocab_ce_fwd", "vocab_ce_fwd_parallel", "vocab_ce_bwd", "max_rel_error", "normwise_error",
 ]
 
 _SQRT2 = math.sqrt(2.0)
@@ -508,6 +509,126 @@ def block_bwd(X, w, dX2, b: int, s: int, heads: int, eps: float = 1e-5, causal: 
             "dln1_g": l1["dgamma"], "dln1_b": l1["dbeta"], "dWqkv": ab["dWqkv"], "dWo": ab["dWo"],
             "dln2_g": l2["dgamma"], "dln2_b": l2["dbeta"], "dA": mb["dA"], "dbA": mb["dbA"],
             "dB": mb["dB"], "dbB": mb["dbB"]}
+
+
+# ---------------------------------------------------------------------------
+# Vocabulary-parallel embedding and cross-entropy ([P3] §4.1, §4.2)
+# ---------------------------------------------------------------------------
+
+def vocab_embed_fwd(ids, E):
+    """Unpartitioned lookup: Y[r] = E[ids[r]]; an id outside [0, V) gives 0."""
+    ids = np.asarray(ids, dtype=np.int64)
+    E = _f64(E)
+    Y = np.zeros((len(ids), E.shape[1]))
+    ok = (ids >= 0) & (ids < E.shape[0])
+    Y[ok] = E[ids[ok]]
+    return Y
+
+
+def vocab_embed_fwd_parallel(ids, E, t: int):
+    """[P3] §4.1: E split by vocabulary rows; shard i looks up the ids in its
+    range [i*V/t, (i+1)*V/t) and returns a zero vector for the others; the
+    partial results are summed (the AllReduce)."""
+    ids = np.asarray(ids, dtype=np.int64)
+    shards = split_rows(E, t)
+    v = shards[0].shape[0]
+    Y = np.zeros((len(ids), shards[0].shape[1]))
+    for i, Ei in enumerate(shards):
+        local = ids - i * v
+        mine = (local >= 0) & (local < v)
+        part = np.zeros_like(Y)
+        part[mine] = Ei[local[mine]]
+        Y = Y + part
+    return Y
+
+
+def vocab_embed_bwd(ids, dY, V: int):
+    """dE[v] = sum of dY[r] over the rows r with ids[r] == v."""
+    ids = np.asarray(ids, dtype=np.int64)
+    dY = _f64(dY)
+    dE = np.zeros((V, dY.shape[1]))
+    ok = (ids >= 0) & (ids < V)
+    np.add.at(dE, ids[ok], dY[ok])
+    return dE
+
+
+def _valid_targets(targets, V: int):
+    """Rows whose target lies outside [0, V) are ignored: loss 0, gradient 0
+    (a reading: the pages only treat in-range targets)."""
+    targets = np.asarray(targets, dtype=np.int64)
+    return targets, (targets >= 0) & (targets < V)
+
+
+def vocab_ce_fwd(X, E, targets):
+    """Unpartitioned cross-entropy of logits = X @ E^T (E [V, h], tied with the
+    input embedding, [P3] §4.2): loss[r] = logsumexp(logits[r]) - logits[r, t_r],
+    total = sum of loss[r] over the rows."""
+    X, E = _f64(X), _f64(E)
+    targets, ok = _valid_targets(targets, E.shape[0])
+    z = X @ E.T
+    m = z.max(axis=1)
+    lse = m + np.log(np.exp(z - m[:, None]).sum(axis=1))
+    rows = np.nonzero(ok)[0]
+    loss = np.zeros(len(targets))
+    loss[rows] = lse[rows] - z[rows, targets[rows]]
+    return {"loss": loss, "lse": lse, "total": float(loss.sum())}
+
+
+def vocab_ce_fwd_parallel(X, E, targets, t: int):
+    """[P3] §4.2 steps 1-6 on t vocabulary shards E_i (rows of E):
+    1. shard i computes its logits z_i = X @ E_i^T;
+    2. its exponential sum, taken relative to the shard's own row maximum
+       (a reading: the page's step 2 has no max subtraction; this is the
+       same value, written so that it cannot overflow);
+    3. the shards' sums are combined, rescaled to the largest maximum, into
+       the global denominator (the AllReduce of b*s values), lse = log of it;
+    4-5. the shard that owns a row's target takes its logit and forms that
+       row's loss, lse - z_target; the shard's local loss is the sum of the
+       losses of the rows whose targets it owns;
+    6. the total loss is the sum of the shards' local losses (the AllReduce
+       of t values)."""
+    X = _f64(X)
+    targets, ok = _valid_targets(targets, E.shape[0])
+    shards = split_rows(E, t)
+    v = shards[0].shape[0]
+    M = X.shape[0]
+    ms, ss = [], []
+    for Ei in shards:                                    # steps 1-2
+        zi = X @ Ei.T
+        mi = zi.max(axis=1)
+        ms.append(mi)
+        ss.append(np.exp(zi - mi[:, None]).sum(axis=1))
+    m = np.max(np.stack(ms), axis=0)                     # step 3
+    total_exp = np.zeros(M)
+    for mi, si in zip(ms, ss):
+        total_exp = total_exp + si * np.exp(mi - m)
+    lse = m + np.log(total_exp)
+    loss = np.zeros(M)
+    local_losses = []
+    for i, Ei in enumerate(shards):                      # steps 4-5
+        local = targets - i * v
+        mine = ok & (local >= 0) & (local < v)
+        rows = np.nonzero(mine)[0]
+        z_t = (X[rows] * _f64(Ei)[local[rows]]).sum(axis=1)
+        loss[rows] = lse[rows] - z_t
+        local_losses.append(float(loss[rows].sum()))
+    return {"loss": loss, "lse": lse, "total": float(sum(local_losses))}   # step 6
+
+
+def vocab_ce_bwd(X, E, targets, dloss):
+    """Gradient of sum_r dloss[r] * loss[r]: dlogits = (softmax - onehot) * dloss
+    on the rows with a valid target (zero on ignored rows), dX = dlogits @ E,
+    dE = dlogits^T @ X."""
+    X, E = _f64(X), _f64(E)
+    targets, ok = _valid_targets(targets, E.shape[0])
+    z = X @ E.T
+    p = np.exp(z - z.max(axis=1, keepdims=True))
+    p = p / p.sum(axis=1, keepdims=True)
+    rows = np.nonzero(ok)[0]
+    p[rows, targets[rows]] -= 1.0
+    p[~ok] = 0.0
+    g = p * _f64(dloss)[:, None]
+    return {"dX": g @ E, "dE": g.T @ X, "dlogits": g}
 
 
 # ---------------------------------------------------------------------------

@@ -520,3 +520,102 @@ def test_planted_layernorm_mistake_is_caught():
     m = _mutant(layernorm_fwd=_ln_no_centering)
     with pytest.raises(AssertionError):
         check_layernorm(m)
+
+
+# ---------------------------------------------------------------------------
+# Vocabulary-parallel embedding and cross-entropy ([P3] §4.1, §4.2)
+# ---------------------------------------------------------------------------
+
+def check_vocab(o):
+    r = _rng(50)
+    V, h = 24, 5
+    E = r.standard_normal((V, h))
+    ids = np.array([0, 23, 7, 7, -1, 24, 12, 3])
+    Y = o.vocab_embed_fwd(ids, E)
+    for i, v in enumerate(ids):  # exact gather; out-of-range ids give zeros
+        assert np.array_equal(Y[i], E[v] if 0 <= v < V else np.zeros(h))
+    for t in (1, 2, 3, 4, 8):
+        assert np.array_equal(o.vocab_embed_fwd_parallel(ids, E, t), Y)
+    dY = _int_mat((8, h), 51)
+    dE = o.vocab_embed_bwd(ids, dY, V)
+    assert np.array_equal(dE[7], dY[2] + dY[3]) and np.array_equal(dE[1], np.zeros(h))
+    assert dE.sum() == dY[[0, 1, 2, 3, 6, 7]].sum()
+    # cross-entropy: all-zero logits give log V; brute force on one row
+    X = r.standard_normal((6, h))
+    tg = np.array([0, 5, 23, 11, 11, 2])
+    assert np.allclose(o.vocab_ce_fwd(X, np.zeros((V, h)), tg)["loss"], math.log(V), rtol=0, atol=1e-14)
+    ce = o.vocab_ce_fwd(X, E, tg)
+    for i in range(6):
+        zs = [sum(X[i, k] * E[v, k] for k in range(h)) for v in range(V)]
+        ref = math.log(sum(math.exp(z) for z in zs)) - zs[tg[i]]
+        assert abs(ce["loss"][i] - ref) < 1e-12
+    assert abs(ce["total"] - sum(ce["loss"])) < 1e-12
+    for t in (1, 2, 3, 4, 8):
+        cp = o.vocab_ce_fwd_parallel(X, E, tg, t)
+        assert np.max(np.abs(cp["loss"] - ce["loss"])) < 1e-12
+        assert np.max(np.abs(cp["lse"] - ce["lse"])) < 1e-12
+        assert abs(cp["total"] - ce["total"]) < 1e-11
+    # large logits: the max-subtracted form stays finite where exp overflows
+    big = o.vocab_ce_fwd_parallel(X * 400.0, E, tg, 4)
+    assert np.all(np.isfinite(big["loss"])) and np.all(big["loss"] >= -1e-9)
+    # an ignored row (target out of range) has loss 0 and no gradient
+    tg2 = tg.copy()
+    tg2[3] = -1
+    tg2[4] = V
+    ce2 = o.vocab_ce_fwd_parallel(X, E, tg2, 3)
+    assert ce2["loss"][3] == 0 and ce2["loss"][4] == 0
+    assert abs(ce2["loss"][[0, 1, 2, 5]] - ce["loss"][[0, 1, 2, 5]]).max() < 1e-12
+    g2 = o.vocab_ce_bwd(X, E, tg2, np.ones(6))
+    assert not g2["dlogits"][3].any() and not g2["dX"][4].any()
+    # softmax rows sum to one, so each valid dlogits row sums to zero
+    assert np.max(np.abs(g2["dlogits"].sum(axis=1))) < 1e-12
+    dl = r.standard_normal(6)
+    loss = lambda: float(np.sum(dl * o.vocab_ce_fwd(X, E, tg)["loss"]))
+    g = o.vocab_ce_bwd(X, E, tg, dl)
+    assert np.max(np.abs(g["dX"] - _fd_grad(loss, X))) < 1e-7
+    assert np.max(np.abs(g["dE"] - _fd_grad(loss, E))) < 1e-7
+
+
+def test_vocab_pins():
+    check_vocab(O)
+
+
+def _ce_without_target(X, E, targets):
+    X, E = np.asarray(X, dtype=np.float64), np.asarray(E, dtype=np.float64)
+    z = X @ E.T
+    m = z.max(axis=1)
+    lse = m + np.log(np.exp(z - m[:, None]).sum(axis=1))
+    loss = lse - z[:, 0]  # mistake: always class 0
+    return {"loss": loss, "lse": lse, "total": float(loss.sum())}
+
+
+def _ce_parallel_unscaled(X, E, targets, t):
+    """Mistake: the shards' exponential sums are added without rescaling
+    them to a common maximum."""
+    X = np.asarray(X, dtype=np.float64)
+    targets = np.asarray(targets, dtype=np.int64)
+    shards = O.split_rows(E, t)
+    tot, ms = 0.0, []
+    for Ei in shards:
+        zi = X @ np.asarray(Ei, dtype=np.float64).T
+        mi = zi.max(axis=1)
+        ms.append(mi)
+        tot = tot + np.exp(zi - mi[:, None]).sum(axis=1)
+    lse = np.max(np.stack(ms), axis=0) + np.log(tot)
+    z = X @ np.asarray(E, dtype=np.float64).T
+    loss = lse - z[np.arange(len(targets)), np.clip(targets, 0, z.shape[1] - 1)]
+    return {"loss": loss, "lse": lse, "total": float(loss.sum())}
+
+
+def _embed_parallel_off_by_one(ids, E, t):
+    ids = np.asarray(ids)
+    return O.vocab_embed_fwd_parallel(np.where(ids >= 0, ids + 1, ids), E, t)
+
+
+@pytest.mark.parametrize("mutant", [dict(vocab_ce_fwd=_ce_without_target),
+                                    dict(vocab_ce_fwd_parallel=_ce_parallel_unscaled),
+                                    dict(vocab_embed_fwd_parallel=_embed_parallel_off_by_one)],
+                         ids=["ce_target", "ce_unscaled", "embed_offset"])
+def test_planted_vocab_mistake_is_caught(mutant):
+    with pytest.raises(AssertionError):
+        check_vocab(_mutant(**mutant))
