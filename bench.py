@@ -221,6 +221,83 @@ class LayerStep:
         return (self.Za, self.Zm, self.dXa, self.dXm)
 
 
+class VocabStep:
+    """The vocabulary-parallel embedding and loss with tied weights, forward
+    and backward: Y = embed(ids); loss = CE(X @ E^T, targets);
+    dE = CE's dE + scatter(dY) (X and dY stand for the hidden states and
+    gradient of the layers in between, which this step does not run)."""
+
+    VOCAB_NAMES = {1: "embed_gather", 2: "embed_scatter_add", 3: "loss_combine",
+                   4: "softmax_grad"}
+
+    def __init__(self, wl, dev):
+        from megatron_tensor_transformer_logical_b200 import binding as L
+        from megatron_tensor_transformer_logical_b200.inputs import make_vocab_inputs
+        self.L, self.wl = L, wl
+        d = {k: v.to(dev) for k, v in make_vocab_inputs(wl).items()}
+        self.ids, self.targets, self.E, self.X, self.dY = (d[k] for k in
+                                                           ("ids", "targets", "E", "X", "dY"))
+        M, h, V = wl.M, wl.h, wl.vocab
+        bf, f32 = torch.bfloat16, torch.float32
+        self.Y = torch.empty(M, h, dtype=bf, device=dev)
+        self.logits = torch.empty(M, V, dtype=bf, device=dev)
+        self.lse = torch.empty(M, dtype=f32, device=dev)
+        self.loss = torch.empty(M, dtype=f32, device=dev)
+        self.total = torch.empty(1, dtype=f32, device=dev)
+        self.dX = torch.empty(M, h, dtype=bf, device=dev)
+        self.dE = torch.empty(V, h, dtype=bf, device=dev)
+        self.ws = L.workspace(L.TP_OP_VOCAB_CE_FWD, M, h, V, 0, wl.t, L.TP_BF16, device=dev)
+
+    def step(self):
+        L, t = self.L, self.wl.t
+        L.tp_vocab_embed_fwd(self.ids, self.E, self.Y, t)
+        L.tp_vocab_ce_fwd(self.X, self.E, self.targets, self.logits, self.lse, self.loss,
+                          self.total, t, self.ws)
+        L.tp_vocab_ce_bwd(self.X, self.E, self.targets, self.logits, self.lse, None, self.logits,
+                          self.dX, self.dE, t)
+        L.tp_vocab_embed_bwd(self.ids, self.dY, self.dE, self.dE, t)
+
+    def flops(self):
+        wl = self.wl
+        return 3 * 2.0 * wl.M * wl.vocab * wl.h
+
+
+def vocab_report(vs, steps, ms, records, peaks, world):
+    """Per-kernel times of the vocabulary step from the launch trace."""
+    per = {}
+    for r in records:
+        if r["kind"] == "vocab":
+            name = VocabStep.VOCAB_NAMES.get(r["tile"], str(r["tile"]))
+        elif r["kind"] == "gemm_tcgen05":
+            name = f'gemm {r["m"]}x{r["n"]}x{r["k"]}'
+        else:
+            name = r["kind"]
+        p = per.setdefault(name, {"ms": 0.0, "n": 0, "bytes": 0.0, "flops": 0.0})
+        p["ms"] += r["ms"]
+        p["n"] += 1
+        p["bytes"] += r["bytes"]
+        p["flops"] += r["flops"]
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    kernels = {}
+    for name, p in per.items():
+        k = {"ms_per_step": round(p["ms"] / steps, 4), "share": round(p["ms"] / ms, 4)}
+        if name.startswith("gemm"):
+            k["tflops"] = round(p["flops"] / (p["ms"] * 1e-3) / 1e12, 1)
+        else:
+            gbs = p["bytes"] / (p["ms"] * 1e-3) / 1e9
+            k["gbs"] = round(gbs, 1)
+            k["frac_of_measured_hbm"] = round(gbs / hbm, 4)
+        kernels[name] = k
+    wl = vs.wl
+    per_step = ms / steps
+    return {"what": "tied embedding + vocabulary-parallel cross-entropy, forward and backward",
+            "M": wl.M, "h": wl.h, "V": wl.vocab, "t": wl.t,
+            "ms_per_step": round(per_step, 4),
+            "tflops": round(world * vs.flops() / (per_step * 1e-3) / 1e12, 2),
+            "tokens_per_s": round(world * wl.M / (per_step * 1e-3), 1),
+            "kernels": kernels}
+
+
 def timed(fn, steps, stream):
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
@@ -286,6 +363,23 @@ def run_libtp(args, rank, world, local_rank, dist):
     barrier()
     block_ms = timed(st.block, args.steps, stream)
     barrier()
+    # The vocabulary-parallel embedding and loss (a second workload).
+    vocab_ms = vocab_records = None
+    vs = None
+    if not args.no_vocab:
+        del st.bsv, st.bg, st.bX2, st.bdX, st.bws_f, st.bws_b
+        vs = VocabStep(WORKLOADS[6], dev)
+        for _ in range(3):
+            vs.step()
+        torch.cuda.synchronize()
+        L.tp_device_status()
+        barrier()
+        L.tp_profile_enable(True)
+        vocab_ms = timed(vs.step, args.steps, stream)
+        vocab_records = L.tp_profile_records()
+        L.tp_profile_enable(False)
+        barrier()
+        del vs.logits
 
     # End to end through the public API: per step, the step's inputs (X, dZ)
     # copied from pinned host memory and its results (Z and dX of both
@@ -323,6 +417,7 @@ def run_libtp(args, rank, world, local_rank, dist):
 
     ms, mlp_ms, mlp_rec_ms = maxall(ms), maxall(mlp_ms), maxall(mlp_rec_ms)
     block_ms = maxall(block_ms)
+    vocab_ms = maxall(vocab_ms) if vocab_ms is not None else None
     e2e_ms = maxall(e2e_ms) if e2e_ms is not None else None
     if rank != 0:
         return None
@@ -401,6 +496,8 @@ def run_libtp(args, rank, world, local_rank, dist):
         "gpu_launches": launches,
         "clocks": clocks,
     }
+    if vocab_ms is not None:
+        out["vocab_fwd_bwd"] = vocab_report(vs, args.steps, vocab_ms, vocab_records, peaks, world)
     if e2e_ms is not None:
         out["e2e"] = {"value": round(world * fl["total"] / (e2e_ms / args.steps * 1e-3) / 1e12, 2),
                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -493,6 +590,7 @@ def main():
     ap.add_argument("--impl", choices=["libtp", "reference"], default="libtp")
     ap.add_argument("--workload", type=int, default=5, choices=[5])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-vocab", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=384)
     ap.add_argument("--ref-sample-tokens", type=int, default=64)

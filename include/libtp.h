@@ -12,6 +12,7 @@
  *   [P2] PyTorch tensor-parallel tutorial (page title "企业官网建设流程全解析"),
  *        §2.2 ParallelAttention, §3.2 ColumnParallelLinear, §3.3 the block.
  *   [P4] "5.1 Tensor并行与算子拆分" §1.1 tensor_parallel_split (divisibility).
+ *   [P3] §4.1 vocabulary-parallel embedding, §4.2 vocabulary-parallel loss.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -69,7 +70,8 @@ typedef enum tp_op {
   TP_OP_ATTN_BWD = 3,
   TP_OP_LN_BWD = 4,
   TP_OP_BLOCK_FWD = 5,
-  TP_OP_BLOCK_BWD = 6
+  TP_OP_BLOCK_BWD = 6,
+  TP_OP_VOCAB_CE_FWD = 7  /* f is the vocabulary size V */
 } tp_op;
 
 /*
@@ -293,6 +295,79 @@ tp_status tp_block_bwd(const void* X, const tp_block_weights* w, const tp_block_
                        void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Vocabulary-parallel input embedding ([P3] §4.1).  E [V, h] is split by rows
+ * into t vocabulary shards of V/t rows.  For each token, the shard whose range
+ * holds ids[r] supplies row ids[r] - i*V/t of its slice and every other shard
+ * supplies a zero row; the shards' rows are summed (the page's AllReduce).
+ * Exactly one shard contributes, so Y[r] = E[ids[r]] exactly; an id outside
+ * [0, V) belongs to no shard and gives a zero row.
+ *   ids [M] int32; E [V, h] dtype; Y [M, h] dtype.  M == 0 is a no-op.
+ * Errors: NULL ids / E / Y; M < 0 or V, h <= 0; V % t != 0 (TP_ERR_SHAPE);
+ *   alignment (h % 8, 16-byte pointers).
+ */
+tp_status tp_vocab_embed_fwd(const int32_t* ids, const void* E, void* Y, int64_t M, int64_t V,
+                             int64_t h, int t, tp_dtype dtype, void* stream);
+
+/*
+ * Backward of tp_vocab_embed_fwd: dE[v] = sum of dY[r] over the rows r with
+ * ids[r] == v (zero for a row of E no token used), plus dE_in[v] when dE_in
+ * is not NULL (the tied output layer's gradient, accumulated; dE_in may be
+ * dE itself).  Each shard writes only its own V/t rows of dE.  Deterministic:
+ * the terms of a row are added in token order, in fp32.
+ *   ids [M] int32; dY [M, h]; dE_in, dE [V, h] dtype; M < 2^28.
+ * Errors: as tp_vocab_embed_fwd; NULL dY (when M > 0) or dE.
+ */
+tp_status tp_vocab_embed_bwd(const int32_t* ids, const void* dY, const void* dE_in, void* dE,
+                             int64_t M, int64_t V, int64_t h, int t, tp_dtype dtype, void* stream);
+
+/*
+ * Vocabulary-parallel cross-entropy, the output layer tied to the input
+ * embedding E ([P3] §4.2), bf16.  With logits = X @ E^T:
+ *   1. shard i computes its logits X @ E_i^T (columns [i*V/t, (i+1)*V/t)) in
+ *      the GEMM; its epilogue rounds them to bf16 (stored in `logits` when
+ *      not NULL) and reduces every 32-column chunk to (max, sum of
+ *      exp(z - max)) over those rounded values;
+ *   2. the chunks of a shard are combined into the shard's local sum;
+ *   3. the shards' sums are combined, each rescaled to the common maximum:
+ *      lse[r] = log sum_v exp(logits[r, v]);
+ *   4-5. the shard owning targets[r] supplies its logit and
+ *      loss[r] = lse[r] - logits[r, targets[r]];
+ *   6. total = sum over shards of the losses of the rows whose target they
+ *      own, i.e. the sum of loss[r].
+ * A row whose target lies outside [0, V) is ignored: loss 0 (its lse is
+ * still written).  Results are deterministic and independent of the GEMM
+ * tile shape.
+ *   X [M, h] bf16; E [V, h] bf16; targets [M] int32; logits [M, V] bf16 or
+ *   NULL (needed by tp_vocab_ce_bwd); lse, loss [M] fp32; total: one fp32 or
+ *   NULL.  V % (8 t) == 0.
+ *   ws: tp_workspace_size(TP_OP_VOCAB_CE_FWD, M, h, V, 0, t, TP_BF16).
+ * Errors: NULL X / E / targets / lse / loss; sizes; alignment; dtype must be
+ *   TP_BF16; workspace.
+ */
+tp_status tp_vocab_ce_fwd(const void* X, const void* E, const int32_t* targets, void* logits,
+                          float* lse, float* loss, float* total, int64_t M, int64_t h, int64_t V,
+                          int t, tp_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Backward of tp_vocab_ce_fwd for the objective sum_r dloss[r] * loss[r]
+ * (dloss NULL: every dloss[r] = 1, the gradient of `total`):
+ *   dlogits[r, v] = (exp(logits[r, v] - lse[r]) - [v == targets[r]]) * dloss[r]
+ *     (zero on ignored rows), stored in bf16;
+ *   dX = dlogits @ E  (the sum over the vocabulary shards of dlogits_i @ E_i,
+ *     accumulated in one fp32 accumulator: the mirror of the column split);
+ *   dE = dlogits^T @ X  (each shard's own rows; overwritten, not accumulated:
+ *     add the input embedding's gradient afterwards with tp_vocab_embed_bwd
+ *     and dE_in = dE).
+ *   logits, lse: from tp_vocab_ce_fwd; dlogits [M, V] bf16 (may be `logits`
+ *   itself, which is then overwritten); dX [M, h], dE [V, h] bf16, each
+ *   skipped when NULL.
+ */
+tp_status tp_vocab_ce_bwd(const void* X, const void* E, const int32_t* targets,
+                          const void* logits, const float* lse, const float* dloss,
+                          void* dlogits, void* dX, void* dE, int64_t M, int64_t h, int64_t V,
+                          int t, tp_dtype dtype, void* stream);
+
+/*
  * Workspace bytes that `op` needs for these sizes (M = b*s tokens; f is
  * ignored by the attention and LayerNorm ops, heads by the MLP and LayerNorm
  * ops).  Returns 0 for invalid arguments.  The size covers the worst case
@@ -316,7 +391,8 @@ typedef enum tp_kernel_kind {
   TP_KIND_ATTN_FWD = 2,      /* attention core forward                       */
   TP_KIND_ATTN_BWD = 3,      /* attention core backward (all its kernels)    */
   TP_KIND_REDUCE = 4,        /* column sums, row terms                       */
-  TP_KIND_COUNT = 5
+  TP_KIND_VOCAB = 5,         /* embedding gather / scatter, loss reductions  */
+  TP_KIND_COUNT = 6
 } tp_kernel_kind;
 
 typedef struct tp_profile_stats {
@@ -337,7 +413,9 @@ int64_t tp_launch_count(void);
 typedef struct tp_launch_record {
   int kind;            /* tp_kernel_kind                                        */
   int tile;            /* GEMM tile: 128/192/256 columns on one SM, 512 = 256x256 */
-                       /* on an SM pair; 0 for other kernels                    */
+                       /* on an SM pair.  TP_KIND_VOCAB: 1 embedding gather,    */
+                       /* 2 embedding scatter-add, 3 loss combination, 4 the    */
+                       /* softmax gradient.  0 for other kernels                */
   int64_t m, n, k;     /* GEMM problem size (0 for other kernels)               */
   double ms;           /* event-timed duration                                  */
   double flops, bytes; /* algorithmic work                                      */

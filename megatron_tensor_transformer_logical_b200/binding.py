@@ -21,17 +21,20 @@ TP_OK, TP_ERR_NULL, TP_ERR_SHAPE, TP_ERR_ALIGN, TP_ERR_DTYPE = 0, 1, 2, 3, 4
 TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_KERNEL, TP_ERR_WORKSPACE = 5, 6, 7, 8
 TP_F32, TP_BF16 = 0, 1
 TP_OP_MLP_FWD, TP_OP_MLP_BWD, TP_OP_ATTN_FWD, TP_OP_ATTN_BWD = 0, 1, 2, 3
-TP_OP_LN_BWD, TP_OP_BLOCK_FWD, TP_OP_BLOCK_BWD = 4, 5, 6
+TP_OP_LN_BWD, TP_OP_BLOCK_FWD, TP_OP_BLOCK_BWD, TP_OP_VOCAB_CE_FWD = 4, 5, 6, 7
 
-TP_KIND_GEMM_TCGEN05, TP_KIND_GEMM_SIMT, TP_KIND_ATTN_FWD, TP_KIND_ATTN_BWD, TP_KIND_REDUCE = range(5)
+(TP_KIND_GEMM_TCGEN05, TP_KIND_GEMM_SIMT, TP_KIND_ATTN_FWD, TP_KIND_ATTN_BWD, TP_KIND_REDUCE,
+ TP_KIND_VOCAB) = range(6)
 KIND_NAMES = {TP_KIND_GEMM_TCGEN05: "gemm_tcgen05", TP_KIND_GEMM_SIMT: "gemm_simt",
-              TP_KIND_ATTN_FWD: "attn_fwd", TP_KIND_ATTN_BWD: "attn_bwd", TP_KIND_REDUCE: "reduce"}
+              TP_KIND_ATTN_FWD: "attn_fwd", TP_KIND_ATTN_BWD: "attn_bwd", TP_KIND_REDUCE: "reduce",
+              TP_KIND_VOCAB: "vocab"}
 
 EXPORTS = ("tp_linear_col", "tp_linear_row", "tp_mlp_fwd", "tp_mlp_bwd", "tp_attn_fwd",
            "tp_attn_bwd", "tp_workspace_size", "tp_last_error", "tp_device_status",
            "tp_version", "tp_profile_enable", "tp_profile_read", "tp_launch_count",
            "tp_mlp_fwd_noalloc", "tp_profile_count", "tp_profile_record", "tp_layernorm_fwd",
-           "tp_layernorm_bwd", "tp_block_fwd", "tp_block_bwd")
+           "tp_layernorm_bwd", "tp_block_fwd", "tp_block_bwd", "tp_vocab_embed_fwd",
+           "tp_vocab_embed_bwd", "tp_vocab_ce_fwd", "tp_vocab_ce_bwd")
 
 _W_FIELDS = ("ln1_g", "ln1_b", "Wqkv", "Wo", "ln2_g", "ln2_b", "A", "bA", "B", "bB")
 _S_FIELDS = ("Xn1", "mean1", "rstd1", "QKV", "O", "LSE", "X1", "Xn2", "mean2", "rstd2", "Y")
@@ -98,6 +101,11 @@ def load() -> ctypes.CDLL:
     L.tp_block_bwd.argtypes = [vp, ctypes.POINTER(BlockWeights), ctypes.POINTER(BlockSaves), vp,
                                vp, ctypes.POINTER(BlockGrads), i64, i64, i64, i64, i32, i32, f32,
                                i32, vp, sz, vp]
+    L.tp_vocab_embed_fwd.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, vp]
+    L.tp_vocab_embed_bwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, vp]
+    L.tp_vocab_ce_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, sz, vp]
+    L.tp_vocab_ce_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32,
+                                  vp]
     L.tp_workspace_size.argtypes = [i32, i64, i64, i64, i32, i32, i32]
     L.tp_workspace_size.restype = sz
     L.tp_last_error.argtypes = []
@@ -243,6 +251,43 @@ def tp_block_bwd(X, w: dict, saves: dict, dX2, dX, grads: dict, b: int, s: int, 
     _check(load().tp_block_bwd(_ptr(X), ctypes.byref(W), ctypes.byref(S), _ptr(dX2), _ptr(dX),
                                ctypes.byref(G), b, s, h, f, heads, t, eps, _dtype(X), _ptr(ws),
                                ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def _ids(t: torch.Tensor) -> int:
+    if t.dtype != torch.int32:
+        raise ValueError("token ids and targets are int32")
+    return _ptr(t)
+
+
+def tp_vocab_embed_fwd(ids, E, Y, t: int, stream=None) -> None:
+    """Y[r] = E[ids[r]] (zero for ids outside [0, V)); ids int32 [M]."""
+    V, h = E.shape
+    _check(load().tp_vocab_embed_fwd(_ids(ids), _ptr(E), _ptr(Y), ids.numel(), V, h, t,
+                                     _dtype(E), _stream(stream)))
+
+
+def tp_vocab_embed_bwd(ids, dY, dE_in, dE, t: int, stream=None) -> None:
+    """dE = scatter-add of dY rows by id (+ dE_in, which may be dE)."""
+    V, h = dE.shape
+    _check(load().tp_vocab_embed_bwd(_ids(ids), _ptr(dY), _ptr(dE_in), _ptr(dE), ids.numel(), V,
+                                     h, t, _dtype(dE), _stream(stream)))
+
+
+def tp_vocab_ce_fwd(X, E, targets, logits, lse, loss, total, t: int, ws, stream=None) -> None:
+    M, h = X.shape
+    V = E.shape[0]
+    _check(load().tp_vocab_ce_fwd(_ptr(X), _ptr(E), _ids(targets), _ptr(logits), _ptr(lse),
+                                  _ptr(loss), _ptr(total), M, h, V, t, _dtype(X), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def tp_vocab_ce_bwd(X, E, targets, logits, lse, dloss, dlogits, dX, dE, t: int,
+                    stream=None) -> None:
+    M, h = X.shape
+    V = E.shape[0]
+    _check(load().tp_vocab_ce_bwd(_ptr(X), _ptr(E), _ids(targets), _ptr(logits), _ptr(lse),
+                                  _ptr(dloss), _ptr(dlogits), _ptr(dX), _ptr(dE), M, h, V, t,
+                                  _dtype(X), _stream(stream)))
 
 
 def tp_device_status(stream=None) -> None:

@@ -603,6 +603,136 @@ tp_status block_bwd(const void* X, const tp_block_weights* w, const tp_block_sav
                               g->dln1_b, M, h, false, inner, stream);
 }
 
+// -------------------------------------------------------------- vocabulary
+
+tp_status vocab_common(int64_t M, int64_t V, int64_t h, int t, tp_dtype dtype) {
+  TP_TRY(check_dtype(dtype));
+  if (M < 0 || V <= 0 || h <= 0) return fail(TP_ERR_SHAPE, "M must be >= 0, V and h positive");
+  TP_TRY(check_t(t));
+  if (V % t != 0) return fail(TP_ERR_SHAPE, "V must be divisible by t (vocabulary split)");
+  if (V > 0x7fffffffLL) return fail(TP_ERR_SHAPE, "V must fit the int32 token ids");
+  TP_TRY(check_rows({h}));
+  return TP_OK;
+}
+
+tp_status vocab_embed_fwd(const int32_t* ids, const void* E, void* Y, int64_t M, int64_t V,
+                          int64_t h, int t, tp_dtype dtype, cudaStream_t stream) {
+  if (ids == nullptr || E == nullptr || Y == nullptr)
+    return fail(TP_ERR_NULL, "ids, E and Y are required");
+  TP_TRY(vocab_common(M, V, h, t, dtype));
+  TP_TRY(check_ptrs_aligned({E, Y}));
+  return launch_embed_fwd(ids, E, Y, M, V, h, t, dtype == TP_F32, stream);
+}
+
+tp_status vocab_embed_bwd(const int32_t* ids, const void* dY, const void* dE_in, void* dE,
+                          int64_t M, int64_t V, int64_t h, int t, tp_dtype dtype,
+                          cudaStream_t stream) {
+  if (dE == nullptr || (M > 0 && (ids == nullptr || dY == nullptr)))
+    return fail(TP_ERR_NULL, "dE is required, and ids and dY when M > 0");
+  TP_TRY(vocab_common(M, V, h, t, dtype));
+  if (M >= (1ll << 28)) return fail(TP_ERR_SHAPE, "embedding backward: M must be below 2^28");
+  TP_TRY(check_ptrs_aligned({dY, dE_in, dE}));
+  return launch_embed_bwd(ids, dY, dE_in, dE, M, V, h, dtype == TP_F32, stream);
+}
+
+int64_t ce_chunks_per_shard(int64_t V, int t) { return (V / t + 31) / 32; }
+
+size_t ce_fwd_ws(int64_t M, int64_t V, int t) {
+  const int64_t ldp = t * ce_chunks_per_shard(V, t);
+  return align_up(static_cast<size_t>(M) * ldp * 8, 256) + align_up(M * 4, 256) +
+         align_up(static_cast<size_t>(t) * 4, 256) + 1024;
+}
+
+tp_status ce_check(int64_t M, int64_t h, int64_t V, int t, tp_dtype dtype) {
+  TP_TRY(vocab_common(M, V, h, t, dtype));
+  if (dtype != TP_BF16) return fail(TP_ERR_DTYPE, "the vocabulary cross-entropy is bf16 only");
+  if ((V / t) % 8 != 0) return fail(TP_ERR_ALIGN, "V / t must be a multiple of 8");
+  return TP_OK;
+}
+
+tp_status vocab_ce_fwd(const void* X, const void* E, const int32_t* targets, void* logits,
+                       float* lse, float* loss, float* total, int64_t M, int64_t h, int64_t V,
+                       int t, tp_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (X == nullptr || E == nullptr || targets == nullptr || lse == nullptr || loss == nullptr)
+    return fail(TP_ERR_NULL, "X, E, targets, lse and loss are required");
+  TP_TRY(ce_check(M, h, V, t, dtype));
+  TP_TRY(check_ptrs_aligned({X, E, logits, ws}));
+  if (M == 0) {
+    if (total == nullptr) return TP_OK;
+    cudaError_t e = cudaMemsetAsync(total, 0, sizeof(float), stream);
+    return e == cudaSuccess ? TP_OK : cuda_fail(e, "cudaMemsetAsync(total)");
+  }
+  if (ws == nullptr || ws_bytes < ce_fwd_ws(M, V, t))
+    return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
+  Carve c(ws, ws_bytes);
+  CEOut ce;
+  ce.cps = static_cast<int>(ce_chunks_per_shard(V, t));
+  ce.ldp = static_cast<int64_t>(t) * ce.cps;
+  ce.part = static_cast<float*>(c.take(static_cast<size_t>(M) * ce.ldp * 8));
+  ce.tlogit = static_cast<float*>(c.take(M * 4));
+  ce.target = targets;
+  float* shard_tot = static_cast<float*>(c.take(static_cast<size_t>(t) * 4));
+  // Step 1: every shard's logits X @ E_i^T in one GEMM whose column tiles
+  // never straddle a shard; the epilogue reduces each 32-column chunk.
+  Gemm g;
+  g.M = M;
+  g.N = V;
+  g.K = h;
+  g.a = {X, h, true};
+  g.b = {E, h, true};  // B(k, v) = E[v, k]
+  g.epi = kEpiCE;
+  g.out = logits;
+  g.ldo = V;
+  g.n_shard = V / t;
+  g.ce = ce;
+  TP_TRY(launch_gemm_bf16(g, stream));
+  // Steps 2-6.
+  return launch_ce_finish(ce, t, M, V, lse, loss, total, shard_tot, stream);
+}
+
+tp_status vocab_ce_bwd(const void* X, const void* E, const int32_t* targets, const void* logits,
+                       const float* lse, const float* dloss, void* dlogits, void* dX, void* dE,
+                       int64_t M, int64_t h, int64_t V, int t, tp_dtype dtype,
+                       cudaStream_t stream) {
+  if (X == nullptr || E == nullptr || targets == nullptr || logits == nullptr || lse == nullptr ||
+      dlogits == nullptr)
+    return fail(TP_ERR_NULL, "X, E, targets, logits, lse and dlogits are required");
+  TP_TRY(ce_check(M, h, V, t, dtype));
+  TP_TRY(check_ptrs_aligned({X, E, logits, dlogits, dX, dE}));
+  if (M == 0) {
+    if (dE == nullptr) return TP_OK;
+    cudaError_t e = cudaMemsetAsync(dE, 0, static_cast<size_t>(V) * h * 2, stream);
+    return e == cudaSuccess ? TP_OK : cuda_fail(e, "cudaMemsetAsync(dE)");
+  }
+  TP_TRY(launch_ce_dlogits(logits, lse, targets, dloss, dlogits, M, V, stream));
+  if (dX != nullptr) {
+    // dX = sum over shards of dlogits_i @ E_i: one K loop over all V.
+    Gemm g;
+    g.M = M;
+    g.N = h;
+    g.K = V;
+    g.a = {dlogits, V, true};
+    g.b = {E, h, false};
+    g.out = dX;
+    g.ldo = h;
+    TP_TRY(launch_gemm_bf16(g, stream));
+  }
+  if (dE != nullptr) {
+    // dE = dlogits^T @ X: row v of dE needs only column v of dlogits, so each
+    // shard's rows come from its own logits.
+    Gemm g;
+    g.M = V;
+    g.N = h;
+    g.K = M;
+    g.a = {dlogits, V, false};
+    g.b = {X, h, false};
+    g.out = dE;
+    g.ldo = h;
+    TP_TRY(launch_gemm_bf16(g, stream));
+  }
+  return TP_OK;
+}
+
 }  // namespace
 }  // namespace tp
 
@@ -702,6 +832,34 @@ tp_status tp_block_bwd(const void* X, const tp_block_weights* w, const tp_block_
                             ws_bytes, static_cast<cudaStream_t>(stream));)
 }
 
+tp_status tp_vocab_embed_fwd(const int32_t* ids, const void* E, void* Y, int64_t M, int64_t V,
+                             int64_t h, int t, tp_dtype dtype, void* stream) {
+  TP_GUARD(return vocab_embed_fwd(ids, E, Y, M, V, h, t, dtype,
+                                  static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_vocab_embed_bwd(const int32_t* ids, const void* dY, const void* dE_in, void* dE,
+                             int64_t M, int64_t V, int64_t h, int t, tp_dtype dtype,
+                             void* stream) {
+  TP_GUARD(return vocab_embed_bwd(ids, dY, dE_in, dE, M, V, h, t, dtype,
+                                  static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_vocab_ce_fwd(const void* X, const void* E, const int32_t* targets, void* logits,
+                          float* lse, float* loss, float* total, int64_t M, int64_t h, int64_t V,
+                          int t, tp_dtype dtype, void* ws, size_t ws_bytes, void* stream) {
+  TP_GUARD(return vocab_ce_fwd(X, E, targets, logits, lse, loss, total, M, h, V, t, dtype, ws,
+                               ws_bytes, static_cast<cudaStream_t>(stream));)
+}
+
+tp_status tp_vocab_ce_bwd(const void* X, const void* E, const int32_t* targets,
+                          const void* logits, const float* lse, const float* dloss,
+                          void* dlogits, void* dX, void* dE, int64_t M, int64_t h, int64_t V,
+                          int t, tp_dtype dtype, void* stream) {
+  TP_GUARD(return vocab_ce_bwd(X, E, targets, logits, lse, dloss, dlogits, dX, dE, M, h, V, t,
+                               dtype, static_cast<cudaStream_t>(stream));)
+}
+
 size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, int t,
                          tp_dtype dtype) {
   try {
@@ -714,6 +872,7 @@ size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, i
       case TP_OP_LN_BWD: return ln_bwd_ws(M, h);
       case TP_OP_BLOCK_FWD: return (heads > 0 && f > 0) ? block_fwd_ws(M, h, f, heads) : 0;
       case TP_OP_BLOCK_BWD: return (heads > 0 && f > 0) ? block_bwd_ws(M, h, f, heads) : 0;
+      case TP_OP_VOCAB_CE_FWD: return (f > 0 && f % t == 0) ? ce_fwd_ws(M, f, t) : 0;
     }
   } catch (...) {
   }

@@ -70,6 +70,11 @@ struct Args {
   long long ldo2;
   const __nv_bfloat16* aux;
   long long ldaux;
+  float2* ce_part;
+  long long ce_ldp;
+  int ce_cps;
+  const int* ce_target;
+  float* ce_tlogit;
   int* status;
 };
 
@@ -231,6 +236,55 @@ __device__ __forceinline__ void epilogue_row32(float (&v)[32], int row, int col0
   if (OUT == kOutF16 && clamped) atomicCAS(a.status, 0, kStatusF16Range);
 }
 
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Cross-entropy epilogue on 32 consecutive columns (vocabulary entries) of
+// one row: "图解Transformer并行计算" §4.2 steps 1-2 for one chunk of a
+// shard.  The logits are rounded to bf16 first, so that the saved logits, the
+// chunk statistics and the target logit all see the same values; the chunk's
+// maximum and its sum of exp(z - max) over its valid columns go to the
+// partial array.  col0 is 32-aligned within its shard and col_end - col0 is
+// a multiple of 8.
+__device__ __forceinline__ void epilogue_ce32(float (&v)[32], int row, int col0, int col_end,
+                                              int tg, const Args& a) {
+  if (row >= a.M) return;
+  const int nv = min(32, col_end - col0);
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+    if (i < nv) mx = fmaxf(mx, v[i]);
+  }
+  if (a.out != nullptr) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+      if (8 * g < nv)
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + (long long)row * a.ldo +
+                                  col0 + 8 * g) = pack8(v + 8 * g);
+  }
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (i < nv) s += exp2f((v[i] - mx) * kLog2e);
+  const int sh = col0 / a.n_shard;
+  const int j = (col0 - sh * a.n_shard) >> 5;
+  a.ce_part[(long long)row * a.ce_ldp + (long long)sh * a.ce_cps + j] = make_float2(mx, s);
+  if (tg >= col0 && tg < col0 + nv) {
+    // v[tg - col0] by a select tree on the index bits (keeps v in registers).
+    const int idx = tg - col0;
+    float w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = (idx & 16) ? v[i + 16] : v[i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = (idx & 8) ? w[i + 8] : w[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = (idx & 4) ? w[i + 4] : w[i];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) w[i] = (idx & 2) ? w[i + 2] : w[i];
+    a.ce_tlogit[row] = (idx & 1) ? w[1] : w[0];
+  }
+}
+
 template <int BN, bool A_KMAJ, bool B_KMAJ, int EPI, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA,
@@ -368,6 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&tfull[acc], acc_phase, args.status, kStatusEpilogueTimeout)) break;
       tc_fence_after();
       const int row = tc.m0 + quarter * 32 + lane;
+      const int tg = (EPI == kEpiCE && row < args.M) ? args.ce_target[row] : -1;
 #pragma unroll 1
       for (int c = 0; c < BN / 2; c += 32) {
         const int cl = half * (BN / 2) + c;
@@ -376,7 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                       static_cast<uint32_t>(acc * BN + cl),
                   v);
-        epilogue_row32<EPI, OUT, false>(v, row, tc.n0 + cl, tc.n_end, args);
+        if constexpr (EPI == kEpiCE)
+          epilogue_ce32(v, row, tc.n0 + cl, tc.n_end, tg, args);
+        else
+          epilogue_row32<EPI, OUT, false>(v, row, tc.n0 + cl, tc.n_end, args);
       }
       tc_fence_before();
       __syncwarp();
@@ -577,6 +635,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&tfull[acc], acc_phase, args.status, kStatusEpilogueTimeout)) break;
       tc_fence_after();
       const int row = tc.m0 + 128 * static_cast<int>(rank) + quarter * 32 + lane;
+      const int tg = (EPI == kEpiCE && row < args.M) ? args.ce_target[row] : -1;
 #pragma unroll 1
       for (int c = 0; c < kPairTN / 2; c += 32) {
         const int cl = half * (kPairTN / 2) + c;
@@ -585,7 +644,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                       static_cast<uint32_t>(acc * kPairTN + cl),
                   v);
-        epilogue_row32<EPI, OUT, false>(v, row, tc.n0 + cl, tc.n_end, args);
+        if constexpr (EPI == kEpiCE)
+          epilogue_ce32(v, row, tc.n0 + cl, tc.n_end, tg, args);
+        else
+          epilogue_row32<EPI, OUT, false>(v, row, tc.n0 + cl, tc.n_end, args);
       }
       tc_fence_before();
       __syncwarp();
@@ -730,6 +792,11 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   a.ldo2 = g.ldo2;
   a.aux = static_cast<const __nv_bfloat16*>(g.aux);
   a.ldaux = g.ldaux;
+  a.ce_part = reinterpret_cast<float2*>(g.ce.part);
+  a.ce_ldp = g.ce.ldp;
+  a.ce_cps = g.ce.cps;
+  a.ce_target = g.ce.target;
+  a.ce_tlogit = g.ce.tlogit;
   a.status = device_status_ptr();
   if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
 
@@ -750,7 +817,8 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
                        (OUT == kOutF32 ? 4.0 : 2.0) * double(g.M) * g.N +
                        (g.out2 ? 2.0 * double(g.M) * g.N : 0.0) +
-                       (g.aux ? 2.0 * double(g.M) * g.N : 0.0);
+                       (g.aux ? 2.0 * double(g.M) * g.N : 0.0) +
+                       (EPI == kEpiCE ? 8.0 * double(g.M) * g.N / 32.0 : 0.0);
   {
     LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, 1, BN, g.M, g.N, g.K);
     kern<<<grid, kThreads, C::kSmemBytes, stream>>>(ta, tb, a);
@@ -777,6 +845,8 @@ tp_status dispatch(const Gemm& g, cudaStream_t s) {
     if (ak && !bk && plain_out) return launch_impl<BN, true, false, kEpiResidual, kOutBF16>(g, s);
   } else if (g.epi == kEpiDGelu) {
     if (ak && bk && plain_out) return launch_impl<BN, true, true, kEpiDGelu, kOutBF16>(g, s);
+  } else if (g.epi == kEpiCE) {
+    if (ak && bk && plain_out) return launch_impl<BN, true, true, kEpiCE, kOutBF16>(g, s);
   } else {
     if (ak && !bk) return by_out<BN, true, false, kEpiStore>(g, s);
     if (ak && bk) return by_out<BN, true, true, kEpiStore>(g, s);
@@ -819,6 +889,11 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   a.ldo2 = g.ldo2;
   a.aux = static_cast<const __nv_bfloat16*>(g.aux);
   a.ldaux = g.ldaux;
+  a.ce_part = reinterpret_cast<float2*>(g.ce.part);
+  a.ce_ldp = g.ce.ldp;
+  a.ce_cps = g.ce.cps;
+  a.ce_target = g.ce.target;
+  a.ce_tlogit = g.ce.tlogit;
   a.status = device_status_ptr();
   if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
 
@@ -851,7 +926,8 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
                        (OUT == kOutF32 ? 4.0 : 2.0) * double(g.M) * g.N +
                        (g.out2 ? 2.0 * double(g.M) * g.N : 0.0) +
-                       (g.aux ? 2.0 * double(g.M) * g.N : 0.0);
+                       (g.aux ? 2.0 * double(g.M) * g.N : 0.0) +
+                       (EPI == kEpiCE ? 8.0 * double(g.M) * g.N / 32.0 : 0.0);
   {
     LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, 1, 512, g.M, g.N, g.K);
     kern<<<2 * clusters, kThreads, kPairSmemBytes, stream>>>(ta, tb, a);
@@ -877,6 +953,8 @@ tp_status dispatch_pair(const Gemm& g, cudaStream_t s) {
     if (ak && !bk && plain_out) return launch_pair<true, false, kEpiResidual, kOutBF16>(g, s);
   } else if (g.epi == kEpiDGelu) {
     if (ak && bk && plain_out) return launch_pair<true, true, kEpiDGelu, kOutBF16>(g, s);
+  } else if (g.epi == kEpiCE) {
+    if (ak && bk && plain_out) return launch_pair<true, true, kEpiCE, kOutBF16>(g, s);
   } else {
     if (ak && !bk) return pair_by_out<true, false, kEpiStore>(g, s);
     if (ak && bk) return pair_by_out<true, true, kEpiStore>(g, s);
@@ -907,6 +985,11 @@ tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream) {
   // stores whole groups of 8 columns, so other shard widths tile plainly
   // (every column is still computed by the same K loop).
   if (gg.n_shard > 0 && (gg.n_shard % 8 != 0 || gg.N % gg.n_shard != 0)) gg.n_shard = 0;
+  if (gg.epi == kEpiCE &&
+      (gg.n_shard <= 0 || gg.ce.part == nullptr || gg.ce.target == nullptr ||
+       gg.ce.tlogit == nullptr || gg.ce.cps != (gg.n_shard + 31) / 32 ||
+       gg.ce.ldp != gg.ce.cps * (gg.N / gg.n_shard)))
+    return fail(TP_ERR_SHAPE, "gemm: inconsistent cross-entropy partial layout");
   switch (choose_tile(gg)) {
     case 512: return dispatch_pair(gg, stream);
     case 128: return dispatch<128>(gg, stream);

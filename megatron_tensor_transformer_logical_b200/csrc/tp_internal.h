@@ -43,6 +43,20 @@ enum Epi : int {
   kEpiBiasGelu = 1,  // v = acc + bias[col]; out = GeLU(v); out2 = v (if out2)
   kEpiDGelu = 2,     // y = aux[row,col]; out = acc * GeLU'(y); out2 = GeLU(y) (if out2)
   kEpiResidual = 3,  // out = acc (+ bias[col]) + aux[row,col]: a residual addition
+  kEpiCE = 4,        // z = bf16(acc); out = z (if out); per 32-column chunk of a
+                     // shard: (max z, sum exp(z - max)) to ce_part; the target's z
+};
+
+// Cross-entropy outputs of a kEpiCE GEMM (columns are vocabulary entries).
+// Chunk j of shard i (columns i*n_shard + [32 j, 32 j + 32)) of row r is
+// part[r * ldp + i * cps + j] = (max, sum of exp(z - max)) over its columns;
+// tlogit[r] = z[r, target[r]] when the target is a column of the GEMM.
+struct CEOut {
+  float* part = nullptr;  // float pairs
+  int64_t ldp = 0;        // pairs per row = shards * cps
+  int cps = 0;            // chunks per shard = ceil(n_shard / 32)
+  const int* target = nullptr;
+  float* tlogit = nullptr;
 };
 
 // One operand of D[M,N] = sum_k A(m,k) B(k,n) stored as a row-major matrix.
@@ -81,6 +95,7 @@ struct Gemm {
   int64_t ldaux = 0;
   int64_t n_shard = 0;         // columns per shard: column tiles never straddle shards
   KOrder korder;
+  CEOut ce;                    // kEpiCE only (requires n_shard % 8 == 0)
 };
 
 // bf16 x bf16 -> fp32 accumulate on tcgen05; out bf16, fp16 or fp32.
@@ -104,6 +119,27 @@ tp_status launch_layernorm_bwd(const void* X, const void* gamma, const float* me
                                const float* rstd, const void* dY, const void* dR, void* dX,
                                void* dgamma, void* dbeta, int64_t M, int64_t h, bool f32,
                                void* scratch, cudaStream_t stream);
+
+// Vocabulary-parallel embedding and loss helpers (HBM-bound kernels).  Their
+// trace records carry one of these codes in the `tile` field.
+enum VocabKernel : int {
+  kVocabEmbedFwd = 1,     // embedding gather
+  kVocabEmbedBwd = 2,     // embedding scatter-add
+  kVocabLossCombine = 3,  // chunk partials -> lse, loss, total
+  kVocabSoftmaxGrad = 4,  // dlogits
+};
+tp_status launch_embed_fwd(const int* ids, const void* E, void* Y, int64_t M, int64_t V,
+                           int64_t h, int t, bool f32, cudaStream_t stream);
+tp_status launch_embed_bwd(const int* ids, const void* dY, const void* dE_in, void* dE,
+                           int64_t M, int64_t V, int64_t h, bool f32, cudaStream_t stream);
+// From the chunk partials of a kEpiCE GEMM: lse, loss and (if not NULL) the
+// total.  `shard_tot` holds t floats of scratch.
+tp_status launch_ce_finish(const CEOut& ce, int t, int64_t M, int64_t V, float* lse, float* loss,
+                           float* total, float* shard_tot, cudaStream_t stream);
+// dlogits = (exp(logits - lse) - onehot(target)) * dloss, bf16, in place allowed.
+tp_status launch_ce_dlogits(const void* logits, const float* lse, const int* target,
+                            const float* dloss, void* dlogits, int64_t M, int64_t V,
+                            cudaStream_t stream);
 
 // Attention core (per head causal softmax attention), bf16 with d = 128.
 struct AttnShape {

@@ -13,7 +13,12 @@ the MLP ``Z = GeLU(X@A)@B`` with ``A`` split by columns and ``B`` by rows
 standalone linear layer in both split modes (same page, §1.1 and §1.2),
 head-wise attention with ``W_o`` split by rows (same page, §3.2), and a
 layer shaped like the 175B case study (hidden 12288, 96 heads) of the
-PyTorch tensor-parallel tutorial (its §5).
+PyTorch tensor-parallel tutorial (its §5).  A sixth workload is the
+vocabulary-parallel embedding and loss of the first page's §4.1-§4.2 at the
+same hidden size; its token ids follow a Zipf law (frequency of the k-th
+most common token proportional to 1/k), the usual shape of natural-text
+token counts, with the ranks scattered over the vocabulary by a seeded
+permutation so that common tokens fall in every shard.
 """
 from __future__ import annotations
 
@@ -39,6 +44,7 @@ class Workload:
     w_std: float = 0.02   # weights ~ N(0, w_std^2)
     bias_std: Optional[float] = None  # None: no bias; 0.0: zero bias buffer
     n_out: int = 0        # standalone linear: output width
+    vocab: int = 0        # vocabulary size V (vocabulary-parallel workload)
 
     @property
     def M(self) -> int:
@@ -60,6 +66,8 @@ WORKLOADS: Dict[int, Workload] = {
                 w_std=0.02),
     5: Workload(5, "175B-shaped layer", b=1, s=2048, h=12288, f=49152,
                 heads=96, t=8, w_std=0.006),
+    6: Workload(6, "vocabulary-parallel embedding + cross-entropy", b=1, s=2048,
+                h=12288, vocab=51200, t=8, w_std=0.02),
 }
 
 
@@ -111,6 +119,33 @@ def make_attn_inputs(wl: Workload, seed: Optional[int] = None) -> Dict[str, torc
         "Wqkv": _draw(gen, (wl.h, 3 * wl.h), wl.w_std, wl.dtype),
         "Wo": _draw(gen, (wl.h, wl.h), wl.w_std, wl.dtype),
         "dZ": _draw(gen, (wl.M, wl.h), 1.0, wl.dtype),
+    }
+
+
+def zipf_ids(n: int, V: int, seed: int, exponent: float = 1.0) -> torch.Tensor:
+    """n int32 token ids in [0, V): rank k (0-based) drawn with probability
+    proportional to 1/(k+1)^exponent, ranks mapped to ids by a seeded
+    permutation of the vocabulary."""
+    gen = torch.Generator().manual_seed(seed)
+    weights = torch.arange(1, V + 1, dtype=torch.float64).pow(-exponent)
+    ranks = torch.multinomial(weights, n, replacement=True, generator=gen)
+    perm = torch.randperm(V, generator=gen)
+    return perm[ranks].to(torch.int32)
+
+
+def make_vocab_inputs(wl: Workload, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """ids [M] int32 (Zipf), targets [M] int32 (the next token: ids shifted by
+    one, the last one drawn), E [V,h] ~ N(0, w_std^2), X [M,h] ~ N(0,1) (the
+    final hidden states fed to the tied output layer), dY [M,h] ~ N(0,1)."""
+    s0 = (wl.seed if seed is None else seed) + 200
+    stream = zipf_ids(wl.M + 1, wl.vocab, s0)
+    gen = torch.Generator().manual_seed(s0 + 1)
+    return {
+        "ids": stream[:-1].contiguous(),
+        "targets": stream[1:].contiguous(),
+        "E": _draw(gen, (wl.vocab, wl.h), wl.w_std, wl.dtype),
+        "X": _draw(gen, (wl.M, wl.h), 1.0, wl.dtype),
+        "dY": _draw(gen, (wl.M, wl.h), 1.0, wl.dtype),
     }
 
 

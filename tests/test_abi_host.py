@@ -154,3 +154,37 @@ def test_layernorm_and_block_validation(lib):
     assert lib.tp_block_fwd(P[0], C.byref(W), P[1], C.byref(S), 1, 64, 512, 2048, 4, 2, 1e-5, L.TP_F32, P[9], big, None) == L.TP_ERR_UNSUPPORTED
     assert lib.tp_workspace_size(L.TP_OP_BLOCK_BWD, 2048, 12288, 49152, 96, 8, L.TP_BF16) > 3 * 2048 * 12288 * 2
     assert lib.tp_workspace_size(L.TP_OP_LN_BWD, 2048, 12288, 0, 0, 1, L.TP_BF16) >= 2 * 296 * 12288 * 4
+
+
+def test_vocab_validation(lib):
+    """Vocabulary-parallel embedding and cross-entropy ("图解Transformer并行计算"
+    §4.1, §4.2): E's rows split over t shards, so V % t must be 0."""
+    big = 1 << 40
+    bf, f32 = L.TP_BF16, L.TP_F32
+    ef, eb = lib.tp_vocab_embed_fwd, lib.tp_vocab_embed_bwd
+    assert ef(None, P[1], P[2], 16, 1024, 64, 4, bf, None) == L.TP_ERR_NULL
+    assert ef(P[0], P[1], P[2], 16, 1026, 64, 4, bf, None) == L.TP_ERR_SHAPE   # V % t
+    assert ef(P[0], P[1], P[2], -1, 1024, 64, 4, bf, None) == L.TP_ERR_SHAPE
+    assert ef(P[0], P[1], P[2], 16, 1024, 60, 4, bf, None) == L.TP_ERR_ALIGN   # h % 8
+    assert ef(P[0], P[1] + 8, P[2], 16, 1024, 64, 4, bf, None) == L.TP_ERR_ALIGN
+    assert ef(P[0], P[1], P[2], 16, 1024, 64, 0, bf, None) == L.TP_ERR_SHAPE
+    assert ef(P[0], P[1], P[2], 16, 1024, 64, 4, 7, None) == L.TP_ERR_DTYPE
+    assert ef(P[0], P[1], P[2], 0, 1024, 64, 4, bf, None) == L.TP_OK          # nothing to do
+    assert eb(P[0], None, None, P[3], 16, 1024, 64, 4, bf, None) == L.TP_ERR_NULL
+    assert eb(P[0], P[1], None, None, 16, 1024, 64, 4, bf, None) == L.TP_ERR_NULL
+    assert eb(P[0], P[1], None, P[3], 1 << 28, 1024, 64, 4, bf, None) == L.TP_ERR_SHAPE
+    cf, cb = lib.tp_vocab_ce_fwd, lib.tp_vocab_ce_bwd
+    ok = (P[0], P[1], P[2], P[3], P[4], P[5], None)
+    assert cf(None, *ok[1:], 64, 256, 1024, 4, bf, P[9], big, None) == L.TP_ERR_NULL
+    assert cf(P[0], P[1], P[2], P[3], None, P[5], None, 64, 256, 1024, 4, bf, P[9], big, None) == L.TP_ERR_NULL
+    assert cf(*ok, 64, 256, 1024, 4, f32, P[9], big, None) == L.TP_ERR_DTYPE  # bf16 only
+    assert cf(*ok, 64, 256, 1004, 8, bf, P[9], big, None) == L.TP_ERR_SHAPE   # V % t
+    assert cf(*ok, 64, 256, 1028, 4, bf, P[9], big, None) == L.TP_ERR_ALIGN   # (V/t) % 8
+    assert cf(*ok, 64, 256, 1024, 4, bf, None, 0, None) == L.TP_ERR_WORKSPACE
+    need = lib.tp_workspace_size(L.TP_OP_VOCAB_CE_FWD, 64, 256, 1024, 0, 4, bf)
+    assert need >= 64 * 1024 // 32 * 8 + 64 * 4
+    assert cf(*ok, 64, 256, 1024, 4, bf, P[9], need - 1, None) == L.TP_ERR_WORKSPACE
+    assert lib.tp_workspace_size(L.TP_OP_VOCAB_CE_FWD, 64, 256, 1026, 0, 4, bf) == 0
+    assert cb(P[0], P[1], P[2], None, P[4], None, P[6], P[7], P[8], 64, 256, 1024, 4, bf, None) == L.TP_ERR_NULL
+    assert cb(P[0], P[1], P[2], P[3], P[4], None, None, P[7], P[8], 64, 256, 1024, 4, bf, None) == L.TP_ERR_NULL
+    assert cb(P[0], P[1], P[2], P[3], P[4], None, P[6], P[7], P[8], 64, 256, 1024, 4, f32, None) == L.TP_ERR_DTYPE
