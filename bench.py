@@ -247,6 +247,7 @@ class VocabStep:
         self.dX = torch.empty(M, h, dtype=bf, device=dev)
         self.dE = torch.empty(V, h, dtype=bf, device=dev)
         self.ws = L.workspace(L.TP_OP_VOCAB_CE_FWD, M, h, V, 0, wl.t, L.TP_BF16, device=dev)
+        self.ws_e = L.workspace(L.TP_OP_VOCAB_EMBED_BWD, M, h, V, 0, wl.t, L.TP_BF16, device=dev)
 
     def step(self):
         L, t = self.L, self.wl.t
@@ -255,7 +256,7 @@ class VocabStep:
                           self.total, t, self.ws)
         L.tp_vocab_ce_bwd(self.X, self.E, self.targets, self.logits, self.lse, None, self.logits,
                           self.dX, self.dE, t)
-        L.tp_vocab_embed_bwd(self.ids, self.dY, self.dE, self.dE, t)
+        L.tp_vocab_embed_bwd(self.ids, self.dY, self.dE, self.dE, t, self.ws_e)
 
     def flops(self):
         wl = self.wl

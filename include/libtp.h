@@ -71,7 +71,8 @@ typedef enum tp_op {
   TP_OP_LN_BWD = 4,
   TP_OP_BLOCK_FWD = 5,
   TP_OP_BLOCK_BWD = 6,
-  TP_OP_VOCAB_CE_FWD = 7  /* f is the vocabulary size V */
+  TP_OP_VOCAB_CE_FWD = 7,   /* f is the vocabulary size V */
+  TP_OP_VOCAB_EMBED_BWD = 8 /* depends on M only */
 } tp_op;
 
 /*
@@ -312,13 +313,17 @@ tp_status tp_vocab_embed_fwd(const int32_t* ids, const void* E, void* Y, int64_t
  * Backward of tp_vocab_embed_fwd: dE[v] = sum of dY[r] over the rows r with
  * ids[r] == v (zero for a row of E no token used), plus dE_in[v] when dE_in
  * is not NULL (the tied output layer's gradient, accumulated; dE_in may be
- * dE itself).  Each shard writes only its own V/t rows of dE.  Deterministic:
- * the terms of a row are added in token order, in fp32.
+ * dE itself, and then only the rows that tokens use are touched).  Each
+ * shard writes only its own V/t rows of dE.  Deterministic: the terms of a
+ * row are added in token order, in fp32.
  *   ids [M] int32; dY [M, h]; dE_in, dE [V, h] dtype; M < 2^28.
- * Errors: as tp_vocab_embed_fwd; NULL dY (when M > 0) or dE.
+ *   ws: tp_workspace_size(TP_OP_VOCAB_EMBED_BWD, M, h, V, 0, t, dtype)
+ *   (may be NULL when M == 0).
+ * Errors: as tp_vocab_embed_fwd; NULL dY (when M > 0) or dE; workspace.
  */
 tp_status tp_vocab_embed_bwd(const int32_t* ids, const void* dY, const void* dE_in, void* dE,
-                             int64_t M, int64_t V, int64_t h, int t, tp_dtype dtype, void* stream);
+                             int64_t M, int64_t V, int64_t h, int t, tp_dtype dtype, void* ws,
+                             size_t ws_bytes, void* stream);
 
 /*
  * Vocabulary-parallel cross-entropy, the output layer tied to the input

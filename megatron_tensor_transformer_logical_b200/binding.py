@@ -22,6 +22,7 @@ TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_KERNEL, TP_ERR_WORKSPACE = 5, 6, 7, 8
 TP_F32, TP_BF16 = 0, 1
 TP_OP_MLP_FWD, TP_OP_MLP_BWD, TP_OP_ATTN_FWD, TP_OP_ATTN_BWD = 0, 1, 2, 3
 TP_OP_LN_BWD, TP_OP_BLOCK_FWD, TP_OP_BLOCK_BWD, TP_OP_VOCAB_CE_FWD = 4, 5, 6, 7
+TP_OP_VOCAB_EMBED_BWD = 8
 
 (TP_KIND_GEMM_TCGEN05, TP_KIND_GEMM_SIMT, TP_KIND_ATTN_FWD, TP_KIND_ATTN_BWD, TP_KIND_REDUCE,
  TP_KIND_VOCAB) = range(6)
@@ -102,7 +103,7 @@ def load() -> ctypes.CDLL:
                                vp, ctypes.POINTER(BlockGrads), i64, i64, i64, i64, i32, i32, f32,
                                i32, vp, sz, vp]
     L.tp_vocab_embed_fwd.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, vp]
-    L.tp_vocab_embed_bwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, vp]
+    L.tp_vocab_embed_bwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, sz, vp]
     L.tp_vocab_ce_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, sz, vp]
     L.tp_vocab_ce_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32,
                                   vp]
@@ -266,11 +267,13 @@ def tp_vocab_embed_fwd(ids, E, Y, t: int, stream=None) -> None:
                                      _dtype(E), _stream(stream)))
 
 
-def tp_vocab_embed_bwd(ids, dY, dE_in, dE, t: int, stream=None) -> None:
+def tp_vocab_embed_bwd(ids, dY, dE_in, dE, t: int, ws, stream=None) -> None:
     """dE = scatter-add of dY rows by id (+ dE_in, which may be dE)."""
     V, h = dE.shape
     _check(load().tp_vocab_embed_bwd(_ids(ids), _ptr(dY), _ptr(dE_in), _ptr(dE), ids.numel(), V,
-                                     h, t, _dtype(dE), _stream(stream)))
+                                     h, t, _dtype(dE), _ptr(ws),
+                                     0 if ws is None else ws.numel() * ws.element_size(),
+                                     _stream(stream)))
 
 
 def tp_vocab_ce_fwd(X, E, targets, logits, lse, loss, total, t: int, ws, stream=None) -> None:

@@ -624,15 +624,19 @@ tp_status vocab_embed_fwd(const int32_t* ids, const void* E, void* Y, int64_t M,
   return launch_embed_fwd(ids, E, Y, M, V, h, t, dtype == TP_F32, stream);
 }
 
+size_t embed_bwd_ws(int64_t M) { return align_up(embed_bwd_scratch_bytes(M), 256) + 256; }
+
 tp_status vocab_embed_bwd(const int32_t* ids, const void* dY, const void* dE_in, void* dE,
-                          int64_t M, int64_t V, int64_t h, int t, tp_dtype dtype,
-                          cudaStream_t stream) {
+                          int64_t M, int64_t V, int64_t h, int t, tp_dtype dtype, void* ws,
+                          size_t ws_bytes, cudaStream_t stream) {
   if (dE == nullptr || (M > 0 && (ids == nullptr || dY == nullptr)))
     return fail(TP_ERR_NULL, "dE is required, and ids and dY when M > 0");
   TP_TRY(vocab_common(M, V, h, t, dtype));
   if (M >= (1ll << 28)) return fail(TP_ERR_SHAPE, "embedding backward: M must be below 2^28");
-  TP_TRY(check_ptrs_aligned({dY, dE_in, dE}));
-  return launch_embed_bwd(ids, dY, dE_in, dE, M, V, h, dtype == TP_F32, stream);
+  TP_TRY(check_ptrs_aligned({dY, dE_in, dE, ws}));
+  if (M > 0 && (ws == nullptr || ws_bytes < embed_bwd_ws(M)))
+    return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
+  return launch_embed_bwd(ids, dY, dE_in, dE, M, V, h, dtype == TP_F32, ws, stream);
 }
 
 int64_t ce_chunks_per_shard(int64_t V, int t) { return (V / t + 31) / 32; }
@@ -839,9 +843,9 @@ tp_status tp_vocab_embed_fwd(const int32_t* ids, const void* E, void* Y, int64_t
 }
 
 tp_status tp_vocab_embed_bwd(const int32_t* ids, const void* dY, const void* dE_in, void* dE,
-                             int64_t M, int64_t V, int64_t h, int t, tp_dtype dtype,
-                             void* stream) {
-  TP_GUARD(return vocab_embed_bwd(ids, dY, dE_in, dE, M, V, h, t, dtype,
+                             int64_t M, int64_t V, int64_t h, int t, tp_dtype dtype, void* ws,
+                             size_t ws_bytes, void* stream) {
+  TP_GUARD(return vocab_embed_bwd(ids, dY, dE_in, dE, M, V, h, t, dtype, ws, ws_bytes,
                                   static_cast<cudaStream_t>(stream));)
 }
 
@@ -873,6 +877,7 @@ size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, i
       case TP_OP_BLOCK_FWD: return (heads > 0 && f > 0) ? block_fwd_ws(M, h, f, heads) : 0;
       case TP_OP_BLOCK_BWD: return (heads > 0 && f > 0) ? block_bwd_ws(M, h, f, heads) : 0;
       case TP_OP_VOCAB_CE_FWD: return (f > 0 && f % t == 0) ? ce_fwd_ws(M, f, t) : 0;
+      case TP_OP_VOCAB_EMBED_BWD: return embed_bwd_ws(M);
     }
   } catch (...) {
   }

@@ -332,6 +332,13 @@ constexpr int kTile64 = 64 * 128 * 2;   // [64 rows x 128] fp16: 16 KB (two 8 KB
 constexpr int kHalf64 = kTile64 / 2;
 constexpr int kTile128x64 = 128 * 64 * 2;  // [128 rows x 64] fp16: 16 KB (one SW128 atom wide)
 
+// The backward kernels run 12 warps: warp 0 TMA, warp 1 MMA, warps 4-11 the
+// element-wise work in two groups of four; group g takes columns
+// [32 g, 32 g + 32) of every 64-column block (and half of the output
+// columns), so each SM sub-partition runs two element-wise warps.
+constexpr int kThreadsB = 384;
+constexpr int kEwWarpsB = 8;
+
 struct BwdArgs {
   int s, h, heads, causal;
   float scale_log2, scale;
@@ -345,7 +352,7 @@ struct BwdArgs {
 // Shared memory: Q 32K | dO 32K | KV[2] (K 16K + V 16K) | dS[2] 16K each.
 constexpr int kSmemDQ = 1024 + 2 * kTile + 2 * (2 * kTile64) + 2 * kTile128x64 + 256;
 
-__global__ void __launch_bounds__(kThreadsA, 1)
+__global__ void __launch_bounds__(kThreadsB, 1)
     attn_bwd_dq_tcgen05(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                         const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -380,7 +387,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&ds_full[i], 4);
+      mbar_init(&ds_full[i], kEwWarpsB);
       mbar_init(&ds_free[i], 1);
     }
     mbar_init(dq_done, 1);
@@ -471,6 +478,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     }
   } else if (warp >= 4) {
     const int quarter = warp & 3;
+    const int grp = (warp - 4) >> 2;  // this warp's column half
+    const int c = grp * 32;
     const int r = quarter * 32 + lane;
     const int qrow = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -489,28 +498,25 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                                      a.status, kStatusAttnTimeout)))
         break;
       tc_fence_after();
-      const int vis = limit - j * kB64;
+      const int vis = limit - j * kB64 - c;  // columns c + i with i < vis are visible
       uint8_t* row = sdS + st * kTile128x64 + (r >> 3) * 1024 + (r & 7) * 128;
+      float sv[32], pv[32];
+      tmem_ld32(tS[st] + lane_off + c, sv);
+      tmem_ld32(tP[st] + lane_off + c, pv);
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < kB64; c += 32) {
-        float sv[32], pv[32];
-        tmem_ld32(tS[st] + lane_off + c, sv);
-        tmem_ld32(tP[st] + lane_off + c, pv);
-        uint32_t pk[16];
+      for (int i = 0; i < 32; i += 2) {
+        float p0 = exp2f(fmaf(sv[i], a.scale_log2, -lse2));
+        float p1 = exp2f(fmaf(sv[i + 1], a.scale_log2, -lse2));
+        p0 = (i < vis) ? p0 : 0.0f;
+        p1 = (i + 1 < vis) ? p1 : 0.0f;
+        pk[i >> 1] = pack_half2(p0 * (pv[i] - dd), p1 * (pv[i + 1] - dd));
+      }
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p0 = exp2f(fmaf(sv[i], a.scale_log2, -lse2));
-          float p1 = exp2f(fmaf(sv[i + 1], a.scale_log2, -lse2));
-          p0 = (c + i < vis) ? p0 : 0.0f;
-          p1 = (c + i + 1 < vis) ? p1 : 0.0f;
-          pk[i >> 1] = pack_half2(p0 * (pv[i] - dd), p1 * (pv[i + 1] - dd));
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = (c >> 3) + q;
-          *reinterpret_cast<uint4*>(row + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
+      for (int q = 0; q < 4; ++q) {
+        const int chunk = (c >> 3) + q;
+        *reinterpret_cast<uint4*>(row + ((chunk ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -521,9 +527,9 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       tc_fence_after();
       __nv_bfloat16* out = a.dqkv + static_cast<long long>(row0 + qrow) * (3LL * a.h) + head * kD;
 #pragma unroll
-      for (int c = 0; c < kD; c += 32) {
+      for (int cc = grp * (kD / 2); cc < (grp + 1) * (kD / 2); cc += 32) {
         float v[32];
-        tmem_ld32(tQ + lane_off + c, v);
+        tmem_ld32(tQ + lane_off + cc, v);
         if (qrow < a.s) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -535,7 +541,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                                                        v[8 * q + 2 * e + 1] * a.scale);
               w[e] = *reinterpret_cast<uint32_t*>(&t);
             }
-            *reinterpret_cast<uint4*>(out + c + 8 * q) = u;
+            *reinterpret_cast<uint4*>(out + cc + 8 * q) = u;
           }
         }
       }
@@ -553,7 +559,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
 // Shared memory: K 32K | V 32K | QdO[2] (Q 16K + dO 16K) | PdS[2] (P^T 16K + dS^T 16K).
 constexpr int kSmemKV = 1024 + 2 * kTile + 2 * (2 * kTile64) + 2 * (2 * kTile128x64) + 256;
 
-__global__ void __launch_bounds__(kThreadsA, 1)
+__global__ void __launch_bounds__(kThreadsB, 1)
     attn_bwd_dkdv_tcgen05(const __grid_constant__ CUtensorMap tmKV128,
                           const __grid_constant__ CUtensorMap tmQ64,
                           const __grid_constant__ CUtensorMap tmdO64, const BwdArgs a) {
@@ -573,6 +579,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   uint64_t* p_free = bars + 9;    // [2]
   uint64_t* acc_done = bars + 11;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  __shared__ __align__(16) float s_stat[kEwWarpsB * 64];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb = static_cast<int>(blockIdx.x);  // early keys see the most queries: first
@@ -589,7 +596,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       mbar_init(&qd_full[i], 1);
       mbar_init(&qd_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], kEwWarpsB);
       mbar_init(&p_free[i], 1);
     }
     mbar_init(acc_done, 1);
@@ -685,13 +692,28 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     }
   } else if (warp >= 4) {
     const int quarter = warp & 3;
+    const int grp = (warp - 4) >> 2;  // this warp's column half
+    const int c = grp * 32;
     const int r = quarter * 32 + lane;
     const int key = k0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.s;
+    // The warp's 32 queries' LSE * log2(e) and D, staged once per block in a
+    // per-warp shared-memory slot (read back as broadcasts).
+    float* wstat = s_stat + (warp - 4) * 64;
     bool ok = true;
     for (int it = 0; it < n_qb && ok; ++it) {
       const int st = it & 1;
+      const int q0 = (i0 + it) * kB64;
+      {
+        const int qs = min(q0 + c + lane, a.s - 1);
+        const float l2 = a.lse[stat + qs] * kLog2eA;
+        const float dq = a.dsum[stat + qs];
+        __syncwarp();  // the previous block's reads of the slot are done
+        wstat[lane] = l2;
+        wstat[32 + lane] = dq;
+        __syncwarp();
+      }
       if (!(ok = mbar_wait(&s_full[st], (static_cast<uint32_t>(it) >> 1) & 1u, a.status,
                            kStatusAttnTimeout)))
         break;
@@ -699,41 +721,40 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                                       a.status, kStatusAttnTimeout)))
         break;
       tc_fence_after();
-      const int q0 = (i0 + it) * kB64;
-      // query q = q0 + c is visible to this key when key <= q (causal) and q < s
-      const int first = a.causal ? max(key - q0, 0) : 0;  // first visible column
-      const int last = min(a.s - q0, kB64);                // one past the last
-      const bool key_ok = key < a.s;
+      // query q = q0 + c + i is visible to this key when key <= q (causal)
+      // and q < s: lo <= i < hi
+      const int lo = (a.causal ? max(key - q0, 0) : 0) - c;
+      const int hi = (key < a.s ? min(a.s - q0, kB64) : 0) - c;
       uint8_t* prow = sPdS + st * (2 * kTile128x64) + (r >> 3) * 1024 + (r & 7) * 128;
       uint8_t* drow = prow + kTile128x64;
+      float sv[32], pv[32];
+      tmem_ld32(tS[st] + lane_off + c, sv);
+      tmem_ld32(tP[st] + lane_off + c, pv);
+      uint32_t pk[16], dk[16];
 #pragma unroll
-      for (int c = 0; c < kB64; c += 32) {
-        float sv[32], pv[32];
-        tmem_ld32(tS[st] + lane_off + c, sv);
-        tmem_ld32(tP[st] + lane_off + c, pv);
-        uint32_t pk[16], dk[16];
+      for (int i = 0; i < 32; i += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(wstat + i);
+        const float4 d4 = *reinterpret_cast<const float4*>(wstat + 32 + i);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        float p[4];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int qa = min(q0 + c + i, a.s - 1), qb2 = min(q0 + c + i + 1, a.s - 1);
-          const float l0 = a.lse[stat + qa] * kLog2eA, l1 = a.lse[stat + qb2] * kLog2eA;
-          const float d0 = a.dsum[stat + qa], d1 = a.dsum[stat + qb2];
-          float p0 = exp2f(fmaf(sv[i], a.scale_log2, -l0));
-          float p1 = exp2f(fmaf(sv[i + 1], a.scale_log2, -l1));
-          const bool v0 = key_ok && (c + i >= first) && (c + i < last);
-          const bool v1 = key_ok && (c + i + 1 >= first) && (c + i + 1 < last);
-          p0 = v0 ? p0 : 0.0f;
-          p1 = v1 ? p1 : 0.0f;
-          pk[i >> 1] = pack_half2(p0, p1);
-          dk[i >> 1] = pack_half2(p0 * (pv[i] - d0), p1 * (pv[i + 1] - d1));
+        for (int e = 0; e < 4; ++e) {
+          p[e] = exp2f(fmaf(sv[i + e], a.scale_log2, -lv[e]));
+          p[e] = (i + e >= lo && i + e < hi) ? p[e] : 0.0f;
         }
+        pk[i >> 1] = pack_half2(p[0], p[1]);
+        pk[(i >> 1) + 1] = pack_half2(p[2], p[3]);
+        dk[i >> 1] = pack_half2(p[0] * (pv[i] - dv[0]), p[1] * (pv[i + 1] - dv[1]));
+        dk[(i >> 1) + 1] = pack_half2(p[2] * (pv[i + 2] - dv[2]), p[3] * (pv[i + 3] - dv[3]));
+      }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int off = ((((c >> 3) + q) ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(prow + off) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-          *reinterpret_cast<uint4*>(drow + off) =
-              make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
-        }
+      for (int q = 0; q < 4; ++q) {
+        const int off = ((((c >> 3) + q) ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(prow + off) =
+            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        *reinterpret_cast<uint4*>(drow + off) =
+            make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -744,10 +765,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       tc_fence_after();
       __nv_bfloat16* out = a.dqkv + static_cast<long long>(row0 + key) * (3LL * a.h);
 #pragma unroll
-      for (int c = 0; c < kD; c += 32) {
+      for (int cc = grp * (kD / 2); cc < (grp + 1) * (kD / 2); cc += 32) {
         float vk[32], vv[32];
-        tmem_ld32(tdK + lane_off + c, vk);
-        tmem_ld32(tdV + lane_off + c, vv);
+        tmem_ld32(tdK + lane_off + cc, vk);
+        tmem_ld32(tdV + lane_off + cc, vv);
         if (key < a.s) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -762,8 +783,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
               wk[e] = *reinterpret_cast<uint32_t*>(&tk);
               wv[e] = *reinterpret_cast<uint32_t*>(&tv);
             }
-            *reinterpret_cast<uint4*>(out + a.h + head * kD + c + 8 * q) = uk;
-            *reinterpret_cast<uint4*>(out + 2 * a.h + head * kD + c + 8 * q) = uv;
+            *reinterpret_cast<uint4*>(out + a.h + head * kD + cc + 8 * q) = uk;
+            *reinterpret_cast<uint4*>(out + 2 * a.h + head * kD + cc + 8 * q) = uv;
           }
         }
       }
@@ -876,8 +897,8 @@ tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const vo
   if (e != cudaSuccess) return cuda_fail(e, "attention bwd smem attribute");
   dim3 gq(static_cast<unsigned>((sh.s + kBM - 1) / kBM), static_cast<unsigned>(sh.b * sh.heads));
   dim3 gk(static_cast<unsigned>((sh.s + kBN - 1) / kBN), static_cast<unsigned>(sh.b * sh.heads));
-  attn_bwd_dq_tcgen05<<<gq, kThreadsA, kSmemDQ, stream>>>(qkv128, qkv64, do128, a);
-  attn_bwd_dkdv_tcgen05<<<gk, kThreadsA, kSmemKV, stream>>>(qkv128, qkv64, do64, a);
+  attn_bwd_dq_tcgen05<<<gq, kThreadsB, kSmemDQ, stream>>>(qkv128, qkv64, do128, a);
+  attn_bwd_dkdv_tcgen05<<<gk, kThreadsB, kSmemKV, stream>>>(qkv128, qkv64, do64, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention bwd (tcgen05) launch");
   return TP_OK;

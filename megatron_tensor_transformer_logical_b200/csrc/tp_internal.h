@@ -130,8 +130,10 @@ enum VocabKernel : int {
 };
 tp_status launch_embed_fwd(const int* ids, const void* E, void* Y, int64_t M, int64_t V,
                            int64_t h, int t, bool f32, cudaStream_t stream);
+size_t embed_bwd_scratch_bytes(int64_t M);
 tp_status launch_embed_bwd(const int* ids, const void* dY, const void* dE_in, void* dE,
-                           int64_t M, int64_t V, int64_t h, bool f32, cudaStream_t stream);
+                           int64_t M, int64_t V, int64_t h, bool f32, void* scratch,
+                           cudaStream_t stream);
 // From the chunk partials of a kEpiCE GEMM: lse, loss and (if not NULL) the
 // total.  `shard_tot` holds t floats of scratch.
 tp_status launch_ce_finish(const CEOut& ce, int t, int64_t M, int64_t V, float* lse, float* loss,

@@ -4,7 +4,10 @@
 // The logits GEMM and its per-chunk reductions run in the tcgen05 GEMM
 // (kEpiCE epilogue); the kernels here are the HBM-bound remainder:
 //   embed_fwd     the masked row lookup of §4.1 (a gather),
-//   embed_bwd     its transpose, a deterministic scatter-add into dE,
+//   embed_bwd     its transpose: dE = dE_in or 0, then a deterministic
+//                 scatter-add of dY into the rows that tokens hit (tokens
+//                 sorted by id, one CTA per run of equal ids; or, for more
+//                 than 16384 tokens, a scan of the ids per 8-row group),
 //   ce_combine    §4.2 steps 2-5: chunk partials -> shard sums -> lse, loss,
 //   ce_shard_loss §4.2 step 6: per-shard loss sums, then their total,
 //   ce_dlogits    the softmax gradient, (exp(z - lse) - onehot) * dloss.
@@ -41,133 +44,321 @@ __global__ void __launch_bounds__(256) embed_fwd_kernel(const int* __restrict__ 
   }
 }
 
-// dE rows [v0, v0 + 8) x one column slice of 256 x 16 bytes per CTA.  The CTA
-// scans all ids in rounds of 2048 tokens, compacts the tokens that hit its 8
-// rows into a shared list in token order, and adds their dY slices into
-// fp32 registers in that order; so every row's sum has a fixed order.
+// The embedding backward in two kernels.  embed_bwd_init writes every row of
+// dE once: dE = dE_in, or zeros (skipped when dE_in is dE itself, the
+// accumulate-in-place case).  embed_bwd_scatter then adds the dY rows into
+// the rows that tokens hit, and touches no other row.
+__global__ void __launch_bounds__(256) embed_bwd_init_kernel(const uint4* __restrict__ src,
+                                                             uint4* __restrict__ dst,
+                                                             int64_t n_vec) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_vec;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[i] = src != nullptr ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+}
+
+// One CTA per group of 8 rows of dE.  It scans the ids in rounds of 2048
+// tokens, compacts the tokens that hit its rows into a shared list in token
+// order (ballots + per-warp counts), and for each 256 x 16-byte column slice
+// adds their dY slices into fp32 registers in that order, then adds the sums
+// to the hit rows of dE (read-modify-write).  The order of every row's sum is
+// fixed, so the result is deterministic without atomics.  A group no token
+// hits exits after one scan.
 constexpr int kEbRows = 8;
 constexpr int kEbThreads = 256;
 constexpr int kEbPerThread = 8;
 constexpr int kEbRound = kEbThreads * kEbPerThread;
 
-template <bool F32>
-__global__ void __launch_bounds__(kEbThreads, 2) embed_bwd_kernel(const int* __restrict__ ids,
-                                                               const void* __restrict__ dY,
-                                                               const void* dE_in, void* dE,
-                                                               int64_t M, int64_t V, int64_t h) {
-  constexpr int EPV = F32 ? 4 : 8;  // elements per 16-byte vector
-  __shared__ int list[kEbRound];
-  __shared__ int counts[kEbPerThread][kEbThreads / 32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * kEbRows;
-  const int64_t c0 = (static_cast<int64_t>(blockIdx.y) * kEbThreads + threadIdx.x) * EPV;
-  const bool col_ok = c0 < h;  // h % EPV == 0: a vector is all in or all out
-  float acc[kEbRows][EPV];
-#pragma unroll
-  for (int r = 0; r < kEbRows; ++r)
-#pragma unroll
-    for (int e = 0; e < EPV; ++e) acc[r][e] = 0.0f;
+struct EbList {
+  int entries[kEbRound];
+  int counts[kEbPerThread][kEbThreads / 32];
+  int total;
+  int rowmask;
+};
 
-  for (int64_t base = 0; base < M; base += kEbRound) {
-    unsigned hits[kEbPerThread];
-    int rows[kEbPerThread];
+// Builds the list of hits among tokens [base, base + 2048); returns its length.
+__device__ __forceinline__ int eb_build_list(const int* __restrict__ ids, int64_t base, int64_t M,
+                                             int64_t v0, int64_t V, EbList& L) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned hits[kEbPerThread];
+  int rows[kEbPerThread];
+  int mask = 0;
 #pragma unroll
-    for (int k = 0; k < kEbPerThread; ++k) {
-      const int64_t tok = base + k * kEbThreads + threadIdx.x;
-      const int64_t id = tok < M ? ids[tok] : -1;
-      const bool hit = id >= v0 && id < v0 + kEbRows && id < V;
-      rows[k] = static_cast<int>(id - v0);
-      hits[k] = __ballot_sync(0xffffffffu, hit);
-      if (lane == 0) counts[k][warp] = __popc(hits[k]);
-    }
-    __syncthreads();
-    // Token order is (k, warp, lane): the slot of a hit is the number of
-    // hits before it in that order.
-    int total = 0;  // hits of the steps before k
-#pragma unroll
-    for (int k = 0; k < kEbPerThread; ++k) {
-      int before = 0, in_k = 0;
-#pragma unroll
-      for (int w = 0; w < kEbThreads / 32; ++w) {
-        const int c = counts[k][w];
-        before += w < warp ? c : 0;
-        in_k += c;
-      }
-      if ((hits[k] >> lane) & 1u) {
-        const int slot = total + before + __popc(hits[k] & ((1u << lane) - 1u));
-        list[slot] = ((k * kEbThreads + static_cast<int>(threadIdx.x)) << 3) | rows[k];
-      }
-      total += in_k;
-    }
-    __syncthreads();
-    if (col_ok) {
-#pragma unroll 4
-      for (int e = 0; e < total; ++e) {
-        const int packed = list[e];
-        const int64_t tok = base + (packed >> 3);
-        const int rr = packed & 7;
-        float x[EPV];
-        if (F32) {
-          const float4 q = *reinterpret_cast<const float4*>(static_cast<const float*>(dY) +
-                                                            tok * h + c0);
-          x[0] = q.x; x[1] = q.y; x[2] = q.z; x[3] = q.w;
-        } else {
-          const uint4 q = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dY) +
-                                                          tok * h + c0);
-          const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
-#pragma unroll
-          for (int i = 0; i < EPV / 2; ++i) {
-            const float2 f = __bfloat1622float2(p[i]);
-            x[2 * i] = f.x;
-            x[2 * i + 1] = f.y;
-          }
-        }
-#pragma unroll
-        for (int r = 0; r < kEbRows; ++r)
-          if (r == rr)
-#pragma unroll
-            for (int i = 0; i < EPV; ++i) acc[r][i] += x[i];
-      }
-    }
-    __syncthreads();  // the list and counts are rewritten by the next round
+  for (int k = 0; k < kEbPerThread; ++k) {
+    const int64_t tok = base + k * kEbThreads + threadIdx.x;
+    const int64_t id = tok < M ? ids[tok] : -1;
+    const bool hit = id >= v0 && id < v0 + kEbRows && id < V;
+    rows[k] = static_cast<int>(id - v0);
+    if (hit) mask |= 1 << rows[k];
+    hits[k] = __ballot_sync(0xffffffffu, hit);
+    if (lane == 0) L.counts[k][warp] = __popc(hits[k]);
   }
-  if (!col_ok) return;
+  if (mask) atomicOr(&L.rowmask, mask);
+  __syncthreads();
+  // Token order is (k, warp, lane): a hit's slot is the number of hits before it.
+  int total = 0;
+#pragma unroll
+  for (int k = 0; k < kEbPerThread; ++k) {
+    int before = 0, in_k = 0;
+#pragma unroll
+    for (int w = 0; w < kEbThreads / 32; ++w) {
+      const int c = L.counts[k][w];
+      before += w < warp ? c : 0;
+      in_k += c;
+    }
+    if ((hits[k] >> lane) & 1u) {
+      const int slot = total + before + __popc(hits[k] & ((1u << lane) - 1u));
+      L.entries[slot] = ((k * kEbThreads + static_cast<int>(threadIdx.x)) << 3) | rows[k];
+    }
+    total += in_k;
+  }
+  __syncthreads();
+  return total;
+}
+
+template <bool F32>
+__device__ __forceinline__ void eb_accumulate(const EbList& L, int n, int64_t base,
+                                              const void* __restrict__ dY, int64_t h, int64_t c0,
+                                              float (&acc)[kEbRows][F32 ? 4 : 8]) {
+  constexpr int EPV = F32 ? 4 : 8;
+#pragma unroll 2
+  for (int e = 0; e < n; ++e) {
+    const int packed = L.entries[e];
+    const int64_t tok = base + (packed >> 3);
+    const int rr = packed & 7;
+    float x[EPV];
+    if (F32) {
+      const float4 q = *reinterpret_cast<const float4*>(static_cast<const float*>(dY) + tok * h +
+                                                        c0);
+      x[0] = q.x; x[1] = q.y; x[2] = q.z; x[3] = q.w;
+    } else {
+      const uint4 q = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dY) +
+                                                      tok * h + c0);
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+      for (int i = 0; i < EPV / 2; ++i) {
+        const float2 f = __bfloat1622float2(p[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kEbRows; ++r)
+      if (r == rr)
+#pragma unroll
+        for (int i = 0; i < EPV; ++i) acc[r][i] += x[i];
+  }
+}
+
+template <bool F32>
+__device__ __forceinline__ void eb_add_rows(void* dE, int64_t v0, int64_t h, int64_t c0,
+                                            int rowmask, const float (&acc)[kEbRows][F32 ? 4 : 8]) {
+  constexpr int EPV = F32 ? 4 : 8;
 #pragma unroll
   for (int r = 0; r < kEbRows; ++r) {
-    const int64_t v = v0 + r;
-    if (v >= V) break;
+    if (!((rowmask >> r) & 1)) continue;
     if (F32) {
-      float* o = static_cast<float*>(dE) + v * h + c0;
-      float4 q = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-      if (dE_in != nullptr) {
-        const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(dE_in) +
-                                                          v * h + c0);
-        q.x += b.x; q.y += b.y; q.z += b.z; q.w += b.w;
-      }
-      *reinterpret_cast<float4*>(o) = q;
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(dE) + (v0 + r) * h + c0);
+      float4 q = *o;
+      q.x += acc[r][0]; q.y += acc[r][1]; q.z += acc[r][2]; q.w += acc[r][3];
+      *o = q;
     } else {
-      float y[EPV];
-#pragma unroll
-      for (int i = 0; i < EPV; ++i) y[i] = acc[r][i];
-      if (dE_in != nullptr) {
-        const uint4 q = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dE_in) +
-                                                        v * h + c0);
-        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
-#pragma unroll
-        for (int i = 0; i < EPV / 2; ++i) {
-          const float2 f = __bfloat1622float2(p[i]);
-          y[2 * i] += f.x;
-          y[2 * i + 1] += f.y;
-        }
-      }
+      uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dE) + (v0 + r) * h + c0);
+      const uint4 q = *o;
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
       uint4 out;
       uint32_t* w = reinterpret_cast<uint32_t*>(&out);
 #pragma unroll
       for (int i = 0; i < EPV / 2; ++i) {
-        __nv_bfloat162 t2 = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
+        const float2 f = __bfloat1622float2(p[i]);
+        __nv_bfloat162 t2 = __floats2bfloat162_rn(f.x + acc[r][2 * i], f.y + acc[r][2 * i + 1]);
         w[i] = *reinterpret_cast<uint32_t*>(&t2);
       }
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dE) + v * h + c0) = out;
+      *o = out;
+    }
+  }
+}
+
+template <bool F32>
+__global__ void __launch_bounds__(kEbThreads, 1) embed_bwd_scatter_kernel(
+    const int* __restrict__ ids, const void* __restrict__ dY, void* dE, int64_t M, int64_t V,
+    int64_t h) {
+  constexpr int EPV = F32 ? 4 : 8;
+  constexpr int64_t kSlice = int64_t(kEbThreads) * EPV;
+  __shared__ EbList L;
+  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * kEbRows;
+  if (threadIdx.x == 0) L.rowmask = 0;
+  __syncthreads();
+  float acc[kEbRows][EPV];
+  if (M <= kEbRound) {
+    // One round: the list is built once and serves every column slice.
+    const int n = eb_build_list(ids, 0, M, v0, V, L);
+    if (n == 0) return;
+    const int rowmask = L.rowmask;
+    for (int64_t c0 = threadIdx.x * EPV; c0 < h; c0 += kSlice) {
+#pragma unroll
+      for (int r = 0; r < kEbRows; ++r)
+#pragma unroll
+        for (int i = 0; i < EPV; ++i) acc[r][i] = 0.0f;
+      eb_accumulate<F32>(L, n, 0, dY, h, c0, acc);
+      eb_add_rows<F32>(dE, v0, h, c0, rowmask, acc);
+    }
+    return;
+  }
+  // Several rounds: the lists are rebuilt for every column slice.
+  for (int64_t s0 = 0; s0 < h; s0 += kSlice) {
+    const int64_t c0 = s0 + threadIdx.x * EPV;
+    const bool col_ok = c0 < h;
+#pragma unroll
+    for (int r = 0; r < kEbRows; ++r)
+#pragma unroll
+      for (int i = 0; i < EPV; ++i) acc[r][i] = 0.0f;
+    for (int64_t base = 0; base < M; base += kEbRound) {
+      const int n = eb_build_list(ids, base, M, v0, V, L);
+      if (col_ok) eb_accumulate<F32>(L, n, base, dY, h, c0, acc);
+      __syncthreads();  // the list is rewritten by the next round
+    }
+    if (col_ok) eb_add_rows<F32>(dE, v0, h, c0, L.rowmask, acc);
+  }
+}
+
+// Sorted form (M <= kSortMax tokens).  embed_sort_kernel, one CTA, sorts the
+// (id, token) pairs by id with a bitonic network in shared memory (keys are
+// unique, so equal ids keep token order), then lists the runs of equal valid
+// ids: run r covers sorted positions [run_start[r], run_start[r + 1]) and
+// has id run_id[r]; ids outside [0, V) sort to the end and form no run.
+constexpr int kSortMax = 16384;
+constexpr int kSortThreads = 1024;
+
+__global__ void __launch_bounds__(kSortThreads) embed_sort_kernel(
+    const int* __restrict__ ids, int M, int n_pow2, int64_t V, int* sorted_tok, int* run_start,
+    int* run_id, int* n_runs) {
+  extern __shared__ unsigned long long keys[];
+  __shared__ int warp_sums[kSortThreads / 32];
+  for (int i = threadIdx.x; i < n_pow2; i += blockDim.x)
+    keys[i] = i < M ? (static_cast<unsigned long long>(static_cast<unsigned>(ids[i])) << 32) |
+                          static_cast<unsigned>(i)
+                    : ~0ull;
+  __syncthreads();
+  for (int k = 2; k <= n_pow2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long a = keys[i], b = keys[ixj];
+          const bool up = (i & k) == 0;
+          if ((a > b) == up) {
+            keys[i] = b;
+            keys[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // Runs: thread t owns the contiguous positions [t*per, (t+1)*per).
+  const int per = (M + kSortThreads - 1) / kSortThreads;
+  const int p0 = threadIdx.x * per, p1 = min(p0 + per, M);
+  int count = 0;
+  for (int p = p0; p < p1; ++p) {
+    const unsigned long long id = keys[p] >> 32;
+    sorted_tok[p] = static_cast<int>(keys[p] & 0xffffffffu);
+    if (id < static_cast<unsigned long long>(V) && (p == 0 || (keys[p - 1] >> 32) != id)) ++count;
+  }
+  // Block-wide exclusive scan of the run counts (warp scans, then warp totals).
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = count;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += v;
+    }
+    warp_sums[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  int r = incl - count + (warp > 0 ? warp_sums[warp - 1] : 0);
+  for (int p = p0; p < p1; ++p) {
+    const unsigned long long id = keys[p] >> 32;
+    if (id < static_cast<unsigned long long>(V) && (p == 0 || (keys[p - 1] >> 32) != id)) {
+      run_start[r] = p;
+      run_id[r] = static_cast<int>(id);
+      ++r;
+    }
+  }
+  if (threadIdx.x == kSortThreads - 1) {
+    const int total = warp_sums[kSortThreads / 32 - 1];
+    *n_runs = total;
+    // End of the last valid run: the first position whose id is not valid.
+    int end = M;
+    for (int p = M - 1; p >= 0 && (keys[p] >> 32) >= static_cast<unsigned long long>(V); --p)
+      end = p;
+    run_start[total] = end;
+  }
+}
+
+// One CTA per (run, 2048-column slice): sums the run's dY rows in token
+// order in fp32 (eight loads in flight per thread) and adds the sum to its
+// row of dE.
+template <bool F32>
+__global__ void __launch_bounds__(256) embed_run_scatter_kernel(
+    const int* __restrict__ sorted_tok, const int* __restrict__ run_start,
+    const int* __restrict__ run_id, const int* __restrict__ n_runs, const void* __restrict__ dY,
+    void* dE, int64_t h) {
+  constexpr int EPV = F32 ? 4 : 8;
+  const int64_t c0 = (static_cast<int64_t>(blockIdx.y) * blockDim.x + threadIdx.x) * EPV;
+  if (c0 >= h) return;
+  const int nr = *n_runs;
+  for (int r = blockIdx.x; r < nr; r += gridDim.x) {
+    const int e0 = run_start[r], e1 = run_start[r + 1];
+    float acc[EPV];
+#pragma unroll
+    for (int i = 0; i < EPV; ++i) acc[i] = 0.0f;
+#pragma unroll 8
+    for (int e = e0; e < e1; ++e) {
+      const int64_t tok = sorted_tok[e];
+      if (F32) {
+        const float4 q = *reinterpret_cast<const float4*>(static_cast<const float*>(dY) +
+                                                          tok * h + c0);
+        acc[0] += q.x; acc[1] += q.y; acc[2] += q.z; acc[3] += q.w;
+      } else {
+        const uint4 q = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dY) +
+                                                        tok * h + c0);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+        for (int i = 0; i < EPV / 2; ++i) {
+          const float2 f = __bfloat1622float2(p[i]);
+          acc[2 * i] += f.x;
+          acc[2 * i + 1] += f.y;
+        }
+      }
+    }
+    const int64_t v = run_id[r];
+    if (F32) {
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(dE) + v * h + c0);
+      float4 q = *o;
+      q.x += acc[0]; q.y += acc[1]; q.z += acc[2]; q.w += acc[3];
+      *o = q;
+    } else {
+      uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dE) + v * h + c0);
+      const uint4 q = *o;
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+      uint4 out;
+      uint32_t* w = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+      for (int i = 0; i < EPV / 2; ++i) {
+        const float2 f = __bfloat1622float2(p[i]);
+        __nv_bfloat162 t2 = __floats2bfloat162_rn(f.x + acc[2 * i], f.y + acc[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&t2);
+      }
+      *o = out;
     }
   }
 }
@@ -310,21 +501,75 @@ tp_status launch_embed_fwd(const int* ids, const void* E, void* Y, int64_t M, in
   return e == cudaSuccess ? TP_OK : cuda_fail(e, "embed_fwd launch");
 }
 
+size_t embed_bwd_scratch_bytes(int64_t M) {
+  if (M > kSortMax) return 0;
+  return static_cast<size_t>(3 * M + 2) * sizeof(int);
+}
+
 tp_status launch_embed_bwd(const int* ids, const void* dY, const void* dE_in, void* dE,
-                           int64_t M, int64_t V, int64_t h, bool f32, cudaStream_t stream) {
-  const int epv = f32 ? 4 : 8;
+                           int64_t M, int64_t V, int64_t h, bool f32, void* scratch,
+                           cudaStream_t stream) {
   const int64_t gx = (V + kEbRows - 1) / kEbRows;
-  const int64_t gy = (h + int64_t(kEbThreads) * epv - 1) / (int64_t(kEbThreads) * epv);
-  if (gx > 0x7fffffffLL || gy > 65535) return fail(TP_ERR_SHAPE, "embedding backward: V or h too large");
+  if (gx > 0x7fffffffLL) return fail(TP_ERR_SHAPE, "embedding backward: V too large");
   const double es = f32 ? 4.0 : 2.0;
-  const double bytes = es * (double(V) * h * (dE_in ? 2.0 : 1.0) + double(M) * h) + 4.0 * M;
-  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+  const bool init = dE_in != dE;  // in place: only the hit rows change
+  const bool sorted = M > 0 && M <= kSortMax;
+  const int64_t hit_rows = M < V ? M : V;
+  // Bytes: the init pass (all of dE written, dE_in read) and at most
+  // min(M, V) rows read and written by the scatter, plus dY and the ids.
+  const double bytes = (init ? es * double(V) * h * (dE_in ? 2.0 : 1.0) : 0.0) +
+                       es * (double(M) * h + 2.0 * double(hit_rows) * h) + 4.0 * M;
+  const int kernels = (init ? 1 : 0) + (M > 0 ? (sorted ? 2 : 1) : 0);
+  const int64_t slices = (h + 256 * (f32 ? 4 : 8) - 1) / (256 * (f32 ? 4 : 8));
+  if (sorted) {
+    static unsigned long long configured = 0;  // one bit per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!(configured & (1ull << (dev & 63)))) {
+      cudaError_t e = cudaFuncSetAttribute(embed_sort_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kSortMax * 8);
+      if (e != cudaSuccess) return cuda_fail(e, "embed_sort smem attribute");
+      configured |= 1ull << (dev & 63);
+    }
+    if (scratch == nullptr) return fail(TP_ERR_WORKSPACE, "embedding backward: workspace missing");
+    if (slices > 65535) return fail(TP_ERR_SHAPE, "embedding backward: h too large");
+  }
   {
-    LaunchScope scope(TP_KIND_VOCAB, double(M) * h, bytes, stream, 1, kVocabEmbedBwd);
-    if (f32)
-      embed_bwd_kernel<true><<<grid, kEbThreads, 0, stream>>>(ids, dY, dE_in, dE, M, V, h);
-    else
-      embed_bwd_kernel<false><<<grid, kEbThreads, 0, stream>>>(ids, dY, dE_in, dE, M, V, h);
+    LaunchScope scope(TP_KIND_VOCAB, double(M) * h, bytes, stream, kernels, kVocabEmbedBwd);
+    if (init) {
+      const int64_t n_vec = V * h * static_cast<int64_t>(es) / 16;
+      const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+      const int64_t blocks = (n_vec + 255) / 256;
+      embed_bwd_init_kernel<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0,
+                              stream>>>(static_cast<const uint4*>(dE_in), static_cast<uint4*>(dE),
+                                        n_vec);
+    }
+    if (sorted) {
+      int* sorted_tok = static_cast<int*>(scratch);
+      int* run_start = sorted_tok + M;
+      int* run_id = run_start + M + 1;
+      int* n_runs = run_id + M;
+      int n_pow2 = 2;
+      while (n_pow2 < M) n_pow2 <<= 1;
+      embed_sort_kernel<<<1, kSortThreads, static_cast<size_t>(n_pow2) * 8, stream>>>(
+          ids, static_cast<int>(M), n_pow2, V, sorted_tok, run_start, run_id, n_runs);
+      const int64_t runs_cap = M < 8192 ? M : 8192;
+      dim3 grid(static_cast<unsigned>(runs_cap), static_cast<unsigned>(slices));
+      if (f32)
+        embed_run_scatter_kernel<true><<<grid, 256, 0, stream>>>(sorted_tok, run_start, run_id,
+                                                                 n_runs, dY, dE, h);
+      else
+        embed_run_scatter_kernel<false><<<grid, 256, 0, stream>>>(sorted_tok, run_start, run_id,
+                                                                  n_runs, dY, dE, h);
+    } else if (M > 0) {
+      if (f32)
+        embed_bwd_scatter_kernel<true><<<static_cast<unsigned>(gx), kEbThreads, 0, stream>>>(
+            ids, dY, dE, M, V, h);
+      else
+        embed_bwd_scatter_kernel<false><<<static_cast<unsigned>(gx), kEbThreads, 0, stream>>>(
+            ids, dY, dE, M, V, h);
+    }
   }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? TP_OK : cuda_fail(e, "embed_bwd launch");

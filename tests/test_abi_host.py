@@ -170,9 +170,13 @@ def test_vocab_validation(lib):
     assert ef(P[0], P[1], P[2], 16, 1024, 64, 0, bf, None) == L.TP_ERR_SHAPE
     assert ef(P[0], P[1], P[2], 16, 1024, 64, 4, 7, None) == L.TP_ERR_DTYPE
     assert ef(P[0], P[1], P[2], 0, 1024, 64, 4, bf, None) == L.TP_OK          # nothing to do
-    assert eb(P[0], None, None, P[3], 16, 1024, 64, 4, bf, None) == L.TP_ERR_NULL
-    assert eb(P[0], P[1], None, None, 16, 1024, 64, 4, bf, None) == L.TP_ERR_NULL
-    assert eb(P[0], P[1], None, P[3], 1 << 28, 1024, 64, 4, bf, None) == L.TP_ERR_SHAPE
+    assert eb(P[0], None, None, P[3], 16, 1024, 64, 4, bf, P[9], big, None) == L.TP_ERR_NULL
+    assert eb(P[0], P[1], None, None, 16, 1024, 64, 4, bf, P[9], big, None) == L.TP_ERR_NULL
+    assert eb(P[0], P[1], None, P[3], 1 << 28, 1024, 64, 4, bf, P[9], big, None) == L.TP_ERR_SHAPE
+    assert eb(P[0], P[1], None, P[3], 16, 1024, 64, 4, bf, None, 0, None) == L.TP_ERR_WORKSPACE
+    need_e = lib.tp_workspace_size(L.TP_OP_VOCAB_EMBED_BWD, 16, 64, 1024, 0, 4, bf)
+    assert need_e >= 3 * 16 * 4
+    assert eb(P[0], P[1], None, P[3], 16, 1024, 64, 4, bf, P[9], need_e - 1, None) == L.TP_ERR_WORKSPACE
     cf, cb = lib.tp_vocab_ce_fwd, lib.tp_vocab_ce_bwd
     ok = (P[0], P[1], P[2], P[3], P[4], P[5], None)
     assert cf(None, *ok[1:], 64, 256, 1024, 4, bf, P[9], big, None) == L.TP_ERR_NULL

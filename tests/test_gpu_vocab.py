@@ -31,6 +31,13 @@ def _gpu():
 
 # ------------------------------------------------------------------ embedding
 
+def embed_bwd(ids, dY, dE_in, dE, t):
+    M = ids.numel()
+    ws = (L.workspace(L.TP_OP_VOCAB_EMBED_BWD, M, dE.shape[1], dE.shape[0], 0, t, L.TP_BF16)
+          if M > 0 else None)
+    L.tp_vocab_embed_bwd(ids, dY, dE_in, dE, t, ws)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("t", [1, 2, 8])
 def test_embed_fwd_exact(dtype, t):
@@ -57,7 +64,7 @@ def test_embed_bwd_integer_exact(dtype, accumulate):
     dY = integer_tensor((M, h), -1, 1, 4, tdt)
     dE_in = integer_tensor((V, h), -4, 4, 5, tdt) if accumulate else None
     dE = torch.full((V, h), float("nan"), dtype=tdt, device="cuda")
-    L.tp_vocab_embed_bwd(cuda(ids), cuda(dY), cuda(dE_in), dE, 4)
+    embed_bwd(cuda(ids), cuda(dY), cuda(dE_in), dE, 4)
     torch.cuda.synchronize()
     ref = O.vocab_embed_bwd(ids.numpy(), dY, V)
     if accumulate:
@@ -74,9 +81,26 @@ def test_embed_bwd_in_place_and_hot_token():
     dY = normal_tensor((M, h), 1.0, 6)
     base = normal_tensor((V, h), 1.0, 7)
     dE = cuda(base.clone())
-    L.tp_vocab_embed_bwd(cuda(ids), cuda(dY), dE, dE, 1)
+    embed_bwd(cuda(ids), cuda(dY), dE, dE, 1)
     torch.cuda.synchronize()
     check(dE, O.vocab_embed_bwd(ids.numpy(), dY, V) + to64(base), "dE (in place)", "bf16")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_embed_bwd_many_tokens_exact(dtype):
+    """More than 16384 tokens: the per-group id scan instead of the sort."""
+    V, h, M = 640, 1032, 20000
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    ids = zipf_ids(M, V, 11, exponent=0.3)
+    ids[::1000] = V + 5
+    dY = integer_tensor((M, h), -1, 1, 12, tdt)
+    dE_in = integer_tensor((V, h), -4, 4, 13, tdt)
+    dE = torch.full((V, h), float("nan"), dtype=tdt, device="cuda")
+    embed_bwd(cuda(ids), cuda(dY), cuda(dE_in), dE, 8)
+    torch.cuda.synchronize()
+    ref = O.vocab_embed_bwd(ids.numpy(), dY, V) + to64(dE_in)
+    assert np.max(np.abs(ref)) < 256
+    assert np.array_equal(to64(dE), ref)
 
 
 def test_embed_bwd_deterministic_and_zero_tokens():
@@ -86,13 +110,13 @@ def test_embed_bwd_deterministic_and_zero_tokens():
     outs = []
     for _ in range(2):
         dE = torch.empty((V, h), dtype=torch.bfloat16, device="cuda")
-        L.tp_vocab_embed_bwd(cuda(ids), cuda(dY), None, dE, 8)
+        embed_bwd(cuda(ids), cuda(dY), None, dE, 8)
         outs.append(dE)
     torch.cuda.synchronize()
     assert torch.equal(outs[0], outs[1])
     check(outs[0], O.vocab_embed_bwd(ids.numpy(), dY, V), "dE", "bf16")
     empty = torch.full((V, h), float("nan"), dtype=torch.bfloat16, device="cuda")
-    L.tp_vocab_embed_bwd(torch.empty(0, dtype=torch.int32, device="cuda"),
+    embed_bwd(torch.empty(0, dtype=torch.int32, device="cuda"),
                          torch.empty(0, h, dtype=torch.bfloat16, device="cuda"), None, empty, 8)
     torch.cuda.synchronize()
     assert not empty.float().abs().sum().item()
@@ -224,7 +248,7 @@ def test_tied_embedding_and_loss_end_to_end():
     dY = torch.empty_like(Y)
     dE = torch.empty_like(Ed)
     L.tp_vocab_ce_bwd(Y, Ed, td, logits, lse, None, logits, dY, dE, wl.t)
-    L.tp_vocab_embed_bwd(cuda(ids), dY, dE, dE, wl.t)
+    embed_bwd(cuda(ids), dY, dE, dE, wl.t)
     torch.cuda.synchronize()
     Y64 = O.vocab_embed_fwd(ids.numpy(), E)
     assert np.array_equal(to64(Y), Y64)
