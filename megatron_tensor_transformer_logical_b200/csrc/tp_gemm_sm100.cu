@@ -730,12 +730,15 @@ int tile_override() {
 
 // Tile kind: 128, 192 or 256 columns on one SM, or 512 = 256 x 256 on an SM
 // pair.  Picks the least estimated time, ceil(tiles / slots) x work per tile
-// / relative rate.  The rates are per-clock throughputs relative to the
-// 256-wide single-SM tile, measured on the 175B-shaped layer's twelve GEMMs
-// under the sustained power cap: with A K-major and B MN-major (the forward
-// linears) the single-SM tile is ~5% faster than the pair; with B K-major
-// (dgrads) or both operands MN-major (wgrads) the pair is 4-10% faster; the
-// 192- and 128-wide tiles only pay where they fill the last wave far better.
+// / relative rate.  The rates are throughputs relative to the 256-wide
+// single-SM tile, measured on the 175B-shaped layer's twelve GEMMs under the
+// sustained power cap with the tile kinds interleaved step by step: with A
+// K-major and B MN-major (the forward linears) the single-SM tile is 3-5%
+// faster than the pair; with both operands MN-major (wgrads) the pair is
+// 6-12% faster; with both K-major (dgrads) the single-SM tile is 3-6% faster
+// in natural K order and the pair 7% faster in the attention's head-group K
+// order.  The 192- and 128-wide tiles run 15% and 30% slower per tile and
+// only pay where they fill the last wave far better.
 int choose_tile(const Gemm& g) {
   const int ov = tile_override();
   if (ov != 0) return ov;
@@ -743,7 +746,7 @@ int choose_tile(const Gemm& g) {
   double best = 1e300;
   int kind = 256;
   const int widths[3] = {256, 192, 128};
-  const double rate[3] = {1.0, 0.8, 0.8};
+  const double rate[3] = {1.0, 0.85, 0.68};
   for (int i = 0; i < 3; ++i) {
     const Plan p = plan_for(g, widths[i]);
     const double t = std::ceil(double(p.m_tiles) * p.n_tiles / sms) * 128.0 * widths[i] / rate[i];
@@ -752,7 +755,13 @@ int choose_tile(const Gemm& g) {
       kind = widths[i];
     }
   }
-  const double pair_rate = (g.a.k_major && !g.b.k_major) ? 0.95 : 1.07;
+  double pair_rate;
+  if (g.a.k_major && !g.b.k_major)
+    pair_rate = 0.96;                                 // forward
+  else if (g.a.k_major && g.b.k_major)
+    pair_rate = g.korder.range_blocks > 0 ? 1.07 : 0.96;  // dgrad
+  else
+    pair_rate = 1.10;                                 // wgrad
   const Plan pp = plan_for(g, kPairTN);
   const double pair_tiles = double((g.M + kPairTM - 1) / kPairTM) * pp.n_tiles;
   const double tp = std::ceil(pair_tiles / std::floor(sms / 2)) * 256.0 * 256.0 / 2.0 / pair_rate;

@@ -321,22 +321,36 @@ __global__ void __launch_bounds__(256) embed_run_scatter_kernel(
     float acc[EPV];
 #pragma unroll
     for (int i = 0; i < EPV; ++i) acc[i] = 0.0f;
-#pragma unroll 8
-    for (int e = e0; e < e1; ++e) {
-      const int64_t tok = sorted_tok[e];
-      if (F32) {
-        const float4 q = *reinterpret_cast<const float4*>(static_cast<const float*>(dY) +
-                                                          tok * h + c0);
-        acc[0] += q.x; acc[1] += q.y; acc[2] += q.z; acc[3] += q.w;
-      } else {
-        const uint4 q = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dY) +
-                                                        tok * h + c0);
-        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+    // Batches of eight rows: the eight loads are issued before any is added,
+    // so a long run (a frequent token) costs one round trip per batch.
+    for (int e = e0; e < e1; e += 8) {
+      uint4 q[8];
 #pragma unroll
-        for (int i = 0; i < EPV / 2; ++i) {
-          const float2 f = __bfloat1622float2(p[i]);
-          acc[2 * i] += f.x;
-          acc[2 * i + 1] += f.y;
+      for (int b = 0; b < 8; ++b) {
+        if (e + b < e1) {
+          const int64_t tok = sorted_tok[e + b];
+          q[b] = F32 ? *reinterpret_cast<const uint4*>(static_cast<const float*>(dY) + tok * h + c0)
+                     : *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dY) +
+                                                       tok * h + c0);
+        } else {
+          q[b] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        if (e + b >= e1) break;  // adds stay in token order; zeros are never added
+        if (F32) {
+          const float* f = reinterpret_cast<const float*>(&q[b]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i] += f[i];
+        } else {
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q[b]);
+#pragma unroll
+          for (int i = 0; i < EPV / 2; ++i) {
+            const float2 f = __bfloat1622float2(p2[i]);
+            acc[2 * i] += f.x;
+            acc[2 * i + 1] += f.y;
+          }
         }
       }
     }

@@ -10,6 +10,11 @@ Cases (175B-shaped layer unless noted; bf16, t = 8):
   attn_fwd    tp_attn_fwd    (QKV GEMM, attention core, Wo GEMM)
   attn_bwd    tp_attn_bwd
   small_gemm  tp_linear_col  X[1024,4096] @ W[4096,8192] (a quick case)
+  vocab_step  the tied vocabulary-parallel embedding + cross-entropy, forward and
+              backward on the seeded vocabulary workload (M=2048, h=12288,
+              V=51200, t=8, Zipf token ids): embedding gather, logits
+              GEMM with the loss epilogue, loss combination, softmax gradient,
+              dX and dE GEMMs, embedding scatter-add
 
 Inputs are seeded N(0,1) / N(0, 0.006^2) tensors made on the device; nothing
 is checked here (the tests do that).  Prints the mean device time per call.
@@ -70,6 +75,26 @@ def make_case(name: str):
         wsb = L.workspace(L.TP_OP_ATTN_BWD, M, h, 0, heads, t, L.TP_BF16)
         return lambda: L.tp_attn_bwd(X, Wqkv, Wo, QKV, O, LSE, dZ, dX, dWqkv, dWo, 1, M, heads, t,
                                      True, wsb)
+    if name == "vocab_step":
+        from .inputs import WORKLOADS, make_vocab_inputs
+        wl = WORKLOADS[6]
+        V = wl.vocab
+        d = {k: v.to("cuda") for k, v in make_vocab_inputs(wl).items()}
+        ids, targets, E, X, dY = d["ids"], d["targets"], d["E"], d["X"], d["dY"]
+        Y, dX = torch.empty(M, h, dtype=bf, device="cuda"), torch.empty(M, h, dtype=bf, device="cuda")
+        logits = torch.empty(M, V, dtype=bf, device="cuda")
+        lse, loss = (torch.empty(M, dtype=torch.float32, device="cuda") for _ in range(2))
+        total = torch.empty(1, dtype=torch.float32, device="cuda")
+        dE = torch.empty_like(E)
+        wsc = L.workspace(L.TP_OP_VOCAB_CE_FWD, M, h, V, 0, t, L.TP_BF16)
+        wse = L.workspace(L.TP_OP_VOCAB_EMBED_BWD, M, h, V, 0, t, L.TP_BF16)
+
+        def step():
+            L.tp_vocab_embed_fwd(ids, E, Y, t)
+            L.tp_vocab_ce_fwd(X, E, targets, logits, lse, loss, total, t, wsc)
+            L.tp_vocab_ce_bwd(X, E, targets, logits, lse, None, logits, dX, dE, t)
+            L.tp_vocab_embed_bwd(ids, dY, dE, dE, t, wse)
+        return step
     raise SystemExit(f"unknown case {name}")
 
 
