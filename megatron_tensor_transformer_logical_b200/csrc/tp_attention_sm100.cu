@@ -348,9 +348,12 @@ struct BwdArgs {
   int* status;
 };
 
-// Q (128 rows, once), dO (128 rows, once), then K_j, V_j (64 rows) in two stages.
-// Shared memory: Q 32K | dO 32K | KV[2] (K 16K + V 16K) | dS[2] 16K each.
-constexpr int kSmemDQ = 1024 + 2 * kTile + 2 * (2 * kTile64) + 2 * kTile128x64 + 256;
+// Q (128 rows, once), dO (128 rows, once), then K_j, V_j (64 rows) in a ring
+// of kKvStages stages (deep enough to cover the L2 latency of a 32 KB load
+// with several blocks of work).
+// Shared memory: Q 32K | dO 32K | KV[4] (K 16K + V 16K) | dS[2] 16K each.
+constexpr int kKvStages = 4;
+constexpr int kSmemDQ = 1024 + 2 * kTile + kKvStages * (2 * kTile64) + 2 * kTile128x64 + 256;
 
 __global__ void __launch_bounds__(kThreadsB, 1)
     attn_bwd_dq_tcgen05(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
@@ -361,16 +364,16 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   uint8_t* sQ = smem;
   uint8_t* sdO = smem + kTile;
   uint8_t* sKV = smem + 2 * kTile;                 // stage st: K at +0, V at +kTile64
-  uint8_t* sdS = sKV + 2 * (2 * kTile64);           // [2] x 16 KB
+  uint8_t* sdS = sKV + kKvStages * (2 * kTile64);   // [2] x 16 KB
   uint64_t* bars = reinterpret_cast<uint64_t*>(sdS + 2 * kTile128x64);
   uint64_t* qd_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* ds_full = bars + 7;   // [2]
-  uint64_t* ds_free = bars + 9;   // [2]
-  uint64_t* dq_done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* kv_full = bars + 1;                   // [kKvStages]
+  uint64_t* kv_empty = kv_full + kKvStages;       // [kKvStages]
+  uint64_t* s_full = kv_empty + kKvStages;        // [2]
+  uint64_t* ds_full = s_full + 2;                 // [2]
+  uint64_t* ds_free = ds_full + 2;                // [2]
+  uint64_t* dq_done = ds_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dq_done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (a.s + kBM - 1) / kBM;
@@ -383,9 +386,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kKvStages; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&ds_full[i], kEwWarpsB);
       mbar_init(&ds_free[i], 1);
@@ -417,17 +422,16 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       tma_load_2d(sdO, &tmdO, qd_full, head * kD, row0 + q0);
       tma_load_2d(sdO + kHalf, &tmdO, qd_full, head * kD + 64, row0 + q0);
       for (int j = 0; j < n_kb && ok; ++j) {
-        const int st = j & 1;
-        if (!(ok = mbar_wait(&kv_empty[st], ((static_cast<uint32_t>(j) >> 1) & 1u) ^ 1u, a.status,
-                             kStatusAttnTimeout)))
-          break;
-        mbar_arrive_expect_tx(&kv_full[st], 2 * kTile64);
-        uint8_t* k_dst = sKV + st * (2 * kTile64);
+        const int ks = j % kKvStages;
+        const uint32_t kph = static_cast<uint32_t>(j / kKvStages) & 1u;
+        if (!(ok = mbar_wait(&kv_empty[ks], kph ^ 1u, a.status, kStatusAttnTimeout))) break;
+        mbar_arrive_expect_tx(&kv_full[ks], 2 * kTile64);
+        uint8_t* k_dst = sKV + ks * (2 * kTile64);
         const int krow = row0 + j * kB64;
-        tma_load_2d(k_dst, &tmKV, &kv_full[st], a.h + head * kD, krow);
-        tma_load_2d(k_dst + kHalf64, &tmKV, &kv_full[st], a.h + head * kD + 64, krow);
-        tma_load_2d(k_dst + kTile64, &tmKV, &kv_full[st], 2 * a.h + head * kD, krow);
-        tma_load_2d(k_dst + kTile64 + kHalf64, &tmKV, &kv_full[st], 2 * a.h + head * kD + 64, krow);
+        tma_load_2d(k_dst, &tmKV, &kv_full[ks], a.h + head * kD, krow);
+        tma_load_2d(k_dst + kHalf64, &tmKV, &kv_full[ks], a.h + head * kD + 64, krow);
+        tma_load_2d(k_dst + kTile64, &tmKV, &kv_full[ks], 2 * a.h + head * kD, krow);
+        tma_load_2d(k_dst + kTile64 + kHalf64, &tmKV, &kv_full[ks], 2 * a.h + head * kD + 64, krow);
       }
     }
   } else if (warp == 1) {
@@ -438,11 +442,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       bool ok = mbar_wait(qd_full, 0, a.status, kStatusAttnTimeout);
       auto issue_sp = [&](int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait(&kv_full[st], (static_cast<uint32_t>(j) >> 1) & 1u, a.status,
+        const int ks = j % kKvStages;
+        if (!mbar_wait(&kv_full[ks], static_cast<uint32_t>(j / kKvStages) & 1u, a.status,
                        kStatusAttnTimeout))
           return false;
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sKV + st * (2 * kTile64));
+        const uint32_t k_addr = smem_u32(sKV + ks * (2 * kTile64));
         const uint32_t v_addr = k_addr + kTile64;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
@@ -464,14 +469,15 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                              kStatusAttnTimeout)))
           break;
         tc_fence_after();
+        const int ks = j % kKvStages;
         const uint32_t ds_addr = smem_u32(sdS + st * kTile128x64);
-        const uint32_t k_addr = smem_u32(sKV + st * (2 * kTile64));
+        const uint32_t k_addr = smem_u32(sKV + ks * (2 * kTile64));
 #pragma unroll
         for (int kk = 0; kk < kB64 / 16; ++kk) {
           umma_bf16(tQ, sw128_desc(ds_addr + kk * 32, 16, 1024),
                     sw128_desc(k_addr + kk * 2048, kHalf64, 1024), kIdQ, (j | kk) != 0 ? 1u : 0u);
         }
-        umma_commit(&kv_empty[st]);
+        umma_commit(&kv_empty[ks]);
         umma_commit(&ds_free[st]);
       }
       if (ok) umma_commit(dq_done);
@@ -554,10 +560,15 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// K, V (128 rows, once), then Q_i, dO_i (64 rows) in two stages; P^T and dS^T
-// tiles [128 keys x 64 queries] in two stages.
-// Shared memory: K 32K | V 32K | QdO[2] (Q 16K + dO 16K) | PdS[2] (P^T 16K + dS^T 16K).
-constexpr int kSmemKV = 1024 + 2 * kTile + 2 * (2 * kTile64) + 2 * (2 * kTile128x64) + 256;
+// K, V (128 rows, once), then Q_i, dO_i (64 rows) with the block's LSE * log2(e)
+// and D in a ring of kQdStages stages; P^T and dS^T tiles [128 keys x 64
+// queries] in two stages.  The TMA warp stages LSE and D (plain loads by its
+// 32 lanes) and counts as the stage's second arrival.
+// Shared memory: K 32K | V 32K | QdO[3] (Q 16K + dO 16K) | PdS[2] (P^T 16K +
+// dS^T 16K) | barriers | stats[3] (128 floats).
+constexpr int kQdStages = 3;
+constexpr int kSmemKV = 1024 + 2 * kTile + kQdStages * (2 * kTile64) + 2 * (2 * kTile128x64) +
+                        256 + kQdStages * 2 * kB64 * 4;
 
 __global__ void __launch_bounds__(kThreadsB, 1)
     attn_bwd_dkdv_tcgen05(const __grid_constant__ CUtensorMap tmKV128,
@@ -568,18 +579,19 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sK = smem;
   uint8_t* sV = smem + kTile;
-  uint8_t* sQdO = smem + 2 * kTile;                     // stage st: Q at +0, dO at +kTile64
-  uint8_t* sPdS = sQdO + 2 * (2 * kTile64);             // stage st: P^T at +0, dS^T at +16K
+  uint8_t* sQdO = smem + 2 * kTile;                     // stage q: Q at +0, dO at +kTile64
+  uint8_t* sPdS = sQdO + kQdStages * (2 * kTile64);     // stage st: P^T at +0, dS^T at +16K
   uint64_t* bars = reinterpret_cast<uint64_t*>(sPdS + 2 * (2 * kTile128x64));
   uint64_t* kv_full = bars + 0;
-  uint64_t* qd_full = bars + 1;   // [2]
-  uint64_t* qd_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* p_full = bars + 7;    // [2]
-  uint64_t* p_free = bars + 9;    // [2]
-  uint64_t* acc_done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
-  __shared__ __align__(16) float s_stat[kEwWarpsB * 64];
+  uint64_t* qd_full = bars + 1;                 // [kQdStages]
+  uint64_t* qd_empty = qd_full + kQdStages;     // [kQdStages]
+  uint64_t* s_full = qd_empty + kQdStages;      // [2]
+  uint64_t* p_full = s_full + 2;                // [2]
+  uint64_t* p_free = p_full + 2;                // [2]
+  uint64_t* acc_done = p_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_done + 1);
+  // stage q: LSE * log2(e) of the block's 64 queries at [0, 64), D at [64, 128)
+  float* s_stat = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb = static_cast<int>(blockIdx.x);  // early keys see the most queries: first
@@ -592,9 +604,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&qd_full[i], 1);
+    for (int i = 0; i < kQdStages; ++i) {
+      mbar_init(&qd_full[i], 2);  // the TMA transaction arrival + the staged statistics
       mbar_init(&qd_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], kEwWarpsB);
       mbar_init(&p_free[i], 1);
@@ -615,8 +629,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   const uint32_t tdV = tmem + 256, tdK = tmem + 384;
 
   if (warp == 0) {
+    const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.s;
+    bool ok = true;
     if (lane == 0) {
-      bool ok = true;
       tma_prefetch_desc(&tmKV128);
       tma_prefetch_desc(&tmQ64);
       tma_prefetch_desc(&tmdO64);
@@ -625,19 +640,30 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       tma_load_2d(sK + kHalf, &tmKV128, kv_full, a.h + head * kD + 64, row0 + k0);
       tma_load_2d(sV, &tmKV128, kv_full, 2 * a.h + head * kD, row0 + k0);
       tma_load_2d(sV + kHalf, &tmKV128, kv_full, 2 * a.h + head * kD + 64, row0 + k0);
-      for (int it = 0; it < n_qb && ok; ++it) {
-        const int st = it & 1;
-        if (!(ok = mbar_wait(&qd_empty[st], ((static_cast<uint32_t>(it) >> 1) & 1u) ^ 1u,
-                             a.status, kStatusAttnTimeout)))
-          break;
-        mbar_arrive_expect_tx(&qd_full[st], 2 * kTile64);
-        uint8_t* dst = sQdO + st * (2 * kTile64);
-        const int qrow = row0 + (i0 + it) * kB64;
-        tma_load_2d(dst, &tmQ64, &qd_full[st], head * kD, qrow);
-        tma_load_2d(dst + kHalf64, &tmQ64, &qd_full[st], head * kD + 64, qrow);
-        tma_load_2d(dst + kTile64, &tmdO64, &qd_full[st], head * kD, qrow);
-        tma_load_2d(dst + kTile64 + kHalf64, &tmdO64, &qd_full[st], head * kD + 64, qrow);
+    }
+    for (int it = 0; it < n_qb && ok; ++it) {
+      const int qs = it % kQdStages;
+      const uint32_t qph = static_cast<uint32_t>(it / kQdStages) & 1u;
+      if (!(ok = mbar_wait(&qd_empty[qs], qph ^ 1u, a.status, kStatusAttnTimeout))) break;
+      const int q0 = (i0 + it) * kB64;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&qd_full[qs], 2 * kTile64);
+        uint8_t* dst = sQdO + qs * (2 * kTile64);
+        const int qrow = row0 + q0;
+        tma_load_2d(dst, &tmQ64, &qd_full[qs], head * kD, qrow);
+        tma_load_2d(dst + kHalf64, &tmQ64, &qd_full[qs], head * kD + 64, qrow);
+        tma_load_2d(dst + kTile64, &tmdO64, &qd_full[qs], head * kD, qrow);
+        tma_load_2d(dst + kTile64 + kHalf64, &tmdO64, &qd_full[qs], head * kD + 64, qrow);
       }
+      float* st_dst = s_stat + qs * (2 * kB64);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int qq = min(q0 + e * 32 + lane, a.s - 1);
+        st_dst[e * 32 + lane] = a.lse[stat + qq] * kLog2eA;
+        st_dst[kB64 + e * 32 + lane] = a.dsum[stat + qq];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qd_full[qs]);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -647,11 +673,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       bool ok = mbar_wait(kv_full, 0, a.status, kStatusAttnTimeout);
       auto issue_sp = [&](int it) -> bool {
         const int st = it & 1;
-        if (!mbar_wait(&qd_full[st], (static_cast<uint32_t>(it) >> 1) & 1u, a.status,
+        const int qs = it % kQdStages;
+        if (!mbar_wait(&qd_full[qs], static_cast<uint32_t>(it / kQdStages) & 1u, a.status,
                        kStatusAttnTimeout))
           return false;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sQdO + st * (2 * kTile64));
+        const uint32_t q_addr = smem_u32(sQdO + qs * (2 * kTile64));
         const uint32_t do_addr = q_addr + kTile64;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
@@ -673,9 +700,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                              kStatusAttnTimeout)))
           break;
         tc_fence_after();
+        const int qs = it % kQdStages;
         const uint32_t pt_addr = smem_u32(sPdS + st * (2 * kTile128x64));
         const uint32_t dst_addr = pt_addr + kTile128x64;
-        const uint32_t q_addr = smem_u32(sQdO + st * (2 * kTile64));
+        const uint32_t q_addr = smem_u32(sQdO + qs * (2 * kTile64));
         const uint32_t do_addr = q_addr + kTile64;
 #pragma unroll
         for (int kk = 0; kk < kB64 / 16; ++kk) {
@@ -685,7 +713,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           umma_bf16(tdK, sw128_desc(dst_addr + kk * 32, 16, 1024),
                     sw128_desc(q_addr + kk * 2048, kHalf64, 1024), kIdAcc, acc);
         }
-        umma_commit(&qd_empty[st]);
+        umma_commit(&qd_empty[qs]);
         umma_commit(&p_free[st]);
       }
       if (ok) umma_commit(acc_done);
@@ -697,30 +725,24 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     const int r = quarter * 32 + lane;
     const int key = k0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.s;
-    // The warp's 32 queries' LSE * log2(e) and D, staged once per block in a
-    // per-warp shared-memory slot (read back as broadcasts).
-    float* wstat = s_stat + (warp - 4) * 64;
     bool ok = true;
     for (int it = 0; it < n_qb && ok; ++it) {
       const int st = it & 1;
+      const int qs = it % kQdStages;
       const int q0 = (i0 + it) * kB64;
-      {
-        const int qs = min(q0 + c + lane, a.s - 1);
-        const float l2 = a.lse[stat + qs] * kLog2eA;
-        const float dq = a.dsum[stat + qs];
-        __syncwarp();  // the previous block's reads of the slot are done
-        wstat[lane] = l2;
-        wstat[32 + lane] = dq;
-        __syncwarp();
-      }
       if (!(ok = mbar_wait(&s_full[st], (static_cast<uint32_t>(it) >> 1) & 1u, a.status,
+                           kStatusAttnTimeout)))
+        break;
+      // The block's statistics were staged before its Q / dO stage completed;
+      // the stage cannot be refilled before this block's products are done.
+      if (!(ok = mbar_wait(&qd_full[qs], static_cast<uint32_t>(it / kQdStages) & 1u, a.status,
                            kStatusAttnTimeout)))
         break;
       if (it >= 2 && !(ok = mbar_wait(&p_free[st], ((static_cast<uint32_t>(it) >> 1) - 1u) & 1u,
                                       a.status, kStatusAttnTimeout)))
         break;
       tc_fence_after();
+      const float* wstat = s_stat + qs * (2 * kB64) + c;
       // query q = q0 + c + i is visible to this key when key <= q (causal)
       // and q < s: lo <= i < hi
       const int lo = (a.causal ? max(key - q0, 0) : 0) - c;
@@ -734,7 +756,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(wstat + i);
-        const float4 d4 = *reinterpret_cast<const float4*>(wstat + 32 + i);
+        const float4 d4 = *reinterpret_cast<const float4*>(wstat + kB64 + i);
         const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
         const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
         float p[4];

@@ -130,3 +130,32 @@ def test_linear_config3_full_size_sampled():
             else:
                 assert torch.equal(Y, first), f"{mode}: t={t} differs from t=1"
             del Y
+
+
+UNCOMMON = {("col", 3): (200, 320, 960), ("col", 5): (200, 320, 960), ("col", 64): (200, 320, 512),
+            ("row", 3): (200, 1536, 320), ("row", 5): (200, 1280, 320), ("row", 64): (200, 4096, 320)}
+
+
+@pytest.mark.parametrize("t", [3, 5, 64])
+@pytest.mark.parametrize("mode", ["col", "row"])
+def test_linear_uncommon_shard_counts(mode, t):
+    """Shard counts that are not powers of two, and the largest allowed (64,
+    8 columns per shard for the column split: the narrowest shard-aligned
+    tiles).  Integer-valued inputs: exact."""
+    M, K, N = UNCOMMON[(mode, t)]
+    X, W = integer_tensor((M, K), -3, 3, 14), integer_tensor((K, N), -3, 3, 15)
+    b = integer_tensor((N,), -8, 8, 16)
+    Xc, Wc, bc = cuda(X), cuda(W), cuda(b)
+    Y = run(mode, Xc, Wc, bc, t, out_dtype=torch.float32)
+    assert np.array_equal(to64(Y), O.linear(X, W, b))
+    if mode == "col":
+        w = N // t
+        for i in (0, t // 2, t - 1):
+            part = run("col", Xc, Wc, bc, t, shard=i, out_dtype=torch.float32)
+            assert torch.equal(part, Y[:, i * w:(i + 1) * w]), i
+    else:
+        parts = [run("row", Xc, Wc, bc, t, shard=i, out_dtype=torch.float32) for i in range(t)]
+        total = parts[0].clone()
+        for p in parts[1:]:
+            total += p
+        assert torch.equal(total, Y)

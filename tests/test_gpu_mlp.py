@@ -124,3 +124,12 @@ def test_mlp_config5_sampled():
     check(out["dbA"][u], bw_units["dbA"], "dbA", "bf16")
     check(out["dB"][u], bw_units["dB"], "dB rows", "bf16")
     check(out["dbB"], bw_units["dbB"], "dbB", "bf16")
+
+
+@pytest.mark.parametrize("t", [3, 64])
+def test_mlp_uncommon_shard_counts(t):
+    """t = 3 (f / t = 256) and t = 64 (f / t = 8, one 8-column group per shard)."""
+    wl = Workload(93, "uncommon t", b=1, s=136, h=128, f=768 if t == 3 else 512, t=t,
+                  w_std=0.05, bias_std=0.05)
+    inp = make_mlp_inputs(wl)
+    compare_full(gpu_mlp(inp, t), inp, "bf16")
