@@ -141,6 +141,64 @@ class ClockSampler:
                 "samples": len(inside)}
 
 
+# ------------------------------------------------------------------- ranks
+class Ranks:
+    """The job's ranks: one process per GPU, each running an independent
+    replica of the step (no collective on the data path).  torch.distributed
+    carries only the barriers around the timed regions and the max over
+    ranks of each timing.  A single process needs no process group."""
+
+    def __init__(self, rank: int = 0, world: int = 1, local_rank: int = 0, dist=None,
+                 backend: str = ""):
+        self.rank, self.world, self.local_rank = rank, world, local_rank
+        self.dist, self.backend = dist, backend
+
+    @classmethod
+    def from_env(cls, backend: str = "nccl", timeout_s: int = 600):
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        if world == 1:
+            return cls(rank, world, local_rank)
+        import datetime
+
+        import torch.distributed as tdist
+        kw = {"timeout": datetime.timedelta(seconds=timeout_s)}
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+            kw["device_id"] = torch.device("cuda", local_rank)
+        tdist.init_process_group(backend, **kw)
+        return cls(rank, world, local_rank, tdist, backend)
+
+    def barrier(self):
+        if self.dist is None:
+            return
+        if self.backend == "nccl":
+            self.dist.barrier(device_ids=[self.local_rank])
+        else:
+            self.dist.barrier()
+
+    def max(self, x):
+        """The maximum of x over the ranks (None stays None on every rank)."""
+        if self.dist is None or x is None:
+            return x
+        dev = torch.device("cuda", self.local_rank) if self.backend == "nccl" else "cpu"
+        t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.destroy_process_group()
+
+
+def job_rate(units_per_rank: float, world: int, ms_max: float, steps: int) -> float:
+    """Whole-job throughput: the units every rank processed in `steps` steps,
+    divided by the slowest rank's time (weak scaling: each rank's work is
+    fixed as the job grows)."""
+    return world * units_per_rank / (ms_max / steps * 1e-3)
+
+
 # ------------------------------------------------------------- libtp arm
 class LayerStep:
     """Device buffers and the four libtp calls of one layer step."""
@@ -376,18 +434,16 @@ def e2e_pipelined(st, steps, stream, barrier):
     return ms, h2d, d2h
 
 
-def run_libtp(args, rank, world, local_rank, dist):
+def run_libtp(args, ranks: Ranks):
     from megatron_tensor_transformer_logical_b200 import binding as L
+    rank, world, local_rank = ranks.rank, ranks.world, ranks.local_rank
+    barrier = ranks.barrier
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = WORKLOADS[args.workload]
     st = LayerStep(wl, dev)
     stream = torch.cuda.current_stream()
     fl = layer_flops(wl.b, wl.s, wl.h, wl.f, wl.heads)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier(device_ids=[local_rank])
 
     for _ in range(args.warmup):
         st.step()
@@ -459,23 +515,18 @@ def run_libtp(args, rank, world, local_rank, dist):
         e2e_ms, h2d, d2h = e2e_pipelined(st, args.steps, stream, barrier)
     L.tp_device_status()
 
-    def maxall(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    maxall = ranks.max
 
     ms, mlp_ms, mlp_rec_ms = maxall(ms), maxall(mlp_ms), maxall(mlp_rec_ms)
     block_ms = maxall(block_ms)
-    vocab_ms = maxall(vocab_ms) if vocab_ms is not None else None
-    e2e_ms = maxall(e2e_ms) if e2e_ms is not None else None
+    vocab_ms = maxall(vocab_ms)
+    e2e_ms = maxall(e2e_ms)
     if rank != 0:
         return None
 
     per_step = ms / args.steps
-    tflops = world * fl["total"] / (per_step * 1e-3) / 1e12
-    tokens = world * wl.M / (per_step * 1e-3)
+    tflops = job_rate(fl["total"], world, ms, args.steps) / 1e12
+    tokens = job_rate(wl.M, world, ms, args.steps)
     peaks, peak_src = load_peaks()
     g = prof["gemm_tcgen05"]
     achieved = g["flops"] / (g["total_ms"] * 1e-3) / 1e12 if g["total_ms"] > 0 else 0.0
@@ -550,7 +601,7 @@ def run_libtp(args, rank, world, local_rank, dist):
     if vocab_ms is not None:
         out["vocab_fwd_bwd"] = vocab_report(vs, args.steps, vocab_ms, vocab_records, peaks, world)
     if e2e_ms is not None:
-        out["e2e"] = {"value": round(world * fl["total"] / (e2e_ms / args.steps * 1e-3) / 1e12, 2),
+        out["e2e"] = {"value": round(job_rate(fl["total"], world, e2e_ms, args.steps) / 1e12, 2),
                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                       "ms_per_step": round(e2e_ms / args.steps, 4)}
     if not args.no_cpu_baseline:
@@ -649,27 +700,20 @@ def main():
     if args.warmup < 3 and args.impl == "libtp":
         ap.error("--warmup must be at least 3")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as tdist
-        if args.impl == "libtp":
-            torch.cuda.set_device(local_rank)
-            tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                     device_id=torch.device("cuda", local_rank))
-            dist = tdist
     if args.impl == "reference":
-        out = run_reference(args, rank, world)
-    else:
-        out = run_libtp(args, rank, world, local_rank, dist)
-    if out is not None:
-        print(json.dumps(out), flush=True)
-    if dist is not None:
-        dist.destroy_process_group()
+        # Rank 0 alone times the oracle; the other ranks exit without work.
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        out = run_reference(args, int(os.environ.get("RANK", "0")), world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    ranks = Ranks.from_env("nccl")
+    try:
+        out = run_libtp(args, ranks)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        ranks.close()
 
 
 if __name__ == "__main__":

@@ -60,6 +60,15 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz;
+// relative error about 2^-22, subnormal results flushed to zero, 2^-inf = 0).
+// The probabilities it produces are rounded to fp16 right after.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 t = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&t);
@@ -249,7 +258,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         float v[32];
         tmem_ld32(tS[st] + lane_off + c, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = exp2f(fmaf(v[i], a.scale_log2, -mx));
+        for (int i = 0; i < 32; ++i) v[i] = ex2_approx(fmaf(v[i], a.scale_log2, -mx));
         if (vis < c + 32) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = (c + i < vis) ? v[i] : 0.0f;
@@ -512,8 +521,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
-        float p0 = exp2f(fmaf(sv[i], a.scale_log2, -lse2));
-        float p1 = exp2f(fmaf(sv[i + 1], a.scale_log2, -lse2));
+        float p0 = ex2_approx(fmaf(sv[i], a.scale_log2, -lse2));
+        float p1 = ex2_approx(fmaf(sv[i + 1], a.scale_log2, -lse2));
         p0 = (i < vis) ? p0 : 0.0f;
         p1 = (i + 1 < vis) ? p1 : 0.0f;
         pk[i >> 1] = pack_half2(p0 * (pv[i] - dd), p1 * (pv[i + 1] - dd));
@@ -762,7 +771,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         float p[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          p[e] = exp2f(fmaf(sv[i + e], a.scale_log2, -lv[e]));
+          p[e] = ex2_approx(fmaf(sv[i + e], a.scale_log2, -lv[e]));
           p[e] = (i + e >= lo && i + e < hi) ? p[e] : 0.0f;
         }
         pk[i >> 1] = pack_half2(p[0], p[1]);
