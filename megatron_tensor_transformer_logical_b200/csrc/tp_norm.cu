@@ -4,16 +4,15 @@
 // LayerNorm is replicated, not partitioned: every logical shard sees the
 // whole normalised row.
 //
-// Forward: one CTA of 512 threads per row; the row (h <= 16384, h % 8 == 0)
-// stays in registers; mean, then the centred variance (two passes over the
-// registers), both in fp32 with block reductions; Y written in the input
-// type, mean and rstd saved in fp32.
-// Backward: a CTA per group of rows; per row g = dY * gamma,
+// Forward: one CTA of 256 threads per row (h <= 16384, h % 8 == 0); the
+// shifted sums of the row give mean and variance in one block reduction
+// (fp32), a second pass over the row writes Y in the input type; mean and
+// rstd are saved in fp32.
+// Backward: dX by one CTA per row, two passes over it (g = dY * gamma;
 //   dX = rstd * (g - mean(g) - xhat * mean(g * xhat)) (+ dR, the residual
-// path's gradient, when given); dgamma / dbeta partial column sums stay in
-// shared memory across the CTA's rows and are summed over CTAs by a second,
-// deterministic pass.  HBM-bound: each element of X and dY is read once,
-// dX written once.
+// path's gradient, when given)); dgamma / dbeta by a column kernel over row
+// chunks of 32 (X and dY read a second time) whose chunk partials a third
+// kernel sums in chunk order (deterministic).  HBM-bound.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -22,9 +21,7 @@
 namespace tp {
 namespace {
 
-constexpr int kLnThreads = 512;
-constexpr int kLnChunks = 4;  // chunks of 8 elements per thread: h <= 512 * 4 * 8 = 16384
-constexpr int kLnMaxH = kLnThreads * kLnChunks * 8;
+constexpr int kLnMaxH = 16384;  // the widest row the library accepts
 
 template <bool F32>
 __device__ __forceinline__ void load8(const void* base, long long off, float* v) {
@@ -62,67 +59,76 @@ __device__ __forceinline__ void store8(void* base, long long off, const float* v
   }
 }
 
-// Sum over the 512 threads of the CTA (all threads get the result).
-__device__ __forceinline__ float block_sum(float v, float* red) {
+// dX of one row per CTA of 256 threads: with xhat = (x - mean) * rstd and
+// g = dY * gamma, dX = rstd * (g - mean(g) - xhat * mean(g * xhat)) (+ dR).
+// Two passes over the row: the first forms both row sums (one block
+// reduction), the second re-reads X and dY (from L2) and writes dX, so a
+// thread holds no row data in registers and several rows run per SM.
+constexpr int kLnBwdThreads = 256;
+
+__device__ __forceinline__ float2 block_sum2(float a, float b, float2* red) {
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
+  for (int s = 16; s > 0; s >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, s);
+    b += __shfl_xor_sync(0xffffffffu, b, s);
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __syncthreads();  // red is free (the previous reduction has been read)
-  if (lane == 0) red[warp] = v;
+  if (lane == 0) red[warp] = make_float2(a, b);
   __syncthreads();
-  float t = lane < kLnThreads / 32 ? red[lane] : 0.0f;
+  float2 t = lane < kLnBwdThreads / 32 ? red[lane] : make_float2(0.0f, 0.0f);
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) t += __shfl_xor_sync(0xffffffffu, t, s);  // every lane: the sum
+  for (int s = 16; s > 0; s >>= 1) {
+    t.x += __shfl_xor_sync(0xffffffffu, t.x, s);
+    t.y += __shfl_xor_sync(0xffffffffu, t.y, s);
+  }
   return t;
 }
 
+// Forward, one row per CTA of 256 threads, two passes over the row: the
+// first forms the sums of (x - K) and (x - K)^2 with K = the row's first
+// element (the shifted-data form of the variance: with K a sample of the row
+// the two sums do not cancel), one block reduction for both; the second pass
+// re-reads the row (from L2) and writes Y.  No row data stays in registers,
+// so several rows run per SM.
 template <bool F32>
-__global__ void __launch_bounds__(kLnThreads)
+__global__ void __launch_bounds__(kLnBwdThreads)
     layernorm_fwd_kernel(const void* X, const void* gamma, const void* beta, void* Y, float* mean,
                          float* rstd, int h, float eps) {
-  __shared__ float red[kLnThreads / 32];
+  __shared__ float2 red[kLnBwdThreads / 32];
   const long long row = blockIdx.x;
+  const long long base = row * h;
   const int nch = h / 8;
-  float x[kLnChunks][8];
-  float s = 0.0f;
+  const float K = F32 ? static_cast<const float*>(X)[base]
+                      : __bfloat162float(static_cast<const __nv_bfloat16*>(X)[base]);
+  float s1 = 0.0f, s2 = 0.0f;
+#pragma unroll 2
+  for (int ch = threadIdx.x; ch < nch; ch += kLnBwdThreads) {
+    float x[8];
+    load8<F32>(X, base + ch * 8, x);
 #pragma unroll
-  for (int k = 0; k < kLnChunks; ++k) {
-    const int ch = threadIdx.x + k * kLnThreads;
-    if (ch < nch) {
-      load8<F32>(X, row * h + ch * 8, x[k]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) s += x[k][i];
+    for (int i = 0; i < 8; ++i) {
+      const float d = x[i] - K;
+      s1 += d;
+      s2 += d * d;
     }
   }
-  const float mu = block_sum(s, red) / h;
-  float q = 0.0f;
+  const float2 m = block_sum2(s1, s2, red);
+  const float d1 = m.x / h;
+  const float mu = K + d1;
+  const float rs = rsqrtf(fmaxf(m.y / h - d1 * d1, 0.0f) + eps);
+#pragma unroll 2
+  for (int ch = threadIdx.x; ch < nch; ch += kLnBwdThreads) {
+    float x[8], g[8], b[8], y[8];
+    load8<F32>(X, base + ch * 8, x);
+    if (gamma != nullptr) load8<F32>(gamma, ch * 8, g);
+    if (beta != nullptr) load8<F32>(beta, ch * 8, b);
 #pragma unroll
-  for (int k = 0; k < kLnChunks; ++k) {
-    const int ch = threadIdx.x + k * kLnThreads;
-    if (ch < nch) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float d = x[k][i] - mu;
-        q += d * d;
-      }
+    for (int i = 0; i < 8; ++i) {
+      y[i] = (x[i] - mu) * rs;
+      if (gamma != nullptr) y[i] *= g[i];
+      if (beta != nullptr) y[i] += b[i];
     }
-  }
-  const float rs = rsqrtf(block_sum(q, red) / h + eps);
-#pragma unroll
-  for (int k = 0; k < kLnChunks; ++k) {
-    const int ch = threadIdx.x + k * kLnThreads;
-    if (ch < nch) {
-      float g[8], b[8], y[8];
-      if (gamma != nullptr) load8<F32>(gamma, ch * 8, g);
-      if (beta != nullptr) load8<F32>(beta, ch * 8, b);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        y[i] = (x[k][i] - mu) * rs;
-        if (gamma != nullptr) y[i] *= g[i];
-        if (beta != nullptr) y[i] += b[i];
-      }
-      store8<F32>(Y, row * h + ch * 8, y);
-    }
+    store8<F32>(Y, base + ch * 8, y);
   }
   if (threadIdx.x == 0) {
     if (mean != nullptr) mean[row] = mu;
@@ -130,69 +136,86 @@ __global__ void __launch_bounds__(kLnThreads)
   }
 }
 
-// Dynamic shared memory: dgamma and dbeta partials, 2 x h floats, laid out
-// [element i of a chunk][chunk] so that consecutive threads touch
-// consecutive words.
 template <bool F32>
-__global__ void __launch_bounds__(kLnThreads)
-    layernorm_bwd_kernel(const void* X, const void* gamma, const float* mean, const float* rstd,
-                         const void* dY, const void* dR, void* dX, float* part_g, float* part_b,
-                         int M, int h, int rows_per_cta) {
-  __shared__ float red[kLnThreads / 32];
-  extern __shared__ float sp[];
+__global__ void __launch_bounds__(kLnBwdThreads)
+    layernorm_bwd_dx_kernel(const void* X, const void* gamma, const float* mean,
+                            const float* rstd, const void* dY, const void* dR, void* dX, int h) {
+  __shared__ float2 red[kLnBwdThreads / 32];
+  const long long row = blockIdx.x;
+  const long long base = row * h;
   const int nch = h / 8;
-  float* sg = sp;      // [8][nch]
-  float* sb = sp + h;  // [8][nch]
-  for (int i = threadIdx.x; i < 2 * h; i += kLnThreads) sp[i] = 0.0f;
-  __syncthreads();
-  const int r0 = blockIdx.x * rows_per_cta;
-  const int r1 = min(r0 + rows_per_cta, M);
-  for (int r = r0; r < r1; ++r) {
-    const long long base = static_cast<long long>(r) * h;
-    const float mu = mean[r], rs = rstd[r];
-    float xh[kLnChunks][8], g[kLnChunks][8];
-    float s1 = 0.0f, s2 = 0.0f;
+  const float mu = mean[row], rs = rstd[row];
+  float s1 = 0.0f, s2 = 0.0f;
+#pragma unroll 2
+  for (int ch = threadIdx.x; ch < nch; ch += kLnBwdThreads) {
+    float x[8], dy[8], gm[8];
+    load8<F32>(X, base + ch * 8, x);
+    load8<F32>(dY, base + ch * 8, dy);
+    if (gamma != nullptr) load8<F32>(gamma, ch * 8, gm);
 #pragma unroll
-    for (int k = 0; k < kLnChunks; ++k) {
-      const int ch = threadIdx.x + k * kLnThreads;
-      if (ch < nch) {
-        float dy[8], gm[8];
-        load8<F32>(X, base + ch * 8, xh[k]);
-        load8<F32>(dY, base + ch * 8, dy);
-        if (gamma != nullptr) load8<F32>(gamma, ch * 8, gm);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          xh[k][i] = (xh[k][i] - mu) * rs;
-          g[k][i] = gamma != nullptr ? dy[i] * gm[i] : dy[i];
-          s1 += g[k][i];
-          s2 += g[k][i] * xh[k][i];
-          sg[i * nch + ch] += dy[i] * xh[k][i];
-          sb[i * nch + ch] += dy[i];
-        }
-      }
-    }
-    const float m1 = block_sum(s1, red) / h;
-    const float m2 = block_sum(s2, red) / h;
-#pragma unroll
-    for (int k = 0; k < kLnChunks; ++k) {
-      const int ch = threadIdx.x + k * kLnThreads;
-      if (ch < nch) {
-        float dx[8], dr[8];
-        if (dR != nullptr) load8<F32>(dR, base + ch * 8, dr);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          dx[i] = rs * (g[k][i] - m1 - xh[k][i] * m2);
-          if (dR != nullptr) dx[i] += dr[i];
-        }
-        store8<F32>(dX, base + ch * 8, dx);
-      }
+    for (int i = 0; i < 8; ++i) {
+      const float g = gamma != nullptr ? dy[i] * gm[i] : dy[i];
+      s1 += g;
+      s2 += g * ((x[i] - mu) * rs);
     }
   }
-  __syncthreads();
-  for (int c = threadIdx.x; c < h; c += kLnThreads) {
-    const long long off = static_cast<long long>(blockIdx.x) * h + c;
-    part_g[off] = sg[(c & 7) * nch + (c >> 3)];
-    part_b[off] = sb[(c & 7) * nch + (c >> 3)];
+  const float2 m = block_sum2(s1, s2, red);
+  const float m1 = m.x / h, m2 = m.y / h;
+#pragma unroll 2
+  for (int ch = threadIdx.x; ch < nch; ch += kLnBwdThreads) {
+    float x[8], dy[8], gm[8], dr[8], dx[8];
+    load8<F32>(X, base + ch * 8, x);
+    load8<F32>(dY, base + ch * 8, dy);
+    if (gamma != nullptr) load8<F32>(gamma, ch * 8, gm);
+    if (dR != nullptr) load8<F32>(dR, base + ch * 8, dr);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float g = gamma != nullptr ? dy[i] * gm[i] : dy[i];
+      dx[i] = rs * (g - m1 - ((x[i] - mu) * rs) * m2);
+      if (dR != nullptr) dx[i] += dr[i];
+    }
+    store8<F32>(dX, base + ch * 8, dx);
+  }
+}
+
+// dgamma / dbeta partial column sums: CTA (column block, row chunk), each
+// thread 8 columns summed over the chunk's rows in row order; the chunk
+// totals are summed in chunk order by column_total_kernel (deterministic).
+constexpr int kLnColThreads = 128;
+constexpr int kLnRowsPerChunk = 32;
+
+template <bool F32>
+__global__ void __launch_bounds__(kLnColThreads)
+    layernorm_bwd_cols_kernel(const void* X, const float* mean, const float* rstd,
+                              const void* dY, float* part_g, float* part_b, int M, int h) {
+  const int c8 = blockIdx.x * kLnColThreads + threadIdx.x;  // chunk of 8 columns
+  if (c8 * 8 >= h) return;
+  const int r0 = blockIdx.y * kLnRowsPerChunk;
+  const int r1 = min(r0 + kLnRowsPerChunk, M);
+  float ag[8], ab[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ag[i] = ab[i] = 0.0f;
+#pragma unroll 4
+  for (int r = r0; r < r1; ++r) {
+    float x[8], dy[8];
+    const long long off = static_cast<long long>(r) * h + c8 * 8;
+    load8<F32>(X, off, x);
+    load8<F32>(dY, off, dy);
+    const float mu = mean[r], rs = rstd[r];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      ag[i] += dy[i] * ((x[i] - mu) * rs);
+      ab[i] += dy[i];
+    }
+  }
+  const long long o = static_cast<long long>(blockIdx.y) * h + c8 * 8;
+  if (part_g != nullptr) {
+    reinterpret_cast<float4*>(part_g + o)[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
+    reinterpret_cast<float4*>(part_g + o)[1] = make_float4(ag[4], ag[5], ag[6], ag[7]);
+  }
+  if (part_b != nullptr) {
+    reinterpret_cast<float4*>(part_b + o)[0] = make_float4(ab[0], ab[1], ab[2], ab[3]);
+    reinterpret_cast<float4*>(part_b + o)[1] = make_float4(ab[4], ab[5], ab[6], ab[7]);
   }
 }
 
@@ -208,9 +231,7 @@ __global__ void column_total_kernel(const float* part, int parts, int h, void* o
     static_cast<__nv_bfloat16*>(out)[c] = __float2bfloat16_rn(s);
 }
 
-constexpr int kLnMaxParts = 296;  // CTAs of the backward: about two per SM
-
-int ln_parts(int64_t M) { return static_cast<int>(M < kLnMaxParts ? M : kLnMaxParts); }
+int ln_parts(int64_t M) { return static_cast<int>((M + kLnRowsPerChunk - 1) / kLnRowsPerChunk); }
 
 }  // namespace
 
@@ -229,10 +250,10 @@ tp_status launch_layernorm_fwd(const void* X, const void* gamma, const void* bet
     return fail(TP_ERR_UNSUPPORTED, "layernorm: h must be a multiple of 8 and at most 16384");
   LaunchScope scope(TP_KIND_REDUCE, 0.0, (f32 ? 4.0 : 2.0) * 2.0 * double(M) * h, stream);
   if (f32)
-    layernorm_fwd_kernel<true><<<static_cast<unsigned>(M), kLnThreads, 0, stream>>>(
+    layernorm_fwd_kernel<true><<<static_cast<unsigned>(M), kLnBwdThreads, 0, stream>>>(
         X, gamma, beta, Y, mean, rstd, static_cast<int>(h), eps);
   else
-    layernorm_fwd_kernel<false><<<static_cast<unsigned>(M), kLnThreads, 0, stream>>>(
+    layernorm_fwd_kernel<false><<<static_cast<unsigned>(M), kLnBwdThreads, 0, stream>>>(
         X, gamma, beta, Y, mean, rstd, static_cast<int>(h), eps);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "layernorm_fwd launch");
@@ -246,37 +267,46 @@ tp_status launch_layernorm_bwd(const void* X, const void* gamma, const float* me
   if (M <= 0) return TP_OK;
   if (h <= 0 || h % 8 != 0 || h > kLnMaxH)
     return fail(TP_ERR_UNSUPPORTED, "layernorm: h must be a multiple of 8 and at most 16384");
+  if (M > 0x7fffffffLL) return fail(TP_ERR_SHAPE, "layernorm: too many rows");
   const int parts = ln_parts(M);
-  const int rows_per = static_cast<int>((M + parts - 1) / parts);
-  const int grid = static_cast<int>((M + rows_per - 1) / rows_per);
-  float* part_g = static_cast<float*>(scratch);
-  float* part_b = part_g + static_cast<size_t>(grid) * h;
-  const int smem = static_cast<int>(2 * h * sizeof(float));
-  cudaError_t e0 = cudaFuncSetAttribute(
-      f32 ? layernorm_bwd_kernel<true> : layernorm_bwd_kernel<false>,
-      cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e0 != cudaSuccess) return cuda_fail(e0, "layernorm_bwd smem attribute");
-  LaunchScope scope(TP_KIND_REDUCE, 0.0, (f32 ? 4.0 : 2.0) * 3.0 * double(M) * h, stream, 3);
+  const bool cols = dgamma != nullptr || dbeta != nullptr;
+  float* part_g = dgamma != nullptr ? static_cast<float*>(scratch) : nullptr;
+  float* part_b = dbeta != nullptr ? static_cast<float*>(scratch) + static_cast<size_t>(parts) * h
+                                   : nullptr;
+  const double es = f32 ? 4.0 : 2.0;
+  const double bytes = es * double(M) * h * (dR != nullptr ? 4.0 : 3.0) +
+                       (cols ? es * 2.0 * double(M) * h + 8.0 * parts * h : 0.0);
+  LaunchScope scope(TP_KIND_REDUCE, 0.0, bytes, stream, cols ? 2 + (dgamma != nullptr) +
+                                                                   (dbeta != nullptr) : 1);
+  const int ih = static_cast<int>(h), im = static_cast<int>(M);
   if (f32)
-    layernorm_bwd_kernel<true><<<grid, kLnThreads, smem, stream>>>(
-        X, gamma, mean, rstd, dY, dR, dX, part_g, part_b, static_cast<int>(M), static_cast<int>(h),
-        rows_per);
+    layernorm_bwd_dx_kernel<true><<<static_cast<unsigned>(M), kLnBwdThreads, 0, stream>>>(
+        X, gamma, mean, rstd, dY, dR, dX, ih);
   else
-    layernorm_bwd_kernel<false><<<grid, kLnThreads, smem, stream>>>(
-        X, gamma, mean, rstd, dY, dR, dX, part_g, part_b, static_cast<int>(M), static_cast<int>(h),
-        rows_per);
-  const unsigned cg = static_cast<unsigned>((h + 255) / 256);
-  if (dgamma != nullptr) {
+    layernorm_bwd_dx_kernel<false><<<static_cast<unsigned>(M), kLnBwdThreads, 0, stream>>>(
+        X, gamma, mean, rstd, dY, dR, dX, ih);
+  if (cols) {
+    dim3 grid(static_cast<unsigned>((h / 8 + kLnColThreads - 1) / kLnColThreads),
+              static_cast<unsigned>(parts));
     if (f32)
-      column_total_kernel<true><<<cg, 256, 0, stream>>>(part_g, grid, static_cast<int>(h), dgamma);
+      layernorm_bwd_cols_kernel<true><<<grid, kLnColThreads, 0, stream>>>(
+          X, mean, rstd, dY, part_g, part_b, im, ih);
     else
-      column_total_kernel<false><<<cg, 256, 0, stream>>>(part_g, grid, static_cast<int>(h), dgamma);
-  }
-  if (dbeta != nullptr) {
-    if (f32)
-      column_total_kernel<true><<<cg, 256, 0, stream>>>(part_b, grid, static_cast<int>(h), dbeta);
-    else
-      column_total_kernel<false><<<cg, 256, 0, stream>>>(part_b, grid, static_cast<int>(h), dbeta);
+      layernorm_bwd_cols_kernel<false><<<grid, kLnColThreads, 0, stream>>>(
+          X, mean, rstd, dY, part_g, part_b, im, ih);
+    const unsigned cg = static_cast<unsigned>((h + 255) / 256);
+    if (dgamma != nullptr) {
+      if (f32)
+        column_total_kernel<true><<<cg, 256, 0, stream>>>(part_g, parts, ih, dgamma);
+      else
+        column_total_kernel<false><<<cg, 256, 0, stream>>>(part_g, parts, ih, dgamma);
+    }
+    if (dbeta != nullptr) {
+      if (f32)
+        column_total_kernel<true><<<cg, 256, 0, stream>>>(part_b, parts, ih, dbeta);
+      else
+        column_total_kernel<false><<<cg, 256, 0, stream>>>(part_b, parts, ih, dbeta);
+    }
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "layernorm_bwd launch");

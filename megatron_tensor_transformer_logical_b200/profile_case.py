@@ -10,6 +10,8 @@ Cases (175B-shaped layer unless noted; bf16, t = 8):
   attn_fwd    tp_attn_fwd    (QKV GEMM, attention core, Wo GEMM)
   attn_bwd    tp_attn_bwd
   small_gemm  tp_linear_col  X[1024,4096] @ W[4096,8192] (a quick case)
+  block       tp_block_fwd + tp_block_bwd: LayerNorm + residual around the attention
+              and the MLP of the 175B-shaped layer (gamma 1, beta 0)
   vocab_step  the tied vocabulary-parallel embedding + cross-entropy, forward and
               backward on the seeded vocabulary workload (M=2048, h=12288,
               V=51200, t=8, Zipf token ids): embedding gather, logits
@@ -75,6 +77,28 @@ def make_case(name: str):
         wsb = L.workspace(L.TP_OP_ATTN_BWD, M, h, 0, heads, t, L.TP_BF16)
         return lambda: L.tp_attn_bwd(X, Wqkv, Wo, QKV, O, LSE, dZ, dX, dWqkv, dWo, 1, M, heads, t,
                                      True, wsb)
+    if name == "block":
+        X, dX2 = _t((M, h), 1.0), _t((M, h), 1.0, seed=4)
+        ones, zeros = torch.ones(h, dtype=bf, device="cuda"), torch.zeros(h, dtype=bf, device="cuda")
+        w = {"ln1_g": ones, "ln1_b": zeros, "Wqkv": _t((h, 3 * h), 0.006, seed=1),
+             "Wo": _t((h, h), 0.006, seed=2), "ln2_g": ones, "ln2_b": zeros,
+             "A": _t((h, f), 0.006, seed=5), "B": _t((f, h), 0.006, seed=6)}
+        e = lambda *sh, dt=bf: torch.empty(*sh, dtype=dt, device="cuda")
+        f32 = torch.float32
+        sv = {"Xn1": e(M, h), "mean1": e(M, dt=f32), "rstd1": e(M, dt=f32),
+              "QKV": e(M, 3 * h, dt=torch.float16), "O": e(M, h), "LSE": e(1, heads, M, dt=f32),
+              "X1": e(M, h), "Xn2": e(M, h), "mean2": e(M, dt=f32), "rstd2": e(M, dt=f32),
+              "Y": e(M, f)}
+        g = {"dln1_g": e(h), "dln1_b": e(h), "dWqkv": e(h, 3 * h), "dWo": e(h, h),
+             "dln2_g": e(h), "dln2_b": e(h), "dA": e(h, f), "dB": e(f, h)}
+        X2, dX = e(M, h), e(M, h)
+        wsf = L.workspace(L.TP_OP_BLOCK_FWD, M, h, f, heads, t, L.TP_BF16)
+        wsb = L.workspace(L.TP_OP_BLOCK_BWD, M, h, f, heads, t, L.TP_BF16)
+
+        def block():
+            L.tp_block_fwd(X, w, X2, sv, 1, M, f, heads, t, 1e-5, wsf)
+            L.tp_block_bwd(X, w, sv, dX2, dX, g, 1, M, f, heads, t, 1e-5, wsb)
+        return block
     if name == "vocab_step":
         from .inputs import WORKLOADS, make_vocab_inputs
         wl = WORKLOADS[6]
