@@ -37,8 +37,10 @@ constexpr int kBM = 128;          // query rows per CTA
 constexpr int kBN = 128;          // keys per block
 constexpr int kTile = 128 * 128 * 2;  // one [128 x 128] fp16 tile: 32 KB
 constexpr int kHalf = kTile / 2;      // one 64-column half: 16 KB
-constexpr int kThreadsA = 256;
-constexpr int kSmemA = 1024 + 6 * kTile + 256;  // Q, K[2], V[2], P, barriers
+constexpr int kThreadsA = 384;
+// Q, K[2], V[2], P, barriers, then the softmax groups' exchange slots:
+// row maxima [2 blocks][2 groups][128 rows] and row sums [2 groups][128].
+constexpr int kSmemA = 1024 + 6 * kTile + 256 + (2 * 2 * 128 + 2 * 128) * 4;
 constexpr float kLog2eA = 1.4426950408889634f;
 constexpr float kLn2A = 0.69314718055994531f;
 
@@ -92,7 +94,11 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   uint64_t* s_full = bars + 9;   // [2]
   uint64_t* p_full = bars + 11;
   uint64_t* o_full = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* x_full = bars + 13;  // [2] both groups' row maxima of a block written
+  uint64_t* l_full = bars + 15;  // both groups' row sums written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  float* x_max = reinterpret_cast<float*>(smem + 6 * kTile + 256);  // [2][2][128]
+  float* x_sum = x_max + 2 * 2 * 128;                                // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (a.s + kBM - 1) / kBM;
@@ -112,8 +118,11 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
     }
-    mbar_init(p_full, 4);  // one arrival per softmax warp
+    mbar_init(p_full, 8);  // one arrival per softmax warp
     mbar_init(o_full, 1);
+    mbar_init(&x_full[0], 8);
+    mbar_init(&x_full[1], 8);
+    mbar_init(l_full, 8);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -198,16 +207,21 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     }
   } else if (warp >= 4) {
     // ----------------------------------------------------------- softmax
+    // Two groups of four warps: group g owns keys [64 g, 64 g + 64) of every
+    // block and output columns [64 g, 64 g + 64); the two halves of a row
+    // agree on its running maximum through shared memory once per block.
     const int quarter = warp & 3;
+    const int grp = (warp - 4) >> 2;
     const int r = quarter * 32 + lane;  // row within the tile = TMEM lane
     const int qrow = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    float o[kD];
+    const int kc0 = grp * 64;           // this group's first key column / output column
+    float o[kD / 2];
 #pragma unroll
-    for (int i = 0; i < kD; ++i) o[i] = 0.0f;
+    for (int i = 0; i < kD / 2; ++i) o[i] = 0.0f;
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
-    uint8_t* prow = sP + (r >> 3) * 1024 + (r & 7) * 128;  // row r in the SW128 layout
+    uint8_t* line = sP + (r >> 3) * 1024 + (r & 7) * 128 + grp * kHalf;  // row r, key half grp
     // Keys [0, limit) are visible to this row (causal: up to the row itself).
     const int limit = a.causal ? min(a.s, qrow + 1) : a.s;
     for (int j = 0; j < n_kb; ++j) {
@@ -216,14 +230,13 @@ __global__ void __launch_bounds__(kThreadsA, 1)
                            kStatusAttnTimeout)))
         break;
       tc_fence_after();
-      const int vis = limit - j * kBN;  // visible keys of this block: [0, vis)
-      // pass 1: row max of the raw scores (the scale is positive, so the max
-      // of the scaled scores is the scaled max)
-      float mraw = -INFINITY;
+      const int vis = limit - j * kBN - kc0;  // visible keys of this half: [0, vis)
+      // pass 1: the half-row max of the raw scores (the scale is positive)
+      float mloc = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kBN; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         float v[32];
-        tmem_ld32(tS[st] + lane_off + c, v);
+        tmem_ld32(tS[st] + lane_off + kc0 + c, v);
         if (vis < c + 32) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = (c + i < vis) ? v[i] : -INFINITY;
@@ -232,31 +245,40 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         for (int w = 16; w >= 1; w >>= 1)
 #pragma unroll
           for (int i = 0; i < w; ++i) v[i] = fmaxf(v[i], v[i + w]);
-        mraw = fmaxf(mraw, v[0]);
+        mloc = fmaxf(mloc, v[0]);
       }
+      // exchange the half-row maxima of block j (slot j & 1)
+      float* xs = x_max + st * 256;
+      xs[grp * 128 + r] = mloc;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&x_full[st]);
+      if (!(ok = mbar_wait(&x_full[st], static_cast<uint32_t>(j >> 1) & 1u, a.status,
+                           kStatusAttnTimeout)))
+        break;
+      const float mraw = fmaxf(mloc, xs[(grp ^ 1) * 128 + r]);
       const float mx = fmaxf(m_run, mraw * a.scale_log2);
       const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - mx);
       m_run = mx;
-      // fold in O_{j-1} (scaled at m_{j-1}) and rescale to m_j
+      // fold in this group's columns of O_{j-1} (scaled at m_{j-1}), rescale to m_j
       if (j > 0) {
         if (!(ok = mbar_wait(o_full, static_cast<uint32_t>(j - 1) & 1u, a.status,
                              kStatusAttnTimeout)))
           break;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kD; c += 32) {
+        for (int c = 0; c < kD / 2; c += 32) {
           float v[32];
-          tmem_ld32(tO + lane_off + c, v);
+          tmem_ld32(tO + lane_off + kc0 + c, v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[c + i] = (o[c + i] + v[i]) * alpha;
         }
       }
-      // pass 2: P = 2^(s * scale - m), row sum, fp16 into the P tile
+      // pass 2: P = 2^(s * scale - m) for this half, row sum, fp16 into the P tile
       float rs = 0.0f;
 #pragma unroll
-      for (int c = 0; c < kBN; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         float v[32];
-        tmem_ld32(tS[st] + lane_off + c, v);
+        tmem_ld32(tS[st] + lane_off + kc0 + c, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = ex2_approx(fmaf(v[i], a.scale_log2, -mx));
         if (vis < c + 32) {
@@ -272,11 +294,10 @@ __global__ void __launch_bounds__(kThreadsA, 1)
           for (int i = 0; i < w; ++i) v[i] += v[i + w];
         rs += v[0];
         // 32 keys = 64 bytes = four 16-byte chunks of the row's 128-byte line
-        // in the 64-key half c / 64; the chunk index is swizzled by (row & 7).
-        uint8_t* line = prow + (c >> 6) * kHalf;
+        // in this group's 64-key half; the chunk index is swizzled by (row & 7).
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int chunk = ((c & 63) >> 3) + q;
+          const int chunk = (c >> 3) + q;
           *reinterpret_cast<uint4*>(line + ((chunk ^ (r & 7)) << 4)) =
               make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
@@ -287,15 +308,23 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
+    // the row sum is the sum of the two halves' sums
+    if (ok) {
+      x_sum[grp * 128 + r] = l_run;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(l_full);
+      ok = mbar_wait(l_full, 0, a.status, kStatusAttnTimeout);
+    }
     if (ok && mbar_wait(o_full, static_cast<uint32_t>(n_kb - 1) & 1u, a.status,
                         kStatusAttnTimeout)) {
       tc_fence_after();
-      const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-      __nv_bfloat16* orow = a.out + static_cast<long long>(row0 + qrow) * a.h + head * kD;
+      const float l_tot = x_sum[r] + x_sum[128 + r];
+      const float inv = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
+      __nv_bfloat16* orow = a.out + static_cast<long long>(row0 + qrow) * a.h + head * kD + kc0;
 #pragma unroll
-      for (int c = 0; c < kD; c += 32) {
+      for (int c = 0; c < kD / 2; c += 32) {
         float v[32];
-        tmem_ld32(tO + lane_off + c, v);
+        tmem_ld32(tO + lane_off + kc0 + c, v);
         if (qrow < a.s) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -312,9 +341,9 @@ __global__ void __launch_bounds__(kThreadsA, 1)
           }
         }
       }
-      if (qrow < a.s)
+      if (qrow < a.s && grp == 0)
         a.lse[(static_cast<long long>(bi) * a.heads + head) * a.s + qrow] =
-            (m_run + log2f(l_run)) * kLn2A;
+            (m_run + log2f(l_tot)) * kLn2A;
     }
   }
 
