@@ -278,6 +278,38 @@ class LayerStep:
     def outputs(self):
         return (self.Za, self.Zm, self.dXa, self.dXm)
 
+    def make_library_gemms(self, dev):
+        """The step's twelve GEMMs as plain torch.matmul calls (cuBLAS) with
+        the same shapes and operand layouts, no epilogues: a library yardstick
+        for the tcgen05 GEMMs, not part of the step."""
+        wl = self.wl
+        M, h, f = wl.M, wl.h, wl.f
+        e = lambda *sh: torch.empty(*sh, dtype=torch.bfloat16, device=dev)
+        self.lib_dqkv = e(M, 3 * h)
+        self.lib_out = {"qkv": e(M, 3 * h), "mh": e(M, h), "hh": e(h, h), "h3h": e(h, 3 * h),
+                        "mf": e(M, f), "fh": e(f, h), "hf": e(h, f)}
+        flops = 0.0
+        for (a, b, c) in ((M, 3 * h, h), (M, h, h), (M, h, h), (h, h, M), (h, 3 * h, M),
+                          (M, h, 3 * h), (M, f, h), (M, h, f), (M, f, h), (f, h, M), (h, f, M),
+                          (M, h, f)):
+            flops += 2.0 * a * b * c
+        self.lib_flops = flops
+
+    def library_gemms(self):
+        o, X, dZ, Y = self.lib_out, self.X, self.dZ, self.Y
+        torch.matmul(X, self.Wqkv, out=o["qkv"])                 # QKV
+        torch.matmul(self.O, self.Wo, out=o["mh"])               # Z = O Wo
+        torch.matmul(dZ, self.Wo.t(), out=o["mh"])               # dO
+        torch.matmul(self.O.t(), dZ, out=o["hh"])                # dWo
+        torch.matmul(X.t(), self.lib_dqkv, out=o["h3h"])         # dWqkv
+        torch.matmul(self.lib_dqkv, self.Wqkv.t(), out=o["mh"])  # dX (attention)
+        torch.matmul(X, self.A, out=o["mf"])                     # Y = X A
+        torch.matmul(Y, self.B, out=o["mh"])                     # Z = H B
+        torch.matmul(dZ, self.B.t(), out=o["mf"])                # dH
+        torch.matmul(Y.t(), dZ, out=o["fh"])                     # dB
+        torch.matmul(X.t(), Y, out=o["hf"])                      # dA
+        torch.matmul(Y, self.A.t(), out=o["mh"])                 # dX (MLP)
+
 
 class VocabStep:
     """The vocabulary-parallel embedding and loss with tied weights, forward
@@ -485,6 +517,14 @@ def run_libtp(args, ranks: Ranks):
     barrier()
     block_ms = timed(st.block, args.steps, stream)
     barrier()
+    # Library yardstick: the same twelve GEMMs as plain cuBLAS calls.
+    st.make_library_gemms(dev)
+    for _ in range(2):
+        st.library_gemms()
+    barrier()
+    lib_ms = timed(st.library_gemms, args.steps, stream)
+    barrier()
+    del st.lib_out, st.lib_dqkv
     # The vocabulary-parallel embedding and loss (a second workload).
     vocab_ms = vocab_records = None
     vs = None
@@ -519,6 +559,7 @@ def run_libtp(args, ranks: Ranks):
 
     ms, mlp_ms, mlp_rec_ms = maxall(ms), maxall(mlp_ms), maxall(mlp_rec_ms)
     block_ms = maxall(block_ms)
+    lib_ms = maxall(lib_ms)
     vocab_ms = maxall(vocab_ms)
     e2e_ms = maxall(e2e_ms)
     if rank != 0:
@@ -580,6 +621,12 @@ def run_libtp(args, ranks: Ranks):
             "ms_per_step": round(block_ms / args.steps, 4),
             "tflops": round(world * fl["total"] / (block_ms / args.steps * 1e-3) / 1e12, 2),
             "overhead_vs_layer_step": round(block_ms / ms - 1.0, 4)},
+        "library_gemm_yardstick": {
+            "what": "the step's 12 GEMMs as plain torch.matmul (cuBLAS), same shapes and layouts, "
+                    "no epilogues; context only, not on the measured path",
+            "ms_per_step": round(lib_ms / args.steps, 4),
+            "tflops": round(st.lib_flops / (lib_ms / args.steps * 1e-3) / 1e12, 2),
+            "libtp_gemm_tflops": round(achieved, 2)},
         "activation_policy": {
             "save_y": {"mlp_ms_per_step": round(mlp_ms / args.steps, 4),
                        "bytes_kept_fwd_to_bwd": wl.M * wl.f * 2},

@@ -376,7 +376,11 @@ tp_status tp_vocab_ce_bwd(const void* X, const void* E, const int32_t* targets,
  * Workspace bytes that `op` needs for these sizes (M = b*s tokens; f is
  * ignored by the attention and LayerNorm ops, heads by the MLP and LayerNorm
  * ops).  Returns 0 for invalid arguments.  The size covers the worst case
- * (recomputed Y / QKV).
+ * (recomputed Y / QKV) and, for the MLP, attention and block ops, scratch of
+ * one fp32 partial tile per SM (about 19 MB on a B200) with which a GEMM
+ * splits its last, partial wave of tiles along K.  Those ops also accept a
+ * workspace without that scratch (the size minus it); their GEMMs then run
+ * the last wave whole.
  */
 size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, int t,
                          tp_dtype dtype);

@@ -129,6 +129,31 @@ struct Carve {
     off += bytes;
     return p;
   }
+  // `bytes` more if the workspace has room for them, else nullptr.
+  void* take_optional(size_t bytes) {
+    const size_t o = align_up(off, 256);
+    if (o + bytes > cap) return nullptr;
+    off = o + bytes;
+    return base + o;
+  }
+};
+
+// The optional part of a workspace: scratch for splitting a GEMM's last
+// partial wave along K.  tp_workspace_size() includes it; a workspace of
+// only the minimum size works without it.
+size_t tail_ws() { return align_up(gemm_tail_scratch_bytes(), 256) + 256; }
+
+struct Tail {
+  void* p = nullptr;
+  size_t bytes = 0;
+  explicit Tail(Carve& c) {
+    p = c.take_optional(gemm_tail_scratch_bytes());
+    bytes = p ? gemm_tail_scratch_bytes() : 0;
+  }
+  void to(Gemm& g) const {
+    g.tail_ws = p;
+    g.tail_ws_bytes = bytes;
+  }
 };
 
 tp_status check_dtype(tp_dtype d) {
@@ -219,14 +244,26 @@ tp_status linear_common(const void* X, const void* W, const void* bias, void* Y,
 
 // --------------------------------------------------------------------- MLP
 
-size_t mlp_fwd_ws(int64_t M, int64_t f, tp_dtype d) { return align_up(M * f * esize(d), 256) + 256; }
+}  // namespace
 
-size_t mlp_bwd_ws(int64_t M, int64_t h, int64_t f, tp_dtype d) {
+size_t mlp_fwd_ws_min(int64_t M, int64_t f, tp_dtype d) {
+  return align_up(M * f * esize(d), 256) + 256;
+}
+
+namespace {
+
+size_t mlp_fwd_ws(int64_t M, int64_t f, tp_dtype d) { return mlp_fwd_ws_min(M, f, d) + tail_ws(); }
+
+size_t mlp_bwd_ws_min(int64_t M, int64_t h, int64_t f, tp_dtype d) {
   const size_t mf = align_up(M * f * esize(d), 256);
   size_t cs = colsum_scratch_bytes(M, f);
   const size_t cs2 = colsum_scratch_bytes(M, h);
   if (cs2 > cs) cs = cs2;
   return 3 * mf + align_up(cs, 256) + 1024;
+}
+
+size_t mlp_bwd_ws(int64_t M, int64_t h, int64_t f, tp_dtype d) {
+  return mlp_bwd_ws_min(M, h, f, d) + tail_ws();
 }
 
 tp_status mlp_fwd(const void* X, const void* A, const void* bA, const void* B, const void* bB,
@@ -239,11 +276,12 @@ tp_status mlp_fwd(const void* X, const void* A, const void* bA, const void* B, c
   if (f % t != 0) return fail(TP_ERR_SHAPE, "f must be divisible by t");
   TP_TRY(check_ptrs_aligned({X, A, bA, B, bB, Z, Ysave, ws}));
   TP_TRY(check_rows({h, f}));
-  if (ws == nullptr || ws_bytes < mlp_fwd_ws(M, f, dtype))
+  if (ws == nullptr || ws_bytes < mlp_fwd_ws_min(M, f, dtype))
     return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
   const bool f32 = dtype == TP_F32;
   Carve c(ws, ws_bytes);
   void* H = c.take(M * f * esize(dtype));
+  const Tail tail(c);
 
   // Column-split first linear with GeLU per shard ([P3] §2.1 steps 1-2).
   Gemm g1;
@@ -255,6 +293,7 @@ tp_status mlp_fwd(const void* X, const void* A, const void* bA, const void* B, c
   g1.bias = bA;
   g1.out2 = Ysave; g1.ldo2 = f;
   g1.n_shard = f / t;
+  tail.to(g1);
   TP_TRY(run(g1, f32, stream));
 
   // Row-split second linear; the t partials are summed in the accumulator
@@ -267,6 +306,7 @@ tp_status mlp_fwd(const void* X, const void* A, const void* bA, const void* B, c
   g2.aux = residual; g2.ldaux = h;
   g2.out = Z; g2.ldo = h; g2.out_f32 = f32;
   g2.bias = bB;
+  tail.to(g2);
   return run(g2, f32, stream);
 }
 
@@ -282,7 +322,7 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
   if (f % t != 0) return fail(TP_ERR_SHAPE, "f must be divisible by t");
   TP_TRY(check_ptrs_aligned({X, A, bA, B, Ysave, dZ, dX, dA, dbA, dB, dbB, ws}));
   TP_TRY(check_rows({h, f}));
-  if (ws == nullptr || ws_bytes < mlp_bwd_ws(M, h, f, dtype))
+  if (ws == nullptr || ws_bytes < mlp_bwd_ws_min(M, h, f, dtype))
     return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
   const bool f32 = dtype == TP_F32;
   const size_t es = esize(dtype);
@@ -293,6 +333,7 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
   size_t cs = colsum_scratch_bytes(M, f);
   if (colsum_scratch_bytes(M, h) > cs) cs = colsum_scratch_bytes(M, h);
   void* scratch = c.take(cs);
+  const Tail tail(c);
 
   const void* Y = Ysave;
   if (Y == nullptr) {
@@ -306,6 +347,7 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
     gr.bias = bA;
     gr.out2 = Yrec; gr.ldo2 = f;
     gr.n_shard = f / t;
+    tail.to(gr);
     TP_TRY(run(gr, f32, stream));
     Y = Yrec;
   }
@@ -320,6 +362,7 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
   g3.out = dY; g3.ldo = f; g3.out_f32 = f32;
   g3.out2 = (Ysave != nullptr) ? H : nullptr; g3.ldo2 = f;
   g3.n_shard = f / t;
+  tail.to(g3);
   TP_TRY(run(g3, f32, stream));
 
   // dB_i = H_i^T @ dZ: shard i's rows of dB, no exchange.
@@ -329,6 +372,7 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
   g4.b = {dZ, h, false};
   g4.epi = kEpiStore;
   g4.out = dB; g4.ldo = h; g4.out_f32 = f32;
+  tail.to(g4);
   TP_TRY(run(g4, f32, stream));
 
   // dA_i = X^T @ dY_i: shard i's columns of dA, no exchange.
@@ -339,6 +383,7 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
   g5.epi = kEpiStore;
   g5.out = dA; g5.ldo = f; g5.out_f32 = f32;
   g5.n_shard = f / t;
+  tail.to(g5);
   TP_TRY(run(g5, f32, stream));
 
   // dX = sum_i dY_i @ A_i^T: shard partials summed in the accumulator.
@@ -348,6 +393,7 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
   g6.b = {A, f, true};  // A [h, f] read as A^T: n = h index, K contiguous
   g6.epi = kEpiStore;
   g6.out = dX; g6.ldo = h; g6.out_f32 = f32;
+  tail.to(g6);
   TP_TRY(run(g6, f32, stream));
 
   if (dbA) TP_TRY(launch_colsum(dY, M, f, f32, dbA, scratch, stream));
@@ -357,17 +403,21 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
 
 // --------------------------------------------------------------- attention
 
-size_t attn_fwd_ws(int64_t M, int64_t h, int heads) {
+size_t attn_fwd_ws_min(int64_t M, int64_t h, int heads) {
   return align_up(M * 3 * h * 2, 256) + align_up(M * h * 2, 256) +
          align_up(static_cast<size_t>(M) * heads * 4, 256) + 1024;
 }
 
-size_t attn_bwd_ws(int64_t M, int64_t h, int heads) {
+size_t attn_fwd_ws(int64_t M, int64_t h, int heads) { return attn_fwd_ws_min(M, h, heads) + tail_ws(); }
+
+size_t attn_bwd_ws_min(int64_t M, int64_t h, int heads) {
   AttnShape sh;
   sh.b = 1; sh.s = M; sh.h = h; sh.heads = heads;
   return 2 * align_up(M * 3 * h * 2, 256) + align_up(M * h * 2, 256) +
          align_up(attn_core_bwd_scratch_bytes(sh), 256) + 1024;
 }
+
+size_t attn_bwd_ws(int64_t M, int64_t h, int heads) { return attn_bwd_ws_min(M, h, heads) + tail_ws(); }
 
 tp_status attn_check(const void* X, const void* Wqkv, const void* Wo, int64_t b, int64_t s,
                      int64_t h, int heads, int t, tp_dtype dtype) {
@@ -393,12 +443,13 @@ tp_status attn_fwd(const void* X, const void* Wqkv, const void* Wo, void* Z, voi
   if (!Z) return fail(TP_ERR_NULL, "Z is required");
   TP_TRY(check_ptrs_aligned({X, Wqkv, Wo, Z, QKVsave, Osave, LSEsave, ws}));
   const int64_t M = b * s;
-  if (ws == nullptr || ws_bytes < attn_fwd_ws(M, h, heads))
+  if (ws == nullptr || ws_bytes < attn_fwd_ws_min(M, h, heads))
     return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
   Carve c(ws, ws_bytes);
   void* QKVw = c.take(M * 3 * h * 2);
   void* Ow = c.take(M * h * 2);
   void* LSEw = c.take(static_cast<size_t>(M) * heads * 4);
+  const Tail tail(c);
   void* QKV = QKVsave ? QKVsave : QKVw;
   void* O = Osave ? Osave : Ow;
   float* LSE = static_cast<float*>(LSEsave ? LSEsave : LSEw);
@@ -410,6 +461,7 @@ tp_status attn_fwd(const void* X, const void* Wqkv, const void* Wo, void* Z, voi
   gq.b = {Wqkv, 3 * h, false};
   gq.out = QKV; gq.ldo = 3 * h; gq.out_f16 = true;  // the attention core reads fp16
   gq.n_shard = h / t;
+  tail.to(gq);
   TP_TRY(launch_gemm_bf16(gq, stream));
 
   AttnShape sh;
@@ -424,6 +476,7 @@ tp_status attn_fwd(const void* X, const void* Wqkv, const void* Wo, void* Z, voi
   go.out = Z; go.ldo = h;
   go.epi = residual ? kEpiResidual : kEpiStore;  // Z = residual + Attn(X) when given
   go.aux = residual; go.ldaux = h;
+  tail.to(go);
   return launch_gemm_bf16(go, stream);
 }
 
@@ -436,7 +489,7 @@ tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* 
     return fail(TP_ERR_NULL, "Osave, LSEsave, dZ, dX, dWqkv and dWo are required");
   TP_TRY(check_ptrs_aligned({X, Wqkv, Wo, QKVsave, Osave, LSEsave, dZ, dX, dWqkv, dWo, ws}));
   const int64_t M = b * s;
-  if (ws == nullptr || ws_bytes < attn_bwd_ws(M, h, heads))
+  if (ws == nullptr || ws_bytes < attn_bwd_ws_min(M, h, heads))
     return fail(TP_ERR_WORKSPACE, "workspace missing or smaller than tp_workspace_size()");
   Carve c(ws, ws_bytes);
   void* QKVw = c.take(M * 3 * h * 2);
@@ -445,6 +498,7 @@ tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* 
   AttnShape sh;
   sh.b = b; sh.s = s; sh.h = h; sh.heads = heads; sh.causal = causal ? 1 : 0;
   void* scratch = c.take(attn_core_bwd_scratch_bytes(sh));
+  const Tail tail(c);
 
   const void* QKV = QKVsave;
   if (QKV == nullptr) {
@@ -454,7 +508,8 @@ tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* 
     gq.b = {Wqkv, 3 * h, false};
     gq.out = QKVw; gq.ldo = 3 * h; gq.out_f16 = true;
     gq.n_shard = h / t;
-    TP_TRY(launch_gemm_bf16(gq, stream));
+    tail.to(gq);
+  TP_TRY(launch_gemm_bf16(gq, stream));
     QKV = QKVw;
   }
 
@@ -465,6 +520,7 @@ tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* 
   g1.b = {Wo, h, true};
   g1.out = dO; g1.ldo = h; g1.out_f16 = true;  // the attention core reads fp16
   g1.n_shard = h / t;
+  tail.to(g1);
   TP_TRY(launch_gemm_bf16(g1, stream));
 
   // dWo_g = O_g^T @ dZ: group g's rows of dWo, no exchange.
@@ -473,6 +529,7 @@ tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* 
   g2.a = {Osave, h, false};
   g2.b = {dZ, h, false};
   g2.out = dWo; g2.ldo = h;
+  tail.to(g2);
   TP_TRY(launch_gemm_bf16(g2, stream));
 
   TP_TRY(launch_attn_core_bwd(sh, QKV, Osave, static_cast<const float*>(LSEsave), dO, dQKV,
@@ -485,6 +542,7 @@ tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* 
   g3.b = {dQKV, 3 * h, false};
   g3.out = dWqkv; g3.ldo = 3 * h;
   g3.n_shard = h / t;
+  tail.to(g3);
   TP_TRY(launch_gemm_bf16(g3, stream));
 
   // dX = sum_g dQKV_g @ Wqkv_g^T: the K loop visits group 0's q, k and v
@@ -501,6 +559,7 @@ tp_status attn_bwd(const void* X, const void* Wqkv, const void* Wo, const void* 
     g4.korder.width = static_cast<int>(width);
     g4.korder.h = static_cast<int>(h);
   }
+  tail.to(g4);
   return launch_gemm_bf16(g4, stream);
 }
 

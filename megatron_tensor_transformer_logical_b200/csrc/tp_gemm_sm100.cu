@@ -75,8 +75,44 @@ struct Args {
   int ce_cps;
   const int* ce_target;
   float* ce_tlogit;
+  // Work units: tiles [0, tail0) whole; each later tile split into
+  // tail_split slices of its K blocks, whose fp32 partial tiles go to
+  // tail_part and are summed (slice order) by gemm_tail_fixup.
+  int units, tail0, tail_split;
+  float* tail_part;
   int* status;
 };
+
+struct Unit {
+  int tile, kb0, kb1;
+  int part;  // index of the partial tile, -1 for a whole tile
+};
+
+__device__ __forceinline__ Unit unit_of(int u, const Args& a) {
+  Unit w;
+  if (u < a.tail0) {
+    w.tile = u;
+    w.kb0 = 0;
+    w.kb1 = a.k_blocks;
+    w.part = -1;
+  } else {
+    const int v = u - a.tail0;
+    const int ks = v % a.tail_split;
+    w.tile = a.tail0 + v / a.tail_split;
+    w.kb0 = ks * a.k_blocks / a.tail_split;
+    w.kb1 = (ks + 1) * a.k_blocks / a.tail_split;
+    w.part = v;
+  }
+  return w;
+}
+
+// 32 fp32 accumulator values of one row into a partial tile (row-major,
+// `ld` floats per row).
+__device__ __forceinline__ void store_partial32(const float (&v)[32], float* dst) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
 
 struct TileCoord {
   int m0, n0, n_end;
@@ -327,7 +363,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = args.m_tiles * args.n_tiles;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -335,9 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const TileCoord tc = tile_coord<BN>(tile, args);
-        for (int kb = 0; kb < args.k_blocks; ++kb) {
+      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
+        const Unit w = unit_of(u, args);
+        const TileCoord tc = tile_coord<BN>(w.tile, args);
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, args.status, kStatusProducerTimeout)) {
             ok = false;
             break;
@@ -376,11 +412,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
+        const Unit w = unit_of(u, args);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.status, kStatusMmaTimeout)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < args.k_blocks; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, args.status, kStatusMmaTimeout)) {
             ok = false;
             break;
@@ -394,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        : sw128_desc(a0 + k * 2048, BK * 128, 1024);
             const uint64_t bd = B_KMAJ ? sw128_desc(b0 + k * 32, 16, 1024)
                                        : sw128_desc(b0 + k * 2048, BK * 128, 1024);
-            umma_bf16(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, ad, bd, kIdesc, (kb != w.kb0 || k != 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           if (++stage == C::kStages) {
@@ -417,11 +454,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = ew >> 2;      // which half of the tile's columns
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const TileCoord tc = tile_coord<BN>(tile, args);
+    for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
+      const Unit w = unit_of(u, args);
+      const TileCoord tc = tile_coord<BN>(w.tile, args);
       if (!mbar_wait(&tfull[acc], acc_phase, args.status, kStatusEpilogueTimeout)) break;
       tc_fence_after();
-      const int row = tc.m0 + quarter * 32 + lane;
+      const int lrow = quarter * 32 + lane;
+      const int row = tc.m0 + lrow;
       const int tg = (EPI == kEpiCE && row < args.M) ? args.ce_target[row] : -1;
 #pragma unroll 1
       for (int c = 0; c < BN / 2; c += 32) {
@@ -431,7 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                       static_cast<uint32_t>(acc * BN + cl),
                   v);
-        if constexpr (EPI == kEpiCE)
+        if (w.part >= 0)  // a K slice of a tail tile: raw partial sums
+          store_partial32(v, args.tail_part + (static_cast<long long>(w.part) * BM + lrow) * BN + cl);
+        else if constexpr (EPI == kEpiCE)
           epilogue_ce32(v, row, tc.n0 + cl, tc.n_end, tg, args);
         else
           epilogue_row32<EPI, OUT, false>(v, row, tc.n0 + cl, tc.n_end, args);
@@ -532,7 +573,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();  // barriers initialised and tensor memory allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = args.m_tiles * args.n_tiles;
   const int cluster_id = static_cast<int>(blockIdx.x >> 1);
   const int num_clusters = static_cast<int>(gridDim.x >> 1);
 
@@ -542,11 +582,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
-        const TileCoord tc = tile_coord_pair(tile, args);
+      for (int u = cluster_id; u < args.units && ok; u += num_clusters) {
+        const Unit w = unit_of(u, args);
+        const TileCoord tc = tile_coord_pair(w.tile, args);
         const int am0 = tc.m0 + 128 * static_cast<int>(rank);
         const int bn0 = tc.n0 + 128 * static_cast<int>(rank);
-        for (int kb = 0; kb < args.k_blocks; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, args.status, kStatusProducerTimeout)) {
             ok = false;
             break;
@@ -584,11 +625,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+      for (int u = cluster_id; u < args.units && ok; u += num_clusters) {
+        const Unit w = unit_of(u, args);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, args.status, kStatusMmaTimeout)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kPairTN);
-        for (int kb = 0; kb < args.k_blocks; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, args.status, kStatusMmaTimeout)) {
             ok = false;
             break;
@@ -602,7 +644,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                        : sw128_desc(a0 + k * 2048, BK * 128, 1024);
             const uint64_t bd = B_KMAJ ? sw128_desc(b0 + k * 32, 16, 1024)
                                        : sw128_desc(b0 + k * 2048, BK * 128, 1024);
-            umma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            umma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb != w.kb0 || k != 0) ? 1u : 0u);
           }
           // Free the stage in both CTAs once these MMAs have read it.
           umma_commit_pair(mapa_shared(smem_u32(&empty[stage]), 0));
@@ -630,11 +672,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                        mapa_shared(smem_u32(&tempty[1]), 0)};
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = cluster_id; tile < num_tiles; tile += num_clusters) {
-      const TileCoord tc = tile_coord_pair(tile, args);
+    for (int u = cluster_id; u < args.units; u += num_clusters) {
+      const Unit w = unit_of(u, args);
+      const TileCoord tc = tile_coord_pair(w.tile, args);
       if (!mbar_wait(&tfull[acc], acc_phase, args.status, kStatusEpilogueTimeout)) break;
       tc_fence_after();
-      const int row = tc.m0 + 128 * static_cast<int>(rank) + quarter * 32 + lane;
+      const int lrow = 128 * static_cast<int>(rank) + quarter * 32 + lane;
+      const int row = tc.m0 + lrow;
       const int tg = (EPI == kEpiCE && row < args.M) ? args.ce_target[row] : -1;
 #pragma unroll 1
       for (int c = 0; c < kPairTN / 2; c += 32) {
@@ -644,7 +688,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                       static_cast<uint32_t>(acc * kPairTN + cl),
                   v);
-        if constexpr (EPI == kEpiCE)
+        if (w.part >= 0)  // a K slice of a tail tile: raw partial sums
+          store_partial32(v, args.tail_part +
+                                 (static_cast<long long>(w.part) * kPairTM + lrow) * kPairTN + cl);
+        else if constexpr (EPI == kEpiCE)
           epilogue_ce32(v, row, tc.n0 + cl, tc.n_end, tg, args);
         else
           epilogue_row32<EPI, OUT, false>(v, row, tc.n0 + cl, tc.n_end, args);
@@ -665,6 +712,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();  // no CTA frees tensor memory while its pair may still use it
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
+}
+
+// Sums the K-slice partials of each tail tile in slice order and applies the
+// GEMM's epilogue, exactly as the GEMM kernel would have for a whole tile.
+// CTA (tail tile, quarter of its rows); a thread handles 32 columns of one row.
+constexpr int kFixupRowGroups = 4;
+
+template <int TM, int TN, bool PAIR, int EPI, int OUT>
+__global__ void __launch_bounds__(256) gemm_tail_fixup(const Args a) {
+  const int ti = blockIdx.x;
+  const int tile = a.tail0 + ti;
+  const TileCoord tc = PAIR ? tile_coord_pair(tile, a) : tile_coord<TN>(tile, a);
+  const float* base = a.tail_part + static_cast<long long>(ti) * a.tail_split * TM * TN;
+  constexpr int kRows = TM / kFixupRowGroups;
+  for (int item = threadIdx.x; item < kRows * (TN / 32); item += blockDim.x) {
+    const int r = blockIdx.y * kRows + item / (TN / 32);
+    const int cl = (item % (TN / 32)) * 32;
+    if (tc.n0 + cl >= tc.n_end || tc.m0 + r >= a.M) continue;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+    for (int ks = 0; ks < a.tail_split; ++ks) {
+      const float4* src = reinterpret_cast<const float4*>(
+          base + (static_cast<long long>(ks) * TM + r) * TN + cl);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 q = src[i];
+        v[4 * i] += q.x;
+        v[4 * i + 1] += q.y;
+        v[4 * i + 2] += q.z;
+        v[4 * i + 3] += q.w;
+      }
+    }
+    epilogue_row32<EPI, OUT, false>(v, tc.m0 + r, tc.n0 + cl, tc.n_end, a);
+  }
+}
+
+// Splitting the last, partial wave of tiles along K: with T tiles on G
+// persistent CTAs (or CTA pairs) and R = T mod G tiles left for the last
+// wave, those R tiles are cut into S = min(G / R, K blocks / 32) K slices, so
+// the last wave keeps R * S of the G workers busy for 1/S of a tile's time;
+// a fixup kernel adds the slices.  Only when at least one full wave exists,
+// the tail is at most half a wave, every slice keeps at least 32 K blocks
+// (shorter slices cost more in partial traffic than they save), and the
+// caller gave scratch for the R * S fp32 partial tiles.  The result of a tail tile differs from the
+// unsplit one only in the grouping of its fp32 sums.
+struct TailPlan {
+  int units, tail0, split;
+};
+
+TailPlan plan_tail(long long tiles, int workers, int k_blocks, size_t part_bytes, const Gemm& g,
+                   int epi) {
+  TailPlan tp{static_cast<int>(tiles), static_cast<int>(tiles), 1};
+  if (epi == kEpiCE || g.tail_ws == nullptr || tiles <= workers) return tp;
+  const long long R = tiles % workers;
+  if (R == 0 || 2 * R > workers) return tp;
+  int S = static_cast<int>(workers / R);
+  if (S > k_blocks / 32) S = k_blocks / 32;
+  if (S < 2 || static_cast<size_t>(R) * S * part_bytes > g.tail_ws_bytes) return tp;
+  tp.tail0 = static_cast<int>(tiles - R);
+  tp.split = S;
+  tp.units = tp.tail0 + static_cast<int>(R) * S;
+  return tp;
 }
 
 // ------------------------------------------------------------------ host side
@@ -822,6 +932,11 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   const long long tiles = static_cast<long long>(p.m_tiles) * p.n_tiles;
   if (tiles == 0) return TP_OK;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+  const TailPlan tp = plan_tail(tiles, grid, a.k_blocks, size_t(BM) * BN * 4, g, EPI);
+  a.units = tp.units;
+  a.tail0 = tp.tail0;
+  a.tail_split = tp.split;
+  a.tail_part = static_cast<float*>(g.tail_ws);
   const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
                        (OUT == kOutF32 ? 4.0 : 2.0) * double(g.M) * g.N +
@@ -829,8 +944,12 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
                        (g.aux ? 2.0 * double(g.M) * g.N : 0.0) +
                        (EPI == kEpiCE ? 8.0 * double(g.M) * g.N / 32.0 : 0.0);
   {
-    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, 1, BN, g.M, g.N, g.K);
+    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, tp.split > 1 ? 2 : 1, BN, g.M,
+                      g.N, g.K);
     kern<<<grid, kThreads, C::kSmemBytes, stream>>>(ta, tb, a);
+    if (tp.split > 1)
+      gemm_tail_fixup<BM, BN, false, EPI, OUT>
+          <<<dim3(static_cast<unsigned>(tiles - tp.tail0), kFixupRowGroups), 256, 0, stream>>>(a);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm_bf16_tcgen05 launch");
@@ -931,6 +1050,11 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   if (tiles == 0) return TP_OK;
   const int mc = max_clusters[dev & 31];
   const int clusters = static_cast<int>(tiles < mc ? tiles : mc);
+  const TailPlan tp = plan_tail(tiles, clusters, a.k_blocks, size_t(kPairTM) * kPairTN * 4, g, EPI);
+  a.units = tp.units;
+  a.tail0 = tp.tail0;
+  a.tail_split = tp.split;
+  a.tail_part = static_cast<float*>(g.tail_ws);
   const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
                        (OUT == kOutF32 ? 4.0 : 2.0) * double(g.M) * g.N +
@@ -938,8 +1062,12 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
                        (g.aux ? 2.0 * double(g.M) * g.N : 0.0) +
                        (EPI == kEpiCE ? 8.0 * double(g.M) * g.N / 32.0 : 0.0);
   {
-    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, 1, 512, g.M, g.N, g.K);
+    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, tp.split > 1 ? 2 : 1, 512, g.M,
+                      g.N, g.K);
     kern<<<2 * clusters, kThreads, kPairSmemBytes, stream>>>(ta, tb, a);
+    if (tp.split > 1)
+      gemm_tail_fixup<kPairTM, kPairTN, true, EPI, OUT>
+          <<<dim3(static_cast<unsigned>(tiles - tp.tail0), kFixupRowGroups), 256, 0, stream>>>(a);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm_bf16_tcgen05_pair launch");
@@ -976,6 +1104,12 @@ tp_status dispatch_pair(const Gemm& g, cudaStream_t s) {
 }
 
 }  // namespace
+
+size_t gemm_tail_scratch_bytes() {
+  // At most one partial tile per persistent CTA (128 x 256 fp32) or per CTA
+  // pair (256 x 256 fp32, half as many pairs).
+  return static_cast<size_t>(sm_count()) * 128 * 256 * 4;
+}
 
 tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return TP_OK;

@@ -96,7 +96,18 @@ struct Gemm {
   int64_t n_shard = 0;         // columns per shard: column tiles never straddle shards
   KOrder korder;
   CEOut ce;                    // kEpiCE only (requires n_shard % 8 == 0)
+  // Scratch for splitting the last partial wave of tiles along K (optional;
+  // gemm_tail_scratch_bytes() is always enough).
+  void* tail_ws = nullptr;
+  size_t tail_ws_bytes = 0;
 };
+
+// Scratch that lets a tcgen05 GEMM split its last wave along K.
+size_t gemm_tail_scratch_bytes();
+
+// The smallest workspace tp_mlp_fwd accepts (without the optional GEMM tail
+// scratch that tp_workspace_size() adds).
+size_t mlp_fwd_ws_min(int64_t M, int64_t f, tp_dtype d);
 
 // bf16 x bf16 -> fp32 accumulate on tcgen05; out bf16, fp16 or fp32.
 tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream);

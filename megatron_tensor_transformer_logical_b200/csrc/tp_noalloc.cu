@@ -63,7 +63,9 @@ extern "C" tp_status tp_mlp_fwd_noalloc(const void* X, const void* A, const void
   try {
     if (dtype != TP_F32 && dtype != TP_BF16) return tp::fail(TP_ERR_DTYPE, "unknown dtype");
     if (M <= 0 || h <= 0 || f <= 0) return tp::fail(TP_ERR_SHAPE, "M, h and f must be positive");
-    const size_t need = tp_workspace_size(TP_OP_MLP_FWD, M, h, f, 0, t < 1 ? 1 : t, dtype);
+    const size_t need = (M > 0 && h > 0 && f > 0 && (dtype == TP_F32 || dtype == TP_BF16))
+                            ? tp::mlp_fwd_ws_min(M, f, dtype)
+                            : 0;
     if (need == 0 || need > tp::kNoAllocScratchBytes)
       return tp::fail(TP_ERR_SHAPE,
                       "tp_mlp_fwd_noalloc: H [M, f] needs " + std::to_string(need) +
