@@ -169,3 +169,46 @@ def test_fp16_range_overflow_is_reported():
     assert e.value.status == L.TP_ERR_KERNEL and "fp16" in str(e.value)
     assert torch.isfinite(QKV.float()).all() and QKV.float().max().item() == 65504.0
     L.tp_device_status()  # the word was cleared
+
+
+def test_attention_with_last_wave_split():
+    """b = 2, s = 2048, h = 4096 (32 heads), t = 8: the dO GEMM (fp16 output,
+    single-SM tiles) and the dX GEMM (SM-pair tiles, head-group K order) both
+    leave a last wave under half full, which they split along K and add back
+    in a fixup kernel; the whole layer is compared with the oracle."""
+    wl = Workload(97, "last-wave split", b=2, s=2048, h=4096, heads=32, t=8, w_std=0.02)
+    inp = make_attn_inputs(wl)
+    compare_full(gpu_attn(inp, wl), inp, wl, True)
+
+
+def test_mlp_with_last_wave_split_all_epilogues():
+    """M = h = f = 4096, t = 8, with biases: each of the six MLP GEMMs leaves a
+    last wave of under half the SMs or SM pairs (512 single-SM or 256 pair
+    tiles on 148 SMs), so the bias + GeLU, GeLU', plain and wgrad epilogues
+    all run through the K-split fixup; compared with the oracle on every
+    output."""
+    from megatron_tensor_transformer_logical_b200.inputs import make_mlp_inputs
+    wl = Workload(98, "mlp last-wave split", b=2, s=2048, h=4096, f=4096, t=8, w_std=0.02,
+                  bias_std=0.02)
+    inp = make_mlp_inputs(wl)
+    d = {k: cuda(v) for k, v in inp.items()}
+    M, h, f = wl.M, wl.h, wl.f
+    Z = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
+    Y = torch.empty(M, f, dtype=torch.bfloat16, device="cuda")
+    n0 = L.tp_launch_count()
+    L.tp_mlp_fwd(d["X"], d["A"], d["bA"], d["B"], d["bB"], Z, Y, wl.t,
+                 L.workspace(L.TP_OP_MLP_FWD, M, h, f, 0, wl.t, L.TP_BF16))
+    # two GEMMs, and a fixup kernel for each GEMM that split its last wave
+    assert L.tp_launch_count() - n0 >= 3, "the forward GEMMs did not split their last wave"
+    g = {k: torch.empty_like(d[k]) for k in ("X", "A", "B")}
+    dbA = torch.empty(f, dtype=torch.bfloat16, device="cuda")
+    dbB = torch.empty(h, dtype=torch.bfloat16, device="cuda")
+    L.tp_mlp_bwd(d["X"], d["A"], d["bA"], d["B"], Y, d["dZ"], g["X"], g["A"], dbA, g["B"], dbB,
+                 wl.t, L.workspace(L.TP_OP_MLP_BWD, M, h, f, 0, wl.t, L.TP_BF16))
+    torch.cuda.synchronize()
+    fw = O.mlp_fwd(inp["X"], inp["A"], inp["bA"], inp["B"], inp["bB"])
+    bw = O.mlp_bwd(inp["X"], inp["A"], inp["bA"], inp["B"], inp["dZ"])
+    check(Z, fw["Z"], "Z", "bf16")
+    check(Y, fw["Y"], "Y", "bf16")
+    for k, v in (("dX", g["X"]), ("dA", g["A"]), ("dB", g["B"]), ("dbA", dbA), ("dbB", dbB)):
+        check(v, bw[k], k, "bf16")
