@@ -159,3 +159,13 @@ def test_linear_uncommon_shard_counts(mode, t):
         for p in parts[1:]:
             total += p
         assert torch.equal(total, Y)
+
+
+@pytest.mark.parametrize("mode", ["col", "row"])
+def test_linear_single_row_exact(mode):
+    """M = 1 with integer-valued inputs: exact for every shard count."""
+    K, N = 512, 1024
+    X, W = integer_tensor((1, K), -3, 3, 17), integer_tensor((K, N), -3, 3, 18)
+    for t in (1, 2, 8):
+        Y = run(mode, cuda(X), cuda(W), None, t, out_dtype=torch.float32)
+        assert np.array_equal(to64(Y), O.linear(X, W, None)), t

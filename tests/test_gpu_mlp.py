@@ -133,3 +133,12 @@ def test_mlp_uncommon_shard_counts(t):
                   w_std=0.05, bias_std=0.05)
     inp = make_mlp_inputs(wl)
     compare_full(gpu_mlp(inp, t), inp, "bf16")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_mlp_single_token(dtype):
+    """M = 1: one row in a 128-row tile (the rest of the tile is out of range)."""
+    wl = Workload(94, "one token", b=1, s=1, h=256, f=1024, t=4, w_std=0.05, bias_std=0.05,
+                  dtype="f32" if dtype == torch.float32 else "bf16")
+    inp = make_mlp_inputs(wl)
+    compare_full(gpu_mlp(inp, wl.t, dtype=dtype), inp, "f32" if dtype == torch.float32 else "bf16")
