@@ -387,51 +387,64 @@ __global__ void __launch_bounds__(256) embed_run_scatter_kernel(
 
 // -------------------------------------------------------------- cross-entropy
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;  // exact: every lane holds the same maximum
+// Folds the pair (m2, s2) into the running pair (m, s), both meaning
+// s * exp(m) = the sum of exp(z) over what was folded in so far.  Commutative
+// bit for bit (one max, two products, one sum), so an xor-shuffle tree leaves
+// every lane with the same pair.
+__device__ __forceinline__ void ms_fold(float& m, float& s, float m2, float s2) {
+  const float nm = fmaxf(m, m2);
+  if (nm == -INFINITY) return;  // both empty
+  s = s * exp2f((m - nm) * kLog2e) + s2 * exp2f((m2 - nm) * kLog2e);
+  m = nm;
 }
 
-// Fixed-shape tree; lane 0's total is broadcast so every lane uses one value.
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
-  return __shfl_sync(0xffffffffu, v, 0);
-}
+constexpr int kCombineThreads = 256;
+constexpr int kCombineBatch = 4;
 
-// One warp per row.  Step 2: the chunks of shard i are combined into the
-// shard's (max m_i, sum s_i of exp(z - m_i)).  Step 3: the shards are
-// combined in shard order, each rescaled to the running maximum, into
-// lse = m + log(S).  Steps 4-5: loss = lse - z[target] (0 if ignored).
-__global__ void __launch_bounds__(256) ce_combine_kernel(const float2* __restrict__ part,
-                                                         int64_t ldp, int cps, int t,
-                                                         const int* __restrict__ target,
-                                                         const float* __restrict__ tlogit,
-                                                         int64_t M, int64_t V, float* lse,
-                                                         float* loss) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= M) return;  // warp-uniform
+// One block per row.  Steps 2-3: the row's chunk pairs (max m_c, sum of
+// exp(z - m_c)) over all shards are folded into one (max, sum) -- each thread
+// a fixed strided share, then a fixed xor tree in the warp and across the
+// block's warps -- and lse = m + log(S); the grouping of a log-sum-exp's terms
+// changes it only by rounding.  Steps 4-5: loss = lse - z[target] (0 if the
+// target is ignored).
+__global__ void __launch_bounds__(kCombineThreads) ce_combine_kernel(
+    const float2* __restrict__ part, int64_t ldp, const int* __restrict__ target,
+    const float* __restrict__ tlogit, int64_t V, float* lse, float* loss) {
+  __shared__ float2 red[kCombineThreads / 32];
+  const int64_t row = blockIdx.x;
   const float2* p = part + row * ldp;
-  float gm = -INFINITY, gs = 0.0f;
-  for (int sh = 0; sh < t; ++sh) {
-    const float2* q = p + static_cast<int64_t>(sh) * cps;
-    float m = -INFINITY;
-    for (int j = lane; j < cps; j += 32) m = fmaxf(m, q[j].x);
-    m = warp_max(m);
-    float s = 0.0f;
-    for (int j = lane; j < cps; j += 32) {
-      const float2 c = q[j];
-      s += c.y * exp2f((c.x - m) * kLog2e);
+  float m = -INFINITY, s = 0.0f;
+  for (int64_t j0 = threadIdx.x; j0 < ldp; j0 += kCombineBatch * kCombineThreads) {
+    float2 c[kCombineBatch];
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u) {
+      const int64_t j = j0 + u * kCombineThreads;
+      c[u] = j < ldp ? p[j] : make_float2(-INFINITY, 0.0f);
     }
-    s = warp_sum(s);
-    const float nm = fmaxf(gm, m);
-    gs = gs * exp2f((gm - nm) * kLog2e) + s * exp2f((m - nm) * kLog2e);
-    gm = nm;
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u) ms_fold(m, s, c[u].x, c[u].y);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    ms_fold(m, s, m2, s2);
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) red[warp] = make_float2(m, s);
+  __syncthreads();
+  if (warp != 0) return;
+  const float2 w = lane < kCombineThreads / 32 ? red[lane] : make_float2(-INFINITY, 0.0f);
+  m = w.x;
+  s = w.y;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    ms_fold(m, s, m2, s2);
   }
   if (lane == 0) {
-    const float l = gm + logf(gs);
+    const float l = m + logf(s);
     lse[row] = l;
     const int tg = target[row];
     loss[row] = (tg >= 0 && tg < V) ? l - tlogit[row] : 0.0f;
@@ -471,36 +484,51 @@ __global__ void ce_total_kernel(const float* __restrict__ shard_tot, int t, floa
   *total = s;
 }
 
-// dlogits = (exp(z - lse) - [col == target]) * dloss over [M, V] bf16, 8
-// columns per thread; rows with an ignored target get zeros.
-__global__ void __launch_bounds__(256) ce_dlogits_kernel(const __nv_bfloat16* logits,
-                                                         const float* __restrict__ lse,
-                                                         const int* __restrict__ target,
-                                                         const float* __restrict__ dloss,
-                                                         __nv_bfloat16* dlogits, int64_t M,
-                                                         int64_t V) {
+// dlogits = (exp(z - lse) - [col == target]) * dloss over [M, V] bf16 in
+// 8-column vectors, each thread's four loads issued before its first store
+// (dlogits may alias logits: every vector is read before the same thread
+// overwrites it); rows with an ignored target get zeros.
+constexpr int kGradThreads = 256;
+constexpr int kGradBatch = 4;  // 16-byte vectors in flight per thread
+
+__global__ void __launch_bounds__(kGradThreads) ce_dlogits_kernel(
+    const __nv_bfloat16* logits, const float* __restrict__ lse, const int* __restrict__ target,
+    const float* __restrict__ dloss, __nv_bfloat16* dlogits, int64_t M, int64_t V) {
   const int64_t nvec = V / 8;
+  const int64_t span = static_cast<int64_t>(kGradBatch) * kGradThreads;
   for (int64_t row = blockIdx.y; row < M; row += gridDim.y) {
     const int64_t tg = target[row];
     const bool ok = tg >= 0 && tg < V;
     const float dl = ok ? (dloss != nullptr ? dloss[row] : 1.0f) : 0.0f;
     const float l2 = lse[row] * kLog2e;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-      const uint4 q = *reinterpret_cast<const uint4*>(logits + row * V + 8 * i);
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
-      uint4 out;
-      uint32_t* w = reinterpret_cast<uint32_t*>(&out);
+    const uint4* zr = reinterpret_cast<const uint4*>(logits + row * V);
+    uint4* gr = reinterpret_cast<uint4*>(dlogits + row * V);
+    for (int64_t i0 = blockIdx.x * span + threadIdx.x; i0 < nvec; i0 += gridDim.x * span) {
+      uint4 q[kGradBatch];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 z = __bfloat1622float2(p[k]);
-        const int64_t c = 8 * i + 2 * k;
-        const float g0 = (ex2_approx(fmaf(z.x, kLog2e, -l2)) - (c == tg ? 1.0f : 0.0f)) * dl;
-        const float g1 = (ex2_approx(fmaf(z.y, kLog2e, -l2)) - (c + 1 == tg ? 1.0f : 0.0f)) * dl;
-        __nv_bfloat162 t2 = __floats2bfloat162_rn(g0, g1);
-        w[k] = *reinterpret_cast<uint32_t*>(&t2);
+      for (int u = 0; u < kGradBatch; ++u) {
+        const int64_t i = i0 + u * kGradThreads;
+        if (i < nvec) q[u] = zr[i];
       }
-      *reinterpret_cast<uint4*>(dlogits + row * V + 8 * i) = out;
+#pragma unroll
+      for (int u = 0; u < kGradBatch; ++u) {
+        const int64_t i = i0 + u * kGradThreads;
+        if (i >= nvec) break;
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q[u]);
+        uint4 out;
+        uint32_t* w = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 z = __bfloat1622float2(p[k]);
+          const int64_t c = 8 * i + 2 * k;
+          const float g0 = (ex2_approx(fmaf(z.x, kLog2e, -l2)) - (c == tg ? 1.0f : 0.0f)) * dl;
+          const float g1 =
+              (ex2_approx(fmaf(z.y, kLog2e, -l2)) - (c + 1 == tg ? 1.0f : 0.0f)) * dl;
+          __nv_bfloat162 t2 = __floats2bfloat162_rn(g0, g1);
+          w[k] = *reinterpret_cast<uint32_t*>(&t2);
+        }
+        gr[i] = out;
+      }
     }
   }
 }
@@ -600,13 +628,12 @@ tp_status launch_embed_bwd(const int* ids, const void* dY, const void* dE_in, vo
 tp_status launch_ce_finish(const CEOut& ce, int t, int64_t M, int64_t V, float* lse, float* loss,
                            float* total, float* shard_tot, cudaStream_t stream) {
   if (M <= 0) return TP_OK;
-  const int64_t blocks = (M + 7) / 8;
+  if (M > 0x7fffffffLL) return fail(TP_ERR_SHAPE, "cross-entropy combine: M too large");
   {
     LaunchScope scope(TP_KIND_VOCAB, 0.0, 8.0 * M * ce.ldp + 20.0 * M, stream,
                       total != nullptr ? 3 : 1, kVocabLossCombine);
-    ce_combine_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        reinterpret_cast<const float2*>(ce.part), ce.ldp, ce.cps, t, ce.target, ce.tlogit, M, V,
-        lse, loss);
+    ce_combine_kernel<<<static_cast<unsigned>(M), kCombineThreads, 0, stream>>>(
+        reinterpret_cast<const float2*>(ce.part), ce.ldp, ce.target, ce.tlogit, V, lse, loss);
     if (total != nullptr) {
       ce_shard_loss_kernel<<<t, 1024, 0, stream>>>(loss, ce.target, M, V / t, shard_tot);
       ce_total_kernel<<<1, 32, 0, stream>>>(shard_tot, t, total);
@@ -621,12 +648,13 @@ tp_status launch_ce_dlogits(const void* logits, const float* lse, const int* tar
                             cudaStream_t stream) {
   if (M <= 0) return TP_OK;
   const int64_t nvec = V / 8;
-  const int64_t gx64 = (nvec + 255) / 256;
+  const int64_t span = static_cast<int64_t>(kGradBatch) * kGradThreads;
+  const int64_t gx64 = (nvec + span - 1) / span;
   const unsigned gx = static_cast<unsigned>(gx64 < 1024 ? gx64 : 1024);
   const unsigned gy = static_cast<unsigned>(M < 65535 ? M : 65535);
   {
     LaunchScope scope(TP_KIND_VOCAB, 0.0, 4.0 * M * V + 12.0 * M, stream, 1, kVocabSoftmaxGrad);
-    ce_dlogits_kernel<<<dim3(gx, gy), 256, 0, stream>>>(
+    ce_dlogits_kernel<<<dim3(gx, gy), kGradThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(logits), lse, target, dloss,
         static_cast<__nv_bfloat16*>(dlogits), M, V);
   }
