@@ -58,18 +58,6 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int m, int n, bool a_mn, bo
          ((static_cast<uint32_t>(n) >> 3) << 17) | ((static_cast<uint32_t>(m) >> 4) << 24);
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz;
-// relative error about 2^-22, subnormal results flushed to zero, 2^-inf = 0).
-// The probabilities it produces are rounded to fp16 right after.
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 t = __floats2half2_rn(a, b);
@@ -303,7 +291,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         }
       }
       l_run = l_run * alpha + rs;
-      fence_proxy_async_smem();  // P stores visible to the tensor core
+      fence_async_smem();  // P stores visible to the tensor core
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
@@ -562,7 +550,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         *reinterpret_cast<uint4*>(row + ((chunk ^ (r & 7)) << 4)) =
             make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
-      fence_proxy_async_smem();
+      fence_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_full[st]);
@@ -816,7 +804,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         *reinterpret_cast<uint4*>(drow + off) =
             make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
       }
-      fence_proxy_async_smem();
+      fence_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[st]);

@@ -22,7 +22,13 @@
 //   warps 4-11  epilogue: tcgen05.ld the accumulator (warp w reads lanes
 //               32*(w%4)..+31, i.e. one output row per thread), apply
 //               bias / GeLU / GeLU' in fp32 and store; the other buffer is
-//               being filled meanwhile.
+//               being filled meanwhile.  Two-byte outputs go through a
+//               32 x 32 shared-memory box per warp and a TMA store (whole
+//               128-byte lines, four shared-memory wavefronts per 512 bytes
+//               instead of one per row), and the operand the epilogue reads
+//               (Y for GeLU', the residual) arrives the same way, so the
+//               epilogue leaves the shared-memory datapath to the tensor
+//               core's operand reads.
 // Every wait is bounded (see mbar_wait): on expiry the kernel records an
 // error code in the device status word and unwinds.
 #include <cuda.h>
@@ -48,14 +54,21 @@ constexpr int kThreads = 384;
 constexpr int kEpiWarps = 8;
 constexpr int kFirstEpiWarp = 4;
 
+// Epilogue staging: per epilogue warp two boxes of 32 rows x 32 two-byte
+// columns (64-byte rows, 64-byte swizzle).
+constexpr int kEpiBoxBytes = 32 * 64;
+constexpr int kEpiStageBytes = kEpiWarps * 2 * kEpiBoxBytes;  // 32 KB
+constexpr int kBarBytes = 256;
+
 template <int BN>
 struct Cfg {
-  static constexpr int kStages = (BN == 256) ? 4 : (BN == 192 ? 5 : 6);
+  static constexpr int kStages = (BN == 128) ? 6 : 4;
   static constexpr int kABytes = BM * BK * 2;
   static constexpr int kBBytes = BN * BK * 2;
   static constexpr int kTmemCols = (2 * BN > 256) ? 512 : 256;  // a power of two
-  static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kBarBytes;
+  static constexpr int kSmemBytes =
+      1024 + kStages * (kABytes + kBBytes) + kEpiStageBytes + kBarBytes;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 struct Args {
@@ -80,6 +93,9 @@ struct Args {
   // tail_part and are summed (slice order) by gemm_tail_fixup.
   int units, tail0, tail_split;
   float* tail_part;
+  // Whole 32-column chunks of a two-byte output go through the shared-memory
+  // boxes and the tensor maps tmO (out), tmO2 (out2) and tmX (aux).
+  int tma_out;
   int* status;
 };
 
@@ -153,13 +169,47 @@ __device__ __forceinline__ int k_coord(int kb, const Args& a) {
   return which * a.kr_h + g * a.kr_width + within * BK;
 }
 
+constexpr float kLog2e = 1.4426950408889634f;
+
+// The standard normal distribution at x: Phi(x) = (1 + erf(x / sqrt 2)) / 2
+// and phi(x) = exp(-x^2 / 2) / sqrt(2 pi), with erf by Abramowitz & Stegun,
+// "Handbook of Mathematical Functions", formula 7.1.26: for z >= 0,
+// erf z = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),
+// t = 1 / (1 + p z), |error| <= 1.5e-7, and erf(-z) = -erf z.  With
+// z = |x| / sqrt 2 the factor exp(-z^2) is the exp(-x^2 / 2) of phi, so one
+// reciprocal and one exponential give both.
+__device__ __forceinline__ void normal_cdf_pdf(float x, float& cdf, float& pdf) {
+  const float z = fabsf(x) * 0.70710678118654752f;
+  const float t = rcp_approx(fmaf(0.3275911f, z, 1.0f));
+  const float poly =
+      t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f),
+                     -0.284496736f),
+               0.254829592f);
+  const float e = ex2_approx(-0.5f * kLog2e * x * x);  // exp(-x^2 / 2)
+  const float q = 0.5f * poly * e;                      // (1 - erf z) / 2
+  cdf = x >= 0.0f ? 1.0f - q : q;
+  pdf = 0.39894228040143268f * e;
+}
+
+// GeLU(x) = x Phi(x) (the erf form).
 __device__ __forceinline__ float gelu_f(float x) {
-  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+  float cdf, pdf;
+  normal_cdf_pdf(x, cdf, pdf);
+  return x * cdf;
+}
+
+// GeLU(x) and GeLU'(x) = Phi(x) + x phi(x) from one evaluation.
+__device__ __forceinline__ void gelu_both_f(float x, float& g, float& gp) {
+  float cdf, pdf;
+  normal_cdf_pdf(x, cdf, pdf);
+  g = x * cdf;
+  gp = fmaf(x, pdf, cdf);
 }
 
 __device__ __forceinline__ float gelu_prime_f(float x) {
-  return 0.5f * (1.0f + erff(x * 0.70710678118654752f)) +
-         x * 0.39894228040143268f * expf(-0.5f * x * x);
+  float cdf, pdf;
+  normal_cdf_pdf(x, cdf, pdf);
+  return fmaf(x, pdf, cdf);
 }
 
 __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
@@ -251,11 +301,16 @@ __device__ __forceinline__ void epilogue_row32(float (&v)[32], int row, int col0
       if (a.out2 != nullptr) {
         float hh[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) hh[i] = gelu_f(y[i]);
+        for (int i = 0; i < 8; ++i) {
+          float gp;
+          gelu_both_f(y[i], hh[i], gp);
+          x[i] *= gp;
+        }
         *reinterpret_cast<uint4*>(a.out2 + (long long)row * a.ldo2 + col) = pack8(hh);
-      }
+      } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] *= gelu_prime_f(y[i]);
+        for (int i = 0; i < 8; ++i) x[i] *= gelu_prime_f(y[i]);
+      }
     }
     if (OUT == kOutF32) {
       float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + (long long)row * a.ldo + col);
@@ -272,7 +327,64 @@ __device__ __forceinline__ void epilogue_row32(float (&v)[32], int row, int col0
   if (OUT == kOutF16 && clamped) atomicCAS(a.status, 0, kStatusF16Range);
 }
 
-constexpr float kLog2e = 1.4426950408889634f;
+// Byte offset of 16-byte chunk j (0-3) of row r in a 32-row x 64-byte box
+// under the 64-byte swizzle (chunk index XOR address bits 7-8; the boxes are
+// 1024-byte aligned).
+__device__ __forceinline__ uint32_t sw64_off(int r, int j) {
+  return static_cast<uint32_t>(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+}
+
+// The epilogue of one row's 32 consecutive columns, all inside the tile's
+// column range, written to the warp's staging boxes (row r of a box = this
+// thread's lane): box0 holds the row of `aux` on entry for the epilogues
+// that read one and receives `out`; box1 receives out2.  Rows past M are
+// computed too and dropped by the TMA store.
+template <int EPI, int OUT>
+__device__ __forceinline__ void epilogue_box32(float (&v)[32], int r, int col0, uint8_t* box0,
+                                               uint8_t* box1, const Args& a) {
+  constexpr bool kAux = (EPI == kEpiResidual || EPI == kEpiDGelu);
+  bool clamped = false;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float* x = v + 8 * g;
+    const int col = col0 + 8 * g;
+    if (EPI != kEpiDGelu && a.bias != nullptr) {
+      float bb[8];
+      unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.bias) + col),
+              bb);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] += bb[i];
+    }
+    float y[8];
+    if (kAux) unpack8(*reinterpret_cast<const uint4*>(box0 + sw64_off(r, g)), y);
+    if (EPI == kEpiResidual) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] += y[i];
+    }
+    if (EPI == kEpiBiasGelu) {
+      if (a.out2 != nullptr) *reinterpret_cast<uint4*>(box1 + sw64_off(r, g)) = pack8(x);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = gelu_f(x[i]);
+    } else if (EPI == kEpiDGelu) {
+      if (a.out2 != nullptr) {
+        float hh[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float gp;
+          gelu_both_f(y[i], hh[i], gp);
+          x[i] *= gp;
+        }
+        *reinterpret_cast<uint4*>(box1 + sw64_off(r, g)) = pack8(hh);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] *= gelu_prime_f(y[i]);
+      }
+    }
+    *reinterpret_cast<uint4*>(box0 + sw64_off(r, g)) =
+        (OUT == kOutF16) ? pack8_f16(x, clamped) : pack8(x);
+  }
+  if (OUT == kOutF16 && clamped) atomicCAS(a.status, 0, kStatusF16Range);
+}
 
 // Cross-entropy epilogue on 32 consecutive columns (vocabulary entries) of
 // one row: "图解Transformer并行计算" §4.2 steps 1-2 for one chunk of a
@@ -280,9 +392,11 @@ constexpr float kLog2e = 1.4426950408889634f;
 // chunk statistics and the target logit all see the same values; the chunk's
 // maximum and its sum of exp(z - max) over its valid columns go to the
 // partial array.  col0 is 32-aligned within its shard and col_end - col0 is
-// a multiple of 8.
+// a multiple of 8.  With a staging box (whole chunks only) the logits go to
+// row `r` of the box instead of global memory.
 __device__ __forceinline__ void epilogue_ce32(float (&v)[32], int row, int col0, int col_end,
-                                              int tg, const Args& a) {
+                                              int tg, const Args& a, uint8_t* box = nullptr,
+                                              int r = 0) {
   if (row >= a.M) return;
   const int nv = min(32, col_end - col0);
   float mx = -INFINITY;
@@ -291,7 +405,10 @@ __device__ __forceinline__ void epilogue_ce32(float (&v)[32], int row, int col0,
     v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
     if (i < nv) mx = fmaxf(mx, v[i]);
   }
-  if (a.out != nullptr) {
+  if (box != nullptr) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) *reinterpret_cast<uint4*>(box + sw64_off(r, g)) = pack8(v + 8 * g);
+  } else if (a.out != nullptr) {
 #pragma unroll
     for (int g = 0; g < 4; ++g)
       if (8 * g < nv)
@@ -321,21 +438,68 @@ __device__ __forceinline__ void epilogue_ce32(float (&v)[32], int row, int col0,
   }
 }
 
+// One 32-column chunk of a whole tile through the warp's staging boxes:
+// wait until the previous chunk's TMA stores have read the boxes, fetch the
+// aux rows (TMA, counted on the warp's own barrier) while the accumulator
+// is read from tensor memory, apply the epilogue into the boxes and store
+// them with TMA.  Rows row0..row0+31 of the output are this warp's lanes.
+// Returns false if the wait for the aux box gave up.
+template <int EPI, int OUT>
+__device__ __forceinline__ bool epilogue_chunk_boxed(uint32_t taddr, int lane, int row, int row0,
+                                                     int col, int col_end, int tg, uint8_t* box0,
+                                                     uint8_t* box1, uint64_t* auxbar,
+                                                     uint32_t& aux_phase, const CUtensorMap* tmO,
+                                                     const CUtensorMap* tmO2,
+                                                     const CUtensorMap* tmX, const Args& a) {
+  constexpr bool kAux = (EPI == kEpiResidual || EPI == kEpiDGelu);
+  constexpr bool kOut2 = (EPI == kEpiBiasGelu || EPI == kEpiDGelu);
+  if (lane == 0) bulk_wait_read<0>();
+  __syncwarp();
+  if (kAux && lane == 0) {
+    mbar_arrive_expect_tx(auxbar, kEpiBoxBytes);
+    tma_load_2d(box0, tmX, auxbar, col, row0);
+  }
+  float v[32];
+  tmem_ld32(taddr, v);
+  if (kAux) {
+    const bool got = mbar_wait(auxbar, aux_phase, a.status, kStatusEpilogueTimeout);
+    aux_phase ^= 1u;
+    if (!__all_sync(0xffffffffu, got)) return false;
+  }
+  if constexpr (EPI == kEpiCE)
+    epilogue_ce32(v, row, col, col_end, tg, a, box0, lane);
+  else
+    epilogue_box32<EPI, OUT>(v, lane, col, box0, box1, a);
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmO, box0, col, row0);
+    if (kOut2 && a.out2 != nullptr) tma_store_2d(tmO2, box1, col, row0);
+    bulk_commit();
+  }
+  return true;
+}
+
 template <int BN, bool A_KMAJ, bool B_KMAJ, int EPI, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA,
-                      const __grid_constant__ CUtensorMap tmB, const Args args) {
+                      const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmO,
+                      const __grid_constant__ CUtensorMap tmO2,
+                      const __grid_constant__ CUtensorMap tmX, const Args args) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kStages * C::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+  uint8_t* sE = sB + C::kStages * C::kBBytes;  // epilogue boxes, 1024-byte aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(sE + kEpiStageBytes);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* auxbar = tempty + 2;  // one per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + kEpiWarps);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -349,11 +513,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], kEpiWarps);
     }
+    for (int i = 0; i < kEpiWarps; ++i) mbar_init(&auxbar[i], 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (args.tma_out) tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -452,9 +618,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - kFirstEpiWarp;
     const int quarter = warp & 3;  // tensor-memory lanes this warp may read
     const int half = ew >> 2;      // which half of the tile's columns
+    uint8_t* box0 = sE + ew * (2 * kEpiBoxBytes);
+    uint8_t* box1 = box0 + kEpiBoxBytes;
+    uint32_t aux_phase = 0;
+    bool ok = true;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
+    for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
       const Unit w = unit_of(u, args);
       const TileCoord tc = tile_coord<BN>(w.tile, args);
       if (!mbar_wait(&tfull[acc], acc_phase, args.status, kStatusEpilogueTimeout)) break;
@@ -465,18 +635,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < BN / 2; c += 32) {
         const int cl = half * (BN / 2) + c;
-        if (tc.n0 + cl >= tc.n_end) break;  // warp-uniform
+        const int col = tc.n0 + cl;
+        if (col >= tc.n_end) break;  // warp-uniform
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(acc * BN + cl);
+        if constexpr (OUT != kOutF32) {
+          if (args.tma_out && w.part < 0 && col + 32 <= tc.n_end) {
+            ok = epilogue_chunk_boxed<EPI, OUT>(taddr, lane, row, tc.m0 + quarter * 32, col,
+                                                tc.n_end, tg, box0, box1, &auxbar[ew], aux_phase,
+                                                &tmO, &tmO2, &tmX, args);
+            if (!ok) break;
+            continue;
+          }
+        }
         float v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                      static_cast<uint32_t>(acc * BN + cl),
-                  v);
+        tmem_ld32(taddr, v);
         if (w.part >= 0)  // a K slice of a tail tile: raw partial sums
           store_partial32(v, args.tail_part + (static_cast<long long>(w.part) * BM + lrow) * BN + cl);
         else if constexpr (EPI == kEpiCE)
-          epilogue_ce32(v, row, tc.n0 + cl, tc.n_end, tg, args);
+          epilogue_ce32(v, row, col, tc.n_end, tg, args);
         else
-          epilogue_row32<EPI, OUT, false>(v, row, tc.n0 + cl, tc.n_end, args);
+          epilogue_row32<EPI, OUT, false>(v, row, col, tc.n_end, args);
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -485,6 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    if (lane == 0) bulk_wait<0>();  // this warp's TMA stores have landed
   }
 
   __syncwarp();  // lane 0 of the producer / MMA warps rejoins its warp
@@ -505,7 +687,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kPairStages = 6;
 constexpr int kPairABytes = 128 * BK * 2;  // 16 KB: this CTA's half of A
 constexpr int kPairBBytes = 128 * BK * 2;  // 16 KB: this CTA's half of B
-constexpr int kPairSmemBytes = 1024 + kPairStages * (kPairABytes + kPairBBytes) + 256;
+constexpr int kPairSmemBytes =
+    1024 + kPairStages * (kPairABytes + kPairBBytes) + kEpiStageBytes + kBarBytes;
+static_assert(kPairSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kPairTM = 256, kPairTN = 256;
 
 __device__ __forceinline__ TileCoord tile_coord_pair(int tile, const Args& a) {
@@ -533,17 +717,22 @@ __device__ __forceinline__ TileCoord tile_coord_pair(int tile, const Args& a) {
 template <bool A_KMAJ, bool B_KMAJ, int EPI, int OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmA,
-                           const __grid_constant__ CUtensorMap tmB, const Args args) {
+                           const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmO,
+                           const __grid_constant__ CUtensorMap tmO2,
+                           const __grid_constant__ CUtensorMap tmX, const Args args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kPairStages * kPairABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPairStages * kPairBBytes);
+  uint8_t* sE = sB + kPairStages * kPairBBytes;  // epilogue boxes, 1024-byte aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(sE + kEpiStageBytes);
   uint64_t* empty = full + kPairStages;
   uint64_t* tfull = empty + kPairStages;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* auxbar = tempty + 2;  // one per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + kEpiWarps);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -559,11 +748,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 2 * kEpiWarps);  // both CTAs' epilogue warps
     }
+    for (int i = 0; i < kEpiWarps; ++i) mbar_init(&auxbar[i], 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (args.tma_out) tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -670,9 +861,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int half = ew >> 2;
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0),
                                        mapa_shared(smem_u32(&tempty[1]), 0)};
+    uint8_t* box0 = sE + ew * (2 * kEpiBoxBytes);
+    uint8_t* box1 = box0 + kEpiBoxBytes;
+    uint32_t aux_phase = 0;
+    bool ok = true;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = cluster_id; u < args.units; u += num_clusters) {
+    for (int u = cluster_id; u < args.units && ok; u += num_clusters) {
       const Unit w = unit_of(u, args);
       const TileCoord tc = tile_coord_pair(w.tile, args);
       if (!mbar_wait(&tfull[acc], acc_phase, args.status, kStatusEpilogueTimeout)) break;
@@ -683,19 +878,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < kPairTN / 2; c += 32) {
         const int cl = half * (kPairTN / 2) + c;
-        if (tc.n0 + cl >= tc.n_end) break;  // warp-uniform
+        const int col = tc.n0 + cl;
+        if (col >= tc.n_end) break;  // warp-uniform
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(acc * kPairTN + cl);
+        if constexpr (OUT != kOutF32) {
+          if (args.tma_out && w.part < 0 && col + 32 <= tc.n_end) {
+            ok = epilogue_chunk_boxed<EPI, OUT>(
+                taddr, lane, row, tc.m0 + 128 * static_cast<int>(rank) + quarter * 32, col,
+                tc.n_end, tg, box0, box1, &auxbar[ew], aux_phase, &tmO, &tmO2, &tmX, args);
+            if (!ok) break;
+            continue;
+          }
+        }
         float v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                      static_cast<uint32_t>(acc * kPairTN + cl),
-                  v);
+        tmem_ld32(taddr, v);
         if (w.part >= 0)  // a K slice of a tail tile: raw partial sums
           store_partial32(v, args.tail_part +
                                  (static_cast<long long>(w.part) * kPairTM + lrow) * kPairTN + cl);
         else if constexpr (EPI == kEpiCE)
-          epilogue_ce32(v, row, tc.n0 + cl, tc.n_end, tg, args);
+          epilogue_ce32(v, row, col, tc.n_end, tg, args);
         else
-          epilogue_row32<EPI, OUT, false>(v, row, tc.n0 + cl, tc.n_end, args);
+          epilogue_row32<EPI, OUT, false>(v, row, col, tc.n_end, args);
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
@@ -704,6 +910,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    if (lane == 0) bulk_wait<0>();  // this warp's TMA stores have landed
   }
   (void)peer;
 
@@ -808,6 +1015,43 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t inner, int64_t outer, int
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Tensor map of the epilogue's 32 x 32 boxes of a row-major two-byte matrix
+// with `cols` columns, `rows` rows and leading dimension `ld`, 64-byte
+// swizzle (the layout sw64_off addresses).
+bool make_box_map(CUtensorMap* m, const void* ptr, int64_t cols, int64_t rows, int64_t ld) {
+  auto fn = encode_fn();
+  if (fn == nullptr || ptr == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The epilogue's tensor maps: output, second output, operand read.
+struct EpiMaps {
+  CUtensorMap o, o2, x;
+};
+
+// Encodes the maps the boxed epilogue needs; false (the epilogue then stores
+// directly) for fp32 outputs, a missing output, or a matrix a tensor map
+// cannot describe.
+template <int EPI, int OUT>
+bool make_epi_maps(const Gemm& g, EpiMaps& e) {
+  std::memset(&e, 0, sizeof(e));
+  if (OUT == kOutF32 || g.out == nullptr) return false;
+  if (!make_box_map(&e.o, g.out, g.N, g.M, g.ldo)) return false;
+  if ((EPI == kEpiBiasGelu || EPI == kEpiDGelu) && g.out2 != nullptr &&
+      !make_box_map(&e.o2, g.out2, g.N, g.M, g.ldo2))
+    return false;
+  if ((EPI == kEpiResidual || EPI == kEpiDGelu) && !make_box_map(&e.x, g.aux, g.N, g.M, g.ldaux))
+    return false;
+  return true;
 }
 
 struct Plan {
@@ -918,6 +1162,8 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   a.ce_tlogit = g.ce.tlogit;
   a.status = device_status_ptr();
   if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
+  EpiMaps em;
+  a.tma_out = make_epi_maps<EPI, OUT>(g, em) ? 1 : 0;
 
   auto kern = gemm_bf16_tcgen05<BN, AK, BKM, EPI, OUT>;
   static int configured_mask = 0;  // one bit per device
@@ -946,7 +1192,7 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   {
     LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, tp.split > 1 ? 2 : 1, BN, g.M,
                       g.N, g.K);
-    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(ta, tb, a);
+    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(ta, tb, em.o, em.o2, em.x, a);
     if (tp.split > 1)
       gemm_tail_fixup<BM, BN, false, EPI, OUT>
           <<<dim3(static_cast<unsigned>(tiles - tp.tail0), kFixupRowGroups), 256, 0, stream>>>(a);
@@ -1024,6 +1270,8 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   a.ce_tlogit = g.ce.tlogit;
   a.status = device_status_ptr();
   if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
+  EpiMaps em;
+  a.tma_out = make_epi_maps<EPI, OUT>(g, em) ? 1 : 0;
 
   auto kern = gemm_bf16_tcgen05_pair<AK, BKM, EPI, OUT>;
   static int configured_mask = 0;
@@ -1064,7 +1312,7 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   {
     LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, tp.split > 1 ? 2 : 1, 512, g.M,
                       g.N, g.K);
-    kern<<<2 * clusters, kThreads, kPairSmemBytes, stream>>>(ta, tb, a);
+    kern<<<2 * clusters, kThreads, kPairSmemBytes, stream>>>(ta, tb, em.o, em.o2, em.x, a);
     if (tp.split > 1)
       gemm_tail_fixup<kPairTM, kPairTN, true, EPI, OUT>
           <<<dim3(static_cast<unsigned>(tiles - tp.tail0), kFixupRowGroups), 256, 0, stream>>>(a);

@@ -14,20 +14,13 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "ptx_sm100.cuh"
 #include "tp_internal.h"
 
 namespace tp {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-
-// 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz;
-// relative error about 2^-22, far below the bf16 rounding of its uses here).
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // ------------------------------------------------------------------ embedding
 

@@ -142,3 +142,43 @@ def test_mlp_single_token(dtype):
                   dtype="f32" if dtype == torch.float32 else "bf16")
     inp = make_mlp_inputs(wl)
     compare_full(gpu_mlp(inp, wl.t, dtype=dtype), inp, "f32" if dtype == torch.float32 else "bf16")
+
+
+def _bf16_ulp(v):
+    """The spacing of bf16 numbers at |v| (8 significant bits)."""
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def test_gelu_epilogues_against_exact_erf():
+    """The GeLU of the first GEMM's epilogue, the GeLU' of the dgrad epilogue
+    and the GeLU the dgrad epilogue recomputes for dB, each against the erf
+    form in fp64 (the oracle's), on one token whose h = 2048 entries sweep
+    [-8, 8] plus special values.  With A = B = I the MLP exposes them
+    exactly: Z = bf16(GeLU(x)) (one product per output), and with dZ = 1
+    the backward gives dbA = bf16(GeLU'(x)) and every column of dB =
+    bf16(GeLU(x)).  The bound is half a bf16 unit of the exact value (the
+    rounding) plus 1e-6 (times |x| for GeLU): the erf approximation's
+    absolute error of 1.5e-7 with the approximate reciprocal, exponential
+    and fp32 rounding on top, still far below a bf16 unit."""
+    h = 2048
+    x = np.linspace(-8.0, 8.0, h)
+    x[:8] = [0.0, 1e-3, -1e-3, 1e-30, -1e-30, 0.5, -0.5, -13.0]
+    X = torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).reshape(1, h)
+    xb = X.double().numpy().ravel()
+    eye = torch.eye(h, dtype=torch.bfloat16)
+    inp = {"X": X, "A": eye, "B": eye.clone(), "bA": None, "bB": None,
+           "dZ": torch.ones(1, h, dtype=torch.bfloat16)}
+    out = gpu_mlp(inp, t=2)
+    g_exact, gp_exact = O.gelu(xb), O.gelu_prime(xb)
+    z = out["Z"].double().cpu().numpy().ravel()
+    dba = out["dbA"].double().cpu().numpy().ravel()
+    db0 = out["dB"][:, 0].double().cpu().numpy().ravel()
+    tol_g = 0.5 * _bf16_ulp(g_exact) + np.abs(xb) * 1e-6 + 1e-30
+    tol_gp = 0.5 * _bf16_ulp(gp_exact) + 1e-6
+    assert np.all(np.abs(z - g_exact) <= tol_g), np.max(np.abs(z - g_exact) / tol_g)
+    assert np.all(np.abs(dba - gp_exact) <= tol_gp), np.max(np.abs(dba - gp_exact) / tol_gp)
+    assert np.all(np.abs(db0 - g_exact) <= tol_g)
+    # The forward and the backward evaluate GeLU the same way, bit for bit.
+    assert np.array_equal(z, db0)
+    assert np.array_equal(out["Y"].double().cpu().numpy().ravel(), xb)
