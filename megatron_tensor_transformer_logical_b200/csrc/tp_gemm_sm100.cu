@@ -37,6 +37,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -1166,14 +1167,17 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   a.tma_out = make_epi_maps<EPI, OUT>(g, em) ? 1 : 0;
 
   auto kern = gemm_bf16_tcgen05<BN, AK, BKM, EPI, OUT>;
-  static int configured_mask = 0;  // one bit per device
+  // Shared-memory opt-in once per device (devices past 31 every launch);
+  // two threads may both set it, which is harmless.
+  static std::atomic<unsigned> configured{0};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(configured_mask & (1 << (dev & 31)))) {
+  const unsigned bit = (dev >= 0 && dev < 32) ? (1u << dev) : 0u;
+  if (bit == 0 || !(configured.load(std::memory_order_acquire) & bit)) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-    configured_mask |= 1 << (dev & 31);
+    configured.fetch_or(bit, std::memory_order_release);
   }
   const long long tiles = static_cast<long long>(p.m_tiles) * p.n_tiles;
   if (tiles == 0) return TP_OK;
@@ -1274,11 +1278,18 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   a.tma_out = make_epi_maps<EPI, OUT>(g, em) ? 1 : 0;
 
   auto kern = gemm_bf16_tcgen05_pair<AK, BKM, EPI, OUT>;
-  static int configured_mask = 0;
-  static int max_clusters[32] = {};
+  // Shared-memory opt-in and the number of co-resident pairs, once per
+  // device (devices past 31 every launch); concurrent first calls compute
+  // the same values.
+  static std::atomic<unsigned> configured{0};
+  static std::atomic<int> max_clusters[32];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(configured_mask & (1 << (dev & 31)))) {
+  const unsigned bit = (dev >= 0 && dev < 32) ? (1u << dev) : 0u;
+  int mc = 0;
+  if (bit != 0 && (configured.load(std::memory_order_acquire) & bit)) {
+    mc = max_clusters[dev].load(std::memory_order_relaxed);
+  } else {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
@@ -1286,17 +1297,17 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
     cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kPairSmemBytes;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+    if (cudaOccupancyMaxActiveClusters(&mc, kern, &cfg) != cudaSuccess || mc <= 0) {
       cudaGetLastError();
-      n = sm_count() / 2;
+      mc = sm_count() / 2;
     }
-    max_clusters[dev & 31] = n;
-    configured_mask |= 1 << (dev & 31);
+    if (bit != 0) {
+      max_clusters[dev].store(mc, std::memory_order_relaxed);
+      configured.fetch_or(bit, std::memory_order_release);
+    }
   }
   const long long tiles = static_cast<long long>(a.m_tiles) * a.n_tiles;
   if (tiles == 0) return TP_OK;
-  const int mc = max_clusters[dev & 31];
   const int clusters = static_cast<int>(tiles < mc ? tiles : mc);
   const TailPlan tp = plan_tail(tiles, clusters, a.k_blocks, size_t(kPairTM) * kPairTN * 4, g, EPI);
   a.units = tp.units;
