@@ -686,8 +686,8 @@ def run_libtp(args, ranks: Ranks):
         out["e2e"] = {"value": round(job_rate(fl["total"], world, e2e_ms, args.steps) / 1e12, 2),
                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                       "ms_per_step": round(e2e_ms / args.steps, 4)}
-    if not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, seconds_hint=args.cpu_sample_tokens)
+    if not args.no_cpu_baseline and world == 1:  # the oracle baseline: rank 0 at N = 1 only
+        out["cpu_baseline"] = cpu_baseline(wl, tokens=args.cpu_sample_tokens)
     return out
 
 
@@ -724,8 +724,10 @@ def oracle_layer_sample(wl, tokens: int, mi=None, ai=None):
     return fn, layer_flops(1, tokens, wl.h, wl.f, wl.heads)["total"]
 
 
-def cpu_baseline(wl, seconds_hint=512):
-    tokens = int(seconds_hint)
+def cpu_baseline(wl, tokens=768):
+    """The oracle as it stands, timed once on the host's cores on the first
+    `tokens` tokens of the layer (exact under the causal mask)."""
+    tokens = int(tokens)
     fn, flops = oracle_layer_sample(wl, tokens)
     t0 = time.perf_counter()
     fn()
@@ -776,7 +778,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-vocab", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=384)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=768)
     ap.add_argument("--ref-sample-tokens", type=int, default=64)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "libtp":
