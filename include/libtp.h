@@ -449,6 +449,32 @@ tp_status tp_device_status(void* stream);
 /* Library version, major * 10000 + minor * 100 + patch. */
 int tp_version(void);
 
+/*
+ * Work plan of the tensor-core GEMM, for tests of its tile scheduler (host
+ * only: no device, no CUDA call).  For D[M, N] = A[M, K] B[K, N] with tile
+ * kind `kind` (128, 192 or 256 output columns per tile on one SM with 128
+ * rows, or 512 = 256 x 256 tiles on an SM pair), column shards of width
+ * `n_shard` (0: none; a width the GEMM cannot align to 8 columns tiles
+ * plainly, as in every entry point), a device of `sms` SMs, and with
+ * (tail_scratch = 1) or without the optional last-wave scratch of the
+ * workspaces, the units the persistent kernel hands out in order: unit u
+ * runs on CTA (or pair) u mod workers.  A whole tile is one unit (part = -1);
+ * the tiles of a short last wave may be split into K slices (part >= 0, the
+ * index of the slice's fp32 partial tile), summed afterwards in slice order.
+ *   out   up to `cap` units (may be NULL to count only), caller-owned HOST memory
+ * Returns the number of units, or -1 for invalid arguments (a size <= 0,
+ * sms < 2, an unknown kind).
+ */
+typedef struct tp_gemm_unit {
+  int32_t m0, rows;    /* output rows [m0, m0 + rows) (clipped to M)            */
+  int32_t n0, n_end;   /* output columns [n0, n_end)                            */
+  int32_t kb0, kb1;    /* K blocks [kb0, kb1), 64 deep                          */
+  int32_t part;        /* partial-tile index of a K slice, -1 for a whole tile  */
+  int32_t tile;        /* output tile index                                     */
+} tp_gemm_unit;
+int64_t tp_gemm_plan(int64_t M, int64_t N, int64_t K, int64_t n_shard, int kind, int sms,
+                     int tail_scratch, tp_gemm_unit* out, int64_t cap);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

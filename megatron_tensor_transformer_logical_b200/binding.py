@@ -35,7 +35,7 @@ EXPORTS = ("tp_linear_col", "tp_linear_row", "tp_mlp_fwd", "tp_mlp_bwd", "tp_att
            "tp_version", "tp_profile_enable", "tp_profile_read", "tp_launch_count",
            "tp_mlp_fwd_noalloc", "tp_profile_count", "tp_profile_record", "tp_layernorm_fwd",
            "tp_layernorm_bwd", "tp_block_fwd", "tp_block_bwd", "tp_vocab_embed_fwd",
-           "tp_vocab_embed_bwd", "tp_vocab_ce_fwd", "tp_vocab_ce_bwd")
+           "tp_vocab_embed_bwd", "tp_vocab_ce_fwd", "tp_vocab_ce_bwd", "tp_gemm_plan")
 
 _W_FIELDS = ("ln1_g", "ln1_b", "Wqkv", "Wo", "ln2_g", "ln2_b", "A", "bA", "B", "bB")
 _S_FIELDS = ("Xn1", "mean1", "rstd1", "QKV", "O", "LSE", "X1", "Xn2", "mean2", "rstd2", "Y")
@@ -58,6 +58,11 @@ class LaunchRecord(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("tile", ctypes.c_int), ("m", ctypes.c_int64),
                 ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("ms", ctypes.c_double),
                 ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
+class GemmUnit(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("m0", "rows", "n0", "n_end", "kb0", "kb1", "part",
+                                              "tile")]
 
 
 class ProfileStats(ctypes.Structure):
@@ -119,11 +124,13 @@ def load() -> ctypes.CDLL:
     L.tp_profile_count.argtypes = []
     L.tp_profile_count.restype = ctypes.c_int64
     L.tp_profile_record.argtypes = [ctypes.c_int64, ctypes.POINTER(LaunchRecord)]
+    L.tp_gemm_plan.argtypes = [i64, i64, i64, i64, i32, i32, i32, ctypes.POINTER(GemmUnit), i64]
     for name in EXPORTS:
         if name not in ("tp_workspace_size", "tp_last_error", "tp_launch_count",
-                        "tp_profile_count"):
+                        "tp_profile_count", "tp_gemm_plan"):
             getattr(L, name).restype = ctypes.c_int
     L.tp_launch_count.restype = ctypes.c_int64
+    L.tp_gemm_plan.restype = ctypes.c_int64
     _lib = L
     return L
 
@@ -325,6 +332,20 @@ def tp_profile_records() -> list:
         out.append({"kind": KIND_NAMES.get(r.kind, str(r.kind)), "tile": r.tile, "m": r.m,
                     "n": r.n, "k": r.k, "ms": r.ms, "flops": r.flops, "bytes": r.bytes})
     return out
+
+
+def tp_gemm_plan(M: int, N: int, K: int, n_shard: int, kind: int, sms: int,
+                 tail_scratch: bool) -> list:
+    """The tensor-core GEMM's work units for one shape (host only), as dicts
+    with m0, rows, n0, n_end, kb0, kb1, part, tile; raises on bad sizes."""
+    L = load()
+    n = int(L.tp_gemm_plan(M, N, K, n_shard, kind, sms, int(tail_scratch), None, 0))
+    if n < 0:
+        raise TPError(TP_ERR_SHAPE, "invalid GEMM plan request")
+    buf = (GemmUnit * max(n, 1))()
+    got = int(L.tp_gemm_plan(M, N, K, n_shard, kind, sms, int(tail_scratch), buf, n))
+    assert got == n
+    return [{f: getattr(buf[i], f) for f, _ in GemmUnit._fields_} for i in range(n)]
 
 
 def workspace(op: int, M: int, h: int, f: int, heads: int, t: int, dtype: int,

@@ -1050,4 +1050,21 @@ tp_status tp_profile_record(int64_t index, tp_launch_record* out) {
 
 int tp_version(void) { return 100; }
 
+int64_t tp_gemm_plan(int64_t M, int64_t N, int64_t K, int64_t n_shard, int kind, int sms,
+                     int tail_scratch, tp_gemm_unit* out, int64_t cap) {
+  try {
+    const int64_t want = (out != nullptr && cap > 0) ? cap : 0;
+    std::vector<tp::GemmPlanUnit> units(static_cast<size_t>(want));
+    const int64_t n = tp::gemm_plan_units(M, N, K, n_shard, kind, sms, tail_scratch != 0,
+                                          units.data(), want);
+    for (int64_t i = 0; i < n && i < want; ++i) {
+      const tp::GemmPlanUnit& u = units[static_cast<size_t>(i)];
+      out[i] = tp_gemm_unit{u.m0, u.rows, u.n0, u.n_end, u.kb0, u.kb1, u.part, u.tile};
+    }
+    return n;
+  } catch (...) {
+    return -1;
+  }
+}
+
 }  // extern "C"

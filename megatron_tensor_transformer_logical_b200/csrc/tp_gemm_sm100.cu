@@ -105,7 +105,7 @@ struct Unit {
   int part;  // index of the partial tile, -1 for a whole tile
 };
 
-__device__ __forceinline__ Unit unit_of(int u, const Args& a) {
+__host__ __device__ __forceinline__ Unit unit_of(int u, const Args& a) {
   Unit w;
   if (u < a.tail0) {
     w.tile = u;
@@ -139,7 +139,7 @@ struct TileCoord {
 // varies fastest, so the CTAs running at one time share B tiles and the
 // band's A rows stay in L2.
 template <int BN>
-__device__ __forceinline__ TileCoord tile_coord(int tile, const Args& a) {
+__host__ __device__ __forceinline__ TileCoord tile_coord(int tile, const Args& a) {
   const int band = a.group_m * a.n_tiles;
   const int g = tile / band;
   const int first_m = g * a.group_m;
@@ -693,7 +693,7 @@ constexpr int kPairSmemBytes =
 static_assert(kPairSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kPairTM = 256, kPairTN = 256;
 
-__device__ __forceinline__ TileCoord tile_coord_pair(int tile, const Args& a) {
+__host__ __device__ __forceinline__ TileCoord tile_coord_pair(int tile, const Args& a) {
   const int band = a.group_m * a.n_tiles;
   const int g = tile / band;
   const int first_m = g * a.group_m;
@@ -970,15 +970,15 @@ struct TailPlan {
   int units, tail0, split;
 };
 
-TailPlan plan_tail(long long tiles, int workers, int k_blocks, size_t part_bytes, const Gemm& g,
-                   int epi) {
+TailPlan plan_tail(long long tiles, int workers, int k_blocks, size_t part_bytes,
+                   size_t scratch_bytes, int epi) {
   TailPlan tp{static_cast<int>(tiles), static_cast<int>(tiles), 1};
-  if (epi == kEpiCE || g.tail_ws == nullptr || tiles <= workers) return tp;
+  if (epi == kEpiCE || scratch_bytes == 0 || tiles <= workers) return tp;
   const long long R = tiles % workers;
   if (R == 0 || 2 * R > workers) return tp;
   int S = static_cast<int>(workers / R);
   if (S > k_blocks / 32) S = k_blocks / 32;
-  if (S < 2 || static_cast<size_t>(R) * S * part_bytes > g.tail_ws_bytes) return tp;
+  if (S < 2 || static_cast<size_t>(R) * S * part_bytes > scratch_bytes) return tp;
   tp.tail0 = static_cast<int>(tiles - R);
   tp.split = S;
   tp.units = tp.tail0 + static_cast<int>(R) * S;
@@ -1074,6 +1074,44 @@ Plan plan_for(const Gemm& g, int bn) {
   return p;
 }
 
+// The tile grid and raster of one GEMM in kernel arguments: 128 x bn tiles
+// on one SM, or 256 x 256 tiles on an SM pair (pair = true, bn = 256).
+// Shared by the launchers and tp_gemm_plan.
+Args plan_args(const Gemm& g, int bn, bool pair) {
+  const Plan p = plan_for(g, bn);
+  Args a{};
+  a.M = static_cast<int>(g.M);
+  a.N = static_cast<int>(g.N);
+  a.K = static_cast<int>(g.K);
+  a.m_tiles = pair ? static_cast<int>((g.M + kPairTM - 1) / kPairTM) : p.m_tiles;
+  a.n_tiles = p.n_tiles;
+  a.k_blocks = static_cast<int>((g.K + BK - 1) / BK);
+  a.group_m = pair ? 8 : 16;
+  a.n_shard = static_cast<int>(g.n_shard);
+  a.n_tiles_per_shard = p.n_tiles_per_shard;
+  a.kr_range_blocks = g.korder.range_blocks;
+  a.kr_t = g.korder.t;
+  a.kr_width = g.korder.width;
+  a.kr_h = g.korder.h;
+  a.units = a.tail0 = static_cast<int>(static_cast<long long>(a.m_tiles) * a.n_tiles);
+  a.tail_split = 1;
+  return a;
+}
+
+// The last-wave K split of `a`'s tiles on `workers` persistent CTAs (or
+// pairs) with partial tiles of `part_bytes` in `scratch_bytes` of caller
+// scratch (0: none), written into a.
+TailPlan plan_tail_args(Args& a, int workers, size_t part_bytes, size_t scratch_bytes, int epi) {
+  const long long tiles = static_cast<long long>(a.m_tiles) * a.n_tiles;
+  const TailPlan tp = plan_tail(tiles, workers, a.k_blocks, part_bytes, scratch_bytes, epi);
+  a.units = tp.units;
+  a.tail0 = tp.tail0;
+  a.tail_split = tp.split;
+  return tp;
+}
+
+size_t tail_bytes(const Gemm& g) { return g.tail_ws != nullptr ? g.tail_ws_bytes : 0; }
+
 // Tile override for tests and tuning: TP_GEMM_TILE = 128 | 256 | pair.
 int tile_override() {
   const char* e = std::getenv("TP_GEMM_TILE");
@@ -1134,21 +1172,7 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
                         : make_map(&tb, g.b.ptr, g.N, g.K, g.b.ld, 64, BK);
   if (!ok_a || !ok_b) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 
-  const Plan p = plan_for(g, BN);
-  Args a;
-  a.M = static_cast<int>(g.M);
-  a.N = static_cast<int>(g.N);
-  a.K = static_cast<int>(g.K);
-  a.m_tiles = p.m_tiles;
-  a.n_tiles = p.n_tiles;
-  a.k_blocks = static_cast<int>((g.K + BK - 1) / BK);
-  a.group_m = 16;
-  a.n_shard = static_cast<int>(g.n_shard);
-  a.n_tiles_per_shard = p.n_tiles_per_shard;
-  a.kr_range_blocks = g.korder.range_blocks;
-  a.kr_t = g.korder.t;
-  a.kr_width = g.korder.width;
-  a.kr_h = g.korder.h;
+  Args a = plan_args(g, BN, false);
   a.out = g.out;
   a.ldo = g.ldo;
   a.bias = g.bias;
@@ -1179,13 +1203,10 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
     configured.fetch_or(bit, std::memory_order_release);
   }
-  const long long tiles = static_cast<long long>(p.m_tiles) * p.n_tiles;
+  const long long tiles = static_cast<long long>(a.m_tiles) * a.n_tiles;
   if (tiles == 0) return TP_OK;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  const TailPlan tp = plan_tail(tiles, grid, a.k_blocks, size_t(BM) * BN * 4, g, EPI);
-  a.units = tp.units;
-  a.tail0 = tp.tail0;
-  a.tail_split = tp.split;
+  const TailPlan tp = plan_tail_args(a, grid, size_t(BM) * BN * 4, tail_bytes(g), EPI);
   a.tail_part = static_cast<float*>(g.tail_ws);
   const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
@@ -1245,21 +1266,7 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   const bool ok_b = BKM ? make_map(&tb, g.b.ptr, g.K, g.N, g.b.ld, BK, 128)
                         : make_map(&tb, g.b.ptr, g.N, g.K, g.b.ld, 64, BK);
   if (!ok_a || !ok_b) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-  const Plan p = plan_for(g, kPairTN);
-  Args a;
-  a.M = static_cast<int>(g.M);
-  a.N = static_cast<int>(g.N);
-  a.K = static_cast<int>(g.K);
-  a.m_tiles = static_cast<int>((g.M + kPairTM - 1) / kPairTM);
-  a.n_tiles = p.n_tiles;
-  a.k_blocks = static_cast<int>((g.K + BK - 1) / BK);
-  a.group_m = 8;
-  a.n_shard = static_cast<int>(g.n_shard);
-  a.n_tiles_per_shard = p.n_tiles_per_shard;
-  a.kr_range_blocks = g.korder.range_blocks;
-  a.kr_t = g.korder.t;
-  a.kr_width = g.korder.width;
-  a.kr_h = g.korder.h;
+  Args a = plan_args(g, kPairTN, true);
   a.out = g.out;
   a.ldo = g.ldo;
   a.bias = g.bias;
@@ -1309,10 +1316,8 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   const long long tiles = static_cast<long long>(a.m_tiles) * a.n_tiles;
   if (tiles == 0) return TP_OK;
   const int clusters = static_cast<int>(tiles < mc ? tiles : mc);
-  const TailPlan tp = plan_tail(tiles, clusters, a.k_blocks, size_t(kPairTM) * kPairTN * 4, g, EPI);
-  a.units = tp.units;
-  a.tail0 = tp.tail0;
-  a.tail_split = tp.split;
+  const TailPlan tp =
+      plan_tail_args(a, clusters, size_t(kPairTM) * kPairTN * 4, tail_bytes(g), EPI);
   a.tail_part = static_cast<float*>(g.tail_ws);
   const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
@@ -1368,6 +1373,43 @@ size_t gemm_tail_scratch_bytes() {
   // At most one partial tile per persistent CTA (128 x 256 fp32) or per CTA
   // pair (256 x 256 fp32, half as many pairs).
   return static_cast<size_t>(sm_count()) * 128 * 256 * 4;
+}
+
+int64_t gemm_plan_units(int64_t M, int64_t N, int64_t K, int64_t n_shard, int kind, int sms,
+                        bool tail_scratch, GemmPlanUnit* out, int64_t cap) {
+  if (M <= 0 || N <= 0 || K <= 0 || sms < 2 || n_shard < 0 || cap < 0 ||
+      (kind != 128 && kind != 192 && kind != 256 && kind != 512))
+    return -1;
+  if (M > (1ll << 31) - BM || N > (1ll << 31) - 256 || K > (1ll << 31) - BK) return -1;
+  Gemm g;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  // the same shard normalisation as launch_gemm_bf16
+  g.n_shard = (n_shard > 0 && n_shard % 8 == 0 && N % n_shard == 0) ? n_shard : 0;
+  const bool pair = kind == 512;
+  const int bn = pair ? kPairTN : kind;
+  Args a = plan_args(g, bn, pair);
+  const long long tiles = static_cast<long long>(a.m_tiles) * a.n_tiles;
+  const int slots = pair ? sms / 2 : sms;  // persistent CTAs, or pairs
+  const int workers = static_cast<int>(tiles < slots ? tiles : slots);
+  const size_t scratch = tail_scratch ? static_cast<size_t>(sms) * 128 * 256 * 4 : 0;
+  plan_tail_args(a, workers, size_t(pair ? kPairTM : BM) * bn * 4, scratch, kEpiStore);
+  for (int u = 0; u < a.units && u < cap && out != nullptr; ++u) {
+    const Unit w = unit_of(u, a);
+    TileCoord tc;
+    if (pair)
+      tc = tile_coord_pair(w.tile, a);
+    else if (bn == 128)
+      tc = tile_coord<128>(w.tile, a);
+    else if (bn == 192)
+      tc = tile_coord<192>(w.tile, a);
+    else
+      tc = tile_coord<256>(w.tile, a);
+    out[u] = GemmPlanUnit{tc.m0, pair ? kPairTM : BM, tc.n0, tc.n_end, w.kb0, w.kb1, w.part,
+                          w.tile};
+  }
+  return a.units;
 }
 
 tp_status launch_gemm_bf16(const Gemm& g, cudaStream_t stream) {

@@ -105,6 +105,21 @@ struct Gemm {
 // Scratch that lets a tcgen05 GEMM split its last wave along K.
 size_t gemm_tail_scratch_bytes();
 
+// One unit of a GEMM work plan: output rows [m0, m0 + rows), columns
+// [n0, n_end), K blocks [kb0, kb1) of 64; part = partial-tile index of a K
+// slice, -1 for a whole tile; tile = the output tile's index.
+struct GemmPlanUnit {
+  int m0, rows, n0, n_end, kb0, kb1, part, tile;
+};
+
+// The units the tcgen05 GEMM would run for D[M, N] = A[M, K] B[K, N] with
+// tile kind 128 / 192 / 256 (one SM) or 512 (256 x 256 on an SM pair), column
+// shards of width n_shard (0: none) and `sms` SMs, with or without the
+// last-wave scratch; host only.  Writes up to cap units to out; returns the
+// number of units, -1 for invalid arguments.
+int64_t gemm_plan_units(int64_t M, int64_t N, int64_t K, int64_t n_shard, int kind, int sms,
+                        bool tail_scratch, GemmPlanUnit* out, int64_t cap);
+
 // The smallest workspace tp_mlp_fwd accepts (without the optional GEMM tail
 // scratch that tp_workspace_size() adds).
 size_t mlp_fwd_ws_min(int64_t M, int64_t f, tp_dtype d);
