@@ -28,7 +28,6 @@ namespace tp {
 namespace {
 
 constexpr int D = 128;            // head dimension
-constexpr int ROW_BYTES = D * 2;  // 256 bytes per row of a [rows][128] bf16 tile
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnArgs {
