@@ -108,7 +108,9 @@ tp_status tp_linear_row(const void* X, const void* W, const void* bias, void* Z,
 
 /*
  * Partitioned MLP forward ([P3] §2.1 steps 1-3, §2.2 MLP_forward_TP):
- *   shard i: Y_i = X @ A_i + bA_i;  H_i = GeLU(Y_i)  (exact erf GeLU, [P2] §3.3);
+ *   shard i: Y_i = X @ A_i + bA_i;  H_i = GeLU(Y_i)  (the erf GeLU, [P2] §3.3:
+ *   fp32 erff for TP_F32; for TP_BF16 erf to within 1.5e-7 (Abramowitz &
+ *   Stegun 7.1.26), far below the bf16 rounding of H);
  *   Z = sum_i H_i @ B_i + bB   (A split by columns, B by rows, f = 4h typically).
  *   X [M, h]; A [h, f]; bA [f] or NULL; B [f, h]; bB [h] or NULL; Z [M, h];
  *   Ysave [M, f] or NULL: receives the pre-activation Y for the backward.
