@@ -4,7 +4,10 @@
 // the causal mask hiding key c from query r when c > r; each head group of
 // §3.2 runs its own heads, so the core runs per (batch, head).
 //
-// One CTA per (batch element, head, 128 query rows), longest rows first:
+// One CTA per (batch element, head, 128 query rows); blockIdx.x is the
+// (batch element, head) and blockIdx.y the row tile, longest rows first, so
+// the CTAs launch in order of decreasing work over all heads (the longest
+// tiles of the last heads do not start in the last wave):
 //   warp 0     TMA: the Q tile once, then K_j and V_j (128 keys each) into a
 //              two-deep ring (fp16, 128-byte swizzle);
 //   warp 1     allocates 512 TMEM columns; one thread issues
@@ -90,8 +93,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (a.s + kBM - 1) / kBM;
-  const int qb = nqb - 1 - static_cast<int>(blockIdx.x);  // longest rows first
-  const int head = blockIdx.y % a.heads, bi = blockIdx.y / a.heads;
+  const int qb = nqb - 1 - static_cast<int>(blockIdx.y);  // longest rows first
+  const int head = blockIdx.x % a.heads, bi = blockIdx.x / a.heads;
   const int q0 = qb * kBM;
   const int n_kb = a.causal ? qb + 1 : nqb;
   const int row0 = bi * a.s;  // first row of this batch element in QKV
@@ -403,8 +406,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (a.s + kBM - 1) / kBM;
-  const int qb = nqb - 1 - static_cast<int>(blockIdx.x);
-  const int head = blockIdx.y % a.heads, bi = blockIdx.y / a.heads;
+  const int qb = nqb - 1 - static_cast<int>(blockIdx.y);  // longest rows first
+  const int head = blockIdx.x % a.heads, bi = blockIdx.x / a.heads;
   const int q0 = qb * kBM;
   const int nkb_all = (a.s + kB64 - 1) / kB64;
   const int n_kb = a.causal ? min(2 * qb + 2, nkb_all) : nkb_all;
@@ -620,8 +623,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   float* s_stat = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb = static_cast<int>(blockIdx.x);  // early keys see the most queries: first
-  const int head = blockIdx.y % a.heads, bi = blockIdx.y / a.heads;
+  const int kb = static_cast<int>(blockIdx.y);  // early keys see the most queries: first
+  const int head = blockIdx.x % a.heads, bi = blockIdx.x / a.heads;
   const int k0 = kb * kBN;
   const int nqb_all = (a.s + kB64 - 1) / kB64;
   const int i0 = a.causal ? (k0 / kB64) : 0;
@@ -864,7 +867,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_attn() {
 tp_status launch_attn_core_fwd_tc(const AttnShape& sh, const void* QKV, void* O, float* LSE,
                                   cudaStream_t stream) {
   if (sh.h / sh.heads != kD) return fail(TP_ERR_UNSUPPORTED, "attention: head dimension must be 128");
-  if (sh.b * sh.heads > 65535) return fail(TP_ERR_SHAPE, "attention: b * heads too large");
+  if ((sh.s + kBM - 1) / kBM > 65535 || sh.b * sh.heads > 0x7fffffffLL)
+    return fail(TP_ERR_SHAPE, "attention: sequence or b * heads too large");
   auto fn = encode_fn_attn();
   if (fn == nullptr) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   CUtensorMap map;
@@ -889,7 +893,7 @@ tp_status launch_attn_core_fwd_tc(const AttnShape& sh, const void* QKV, void* O,
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemA);
   if (e != cudaSuccess) return cuda_fail(e, "attention fwd smem attribute");
-  dim3 grid(static_cast<unsigned>((sh.s + kBM - 1) / kBM), static_cast<unsigned>(sh.b * sh.heads));
+  dim3 grid(static_cast<unsigned>(sh.b * sh.heads), static_cast<unsigned>((sh.s + kBM - 1) / kBM));
   const double pairs = sh.causal ? 0.5 * double(sh.s) * sh.s : double(sh.s) * sh.s;
   {
     LaunchScope scope(TP_KIND_ATTN_FWD, 4.0 * kD * pairs * double(sh.b) * sh.heads,
@@ -920,7 +924,8 @@ tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const vo
                                   const float* LSE, const float* dsum, void* dQKV,
                                   cudaStream_t stream) {
   if (sh.h / sh.heads != kD) return fail(TP_ERR_UNSUPPORTED, "attention: head dimension must be 128");
-  if (sh.b * sh.heads > 65535) return fail(TP_ERR_SHAPE, "attention: b * heads too large");
+  if ((sh.s + kBM - 1) / kBM > 65535 || sh.b * sh.heads > 0x7fffffffLL)
+    return fail(TP_ERR_SHAPE, "attention: sequence or b * heads too large");
   const int64_t M = sh.b * sh.s;
   CUtensorMap qkv128, qkv64, do128, do64;
   if (!make_map_f16(&qkv128, QKV, 3 * sh.h, M, 128) || !make_map_f16(&qkv64, QKV, 3 * sh.h, M, 64) ||
@@ -944,8 +949,9 @@ tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const vo
     e = cudaFuncSetAttribute(attn_bwd_dkdv_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemKV);
   if (e != cudaSuccess) return cuda_fail(e, "attention bwd smem attribute");
-  dim3 gq(static_cast<unsigned>((sh.s + kBM - 1) / kBM), static_cast<unsigned>(sh.b * sh.heads));
-  dim3 gk(static_cast<unsigned>((sh.s + kBN - 1) / kBN), static_cast<unsigned>(sh.b * sh.heads));
+  // (batch element, head) fastest: the CTAs launch in order of decreasing work
+  dim3 gq(static_cast<unsigned>(sh.b * sh.heads), static_cast<unsigned>((sh.s + kBM - 1) / kBM));
+  dim3 gk(static_cast<unsigned>(sh.b * sh.heads), static_cast<unsigned>((sh.s + kBN - 1) / kBN));
   attn_bwd_dq_tcgen05<<<gq, kThreadsB, kSmemDQ, stream>>>(qkv128, qkv64, do128, a);
   attn_bwd_dkdv_tcgen05<<<gk, kThreadsB, kSmemKV, stream>>>(qkv128, qkv64, do64, a);
   e = cudaGetLastError();
