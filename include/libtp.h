@@ -36,8 +36,13 @@
  *   fp32 work runs on the CUDA cores in fp32.
  * - No C++ exception crosses this interface.  A non-TP_OK status leaves a
  *   message for tp_last_error().  TP_ERR_CUDA reports a launch error.  Errors
- *   that kernels detect while running (a bounded wait that expired) are
- *   recorded in a device status word, read by tp_device_status().
+ *   that kernels detect while running (a bounded wait that expired) and
+ *   conditions they flag (an fp16 intermediate saturated) are recorded in a
+ *   per-device status, read by tp_device_status().  Neither stops a later
+ *   call: a flag is never read by a kernel, and a timeout makes only the
+ *   other waits of its own launch give up early (each launch carries its own
+ *   generation number).  No call checks or clears the status on entry; the
+ *   record stays until tp_device_status() reads it.
  */
 #ifndef LIBTP_H_
 #define LIBTP_H_
@@ -129,14 +134,18 @@ tp_status tp_mlp_fwd(const void* X, const void* A, const void* bA, const void* B
  * synchronisation, a plugin interface that passes only inputs and outputs).
  * The source pages have no counterpart: this is a deployment variant.
  *   Same arguments, arithmetic and kernels as tp_mlp_fwd; the intermediate
- *   H [M, f] lives in a fixed 64 MiB (67108864-byte) array compiled into
+ *   H [M, f] lives in a fixed array of 64 MiB + 256 bytes compiled into
  *   libtp, which every GPU that loads the library holds until the process
- *   exits.  M * f * element size must not exceed 64 MiB (H alone; so
- *   M * f <= 33554432 for bf16, 16777216 for fp32), otherwise TP_ERR_SHAPE
- *   with a message saying so.  Allocates nothing and calls no allocator.
+ *   exits.  M * f * element size must not exceed 64 MiB = 67108864 bytes
+ *   (H alone; so M * f <= 33554432 for bf16, 16777216 for fp32; exactly
+ *   that much is accepted), otherwise TP_ERR_SHAPE with a message saying so.
+ *   Allocates nothing and calls no allocator.
  *   The first call on each device looks up the array's device address with
  *   cudaGetSymbolAddress (that device must be current); make that first call
- *   before any stream capture.  Every call shares the one array and it keeps
+ *   before any stream capture.  The address is cached per device and CUDA
+ *   context: after cudaDeviceReset (or with another context current) the
+ *   next call looks it up again, so that call, too, should come before any
+ *   stream capture.  Every call shares the one array and it keeps
  *   the previous call's contents; nothing in it needs to start at zero (H is
  *   fully written before it is read).  Calls whose executions overlap on the
  *   GPU (on different streams, or on several host threads) race on it.
@@ -441,12 +450,27 @@ tp_status tp_profile_record(int64_t index, tp_launch_record* out);
 const char* tp_last_error(void);
 
 /*
- * Synchronizes `stream`, then reads and clears the device status word of the
- * current device.  TP_OK, TP_ERR_KERNEL (a kernel gave up a bounded wait, or
- * an fp16 attention intermediate was saturated; the message says which) or
- * TP_ERR_CUDA.
+ * Synchronizes `stream`, then reads and clears the status of the current
+ * device.  TP_OK, TP_ERR_KERNEL (a kernel gave up a bounded wait since the
+ * last read, or an fp16 attention intermediate was saturated; the message
+ * says which, a timeout first) or TP_ERR_CUDA.  Outputs of the launch that
+ * gave up a wait are incomplete; outputs of every other launch are not
+ * affected.  The same launch replayed from a captured CUDA graph keeps its
+ * generation, so after a timeout read this before replaying the graph.
  */
 tp_status tp_device_status(void* stream);
+
+/*
+ * Self-test of the kernels' bounded waits (failure detection without a GPU
+ * fault): launches one small kernel on `stream` in which one warp waits on an
+ * mbarrier that nothing ever completes, giving up after `limit_ns`
+ * nanoseconds, and a second warp waits on it with the default 2 s limit and
+ * must be released by the first one's abort.  No copy or tensor-core work is
+ * in flight, so the kernel returns normally; the following
+ * tp_device_status() then returns TP_ERR_KERNEL ("bounded-wait self-test").
+ * limit_ns must be in [1e3, 2e9] (else TP_ERR_SHAPE).
+ */
+tp_status tp_selftest_bounded_wait(int64_t limit_ns, void* stream);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int tp_version(void);

@@ -35,7 +35,8 @@ EXPORTS = ("tp_linear_col", "tp_linear_row", "tp_mlp_fwd", "tp_mlp_bwd", "tp_att
            "tp_version", "tp_profile_enable", "tp_profile_read", "tp_launch_count",
            "tp_mlp_fwd_noalloc", "tp_profile_count", "tp_profile_record", "tp_layernorm_fwd",
            "tp_layernorm_bwd", "tp_block_fwd", "tp_block_bwd", "tp_vocab_embed_fwd",
-           "tp_vocab_embed_bwd", "tp_vocab_ce_fwd", "tp_vocab_ce_bwd", "tp_gemm_plan")
+           "tp_vocab_embed_bwd", "tp_vocab_ce_fwd", "tp_vocab_ce_bwd", "tp_gemm_plan",
+           "tp_selftest_bounded_wait")
 
 _W_FIELDS = ("ln1_g", "ln1_b", "Wqkv", "Wo", "ln2_g", "ln2_b", "A", "bA", "B", "bB")
 _S_FIELDS = ("Xn1", "mean1", "rstd1", "QKV", "O", "LSE", "X1", "Xn2", "mean2", "rstd2", "Y")
@@ -117,6 +118,7 @@ def load() -> ctypes.CDLL:
     L.tp_last_error.argtypes = []
     L.tp_last_error.restype = ctypes.c_char_p
     L.tp_device_status.argtypes = [vp]
+    L.tp_selftest_bounded_wait.argtypes = [i64, vp]
     L.tp_version.argtypes = []
     L.tp_profile_enable.argtypes = [i32]
     L.tp_profile_read.argtypes = [i32, ctypes.POINTER(ProfileStats)]
@@ -302,6 +304,10 @@ def tp_vocab_ce_bwd(X, E, targets, logits, lse, dloss, dlogits, dX, dE, t: int,
 
 def tp_device_status(stream=None) -> None:
     _check(load().tp_device_status(_stream(stream)))
+
+
+def tp_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
+    _check(load().tp_selftest_bounded_wait(int(limit_ns), _stream(stream)))
 
 
 def tp_version() -> int:

@@ -8,14 +8,41 @@
 
 namespace tp {
 
-// Codes written to the device status word when a bounded wait gives up.
+// Codes recorded in DeviceStatus::code when a bounded wait gives up.
 enum : int {
   kStatusOk = 0,
   kStatusProducerTimeout = 0x101,
   kStatusMmaTimeout = 0x102,
   kStatusEpilogueTimeout = 0x103,
   kStatusAttnTimeout = 0x104,
-  kStatusF16Range = 0x201,  // a value outside the fp16 range was saturated
+  kStatusSelftestTimeout = 0x105,  // the bounded-wait self-test kernel
+};
+
+// Bits of DeviceStatus::flags: conditions that are reported but stop nothing.
+enum : int {
+  kFlagF16Range = 0x1,  // a value outside the fp16 range was saturated
+};
+
+// Per-device status, one instance in device memory.  Timeouts and flags are
+// kept apart so that a flag can never make a wait give up:
+//   abort_gen  the generation of the latest launch in which a wait gave up;
+//              the waits of a launch abort early only when it is >= their
+//              own generation, so an old timeout stops no later launch;
+//   code       the first timeout code not yet read by the host;
+//   flags      sticky flag bits (kFlag*), read by no wait.
+// The host reads and clears all three (tp_device_status).
+struct DeviceStatus {
+  unsigned long long abort_gen;
+  int code;
+  int flags;
+};
+
+// What a kernel's bounded waits need: the status, this launch's generation
+// (a per-process counter, so every launch has its own) and the wait limit.
+struct WaitCtl {
+  DeviceStatus* st;
+  unsigned long long gen;
+  unsigned long long limit_ns;
 };
 
 // A wait that has not completed after this long is treated as a hang: the
@@ -64,10 +91,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits until the phase with the given parity has completed.  Gives up (and
-// records `code` in *status) after kWaitLimitNs, or as soon as another CTA
-// has recorded an error; returns false then.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
+// Waits until the phase with the given parity has completed.  Gives up after
+// w.limit_ns (recording `code` and this launch's generation), or as soon as
+// another CTA of this launch (or of a later one) has given up; returns false
+// then.  Flags in the status never stop a wait.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w,
                                           int code) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
@@ -75,13 +103,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 255u) == 0) {
-      if (*reinterpret_cast<volatile int*>(status) != 0) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicCAS(status, 0, code);
+      if (*reinterpret_cast<volatile unsigned long long*>(&w.st->abort_gen) >= w.gen) return false;
+      if (globaltimer_ns() - t0 > w.limit_ns) {
+        atomicCAS(&w.st->code, 0, code);
+        atomicMax(&w.st->abort_gen, w.gen);
         return false;
       }
     }
   }
+}
+
+// Sets flag bits in the status (sticky until the host reads them).
+__device__ __forceinline__ void status_flag(const WaitCtl& w, int bits) {
+  atomicOr(&w.st->flags, bits);
 }
 
 // ------------------------------------------------------------- arithmetic

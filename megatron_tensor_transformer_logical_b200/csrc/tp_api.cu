@@ -1,6 +1,7 @@
 // libtp C entry points: host-side validation, the shard planner (how each
 // partitioned operation of the pages maps onto kernel launches), workspace
 // carving and the device status word.  Nothing here computes on the host.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -10,6 +11,7 @@
 #include <atomic>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "../../include/libtp.h"
@@ -23,8 +25,9 @@ thread_local std::string g_last_error;
 constexpr int kMaxDevices = 64;
 }  // namespace
 
-// Device status word: kernels that give up a bounded wait record a code here.
-__device__ int g_tp_status_word;
+// Device status: kernels that give up a bounded wait record a code here, and
+// the fp16-saturating epilogue sets a flag (DeviceStatus in ptx_sm100.cuh).
+__device__ DeviceStatus g_tp_status;
 
 tp_status fail(tp_status st, const std::string& msg) {
   g_last_error = msg;
@@ -36,18 +39,61 @@ tp_status cuda_fail(cudaError_t e, const char* where) {
   return TP_ERR_CUDA;
 }
 
-int* device_status_ptr() {
-  static int* ptrs[kMaxDevices] = {};
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static const std::pair<GetCurrent, GetId> fns = [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    const bool ok =
+        cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &q1) == cudaSuccess &&
+        q1 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &q2) == cudaSuccess &&
+        q2 == cudaDriverEntryPointSuccess;
+    return ok ? std::make_pair(reinterpret_cast<GetCurrent>(a), reinterpret_cast<GetId>(b))
+              : std::make_pair(static_cast<GetCurrent>(nullptr), static_cast<GetId>(nullptr));
+  }();
+  if (fns.first == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (fns.first(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (fns.second(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+DeviceStatus* device_status_ptr() {
+  // Cached per device together with the context it was resolved in: a new
+  // context on the device (after cudaDeviceReset, say) loads libtp's device
+  // code again, possibly elsewhere, so the address is looked up again.
+  static DeviceStatus* ptrs[kMaxDevices] = {};
+  static unsigned long long ctx_ids[kMaxDevices] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (ptrs[dev] == nullptr) {
+  const unsigned long long id = current_context_id();
+  if (ptrs[dev] == nullptr || id == 0 || id != ctx_ids[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_tp_status_word) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<int*>(p);
+    if (cudaGetSymbolAddress(&p, g_tp_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<DeviceStatus*>(p);
+    ctx_ids[dev] = current_context_id();  // the lookup made the context current
   }
   return ptrs[dev];
+}
+
+namespace {
+// Launch generations start at 1, so a cleared status (abort_gen 0) stops no
+// wait.
+std::atomic<unsigned long long> g_launch_gen{0};
+}  // namespace
+
+WaitCtl wait_ctl() {
+  WaitCtl w;
+  w.st = device_status_ptr();
+  w.gen = g_launch_gen.fetch_add(1, std::memory_order_relaxed) + 1;
+  w.limit_ns = kWaitLimitNs;
+  return w;
 }
 
 int sm_count() {
@@ -117,6 +163,15 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline size_t esize(tp_dtype d) { return d == TP_F32 ? 4 : 2; }
+
+// Every size is below 2^31 - 256 (the kernels index rows and columns with
+// 32-bit integers), which also keeps every byte count below 2^63.
+constexpr int64_t kMaxDim = (1ll << 31) - 256;
+inline bool dims_ok(std::initializer_list<int64_t> ds) {
+  for (int64_t d : ds)
+    if (d > kMaxDim) return false;
+  return true;
+}
 
 // Bump allocator over the caller's workspace.
 struct Carve {
@@ -199,6 +254,7 @@ tp_status linear_common(const void* X, const void* W, const void* bias, void* Y,
   if (dtype == TP_F32 && out_dtype != TP_F32)
     return fail(TP_ERR_DTYPE, "fp32 inputs need an fp32 output");
   if (M <= 0 || K <= 0 || N <= 0) return fail(TP_ERR_SHAPE, "M, K and N must be positive");
+  if (!dims_ok({M, K, N})) return fail(TP_ERR_SHAPE, "M, K and N must be below 2^31 - 256");
   TP_TRY(check_t(t));
   if (shard >= t) return fail(TP_ERR_SHAPE, "shard must be < t");
   const int64_t split = col ? N : K;
@@ -272,6 +328,7 @@ tp_status mlp_fwd(const void* X, const void* A, const void* bA, const void* B, c
   if (!X || !A || !B || !Z) return fail(TP_ERR_NULL, "X, A, B and Z are required");
   TP_TRY(check_dtype(dtype));
   if (M <= 0 || h <= 0 || f <= 0) return fail(TP_ERR_SHAPE, "M, h and f must be positive");
+  if (!dims_ok({M, h, f})) return fail(TP_ERR_SHAPE, "M, h and f must be below 2^31 - 256");
   TP_TRY(check_t(t));
   if (f % t != 0) return fail(TP_ERR_SHAPE, "f must be divisible by t");
   TP_TRY(check_ptrs_aligned({X, A, bA, B, bB, Z, Ysave, ws}));
@@ -318,6 +375,7 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
     return fail(TP_ERR_NULL, "X, A, B, dZ, dX, dA and dB are required");
   TP_TRY(check_dtype(dtype));
   if (M <= 0 || h <= 0 || f <= 0) return fail(TP_ERR_SHAPE, "M, h and f must be positive");
+  if (!dims_ok({M, h, f})) return fail(TP_ERR_SHAPE, "M, h and f must be below 2^31 - 256");
   TP_TRY(check_t(t));
   if (f % t != 0) return fail(TP_ERR_SHAPE, "f must be divisible by t");
   TP_TRY(check_ptrs_aligned({X, A, bA, B, Ysave, dZ, dX, dA, dbA, dB, dbB, ws}));
@@ -430,7 +488,7 @@ tp_status attn_check(const void* X, const void* Wqkv, const void* Wo, int64_t b,
   if (h % heads != 0) return fail(TP_ERR_SHAPE, "h must be divisible by heads");
   if (heads % t != 0) return fail(TP_ERR_SHAPE, "heads must be divisible by t");
   if (h / heads != 128) return fail(TP_ERR_UNSUPPORTED, "head dimension must be 128");
-  if (b * s > (1ll << 31) - 256) return fail(TP_ERR_SHAPE, "too many tokens");
+  if (!dims_ok({b, s, 3 * h}) || b * s > kMaxDim) return fail(TP_ERR_SHAPE, "too many tokens");
   TP_TRY(check_rows({h}));
   return TP_OK;
 }
@@ -569,6 +627,7 @@ tp_status ln_check(const void* X, const void* Y, int64_t M, int64_t h, tp_dtype 
   if (!X || !Y) return fail(TP_ERR_NULL, "X and Y are required");
   TP_TRY(check_dtype(dtype));
   if (M <= 0 || h <= 0) return fail(TP_ERR_SHAPE, "M and h must be positive");
+  if (!dims_ok({M, h})) return fail(TP_ERR_SHAPE, "M and h must be below 2^31 - 256");
   TP_TRY(check_rows({h}));
   if (h > layernorm_max_h()) return fail(TP_ERR_UNSUPPORTED, "layernorm: h must be at most 16384");
   return TP_OK;
@@ -810,6 +869,30 @@ using namespace tp;
     return fail(TP_ERR_UNSUPPORTED, "internal error");              \
   }
 
+namespace tp {
+namespace {
+// The bounded-wait self-test: an mbarrier that nothing ever arrives on.
+// Warp 0 waits on it with the short limit `short_ns` and gives up, recording
+// kStatusSelftestTimeout; warp 1 waits with the default limit and must be
+// released early by warp 0's abort (same launch generation).  No copy or
+// tensor-core work is in flight, so giving up leaves nothing behind.
+__global__ void bounded_wait_selftest_kernel(WaitCtl w, unsigned long long short_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) {
+    WaitCtl mine = w;
+    if (threadIdx.x == 0) mine.limit_ns = short_ns;
+    mbar_wait(&bar, 0, mine, kStatusSelftestTimeout);
+  }
+  __syncwarp();
+}
+}  // namespace
+}  // namespace tp
+
 extern "C" {
 
 tp_status tp_linear_col(const void* X, const void* W, const void* bias, void* Y, int64_t M,
@@ -927,6 +1010,7 @@ size_t tp_workspace_size(tp_op op, int64_t M, int64_t h, int64_t f, int heads, i
                          tp_dtype dtype) {
   try {
     if (M <= 0 || h <= 0 || t < 1 || (dtype != TP_F32 && dtype != TP_BF16)) return 0;
+    if (!dims_ok({M, h, f})) return 0;
     switch (op) {
       case TP_OP_MLP_FWD: return f > 0 ? mlp_fwd_ws(M, f, dtype) : 0;
       case TP_OP_MLP_BWD: return f > 0 ? mlp_bwd_ws(M, h, f, dtype) : 0;
@@ -950,28 +1034,52 @@ tp_status tp_device_status(void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-    int* p = device_status_ptr();
-    if (p == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
-    int v = 0;
-    e = cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
-    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
-    if (v != 0) {
-      const int zero = 0;
-      cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
-      char buf[128];
-      const char* who = v == kStatusProducerTimeout   ? "GEMM TMA producer"
-                        : v == kStatusMmaTimeout      ? "GEMM MMA issuer"
-                        : v == kStatusEpilogueTimeout ? "GEMM epilogue"
-                        : v == kStatusAttnTimeout     ? "attention kernel"
-                                                      : "unknown";
-      if (v == kStatusF16Range)
-        std::snprintf(buf, sizeof(buf),
-                      "an fp16 attention intermediate (QKV or dO) exceeded the fp16 range and "
-                      "was saturated (code 0x%x)", v);
-      else
-        std::snprintf(buf, sizeof(buf), "kernel gave up a bounded wait (code 0x%x, %s)", v, who);
+    DeviceStatus* p = device_status_ptr();
+    if (p == nullptr) return fail(TP_ERR_CUDA, "device status unavailable");
+    DeviceStatus v{};
+    e = cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+    if (v.code == 0 && v.flags == 0 && v.abort_gen == 0) return TP_OK;
+    const DeviceStatus zero{};
+    e = cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status");
+    const char* sat = (v.flags & kFlagF16Range) ? "; an fp16 attention intermediate (QKV or dO) "
+                                                  "exceeded the fp16 range and was saturated"
+                                                : "";
+    char buf[256];
+    if (v.code != 0) {
+      const char* who = v.code == kStatusProducerTimeout   ? "GEMM TMA producer"
+                        : v.code == kStatusMmaTimeout      ? "GEMM MMA issuer"
+                        : v.code == kStatusEpilogueTimeout ? "GEMM epilogue"
+                        : v.code == kStatusAttnTimeout     ? "attention kernel"
+                        : v.code == kStatusSelftestTimeout ? "bounded-wait self-test"
+                                                           : "unknown";
+      std::snprintf(buf, sizeof(buf), "kernel gave up a bounded wait (code 0x%x, %s)%s", v.code,
+                    who, sat);
       return fail(TP_ERR_KERNEL, buf);
     }
+    if (v.flags & kFlagF16Range) {
+      std::snprintf(buf, sizeof(buf),
+                    "an fp16 attention intermediate (QKV or dO) exceeded the fp16 range and was "
+                    "saturated (flags 0x%x)", v.flags);
+      return fail(TP_ERR_KERNEL, buf);
+    }
+    return TP_OK;
+  } catch (...) {
+    return fail(TP_ERR_UNSUPPORTED, "internal error");
+  }
+}
+
+tp_status tp_selftest_bounded_wait(int64_t limit_ns, void* stream) {
+  try {
+    if (limit_ns < 1000 || limit_ns > static_cast<int64_t>(kWaitLimitNs))
+      return fail(TP_ERR_SHAPE, "limit_ns must be in [1e3, 2e9]");
+    WaitCtl w = wait_ctl();
+    if (w.st == nullptr) return fail(TP_ERR_CUDA, "device status unavailable");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    bounded_wait_selftest_kernel<<<1, 64, 0, s>>>(w, static_cast<unsigned long long>(limit_ns));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "bounded-wait self-test launch");
     return TP_OK;
   } catch (...) {
     return fail(TP_ERR_UNSUPPORTED, "internal error");

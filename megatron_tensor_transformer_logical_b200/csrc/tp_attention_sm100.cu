@@ -52,7 +52,7 @@ struct FwdArgs {
   float scale_log2;
   __nv_bfloat16* out;  // O [M, h]
   float* lse;          // [b, heads, s]
-  int* status;
+  WaitCtl status;
 };
 
 // kind::f16 instruction descriptor with fp16 A/B and fp32 D.
@@ -374,7 +374,7 @@ struct BwdArgs {
   const float* lse;   // [b, heads, s]
   const float* dsum;  // [b, heads, s]
   __nv_bfloat16* dqkv;  // [M, 3h]
-  int* status;
+  WaitCtl status;
 };
 
 // Q (128 rows, once), dO (128 rows, once), then K_j, V_j (64 rows) in a ring
@@ -888,8 +888,8 @@ tp_status launch_attn_core_fwd_tc(const AttnShape& sh, const void* QKV, void* O,
   a.scale_log2 = kLog2eA / std::sqrt(static_cast<float>(kD));
   a.out = static_cast<__nv_bfloat16*>(O);
   a.lse = LSE;
-  a.status = device_status_ptr();
-  if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
+  a.status = wait_ctl();
+  if (a.status.st == nullptr) return fail(TP_ERR_CUDA, "device status unavailable");
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemA);
   if (e != cudaSuccess) return cuda_fail(e, "attention fwd smem attribute");
@@ -941,8 +941,8 @@ tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const vo
   a.lse = LSE;
   a.dsum = dsum;
   a.dqkv = static_cast<__nv_bfloat16*>(dQKV);
-  a.status = device_status_ptr();
-  if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
+  a.status = wait_ctl();
+  if (a.status.st == nullptr) return fail(TP_ERR_CUDA, "device status unavailable");
   cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_tcgen05,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDQ);
   if (e == cudaSuccess)

@@ -97,7 +97,7 @@ struct Args {
   // Whole 32-column chunks of a two-byte output go through the shared-memory
   // boxes and the tensor maps tmO (out), tmO2 (out2) and tmX (aux).
   int tma_out;
-  int* status;
+  WaitCtl status;
 };
 
 struct Unit {
@@ -325,7 +325,7 @@ __device__ __forceinline__ void epilogue_row32(float (&v)[32], int row, int col0
           pack8(x);
     }
   }
-  if (OUT == kOutF16 && clamped) atomicCAS(a.status, 0, kStatusF16Range);
+  if (OUT == kOutF16 && clamped) status_flag(a.status, kFlagF16Range);
 }
 
 // Byte offset of 16-byte chunk j (0-3) of row r in a 32-row x 64-byte box
@@ -384,7 +384,7 @@ __device__ __forceinline__ void epilogue_box32(float (&v)[32], int r, int col0, 
     *reinterpret_cast<uint4*>(box0 + sw64_off(r, g)) =
         (OUT == kOutF16) ? pack8_f16(x, clamped) : pack8(x);
   }
-  if (OUT == kOutF16 && clamped) atomicCAS(a.status, 0, kStatusF16Range);
+  if (OUT == kOutF16 && clamped) status_flag(a.status, kFlagF16Range);
 }
 
 // Cross-entropy epilogue on 32 consecutive columns (vocabulary entries) of
@@ -1185,8 +1185,8 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   a.ce_cps = g.ce.cps;
   a.ce_target = g.ce.target;
   a.ce_tlogit = g.ce.tlogit;
-  a.status = device_status_ptr();
-  if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
+  a.status = wait_ctl();
+  if (a.status.st == nullptr) return fail(TP_ERR_CUDA, "device status unavailable");
   EpiMaps em;
   a.tma_out = make_epi_maps<EPI, OUT>(g, em) ? 1 : 0;
 
@@ -1279,8 +1279,8 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   a.ce_cps = g.ce.cps;
   a.ce_target = g.ce.target;
   a.ce_tlogit = g.ce.tlogit;
-  a.status = device_status_ptr();
-  if (a.status == nullptr) return fail(TP_ERR_CUDA, "device status word unavailable");
+  a.status = wait_ctl();
+  if (a.status.st == nullptr) return fail(TP_ERR_CUDA, "device status unavailable");
   EpiMaps em;
   a.tma_out = make_epi_maps<EPI, OUT>(g, em) ? 1 : 0;
 

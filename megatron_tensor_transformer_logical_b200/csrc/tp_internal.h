@@ -8,6 +8,7 @@
 #include <string>
 
 #include "../../include/libtp.h"
+#include "ptx_sm100.cuh"
 
 namespace tp {
 
@@ -15,10 +16,17 @@ namespace tp {
 tp_status fail(tp_status st, const std::string& msg);
 tp_status cuda_fail(cudaError_t e, const char* where);
 
-// Device status word of the current device (kernels record bounded-wait
-// expiry there); resolved once per device with cudaGetSymbolAddress.
-int* device_status_ptr();
+// Status of the current device (kernels record bounded-wait expiry and
+// flags there); resolved once per device with cudaGetSymbolAddress.
+DeviceStatus* device_status_ptr();
+// Bounded-wait control for one kernel launch on the current device: its
+// status, a fresh generation and the default wait limit.  st is nullptr if
+// the status could not be resolved.
+WaitCtl wait_ctl();
 int sm_count();
+// Unique id of the current CUDA context (cuCtxGetId), 0 if there is none or
+// it cannot be queried.  Caches of device-symbol addresses key on it.
+unsigned long long current_context_id();
 
 // Brackets one kernel launch: counts it and, while profiling is enabled,
 // records a start/stop event pair on `stream` with its kind and work.

@@ -192,3 +192,29 @@ def test_vocab_validation(lib):
     assert cb(P[0], P[1], P[2], None, P[4], None, P[6], P[7], P[8], 64, 256, 1024, 4, bf, None) == L.TP_ERR_NULL
     assert cb(P[0], P[1], P[2], P[3], P[4], None, None, P[7], P[8], 64, 256, 1024, 4, bf, None) == L.TP_ERR_NULL
     assert cb(P[0], P[1], P[2], P[3], P[4], None, P[6], P[7], P[8], 64, 256, 1024, 4, f32, None) == L.TP_ERR_DTYPE
+
+
+def test_selftest_limit_validation(lib):
+    assert lib.tp_selftest_bounded_wait(999, None) == L.TP_ERR_SHAPE
+    assert lib.tp_selftest_bounded_wait(2_000_000_001, None) == L.TP_ERR_SHAPE
+
+
+def test_absurd_sizes_are_rejected_before_any_product_overflows(lib):
+    big = 1 << 40
+    huge = 1 << 32
+    assert lib.tp_workspace_size(L.TP_OP_MLP_FWD, huge, 512, huge, 0, 8, L.TP_BF16) == 0
+    assert lib.tp_mlp_fwd(P[0], P[1], None, P[2], None, P[3], None, huge, 512, huge, 8,
+                          L.TP_BF16, P[9], big, None) == L.TP_ERR_SHAPE
+    assert lib.tp_linear_col(P[0], P[1], None, P[2], huge, 512, 512, 1, -1, L.TP_BF16,
+                             L.TP_BF16, None) == L.TP_ERR_SHAPE
+    assert lib.tp_attn_fwd(P[0], P[1], P[2], P[3], None, None, None, huge, huge, 512, 4, 2, 1,
+                           L.TP_BF16, P[9], big, None) == L.TP_ERR_SHAPE
+
+
+@pytest.mark.parametrize("M,f", [(1 << 32, 1 << 32), (4096, 8200), (1, (1 << 25) + 8)])
+def test_noalloc_rejects_sizes_beyond_its_array_on_the_host(lib, M, f):
+    # 2^32 x 2^32 would wrap a 64-bit byte count; the others are just past
+    # the 64 MiB limit on H (bf16).  All are rejected before any CUDA call.
+    assert lib.tp_mlp_fwd_noalloc(P[0], P[1], None, P[2], None, P[3], None, M, 512, f, 8,
+                                  L.TP_BF16, None) == L.TP_ERR_SHAPE
+    assert b"64 MiB" in lib.tp_last_error()

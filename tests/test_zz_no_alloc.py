@@ -14,6 +14,7 @@ import torch
 
 from megatron_tensor_transformer_logical_b200 import binding as L
 from megatron_tensor_transformer_logical_b200.inputs import Workload, make_mlp_inputs
+from oracle import tp_oracle as O
 from tests.parity import check, cuda, need_gpu
 
 pytestmark = pytest.mark.gpu
@@ -49,6 +50,30 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(dtype):
         Zn, Yn = _run(inp, wl.t, noalloc=True)
         check(Zn, Zr.double().cpu().numpy(), f"Z {wl.name}", dtype)
         check(Yn, Yr.double().cpu().numpy(), f"Ysave {wl.name}", dtype)
+        # and against the CPU oracle ("图解Transformer并行计算" §2.1)
+        fw = O.mlp_fwd(inp["X"], inp["A"], inp["bA"], inp["B"], inp["bB"])
+        check(Zn, fw["Z"], f"Z {wl.name} vs oracle", dtype)
+        check(Yn, fw["Y"], f"Ysave {wl.name} vs oracle", dtype)
+
+
+def test_noalloc_accepts_exactly_its_limit():
+    """H of exactly 64 MiB (M * f = 2^25 bf16 elements) is accepted and gives
+    the workspace entry point's result; 8 more columns are rejected."""
+    need_gpu()
+    wl = Workload(99, "noalloc limit", b=1, s=4096, h=64, f=8192, t=8, dtype="bf16",
+                  w_std=0.05, bias_std=0.05)
+    inp = make_mlp_inputs(wl)
+    Zr, Yr = _run(inp, wl.t, noalloc=False)
+    Zn, Yn = _run(inp, wl.t, noalloc=True)
+    check(Zn, Zr.double().cpu().numpy(), "Z at the limit", "bf16")
+    check(Yn, Yr.double().cpu().numpy(), "Ysave at the limit", "bf16")
+    X = torch.zeros(4096, 64, dtype=torch.bfloat16, device="cuda")
+    A = torch.zeros(64, 8200, dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros(8200, 64, dtype=torch.bfloat16, device="cuda")
+    Z = torch.zeros(4096, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(L.TPError) as e:
+        L.tp_mlp_fwd_noalloc(X, A, None, B, None, Z, None, 8)
+    assert e.value.status == L.TP_ERR_SHAPE and "64 MiB" in str(e.value)
 
 
 def test_noalloc_rejects_sizes_beyond_its_array():
