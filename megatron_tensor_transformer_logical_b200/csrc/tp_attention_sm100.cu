@@ -4,21 +4,24 @@
 // the causal mask hiding key c from query r when c > r; each head group of
 // §3.2 runs its own heads, so the core runs per (batch, head).
 //
-// One CTA per (batch element, head, 128 query rows); blockIdx.x is the
-// (batch element, head) and blockIdx.y the row tile, longest rows first, so
-// the CTAs launch in order of decreasing work over all heads (the longest
-// tiles of the last heads do not start in the last wave):
-//   warp 0     TMA: the Q tile once, then K_j and V_j (128 keys each) into a
-//              two-deep ring (fp16, 128-byte swizzle);
-//   warp 1     allocates 512 TMEM columns; one thread issues
-//              S_j = Q K_j^T (128 x 128, K = d = 128) into one of two S
-//              buffers, so S_{j+1} is computed while S_j is being
-//              normalised, and O_j = P_j V_j into an O buffer;
-//   warps 4-7  softmax: thread i owns query row i = TMEM lane i, so the
-//              row max and sum need no shuffles; P_j (fp16) is written to
-//              shared memory in the MMA's K-major swizzled layout; the
-//              output is accumulated and rescaled in registers:
-//                O <- (O + P_{j-1} V_{j-1}) * 2^(m_{j-1} - m_j).
+// One CTA per (batch element, head, pair of adjacent 128-row query tiles);
+// blockIdx.x is the (batch element, head) and blockIdx.y the pair, longest
+// rows first, so the CTAs launch in order of decreasing work over all heads.
+// The two tiles share each K / V block and take turns on the tensor core: one
+// tile's softmax runs while the other tile's products are computed.
+//   warp 0      TMA: both Q tiles once, then K_j and V_j (128 keys each) into
+//               two-deep rings (fp16, 128-byte swizzle);
+//   warp 1      allocates 512 TMEM columns; one thread issues, per key block,
+//               P_0 V_j, S_0 = Q_0 K_{j+1}^T, P_1 V_j, S_1 = Q_1 K_{j+1}^T;
+//   warps 4-7   softmax of tile 0, warps 8-11 of tile 1: thread i owns query
+//               row i = TMEM lane i, so row max and sum need no shuffles;
+//               P_j (fp16) is written back into tensor memory over its S
+//               columns and is the tensor-memory A operand of P V, which
+//               accumulates O in tensor memory.
+// O and the row sum are kept relative to a row maximum that is raised only
+// when the new maximum exceeds it by more than 2^8 (then O is rescaled in
+// tensor memory); P stays below 2^8, and the final O / l uses the same
+// maximum, so the result does not depend on when the maximum was raised.
 // Scores are kept in the log2 domain (scaled by log2(e)/sqrt(d)); the saved
 // LSE is the natural log of the softmax denominator.  Every wait is bounded.
 #include <cuda.h>
@@ -41,9 +44,12 @@ constexpr int kBN = 128;          // keys per block
 constexpr int kTile = 128 * 128 * 2;  // one [128 x 128] fp16 tile: 32 KB
 constexpr int kHalf = kTile / 2;      // one 64-column half: 16 KB
 constexpr int kThreadsA = 384;
-// Q, K[2], V[2], P, barriers, then the softmax groups' exchange slots:
-// row maxima [2 blocks][2 groups][128 rows] and row sums [2 groups][128].
-constexpr int kSmemA = 1024 + 6 * kTile + 256 + (2 * 2 * 128 + 2 * 128) * 4;
+// Q of both tiles, K[2], V[2], barriers.
+constexpr int kSmemA = 1024 + 6 * kTile + 256;
+// O and the row sum keep the scale of a stale row maximum until the maximum
+// has risen by more than 2^8 (log2 units); the final 1/l uses the same
+// maximum, so the result is exact either way, and P stays below 2^8.
+constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLog2eA = 1.4426950408889634f;
 constexpr float kLn2A = 0.69314718055994531f;
 
@@ -67,36 +73,91 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&t);
 }
 
+// The raw-score maximum over this row's visible keys [0, vis) of one block.
+__device__ __forceinline__ float row_max_visible(uint32_t srow, int vis) {
+  float mx = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < kBN; c += 32) {
+    float v[32];
+    tmem_ld32(srow + c, v);
+    if (vis < c + 32) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = (c + i < vis) ? v[i] : -INFINITY;
+    }
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+      for (int i = 0; i < w; ++i) v[i] = fmaxf(v[i], v[i + w]);
+    mx = fmaxf(mx, v[0]);
+  }
+  return mx;
+}
+
+// P = 2^(s * scale_log2 - m) over one block row (masked keys 0), packed to
+// fp16 pairs in registers; returns the row sum of P and, in *mraw, the raw
+// maximum over the visible keys.
+__device__ __forceinline__ float exp_row(uint32_t srow, int vis, float scale_log2, float m,
+                                         uint32_t (&pk)[kBN / 2], float* mraw) {
+  float rs = 0.0f, mx = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < kBN; c += 32) {
+    float v[32];
+    tmem_ld32(srow + c, v);
+    if (vis >= c + 32) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        mx = fmaxf(mx, v[i]);
+        v[i] = ex2_approx(fmaf(v[i], scale_log2, -m));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const bool in = c + i < vis;
+        mx = fmaxf(mx, in ? v[i] : -INFINITY);
+        v[i] = in ? ex2_approx(fmaf(v[i], scale_log2, -m)) : 0.0f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[c / 2 + i] = pack_half2(v[2 * i], v[2 * i + 1]);
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+      for (int i = 0; i < w; ++i) v[i] += v[i + w];
+    rs += v[0];
+  }
+  *mraw = mx;
+  return rs;
+}
+
 __global__ void __launch_bounds__(kThreadsA, 1)
     attn_fwd_tcgen05(const __grid_constant__ CUtensorMap tmQKV, const FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + kTile;          // 2 stages
-  uint8_t* sV = smem + 3 * kTile;      // 2 stages
-  uint8_t* sP = smem + 5 * kTile;
+  uint8_t* sQ = smem;              // [2] query tiles
+  uint8_t* sK = smem + 2 * kTile;  // [2] stages
+  uint8_t* sV = smem + 4 * kTile;  // [2] stages
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * kTile);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* v_full = bars + 3;   // [2]
-  uint64_t* k_empty = bars + 5;  // [2]
-  uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2]
-  uint64_t* p_full = bars + 11;
-  uint64_t* o_full = bars + 12;
-  uint64_t* x_full = bars + 13;  // [2] both groups' row maxima of a block written
-  uint64_t* l_full = bars + 15;  // both groups' row sums written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
-  float* x_max = reinterpret_cast<float*>(smem + 6 * kTile + 256);  // [2][2][128]
-  float* x_sum = x_max + 2 * 2 * 128;                                // [2][128]
+  uint64_t* k_full = bars + 1;    // [2] stages
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2] tiles: S ready (and the previous P V done)
+  uint64_t* p_full = bars + 11;   // [2] tiles: P stored (and O rescaled)
+  uint64_t* o_full = bars + 13;   // [2] tiles: P V done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (a.s + kBM - 1) / kBM;
-  const int qb = nqb - 1 - static_cast<int>(blockIdx.y);  // longest rows first
+  const int npairs = (nqb + 1) / 2;
+  const int pair = npairs - 1 - static_cast<int>(blockIdx.y);  // longest rows first
   const int head = blockIdx.x % a.heads, bi = blockIdx.x / a.heads;
-  const int q0 = qb * kBM;
-  const int n_kb = a.causal ? qb + 1 : nqb;
+  const int qb0 = 2 * pair;  // query tiles qb0 and qb0 + 1
+  const bool valid1 = qb0 + 1 < nqb;
+  const int n0 = a.causal ? qb0 + 1 : nqb;                      // key blocks of tile 0
+  const int n1 = valid1 ? (a.causal ? qb0 + 2 : nqb) : 0;       // and of tile 1
+  const int n_max = max(n0, n1);
   const int row0 = bi * a.s;  // first row of this batch element in QKV
   const int qcol = head * kD, kcol = a.h + head * kD, vcol = 2 * a.h + head * kD;
 
@@ -104,16 +165,13 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
       mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);  // one arrival per warp of the tile's softmax group
+      mbar_init(&o_full[i], 1);
     }
-    mbar_init(p_full, 8);  // one arrival per softmax warp
-    mbar_init(o_full, 1);
-    mbar_init(&x_full[0], 8);
-    mbar_init(&x_full[1], 8);
-    mbar_init(l_full, 8);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -124,18 +182,22 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 128};
-  const uint32_t tO = tmem + 256;
+  // Tile x: S_x at columns [256 x, 256 x + 128) (P_x, fp16 pairs, over its
+  // first 64 columns), O_x at [256 x + 128, 256 x + 256).
+  auto tS = [tmem](int x) { return tmem + static_cast<uint32_t>(256 * x); };
+  auto tO = [tmem](int x) { return tmem + static_cast<uint32_t>(256 * x + 128); };
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------- TMA producer
       bool ok = true;
       tma_prefetch_desc(&tmQKV);
-      mbar_arrive_expect_tx(q_full, kTile);
-      tma_load_2d(sQ, &tmQKV, q_full, qcol, row0 + q0);
-      tma_load_2d(sQ + kHalf, &tmQKV, q_full, qcol + 64, row0 + q0);
-      for (int j = 0; j < n_kb && ok; ++j) {
+      mbar_arrive_expect_tx(q_full, (valid1 ? 2 : 1) * kTile);
+      for (int x = 0; x < (valid1 ? 2 : 1); ++x) {
+        tma_load_2d(sQ + x * kTile, &tmQKV, q_full, qcol, row0 + (qb0 + x) * kBM);
+        tma_load_2d(sQ + x * kTile + kHalf, &tmQKV, q_full, qcol + 64, row0 + (qb0 + x) * kBM);
+      }
+      for (int j = 0; j < n_max && ok; ++j) {
         const int st = j & 1;
         const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
         const int krow = row0 + j * kBN;
@@ -152,170 +214,139 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // --------------------------------------------------------- MMA issuer
+      // Per key block j: P_a V_j, S_a(j+1), P_b V_j, S_b(j+1).  The MMAs of
+      // this thread run in issue order, so S_x(j+1) overwrites P_x(j) only
+      // after P_x(j) V_j has read it, and the commit of S_x(j+1) also covers
+      // P_x(j) V_j (the softmax may rescale O_x once S_x(j+1) is ready).
       constexpr uint32_t kIdS = idesc_f16_f32(128, 128, false, false);  // Q K^T
       constexpr uint32_t kIdO = idesc_f16_f32(128, 128, false, true);   // P V
-      const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
-      bool ok = mbar_wait(q_full, 0, a.status, kStatusAttnTimeout);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&k_full[st], static_cast<uint32_t>(j >> 1) & 1u, a.status,
-                       kStatusAttnTimeout))
-          return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + st * kTile);
+      auto issue_s = [&](int x, int j) {
+        const uint32_t q_addr = smem_u32(sQ + x * kTile);
+        const uint32_t k_addr = smem_u32(sK + (j & 1) * kTile);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          umma_bf16(tS[st], sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
+          umma_bf16(tS(x), sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
                     kIdS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[st]);
-        umma_commit(&k_empty[st]);
-        return true;
+        umma_commit(&s_full[x]);
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < n_kb && ok; ++j) {
-        if (j + 1 < n_kb && !(ok = issue_s(j + 1))) break;
-        // P_j written by the softmax warps (which also read O_{j-1} already).
-        if (!(ok = mbar_wait(p_full, static_cast<uint32_t>(j) & 1u, a.status, kStatusAttnTimeout)))
-          break;
+      auto issue_pv = [&](int x, int j) {
+        const uint32_t v_addr = smem_u32(sV + (j & 1) * kTile);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)  // 16 keys: 8 columns of fp16 pairs
+          umma_f16_ts(tO(x), tS(x) + static_cast<uint32_t>(kk * 8),
+                      sw128_desc(v_addr + kk * 16 * 128, kHalf, 1024), kIdO,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&o_full[x]);
+      };
+      bool ok = mbar_wait(q_full, 0, a.status, kStatusAttnTimeout) &&
+                mbar_wait(&k_full[0], 0, a.status, kStatusAttnTimeout);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (n1 > 0) issue_s(1, 0);
+        umma_commit(&k_empty[0]);
+      }
+      for (int j = 0; j < n_max && ok; ++j) {
         const int st = j & 1;
         if (!(ok = mbar_wait(&v_full[st], static_cast<uint32_t>(j >> 1) & 1u, a.status,
                              kStatusAttnTimeout)))
           break;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sV + st * kTile);
+        bool k_next = false;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t poff = (kk >> 2) * kHalf + (kk & 3) * 32;  // P: K-major over keys
-          const uint32_t voff = kk * 16 * 128;                       // V: MN-major, 16 key rows
-          umma_bf16(tO, sw128_desc(p_addr + poff, 16, 1024),
-                    sw128_desc(v_addr + voff, kHalf, 1024), kIdO, kk > 0 ? 1u : 0u);
+        for (int x = 0; x < 2; ++x) {
+          const int nx = x ? n1 : n0;
+          if (!ok || j >= nx) continue;
+          if (!(ok = mbar_wait(&p_full[x], static_cast<uint32_t>(j) & 1u, a.status,
+                               kStatusAttnTimeout)))
+            break;
+          tc_fence_after();
+          issue_pv(x, j);
+          if (j + 1 < nx) {
+            if (!k_next) {
+              if (!(ok = mbar_wait(&k_full[(j + 1) & 1], static_cast<uint32_t>((j + 1) >> 1) & 1u,
+                                   a.status, kStatusAttnTimeout)))
+                break;
+              tc_fence_after();
+              k_next = true;
+            }
+            issue_s(x, j + 1);
+          }
         }
-        umma_commit(o_full);
+        if (!ok) break;
+        if (k_next) umma_commit(&k_empty[(j + 1) & 1]);
         umma_commit(&v_empty[st]);
       }
     }
   } else if (warp >= 4) {
     // ----------------------------------------------------------- softmax
-    // Two groups of four warps: group g owns keys [64 g, 64 g + 64) of every
-    // block and output columns [64 g, 64 g + 64); the two halves of a row
-    // agree on its running maximum through shared memory once per block.
+    // Warps 4-7 take tile 0, warps 8-11 tile 1; thread i of a group owns
+    // query row i of its tile = tensor-memory lane i.
+    const int x = (warp - 4) >> 2;
     const int quarter = warp & 3;
-    const int grp = (warp - 4) >> 2;
-    const int r = quarter * 32 + lane;  // row within the tile = TMEM lane
-    const int qrow = q0 + r;
+    const int r = quarter * 32 + lane;
+    const int qrow = (qb0 + x) * kBM + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int kc0 = grp * 64;           // this group's first key column / output column
-    float o[kD / 2];
-#pragma unroll
-    for (int i = 0; i < kD / 2; ++i) o[i] = 0.0f;
-    float m_run = -INFINITY, l_run = 0.0f;
-    bool ok = true;
-    uint8_t* line = sP + (r >> 3) * 1024 + (r & 7) * 128 + grp * kHalf;  // row r, key half grp
+    const uint32_t srow = tS(x) + lane_off, orow_t = tO(x) + lane_off;
+    const int nx = x ? n1 : n0;
     // Keys [0, limit) are visible to this row (causal: up to the row itself).
     const int limit = a.causal ? min(a.s, qrow + 1) : a.s;
-    for (int j = 0; j < n_kb; ++j) {
-      const int st = j & 1;
-      if (!(ok = mbar_wait(&s_full[st], static_cast<uint32_t>(j >> 1) & 1u, a.status,
+    float m_used = -INFINITY, l_run = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nx; ++j) {
+      if (!(ok = mbar_wait(&s_full[x], static_cast<uint32_t>(j) & 1u, a.status,
                            kStatusAttnTimeout)))
         break;
       tc_fence_after();
-      const int vis = limit - j * kBN - kc0;  // visible keys of this half: [0, vis)
-      // pass 1: the half-row max of the raw scores (the scale is positive)
-      float mloc = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 64; c += 32) {
-        float v[32];
-        tmem_ld32(tS[st] + lane_off + kc0 + c, v);
-        if (vis < c + 32) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = (c + i < vis) ? v[i] : -INFINITY;
-        }
-#pragma unroll
-        for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-          for (int i = 0; i < w; ++i) v[i] = fmaxf(v[i], v[i + w]);
-        mloc = fmaxf(mloc, v[0]);
-      }
-      // exchange the half-row maxima of block j (slot j & 1)
-      float* xs = x_max + st * 256;
-      xs[grp * 128 + r] = mloc;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&x_full[st]);
-      if (!(ok = mbar_wait(&x_full[st], static_cast<uint32_t>(j >> 1) & 1u, a.status,
-                           kStatusAttnTimeout)))
-        break;
-      const float mraw = fmaxf(mloc, xs[(grp ^ 1) * 128 + r]);
-      const float mx = fmaxf(m_run, mraw * a.scale_log2);
-      const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - mx);
-      m_run = mx;
-      // fold in this group's columns of O_{j-1} (scaled at m_{j-1}), rescale to m_j
+      const int vis = limit - j * kBN;  // visible keys of this block: [0, vis), vis >= 1
+      if (j == 0) m_used = row_max_visible(srow, vis) * a.scale_log2;
+      uint32_t pk[kBN / 2];
+      float mraw;
+      float rs = exp_row(srow, vis, a.scale_log2, m_used, pk, &mraw);
       if (j > 0) {
-        if (!(ok = mbar_wait(o_full, static_cast<uint32_t>(j - 1) & 1u, a.status,
-                             kStatusAttnTimeout)))
-          break;
-        tc_fence_after();
+        const float m_new = mraw * a.scale_log2;
+        const bool need = m_new > m_used + kRescaleLog2;
+        if (__any_sync(0xffffffffu, need)) {
+          // Rare: the maximum rose by more than 2^8.  Recompute P at the new
+          // maximum (S is still intact: P has not been stored yet) and
+          // rescale O (P_{j-1} V_{j-1} completed before S_j) and l.
+          const float alpha = need ? ex2_approx(m_used - m_new) : 1.0f;
+          if (need) m_used = m_new;
+          rs = exp_row(srow, vis, a.scale_log2, m_used, pk, &mraw);
+#pragma unroll 1
+          for (int c = 0; c < kD; c += 32) {
+            float o[32];
+            tmem_ld32(orow_t + c, o);
 #pragma unroll
-        for (int c = 0; c < kD / 2; c += 32) {
-          float v[32];
-          tmem_ld32(tO + lane_off + kc0 + c, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[c + i] = (o[c + i] + v[i]) * alpha;
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(orow_t + c, o);
+          }
+          l_run *= alpha;
         }
       }
-      // pass 2: P = 2^(s * scale - m) for this half, row sum, fp16 into the P tile
-      float rs = 0.0f;
+      l_run += rs;
 #pragma unroll
-      for (int c = 0; c < 64; c += 32) {
-        float v[32];
-        tmem_ld32(tS[st] + lane_off + kc0 + c, v);
+      for (int c = 0; c < kBN / 2; c += 16) {
+        uint32_t q16[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = ex2_approx(fmaf(v[i], a.scale_log2, -mx));
-        if (vis < c + 32) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = (c + i < vis) ? v[i] : 0.0f;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_half2(v[2 * i], v[2 * i + 1]);
-#pragma unroll
-        for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-          for (int i = 0; i < w; ++i) v[i] += v[i + w];
-        rs += v[0];
-        // 32 keys = 64 bytes = four 16-byte chunks of the row's 128-byte line
-        // in this group's 64-key half; the chunk index is swizzled by (row & 7).
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = (c >> 3) + q;
-          *reinterpret_cast<uint4*>(line + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
+        for (int i = 0; i < 16; ++i) q16[i] = pk[c + i];
+        tmem_st16(srow + c, q16);
       }
-      l_run = l_run * alpha + rs;
-      fence_async_smem();  // P stores visible to the tensor core
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[x]);
     }
-    // the row sum is the sum of the two halves' sums
-    if (ok) {
-      x_sum[grp * 128 + r] = l_run;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(l_full);
-      ok = mbar_wait(l_full, 0, a.status, kStatusAttnTimeout);
-    }
-    if (ok && mbar_wait(o_full, static_cast<uint32_t>(n_kb - 1) & 1u, a.status,
-                        kStatusAttnTimeout)) {
+    if (ok && nx > 0 &&
+        mbar_wait(&o_full[x], static_cast<uint32_t>(nx - 1) & 1u, a.status, kStatusAttnTimeout)) {
       tc_fence_after();
-      const float l_tot = x_sum[r] + x_sum[128 + r];
-      const float inv = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
-      __nv_bfloat16* orow = a.out + static_cast<long long>(row0 + qrow) * a.h + head * kD + kc0;
-#pragma unroll
-      for (int c = 0; c < kD / 2; c += 32) {
+      const float inv = 1.0f / l_run;
+      __nv_bfloat16* orow = a.out + static_cast<long long>(row0 + qrow) * a.h + head * kD;
+#pragma unroll 1
+      for (int c = 0; c < kD; c += 32) {
         float v[32];
-        tmem_ld32(tO + lane_off + kc0 + c, v);
+        tmem_ld32(orow_t + c, v);
         if (qrow < a.s) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -324,17 +355,16 @@ __global__ void __launch_bounds__(kThreadsA, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int i = 8 * q + 2 * e;
-              __nv_bfloat162 t = __floats2bfloat162_rn((o[c + i] + v[i]) * inv,
-                                                       (o[c + i + 1] + v[i + 1]) * inv);
+              __nv_bfloat162 t = __floats2bfloat162_rn(v[i] * inv, v[i + 1] * inv);
               w[e] = *reinterpret_cast<uint32_t*>(&t);
             }
             *reinterpret_cast<uint4*>(orow + c + 8 * q) = u;
           }
         }
       }
-      if (qrow < a.s && grp == 0)
+      if (qrow < a.s)
         a.lse[(static_cast<long long>(bi) * a.heads + head) * a.s + qrow] =
-            (m_run + log2f(l_tot)) * kLn2A;
+            (m_used + log2f(l_run)) * kLn2A;
     }
   }
 
@@ -893,7 +923,8 @@ tp_status launch_attn_core_fwd_tc(const AttnShape& sh, const void* QKV, void* O,
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemA);
   if (e != cudaSuccess) return cuda_fail(e, "attention fwd smem attribute");
-  dim3 grid(static_cast<unsigned>(sh.b * sh.heads), static_cast<unsigned>((sh.s + kBM - 1) / kBM));
+  const int64_t nqb = (sh.s + kBM - 1) / kBM;
+  dim3 grid(static_cast<unsigned>(sh.b * sh.heads), static_cast<unsigned>((nqb + 1) / 2));
   const double pairs = sh.causal ? 0.5 * double(sh.s) * sh.s : double(sh.s) * sh.s;
   {
     LaunchScope scope(TP_KIND_ATTN_FWD, 4.0 * kD * pairs * double(sh.b) * sh.heads,
