@@ -377,24 +377,22 @@ __global__ void __launch_bounds__(kThreadsA, 1)
 
 
 // ------------------------------------------------------------------ backward
-// Two kernels, no atomics (deterministic), both on tcgen05 with the same
-// warp roles as the forward; P and dS are recomputed from the saved LSE:
+// Two kernels, no atomics (deterministic), both on tcgen05; P and dS are
+// recomputed from the saved LSE:
 //   P = 2^(S * scale_log2 - LSE * log2e),  dS = P * (dP - D),  D = rowsum(dO * O).
-// dQ kernel  (per 128 query rows, 64-key blocks):
-//   S = Q K^T, dP = dO V^T (TMEM, two buffers) -> dS (fp16, shared memory)
-//   -> dQ += dS K (TMEM); dQ is scaled by 1/sqrt(d) at the end.
+// dQ kernel (per pair of 128-row query tiles of one head, 64-key blocks; the
+// two tiles share each K / V block and take turns on the tensor core):
+//   S = Q K^T, dP = dO V^T (TMEM) -> dS (fp16, written back into tensor
+//   memory over S) -> dQ += dS K (dS the tensor-memory A operand); dQ is
+//   scaled by 1/sqrt(d) at the end.
 // dK/dV kernel (per 128 keys, 64-query blocks):
-//   S^T = K Q^T, dP^T = V dO^T (TMEM, two buffers) -> P^T, dS^T (shared memory)
-//   -> dV += P^T dO, dK += dS^T Q (TMEM); dK is scaled by 1/sqrt(d) at the end.
+//   S^T = K Q^T, dP^T = V dO^T (TMEM, two buffers) -> P^T, dS^T (fp16, back
+//   into tensor memory over S^T and dP^T) -> dV += P^T dO, dK += dS^T Q
+//   (tensor-memory A operands); dK is scaled by 1/sqrt(d) at the end.
 constexpr int kB64 = 64;
 constexpr int kTile64 = 64 * 128 * 2;   // [64 rows x 128] fp16: 16 KB (two 8 KB halves)
 constexpr int kHalf64 = kTile64 / 2;
-constexpr int kTile128x64 = 128 * 64 * 2;  // [128 rows x 64] fp16: 16 KB (one SW128 atom wide)
 
-// The backward kernels run 12 warps: warp 0 TMA, warp 1 MMA, warps 4-11 the
-// element-wise work in two groups of four; group g takes columns
-// [32 g, 32 g + 32) of every 64-column block (and half of the output
-// columns), so each SM sub-partition runs two element-wise warps.
 constexpr int kThreadsB = 384;
 constexpr int kEwWarpsB = 8;
 
@@ -407,12 +405,42 @@ struct BwdArgs {
   WaitCtl status;
 };
 
-// Q (128 rows, once), dO (128 rows, once), then K_j, V_j (64 rows) in a ring
-// of kKvStages stages (deep enough to cover the L2 latency of a 32 KB load
-// with several blocks of work).
-// Shared memory: Q 32K | dO 32K | KV[4] (K 16K + V 16K) | dS[2] 16K each.
-constexpr int kKvStages = 4;
-constexpr int kSmemDQ = 1024 + 2 * kTile + kKvStages * (2 * kTile64) + 2 * kTile128x64 + 256;
+// Two warp-collective loads of 32 lanes x 32 columns with a single wait.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, float (&va)[32], uint32_t tb,
+                                            float (&vb)[32]) {
+  uint32_t a[32], b[32];
+#define TP_LD32(dst, addr)                                                                  \
+  asm volatile(                                                                            \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "                                            \
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "            \
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "  \
+      "[%32];"                                                                             \
+      : "=r"(dst[0]), "=r"(dst[1]), "=r"(dst[2]), "=r"(dst[3]), "=r"(dst[4]),             \
+        "=r"(dst[5]), "=r"(dst[6]), "=r"(dst[7]), "=r"(dst[8]), "=r"(dst[9]),             \
+        "=r"(dst[10]), "=r"(dst[11]), "=r"(dst[12]), "=r"(dst[13]), "=r"(dst[14]),        \
+        "=r"(dst[15]), "=r"(dst[16]), "=r"(dst[17]), "=r"(dst[18]), "=r"(dst[19]),        \
+        "=r"(dst[20]), "=r"(dst[21]), "=r"(dst[22]), "=r"(dst[23]), "=r"(dst[24]),        \
+        "=r"(dst[25]), "=r"(dst[26]), "=r"(dst[27]), "=r"(dst[28]), "=r"(dst[29]),        \
+        "=r"(dst[30]), "=r"(dst[31])                                                       \
+      : "r"(addr)                                                                          \
+      : "memory")
+  TP_LD32(a, ta);
+  TP_LD32(b, tb);
+#undef TP_LD32
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  // The wait orders the loads; the copies below cannot move above it (the
+  // asm is volatile with a memory clobber).
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    va[i] = __uint_as_float(a[i]);
+    vb[i] = __uint_as_float(b[i]);
+  }
+}
+
+// dQ kernel.  Shared memory: Q[2] 32K each | dO[2] 32K each | KV ring of
+// kKvStages stages (K 16K + V 16K) | barriers.
+constexpr int kKvStages = 3;
+constexpr int kSmemDQ = 1024 + 4 * kTile + kKvStages * (2 * kTile64) + 256;
 
 __global__ void __launch_bounds__(kThreadsB, 1)
     attn_bwd_dq_tcgen05(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
@@ -420,27 +448,29 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sdO = smem + kTile;
-  uint8_t* sKV = smem + 2 * kTile;                 // stage st: K at +0, V at +kTile64
-  uint8_t* sdS = sKV + kKvStages * (2 * kTile64);   // [2] x 16 KB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sdS + 2 * kTile128x64);
+  uint8_t* sQ = smem;                  // [2] tiles
+  uint8_t* sdO = smem + 2 * kTile;     // [2] tiles
+  uint8_t* sKV = smem + 4 * kTile;     // stage st: K at +0, V at +kTile64
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + kKvStages * (2 * kTile64));
   uint64_t* qd_full = bars + 0;
   uint64_t* kv_full = bars + 1;                   // [kKvStages]
   uint64_t* kv_empty = kv_full + kKvStages;       // [kKvStages]
-  uint64_t* s_full = kv_empty + kKvStages;        // [2]
-  uint64_t* ds_full = s_full + 2;                 // [2]
-  uint64_t* ds_free = ds_full + 2;                // [2]
-  uint64_t* dq_done = ds_free + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dq_done + 1);
+  uint64_t* s_full = kv_empty + kKvStages;        // [2] tiles: S, dP ready
+  uint64_t* ds_full = s_full + 2;                 // [2] tiles: dS stored
+  uint64_t* dq_done = ds_full + 2;                // [2] tiles
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dq_done + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (a.s + kBM - 1) / kBM;
-  const int qb = nqb - 1 - static_cast<int>(blockIdx.y);  // longest rows first
+  const int npairs = (nqb + 1) / 2;
+  const int pair = npairs - 1 - static_cast<int>(blockIdx.y);  // longest rows first
   const int head = blockIdx.x % a.heads, bi = blockIdx.x / a.heads;
-  const int q0 = qb * kBM;
+  const int qb0 = 2 * pair;
+  const bool valid1 = qb0 + 1 < nqb;
   const int nkb_all = (a.s + kB64 - 1) / kB64;
-  const int n_kb = a.causal ? min(2 * qb + 2, nkb_all) : nkb_all;
+  const int n0 = a.causal ? min(2 * qb0 + 2, nkb_all) : nkb_all;
+  const int n1 = valid1 ? (a.causal ? min(2 * qb0 + 4, nkb_all) : nkb_all) : 0;
+  const int n_max = max(n0, n1);
   const int row0 = bi * a.s;
 
   if (threadIdx.x == 0) {
@@ -451,10 +481,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&ds_full[i], kEwWarpsB);
-      mbar_init(&ds_free[i], 1);
+      mbar_init(&ds_full[i], 4);  // the tile's four element-wise warps
+      mbar_init(&dq_done[i], 1);
     }
-    mbar_init(dq_done, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -465,9 +494,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 64};
-  const uint32_t tP[2] = {tmem + 128, tmem + 192};
-  const uint32_t tQ = tmem + 256;
+  // Tile x: S_x at [256 x, +64) (dS_x, fp16 pairs, over its first 32
+  // columns), dP_x at [256 x + 64, +64), dQ_x at [256 x + 128, +128).
+  auto tS = [tmem](int x) { return tmem + static_cast<uint32_t>(256 * x); };
+  auto tP = [tmem](int x) { return tmem + static_cast<uint32_t>(256 * x + 64); };
+  auto tQ = [tmem](int x) { return tmem + static_cast<uint32_t>(256 * x + 128); };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -475,12 +506,15 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmKV);
       tma_prefetch_desc(&tmdO);
-      mbar_arrive_expect_tx(qd_full, 2 * kTile);
-      tma_load_2d(sQ, &tmQ, qd_full, head * kD, row0 + q0);
-      tma_load_2d(sQ + kHalf, &tmQ, qd_full, head * kD + 64, row0 + q0);
-      tma_load_2d(sdO, &tmdO, qd_full, head * kD, row0 + q0);
-      tma_load_2d(sdO + kHalf, &tmdO, qd_full, head * kD + 64, row0 + q0);
-      for (int j = 0; j < n_kb && ok; ++j) {
+      mbar_arrive_expect_tx(qd_full, (valid1 ? 2 : 1) * 2 * kTile);
+      for (int x = 0; x < (valid1 ? 2 : 1); ++x) {
+        const int qr = row0 + (qb0 + x) * kBM;
+        tma_load_2d(sQ + x * kTile, &tmQ, qd_full, head * kD, qr);
+        tma_load_2d(sQ + x * kTile + kHalf, &tmQ, qd_full, head * kD + 64, qr);
+        tma_load_2d(sdO + x * kTile, &tmdO, qd_full, head * kD, qr);
+        tma_load_2d(sdO + x * kTile + kHalf, &tmdO, qd_full, head * kD + 64, qr);
+      }
+      for (int j = 0; j < n_max && ok; ++j) {
         const int ks = j % kKvStages;
         const uint32_t kph = static_cast<uint32_t>(j / kKvStages) & 1u;
         if (!(ok = mbar_wait(&kv_empty[ks], kph ^ 1u, a.status, kStatusAttnTimeout))) break;
@@ -495,58 +529,74 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      // Per key block j: dQ_0 += dS_0 K_j, S_0 / dP_0 of block j + 1, then the
+      // same for tile 1.  The MMAs run in issue order, so S_x(j + 1)
+      // overwrites dS_x(j) only after dQ_x's product has read it.
       constexpr uint32_t kIdSP = idesc_f16_f32(128, 64, false, false);  // Q K^T, dO V^T
       constexpr uint32_t kIdQ = idesc_f16_f32(128, 128, false, true);   // dS K
-      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sdO);
-      bool ok = mbar_wait(qd_full, 0, a.status, kStatusAttnTimeout);
-      auto issue_sp = [&](int j) -> bool {
-        const int st = j & 1;
-        const int ks = j % kKvStages;
-        if (!mbar_wait(&kv_full[ks], static_cast<uint32_t>(j / kKvStages) & 1u, a.status,
-                       kStatusAttnTimeout))
-          return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sKV + ks * (2 * kTile64));
+      auto issue_sp = [&](int x, int j) {
+        const uint32_t q_addr = smem_u32(sQ + x * kTile), do_addr = smem_u32(sdO + x * kTile);
+        const uint32_t k_addr = smem_u32(sKV + (j % kKvStages) * (2 * kTile64));
         const uint32_t v_addr = k_addr + kTile64;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t a_off = (kk >> 2) * kHalf + (kk & 3) * 32;
           const uint32_t b_off = (kk >> 2) * kHalf64 + (kk & 3) * 32;
-          umma_bf16(tS[st], sw128_desc(q_addr + a_off, 16, 1024),
+          umma_bf16(tS(x), sw128_desc(q_addr + a_off, 16, 1024),
                     sw128_desc(k_addr + b_off, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
-          umma_bf16(tP[st], sw128_desc(do_addr + a_off, 16, 1024),
+          umma_bf16(tP(x), sw128_desc(do_addr + a_off, 16, 1024),
                     sw128_desc(v_addr + b_off, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[st]);
-        return true;
+        umma_commit(&s_full[x]);
       };
-      if (ok) ok = issue_sp(0);
-      for (int j = 0; j < n_kb && ok; ++j) {
-        if (j + 1 < n_kb && !(ok = issue_sp(j + 1))) break;
-        const int st = j & 1;
-        if (!(ok = mbar_wait(&ds_full[st], (static_cast<uint32_t>(j) >> 1) & 1u, a.status,
-                             kStatusAttnTimeout)))
-          break;
+      bool ok = mbar_wait(qd_full, 0, a.status, kStatusAttnTimeout) &&
+                mbar_wait(&kv_full[0], 0, a.status, kStatusAttnTimeout);
+      if (ok) {
         tc_fence_after();
-        const int ks = j % kKvStages;
-        const uint32_t ds_addr = smem_u32(sdS + st * kTile128x64);
-        const uint32_t k_addr = smem_u32(sKV + ks * (2 * kTile64));
-#pragma unroll
-        for (int kk = 0; kk < kB64 / 16; ++kk) {
-          umma_bf16(tQ, sw128_desc(ds_addr + kk * 32, 16, 1024),
-                    sw128_desc(k_addr + kk * 2048, kHalf64, 1024), kIdQ, (j | kk) != 0 ? 1u : 0u);
-        }
-        umma_commit(&kv_empty[ks]);
-        umma_commit(&ds_free[st]);
+        issue_sp(0, 0);
+        if (n1 > 0) issue_sp(1, 0);
       }
-      if (ok) umma_commit(dq_done);
+      for (int j = 0; j < n_max && ok; ++j) {
+        bool kv_next = false;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int nx = x ? n1 : n0;
+          if (!ok || j >= nx) continue;
+          if (!(ok = mbar_wait(&ds_full[x], static_cast<uint32_t>(j) & 1u, a.status,
+                               kStatusAttnTimeout)))
+            break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sKV + (j % kKvStages) * (2 * kTile64));
+#pragma unroll
+          for (int kk = 0; kk < kB64 / 16; ++kk)  // 16 keys: 8 columns of fp16 pairs
+            umma_f16_ts(tQ(x), tS(x) + static_cast<uint32_t>(kk * 8),
+                        sw128_desc(k_addr + kk * 2048, kHalf64, 1024), kIdQ,
+                        (j | kk) != 0 ? 1u : 0u);
+          if (j + 1 < nx) {
+            if (!kv_next) {
+              const int ks = (j + 1) % kKvStages;
+              if (!(ok = mbar_wait(&kv_full[ks], static_cast<uint32_t>((j + 1) / kKvStages) & 1u,
+                                   a.status, kStatusAttnTimeout)))
+                break;
+              tc_fence_after();
+              kv_next = true;
+            }
+            issue_sp(x, j + 1);
+          } else {
+            umma_commit(&dq_done[x]);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&kv_empty[j % kKvStages]);
+      }
     }
   } else if (warp >= 4) {
+    // Warps 4-7 take tile 0, warps 8-11 tile 1; thread i owns query row i.
+    const int x = (warp - 4) >> 2;
     const int quarter = warp & 3;
-    const int grp = (warp - 4) >> 2;  // this warp's column half
-    const int c = grp * 32;
     const int r = quarter * 32 + lane;
-    const int qrow = q0 + r;
+    const int qrow = (qb0 + x) * kBM + r;
+    const int nx = x ? n1 : n0;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.s;
     const int qc = min(qrow, a.s - 1);
@@ -554,47 +604,49 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     const float dd = a.dsum[stat + qc];
     const int limit = a.causal ? min(a.s, qrow + 1) : a.s;
     bool ok = true;
-    for (int j = 0; j < n_kb && ok; ++j) {
-      const int st = j & 1;
-      if (!(ok = mbar_wait(&s_full[st], (static_cast<uint32_t>(j) >> 1) & 1u, a.status,
+    for (int j = 0; j < nx && ok; ++j) {
+      if (!(ok = mbar_wait(&s_full[x], static_cast<uint32_t>(j) & 1u, a.status,
                            kStatusAttnTimeout)))
         break;
-      if (j >= 2 && !(ok = mbar_wait(&ds_free[st], ((static_cast<uint32_t>(j) >> 1) - 1u) & 1u,
-                                     a.status, kStatusAttnTimeout)))
-        break;
       tc_fence_after();
-      const int vis = limit - j * kB64 - c;  // columns c + i with i < vis are visible
-      uint8_t* row = sdS + st * kTile128x64 + (r >> 3) * 1024 + (r & 7) * 128;
-      float sv[32], pv[32];
-      tmem_ld32(tS[st] + lane_off + c, sv);
-      tmem_ld32(tP[st] + lane_off + c, pv);
-      uint32_t pk[16];
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float p0 = ex2_approx(fmaf(sv[i], a.scale_log2, -lse2));
-        float p1 = ex2_approx(fmaf(sv[i + 1], a.scale_log2, -lse2));
-        p0 = (i < vis) ? p0 : 0.0f;
-        p1 = (i + 1 < vis) ? p1 : 0.0f;
-        pk[i >> 1] = pack_half2(p0 * (pv[i] - dd), p1 * (pv[i + 1] - dd));
-      }
+      for (int c = 0; c < kB64; c += 32) {
+        const int vis = limit - j * kB64 - c;  // columns c + i with i < vis are visible
+        float sv[32], pv[32];
+        tmem_ld32x2(tS(x) + lane_off + c, sv, tP(x) + lane_off + c, pv);
+        uint32_t pk[16];
+        if (vis >= 32) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int chunk = (c >> 3) + q;
-        *reinterpret_cast<uint4*>(row + ((chunk ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          for (int i = 0; i < 32; i += 2) {
+            const float p0 = ex2_approx(fmaf(sv[i], a.scale_log2, -lse2));
+            const float p1 = ex2_approx(fmaf(sv[i + 1], a.scale_log2, -lse2));
+            pk[i >> 1] = pack_half2(p0 * (pv[i] - dd), p1 * (pv[i + 1] - dd));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float p0 = ex2_approx(fmaf(sv[i], a.scale_log2, -lse2));
+            float p1 = ex2_approx(fmaf(sv[i + 1], a.scale_log2, -lse2));
+            p0 = (i < vis) ? p0 : 0.0f;
+            p1 = (i + 1 < vis) ? p1 : 0.0f;
+            pk[i >> 1] = pack_half2(p0 * (pv[i] - dd), p1 * (pv[i + 1] - dd));
+          }
+        }
+        // dS columns [c / 2, c / 2 + 16): S columns this thread has read.
+        tmem_st16(tS(x) + lane_off + c / 2, pk);
       }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_full[st]);
+      if (lane == 0) mbar_arrive(&ds_full[x]);
     }
-    if (ok && mbar_wait(dq_done, 0, a.status, kStatusAttnTimeout)) {
+    if (ok && nx > 0 && mbar_wait(&dq_done[x], 0, a.status, kStatusAttnTimeout)) {
       tc_fence_after();
       __nv_bfloat16* out = a.dqkv + static_cast<long long>(row0 + qrow) * (3LL * a.h) + head * kD;
-#pragma unroll
-      for (int cc = grp * (kD / 2); cc < (grp + 1) * (kD / 2); cc += 32) {
+#pragma unroll 1
+      for (int cc = 0; cc < kD; cc += 32) {
         float v[32];
-        tmem_ld32(tQ + lane_off + cc, v);
+        tmem_ld32(tQ(x) + lane_off + cc, v);
         if (qrow < a.s) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -620,14 +672,15 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 }
 
 // K, V (128 rows, once), then Q_i, dO_i (64 rows) with the block's LSE * log2(e)
-// and D in a ring of kQdStages stages; P^T and dS^T tiles [128 keys x 64
-// queries] in two stages.  The TMA warp stages LSE and D (plain loads by its
-// 32 lanes) and counts as the stage's second arrival.
-// Shared memory: K 32K | V 32K | QdO[3] (Q 16K + dO 16K) | PdS[2] (P^T 16K +
-// dS^T 16K) | barriers | stats[3] (128 floats).
-constexpr int kQdStages = 3;
-constexpr int kSmemKV = 1024 + 2 * kTile + kQdStages * (2 * kTile64) + 2 * (2 * kTile128x64) +
-                        256 + kQdStages * 2 * kB64 * 4;
+// and D in a ring of kQdStages stages.  The TMA warp stages LSE and D (plain
+// loads by its 32 lanes) and counts as the stage's second arrival.
+// Shared memory: K 32K | V 32K | QdO[4] (Q 16K + dO 16K) | barriers | stats[4]
+// (128 floats).  P^T and dS^T live in tensor memory: element-wise group g
+// (query columns [32 g, 32 g + 32) of a block) writes its fp16 pairs over
+// the 16 columns starting at column 32 g of the S^T (P^T) and dP^T (dS^T)
+// buffers, columns only it has read.
+constexpr int kQdStages = 4;
+constexpr int kSmemKV = 1024 + 2 * kTile + kQdStages * (2 * kTile64) + 256 + kQdStages * 2 * kB64 * 4;
 
 __global__ void __launch_bounds__(kThreadsB, 1)
     attn_bwd_dkdv_tcgen05(const __grid_constant__ CUtensorMap tmKV128,
@@ -639,15 +692,13 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   uint8_t* sK = smem;
   uint8_t* sV = smem + kTile;
   uint8_t* sQdO = smem + 2 * kTile;                     // stage q: Q at +0, dO at +kTile64
-  uint8_t* sPdS = sQdO + kQdStages * (2 * kTile64);     // stage st: P^T at +0, dS^T at +16K
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sPdS + 2 * (2 * kTile128x64));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sQdO + kQdStages * (2 * kTile64));
   uint64_t* kv_full = bars + 0;
   uint64_t* qd_full = bars + 1;                 // [kQdStages]
   uint64_t* qd_empty = qd_full + kQdStages;     // [kQdStages]
   uint64_t* s_full = qd_empty + kQdStages;      // [2]
   uint64_t* p_full = s_full + 2;                // [2]
-  uint64_t* p_free = p_full + 2;                // [2]
-  uint64_t* acc_done = p_free + 2;
+  uint64_t* acc_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_done + 1);
   // stage q: LSE * log2(e) of the block's 64 queries at [0, 64), D at [64, 128)
   float* s_stat = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
@@ -670,7 +721,6 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], kEwWarpsB);
-      mbar_init(&p_free[i], 1);
     }
     mbar_init(acc_done, 1);
     fence_mbar_init();
@@ -683,8 +733,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 64};
-  const uint32_t tP[2] = {tmem + 128, tmem + 192};
+  // S^T buffers at columns 0 and 64, dP^T at 128 and 192, dV at 256, dK at 384.
+  auto tS = [tmem](int st) { return tmem + static_cast<uint32_t>(64 * st); };
+  auto tP = [tmem](int st) { return tmem + static_cast<uint32_t>(128 + 64 * st); };
   const uint32_t tdV = tmem + 256, tdK = tmem + 384;
 
   if (warp == 0) {
@@ -743,9 +794,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t a_off = (kk >> 2) * kHalf + (kk & 3) * 32;
           const uint32_t b_off = (kk >> 2) * kHalf64 + (kk & 3) * 32;
-          umma_bf16(tS[st], sw128_desc(k_addr + a_off, 16, 1024),
+          umma_bf16(tS(st), sw128_desc(k_addr + a_off, 16, 1024),
                     sw128_desc(q_addr + b_off, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
-          umma_bf16(tP[st], sw128_desc(v_addr + a_off, 16, 1024),
+          umma_bf16(tP(st), sw128_desc(v_addr + a_off, 16, 1024),
                     sw128_desc(do_addr + b_off, 16, 1024), kIdSP, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[st]);
@@ -753,6 +804,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       };
       if (ok && n_qb > 0) ok = issue_sp(0);
       for (int it = 0; it < n_qb && ok; ++it) {
+        // S^T / dP^T of block it + 1 go into the other buffers, whose P^T /
+        // dS^T the products of block it - 1 (issued before) have read.
         if (it + 1 < n_qb && !(ok = issue_sp(it + 1))) break;
         const int st = it & 1;
         if (!(ok = mbar_wait(&p_full[st], (static_cast<uint32_t>(it) >> 1) & 1u, a.status,
@@ -760,20 +813,19 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           break;
         tc_fence_after();
         const int qs = it % kQdStages;
-        const uint32_t pt_addr = smem_u32(sPdS + st * (2 * kTile128x64));
-        const uint32_t dst_addr = pt_addr + kTile128x64;
         const uint32_t q_addr = smem_u32(sQdO + qs * (2 * kTile64));
         const uint32_t do_addr = q_addr + kTile64;
 #pragma unroll
         for (int kk = 0; kk < kB64 / 16; ++kk) {
+          // queries [16 kk, 16 kk + 16): group kk / 2's columns, 8 columns each
+          const uint32_t col = static_cast<uint32_t>(32 * (kk >> 1) + 8 * (kk & 1));
           const uint32_t acc = (it | kk) != 0 ? 1u : 0u;
-          umma_bf16(tdV, sw128_desc(pt_addr + kk * 32, 16, 1024),
-                    sw128_desc(do_addr + kk * 2048, kHalf64, 1024), kIdAcc, acc);
-          umma_bf16(tdK, sw128_desc(dst_addr + kk * 32, 16, 1024),
-                    sw128_desc(q_addr + kk * 2048, kHalf64, 1024), kIdAcc, acc);
+          umma_f16_ts(tdV, tS(st) + col, sw128_desc(do_addr + kk * 2048, kHalf64, 1024), kIdAcc,
+                      acc);
+          umma_f16_ts(tdK, tP(st) + col, sw128_desc(q_addr + kk * 2048, kHalf64, 1024), kIdAcc,
+                      acc);
         }
         umma_commit(&qd_empty[qs]);
-        umma_commit(&p_free[st]);
       }
       if (ok) umma_commit(acc_done);
     }
@@ -797,20 +849,14 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       if (!(ok = mbar_wait(&qd_full[qs], static_cast<uint32_t>(it / kQdStages) & 1u, a.status,
                            kStatusAttnTimeout)))
         break;
-      if (it >= 2 && !(ok = mbar_wait(&p_free[st], ((static_cast<uint32_t>(it) >> 1) - 1u) & 1u,
-                                      a.status, kStatusAttnTimeout)))
-        break;
       tc_fence_after();
       const float* wstat = s_stat + qs * (2 * kB64) + c;
       // query q = q0 + c + i is visible to this key when key <= q (causal)
       // and q < s: lo <= i < hi
       const int lo = (a.causal ? max(key - q0, 0) : 0) - c;
       const int hi = (key < a.s ? min(a.s - q0, kB64) : 0) - c;
-      uint8_t* prow = sPdS + st * (2 * kTile128x64) + (r >> 3) * 1024 + (r & 7) * 128;
-      uint8_t* drow = prow + kTile128x64;
       float sv[32], pv[32];
-      tmem_ld32(tS[st] + lane_off + c, sv);
-      tmem_ld32(tP[st] + lane_off + c, pv);
+      tmem_ld32x2(tS(st) + lane_off + c, sv, tP(st) + lane_off + c, pv);
       uint32_t pk[16], dk[16];
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
@@ -829,15 +875,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         dk[i >> 1] = pack_half2(p[0] * (pv[i] - dv[0]), p[1] * (pv[i + 1] - dv[1]));
         dk[(i >> 1) + 1] = pack_half2(p[2] * (pv[i + 2] - dv[2]), p[3] * (pv[i + 3] - dv[3]));
       }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int off = ((((c >> 3) + q) ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(prow + off) =
-            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        *reinterpret_cast<uint4*>(drow + off) =
-            make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
-      }
-      fence_async_smem();
+      tmem_st16(tS(st) + lane_off + c, pk);  // P^T over this group's S^T columns
+      tmem_st16(tP(st) + lane_off + c, dk);  // dS^T over its dP^T columns
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[st]);
@@ -981,7 +1021,8 @@ tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const vo
                              kSmemKV);
   if (e != cudaSuccess) return cuda_fail(e, "attention bwd smem attribute");
   // (batch element, head) fastest: the CTAs launch in order of decreasing work
-  dim3 gq(static_cast<unsigned>(sh.b * sh.heads), static_cast<unsigned>((sh.s + kBM - 1) / kBM));
+  const int64_t nqb = (sh.s + kBM - 1) / kBM;
+  dim3 gq(static_cast<unsigned>(sh.b * sh.heads), static_cast<unsigned>((nqb + 1) / 2));
   dim3 gk(static_cast<unsigned>(sh.b * sh.heads), static_cast<unsigned>((sh.s + kBN - 1) / kBN));
   attn_bwd_dq_tcgen05<<<gq, kThreadsB, kSmemDQ, stream>>>(qkv128, qkv64, do128, a);
   attn_bwd_dkdv_tcgen05<<<gk, kThreadsB, kSmemKV, stream>>>(qkv128, qkv64, do64, a);

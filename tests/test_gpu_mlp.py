@@ -109,8 +109,13 @@ def test_mlp_config5_sampled():
     inp = make_mlp_inputs(wl)
     out = gpu_mlp(inp, wl.t)
     rng = np.random.default_rng(5)
-    rows = np.unique(np.r_[0, wl.M - 1, rng.integers(0, wl.M, 6)])
-    units = np.unique(np.r_[0, wl.f - 1, wl.f // wl.t, rng.integers(0, wl.f, 13)])
+    # one row from every 128-row tile, and one hidden unit from every 256-wide
+    # column tile of each shard's first and last tiles, plus the edges
+    rows = np.unique(np.r_[0, wl.M - 1, [rng.integers(i, i + 128) for i in range(0, wl.M, 128)]])
+    shard = wl.f // wl.t
+    units = np.unique(np.r_[0, wl.f - 1, [rng.integers(i, i + 256) for i in range(0, wl.f, shard)],
+                            [rng.integers(i - 256, i) for i in range(shard, wl.f + 1, shard)],
+                            rng.integers(0, wl.f, 8)])
     X64, dZ64 = to64(inp["X"]), to64(inp["dZ"])
     A64, B64 = to64(inp["A"]), to64(inp["B"])
     fw = O.mlp_fwd(X64[rows], A64, None, B64, None)
