@@ -486,6 +486,111 @@ def e2e_pipelined(st, steps, stream, barrier):
     return ms, h2d, d2h
 
 
+def other_configs(dev, stream, steps, barrier, peak):
+    """Throughput of the other workloads of the build, each on its own
+    buffers, timed with CUDA events over `steps` calls after two warm-up calls:
+    GPT-2-small MLP fwd+bwd with biases (t = 4), the standalone column- and
+    row-split linears at t = 1, 2, 4, 8, and head-wise attention fwd+bwd
+    (b = 4, s = 2048, h = 4096, 32 heads, t = 8)."""
+    from megatron_tensor_transformer_logical_b200 import binding as L
+    from megatron_tensor_transformer_logical_b200.inputs import (make_attn_inputs,
+                                                                 make_linear_inputs,
+                                                                 make_mlp_inputs)
+    bf = torch.bfloat16
+    out = {}
+
+    def rate(flops, ms):
+        tf = flops / (ms / steps * 1e-3) / 1e12
+        return {"tflops": round(tf, 2), "frac_of_nominal_2250": round(tf / NOMINAL_BF16_TFLOPS, 4),
+                "frac_of_measured_sustained": round(tf / peak, 4)}
+
+    def run(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        L.tp_device_status()
+        barrier()
+        L.tp_profile_enable(True)
+        ms = timed(fn, steps, stream)
+        prof = {name: L.tp_profile_read(k) for k, name in L.KIND_NAMES.items()}
+        L.tp_profile_enable(False)
+        barrier()
+        return ms, prof
+
+    def kernel_split(prof, ms):
+        return {name: {"ms_per_step": round(p["total_ms"] / steps, 4),
+                       "share": round(p["total_ms"] / ms, 4)}
+                for name, p in prof.items() if p["launches"]}
+
+    # Workload 2: GPT-2-small MLP with biases, fwd + bwd (both bias gradients).
+    wl = WORKLOADS[2]
+    d = {k: v.to(dev) for k, v in make_mlp_inputs(wl).items()}
+    M, h, f = wl.M, wl.h, wl.f
+    e = lambda *sh: torch.empty(*sh, dtype=bf, device=dev)
+    Z, Y, dX, dA, dB, dbA, dbB = e(M, h), e(M, f), e(M, h), e(h, f), e(f, h), e(f), e(h)
+    wsf = L.workspace(L.TP_OP_MLP_FWD, M, h, f, 0, wl.t, L.TP_BF16, device=dev)
+    wsb = L.workspace(L.TP_OP_MLP_BWD, M, h, f, 0, wl.t, L.TP_BF16, device=dev)
+
+    def mlp2():
+        L.tp_mlp_fwd(d["X"], d["A"], d["bA"], d["B"], d["bB"], Z, Y, wl.t, wsf)
+        L.tp_mlp_bwd(d["X"], d["A"], d["bA"], d["B"], Y, d["dZ"], dX, dA, dbA, dB, dbB, wl.t, wsb)
+    ms, prof = run(mlp2)
+    fl = 3 * (2.0 * M * f * h * 2)
+    out["2"] = {"workload": f"{wl.name}: MLP fwd+bwd with biases (dbA, dbB), t={wl.t}",
+                "M": M, "h": h, "f": f, "ms_per_step": round(ms / steps, 4),
+                "tokens_per_s": round(M / (ms / steps * 1e-3), 1), **rate(fl, ms),
+                "kernels": kernel_split(prof, ms)}
+    del d, Z, Y, dX, dA, dB, dbA, dbB, wsf, wsb
+
+    # Workload 3: standalone column- and row-split linears.
+    wl = WORKLOADS[3]
+    d = {k: v.to(dev) for k, v in make_linear_inputs(wl).items()}
+    M, K, N = wl.M, wl.h, wl.n_out
+    Yc, Zr = e(M, N), e(M, N)
+    sweep = {}
+    for t in (1, 2, 4, 8):
+        msc, _ = run(lambda: L.tp_linear_col(d["X"], d["W"], None, Yc, t))
+        msr, _ = run(lambda: L.tp_linear_row(d["X"], d["W"], None, Zr, t))
+        fl = 2.0 * M * N * K
+        sweep[f"t{t}"] = {"col": {"ms_per_call": round(msc / steps, 4), **rate(fl, msc)},
+                          "row": {"ms_per_call": round(msr / steps, 4), **rate(fl, msr)}}
+    out["3"] = {"workload": f"{wl.name}: X[{M},{K}] @ W[{K},{N}]", "tokens_per_call": M,
+                "sweep": sweep}
+    del d, Yc, Zr
+
+    # Workload 4: head-wise attention fwd + bwd.
+    wl = WORKLOADS[4]
+    d = {k: v.to(dev) for k, v in make_attn_inputs(wl).items()}
+    M, h = wl.M, wl.h
+    Za, Os, dXa, dWo = e(M, h), e(M, h), e(M, h), e(h, h)
+    QKV = torch.empty(M, 3 * h, dtype=torch.float16, device=dev)
+    LSE = torch.empty(wl.b, wl.heads, wl.s, dtype=torch.float32, device=dev)
+    dWqkv = e(h, 3 * h)
+    wsf = L.workspace(L.TP_OP_ATTN_FWD, M, h, 0, wl.heads, wl.t, L.TP_BF16, device=dev)
+    wsb = L.workspace(L.TP_OP_ATTN_BWD, M, h, 0, wl.heads, wl.t, L.TP_BF16, device=dev)
+
+    def attn4():
+        L.tp_attn_fwd(d["X"], d["Wqkv"], d["Wo"], Za, QKV, Os, LSE, wl.b, wl.s, wl.heads, wl.t,
+                      True, wsf)
+        L.tp_attn_bwd(d["X"], d["Wqkv"], d["Wo"], QKV, Os, LSE, d["dZ"], dXa, dWqkv, dWo, wl.b,
+                      wl.s, wl.heads, wl.t, True, wsb)
+    ms, prof = run(attn4)
+    lf = layer_flops(wl.b, wl.s, wl.h, 4 * wl.h, wl.heads)
+    fl = lf["attn_fwd"] + lf["attn_bwd"]
+    core = {}
+    for name in ("attn_fwd", "attn_bwd"):
+        p = prof[name]
+        if p["launches"]:
+            core[name] = {"ms_per_step": round(p["total_ms"] / steps, 4),
+                          "tflops": round(p["flops"] / (p["total_ms"] * 1e-3) / 1e12, 1)}
+    out["4"] = {"workload": f"{wl.name}: attention fwd+bwd, b={wl.b}, s={wl.s}, h={wl.h}, "
+                            f"{wl.heads} heads, t={wl.t}, causal",
+                "ms_per_step": round(ms / steps, 4),
+                "tokens_per_s": round(M / (ms / steps * 1e-3), 1), **rate(fl, ms),
+                "attention_core": core, "kernels": kernel_split(prof, ms)}
+    return out
+
+
 def run_libtp(args, ranks: Ranks):
     from megatron_tensor_transformer_logical_b200 import binding as L
     rank, world, local_rank = ranks.rank, ranks.world, ranks.local_rank
@@ -573,6 +678,15 @@ def run_libtp(args, ranks: Ranks):
         L.tp_profile_enable(False)
         barrier()
         del vs.logits
+
+    # The build's other workloads (MLP with biases, linear sweep, attention).
+    others = None
+    if not args.no_configs:
+        peaks_, _ = load_peaks()
+        others = other_configs(dev, stream, args.steps, barrier,
+                               float(peaks_.get("bf16_tflops_sustained",
+                                                FALLBACK_PEAKS["bf16_tflops_sustained"])))
+        L.tp_device_status()
 
     # End to end through the public API: per step, the step's inputs (X, dZ)
     # copied from pinned host memory and its results (Z and dX of both
@@ -682,6 +796,8 @@ def run_libtp(args, ranks: Ranks):
     }
     if vocab_ms is not None:
         out["vocab_fwd_bwd"] = vocab_report(vs, args.steps, vocab_ms, vocab_records, peaks, world)
+    if others is not None:
+        out["other_workloads"] = others
     if e2e_ms is not None:
         out["e2e"] = {"value": round(job_rate(fl["total"], world, e2e_ms, args.steps) / 1e12, 2),
                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -777,6 +893,8 @@ def main():
     ap.add_argument("--workload", type=int, default=5, choices=[5])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-vocab", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (MLP with biases, linear sweep, attention)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=768)
     ap.add_argument("--ref-sample-tokens", type=int, default=64)

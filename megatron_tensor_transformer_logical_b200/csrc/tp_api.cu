@@ -310,12 +310,20 @@ namespace {
 
 size_t mlp_fwd_ws(int64_t M, int64_t f, tp_dtype d) { return mlp_fwd_ws_min(M, f, d) + tail_ws(); }
 
-size_t mlp_bwd_ws_min(int64_t M, int64_t h, int64_t f, tp_dtype d) {
-  const size_t mf = align_up(M * f * esize(d), 256);
+// Column-sum scratch of the MLP backward: the two-pass sums of dY and dZ,
+// or the GeLU' GEMM's per-32-row partials of dY (ceil(M / 32) x f floats).
+size_t mlp_bwd_colsum_bytes(int64_t M, int64_t h, int64_t f) {
   size_t cs = colsum_scratch_bytes(M, f);
   const size_t cs2 = colsum_scratch_bytes(M, h);
+  const size_t cs3 = static_cast<size_t>((M + 31) / 32) * static_cast<size_t>(f) * 4;
   if (cs2 > cs) cs = cs2;
-  return 3 * mf + align_up(cs, 256) + 1024;
+  if (cs3 > cs) cs = cs3;
+  return cs;
+}
+
+size_t mlp_bwd_ws_min(int64_t M, int64_t h, int64_t f, tp_dtype d) {
+  const size_t mf = align_up(M * f * esize(d), 256);
+  return 3 * mf + align_up(mlp_bwd_colsum_bytes(M, h, f), 256) + 1024;
 }
 
 size_t mlp_bwd_ws(int64_t M, int64_t h, int64_t f, tp_dtype d) {
@@ -388,9 +396,7 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
   void* dY = c.take(M * f * es);
   void* H = c.take(M * f * es);
   void* Yrec = c.take(M * f * es);
-  size_t cs = colsum_scratch_bytes(M, f);
-  if (colsum_scratch_bytes(M, h) > cs) cs = colsum_scratch_bytes(M, h);
-  void* scratch = c.take(cs);
+  void* scratch = c.take(mlp_bwd_colsum_bytes(M, h, f));
   const Tail tail(c);
 
   const void* Y = Ysave;
@@ -420,6 +426,10 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
   g3.out = dY; g3.ldo = f; g3.out_f32 = f32;
   g3.out2 = (Ysave != nullptr) ? H : nullptr; g3.ldo2 = f;
   g3.n_shard = f / t;
+  // dbA_i = colsum(dY_i): on the tensor-core path the epilogue writes the
+  // column sums of each 32-row group of dY (fp32, before rounding).
+  const bool fused_dba = dbA != nullptr && !f32;
+  if (fused_dba) g3.csum_part = static_cast<float*>(scratch);
   tail.to(g3);
   TP_TRY(run(g3, f32, stream));
 
@@ -454,7 +464,11 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
   tail.to(g6);
   TP_TRY(run(g6, f32, stream));
 
-  if (dbA) TP_TRY(launch_colsum(dY, M, f, f32, dbA, scratch, stream));
+  if (fused_dba)
+    TP_TRY(launch_colsum_finish(static_cast<const float*>(scratch), (M + 31) / 32, f, false, dbA,
+                                stream));
+  else if (dbA)
+    TP_TRY(launch_colsum(dY, M, f, f32, dbA, scratch, stream));
   if (dbB) TP_TRY(launch_colsum(dZ, M, h, f32, dbB, scratch, stream));
   return TP_OK;
 }

@@ -44,28 +44,37 @@ struct AttnArgs {
 };
 
 // ------------------------------------------------------- backward: D term
-// D[bi, head, r] = sum_e dO[row, head*d + e] * O[row, head*d + e]; one warp
-// per (row, head).
-__global__ void attn_bwd_dsum_kernel(const AttnArgs a, float* dsum, long long M) {
-  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (wid >= M * a.heads) return;
-  const long long row = wid / a.heads;
-  const int head = static_cast<int>(wid - row * a.heads);
-  const long long off = row * a.h + head * D + lane * 4;
-  const uint2 ov = *reinterpret_cast<const uint2*>(a.o + off);
-  const uint2 dv = *reinterpret_cast<const uint2*>(a.dout + off);
-  const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-  const __half2* d2 = reinterpret_cast<const __half2*>(&dv);
+// D[bi, head, r] = sum_e dO[row, head*d + e] * O[row, head*d + e].  Sixteen
+// threads per (row, head), each with 16-byte loads of 8 elements of O and
+// dO (a warp reads two heads' 512 contiguous bytes of each), the 16 partial
+// sums added by four shuffle steps.  HBM-bound: 4 bytes read per element.
+__global__ void __launch_bounds__(256) attn_bwd_dsum_kernel(const AttnArgs a, float* dsum,
+                                                             long long M) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long pair = t >> 4;  // (row, head), head fastest
+  const int l16 = threadIdx.x & 15;
+  const bool in = pair < M * a.heads;
   float acc = 0.0f;
+  long long row = 0;
+  int head = 0;
+  if (in) {
+    row = pair / a.heads;
+    head = static_cast<int>(pair - row * a.heads);
+    const long long off = row * a.h + head * D + l16 * 8;
+    const uint4 ov = *reinterpret_cast<const uint4*>(a.o + off);
+    const uint4 dv = *reinterpret_cast<const uint4*>(a.dout + off);
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __half2* d2 = reinterpret_cast<const __half2*>(&dv);
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float2 x = __bfloat1622float2(o2[i]), y = __half22float2(d2[i]);
-    acc += x.x * y.x + x.y * y.y;
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(o2[i]), y = __half22float2(d2[i]);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
+    }
   }
 #pragma unroll
-  for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
-  if (lane == 0) {
+  for (int sh = 8; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+  if (in && l16 == 0) {
     const long long bi = row / a.s, r = row - bi * a.s;
     dsum[(bi * a.heads + head) * a.s + r] = acc;
   }
@@ -114,10 +123,10 @@ tp_status launch_attn_core_bwd(const AttnShape& sh, const void* QKV, const void*
   a.dsum = dsum;
   a.out = static_cast<__nv_bfloat16*>(dQKV);
   const long long M = sh.b * sh.s;
-  const long long warps = M * sh.heads;
+  const long long threads = M * sh.heads * 16;
   LaunchScope scope(TP_KIND_ATTN_BWD, 2.5 * core_flops(sh), 2.0 * double(M) * 8 * sh.h, stream,
                     3);
-  attn_bwd_dsum_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, stream>>>(a, dsum, M);
+  attn_bwd_dsum_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(a, dsum, M);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention bwd (D term) launch");
   return launch_attn_core_bwd_tc(sh, QKV, dO, LSE, dsum, dQKV, stream);

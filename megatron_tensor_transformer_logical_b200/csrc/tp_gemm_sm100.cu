@@ -97,6 +97,10 @@ struct Args {
   // Whole 32-column chunks of a two-byte output go through the shared-memory
   // boxes and the tensor maps tmO (out), tmO2 (out2) and tmX (aux).
   int tma_out;
+  // kEpiDGelu only: column sums of the output (fp32, before rounding) per
+  // 32-row group, csum_part[(row / 32) * csum_ld + col]; nullptr: none.
+  float* csum_part;
+  long long csum_ld;
   WaitCtl status;
 };
 
@@ -328,6 +332,43 @@ __device__ __forceinline__ void epilogue_row32(float (&v)[32], int row, int col0
   if (OUT == kOutF16 && clamped) status_flag(a.status, kFlagF16Range);
 }
 
+// Column sums of one warp's 32 rows x 32 columns (thread = row, v = its 32
+// columns): five butterfly steps, after which lane c holds the sum of column
+// c over the warp's rows (a fixed order, so the result is deterministic).
+// Destroys v.  Every lane of the warp must call it with the same columns.
+__device__ __forceinline__ float warp_colsum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool up = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = up ? v[i] : v[i + w];
+      const float keep = up ? v[i + w] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return v[0];
+}
+
+// The bias gradient of a GeLU' epilogue: after the epilogue has left the
+// output values of rows row0 + lane (row0 a multiple of 32) and columns
+// [col0, col0 + 32) in v, adds this warp's 32-row column sums to the
+// partial array (rows past M and columns past col_end count as zero).
+template <int EPI>
+__device__ __forceinline__ void epilogue_colsum(float (&v)[32], int row, int col0, int col_end,
+                                                int lane, const Args& a) {
+  if constexpr (EPI == kEpiDGelu) {
+    if (a.csum_part == nullptr) return;
+    if (row >= a.M) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+    }
+    const float sum = warp_colsum32(v, lane);
+    if (col0 + lane < col_end)
+      a.csum_part[static_cast<long long>(row >> 5) * a.csum_ld + col0 + lane] = sum;
+  }
+}
+
 // Byte offset of 16-byte chunk j (0-3) of row r in a 32-row x 64-byte box
 // under the 64-byte swizzle (chunk index XOR address bits 7-8; the boxes are
 // 1024-byte aligned).
@@ -471,6 +512,7 @@ __device__ __forceinline__ bool epilogue_chunk_boxed(uint32_t taddr, int lane, i
     epilogue_ce32(v, row, col, col_end, tg, a, box0, lane);
   else
     epilogue_box32<EPI, OUT>(v, lane, col, box0, box1, a);
+  epilogue_colsum<EPI>(v, row, col, col_end, lane, a);
   fence_async_smem();
   __syncwarp();
   if (lane == 0) {
@@ -655,8 +697,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           store_partial32(v, args.tail_part + (static_cast<long long>(w.part) * BM + lrow) * BN + cl);
         else if constexpr (EPI == kEpiCE)
           epilogue_ce32(v, row, col, tc.n_end, tg, args);
-        else
+        else {
           epilogue_row32<EPI, OUT, false>(v, row, col, tc.n_end, args);
+          epilogue_colsum<EPI>(v, row, col, tc.n_end, lane, args);
+        }
       }
       if (!ok) break;
       tc_fence_before();
@@ -899,8 +943,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                  (static_cast<long long>(w.part) * kPairTM + lrow) * kPairTN + cl);
         else if constexpr (EPI == kEpiCE)
           epilogue_ce32(v, row, col, tc.n_end, tg, args);
-        else
+        else {
           epilogue_row32<EPI, OUT, false>(v, row, col, tc.n_end, args);
+          epilogue_colsum<EPI>(v, row, col, tc.n_end, lane, args);
+        }
       }
       if (!ok) break;
       tc_fence_before();
@@ -933,11 +979,15 @@ __global__ void __launch_bounds__(256) gemm_tail_fixup(const Args a) {
   const int tile = a.tail0 + ti;
   const TileCoord tc = PAIR ? tile_coord_pair(tile, a) : tile_coord<TN>(tile, a);
   const float* base = a.tail_part + static_cast<long long>(ti) * a.tail_split * TM * TN;
-  constexpr int kRows = TM / kFixupRowGroups;
+  constexpr int kRows = TM / kFixupRowGroups;  // a multiple of 32
+  static_assert(kRows % 32 == 0, "fixup: a warp takes 32 rows of one chunk");
+  const int lane = threadIdx.x & 31;
+  // Item = (32-column chunk, row): the 32 lanes of a warp take 32 consecutive
+  // rows of one chunk (warp-uniform loop and chunk, as the column sums need).
   for (int item = threadIdx.x; item < kRows * (TN / 32); item += blockDim.x) {
-    const int r = blockIdx.y * kRows + item / (TN / 32);
-    const int cl = (item % (TN / 32)) * 32;
-    if (tc.n0 + cl >= tc.n_end || tc.m0 + r >= a.M) continue;
+    const int r = blockIdx.y * kRows + item % kRows;
+    const int cl = (item / kRows) * 32;
+    if (tc.n0 + cl >= tc.n_end) continue;  // warp-uniform
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = 0.0f;
@@ -954,18 +1004,24 @@ __global__ void __launch_bounds__(256) gemm_tail_fixup(const Args a) {
       }
     }
     epilogue_row32<EPI, OUT, false>(v, tc.m0 + r, tc.n0 + cl, tc.n_end, a);
+    epilogue_colsum<EPI>(v, tc.m0 + r, tc.n0 + cl, tc.n_end, lane, a);
   }
 }
 
-// Splitting the last, partial wave of tiles along K: with T tiles on G
-// persistent CTAs (or CTA pairs) and R = T mod G tiles left for the last
-// wave, those R tiles are cut into S = min(G / R, K blocks / 32) K slices, so
-// the last wave keeps R * S of the G workers busy for 1/S of a tile's time;
-// a fixup kernel adds the slices.  Only when at least one full wave exists,
-// the tail is at most half a wave, every slice keeps at least 32 K blocks
-// (shorter slices cost more in partial traffic than they save), and the
-// caller gave scratch for the R * S fp32 partial tiles.  The result of a tail tile differs from the
-// unsplit one only in the grouping of its fp32 sums.
+// Splitting tiles along K when the tiles alone would leave SMs idle:
+// * the last, partial wave: with T tiles on G persistent CTAs (or CTA pairs)
+//   and R = T mod G tiles left for the last wave (at most half a wave),
+//   those R tiles are cut into S = min(G / R, K blocks / 32) K slices, so
+//   the last wave keeps R * S of the G workers busy for 1/S of a tile's time;
+// * fewer tiles than workers (T < G): all T tiles are cut into
+//   S = min(G / T, K blocks / 32) slices, so T * S workers share them.
+// A fixup kernel adds the slices.  Only when every slice keeps at least 32 K
+// blocks (shorter slices cost more in partial traffic than they save) and
+// the caller gave scratch for the R * S fp32 partial tiles.  The result of a
+// split tile differs from the unsplit one only in the grouping of its fp32
+// sums.
+constexpr int kMinSliceBlocks = 32;
+
 struct TailPlan {
   int units, tail0, split;
 };
@@ -973,11 +1029,16 @@ struct TailPlan {
 TailPlan plan_tail(long long tiles, int workers, int k_blocks, size_t part_bytes,
                    size_t scratch_bytes, int epi) {
   TailPlan tp{static_cast<int>(tiles), static_cast<int>(tiles), 1};
-  if (epi == kEpiCE || scratch_bytes == 0 || tiles <= workers) return tp;
-  const long long R = tiles % workers;
-  if (R == 0 || 2 * R > workers) return tp;
+  if (epi == kEpiCE || scratch_bytes == 0 || tiles == 0) return tp;
+  long long R;
+  if (tiles < workers) {
+    R = tiles;
+  } else {
+    R = tiles % workers;
+    if (R == 0 || 2 * R > workers) return tp;
+  }
   int S = static_cast<int>(workers / R);
-  if (S > k_blocks / 32) S = k_blocks / 32;
+  if (S > k_blocks / kMinSliceBlocks) S = k_blocks / kMinSliceBlocks;
   if (S < 2 || static_cast<size_t>(R) * S * part_bytes > scratch_bytes) return tp;
   tp.tail0 = static_cast<int>(tiles - R);
   tp.split = S;
@@ -1185,6 +1246,8 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   a.ce_cps = g.ce.cps;
   a.ce_target = g.ce.target;
   a.ce_tlogit = g.ce.tlogit;
+  a.csum_part = EPI == kEpiDGelu ? g.csum_part : nullptr;
+  a.csum_ld = g.N;
   a.status = wait_ctl();
   if (a.status.st == nullptr) return fail(TP_ERR_CUDA, "device status unavailable");
   EpiMaps em;
@@ -1205,8 +1268,8 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   }
   const long long tiles = static_cast<long long>(a.m_tiles) * a.n_tiles;
   if (tiles == 0) return TP_OK;
-  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  const TailPlan tp = plan_tail_args(a, grid, size_t(BM) * BN * 4, tail_bytes(g), EPI);
+  const TailPlan tp = plan_tail_args(a, sm_count(), size_t(BM) * BN * 4, tail_bytes(g), EPI);
+  const int grid = static_cast<int>(tp.units < sm_count() ? tp.units : sm_count());
   a.tail_part = static_cast<float*>(g.tail_ws);
   const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
@@ -1279,6 +1342,8 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   a.ce_cps = g.ce.cps;
   a.ce_target = g.ce.target;
   a.ce_tlogit = g.ce.tlogit;
+  a.csum_part = EPI == kEpiDGelu ? g.csum_part : nullptr;
+  a.csum_ld = g.N;
   a.status = wait_ctl();
   if (a.status.st == nullptr) return fail(TP_ERR_CUDA, "device status unavailable");
   EpiMaps em;
@@ -1315,9 +1380,8 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   }
   const long long tiles = static_cast<long long>(a.m_tiles) * a.n_tiles;
   if (tiles == 0) return TP_OK;
-  const int clusters = static_cast<int>(tiles < mc ? tiles : mc);
-  const TailPlan tp =
-      plan_tail_args(a, clusters, size_t(kPairTM) * kPairTN * 4, tail_bytes(g), EPI);
+  const TailPlan tp = plan_tail_args(a, mc, size_t(kPairTM) * kPairTN * 4, tail_bytes(g), EPI);
+  const int clusters = static_cast<int>(tp.units < mc ? tp.units : mc);
   a.tail_part = static_cast<float*>(g.tail_ws);
   const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
@@ -1390,11 +1454,9 @@ int64_t gemm_plan_units(int64_t M, int64_t N, int64_t K, int64_t n_shard, int ki
   const bool pair = kind == 512;
   const int bn = pair ? kPairTN : kind;
   Args a = plan_args(g, bn, pair);
-  const long long tiles = static_cast<long long>(a.m_tiles) * a.n_tiles;
   const int slots = pair ? sms / 2 : sms;  // persistent CTAs, or pairs
-  const int workers = static_cast<int>(tiles < slots ? tiles : slots);
   const size_t scratch = tail_scratch ? static_cast<size_t>(sms) * 128 * 256 * 4 : 0;
-  plan_tail_args(a, workers, size_t(pair ? kPairTM : BM) * bn * 4, scratch, kEpiStore);
+  plan_tail_args(a, slots, size_t(pair ? kPairTM : BM) * bn * 4, scratch, kEpiStore);
   for (int u = 0; u < a.units && u < cap && out != nullptr; ++u) {
     const Unit w = unit_of(u, a);
     TileCoord tc;

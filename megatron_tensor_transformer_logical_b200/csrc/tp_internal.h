@@ -104,6 +104,10 @@ struct Gemm {
   int64_t n_shard = 0;         // columns per shard: column tiles never straddle shards
   KOrder korder;
   CEOut ce;                    // kEpiCE only (requires n_shard % 8 == 0)
+  // kEpiDGelu on the tensor-core path: per-32-row column sums of the output
+  // (fp32, before rounding) to csum_part[(row / 32) * N + col], ceil(M / 32)
+  // rows; finish with launch_colsum_finish.  nullptr: none.
+  float* csum_part = nullptr;
   // Scratch for splitting the last partial wave of tiles along K (optional;
   // gemm_tail_scratch_bytes() is always enough).
   void* tail_ws = nullptr;
@@ -142,6 +146,9 @@ tp_status launch_gemm_f32(const Gemm& g, cudaStream_t stream);
 size_t colsum_scratch_bytes(int64_t rows, int64_t cols);
 tp_status launch_colsum(const void* in, int64_t rows, int64_t cols, bool f32, void* out,
                         void* scratch, cudaStream_t stream);
+// out[c] = sum over k < chunks of part[k * cols + c], in k order (bf16 or f32).
+tp_status launch_colsum_finish(const float* part, int64_t chunks, int64_t cols, bool f32,
+                               void* out, cudaStream_t stream);
 
 // LayerNorm over rows of [M, h] (h % 8 == 0, h <= layernorm_max_h()).
 int64_t layernorm_max_h();

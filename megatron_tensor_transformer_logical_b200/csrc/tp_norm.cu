@@ -88,8 +88,12 @@ __device__ __forceinline__ float2 block_sum2(float a, float b, float2* red) {
 // first forms the sums of (x - K) and (x - K)^2 with K = the row's first
 // element (the shifted-data form of the variance: with K a sample of the row
 // the two sums do not cancel), one block reduction for both; the second pass
-// re-reads the row (from L2) and writes Y.  No row data stays in registers,
-// so several rows run per SM.
+// re-reads the row (from L2) and writes Y.  Each pass issues all of a
+// thread's 16-byte loads (at most 8 at h = 16384) before using them, so a
+// CTA keeps its whole row in flight; no row data stays in registers across
+// the reduction, so several rows run per SM.
+constexpr int kLnMaxChunks = kLnMaxH / 8 / kLnBwdThreads;  // 8
+
 template <bool F32>
 __global__ void __launch_bounds__(kLnBwdThreads)
     layernorm_fwd_kernel(const void* X, const void* gamma, const void* beta, void* Y, float* mean,
@@ -101,22 +105,53 @@ __global__ void __launch_bounds__(kLnBwdThreads)
   const float K = F32 ? static_cast<const float*>(X)[base]
                       : __bfloat162float(static_cast<const __nv_bfloat16*>(X)[base]);
   float s1 = 0.0f, s2 = 0.0f;
-#pragma unroll 2
-  for (int ch = threadIdx.x; ch < nch; ch += kLnBwdThreads) {
-    float x[8];
-    load8<F32>(X, base + ch * 8, x);
+  {
+    // the raw 16-byte words (bf16: one per chunk, 32 registers at most)
+    constexpr int kWords = F32 ? 2 : 1;
+    uint4 raw[kLnMaxChunks * kWords];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float d = x[i] - K;
-      s1 += d;
-      s2 += d * d;
+    for (int k = 0; k < kLnMaxChunks; ++k) {
+      const int ch = threadIdx.x + k * kLnBwdThreads;
+      if (ch < nch) {
+        const uint4* p =
+            F32 ? reinterpret_cast<const uint4*>(static_cast<const float*>(X) + base + ch * 8)
+                : reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(X) + base +
+                                                 ch * 8);
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) raw[k * kWords + w] = p[w];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kLnMaxChunks; ++k) {
+      if (threadIdx.x + k * kLnBwdThreads < nch) {
+        float x[8];
+        if (F32) {
+          const float* f = reinterpret_cast<const float*>(&raw[k * kWords]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[i] = f[i];
+        } else {
+          const __nv_bfloat162* q = reinterpret_cast<const __nv_bfloat162*>(&raw[k * kWords]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 t = __bfloat1622float2(q[i]);
+            x[2 * i] = t.x;
+            x[2 * i + 1] = t.y;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float d = x[i] - K;
+          s1 += d;
+          s2 += d * d;
+        }
+      }
     }
   }
   const float2 m = block_sum2(s1, s2, red);
   const float d1 = m.x / h;
   const float mu = K + d1;
   const float rs = rsqrtf(fmaxf(m.y / h - d1 * d1, 0.0f) + eps);
-#pragma unroll 2
+#pragma unroll 4
   for (int ch = threadIdx.x; ch < nch; ch += kLnBwdThreads) {
     float x[8], g[8], b[8], y[8];
     load8<F32>(X, base + ch * 8, x);

@@ -17,6 +17,19 @@ Cases (175B-shaped layer unless noted; bf16, t = 8):
               V=51200, t=8, Zipf token ids): embedding gather, logits
               GEMM with the loss epilogue, loss combination, softmax gradient,
               dX and dE GEMMs, embedding scatter-add
+  layernorm   tp_layernorm_fwd + tp_layernorm_bwd on X[8192,12288] (201 MB, larger
+              than L2), gamma and beta, with a residual gradient
+  mlp_bwd_bias tp_mlp_bwd with both bias gradients, M=8192, h=12288, f=1024, t=8:
+              dbB = colsum(dZ [8192,12288]) runs the two-pass column sum over 201 MB,
+              dbA the GeLU' epilogue's partials and the finishing pass
+  attn_bwd_big tp_attn_bwd at b=2, s=4096, h=6144 (48 heads; about 2.7 GB on the
+              device): the D = rowsum(dO * O) kernel reads 2 x 100 MB
+  linear_f32  tp_linear_col in fp32, X[4096,4096] @ W[4096,4096] (the CUDA-core path)
+  mlp_bwd_quarter tp_mlp_bwd with f = 12288 (a quarter of the layer's width; about 2 GB on
+              the device): the four backward GEMMs with the 175B-shaped M and h
+  attn_small  tp_attn_fwd + tp_attn_bwd on one head group of the 175B-shaped layer:
+              b=1, s=2048, h=1536 (12 heads of 128), t=1, causal (a small case for
+              full ncu captures of the attention kernels)
 
 Inputs are seeded N(0,1) / N(0, 0.006^2) tensors made on the device; nothing
 is checked here (the tests do that).  Prints the mean device time per call.
@@ -119,6 +132,76 @@ def make_case(name: str):
             L.tp_vocab_ce_bwd(X, E, targets, logits, lse, None, logits, dX, dE, t)
             L.tp_vocab_embed_bwd(ids, dY, dE, dE, t, wse)
         return step
+    if name == "layernorm":
+        Mb = 8192
+        X, dY, dR = _t((Mb, h), 1.0), _t((Mb, h), 1.0, seed=1), _t((Mb, h), 1.0, seed=2)
+        g, b = 1.0 + _t((h,), 0.1, seed=3), _t((h,), 0.1, seed=4)
+        Y, dX = torch.empty_like(X), torch.empty_like(X)
+        mean = torch.empty(Mb, dtype=torch.float32, device="cuda")
+        rstd = torch.empty_like(mean)
+        dg, db = torch.empty_like(g), torch.empty_like(b)
+        ws = L.workspace(L.TP_OP_LN_BWD, Mb, h, 0, 0, 1, L.TP_BF16)
+
+        def ln():
+            L.tp_layernorm_fwd(X, g, b, Y, mean, rstd, 1e-5)
+            L.tp_layernorm_bwd(X, g, mean, rstd, dY, dR, dX, dg, db, ws)
+        return ln
+    if name == "mlp_bwd_bias":
+        Mb, fb = 8192, 1024
+        X, A, B = _t((Mb, h), 1.0), _t((h, fb), 0.006, seed=1), _t((fb, h), 0.006, seed=2)
+        bA, bB = _t((fb,), 0.01, seed=5), _t((h,), 0.01, seed=6)
+        dZ = _t((Mb, h), 1.0, seed=3)
+        Z, Y = torch.empty(Mb, h, dtype=bf, device="cuda"), torch.empty(Mb, fb, dtype=bf, device="cuda")
+        L.tp_mlp_fwd(X, A, bA, B, bB, Z, Y, t, L.workspace(L.TP_OP_MLP_FWD, Mb, h, fb, 0, t, L.TP_BF16))
+        dX, dA, dB = torch.empty_like(X), torch.empty_like(A), torch.empty_like(B)
+        dbA, dbB = torch.empty_like(bA), torch.empty_like(bB)
+        wsb = L.workspace(L.TP_OP_MLP_BWD, Mb, h, fb, 0, t, L.TP_BF16)
+        return lambda: L.tp_mlp_bwd(X, A, bA, B, Y, dZ, dX, dA, dbA, dB, dbB, t, wsb)
+    if name == "attn_bwd_big":
+        b2, s2 = 2, 4096
+        Mb = b2 * s2
+        h, heads = 6144, 48
+        X, Wqkv, Wo = _t((Mb, h), 1.0), _t((h, 3 * h), 0.006, seed=1), _t((h, h), 0.006, seed=2)
+        dZ = _t((Mb, h), 1.0, seed=3)
+        Z = torch.empty(Mb, h, dtype=bf, device="cuda")
+        QKV = torch.empty(Mb, 3 * h, dtype=torch.float16, device="cuda")
+        O = torch.empty(Mb, h, dtype=bf, device="cuda")
+        LSE = torch.empty(b2, heads, s2, dtype=torch.float32, device="cuda")
+        L.tp_attn_fwd(X, Wqkv, Wo, Z, QKV, O, LSE, b2, s2, heads, t, True,
+                      L.workspace(L.TP_OP_ATTN_FWD, Mb, h, 0, heads, t, L.TP_BF16))
+        dX, dWqkv, dWo = torch.empty_like(X), torch.empty_like(Wqkv), torch.empty_like(Wo)
+        wsb = L.workspace(L.TP_OP_ATTN_BWD, Mb, h, 0, heads, t, L.TP_BF16)
+        return lambda: L.tp_attn_bwd(X, Wqkv, Wo, QKV, O, LSE, dZ, dX, dWqkv, dWo, b2, s2, heads,
+                                     t, True, wsb)
+    if name == "mlp_bwd_quarter":
+        fq = 12288
+        X, A, B = _t((M, h), 1.0), _t((h, fq), 0.006, seed=1), _t((fq, h), 0.006, seed=2)
+        dZ = _t((M, h), 1.0, seed=3)
+        Z, Y = torch.empty(M, h, dtype=bf, device="cuda"), torch.empty(M, fq, dtype=bf, device="cuda")
+        L.tp_mlp_fwd(X, A, None, B, None, Z, Y, t, L.workspace(L.TP_OP_MLP_FWD, M, h, fq, 0, t, L.TP_BF16))
+        dX, dA, dB = torch.empty_like(X), torch.empty_like(A), torch.empty_like(B)
+        wsb = L.workspace(L.TP_OP_MLP_BWD, M, h, fq, 0, t, L.TP_BF16)
+        return lambda: L.tp_mlp_bwd(X, A, None, B, Y, dZ, dX, dA, None, dB, None, t, wsb)
+    if name == "attn_small":
+        hs, hd = 1536, 12
+        X, Wqkv, Wo = _t((M, hs), 1.0), _t((hs, 3 * hs), 0.02, seed=1), _t((hs, hs), 0.02, seed=2)
+        dZ = _t((M, hs), 1.0, seed=3)
+        Z = torch.empty(M, hs, dtype=bf, device="cuda")
+        QKV = torch.empty(M, 3 * hs, dtype=torch.float16, device="cuda")
+        O = torch.empty(M, hs, dtype=bf, device="cuda")
+        LSE = torch.empty(1, hd, M, dtype=torch.float32, device="cuda")
+        dX, dWqkv, dWo = torch.empty_like(X), torch.empty_like(Wqkv), torch.empty_like(Wo)
+        wsf = L.workspace(L.TP_OP_ATTN_FWD, M, hs, 0, hd, 1, L.TP_BF16)
+        wsb = L.workspace(L.TP_OP_ATTN_BWD, M, hs, 0, hd, 1, L.TP_BF16)
+
+        def small():
+            L.tp_attn_fwd(X, Wqkv, Wo, Z, QKV, O, LSE, 1, M, hd, 1, True, wsf)
+            L.tp_attn_bwd(X, Wqkv, Wo, QKV, O, LSE, dZ, dX, dWqkv, dWo, 1, M, hd, 1, True, wsb)
+        return small
+    if name == "linear_f32":
+        X, W = _t((4096, 4096), 1.0, torch.float32), _t((4096, 4096), 0.02, torch.float32, seed=1)
+        Y = torch.empty(4096, 4096, dtype=torch.float32, device="cuda")
+        return lambda: L.tp_linear_col(X, W, None, Y, 2)
     raise SystemExit(f"unknown case {name}")
 
 

@@ -10,7 +10,9 @@ element exactly once over the whole K range:
   columns: the column split of "图解Transformer并行计算" §1.2);
 * each tile's units cover its K blocks [0, ceil(K / 64)) exactly once, in
   order: one whole unit, or K slices with distinct partial-tile indices
-  that fit the last-wave scratch (split only in the last, short wave);
+  that fit the scratch (split only in the last, short wave, or every tile
+  when there are fewer tiles than persistent CTAs), each slice at least 32
+  K blocks deep;
 * every unit is a tile of the grid and the unit count matches the plan.
 """
 import random
@@ -55,11 +57,17 @@ def _check_plan(M, N, K, n_shard, kind, sms, scratch):
         assert scratch, "K slices need the last-wave scratch"
         assert max(parts) + 1 == len(parts)
         assert len(parts) * rows * cols * 4 <= sms * 128 * 256 * 4
-        # only the last tiles (the short last wave) are split, at most half a wave
         n_tiles = len(by_tile)
-        workers = min(n_tiles, sms // 2 if kind == 512 else sms)
-        assert sorted(split_tiles) == list(range(n_tiles - len(split_tiles), n_tiles))
-        assert 2 * len(split_tiles) <= workers
+        slots = sms // 2 if kind == 512 else sms
+        if n_tiles < slots:
+            # fewer tiles than workers: every tile is split, within the workers
+            assert sorted(split_tiles) == list(range(n_tiles))
+            assert len(parts) <= slots
+        else:
+            # only the last tiles (the short last wave) are split, at most half a wave
+            assert sorted(split_tiles) == list(range(n_tiles - len(split_tiles), n_tiles))
+            assert 2 * len(split_tiles) <= slots
+            assert len(split_tiles) == n_tiles % slots
         # every slice is at least 32 K blocks deep
         assert all(v["kb1"] - v["kb0"] >= 32 for t in split_tiles for v in by_tile[t][:-1])
     # spatial coverage: per row band, the column ranges partition [0, N)
@@ -116,6 +124,17 @@ def test_short_last_wave_is_split():
     assert sum(u["part"] >= 0 for u in units) == 28 * 5
     units = L.tp_gemm_plan(2048, 12288, 49152, 0, 256, 148, False)
     assert len(units) == 768 and all(u["part"] == -1 for u in units)
+
+
+def test_tile_starved_gemm_is_split():
+    """A wgrad of the GPT-2-small MLP (M = 3072, N = 768, K = 8192): 72 tiles
+    of 128 x 256 for 148 SMs, so every tile is cut into two K slices of 64
+    blocks (144 units); without the scratch the 72 tiles run whole."""
+    units = L.tp_gemm_plan(3072, 768, 8192, 0, 256, 148, True)
+    assert len(units) == 144 and all(u["part"] >= 0 for u in units)
+    assert {u["kb1"] - u["kb0"] for u in units} == {64}
+    units = L.tp_gemm_plan(3072, 768, 8192, 0, 256, 148, False)
+    assert len(units) == 72
 
 
 def test_invalid_plan_requests():
