@@ -76,16 +76,18 @@ def gemm_source_hash():
 
 
 def traffic_per_launch():
-    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
-    taken on the current kernel source; otherwise None."""
+    """DRAM bytes per GEMM launch from the committed ncu capture (and the
+    launches it covers, with their algorithmic bytes), if it was taken on the
+    current kernel source; otherwise (None, None, None)."""
     p = os.path.join(ROOT, "profiles", "gemm_tcgen05_traffic.json")
     if not os.path.exists(p):
-        return None
+        return None, None, None
     with open(p) as fh:
         d = json.load(fh)
     if d.get("source_sha256_16") != gemm_source_hash():
-        return None
-    return d.get("dram_bytes_per_launch")
+        return None, None, None
+    return (d.get("dram_bytes_per_launch"), d.get("scope"),
+            d.get("algorithmic_bytes_per_launch"))
 
 
 # ------------------------------------------------------------ clock sampling
@@ -717,7 +719,7 @@ def run_libtp(args, ranks: Ranks):
     g = prof["gemm_tcgen05"]
     achieved = g["flops"] / (g["total_ms"] * 1e-3) / 1e12 if g["total_ms"] > 0 else 0.0
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    traffic = traffic_per_launch()
+    traffic, traffic_scope, traffic_alg = traffic_per_launch()
     mlp_tflops = world * (fl["mlp_fwd"] + fl["mlp_bwd"]) / (mlp_ms / args.steps * 1e-3) / 1e12
     gemms = {}
     for r in records:
@@ -787,6 +789,8 @@ def run_libtp(args, ranks: Ranks):
                      "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_src} bf16_tflops_sustained",
                      "traffic": traffic,
+                     "traffic_scope": traffic_scope,
+                     "traffic_algorithmic_bytes_per_launch": traffic_alg,
                      "algorithmic_bytes_per_launch": (g["bytes"] / g["launches"]) if g["launches"] else None,
                      "flops_per_launch": (g["flops"] / g["launches"]) if g["launches"] else None},
         "kernels": kernels,

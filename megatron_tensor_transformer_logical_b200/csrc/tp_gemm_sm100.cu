@@ -91,9 +91,12 @@ struct Args {
   float* ce_tlogit;
   // Work units: tiles [0, tail0) whole; each later tile split into
   // tail_split slices of its K blocks, whose fp32 partial tiles go to
-  // tail_part and are summed (slice order) by gemm_tail_fixup.
+  // tail_part; the CTA that stores a tile's last slice adds them (slice
+  // order) and applies the epilogue (tail_ctr: one arrival counter per split
+  // tile, per CTA of a pair).
   int units, tail0, tail_split;
   float* tail_part;
+  unsigned long long* tail_ctr;
   // Whole 32-column chunks of a two-byte output go through the shared-memory
   // boxes and the tensor maps tmO (out), tmO2 (out2) and tmX (aux).
   int tma_out;
@@ -133,6 +136,22 @@ __device__ __forceinline__ void store_partial32(const float (&v)[32], float* dst
   float4* d = reinterpret_cast<float4*>(dst);
 #pragma unroll
   for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
+// Counts one arrival of a split tile's slice on its counter and returns
+// whether it was the last of `split`.  The counter holds (launch generation
+// << 8) | arrivals, so the counters need no clearing between launches: a
+// value from an earlier launch counts as zero.  One thread calls it, after
+// the CTA's partial-tile stores and a __threadfence().
+__device__ __forceinline__ bool tail_ticket(unsigned long long* ctr, unsigned long long gen,
+                                            int split) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(ctr);
+  for (;;) {
+    const unsigned long long want = ((cur >> 8) == gen) ? cur + 1ull : ((gen << 8) | 1ull);
+    const unsigned long long prev = atomicCAS(ctr, cur, want);
+    if (prev == cur) return static_cast<int>(want & 0xffull) == split;
+    cur = prev;  // another slice arrived in between: retry on its value
+  }
 }
 
 struct TileCoord {
@@ -523,6 +542,58 @@ __device__ __forceinline__ bool epilogue_chunk_boxed(uint32_t taddr, int lane, i
   return true;
 }
 
+// The final pass over a split tile, run by the CTA that stored its last
+// slice: each epilogue thread adds its row's 32-column chunks of the
+// tile's slices in slice order (L2 loads: other SMs wrote them) and applies
+// the epilogue, as a whole tile's epilogue would; `lrow` is the row within
+// the TM x TN partial tile, `half` the epilogue warp's half of the columns.
+template <int TM, int TN, int EPI, int OUT>
+__device__ __forceinline__ void tail_finish(const Args& a, const TileCoord& tc, int ti, int lrow,
+                                            int row, int half, int lane) {
+  const float* base = a.tail_part + static_cast<long long>(ti) * a.tail_split * TM * TN;
+#pragma unroll 1
+  for (int c = 0; c < TN / 2; c += 32) {
+    const int cl = half * (TN / 2) + c;
+    const int col = tc.n0 + cl;
+    if (col >= tc.n_end) break;  // warp-uniform
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+    for (int ks = 0; ks < a.tail_split; ++ks) {
+      const float4* src = reinterpret_cast<const float4*>(
+          base + (static_cast<long long>(ks) * TM + lrow) * TN + cl);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 q = __ldcg(src + i);
+        v[4 * i] += q.x;
+        v[4 * i + 1] += q.y;
+        v[4 * i + 2] += q.z;
+        v[4 * i + 3] += q.w;
+      }
+    }
+    epilogue_row32<EPI, OUT, false>(v, row, col, tc.n_end, a);
+    epilogue_colsum<EPI>(v, row, col, tc.n_end, lane, a);
+  }
+}
+
+// After a CTA's epilogue warps stored their parts of a slice of split tile
+// ti (counter slot `slot`): the last CTA to do so for that tile finishes it.
+// Called by all epilogue warps of the CTA together (named barrier 1).
+template <int TM, int TN, int EPI, int OUT>
+__device__ __forceinline__ void tail_arrive(const Args& a, const TileCoord& tc, int ti, int slot,
+                                            int lrow, int row, int half, int lane, int ew,
+                                            int* flag) {
+  __threadfence();
+  named_sync(1, kEpiWarps * 32);
+  if (ew == 0 && lane == 0)
+    *flag = tail_ticket(a.tail_ctr + slot, a.status.gen, a.tail_split) ? 1 : 0;
+  named_sync(1, kEpiWarps * 32);
+  if (*reinterpret_cast<volatile int*>(flag)) {
+    __threadfence();
+    tail_finish<TM, TN, EPI, OUT>(a, tc, ti, lrow, row, half, lane);
+  }
+}
+
 template <int BN, bool A_KMAJ, bool B_KMAJ, int EPI, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA,
@@ -543,6 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* auxbar = tempty + 2;  // one per epilogue warp
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + kEpiWarps);
+  int* tail_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -706,6 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (w.part >= 0)
+        tail_arrive<BM, BN, EPI, OUT>(args, tc, w.tile - args.tail0, w.tile - args.tail0, lrow,
+                                      row, half, lane, ew, tail_flag);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -778,6 +853,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* auxbar = tempty + 2;  // one per epilogue warp
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + kEpiWarps);
+  int* tail_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -952,6 +1028,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
+      if (w.part >= 0)  // each CTA of the pair finishes its own 128 rows
+        tail_arrive<kPairTM, kPairTN, EPI, OUT>(args, tc, w.tile - args.tail0,
+                                                2 * (w.tile - args.tail0) + static_cast<int>(rank),
+                                                lrow, row, half, lane, ew, tail_flag);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -968,59 +1048,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
 }
 
-// Sums the K-slice partials of each tail tile in slice order and applies the
-// GEMM's epilogue, exactly as the GEMM kernel would have for a whole tile.
-// CTA (tail tile, quarter of its rows); a thread handles 32 columns of one row.
-constexpr int kFixupRowGroups = 4;
-
-template <int TM, int TN, bool PAIR, int EPI, int OUT>
-__global__ void __launch_bounds__(256) gemm_tail_fixup(const Args a) {
-  const int ti = blockIdx.x;
-  const int tile = a.tail0 + ti;
-  const TileCoord tc = PAIR ? tile_coord_pair(tile, a) : tile_coord<TN>(tile, a);
-  const float* base = a.tail_part + static_cast<long long>(ti) * a.tail_split * TM * TN;
-  constexpr int kRows = TM / kFixupRowGroups;  // a multiple of 32
-  static_assert(kRows % 32 == 0, "fixup: a warp takes 32 rows of one chunk");
-  const int lane = threadIdx.x & 31;
-  // Item = (32-column chunk, row): the 32 lanes of a warp take 32 consecutive
-  // rows of one chunk (warp-uniform loop and chunk, as the column sums need).
-  for (int item = threadIdx.x; item < kRows * (TN / 32); item += blockDim.x) {
-    const int r = blockIdx.y * kRows + item % kRows;
-    const int cl = (item / kRows) * 32;
-    if (tc.n0 + cl >= tc.n_end) continue;  // warp-uniform
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-    for (int ks = 0; ks < a.tail_split; ++ks) {
-      const float4* src = reinterpret_cast<const float4*>(
-          base + (static_cast<long long>(ks) * TM + r) * TN + cl);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 q = src[i];
-        v[4 * i] += q.x;
-        v[4 * i + 1] += q.y;
-        v[4 * i + 2] += q.z;
-        v[4 * i + 3] += q.w;
-      }
-    }
-    epilogue_row32<EPI, OUT, false>(v, tc.m0 + r, tc.n0 + cl, tc.n_end, a);
-    epilogue_colsum<EPI>(v, tc.m0 + r, tc.n0 + cl, tc.n_end, lane, a);
-  }
-}
-
 // Splitting tiles along K when the tiles alone would leave SMs idle:
 // * the last, partial wave: with T tiles on G persistent CTAs (or CTA pairs)
 //   and R = T mod G tiles left for the last wave (at most half a wave),
-//   those R tiles are cut into S = min(G / R, K blocks / 32) K slices, so
+//   those R tiles are cut into S = min(G / R, K blocks / B) K slices, so
 //   the last wave keeps R * S of the G workers busy for 1/S of a tile's time;
 // * fewer tiles than workers (T < G): all T tiles are cut into
-//   S = min(G / T, K blocks / 32) slices, so T * S workers share them.
-// A fixup kernel adds the slices.  Only when every slice keeps at least 32 K
-// blocks (shorter slices cost more in partial traffic than they save) and
-// the caller gave scratch for the R * S fp32 partial tiles.  The result of a
+//   S = min(G / T, K blocks / B) slices, so T * S workers share them.
+// The CTA that stores a tile's last slice adds the slices (tail_finish).
+// B = 32 K blocks (shorter slices cost more in partial traffic than they
+// save), or 16 for a GEMM of fewer than four waves, whose last wave is a
+// large share of its time; and only when the caller gave scratch for the
+// R * S fp32 partial tiles.  The result of a
 // split tile differs from the unsplit one only in the grouping of its fp32
 // sums.
 constexpr int kMinSliceBlocks = 32;
+// The split tiles' arrival counters sit at the start of the scratch (at most
+// one tile per worker, two counters per tile for a CTA pair), the partial
+// tiles after them.
+constexpr size_t kTailCtrBytes = 4096;
 
 struct TailPlan {
   int units, tail0, split;
@@ -1029,7 +1075,8 @@ struct TailPlan {
 TailPlan plan_tail(long long tiles, int workers, int k_blocks, size_t part_bytes,
                    size_t scratch_bytes, int epi) {
   TailPlan tp{static_cast<int>(tiles), static_cast<int>(tiles), 1};
-  if (epi == kEpiCE || scratch_bytes == 0 || tiles == 0) return tp;
+  if (epi == kEpiCE || scratch_bytes <= kTailCtrBytes || tiles == 0) return tp;
+  scratch_bytes -= kTailCtrBytes;
   long long R;
   if (tiles < workers) {
     R = tiles;
@@ -1037,8 +1084,11 @@ TailPlan plan_tail(long long tiles, int workers, int k_blocks, size_t part_bytes
     R = tiles % workers;
     if (R == 0 || 2 * R > workers) return tp;
   }
+  // A GEMM of fewer than 4 waves loses a large share of its time to the
+  // short last wave, so its slices may be as short as 16 K blocks.
+  const int min_slice = tiles < 4LL * workers ? kMinSliceBlocks / 2 : kMinSliceBlocks;
   int S = static_cast<int>(workers / R);
-  if (S > k_blocks / kMinSliceBlocks) S = k_blocks / kMinSliceBlocks;
+  if (S > k_blocks / min_slice) S = k_blocks / min_slice;
   if (S < 2 || static_cast<size_t>(R) * S * part_bytes > scratch_bytes) return tp;
   tp.tail0 = static_cast<int>(tiles - R);
   tp.split = S;
@@ -1270,7 +1320,8 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   if (tiles == 0) return TP_OK;
   const TailPlan tp = plan_tail_args(a, sm_count(), size_t(BM) * BN * 4, tail_bytes(g), EPI);
   const int grid = static_cast<int>(tp.units < sm_count() ? tp.units : sm_count());
-  a.tail_part = static_cast<float*>(g.tail_ws);
+  a.tail_ctr = static_cast<unsigned long long*>(g.tail_ws);
+  a.tail_part = reinterpret_cast<float*>(static_cast<char*>(g.tail_ws) + kTailCtrBytes);
   const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
                        (OUT == kOutF32 ? 4.0 : 2.0) * double(g.M) * g.N +
@@ -1278,12 +1329,8 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
                        (g.aux ? 2.0 * double(g.M) * g.N : 0.0) +
                        (EPI == kEpiCE ? 8.0 * double(g.M) * g.N / 32.0 : 0.0);
   {
-    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, tp.split > 1 ? 2 : 1, BN, g.M,
-                      g.N, g.K);
+    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, 1, BN, g.M, g.N, g.K);
     kern<<<grid, kThreads, C::kSmemBytes, stream>>>(ta, tb, em.o, em.o2, em.x, a);
-    if (tp.split > 1)
-      gemm_tail_fixup<BM, BN, false, EPI, OUT>
-          <<<dim3(static_cast<unsigned>(tiles - tp.tail0), kFixupRowGroups), 256, 0, stream>>>(a);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm_bf16_tcgen05 launch");
@@ -1382,7 +1429,8 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
   if (tiles == 0) return TP_OK;
   const TailPlan tp = plan_tail_args(a, mc, size_t(kPairTM) * kPairTN * 4, tail_bytes(g), EPI);
   const int clusters = static_cast<int>(tp.units < mc ? tp.units : mc);
-  a.tail_part = static_cast<float*>(g.tail_ws);
+  a.tail_ctr = static_cast<unsigned long long*>(g.tail_ws);
+  a.tail_part = reinterpret_cast<float*>(static_cast<char*>(g.tail_ws) + kTailCtrBytes);
   const double flops = 2.0 * double(g.M) * double(g.N) * double(g.K);
   const double bytes = 2.0 * (double(g.M) * g.K + double(g.K) * g.N) +
                        (OUT == kOutF32 ? 4.0 : 2.0) * double(g.M) * g.N +
@@ -1390,12 +1438,8 @@ tp_status launch_pair(const Gemm& g, cudaStream_t stream) {
                        (g.aux ? 2.0 * double(g.M) * g.N : 0.0) +
                        (EPI == kEpiCE ? 8.0 * double(g.M) * g.N / 32.0 : 0.0);
   {
-    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, tp.split > 1 ? 2 : 1, 512, g.M,
-                      g.N, g.K);
+    LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, 1, 512, g.M, g.N, g.K);
     kern<<<2 * clusters, kThreads, kPairSmemBytes, stream>>>(ta, tb, em.o, em.o2, em.x, a);
-    if (tp.split > 1)
-      gemm_tail_fixup<kPairTM, kPairTN, true, EPI, OUT>
-          <<<dim3(static_cast<unsigned>(tiles - tp.tail0), kFixupRowGroups), 256, 0, stream>>>(a);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm_bf16_tcgen05_pair launch");
@@ -1434,9 +1478,9 @@ tp_status dispatch_pair(const Gemm& g, cudaStream_t s) {
 }  // namespace
 
 size_t gemm_tail_scratch_bytes() {
-  // At most one partial tile per persistent CTA (128 x 256 fp32) or per CTA
-  // pair (256 x 256 fp32, half as many pairs).
-  return static_cast<size_t>(sm_count()) * 128 * 256 * 4;
+  // The arrival counters, then at most one partial tile per persistent CTA
+  // (128 x 256 fp32) or per CTA pair (256 x 256 fp32, half as many pairs).
+  return kTailCtrBytes + static_cast<size_t>(sm_count()) * 128 * 256 * 4;
 }
 
 int64_t gemm_plan_units(int64_t M, int64_t N, int64_t K, int64_t n_shard, int kind, int sms,
@@ -1455,7 +1499,8 @@ int64_t gemm_plan_units(int64_t M, int64_t N, int64_t K, int64_t n_shard, int ki
   const int bn = pair ? kPairTN : kind;
   Args a = plan_args(g, bn, pair);
   const int slots = pair ? sms / 2 : sms;  // persistent CTAs, or pairs
-  const size_t scratch = tail_scratch ? static_cast<size_t>(sms) * 128 * 256 * 4 : 0;
+  const size_t scratch =
+      tail_scratch ? kTailCtrBytes + static_cast<size_t>(sms) * 128 * 256 * 4 : 0;
   plan_tail_args(a, slots, size_t(pair ? kPairTM : BM) * bn * 4, scratch, kEpiStore);
   for (int u = 0; u < a.units && u < cap && out != nullptr; ++u) {
     const Unit w = unit_of(u, a);

@@ -27,9 +27,10 @@ Cases (175B-shaped layer unless noted; bf16, t = 8):
   linear_f32  tp_linear_col in fp32, X[4096,4096] @ W[4096,4096] (the CUDA-core path)
   mlp_bwd_quarter tp_mlp_bwd with f = 12288 (a quarter of the layer's width; about 2 GB on
               the device): the four backward GEMMs with the 175B-shaped M and h
-  attn_small  tp_attn_fwd + tp_attn_bwd on one head group of the 175B-shaped layer:
-              b=1, s=2048, h=1536 (12 heads of 128), t=1, causal (a small case for
-              full ncu captures of the attention kernels)
+  attn_small  tp_attn_fwd + tp_attn_bwd on two head groups of the 175B-shaped layer:
+              b=1, s=2048, h=3072 (24 heads of 128, 192 forward CTAs, more than one
+              per SM), t=2, causal (a small case for full ncu captures of the
+              attention kernels)
 
 Inputs are seeded N(0,1) / N(0, 0.006^2) tensors made on the device; nothing
 is checked here (the tests do that).  Prints the mean device time per call.
@@ -183,7 +184,7 @@ def make_case(name: str):
         wsb = L.workspace(L.TP_OP_MLP_BWD, M, h, fq, 0, t, L.TP_BF16)
         return lambda: L.tp_mlp_bwd(X, A, None, B, Y, dZ, dX, dA, None, dB, None, t, wsb)
     if name == "attn_small":
-        hs, hd = 1536, 12
+        hs, hd = 3072, 24
         X, Wqkv, Wo = _t((M, hs), 1.0), _t((hs, 3 * hs), 0.02, seed=1), _t((hs, hs), 0.02, seed=2)
         dZ = _t((M, hs), 1.0, seed=3)
         Z = torch.empty(M, hs, dtype=bf, device="cuda")
@@ -191,12 +192,12 @@ def make_case(name: str):
         O = torch.empty(M, hs, dtype=bf, device="cuda")
         LSE = torch.empty(1, hd, M, dtype=torch.float32, device="cuda")
         dX, dWqkv, dWo = torch.empty_like(X), torch.empty_like(Wqkv), torch.empty_like(Wo)
-        wsf = L.workspace(L.TP_OP_ATTN_FWD, M, hs, 0, hd, 1, L.TP_BF16)
-        wsb = L.workspace(L.TP_OP_ATTN_BWD, M, hs, 0, hd, 1, L.TP_BF16)
+        wsf = L.workspace(L.TP_OP_ATTN_FWD, M, hs, 0, hd, 2, L.TP_BF16)
+        wsb = L.workspace(L.TP_OP_ATTN_BWD, M, hs, 0, hd, 2, L.TP_BF16)
 
         def small():
-            L.tp_attn_fwd(X, Wqkv, Wo, Z, QKV, O, LSE, 1, M, hd, 1, True, wsf)
-            L.tp_attn_bwd(X, Wqkv, Wo, QKV, O, LSE, dZ, dX, dWqkv, dWo, 1, M, hd, 1, True, wsb)
+            L.tp_attn_fwd(X, Wqkv, Wo, Z, QKV, O, LSE, 1, M, hd, 2, True, wsf)
+            L.tp_attn_bwd(X, Wqkv, Wo, QKV, O, LSE, dZ, dX, dWqkv, dWo, 1, M, hd, 2, True, wsb)
         return small
     if name == "linear_f32":
         X, W = _t((4096, 4096), 1.0, torch.float32), _t((4096, 4096), 0.02, torch.float32, seed=1)

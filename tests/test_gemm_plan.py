@@ -12,7 +12,7 @@ element exactly once over the whole K range:
   order: one whole unit, or K slices with distinct partial-tile indices
   that fit the scratch (split only in the last, short wave, or every tile
   when there are fewer tiles than persistent CTAs), each slice at least 32
-  K blocks deep;
+  K blocks deep (16 for a GEMM of fewer than four waves);
 * every unit is a tile of the grid and the unit count matches the plan.
 """
 import random
@@ -68,8 +68,10 @@ def _check_plan(M, N, K, n_shard, kind, sms, scratch):
             assert sorted(split_tiles) == list(range(n_tiles - len(split_tiles), n_tiles))
             assert 2 * len(split_tiles) <= slots
             assert len(split_tiles) == n_tiles % slots
-        # every slice is at least 32 K blocks deep
-        assert all(v["kb1"] - v["kb0"] >= 32 for t in split_tiles for v in by_tile[t][:-1])
+        # every slice is at least 32 K blocks deep (16 when the GEMM has
+        # fewer than four waves of tiles)
+        depth = 16 if n_tiles < 4 * slots else 32
+        assert all(v["kb1"] - v["kb0"] >= depth for t in split_tiles for v in by_tile[t][:-1])
     # spatial coverage: per row band, the column ranges partition [0, N)
     bands = {}
     for tile, us in by_tile.items():
@@ -135,6 +137,15 @@ def test_tile_starved_gemm_is_split():
     assert {u["kb1"] - u["kb0"] for u in units} == {64}
     units = L.tp_gemm_plan(3072, 768, 8192, 0, 256, 148, False)
     assert len(units) == 72
+
+
+def test_short_gemm_splits_its_last_wave_finer():
+    """The GPT-2-small MLP's second GEMM (M = 8192, N = 768, K = 3072):
+    192 tiles on 148 SMs, 1.3 waves; the 44 tiles of the last wave are cut
+    into three slices of 16 K blocks."""
+    units = L.tp_gemm_plan(8192, 768, 3072, 0, 256, 148, True)
+    assert len(units) == 148 + 44 * 3
+    assert {u["kb1"] - u["kb0"] for u in units if u["part"] >= 0} == {16}
 
 
 def test_invalid_plan_requests():
