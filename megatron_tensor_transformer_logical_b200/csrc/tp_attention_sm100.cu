@@ -99,31 +99,45 @@ __device__ __forceinline__ float row_max_visible(uint32_t srow, int vis) {
 __device__ __forceinline__ float exp_row(uint32_t srow, int vis, float scale_log2, float m,
                                          uint32_t (&pk)[kBN / 2], float* mraw) {
   float rs = 0.0f, mx = -INFINITY;
+  // The next chunk's tensor-memory load is in flight while this one is
+  // computed (one wait per chunk, after the computation).
+  uint32_t nx[32];
+  tmem_ld32_nowait(srow, nx);
+  tmem_wait_ld(nx);
 #pragma unroll
   for (int c = 0; c < kBN; c += 32) {
     float v[32];
-    tmem_ld32(srow + c, v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(nx[i]);
+    if (c + 32 < kBN) tmem_ld32_nowait(srow + c + 32, nx);
+    // the chunk's maximum by a tree (depth 5, not a chain of 32)
+    float w[16];
     if (vis >= c + 32) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        mx = fmaxf(mx, v[i]);
-        v[i] = ex2_approx(fmaf(v[i], scale_log2, -m));
-      }
+      for (int i = 0; i < 16; ++i) w[i] = fmaxf(v[i], v[i + 16]);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = ex2_approx(fmaf(v[i], scale_log2, -m));
     } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const bool in = c + i < vis;
-        mx = fmaxf(mx, in ? v[i] : -INFINITY);
-        v[i] = in ? ex2_approx(fmaf(v[i], scale_log2, -m)) : 0.0f;
-      }
+      for (int i = 0; i < 16; ++i)
+        w[i] = fmaxf(c + i < vis ? v[i] : -INFINITY, c + i + 16 < vis ? v[i + 16] : -INFINITY);
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        v[i] = (c + i < vis) ? ex2_approx(fmaf(v[i], scale_log2, -m)) : 0.0f;
     }
+#pragma unroll
+    for (int k = 8; k >= 1; k >>= 1)
+#pragma unroll
+      for (int i = 0; i < k; ++i) w[i] = fmaxf(w[i], w[i + k]);
+    mx = fmaxf(mx, w[0]);
 #pragma unroll
     for (int i = 0; i < 16; ++i) pk[c / 2 + i] = pack_half2(v[2 * i], v[2 * i + 1]);
 #pragma unroll
-    for (int w = 16; w >= 1; w >>= 1)
+    for (int k = 16; k >= 1; k >>= 1)
 #pragma unroll
-      for (int i = 0; i < w; ++i) v[i] += v[i + w];
+      for (int i = 0; i < k; ++i) v[i] += v[i + k];
     rs += v[0];
+    if (c + 32 < kBN) tmem_wait_ld(nx);
   }
   *mraw = mx;
   return rs;
