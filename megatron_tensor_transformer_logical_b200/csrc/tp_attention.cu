@@ -45,55 +45,38 @@ struct AttnArgs {
 
 // ------------------------------------------------------- backward: D term
 // D[bi, head, r] = sum_e dO[row, head*d + e] * O[row, head*d + e].  Sixteen
-// threads per (row, head) with 16-byte loads of 8 elements of O and dO
-// (256 contiguous bytes of each per group), the 16 partial sums added by four
-// shuffle steps.  The pairs are taken in the order of D (r fastest), so a
-// warp's two results are adjacent; the grid is a few CTAs per SM striding
-// over the pairs, four pairs per group in flight.  O is read once here and
-// never again (evict-first); dO stays in L2 for the dQ and dK/dV kernels.
-// HBM-bound: 4 bytes read per element.
-constexpr int kDsumUnroll = 4;
-
+// threads per (row, head), each with 16-byte loads of 8 elements of O and
+// dO (a warp reads two heads' 512 contiguous bytes of each), the 16 partial
+// sums added by four shuffle steps.  HBM-bound: 4 bytes read per element.
 __global__ void __launch_bounds__(256) attn_bwd_dsum_kernel(const AttnArgs a, float* dsum,
                                                              long long M) {
-  const long long total = M * a.heads;
-  const int lane = threadIdx.x & 31, l16 = lane & 15;
-  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const long long stride = 2 * warps;  // pairs per sweep of the grid
-  // First pair of this warp (even): warp-uniform, so every lane takes the
-  // same trips through the loop and the shuffles see the whole warp.
-  long long base = 2 * (static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5));
-  for (; base < total; base += kDsumUnroll * stride) {
-    uint4 ov[kDsumUnroll], dv[kDsumUnroll];
-    long long q[kDsumUnroll];
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long pair = t >> 4;  // (row, head), head fastest
+  const int l16 = threadIdx.x & 15;
+  const bool in = pair < M * a.heads;
+  float acc = 0.0f;
+  long long row = 0;
+  int head = 0;
+  if (in) {
+    row = pair / a.heads;
+    head = static_cast<int>(pair - row * a.heads);
+    const long long off = row * a.h + head * D + l16 * 8;
+    const uint4 ov = *reinterpret_cast<const uint4*>(a.o + off);
+    const uint4 dv = *reinterpret_cast<const uint4*>(a.dout + off);
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __half2* d2 = reinterpret_cast<const __half2*>(&dv);
 #pragma unroll
-    for (int u = 0; u < kDsumUnroll; ++u) {
-      q[u] = base + u * stride + (lane >> 4);
-      ov[u] = make_uint4(0u, 0u, 0u, 0u);
-      dv[u] = ov[u];
-      if (q[u] < total) {
-        const long long bh = q[u] / a.s, r = q[u] - bh * a.s;
-        const long long bi = bh / a.heads, head = bh - bi * a.heads;
-        const long long off = (bi * a.s + r) * a.h + head * D + l16 * 8;
-        ov[u] = __ldcs(reinterpret_cast<const uint4*>(a.o + off));
-        dv[u] = *reinterpret_cast<const uint4*>(a.dout + off);
-      }
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(o2[i]), y = __half22float2(d2[i]);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
     }
+  }
 #pragma unroll
-    for (int u = 0; u < kDsumUnroll; ++u) {
-      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov[u]);
-      const __half2* d2 = reinterpret_cast<const __half2*>(&dv[u]);
-      float acc = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 x = __bfloat1622float2(o2[i]), y = __half22float2(d2[i]);
-        acc = fmaf(x.x, y.x, acc);
-        acc = fmaf(x.y, y.y, acc);
-      }
-#pragma unroll
-      for (int sh = 8; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
-      if (l16 == 0 && q[u] < total) dsum[q[u]] = acc;
-    }
+  for (int sh = 8; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+  if (in && l16 == 0) {
+    const long long bi = row / a.s, r = row - bi * a.s;
+    dsum[(bi * a.heads + head) * a.s + r] = acc;
   }
 }
 
@@ -140,13 +123,10 @@ tp_status launch_attn_core_bwd(const AttnShape& sh, const void* QKV, const void*
   a.dsum = dsum;
   a.out = static_cast<__nv_bfloat16*>(dQKV);
   const long long M = sh.b * sh.s;
-  const long long warps_needed = (M * sh.heads + 1) / 2;
-  long long blocks = (warps_needed + 7) / 8;
-  const long long most = 8LL * sm_count();  // 8 CTAs of 256 threads fill an SM
-  if (blocks > most) blocks = most;
+  const long long threads = M * sh.heads * 16;
   LaunchScope scope(TP_KIND_ATTN_BWD, 2.5 * core_flops(sh), 2.0 * double(M) * 8 * sh.h, stream,
                     3);
-  attn_bwd_dsum_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(a, dsum, M);
+  attn_bwd_dsum_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(a, dsum, M);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention bwd (D term) launch");
   return launch_attn_core_bwd_tc(sh, QKV, dO, LSE, dsum, dQKV, stream);
