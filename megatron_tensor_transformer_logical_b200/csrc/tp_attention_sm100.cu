@@ -73,6 +73,26 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&t);
 }
 
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// max(m, v[0..31]) by three-input maxima: 16 instructions, depth 4.
+__device__ __forceinline__ float max32(const float (&v)[32], float m) {
+  float w[12];
+#pragma unroll
+  for (int k = 0; k < 10; ++k) w[k] = max3f(v[3 * k], v[3 * k + 1], v[3 * k + 2]);
+  w[10] = v[30];
+  w[11] = v[31];
+  float x[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) x[k] = max3f(w[3 * k], w[3 * k + 1], w[3 * k + 2]);
+  return max3f(max3f(x[0], x[1], x[2]), x[3], m);
+}
+
 // The raw-score maximum over this row's visible keys [0, vis) of one block.
 __device__ __forceinline__ float row_max_visible(uint32_t srow, int vis) {
   float mx = -INFINITY;
@@ -84,21 +104,22 @@ __device__ __forceinline__ float row_max_visible(uint32_t srow, int vis) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = (c + i < vis) ? v[i] : -INFINITY;
     }
-#pragma unroll
-    for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-      for (int i = 0; i < w; ++i) v[i] = fmaxf(v[i], v[i + w]);
-    mx = fmaxf(mx, v[0]);
+    mx = max32(v, mx);
   }
   return mx;
 }
 
 // P = 2^(s * scale_log2 - m) over one block row (masked keys 0), packed to
 // fp16 pairs in registers; returns the row sum of P and, in *mraw, the raw
-// maximum over the visible keys.
+// maximum over the visible keys.  The softmax is bound by instruction issue,
+// so the arithmetic is paired where sm_100 allows it: the scale-and-shift as
+// two-wide fused multiply-adds, the row sum as two-wide adds, the maximum by
+// three-input maxima.
 __device__ __forceinline__ float exp_row(uint32_t srow, int vis, float scale_log2, float m,
                                          uint32_t (&pk)[kBN / 2], float* mraw) {
-  float rs = 0.0f, mx = -INFINITY;
+  const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m, -m);
+  float2 acc = make_float2(0.0f, 0.0f);
+  float mx = -INFINITY;
   // The next chunk's tensor-memory load is in flight while this one is
   // computed (one wait per chunk, after the computation).
   uint32_t nx[32];
@@ -110,37 +131,36 @@ __device__ __forceinline__ float exp_row(uint32_t srow, int vis, float scale_log
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(nx[i]);
     if (c + 32 < kBN) tmem_ld32_nowait(srow + c + 32, nx);
-    // the chunk's maximum by a tree (depth 5, not a chain of 32)
-    float w[16];
+    float2 u[16];
     if (vis >= c + 32) {
+      mx = max32(v, mx);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) w[i] = fmaxf(v[i], v[i + 16]);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = ex2_approx(fmaf(v[i], scale_log2, -m));
+      for (int i = 0; i < 16; ++i) {
+        const float2 t = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), sc2, nm2);
+        u[i] = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+      }
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        w[i] = fmaxf(c + i < vis ? v[i] : -INFINITY, c + i + 16 < vis ? v[i + 16] : -INFINITY);
+      for (int i = 0; i < 16; ++i) {
+        const float2 t = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), sc2, nm2);
+        u[i] = make_float2(c + 2 * i < vis ? ex2_approx(t.x) : 0.0f,
+                           c + 2 * i + 1 < vis ? ex2_approx(t.y) : 0.0f);
+      }
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        v[i] = (c + i < vis) ? ex2_approx(fmaf(v[i], scale_log2, -m)) : 0.0f;
+      for (int i = 0; i < 32; ++i) v[i] = (c + i < vis) ? v[i] : -INFINITY;
+      mx = max32(v, mx);
     }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[c / 2 + i] = pack_half2(u[i].x, u[i].y);
 #pragma unroll
     for (int k = 8; k >= 1; k >>= 1)
 #pragma unroll
-      for (int i = 0; i < k; ++i) w[i] = fmaxf(w[i], w[i + k]);
-    mx = fmaxf(mx, w[0]);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) pk[c / 2 + i] = pack_half2(v[2 * i], v[2 * i + 1]);
-#pragma unroll
-    for (int k = 16; k >= 1; k >>= 1)
-#pragma unroll
-      for (int i = 0; i < k; ++i) v[i] += v[i + k];
-    rs += v[0];
+      for (int i = 0; i < k; ++i) u[i] = __fadd2_rn(u[i], u[i + k]);
+    acc = __fadd2_rn(acc, u[0]);
     if (c + 32 < kBN) tmem_wait_ld(nx);
   }
   *mraw = mx;
-  return rs;
+  return acc.x + acc.y;
 }
 
 __global__ void __launch_bounds__(kThreadsA, 1)
@@ -616,6 +636,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     const int qc = min(qrow, a.s - 1);
     const float lse2 = a.lse[stat + qc] * kLog2eA;
     const float dd = a.dsum[stat + qc];
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+    const float2 nl2 = make_float2(-lse2, -lse2), nd2 = make_float2(-dd, -dd);
     const int limit = a.causal ? min(a.s, qrow + 1) : a.s;
     bool ok = true;
     for (int j = 0; j < nx && ok; ++j) {
@@ -629,21 +651,25 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         float sv[32], pv[32];
         tmem_ld32x2(tS(x) + lane_off + c, sv, tP(x) + lane_off + c, pv);
         uint32_t pk[16];
+        // dS = P (dP - D), P = 2^(S scale_log2 - lse2), two entries per step
+        // (two-wide fused multiply-add, add and multiply: the same roundings
+        // as the one-wide forms).
         if (vis >= 32) {
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float p0 = ex2_approx(fmaf(sv[i], a.scale_log2, -lse2));
-            const float p1 = ex2_approx(fmaf(sv[i + 1], a.scale_log2, -lse2));
-            pk[i >> 1] = pack_half2(p0 * (pv[i] - dd), p1 * (pv[i + 1] - dd));
+            const float2 t = __ffma2_rn(make_float2(sv[i], sv[i + 1]), sc2, nl2);
+            const float2 p = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+            const float2 g = __fmul2_rn(p, __fadd2_rn(make_float2(pv[i], pv[i + 1]), nd2));
+            pk[i >> 1] = pack_half2(g.x, g.y);
           }
         } else {
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            float p0 = ex2_approx(fmaf(sv[i], a.scale_log2, -lse2));
-            float p1 = ex2_approx(fmaf(sv[i + 1], a.scale_log2, -lse2));
-            p0 = (i < vis) ? p0 : 0.0f;
-            p1 = (i + 1 < vis) ? p1 : 0.0f;
-            pk[i >> 1] = pack_half2(p0 * (pv[i] - dd), p1 * (pv[i + 1] - dd));
+            const float2 t = __ffma2_rn(make_float2(sv[i], sv[i + 1]), sc2, nl2);
+            const float2 p = make_float2(i < vis ? ex2_approx(t.x) : 0.0f,
+                                         i + 1 < vis ? ex2_approx(t.y) : 0.0f);
+            const float2 g = __fmul2_rn(p, __fadd2_rn(make_float2(pv[i], pv[i + 1]), nd2));
+            pk[i >> 1] = pack_half2(g.x, g.y);
           }
         }
         // dS columns [c / 2, c / 2 + 16): S columns this thread has read.
@@ -714,7 +740,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   uint64_t* p_full = s_full + 2;                // [2]
   uint64_t* acc_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_done + 1);
-  // stage q: LSE * log2(e) of the block's 64 queries at [0, 64), D at [64, 128)
+  // stage q: -LSE * log2(e) of the block's 64 queries at [0, 64), -D at [64, 128)
   float* s_stat = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -783,8 +809,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int qq = min(q0 + e * 32 + lane, a.s - 1);
-        st_dst[e * 32 + lane] = a.lse[stat + qq] * kLog2eA;
-        st_dst[kB64 + e * 32 + lane] = a.dsum[stat + qq];
+        st_dst[e * 32 + lane] = -(a.lse[stat + qq] * kLog2eA);
+        st_dst[kB64 + e * 32 + lane] = -a.dsum[stat + qq];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&qd_full[qs]);
@@ -850,6 +876,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     const int r = quarter * 32 + lane;
     const int key = k0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
     bool ok = true;
     for (int it = 0; it < n_qb && ok; ++it) {
       const int st = it & 1;
@@ -872,22 +899,23 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       float sv[32], pv[32];
       tmem_ld32x2(tS(st) + lane_off + c, sv, tP(st) + lane_off + c, pv);
       uint32_t pk[16], dk[16];
+      // P^T = 2^(S^T scale_log2 - lse2) and dS^T = P^T (dP^T - D), two
+      // entries per step (two-wide arithmetic, the one-wide roundings); the
+      // staged statistics are negated.  Blocks off the diagonal skip the mask.
+      const bool full = lo <= 0 && hi >= 32;
 #pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(wstat + i);
-        const float4 d4 = *reinterpret_cast<const float4*>(wstat + kB64 + i);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-        float p[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          p[e] = ex2_approx(fmaf(sv[i + e], a.scale_log2, -lv[e]));
-          p[e] = (i + e >= lo && i + e < hi) ? p[e] : 0.0f;
+      for (int i = 0; i < 32; i += 2) {
+        const float2 nl = *reinterpret_cast<const float2*>(wstat + i);
+        const float2 nd = *reinterpret_cast<const float2*>(wstat + kB64 + i);
+        const float2 t = __ffma2_rn(make_float2(sv[i], sv[i + 1]), sc2, nl);
+        float2 p = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+        if (!full) {
+          p.x = (i >= lo && i < hi) ? p.x : 0.0f;
+          p.y = (i + 1 >= lo && i + 1 < hi) ? p.y : 0.0f;
         }
-        pk[i >> 1] = pack_half2(p[0], p[1]);
-        pk[(i >> 1) + 1] = pack_half2(p[2], p[3]);
-        dk[i >> 1] = pack_half2(p[0] * (pv[i] - dv[0]), p[1] * (pv[i + 1] - dv[1]));
-        dk[(i >> 1) + 1] = pack_half2(p[2] * (pv[i + 2] - dv[2]), p[3] * (pv[i + 3] - dv[3]));
+        pk[i >> 1] = pack_half2(p.x, p.y);
+        const float2 g = __fmul2_rn(p, __fadd2_rn(make_float2(pv[i], pv[i + 1]), nd));
+        dk[i >> 1] = pack_half2(g.x, g.y);
       }
       tmem_st16(tS(st) + lane_off + c, pk);  // P^T over this group's S^T columns
       tmem_st16(tP(st) + lane_off + c, dk);  // dS^T over its dP^T columns
