@@ -22,6 +22,9 @@
 // when the new maximum exceeds it by more than 2^8 (then O is rescaled in
 // tensor memory); P stays below 2^8, and the final O / l uses the same
 // maximum, so the result does not depend on when the maximum was raised.
+// The maximum of a block after the first is formed only when its row sum of
+// P exceeds 255 (which any key more than 2^8 above the maximum in use
+// forces), so the common block costs the exponentials and the sum alone.
 // Scores are kept in the log2 domain (scaled by log2(e)/sqrt(d)); the saved
 // LSE is the natural log of the softmax denominator.  Every wait is bounded.
 #include <cuda.h>
@@ -50,6 +53,10 @@ constexpr int kSmemA = 1024 + 6 * kTile + 256;
 // has risen by more than 2^8 (log2 units); the final 1/l uses the same
 // maximum, so the result is exact either way, and P stays below 2^8.
 constexpr float kRescaleLog2 = 8.0f;
+// A block's row sum of P above this may hide a key more than 2^8 above the
+// maximum in use (that key's P alone is 2^8 up to the rounding of its
+// exponent), so the exact block maximum is formed and compared.
+constexpr float kCheckSum = 255.0f;
 constexpr float kLog2eA = 1.4426950408889634f;
 constexpr float kLn2A = 0.69314718055994531f;
 
@@ -110,16 +117,16 @@ __device__ __forceinline__ float row_max_visible(uint32_t srow, int vis) {
 }
 
 // P = 2^(s * scale_log2 - m) over one block row (masked keys 0), packed to
-// fp16 pairs in registers; returns the row sum of P and, in *mraw, the raw
-// maximum over the visible keys.  The softmax is bound by instruction issue,
-// so the arithmetic is paired where sm_100 allows it: the scale-and-shift as
-// two-wide fused multiply-adds, the row sum as two-wide adds, the maximum by
-// three-input maxima.
+// fp16 pairs in registers; returns the row sum of P.  The softmax is bound by
+// instruction issue, so the arithmetic is paired where sm_100 allows it: the
+// scale-and-shift as two-wide fused multiply-adds, the row sum as two-wide
+// adds.  The block's maximum is not formed here: a sum above kCheckSum is
+// what sends the caller to the exact maximum (a key 2^8 above m alone makes
+// the sum exceed it).
 __device__ __forceinline__ float exp_row(uint32_t srow, int vis, float scale_log2, float m,
-                                         uint32_t (&pk)[kBN / 2], float* mraw) {
+                                         uint32_t (&pk)[kBN / 2]) {
   const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m, -m);
   float2 acc = make_float2(0.0f, 0.0f);
-  float mx = -INFINITY;
   // The next chunk's tensor-memory load is in flight while this one is
   // computed (one wait per chunk, after the computation).
   uint32_t nx[32];
@@ -133,7 +140,6 @@ __device__ __forceinline__ float exp_row(uint32_t srow, int vis, float scale_log
     if (c + 32 < kBN) tmem_ld32_nowait(srow + c + 32, nx);
     float2 u[16];
     if (vis >= c + 32) {
-      mx = max32(v, mx);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float2 t = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), sc2, nm2);
@@ -146,9 +152,6 @@ __device__ __forceinline__ float exp_row(uint32_t srow, int vis, float scale_log
         u[i] = make_float2(c + 2 * i < vis ? ex2_approx(t.x) : 0.0f,
                            c + 2 * i + 1 < vis ? ex2_approx(t.y) : 0.0f);
       }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = (c + i < vis) ? v[i] : -INFINITY;
-      mx = max32(v, mx);
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) pk[c / 2 + i] = pack_half2(u[i].x, u[i].y);
@@ -159,7 +162,6 @@ __device__ __forceinline__ float exp_row(uint32_t srow, int vis, float scale_log
     acc = __fadd2_rn(acc, u[0]);
     if (c + 32 < kBN) tmem_wait_ld(nx);
   }
-  *mraw = mx;
   return acc.x + acc.y;
 }
 
@@ -336,18 +338,19 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       const int vis = limit - j * kBN;  // visible keys of this block: [0, vis), vis >= 1
       if (j == 0) m_used = row_max_visible(srow, vis) * a.scale_log2;
       uint32_t pk[kBN / 2];
-      float mraw;
-      float rs = exp_row(srow, vis, a.scale_log2, m_used, pk, &mraw);
-      if (j > 0) {
-        const float m_new = mraw * a.scale_log2;
+      float rs = exp_row(srow, vis, a.scale_log2, m_used, pk);
+      // Block 0 set the maximum in use, so its P <= 1.  Later blocks: a row
+      // sum above kCheckSum (rare) sends the warp to the exact maximum.
+      if (j > 0 && __any_sync(0xffffffffu, rs > kCheckSum)) {
+        const float m_new = row_max_visible(srow, vis) * a.scale_log2;
         const bool need = m_new > m_used + kRescaleLog2;
         if (__any_sync(0xffffffffu, need)) {
-          // Rare: the maximum rose by more than 2^8.  Recompute P at the new
+          // The maximum rose by more than 2^8.  Recompute P at the new
           // maximum (S is still intact: P has not been stored yet) and
           // rescale O (P_{j-1} V_{j-1} completed before S_j) and l.
           const float alpha = need ? ex2_approx(m_used - m_new) : 1.0f;
           if (need) m_used = m_new;
-          rs = exp_row(srow, vis, a.scale_log2, m_used, pk, &mraw);
+          rs = exp_row(srow, vis, a.scale_log2, m_used, pk);
 #pragma unroll 1
           for (int c = 0; c < kD; c += 32) {
             float o[32];

@@ -65,6 +65,49 @@ def test_attention_small_ragged(monkeypatch, causal, save_qkv, tile):
     compare_full(gpu_attn(inp, wl, causal, save_qkv), inp, wl, causal)
 
 
+@pytest.mark.parametrize("causal", [True, False], ids=["causal", "full"])
+def test_attention_row_maximum_rising_across_blocks(causal):
+    """Scores that rise by about 30 (log2 units) from one 128-key block to
+    the next, so the forward raises its row maximum and rescales O and the
+    row sum in tensor memory at every block ("图解Transformer并行计算" §3.2
+    step 2: the softmax must not depend on when the maximum is raised).
+    Column 0 of X is a ramp and feeds q[0] and k[0] of every head alone,
+    through exact power-of-two weights, so the large score component is exact
+    in fp16.
+
+    The forward is compared in both masks.  The backward is compared under
+    the causal mask only: with every row as sharp as this and all keys
+    visible, D = rowsum(dO * O) taken from the bf16-rounded O moves the score
+    gradient P (dP - D) enough that dX sits at the bf16 bar (5.9e-3
+    normwise measured; a rounding-point emulation in fp64 gives the same,
+    and 2.3e-3 with O unrounded)."""
+    wl = Workload(86, "attn rising max", b=1, s=520, h=256, heads=2, t=2, w_std=0.05)
+    inp = make_attn_inputs(wl)
+    X, W = inp["X"].clone(), inp["Wqkv"].clone()
+    ramp = torch.round(torch.arange(wl.s, dtype=torch.float64) * (64.0 / wl.s)) / 16.0
+    X[:, 0] = ramp.to(X.dtype)  # 0 .. 4 in steps of 1/16: exact in bf16
+    for head in range(wl.heads):
+        for col in (head * 128, wl.h + head * 128):  # q[0] and k[0] of the head
+            W[:, col] = 0.0
+            W[0, col] = 8.0
+    inp["X"], inp["Wqkv"] = X, W
+    # The construction does what it says: for the last row, the best score of
+    # each key block exceeds that of the block before by more than 8.
+    x64, w64 = to64(X), to64(W)
+    q, k = x64 @ w64[:, :128], x64 @ w64[:, wl.h:wl.h + 128]
+    t = (q[-1] @ k.T) / np.sqrt(128.0) / np.log(2.0)
+    assert all(t[128 * (i + 1):128 * (i + 2)].max() - t[128 * i:128 * (i + 1)].max() > 8.0
+               for i in range(3))
+    out = gpu_attn(inp, wl, causal)
+    if causal:
+        compare_full(out, inp, wl, causal)
+        return
+    fw = O.attn_fwd(inp["X"], inp["Wqkv"], inp["Wo"], wl.b, wl.s, wl.heads, causal)
+    for key in ("Z", "O", "QKV"):
+        check(out[key], fw[key], key, "bf16")
+    assert np.max(np.abs(to64(out["LSE"]) - fw["LSE"])) < 2e-2
+
+
 def test_attention_single_token_and_short():
     # s = 1 (a row that sees only itself: O = V) and s = 3.
     for s in (1, 3):
