@@ -483,8 +483,10 @@ size_t attn_fwd_ws_min(int64_t M, int64_t h, int heads) {
 size_t attn_fwd_ws(int64_t M, int64_t h, int heads) { return attn_fwd_ws_min(M, h, heads) + tail_ws(); }
 
 size_t attn_bwd_ws_min(int64_t M, int64_t h, int heads) {
+  // The row terms take the most room with one token per sequence (every row
+  // padded to 4 floats): b = M, s = 1 bounds every split of M.
   AttnShape sh;
-  sh.b = 1; sh.s = M; sh.h = h; sh.heads = heads;
+  sh.b = M; sh.s = 1; sh.h = h; sh.heads = heads;
   return 2 * align_up(M * 3 * h * 2, 256) + align_up(M * h * 2, 256) +
          align_up(attn_core_bwd_scratch_bytes(sh), 256) + 1024;
 }

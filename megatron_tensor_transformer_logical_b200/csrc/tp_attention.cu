@@ -20,6 +20,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 
 #include "tp_internal.h"
@@ -35,7 +36,6 @@ struct AttnArgs {
   const __nv_bfloat16* o;    // [M, h] bf16
   const __half* dout;        // [M, h] fp16
   const float* lse;          // [b, heads, s]
-  const float* dsum;         // [b, heads, s]: rowsum(dO * O)
   __nv_bfloat16* out;        // O (fwd) or dQKV (bwd)
   float* lse_out;
   int s, h, heads, causal;
@@ -48,8 +48,11 @@ struct AttnArgs {
 // threads per (row, head), each with 16-byte loads of 8 elements of O and
 // dO (a warp reads two heads' 512 contiguous bytes of each), the 16 partial
 // sums added by four shuffle steps.  HBM-bound: 4 bytes read per element.
-__global__ void __launch_bounds__(256) attn_bwd_dsum_kernel(const AttnArgs a, float* dsum,
-                                                             long long M) {
+// Writes the backward's row terms in the form the tcgen05 kernels take:
+// nd = -D and nlse = -LSE * log2(e), rows of sp floats per (batch element,
+// head); the same threads also zero the row padding and the 64-float tail.
+__global__ void __launch_bounds__(256) attn_bwd_dsum_kernel(const AttnArgs a, float* nlse,
+                                                             float* nd, long long M, int sp) {
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long pair = t >> 4;  // (row, head), head fastest
   const int l16 = threadIdx.x & 15;
@@ -76,7 +79,20 @@ __global__ void __launch_bounds__(256) attn_bwd_dsum_kernel(const AttnArgs a, fl
   for (int sh = 8; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
   if (in && l16 == 0) {
     const long long bi = row / a.s, r = row - bi * a.s;
-    dsum[(bi * a.heads + head) * a.s + r] = acc;
+    const long long q = bi * a.heads + head;
+    nd[q * sp + r] = -acc;
+    nlse[q * sp + r] = -(a.lse[q * a.s + r] * kLog2e);
+  }
+  const long long rows = M / a.s * a.heads;
+  const int padr = sp - a.s;
+  if (t < rows * padr) {
+    const long long i = t / padr * sp + a.s + t % padr;
+    nd[i] = 0.0f;
+    nlse[i] = 0.0f;
+  } else if (t < rows * padr + 64) {
+    const long long i = rows * sp + (t - rows * padr);
+    nd[i] = 0.0f;
+    nlse[i] = 0.0f;
   }
 }
 
@@ -105,8 +121,11 @@ tp_status launch_attn_core_fwd(const AttnShape& sh, const void* QKV, void* O, fl
   return launch_attn_core_fwd_tc(sh, QKV, O, LSE, stream);
 }
 
+// Two arrays of row terms, each [b * heads] rows of attn_stat_stride(s)
+// floats and a 64-float tail, 256-byte aligned.
 size_t attn_core_bwd_scratch_bytes(const AttnShape& sh) {
-  return static_cast<size_t>(sh.b * sh.s) * static_cast<size_t>(sh.heads) * sizeof(float);
+  const size_t n = static_cast<size_t>(sh.b * sh.heads) * attn_stat_stride(sh.s) + 64;
+  return 2 * ((n * sizeof(float) + 255) / 256 * 256);
 }
 
 tp_status launch_attn_core_bwd(const AttnShape& sh, const void* QKV, const void* O,
@@ -119,17 +138,21 @@ tp_status launch_attn_core_bwd(const AttnShape& sh, const void* QKV, const void*
   a.o = static_cast<const __nv_bfloat16*>(O);
   a.dout = static_cast<const __half*>(dO);
   a.lse = LSE;
-  float* dsum = static_cast<float*>(scratch);
-  a.dsum = dsum;
   a.out = static_cast<__nv_bfloat16*>(dQKV);
+  const int64_t sp = attn_stat_stride(sh.s);
+  const size_t half = attn_core_bwd_scratch_bytes(sh) / 2;
+  float* nlse = static_cast<float*>(scratch);
+  float* nd = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + half);
   const long long M = sh.b * sh.s;
-  const long long threads = M * sh.heads * 16;
+  const long long pad = sh.b * sh.heads * (sp - sh.s) + 64;
+  const long long threads = std::max(M * sh.heads * 16, pad);
   LaunchScope scope(TP_KIND_ATTN_BWD, 2.5 * core_flops(sh), 2.0 * double(M) * 8 * sh.h, stream,
                     3);
-  attn_bwd_dsum_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(a, dsum, M);
+  attn_bwd_dsum_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+      a, nlse, nd, M, static_cast<int>(sp));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention bwd (D term) launch");
-  return launch_attn_core_bwd_tc(sh, QKV, dO, LSE, dsum, dQKV, stream);
+  return launch_attn_core_bwd_tc(sh, QKV, dO, nlse, nd, dQKV, stream);
 }
 
 }  // namespace tp

@@ -436,8 +436,12 @@ constexpr int kEwWarpsB = 8;
 struct BwdArgs {
   int s, h, heads, causal;
   float scale_log2, scale;
-  const float* lse;   // [b, heads, s]
-  const float* dsum;  // [b, heads, s]
+  // Row terms of the backward, [b * heads] rows of sp floats (s rounded up
+  // to 4, zero beyond s, 64 zeros after the last row): -LSE * log2(e) and
+  // -D with D = rowsum(dO * O).
+  const float* nlse;
+  const float* nd;
+  int sp;
   __nv_bfloat16* dqkv;  // [M, 3h]
   WaitCtl status;
 };
@@ -635,12 +639,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     const int qrow = (qb0 + x) * kBM + r;
     const int nx = x ? n1 : n0;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.s;
+    const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.sp;
     const int qc = min(qrow, a.s - 1);
-    const float lse2 = a.lse[stat + qc] * kLog2eA;
-    const float dd = a.dsum[stat + qc];
+    const float nl = a.nlse[stat + qc], ndd = a.nd[stat + qc];
     const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-    const float2 nl2 = make_float2(-lse2, -lse2), nd2 = make_float2(-dd, -dd);
+    const float2 nl2 = make_float2(nl, nl), nd2 = make_float2(ndd, ndd);
     const int limit = a.causal ? min(a.s, qrow + 1) : a.s;
     bool ok = true;
     for (int j = 0; j < nx && ok; ++j) {
@@ -714,9 +717,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// K, V (128 rows, once), then Q_i, dO_i (64 rows) with the block's LSE * log2(e)
-// and D in a ring of kQdStages stages.  The TMA warp stages LSE and D (plain
-// loads by its 32 lanes) and counts as the stage's second arrival.
+// K, V (128 rows, once), then Q_i, dO_i (64 rows) with the block's row
+// terms -LSE * log2(e) and -D in a ring of kQdStages stages, all of a stage
+// copied asynchronously (tensor loads and two 256-byte bulk copies on the
+// stage's barrier), so the TMA warp never waits on a load itself.
 // Shared memory: K 32K | V 32K | QdO[4] (Q 16K + dO 16K) | barriers | stats[4]
 // (128 floats).  P^T and dS^T live in tensor memory: element-wise group g
 // (query columns [32 g, 32 g + 32) of a block) writes its fp16 pairs over
@@ -758,7 +762,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int i = 0; i < kQdStages; ++i) {
-      mbar_init(&qd_full[i], 2);  // the TMA transaction arrival + the staged statistics
+      mbar_init(&qd_full[i], 1);  // the TMA warp's arrival; the copies count as transactions
       mbar_init(&qd_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -782,7 +786,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   const uint32_t tdV = tmem + 256, tdK = tmem + 384;
 
   if (warp == 0) {
-    const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.s;
+    const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.sp;
     bool ok = true;
     if (lane == 0) {
       tma_prefetch_desc(&tmKV128);
@@ -800,23 +804,20 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       if (!(ok = mbar_wait(&qd_empty[qs], qph ^ 1u, a.status, kStatusAttnTimeout))) break;
       const int q0 = (i0 + it) * kB64;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&qd_full[qs], 2 * kTile64);
+        // Q, dO and the block's 64 row terms of each kind (256 bytes from
+        // a 16-byte aligned row offset; past s they are zeros or the next
+        // row's finite values, which the mask never lets through).
+        mbar_arrive_expect_tx(&qd_full[qs], 2 * kTile64 + 2 * kB64 * 4);
         uint8_t* dst = sQdO + qs * (2 * kTile64);
         const int qrow = row0 + q0;
         tma_load_2d(dst, &tmQ64, &qd_full[qs], head * kD, qrow);
         tma_load_2d(dst + kHalf64, &tmQ64, &qd_full[qs], head * kD + 64, qrow);
         tma_load_2d(dst + kTile64, &tmdO64, &qd_full[qs], head * kD, qrow);
         tma_load_2d(dst + kTile64 + kHalf64, &tmdO64, &qd_full[qs], head * kD + 64, qrow);
+        float* st_dst = s_stat + qs * (2 * kB64);
+        bulk_load(st_dst, a.nlse + stat + q0, kB64 * 4, &qd_full[qs]);
+        bulk_load(st_dst + kB64, a.nd + stat + q0, kB64 * 4, &qd_full[qs]);
       }
-      float* st_dst = s_stat + qs * (2 * kB64);
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int qq = min(q0 + e * 32 + lane, a.s - 1);
-        st_dst[e * 32 + lane] = -(a.lse[stat + qq] * kLog2eA);
-        st_dst[kB64 + e * 32 + lane] = -a.dsum[stat + qq];
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qd_full[qs]);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -1035,9 +1036,9 @@ bool make_map_f16(CUtensorMap* m, const void* ptr, int64_t cols, int64_t rows, i
 }
 }  // namespace
 
-// D = rowsum(dO * O) must already be in `dsum`.
+// The row terms -LSE * log2(e) and -D must already be in `nlse` and `nd`.
 tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const void* dO,
-                                  const float* LSE, const float* dsum, void* dQKV,
+                                  const float* nlse, const float* nd, void* dQKV,
                                   cudaStream_t stream) {
   if (sh.h / sh.heads != kD) return fail(TP_ERR_UNSUPPORTED, "attention: head dimension must be 128");
   if ((sh.s + kBM - 1) / kBM > 65535 || sh.b * sh.heads > 0x7fffffffLL)
@@ -1054,8 +1055,9 @@ tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const vo
   a.causal = sh.causal;
   a.scale = 1.0f / std::sqrt(static_cast<float>(kD));
   a.scale_log2 = a.scale * kLog2eA;
-  a.lse = LSE;
-  a.dsum = dsum;
+  a.nlse = nlse;
+  a.nd = nd;
+  a.sp = static_cast<int>(attn_stat_stride(sh.s));
   a.dqkv = static_cast<__nv_bfloat16*>(dQKV);
   a.status = wait_ctl();
   if (a.status.st == nullptr) return fail(TP_ERR_CUDA, "device status unavailable");

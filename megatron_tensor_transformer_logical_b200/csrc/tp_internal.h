@@ -196,12 +196,17 @@ tp_status launch_attn_core_fwd(const AttnShape& sh, const void* QKV, void* O, fl
 // The tcgen05 / TMEM forward that launch_attn_core_fwd runs.
 tp_status launch_attn_core_fwd_tc(const AttnShape& sh, const void* QKV, void* O, float* LSE,
                                   cudaStream_t stream);
-// The tcgen05 dQ and dK/dV kernels; D = rowsum(dO * O) must be in `dsum`.
+// Row stride of the backward's row terms: s rounded up to 4 floats, so each
+// row starts 16-byte aligned for the bulk copies of the dK/dV kernel.
+inline int64_t attn_stat_stride(int64_t s) { return (s + 3) / 4 * 4; }
+// The tcgen05 dQ and dK/dV kernels, given the row terms -LSE * log2(e) in
+// `nlse` and -D = -rowsum(dO * O) in `nd`: [b * heads] rows of
+// attn_stat_stride(s) floats, zero beyond s, and 64 zeros after the last row.
 tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const void* dO,
-                                  const float* LSE, const float* dsum, void* dQKV,
+                                  const float* nlse, const float* nd, void* dQKV,
                                   cudaStream_t stream);
 // dO [M, h]; writes dQKV [M, 3h] (bf16).  `scratch` holds
-// attn_core_bwd_scratch_bytes bytes (fp32 dQ accumulator and row terms).
+// attn_core_bwd_scratch_bytes bytes (the two arrays of row terms).
 size_t attn_core_bwd_scratch_bytes(const AttnShape& sh);
 tp_status launch_attn_core_bwd(const AttnShape& sh, const void* QKV, const void* O,
                                const float* LSE, const void* dO, void* dQKV, void* scratch,
