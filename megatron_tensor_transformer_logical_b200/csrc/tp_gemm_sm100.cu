@@ -201,39 +201,69 @@ constexpr float kLog2e = 1.4426950408889634f;
 // erf z = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),
 // t = 1 / (1 + p z), |error| <= 1.5e-7, and erf(-z) = -erf z.  With
 // z = |x| / sqrt 2 the factor exp(-z^2) is the exp(-x^2 / 2) of phi, so one
-// reciprocal and one exponential give both.
-__device__ __forceinline__ void normal_cdf_pdf(float x, float& cdf, float& pdf) {
-  const float z = fabsf(x) * 0.70710678118654752f;
-  const float t = rcp_approx(fmaf(0.3275911f, z, 1.0f));
-  const float poly =
-      t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f),
-                     -0.284496736f),
-               0.254829592f);
-  const float e = ex2_approx(-0.5f * kLog2e * x * x);  // exp(-x^2 / 2)
-  const float q = 0.5f * poly * e;                      // (1 - erf z) / 2
-  cdf = x >= 0.0f ? 1.0f - q : q;
-  pdf = 0.39894228040143268f * e;
+// reciprocal and one exponential give both.  GeLU(x) = x Phi(x) (the erf
+// form) and GeLU'(x) = Phi(x) + x phi(x).  Two values at a time, on sm_100's
+// two-wide fp32 instructions (each lane rounded as the one-wide form): on
+// short-K GEMMs the epilogue's instruction issue, not the tensor core, sets
+// the pace.
+__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+
+__device__ __forceinline__ void normal_cdf_pdf2(float2 x, float2& cdf, float2& pdf) {
+  const float2 z = __fmul2_rn(make_float2(fabsf(x.x), fabsf(x.y)), f2(0.70710678118654752f));
+  const float2 d = __ffma2_rn(f2(0.3275911f), z, f2(1.0f));
+  const float2 t = make_float2(rcp_approx(d.x), rcp_approx(d.y));
+  float2 p = __ffma2_rn(t, f2(1.061405429f), f2(-1.453152027f));
+  p = __ffma2_rn(t, p, f2(1.421413741f));
+  p = __ffma2_rn(t, p, f2(-0.284496736f));
+  p = __ffma2_rn(t, p, f2(0.254829592f));
+  const float2 poly = __fmul2_rn(t, p);
+  const float2 arg = __fmul2_rn(__fmul2_rn(x, f2(-0.5f * kLog2e)), x);
+  const float2 e = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));  // exp(-x^2 / 2)
+  const float2 q = __fmul2_rn(__fmul2_rn(f2(0.5f), poly), e);         // (1 - erf z) / 2
+  const float2 r = __fadd2_rn(f2(1.0f), make_float2(-q.x, -q.y));
+  cdf = make_float2(x.x >= 0.0f ? r.x : q.x, x.y >= 0.0f ? r.y : q.y);
+  pdf = __fmul2_rn(f2(0.39894228040143268f), e);
 }
 
-// GeLU(x) = x Phi(x) (the erf form).
-__device__ __forceinline__ float gelu_f(float x) {
-  float cdf, pdf;
-  normal_cdf_pdf(x, cdf, pdf);
-  return x * cdf;
+// GeLU on eight values, in pairs.
+__device__ __forceinline__ void gelu8(float* x) {
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const float2 v = make_float2(x[i], x[i + 1]);
+    float2 cdf, pdf;
+    normal_cdf_pdf2(v, cdf, pdf);
+    const float2 g = __fmul2_rn(v, cdf);
+    x[i] = g.x;
+    x[i + 1] = g.y;
+  }
 }
 
-// GeLU(x) and GeLU'(x) = Phi(x) + x phi(x) from one evaluation.
-__device__ __forceinline__ void gelu_both_f(float x, float& g, float& gp) {
-  float cdf, pdf;
-  normal_cdf_pdf(x, cdf, pdf);
-  g = x * cdf;
-  gp = fmaf(x, pdf, cdf);
+// x *= GeLU'(y) on eight values, in pairs; with hh, also hh = GeLU(y).
+__device__ __forceinline__ void dgelu8(float* x, const float* y, float* hh) {
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const float2 v = make_float2(y[i], y[i + 1]);
+    float2 cdf, pdf;
+    normal_cdf_pdf2(v, cdf, pdf);
+    if (hh != nullptr) {
+      const float2 g = __fmul2_rn(v, cdf);
+      hh[i] = g.x;
+      hh[i + 1] = g.y;
+    }
+    const float2 r = __fmul2_rn(make_float2(x[i], x[i + 1]), __ffma2_rn(v, pdf, cdf));
+    x[i] = r.x;
+    x[i + 1] = r.y;
+  }
 }
 
-__device__ __forceinline__ float gelu_prime_f(float x) {
-  float cdf, pdf;
-  normal_cdf_pdf(x, cdf, pdf);
-  return fmaf(x, pdf, cdf);
+// x += b on eight values, in pairs.
+__device__ __forceinline__ void add8(float* x, const float* b) {
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const float2 r = __fadd2_rn(make_float2(x[i], x[i + 1]), make_float2(b[i], b[i + 1]));
+    x[i] = r.x;
+    x[i + 1] = r.y;
+  }
 }
 
 __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
@@ -305,35 +335,26 @@ __device__ __forceinline__ void epilogue_row32(float (&v)[32], int row, int col0
         unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.bias) + col),
                 bb);
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] += bb[i];
+      add8(x, bb);
     }
     if (EPI == kEpiResidual) {
       float rr[8];
       unpack8(*reinterpret_cast<const uint4*>(a.aux + (long long)row * a.ldaux + col), rr);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] += rr[i];
+      add8(x, rr);
     }
     if (EPI == kEpiBiasGelu) {
       if (a.out2 != nullptr)
         *reinterpret_cast<uint4*>(a.out2 + (long long)row * a.ldo2 + col) = pack8(x);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = gelu_f(x[i]);
+      gelu8(x);
     } else if (EPI == kEpiDGelu) {
       float y[8];
       unpack8(*reinterpret_cast<const uint4*>(a.aux + (long long)row * a.ldaux + col), y);
       if (a.out2 != nullptr) {
         float hh[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float gp;
-          gelu_both_f(y[i], hh[i], gp);
-          x[i] *= gp;
-        }
+        dgelu8(x, y, hh);
         *reinterpret_cast<uint4*>(a.out2 + (long long)row * a.ldo2 + col) = pack8(hh);
       } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] *= gelu_prime_f(y[i]);
+        dgelu8(x, y, nullptr);
       }
     }
     if (OUT == kOutF32) {
@@ -413,32 +434,21 @@ __device__ __forceinline__ void epilogue_box32(float (&v)[32], int r, int col0, 
       float bb[8];
       unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.bias) + col),
               bb);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] += bb[i];
+      add8(x, bb);
     }
     float y[8];
     if (kAux) unpack8(*reinterpret_cast<const uint4*>(box0 + sw64_off(r, g)), y);
-    if (EPI == kEpiResidual) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] += y[i];
-    }
+    if (EPI == kEpiResidual) add8(x, y);
     if (EPI == kEpiBiasGelu) {
       if (a.out2 != nullptr) *reinterpret_cast<uint4*>(box1 + sw64_off(r, g)) = pack8(x);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = gelu_f(x[i]);
+      gelu8(x);
     } else if (EPI == kEpiDGelu) {
       if (a.out2 != nullptr) {
         float hh[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float gp;
-          gelu_both_f(y[i], hh[i], gp);
-          x[i] *= gp;
-        }
+        dgelu8(x, y, hh);
         *reinterpret_cast<uint4*>(box1 + sw64_off(r, g)) = pack8(hh);
       } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] *= gelu_prime_f(y[i]);
+        dgelu8(x, y, nullptr);
       }
     }
     *reinterpret_cast<uint4*>(box0 + sw64_off(r, g)) =
