@@ -435,6 +435,7 @@ constexpr int kEwWarpsB = 8;
 
 struct BwdArgs {
   int s, h, heads, causal;
+  int bh, kv_items;  // b * heads; dK/dV work items (key tiles of all heads)
   float scale_log2, scale;
   // Row terms of the backward, [b * heads] rows of sp floats (s rounded up
   // to 4, zero beyond s, 64 zeros after the last row): -LSE * log2(e) and
@@ -729,6 +730,40 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 constexpr int kQdStages = 4;
 constexpr int kSmemKV = 1024 + 2 * kTile + kQdStages * (2 * kTile64) + 256 + kQdStages * 2 * kB64 * 4;
 
+// Work item k of the dK/dV kernel (k = 0 the longest): key tile k / (b *
+// heads) of one (batch element, head); under the causal mask the early key
+// tiles see the most query blocks.
+struct KvItem {
+  int bi, head, k0, i0, n_qb;  // first key, first query block, query blocks
+};
+
+__device__ __forceinline__ KvItem kv_item(int k, const BwdArgs& a) {
+  KvItem it;
+  const int bh = k % a.bh, kb = k / a.bh;
+  it.head = bh % a.heads;
+  it.bi = bh / a.heads;
+  it.k0 = kb * kBN;
+  const int nqb_all = (a.s + kB64 - 1) / kB64;
+  it.i0 = a.causal ? it.k0 / kB64 : 0;
+  it.n_qb = nqb_all - it.i0;  // >= 1: k0 < s
+  return it;
+}
+
+// The r-th item of this CTA, or -1: rounds of gridDim.x items in snake order
+// (even rounds from CTA 0 up, odd rounds down), so long and short key tiles
+// even out over the CTAs.
+__device__ __forceinline__ int kv_item_index(int r, const BwdArgs& a) {
+  const long long g = gridDim.x, c = blockIdx.x;
+  const long long k = r * g + ((r & 1) ? g - 1 - c : c);
+  return k < a.kv_items ? static_cast<int>(k) : -1;
+}
+
+// Persistent: one CTA per SM walks its key tiles.  The Q / dO ring runs on
+// across items; an item's K and V are loaded once the previous item's last
+// S^T / dP^T products are done (kv_empty), and its first dV, dK products
+// wait until the previous item's epilogue has read the accumulators
+// (acc_empty), so the next key tile's loads and first products overlap the
+// current one's epilogue.
 __global__ void __launch_bounds__(kThreadsB, 1)
     attn_bwd_dkdv_tcgen05(const __grid_constant__ CUtensorMap tmKV128,
                           const __grid_constant__ CUtensorMap tmQ64,
@@ -741,26 +776,22 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   uint8_t* sQdO = smem + 2 * kTile;                     // stage q: Q at +0, dO at +kTile64
   uint64_t* bars = reinterpret_cast<uint64_t*>(sQdO + kQdStages * (2 * kTile64));
   uint64_t* kv_full = bars + 0;
-  uint64_t* qd_full = bars + 1;                 // [kQdStages]
+  uint64_t* kv_empty = bars + 1;                // the item's last S^T / dP^T done
+  uint64_t* qd_full = bars + 2;                 // [kQdStages]
   uint64_t* qd_empty = qd_full + kQdStages;     // [kQdStages]
   uint64_t* s_full = qd_empty + kQdStages;      // [2]
   uint64_t* p_full = s_full + 2;                // [2]
-  uint64_t* acc_done = p_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_done + 1);
+  uint64_t* acc_done = p_full + 2;              // the item's last dV, dK products done
+  uint64_t* acc_empty = acc_done + 1;           // the epilogue has read dV, dK
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   // stage q: -LSE * log2(e) of the block's 64 queries at [0, 64), -D at [64, 128)
   float* s_stat = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb = static_cast<int>(blockIdx.y);  // early keys see the most queries: first
-  const int head = blockIdx.x % a.heads, bi = blockIdx.x / a.heads;
-  const int k0 = kb * kBN;
-  const int nqb_all = (a.s + kB64 - 1) / kB64;
-  const int i0 = a.causal ? (k0 / kB64) : 0;
-  const int n_qb = nqb_all - i0;
-  const int row0 = bi * a.s;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
     for (int i = 0; i < kQdStages; ++i) {
       mbar_init(&qd_full[i], 1);  // the TMA warp's arrival; the copies count as transactions
       mbar_init(&qd_empty[i], 1);
@@ -770,6 +801,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       mbar_init(&p_full[i], kEwWarpsB);
     }
     mbar_init(acc_done, 1);
+    mbar_init(acc_empty, kEwWarpsB);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -786,37 +818,45 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   const uint32_t tdV = tmem + 256, tdK = tmem + 384;
 
   if (warp == 0) {
-    const long long stat = (static_cast<long long>(bi) * a.heads + head) * a.sp;
-    bool ok = true;
     if (lane == 0) {
       tma_prefetch_desc(&tmKV128);
       tma_prefetch_desc(&tmQ64);
       tma_prefetch_desc(&tmdO64);
-      mbar_arrive_expect_tx(kv_full, 2 * kTile);
-      tma_load_2d(sK, &tmKV128, kv_full, a.h + head * kD, row0 + k0);
-      tma_load_2d(sK + kHalf, &tmKV128, kv_full, a.h + head * kD + 64, row0 + k0);
-      tma_load_2d(sV, &tmKV128, kv_full, 2 * a.h + head * kD, row0 + k0);
-      tma_load_2d(sV + kHalf, &tmKV128, kv_full, 2 * a.h + head * kD + 64, row0 + k0);
-    }
-    for (int it = 0; it < n_qb && ok; ++it) {
-      const int qs = it % kQdStages;
-      const uint32_t qph = static_cast<uint32_t>(it / kQdStages) & 1u;
-      if (!(ok = mbar_wait(&qd_empty[qs], qph ^ 1u, a.status, kStatusAttnTimeout))) break;
-      const int q0 = (i0 + it) * kB64;
-      if (lane == 0) {
-        // Q, dO and the block's 64 row terms of each kind (256 bytes from
-        // a 16-byte aligned row offset; past s they are zeros or the next
-        // row's finite values, which the mask never lets through).
-        mbar_arrive_expect_tx(&qd_full[qs], 2 * kTile64 + 2 * kB64 * 4);
-        uint8_t* dst = sQdO + qs * (2 * kTile64);
-        const int qrow = row0 + q0;
-        tma_load_2d(dst, &tmQ64, &qd_full[qs], head * kD, qrow);
-        tma_load_2d(dst + kHalf64, &tmQ64, &qd_full[qs], head * kD + 64, qrow);
-        tma_load_2d(dst + kTile64, &tmdO64, &qd_full[qs], head * kD, qrow);
-        tma_load_2d(dst + kTile64 + kHalf64, &tmdO64, &qd_full[qs], head * kD + 64, qrow);
-        float* st_dst = s_stat + qs * (2 * kB64);
-        bulk_load(st_dst, a.nlse + stat + q0, kB64 * 4, &qd_full[qs]);
-        bulk_load(st_dst + kB64, a.nd + stat + q0, kB64 * 4, &qd_full[qs]);
+      bool ok = true;
+      long long g = 0;  // query blocks loaded so far: the ring position
+      for (int r = 0; ok; ++r) {
+        const int k = kv_item_index(r, a);
+        if (k < 0) break;
+        const KvItem it = kv_item(k, a);
+        const int row0 = it.bi * a.s;
+        if (!(ok = mbar_wait(kv_empty, static_cast<uint32_t>(r & 1) ^ 1u, a.status,
+                             kStatusAttnTimeout)))
+          break;
+        mbar_arrive_expect_tx(kv_full, 2 * kTile);
+        tma_load_2d(sK, &tmKV128, kv_full, a.h + it.head * kD, row0 + it.k0);
+        tma_load_2d(sK + kHalf, &tmKV128, kv_full, a.h + it.head * kD + 64, row0 + it.k0);
+        tma_load_2d(sV, &tmKV128, kv_full, 2 * a.h + it.head * kD, row0 + it.k0);
+        tma_load_2d(sV + kHalf, &tmKV128, kv_full, 2 * a.h + it.head * kD + 64, row0 + it.k0);
+        const long long stat = (static_cast<long long>(it.bi) * a.heads + it.head) * a.sp;
+        for (int j = 0; j < it.n_qb && ok; ++j, ++g) {
+          const int qs = static_cast<int>(g % kQdStages);
+          const uint32_t qph = static_cast<uint32_t>(g / kQdStages) & 1u;
+          if (!(ok = mbar_wait(&qd_empty[qs], qph ^ 1u, a.status, kStatusAttnTimeout))) break;
+          const int q0 = (it.i0 + j) * kB64;
+          // Q, dO and the block's 64 row terms of each kind (256 bytes from
+          // a 16-byte aligned row offset; past s they are zeros or the next
+          // row's finite values, which the mask never lets through).
+          mbar_arrive_expect_tx(&qd_full[qs], 2 * kTile64 + 2 * kB64 * 4);
+          uint8_t* dst = sQdO + qs * (2 * kTile64);
+          const int qrow = row0 + q0;
+          tma_load_2d(dst, &tmQ64, &qd_full[qs], it.head * kD, qrow);
+          tma_load_2d(dst + kHalf64, &tmQ64, &qd_full[qs], it.head * kD + 64, qrow);
+          tma_load_2d(dst + kTile64, &tmdO64, &qd_full[qs], it.head * kD, qrow);
+          tma_load_2d(dst + kTile64 + kHalf64, &tmdO64, &qd_full[qs], it.head * kD + 64, qrow);
+          float* st_dst = s_stat + qs * (2 * kB64);
+          bulk_load(st_dst, a.nlse + stat + q0, kB64 * 4, &qd_full[qs]);
+          bulk_load(st_dst + kB64, a.nd + stat + q0, kB64 * 4, &qd_full[qs]);
+        }
       }
     }
   } else if (warp == 1) {
@@ -824,11 +864,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       constexpr uint32_t kIdSP = idesc_f16_f32(128, 64, false, false);  // K Q^T, V dO^T
       constexpr uint32_t kIdAcc = idesc_f16_f32(128, 128, false, true);  // P^T dO, dS^T Q
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      bool ok = mbar_wait(kv_full, 0, a.status, kStatusAttnTimeout);
-      auto issue_sp = [&](int it) -> bool {
-        const int st = it & 1;
-        const int qs = it % kQdStages;
-        if (!mbar_wait(&qd_full[qs], static_cast<uint32_t>(it / kQdStages) & 1u, a.status,
+      // S^T / dP^T of ring position gg into buffer gg & 1, whose P^T / dS^T
+      // the products of position gg - 2 (issued before) have read.
+      auto issue_sp = [&](long long gg) -> bool {
+        const int st = static_cast<int>(gg & 1);
+        const int qs = static_cast<int>(gg % kQdStages);
+        if (!mbar_wait(&qd_full[qs], static_cast<uint32_t>(gg / kQdStages) & 1u, a.status,
                        kStatusAttnTimeout))
           return false;
         tc_fence_after();
@@ -846,91 +887,120 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         umma_commit(&s_full[st]);
         return true;
       };
-      if (ok && n_qb > 0) ok = issue_sp(0);
-      for (int it = 0; it < n_qb && ok; ++it) {
-        // S^T / dP^T of block it + 1 go into the other buffers, whose P^T /
-        // dS^T the products of block it - 1 (issued before) have read.
-        if (it + 1 < n_qb && !(ok = issue_sp(it + 1))) break;
-        const int st = it & 1;
-        if (!(ok = mbar_wait(&p_full[st], (static_cast<uint32_t>(it) >> 1) & 1u, a.status,
+      bool ok = true;
+      long long g = 0;  // query blocks of the items before this one
+      for (int r = 0; ok; ++r) {
+        const int k = kv_item_index(r, a);
+        if (k < 0) break;
+        const KvItem it = kv_item(k, a);
+        if (!(ok = mbar_wait(kv_full, static_cast<uint32_t>(r & 1), a.status,
                              kStatusAttnTimeout)))
           break;
-        tc_fence_after();
-        const int qs = it % kQdStages;
-        const uint32_t q_addr = smem_u32(sQdO + qs * (2 * kTile64));
-        const uint32_t do_addr = q_addr + kTile64;
+        if (!(ok = issue_sp(g))) break;
+        if (it.n_qb == 1) umma_commit(kv_empty);
+        for (int j = 0; j < it.n_qb && ok; ++j) {
+          const long long gj = g + j;
+          if (j + 1 < it.n_qb) {
+            if (!(ok = issue_sp(gj + 1))) break;
+            if (j + 2 == it.n_qb) umma_commit(kv_empty);  // the item's last S^T / dP^T
+          }
+          const int st = static_cast<int>(gj & 1);
+          if (!(ok = mbar_wait(&p_full[st], static_cast<uint32_t>(gj >> 1) & 1u, a.status,
+                               kStatusAttnTimeout)))
+            break;
+          // The item's first dV, dK products overwrite the accumulators: the
+          // previous item's epilogue must have read them.
+          if (j == 0 && r > 0 &&
+              !(ok = mbar_wait(acc_empty, static_cast<uint32_t>((r - 1) & 1), a.status,
+                               kStatusAttnTimeout)))
+            break;
+          tc_fence_after();
+          const int qs = static_cast<int>(gj % kQdStages);
+          const uint32_t q_addr = smem_u32(sQdO + qs * (2 * kTile64));
+          const uint32_t do_addr = q_addr + kTile64;
 #pragma unroll
-        for (int kk = 0; kk < kB64 / 16; ++kk) {
-          // queries [16 kk, 16 kk + 16): group kk / 2's columns, 8 columns each
-          const uint32_t col = static_cast<uint32_t>(32 * (kk >> 1) + 8 * (kk & 1));
-          const uint32_t acc = (it | kk) != 0 ? 1u : 0u;
-          umma_f16_ts(tdV, tS(st) + col, sw128_desc(do_addr + kk * 2048, kHalf64, 1024), kIdAcc,
-                      acc);
-          umma_f16_ts(tdK, tP(st) + col, sw128_desc(q_addr + kk * 2048, kHalf64, 1024), kIdAcc,
-                      acc);
+          for (int kk = 0; kk < kB64 / 16; ++kk) {
+            // queries [16 kk, 16 kk + 16): group kk / 2's columns, 8 columns each
+            const uint32_t col = static_cast<uint32_t>(32 * (kk >> 1) + 8 * (kk & 1));
+            const uint32_t acc = (j | kk) != 0 ? 1u : 0u;
+            umma_f16_ts(tdV, tS(st) + col, sw128_desc(do_addr + kk * 2048, kHalf64, 1024),
+                        kIdAcc, acc);
+            umma_f16_ts(tdK, tP(st) + col, sw128_desc(q_addr + kk * 2048, kHalf64, 1024),
+                        kIdAcc, acc);
+          }
+          umma_commit(&qd_empty[qs]);
         }
-        umma_commit(&qd_empty[qs]);
+        if (ok) umma_commit(acc_done);
+        g += it.n_qb;
       }
-      if (ok) umma_commit(acc_done);
     }
   } else if (warp >= 4) {
     const int quarter = warp & 3;
     const int grp = (warp - 4) >> 2;  // this warp's column half
     const int c = grp * 32;
     const int r = quarter * 32 + lane;
-    const int key = k0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
     bool ok = true;
-    for (int it = 0; it < n_qb && ok; ++it) {
-      const int st = it & 1;
-      const int qs = it % kQdStages;
-      const int q0 = (i0 + it) * kB64;
-      if (!(ok = mbar_wait(&s_full[st], (static_cast<uint32_t>(it) >> 1) & 1u, a.status,
-                           kStatusAttnTimeout)))
-        break;
-      // The block's statistics were staged before its Q / dO stage completed;
-      // the stage cannot be refilled before this block's products are done.
-      if (!(ok = mbar_wait(&qd_full[qs], static_cast<uint32_t>(it / kQdStages) & 1u, a.status,
-                           kStatusAttnTimeout)))
-        break;
-      tc_fence_after();
-      const float* wstat = s_stat + qs * (2 * kB64) + c;
-      // query q = q0 + c + i is visible to this key when key <= q (causal)
-      // and q < s: lo <= i < hi
-      const int lo = (a.causal ? max(key - q0, 0) : 0) - c;
-      const int hi = (key < a.s ? min(a.s - q0, kB64) : 0) - c;
-      float sv[32], pv[32];
-      tmem_ld32x2(tS(st) + lane_off + c, sv, tP(st) + lane_off + c, pv);
-      uint32_t pk[16], dk[16];
-      // P^T = 2^(S^T scale_log2 - lse2) and dS^T = P^T (dP^T - D), two
-      // entries per step (two-wide arithmetic, the one-wide roundings); the
-      // staged statistics are negated.  Blocks off the diagonal skip the mask.
-      const bool full = lo <= 0 && hi >= 32;
+    long long gb = 0;  // query blocks of the items before this one
+    for (int ri = 0; ok; ++ri) {
+      const int k = kv_item_index(ri, a);
+      if (k < 0) break;
+      const KvItem it = kv_item(k, a);
+      const int key = it.k0 + r;
+      for (int j = 0; j < it.n_qb; ++j) {
+        const long long gj = gb + j;
+        const int st = static_cast<int>(gj & 1);
+        const int qs = static_cast<int>(gj % kQdStages);
+        const int q0 = (it.i0 + j) * kB64;
+        if (!(ok = mbar_wait(&s_full[st], static_cast<uint32_t>(gj >> 1) & 1u, a.status,
+                             kStatusAttnTimeout)))
+          break;
+        // The block's statistics were staged with its Q / dO stage; the stage
+        // cannot be refilled before this block's products are done.
+        if (!(ok = mbar_wait(&qd_full[qs], static_cast<uint32_t>(gj / kQdStages) & 1u, a.status,
+                             kStatusAttnTimeout)))
+          break;
+        tc_fence_after();
+        const float* wstat = s_stat + qs * (2 * kB64) + c;
+        // query q = q0 + c + i is visible to this key when key <= q (causal)
+        // and q < s: lo <= i < hi
+        const int lo = (a.causal ? max(key - q0, 0) : 0) - c;
+        const int hi = (key < a.s ? min(a.s - q0, kB64) : 0) - c;
+        float sv[32], pv[32];
+        tmem_ld32x2(tS(st) + lane_off + c, sv, tP(st) + lane_off + c, pv);
+        uint32_t pk[16], dk[16];
+        // P^T = 2^(S^T scale_log2 - lse2) and dS^T = P^T (dP^T - D), two
+        // entries per step (two-wide arithmetic, the one-wide roundings); the
+        // staged statistics are negated.  Blocks off the diagonal skip the mask.
+        const bool full = lo <= 0 && hi >= 32;
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float2 nl = *reinterpret_cast<const float2*>(wstat + i);
-        const float2 nd = *reinterpret_cast<const float2*>(wstat + kB64 + i);
-        const float2 t = __ffma2_rn(make_float2(sv[i], sv[i + 1]), sc2, nl);
-        float2 p = make_float2(ex2_approx(t.x), ex2_approx(t.y));
-        if (!full) {
-          p.x = (i >= lo && i < hi) ? p.x : 0.0f;
-          p.y = (i + 1 >= lo && i + 1 < hi) ? p.y : 0.0f;
+        for (int i = 0; i < 32; i += 2) {
+          const float2 nl = *reinterpret_cast<const float2*>(wstat + i);
+          const float2 nd = *reinterpret_cast<const float2*>(wstat + kB64 + i);
+          const float2 t = __ffma2_rn(make_float2(sv[i], sv[i + 1]), sc2, nl);
+          float2 p = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+          if (!full) {
+            p.x = (i >= lo && i < hi) ? p.x : 0.0f;
+            p.y = (i + 1 >= lo && i + 1 < hi) ? p.y : 0.0f;
+          }
+          pk[i >> 1] = pack_half2(p.x, p.y);
+          const float2 g = __fmul2_rn(p, __fadd2_rn(make_float2(pv[i], pv[i + 1]), nd));
+          dk[i >> 1] = pack_half2(g.x, g.y);
         }
-        pk[i >> 1] = pack_half2(p.x, p.y);
-        const float2 g = __fmul2_rn(p, __fadd2_rn(make_float2(pv[i], pv[i + 1]), nd));
-        dk[i >> 1] = pack_half2(g.x, g.y);
+        tmem_st16(tS(st) + lane_off + c, pk);  // P^T over this group's S^T columns
+        tmem_st16(tP(st) + lane_off + c, dk);  // dS^T over its dP^T columns
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[st]);
       }
-      tmem_st16(tS(st) + lane_off + c, pk);  // P^T over this group's S^T columns
-      tmem_st16(tP(st) + lane_off + c, dk);  // dS^T over its dP^T columns
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[st]);
-    }
-    if (ok && n_qb > 0 && mbar_wait(acc_done, 0, a.status, kStatusAttnTimeout)) {
+      if (!ok) break;
+      gb += it.n_qb;
+      if (!(ok = mbar_wait(acc_done, static_cast<uint32_t>(ri & 1), a.status, kStatusAttnTimeout)))
+        break;
       tc_fence_after();
-      __nv_bfloat16* out = a.dqkv + static_cast<long long>(row0 + key) * (3LL * a.h);
+      __nv_bfloat16* out = a.dqkv + (static_cast<long long>(it.bi) * a.s + key) * (3LL * a.h);
 #pragma unroll
       for (int cc = grp * (kD / 2); cc < (grp + 1) * (kD / 2); cc += 32) {
         float vk[32], vv[32];
@@ -950,13 +1020,18 @@ __global__ void __launch_bounds__(kThreadsB, 1)
               wk[e] = *reinterpret_cast<uint32_t*>(&tk);
               wv[e] = *reinterpret_cast<uint32_t*>(&tv);
             }
-            *reinterpret_cast<uint4*>(out + a.h + head * kD + cc + 8 * q) = uk;
-            *reinterpret_cast<uint4*>(out + 2 * a.h + head * kD + cc + 8 * q) = uv;
+            *reinterpret_cast<uint4*>(out + a.h + it.head * kD + cc + 8 * q) = uk;
+            *reinterpret_cast<uint4*>(out + 2 * a.h + it.head * kD + cc + 8 * q) = uv;
           }
         }
       }
+
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
+
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -1070,7 +1145,11 @@ tp_status launch_attn_core_bwd_tc(const AttnShape& sh, const void* QKV, const vo
   // (batch element, head) fastest: the CTAs launch in order of decreasing work
   const int64_t nqb = (sh.s + kBM - 1) / kBM;
   dim3 gq(static_cast<unsigned>(sh.b * sh.heads), static_cast<unsigned>((nqb + 1) / 2));
-  dim3 gk(static_cast<unsigned>(sh.b * sh.heads), static_cast<unsigned>((sh.s + kBN - 1) / kBN));
+  const int64_t kv_items = sh.b * sh.heads * ((sh.s + kBN - 1) / kBN);
+  if (kv_items > 0x7fffffffLL) return fail(TP_ERR_SHAPE, "attention: too many key tiles");
+  a.bh = static_cast<int>(sh.b * sh.heads);
+  a.kv_items = static_cast<int>(kv_items);
+  const unsigned gk = static_cast<unsigned>(std::min<int64_t>(kv_items, sm_count()));
   attn_bwd_dq_tcgen05<<<gq, kThreadsB, kSmemDQ, stream>>>(qkv128, qkv64, do128, a);
   attn_bwd_dkdv_tcgen05<<<gk, kThreadsB, kSmemKV, stream>>>(qkv128, qkv64, do64, a);
   e = cudaGetLastError();
