@@ -1252,7 +1252,10 @@ int tile_override() {
 // 6-12% faster; with both K-major (dgrads) the single-SM tile is 3-6% faster
 // in natural K order and the pair 7% faster in the attention's head-group K
 // order.  The 192- and 128-wide tiles run 15% and 30% slower per tile and
-// only pay where they fill the last wave far better.
+// only pay where they fill the last wave far better.  With at most 16 K
+// blocks the per-tile epilogue, not the main loop, sets the pace and the
+// narrower tiles lose only 4% and 10% (workload 2's K = 768 GEMMs: 60 us on
+// 192-wide tiles against 66 us on 256-wide ones).
 int choose_tile(const Gemm& g) {
   const int ov = tile_override();
   if (ov != 0) return ov;
@@ -1260,7 +1263,8 @@ int choose_tile(const Gemm& g) {
   double best = 1e300;
   int kind = 256;
   const int widths[3] = {256, 192, 128};
-  const double rate[3] = {1.0, 0.85, 0.68};
+  const bool short_k = (g.K + BK - 1) / BK <= 16;
+  const double rate[3] = {1.0, short_k ? 0.96 : 0.85, short_k ? 0.90 : 0.68};
   for (int i = 0; i < 3; ++i) {
     const Plan p = plan_for(g, widths[i]);
     const double t = std::ceil(double(p.m_tiles) * p.n_tiles / sms) * 128.0 * widths[i] / rate[i];
