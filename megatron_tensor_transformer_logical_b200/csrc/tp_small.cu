@@ -88,26 +88,29 @@ __global__ void __launch_bounds__(kColsumThreads)
 }
 
 // Second pass: out[c] = the sum of the chunk partials of column c.  A CTA of
-// 256 threads takes 32 columns: warp w adds chunks w, w + 8, w + 16, ... of
-// its lane's column (128-byte rows), then the 8 warp sums are added in warp
-// order (deterministic).
+// 1024 threads takes 32 columns: warp w adds chunks w, w + 32, w + 64, ...
+// of its lane's column (128-byte rows, eight loads in flight), then the 32
+// warp sums are added in warp order (deterministic).  Few columns (768 for
+// a GPT-2-small bias) still give every thread only a handful of loads.
+constexpr int kFinalWarps = 32;
+
 template <bool F32>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kFinalWarps * 32)
     colsum_final(const float* part, int64_t chunks, int64_t cols, void* out) {
-  __shared__ float red[8][32];
+  __shared__ float red[kFinalWarps][32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t c = static_cast<int64_t>(blockIdx.x) * 32 + lane;
   float s = 0.0f;
   if (c < cols) {
-#pragma unroll 4
-    for (int64_t k = w; k < chunks; k += 8) s += part[k * cols + c];
+#pragma unroll 8
+    for (int64_t k = w; k < chunks; k += kFinalWarps) s += part[k * cols + c];
   }
   red[w][lane] = s;
   __syncthreads();
   if (w == 0 && c < cols) {
     float t = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) t += red[i][lane];
+    for (int i = 0; i < kFinalWarps; ++i) t += red[i][lane];
     if (F32)
       static_cast<float*>(out)[c] = t;
     else
@@ -135,11 +138,11 @@ tp_status launch_colsum(const void* in, int64_t rows, int64_t cols, bool f32, vo
                  stream, 2);
   if (f32) {
     colsum_partial<true><<<g1, kColsumThreads, 0, stream>>>(in, rows, cols, p.rows_per_chunk, part);
-    colsum_final<true><<<g2, 256, 0, stream>>>(part, p.chunks, cols, out);
+    colsum_final<true><<<g2, kFinalWarps * 32, 0, stream>>>(part, p.chunks, cols, out);
   } else {
     colsum_partial<false><<<g1, kColsumThreads, 0, stream>>>(in, rows, cols, p.rows_per_chunk,
                                                              part);
-    colsum_final<false><<<g2, 256, 0, stream>>>(part, p.chunks, cols, out);
+    colsum_final<false><<<g2, kFinalWarps * 32, 0, stream>>>(part, p.chunks, cols, out);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "colsum launch");
@@ -152,9 +155,9 @@ tp_status launch_colsum_finish(const float* part, int64_t chunks, int64_t cols, 
   dim3 g(static_cast<unsigned>((cols + 31) / 32));
   LaunchScope s1(TP_KIND_REDUCE, double(chunks) * cols, 4.0 * chunks * cols, stream);
   if (f32)
-    colsum_final<true><<<g, 256, 0, stream>>>(part, chunks, cols, out);
+    colsum_final<true><<<g, kFinalWarps * 32, 0, stream>>>(part, chunks, cols, out);
   else
-    colsum_final<false><<<g, 256, 0, stream>>>(part, chunks, cols, out);
+    colsum_final<false><<<g, kFinalWarps * 32, 0, stream>>>(part, chunks, cols, out);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "colsum finish launch");
   return TP_OK;
