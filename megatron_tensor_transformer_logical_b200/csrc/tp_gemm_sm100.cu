@@ -132,10 +132,17 @@ __host__ __device__ __forceinline__ Unit unit_of(int u, const Args& a) {
 
 // 32 fp32 accumulator values of one row into a partial tile (row-major,
 // `ld` floats per row).
-__device__ __forceinline__ void store_partial32(const float (&v)[32], float* dst) {
-  float4* d = reinterpret_cast<float4*>(dst);
+// A split tile's fp32 partial of TM x TN is laid out as [TN / 4][TM][4]
+// (four columns of one row together, rows next to each other), so a warp,
+// whose lanes hold 32 consecutive rows, stores and loads 512 contiguous
+// bytes per instruction.  Columns [cl, cl + 32) of row lrow:
+template <int TM>
+__device__ __forceinline__ void store_partial32(const float (&v)[32], float* slice, int lrow,
+                                                int cl) {
+  float4* d = reinterpret_cast<float4*>(slice) + (cl >> 2) * TM + lrow;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  for (int i = 0; i < 8; ++i)
+    d[i * TM] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
 
 // Counts one arrival of a split tile's slice on its counter and returns
@@ -569,12 +576,13 @@ __device__ __forceinline__ void tail_finish(const Args& a, const TileCoord& tc, 
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+#pragma unroll 2
     for (int ks = 0; ks < a.tail_split; ++ks) {
-      const float4* src = reinterpret_cast<const float4*>(
-          base + (static_cast<long long>(ks) * TM + lrow) * TN + cl);
+      const float4* src = reinterpret_cast<const float4*>(base + static_cast<long long>(ks) * TM * TN) +
+                          (cl >> 2) * TM + lrow;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float4 q = __ldcg(src + i);
+        const float4 q = __ldcg(src + i * TM);
         v[4 * i] += q.x;
         v[4 * i + 1] += q.y;
         v[4 * i + 2] += q.z;
@@ -776,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[32];
         tmem_ld32(taddr, v);
         if (w.part >= 0)  // a K slice of a tail tile: raw partial sums
-          store_partial32(v, args.tail_part + (static_cast<long long>(w.part) * BM + lrow) * BN + cl);
+          store_partial32<BM>(v, args.tail_part + static_cast<long long>(w.part) * BM * BN, lrow, cl);
         else if constexpr (EPI == kEpiCE)
           epilogue_ce32(v, row, col, tc.n_end, tg, args);
         else {
@@ -1025,8 +1033,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float v[32];
         tmem_ld32(taddr, v);
         if (w.part >= 0)  // a K slice of a tail tile: raw partial sums
-          store_partial32(v, args.tail_part +
-                                 (static_cast<long long>(w.part) * kPairTM + lrow) * kPairTN + cl);
+          store_partial32<kPairTM>(
+              v, args.tail_part + static_cast<long long>(w.part) * kPairTM * kPairTN, lrow, cl);
         else if constexpr (EPI == kEpiCE)
           epilogue_ce32(v, row, col, tc.n_end, tg, args);
         else {
