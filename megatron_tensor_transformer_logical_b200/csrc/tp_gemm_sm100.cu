@@ -1250,9 +1250,23 @@ int tile_override() {
   return (v == 128 || v == 192 || v == 256) ? v : 0;
 }
 
+// Estimated time of T tiles of `tile_work` each on `workers` persistent CTAs
+// (or pairs): whole waves, except that a GEMM with fewer tiles than workers
+// counts the K slices plan_tail cuts every tile into (a short last wave's
+// split is left out of the estimate: measured, it does not repay the
+// narrower tiles it would displace).
+double est_tiles(const Gemm& g, long long T, int workers, size_t part_bytes, double tile_work) {
+  if (T < workers) {
+    const int k_blocks = static_cast<int>((g.K + BK - 1) / BK);
+    const TailPlan tp = plan_tail(T, workers, k_blocks, part_bytes, tail_bytes(g), g.epi);
+    if (tp.split > 1) return tile_work / tp.split;
+  }
+  return std::ceil(double(T) / workers) * tile_work;
+}
+
 // Tile kind: 128, 192 or 256 columns on one SM, or 512 = 256 x 256 on an SM
-// pair.  Picks the least estimated time, ceil(tiles / slots) x work per tile
-// / relative rate.  The rates are throughputs relative to the 256-wide
+// pair.  Picks the least estimated time, est_tiles with the work per tile
+// divided by a relative rate.  The rates are throughputs relative to the 256-wide
 // single-SM tile, measured on the 175B-shaped layer's twelve GEMMs under the
 // sustained power cap with the tile kinds interleaved step by step: with A
 // K-major and B MN-major (the forward linears) the single-SM tile is 3-5%
@@ -1275,7 +1289,9 @@ int choose_tile(const Gemm& g) {
   const double rate[3] = {1.0, short_k ? 0.96 : 0.85, short_k ? 0.90 : 0.68};
   for (int i = 0; i < 3; ++i) {
     const Plan p = plan_for(g, widths[i]);
-    const double t = std::ceil(double(p.m_tiles) * p.n_tiles / sms) * 128.0 * widths[i] / rate[i];
+    const double t = est_tiles(g, static_cast<long long>(p.m_tiles) * p.n_tiles,
+                               static_cast<int>(sms), size_t(BM) * widths[i] * 4,
+                               128.0 * widths[i] / rate[i]);
     if (t < best * 0.999) {
       best = t;
       kind = widths[i];
@@ -1289,8 +1305,9 @@ int choose_tile(const Gemm& g) {
   else
     pair_rate = 1.10;                                 // wgrad
   const Plan pp = plan_for(g, kPairTN);
-  const double pair_tiles = double((g.M + kPairTM - 1) / kPairTM) * pp.n_tiles;
-  const double tp = std::ceil(pair_tiles / std::floor(sms / 2)) * 256.0 * 256.0 / 2.0 / pair_rate;
+  const long long pair_tiles = (g.M + kPairTM - 1) / kPairTM * pp.n_tiles;
+  const double tp = est_tiles(g, pair_tiles, static_cast<int>(sms) / 2,
+                              size_t(kPairTM) * kPairTN * 4, 256.0 * 256.0 / 2.0 / pair_rate);
   if (tp < best * 0.999) kind = 512;
   return kind;
 }
