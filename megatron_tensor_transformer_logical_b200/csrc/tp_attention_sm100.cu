@@ -422,7 +422,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
 //   S = Q K^T, dP = dO V^T (TMEM) -> dS (fp16, written back into tensor
 //   memory over S) -> dQ += dS K (dS the tensor-memory A operand); dQ is
 //   scaled by 1/sqrt(d) at the end.
-// dK/dV kernel (per 128 keys, 64-query blocks):
+// dK/dV kernel (per 128 keys, 64-query blocks; persistent, one CTA per SM
+// taking its key tiles in turn):
 //   S^T = K Q^T, dP^T = V dO^T (TMEM, two buffers) -> P^T, dS^T (fp16, back
 //   into tensor memory over S^T and dP^T) -> dV += P^T dO, dK += dS^T Q
 //   (tensor-memory A operands); dK is scaled by 1/sqrt(d) at the end.
