@@ -52,17 +52,22 @@ struct AttnArgs {
 // nd = -D and nlse = -LSE * log2(e), rows of sp floats per (batch element,
 // head); the same threads also zero the row padding and the 64-float tail.
 __global__ void __launch_bounds__(256) attn_bwd_dsum_kernel(const AttnArgs a, float* nlse,
-                                                             float* nd, long long M, int sp) {
+                                                             float* nd, long long M,
+                                                             long long rows, int sp) {
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long pair = t >> 4;  // (row, head), head fastest
   const int l16 = threadIdx.x & 15;
   const bool in = pair < M * a.heads;
-  float acc = 0.0f;
-  long long row = 0;
-  int head = 0;
+  float acc = 0.0f, lse = 0.0f;
+  long long dst = 0;
   if (in) {
-    row = pair / a.heads;
-    head = static_cast<int>(pair - row * a.heads);
+    const long long row = pair / a.heads;
+    const int head = static_cast<int>(pair - row * a.heads);
+    const long long bi = row / a.s, r = row - bi * a.s;
+    const long long q = bi * a.heads + head;
+    dst = q * sp + r;
+    // The group's LSE load goes out with its O and dO loads.
+    if (l16 == 0) lse = a.lse[q * a.s + r];
     const long long off = row * a.h + head * D + l16 * 8;
     const uint4 ov = *reinterpret_cast<const uint4*>(a.o + off);
     const uint4 dv = *reinterpret_cast<const uint4*>(a.dout + off);
@@ -78,12 +83,9 @@ __global__ void __launch_bounds__(256) attn_bwd_dsum_kernel(const AttnArgs a, fl
 #pragma unroll
   for (int sh = 8; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
   if (in && l16 == 0) {
-    const long long bi = row / a.s, r = row - bi * a.s;
-    const long long q = bi * a.heads + head;
-    nd[q * sp + r] = -acc;
-    nlse[q * sp + r] = -(a.lse[q * a.s + r] * kLog2e);
+    nd[dst] = -acc;
+    nlse[dst] = -(lse * kLog2e);
   }
-  const long long rows = M / a.s * a.heads;
   const int padr = sp - a.s;
   if (t < rows * padr) {
     const long long i = t / padr * sp + a.s + t % padr;
@@ -149,7 +151,7 @@ tp_status launch_attn_core_bwd(const AttnShape& sh, const void* QKV, const void*
   LaunchScope scope(TP_KIND_ATTN_BWD, 2.5 * core_flops(sh), 2.0 * double(M) * 8 * sh.h, stream,
                     3);
   attn_bwd_dsum_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
-      a, nlse, nd, M, static_cast<int>(sp));
+      a, nlse, nd, M, sh.b * sh.heads, static_cast<int>(sp));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention bwd (D term) launch");
   return launch_attn_core_bwd_tc(sh, QKV, dO, nlse, nd, dQKV, stream);
