@@ -113,6 +113,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Counts one arrival on a counter shared by `count` arrivals of one launch
+// and returns whether it was the last.  The counter holds (launch generation
+// << 8) | arrivals (count < 256), so counters need no clearing between
+// launches: a value from an earlier launch counts as zero.  One thread calls
+// it, after its CTA's stores of what the last arrival will read and a
+// __threadfence().
+__device__ __forceinline__ bool gen_ticket(unsigned long long* ctr, unsigned long long gen,
+                                           int count) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(ctr);
+  for (;;) {
+    const unsigned long long want = ((cur >> 8) == gen) ? cur + 1ull : ((gen << 8) | 1ull);
+    const unsigned long long prev = atomicCAS(ctr, cur, want);
+    if (prev == cur) return static_cast<int>(want & 0xffull) == count;
+    cur = prev;  // another arrival came in between: retry on its value
+  }
+}
+
 // Sets flag bits in the status (sticky until the host reads them).
 __device__ __forceinline__ void status_flag(const WaitCtl& w, int bits) {
   atomicOr(&w.st->flags, bits);

@@ -9,6 +9,8 @@
 #include <cstring>
 #include <exception>
 #include <atomic>
+#include <chrono>
+#include <cstdint>
 #include <mutex>
 #include <string>
 #include <utility>
@@ -83,9 +85,19 @@ DeviceStatus* device_status_ptr() {
 }
 
 namespace {
-// Launch generations start at 1, so a cleared status (abort_gen 0) stops no
-// wait.
-std::atomic<unsigned long long> g_launch_gen{0};
+// Launch generations start from a value drawn when the library loads (the
+// clock and an address, below 2^47), so arrival counters left in reused
+// device memory by another process, or by another load of this library,
+// carry no current generation; they are never 0, so a cleared status
+// (abort_gen 0) stops no wait.
+unsigned long long first_launch_gen() {
+  const unsigned long long t = static_cast<unsigned long long>(
+      std::chrono::steady_clock::now().time_since_epoch().count());
+  const unsigned long long a = static_cast<unsigned long long>(
+      reinterpret_cast<uintptr_t>(&first_launch_gen));
+  return ((t * 0x9E3779B97F4A7C15ull) ^ (a >> 4)) & ((1ull << 47) - 1);
+}
+std::atomic<unsigned long long> g_launch_gen{first_launch_gen()};
 }  // namespace
 
 WaitCtl wait_ctl() {
@@ -310,12 +322,18 @@ namespace {
 
 size_t mlp_fwd_ws(int64_t M, int64_t f, tp_dtype d) { return mlp_fwd_ws_min(M, f, d) + tail_ws(); }
 
-// Column-sum scratch of the MLP backward: the two-pass sums of dY and dZ,
-// or the GeLU' GEMM's per-32-row partials of dY (ceil(M / 32) x f floats).
+// The GeLU' GEMM's per-32-row partials of dY: ceil(M / 32) x f floats.
+size_t dba_partial_bytes(int64_t M, int64_t f) {
+  return static_cast<size_t>((M + 31) / 32) * static_cast<size_t>(f) * 4;
+}
+
+// Column-sum scratch of the MLP backward: the two-pass sums of dY and dZ
+// (fp32 path), or the GeLU' GEMM's partials of dY followed by the scratch of
+// the one-launch bias gradients (bf16 path).
 size_t mlp_bwd_colsum_bytes(int64_t M, int64_t h, int64_t f) {
   size_t cs = colsum_scratch_bytes(M, f);
   const size_t cs2 = colsum_scratch_bytes(M, h);
-  const size_t cs3 = static_cast<size_t>((M + 31) / 32) * static_cast<size_t>(f) * 4;
+  const size_t cs3 = align_up(dba_partial_bytes(M, f), 256) + mlp_bias_grads_scratch_bytes(M, h);
   if (cs2 > cs) cs = cs2;
   if (cs3 > cs) cs = cs3;
   return cs;
@@ -464,12 +482,14 @@ tp_status mlp_bwd(const void* X, const void* A, const void* bA, const void* B, c
   tail.to(g6);
   TP_TRY(run(g6, f32, stream));
 
-  if (fused_dba)
-    TP_TRY(launch_colsum_finish(static_cast<const float*>(scratch), (M + 31) / 32, f, false, dbA,
-                                stream));
-  else if (dbA)
-    TP_TRY(launch_colsum(dY, M, f, f32, dbA, scratch, stream));
-  if (dbB) TP_TRY(launch_colsum(dZ, M, h, f32, dbB, scratch, stream));
+  if (!f32)  // one launch: dbA from the partials, dbB = colsum(dZ)
+    TP_TRY(launch_mlp_bias_grads(
+        dZ, M, h, dbB, static_cast<const float*>(scratch), f, dbA,
+        static_cast<char*>(scratch) + align_up(dba_partial_bytes(M, f), 256), stream));
+  else {
+    if (dbA) TP_TRY(launch_colsum(dY, M, f, f32, dbA, scratch, stream));
+    if (dbB) TP_TRY(launch_colsum(dZ, M, h, f32, dbB, scratch, stream));
+  }
   return TP_OK;
 }
 

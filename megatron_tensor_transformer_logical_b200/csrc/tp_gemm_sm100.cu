@@ -72,6 +72,22 @@ struct Cfg {
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
+// Epilogues that read an operand (`aux`: Y for GeLU', the residual) fetch
+// it one 32-column chunk ahead into two more boxes per epilogue warp where
+// shared memory has room for them (BN = 192: four 40 KB stages), so the
+// fetch of the next chunk's rows overlaps the current chunk instead of
+// being waited for at the start of every chunk; elsewhere the aux rows come
+// into the output box at the start of their own chunk.
+template <int BN, int EPI>
+struct AuxAhead {
+  static constexpr bool kOn = BN == 192 && (EPI == kEpiResidual || EPI == kEpiDGelu);
+  static constexpr int kBytes = kOn ? kEpiWarps * 2 * kEpiBoxBytes : 0;
+  static constexpr int kBars = kOn ? 2 * kEpiWarps : kEpiWarps;
+  static constexpr int kSmemBytes = Cfg<BN>::kSmemBytes + kBytes;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  static_assert((4 + 2 * Cfg<BN>::kStages + kBars) * 8 + 8 <= kBarBytes, "barrier area");
+};
+
 struct Args {
   int M, N, K;
   int m_tiles, n_tiles, k_blocks, group_m;
@@ -143,22 +159,6 @@ __device__ __forceinline__ void store_partial32(const float (&v)[32], float* sli
 #pragma unroll
   for (int i = 0; i < 8; ++i)
     d[i * TM] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-}
-
-// Counts one arrival of a split tile's slice on its counter and returns
-// whether it was the last of `split`.  The counter holds (launch generation
-// << 8) | arrivals, so the counters need no clearing between launches: a
-// value from an earlier launch counts as zero.  One thread calls it, after
-// the CTA's partial-tile stores and a __threadfence().
-__device__ __forceinline__ bool tail_ticket(unsigned long long* ctr, unsigned long long gen,
-                                            int split) {
-  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(ctr);
-  for (;;) {
-    const unsigned long long want = ((cur >> 8) == gen) ? cur + 1ull : ((gen << 8) | 1ull);
-    const unsigned long long prev = atomicCAS(ctr, cur, want);
-    if (prev == cur) return static_cast<int>(want & 0xffull) == split;
-    cur = prev;  // another slice arrived in between: retry on its value
-  }
 }
 
 struct TileCoord {
@@ -425,12 +425,13 @@ __device__ __forceinline__ uint32_t sw64_off(int r, int j) {
 
 // The epilogue of one row's 32 consecutive columns, all inside the tile's
 // column range, written to the warp's staging boxes (row r of a box = this
-// thread's lane): box0 holds the row of `aux` on entry for the epilogues
-// that read one and receives `out`; box1 receives out2.  Rows past M are
+// thread's lane): abox holds the row of `aux` for the epilogues that read
+// one (it may be box0), box0 receives `out` and box1 out2.  Rows past M are
 // computed too and dropped by the TMA store.
 template <int EPI, int OUT>
 __device__ __forceinline__ void epilogue_box32(float (&v)[32], int r, int col0, uint8_t* box0,
-                                               uint8_t* box1, const Args& a) {
+                                               uint8_t* box1, const uint8_t* abox,
+                                               const Args& a) {
   constexpr bool kAux = (EPI == kEpiResidual || EPI == kEpiDGelu);
   bool clamped = false;
 #pragma unroll
@@ -444,7 +445,7 @@ __device__ __forceinline__ void epilogue_box32(float (&v)[32], int r, int col0, 
       add8(x, bb);
     }
     float y[8];
-    if (kAux) unpack8(*reinterpret_cast<const uint4*>(box0 + sw64_off(r, g)), y);
+    if (kAux) unpack8(*reinterpret_cast<const uint4*>(abox + sw64_off(r, g)), y);
     if (EPI == kEpiResidual) add8(x, y);
     if (EPI == kEpiBiasGelu) {
       if (a.out2 != nullptr) *reinterpret_cast<uint4*>(box1 + sw64_off(r, g)) = pack8(x);
@@ -547,7 +548,37 @@ __device__ __forceinline__ bool epilogue_chunk_boxed(uint32_t taddr, int lane, i
   if constexpr (EPI == kEpiCE)
     epilogue_ce32(v, row, col, col_end, tg, a, box0, lane);
   else
-    epilogue_box32<EPI, OUT>(v, lane, col, box0, box1, a);
+    epilogue_box32<EPI, OUT>(v, lane, col, box0, box1, box0, a);
+  epilogue_colsum<EPI>(v, row, col, col_end, lane, a);
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmO, box0, col, row0);
+    if (kOut2 && a.out2 != nullptr) tma_store_2d(tmO2, box1, col, row0);
+    bulk_commit();
+  }
+  return true;
+}
+
+// One 32-column chunk of a whole tile for an epilogue that reads `aux`,
+// whose rows were requested earlier into `abox` (counted on `abar`, wait
+// parity `aphase`): as epilogue_chunk_boxed, without fetching them here.
+// Returns false if the wait for the aux box gave up.
+template <int EPI, int OUT>
+__device__ __forceinline__ bool epilogue_chunk_ahead(uint32_t taddr, int lane, int row, int row0,
+                                                     int col, int col_end, uint8_t* box0,
+                                                     uint8_t* box1, const uint8_t* abox,
+                                                     uint64_t* abar, uint32_t aphase,
+                                                     const CUtensorMap* tmO,
+                                                     const CUtensorMap* tmO2, const Args& a) {
+  constexpr bool kOut2 = (EPI == kEpiBiasGelu || EPI == kEpiDGelu);
+  if (lane == 0) bulk_wait_read<0>();
+  __syncwarp();
+  float v[32];
+  tmem_ld32(taddr, v);
+  const bool got = mbar_wait(abar, aphase, a.status, kStatusEpilogueTimeout);
+  if (!__all_sync(0xffffffffu, got)) return false;
+  epilogue_box32<EPI, OUT>(v, lane, col, box0, box1, abox, a);
   epilogue_colsum<EPI>(v, row, col, col_end, lane, a);
   fence_async_smem();
   __syncwarp();
@@ -604,7 +635,7 @@ __device__ __forceinline__ void tail_arrive(const Args& a, const TileCoord& tc, 
   __threadfence();
   named_sync(1, kEpiWarps * 32);
   if (ew == 0 && lane == 0)
-    *flag = tail_ticket(a.tail_ctr + slot, a.status.gen, a.tail_split) ? 1 : 0;
+    *flag = gen_ticket(a.tail_ctr + slot, a.status.gen, a.tail_split) ? 1 : 0;
   named_sync(1, kEpiWarps * 32);
   if (*reinterpret_cast<volatile int*>(flag)) {
     __threadfence();
@@ -620,18 +651,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmO2,
                       const __grid_constant__ CUtensorMap tmX, const Args args) {
   using C = Cfg<BN>;
+  using AX = AuxAhead<BN, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kStages * C::kABytes;
   uint8_t* sE = sB + C::kStages * C::kBBytes;  // epilogue boxes, 1024-byte aligned
-  uint64_t* full = reinterpret_cast<uint64_t*>(sE + kEpiStageBytes);
+  uint8_t* sX = sE + kEpiStageBytes;           // aux boxes fetched ahead (AX::kOn)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sX + AX::kBytes);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
-  uint64_t* auxbar = tempty + 2;  // one per epilogue warp
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + kEpiWarps);
+  uint64_t* auxbar = tempty + 2;  // one (two with AX::kOn) per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + AX::kBars);
   int* tail_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -646,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], kEpiWarps);
     }
-    for (int i = 0; i < kEpiWarps; ++i) mbar_init(&auxbar[i], 1);
+    for (int i = 0; i < AX::kBars; ++i) mbar_init(&auxbar[i], 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -754,6 +787,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* box0 = sE + ew * (2 * kEpiBoxBytes);
     uint8_t* box1 = box0 + kEpiBoxBytes;
     uint32_t aux_phase = 0;
+    // Aux fetched ahead (AX::kOn): the chunk (unit ax_u, column offset ax_c)
+    // whose rows are on their way into aux box ax_slot (ax_u < 0: none);
+    // ax_par holds each box's wait parity.
+    uint8_t* xbox = sX + ew * (2 * kEpiBoxBytes);
+    int ax_u = -1, ax_c = 0, ax_slot = 0;
+    uint32_t ax_par = 0;
+    auto ax_fetch = [&](int slot, int col, int row0) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&auxbar[2 * ew + slot], kEpiBoxBytes);
+        tma_load_2d(xbox + slot * kEpiBoxBytes, &tmX, &auxbar[2 * ew + slot], col, row0);
+      }
+    };
     bool ok = true;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -774,9 +819,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                                static_cast<uint32_t>(acc * BN + cl);
         if constexpr (OUT != kOutF32) {
           if (args.tma_out && w.part < 0 && col + 32 <= tc.n_end) {
-            ok = epilogue_chunk_boxed<EPI, OUT>(taddr, lane, row, tc.m0 + quarter * 32, col,
-                                                tc.n_end, tg, box0, box1, &auxbar[ew], aux_phase,
-                                                &tmO, &tmO2, &tmX, args);
+            if constexpr (AX::kOn) {
+              // This chunk's aux rows: requested by the previous chunk, else now.
+              const int slot = ax_slot;
+              if (ax_u != u || ax_c != c) ax_fetch(slot, col, tc.m0 + quarter * 32);
+              // Request the next chunk's: the next one of this tile, or the
+              // first one of this CTA's next unit.
+              ax_u = -1;
+              if (c + 32 < BN / 2) {
+                if (col + 64 <= tc.n_end) {
+                  ax_fetch(slot ^ 1, col + 32, tc.m0 + quarter * 32);
+                  ax_u = u;
+                  ax_c = c + 32;
+                }
+              } else if (u + static_cast<int>(gridDim.x) < args.units) {
+                const int un = u + static_cast<int>(gridDim.x);
+                const Unit wn = unit_of(un, args);
+                const TileCoord tn = tile_coord<BN>(wn.tile, args);
+                const int coln = tn.n0 + half * (BN / 2);
+                if (wn.part < 0 && coln + 32 <= tn.n_end) {
+                  ax_fetch(slot ^ 1, coln, tn.m0 + quarter * 32);
+                  ax_u = un;
+                  ax_c = 0;
+                }
+              }
+              ax_slot = slot ^ 1;
+              ok = epilogue_chunk_ahead<EPI, OUT>(
+                  taddr, lane, row, tc.m0 + quarter * 32, col, tc.n_end, box0, box1,
+                  xbox + slot * kEpiBoxBytes, &auxbar[2 * ew + slot], (ax_par >> slot) & 1u,
+                  &tmO, &tmO2, args);
+              ax_par ^= 1u << slot;
+            } else {
+              ok = epilogue_chunk_boxed<EPI, OUT>(taddr, lane, row, tc.m0 + quarter * 32, col,
+                                                  tc.n_end, tg, box0, box1, &auxbar[ew],
+                                                  aux_phase, &tmO, &tmO2, &tmX, args);
+            }
             if (!ok) break;
             continue;
           }
@@ -804,6 +881,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    // An aux fetch still in flight (only after a wait gave up): let it land
+    // before the CTA's shared memory goes away.
+    if (AX::kOn && ax_u >= 0)
+      mbar_wait(&auxbar[2 * ew + ax_slot], (ax_par >> ax_slot) & 1u, args.status,
+                kStatusEpilogueTimeout);
     if (lane == 0) bulk_wait<0>();  // this warp's TMA stores have landed
   }
 
@@ -1351,7 +1433,8 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   const unsigned bit = (dev >= 0 && dev < 32) ? (1u << dev) : 0u;
   if (bit == 0 || !(configured.load(std::memory_order_acquire) & bit)) {
     cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AuxAhead<BN, EPI>::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
     configured.fetch_or(bit, std::memory_order_release);
   }
@@ -1369,7 +1452,8 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
                        (EPI == kEpiCE ? 8.0 * double(g.M) * g.N / 32.0 : 0.0);
   {
     LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, 1, BN, g.M, g.N, g.K);
-    kern<<<grid, kThreads, C::kSmemBytes, stream>>>(ta, tb, em.o, em.o2, em.x, a);
+    kern<<<grid, kThreads, AuxAhead<BN, EPI>::kSmemBytes, stream>>>(ta, tb, em.o, em.o2, em.x,
+                                                                       a);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm_bf16_tcgen05 launch");

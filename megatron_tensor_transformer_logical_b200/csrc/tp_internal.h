@@ -149,6 +149,15 @@ tp_status launch_colsum(const void* in, int64_t rows, int64_t cols, bool f32, vo
 // out[c] = sum over k < chunks of part[k * cols + c], in k order (bf16 or f32).
 tp_status launch_colsum_finish(const float* part, int64_t chunks, int64_t cols, bool f32,
                                void* out, cudaStream_t stream);
+// Both bias gradients of the bf16 MLP backward in one launch: dbB =
+// colsum(dZ) for dZ [M, h], and dbA from partA, the GeLU' GEMM's per-32-row
+// partials ([ceil(M / 32), f] fp32).  Either output may be nullptr (then its
+// part is skipped).  `scratch` holds mlp_bias_grads_scratch_bytes(M, h)
+// bytes (chunk partials and arrival counters, cleared here on `stream`).
+size_t mlp_bias_grads_scratch_bytes(int64_t M, int64_t h);
+tp_status launch_mlp_bias_grads(const void* dZ, int64_t M, int64_t h, void* dbB,
+                                const float* partA, int64_t f, void* dbA, void* scratch,
+                                cudaStream_t stream);
 
 // LayerNorm over rows of [M, h] (h % 8 == 0, h <= layernorm_max_h()).
 int64_t layernorm_max_h();

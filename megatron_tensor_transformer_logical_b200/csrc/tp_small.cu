@@ -118,7 +118,167 @@ __global__ void __launch_bounds__(kFinalWarps * 32)
   }
 }
 
+// Both bias gradients of the MLP backward on the bf16 tensor-core path in one
+// launch (the two passes above cost three launches there):
+// * dbB = colsum(dZ): CTA (column block of 64, row chunk) sums its rows into
+//   fp32 partials (8 groups of 8 columns x 32 row phases, the phases added
+//   in order through shared memory); the CTA whose arrival on the column
+//   block's counter is the last adds the block's chunk partials in chunk
+//   order (16 groups of 4 columns x 16 chunk phases, phases in order);
+// * dbA: CTAs past those add the GeLU' GEMM's per-32-row partials of dY in
+//   the same 16 x 16 arrangement.
+// Which CTA arrives last varies; the order of every sum does not, so the
+// result is deterministic.  The counters are cleared on the stream before
+// the launch (one atomicAdd per arrival: a compare-and-swap loop retried
+// under 64-way contention costs tens of microseconds).
+constexpr int kBiasCols = 64;
+constexpr int kBiasThreads = 256;
+
+struct BiasPlan {
+  int64_t chunk_rows, chunks, col_blocks;
+};
+
+BiasPlan bias_plan(int64_t rows, int64_t cols) {
+  BiasPlan p;
+  p.chunk_rows = 128 * ((rows + 8191) / 8192);
+  p.chunks = (rows + p.chunk_rows - 1) / p.chunk_rows;
+  p.col_blocks = (cols + kBiasCols - 1) / kBiasCols;
+  return p;
+}
+
+struct BiasArgs {
+  const __nv_bfloat16* dZ;  // [M, h]
+  int64_t M, h, chunk_rows, chunks, col_blocks;
+  int nb;                   // CTAs of the dbB part (0: no dbB)
+  float* partB;             // [chunks, h]
+  unsigned int* ctr;        // [col_blocks], zero at launch
+  __nv_bfloat16* dbB;
+  const float* partA;       // [rowsA, f]
+  int64_t rowsA, f;
+  __nv_bfloat16* dbA;
+};
+
+// out[c .. c+3] = the 16 phases' float4 partials of group g, added in order.
+__device__ __forceinline__ void bias_finish4(const float4 (&red)[16][16], int g,
+                                             __nv_bfloat16* out) {
+  float4 t = red[0][g];
+#pragma unroll
+  for (int q = 1; q < 16; ++q) {
+    const float4 v = red[q][g];
+    t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
+  }
+  __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out);
+  o[0] = __floats2bfloat162_rn(t.x, t.y);
+  o[1] = __floats2bfloat162_rn(t.z, t.w);
+}
+
+__global__ void __launch_bounds__(kBiasThreads) mlp_bias_grads(const BiasArgs a) {
+  __shared__ float4 red[16][16];
+  __shared__ float redB[32][kBiasCols];
+  __shared__ int last;
+  const int tid = static_cast<int>(threadIdx.x);
+  const int g4 = tid & 15, q = tid >> 4;  // float4 group, phase (the sums of partials)
+  if (static_cast<int>(blockIdx.x) < a.nb) {
+    const int64_t cb = blockIdx.x % a.col_blocks, ch = blockIdx.x / a.col_blocks;
+    const int g = tid & 7, p = tid >> 3;
+    const int64_t c = cb * kBiasCols + g * 8;
+    const int64_t r0 = ch * a.chunk_rows;
+    const int64_t r1 = r0 + a.chunk_rows < a.M ? r0 + a.chunk_rows : a.M;
+    float s[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    if (c < a.h) {
+#pragma unroll 4
+      for (int64_t r = r0 + p; r < r1; r += 32) {
+        const uint4 u = *reinterpret_cast<const uint4*>(a.dZ + r * a.h + c);
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(hv[i]);
+          s[2 * i] += f.x;
+          s[2 * i + 1] += f.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) redB[p][g * 8 + i] = s[i];
+    __syncthreads();
+    if (tid < kBiasCols && cb * kBiasCols + tid < a.h) {
+      float t = 0.0f;
+#pragma unroll 8
+      for (int k = 0; k < 32; ++k) t += redB[k][tid];
+      a.partB[ch * a.h + cb * kBiasCols + tid] = t;
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last = atomicAdd(a.ctr + cb, 1u) + 1u == static_cast<unsigned>(a.chunks);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    const int64_t c4 = cb * kBiasCols + g4 * 4;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (c4 < a.h) {
+#pragma unroll 4
+      for (int64_t k = q; k < a.chunks; k += 16) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(a.partB + k * a.h + c4));
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+    }
+    red[q][g4] = acc;
+    __syncthreads();
+    if (tid < 16 && c4 < a.h) bias_finish4(red, g4, a.dbB + c4);
+  } else {
+    const int64_t c4 = (static_cast<int64_t>(blockIdx.x) - a.nb) * kBiasCols + g4 * 4;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (c4 < a.f) {
+#pragma unroll 8
+      for (int64_t k = q; k < a.rowsA; k += 16) {
+        const float4 v = *reinterpret_cast<const float4*>(a.partA + k * a.f + c4);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+    }
+    red[q][g4] = acc;
+    __syncthreads();
+    if (tid < 16 && c4 < a.f) bias_finish4(red, g4, a.dbA + c4);
+  }
+}
+
 }  // namespace
+
+size_t mlp_bias_grads_scratch_bytes(int64_t M, int64_t h) {
+  const BiasPlan p = bias_plan(M, h);
+  return static_cast<size_t>(p.chunks) * static_cast<size_t>(h) * 4 +
+         static_cast<size_t>(p.col_blocks) * 4;
+}
+
+tp_status launch_mlp_bias_grads(const void* dZ, int64_t M, int64_t h, void* dbB,
+                                const float* partA, int64_t f, void* dbA, void* scratch,
+                                cudaStream_t stream) {
+  if (M <= 0 || (dbA == nullptr && dbB == nullptr)) return TP_OK;
+  if (h % 8 != 0 || f % 8 != 0) return fail(TP_ERR_ALIGN, "bias grads: widths must be multiples of 8");
+  const BiasPlan p = bias_plan(M, h);
+  BiasArgs a;
+  a.dZ = static_cast<const __nv_bfloat16*>(dZ);
+  a.M = M; a.h = h;
+  a.chunk_rows = p.chunk_rows; a.chunks = p.chunks; a.col_blocks = p.col_blocks;
+  a.nb = dbB != nullptr ? static_cast<int>(p.col_blocks * p.chunks) : 0;
+  a.partB = static_cast<float*>(scratch);
+  a.ctr = reinterpret_cast<unsigned int*>(static_cast<char*>(scratch) +
+                                          static_cast<size_t>(p.chunks) * h * 4);
+  a.dbB = static_cast<__nv_bfloat16*>(dbB);
+  a.partA = partA;
+  a.rowsA = (M + 31) / 32;
+  a.f = f;
+  a.dbA = static_cast<__nv_bfloat16*>(dbA);
+  const int na = dbA != nullptr ? static_cast<int>((f + kBiasCols - 1) / kBiasCols) : 0;
+  LaunchScope s1(TP_KIND_REDUCE, double(M) * h + double(a.rowsA) * f,
+                 2.0 * M * h + 8.0 * p.chunks * h + 4.0 * a.rowsA * f, stream);
+  cudaError_t e = cudaSuccess;
+  if (a.nb > 0) e = cudaMemsetAsync(a.ctr, 0, static_cast<size_t>(p.col_blocks) * 4, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "bias grads counters");
+  mlp_bias_grads<<<a.nb + na, kBiasThreads, 0, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "bias grads launch");
+  return TP_OK;
+}
 
 size_t colsum_scratch_bytes(int64_t rows, int64_t cols) {
   return static_cast<size_t>(colsum_plan(rows, cols).chunks) * static_cast<size_t>(cols) *

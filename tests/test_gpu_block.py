@@ -94,7 +94,12 @@ def gpu_block(w, X, dX2, b, s, f, heads, t, eps=1e-5):
     return X2, sv, dX, g
 
 
-def test_block_small_vs_oracle():
+@pytest.mark.parametrize("tile", ["auto", "192"])
+def test_block_small_vs_oracle(monkeypatch, tile):
+    """Tile 192 takes the residual epilogues through the aux rows fetched a
+    chunk ahead, across a ragged column tile and from one unit to the next."""
+    if tile != "auto":
+        monkeypatch.setenv("TP_GEMM_TILE", tile)
     b, s, h, f, heads, t = 2, 96, 256, 1024, 2, 2
     w, X, dX2 = make_block(b, s, h, f, heads, 7)
     X2, sv, dX, g = gpu_block(w, X, dX2, b, s, f, heads, t)

@@ -81,6 +81,17 @@ def test_mlp_fp32_shard_counts(t):
     compare_full(gpu_mlp(inp, t, dtype=torch.float32), inp, "f32")
 
 
+def test_mlp_bias_grads_many_row_chunks():
+    """M = 8200 rows: the bias-gradient pass takes 256-row chunks (33 of them,
+    the last ragged) and a ragged last column block of dZ (h = 264) and of
+    the dY partials (f = 544)."""
+    wl = Workload(93, "bias chunks", b=1, s=8200, h=264, f=544, t=2, w_std=0.05,
+                  bias_std=0.05)
+    inp = make_mlp_inputs(wl)
+    out = gpu_mlp(inp, wl.t)
+    compare_full(out, inp, "bf16")
+
+
 def test_mlp_config2_bf16():
     wl = WORKLOADS[2]
     inp = make_mlp_inputs(wl)
