@@ -127,6 +127,10 @@ __global__ void __launch_bounds__(kFinalWarps * 32)
 //   order (16 groups of 4 columns x 16 chunk phases, phases in order);
 // * dbA: CTAs past those add the GeLU' GEMM's per-32-row partials of dY in
 //   the same 16 x 16 arrangement.
+// 64-column blocks keep many short CTAs in flight for a narrow dZ (workload
+// 2's h = 768: 516 CTAs of 192 rows); 256-column blocks (a warp reading 512
+// contiguous bytes of a row) measured 8% faster on a 12288-wide dZ but 2%
+// slower on workload 2's MLP backward.
 // Which CTA arrives last varies; the order of every sum does not, so the
 // result is deterministic.  The counters are cleared on the stream before
 // the launch (one atomicAdd per arrival: a compare-and-swap loop retried
@@ -138,11 +142,18 @@ struct BiasPlan {
   int64_t chunk_rows, chunks, col_blocks;
 };
 
+// At most four CTAs per SM of a 148-SM B200, one wave (a fixed target, so
+// the scratch size does not depend on the device), and at most 64 row
+// chunks of a multiple of 32 rows: wide inputs get few, long chunks that
+// stream, narrow ones many short chunks.
 BiasPlan bias_plan(int64_t rows, int64_t cols) {
   BiasPlan p;
-  p.chunk_rows = 128 * ((rows + 8191) / 8192);
-  p.chunks = (rows + p.chunk_rows - 1) / p.chunk_rows;
   p.col_blocks = (cols + kBiasCols - 1) / kBiasCols;
+  int64_t want = 4 * 148 / p.col_blocks;
+  if (want > 64) want = 64;
+  if (want < 1) want = 1;
+  p.chunk_rows = ((rows + want - 1) / want + 31) / 32 * 32;
+  p.chunks = (rows + p.chunk_rows - 1) / p.chunk_rows;
   return p;
 }
 
@@ -158,13 +169,14 @@ struct BiasArgs {
   __nv_bfloat16* dbA;
 };
 
-// out[c .. c+3] = the 16 phases' float4 partials of group g, added in order.
-__device__ __forceinline__ void bias_finish4(const float4 (&red)[16][16], int g,
-                                             __nv_bfloat16* out) {
-  float4 t = red[0][g];
+// out[0..3] = the P phases' float4 partials of group g (red[q * G + g]),
+// added in phase order.
+template <int P, int G>
+__device__ __forceinline__ void bias_finish4(const float4* red, int g, __nv_bfloat16* out) {
+  float4 t = red[g];
 #pragma unroll
-  for (int q = 1; q < 16; ++q) {
-    const float4 v = red[q][g];
+  for (int q = 1; q < P; ++q) {
+    const float4 v = red[q * G + g];
     t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
   }
   __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out);
@@ -173,11 +185,10 @@ __device__ __forceinline__ void bias_finish4(const float4 (&red)[16][16], int g,
 }
 
 __global__ void __launch_bounds__(kBiasThreads) mlp_bias_grads(const BiasArgs a) {
-  __shared__ float4 red[16][16];
   __shared__ float redB[32][kBiasCols];
+  __shared__ float4 red4[256];
   __shared__ int last;
   const int tid = static_cast<int>(threadIdx.x);
-  const int g4 = tid & 15, q = tid >> 4;  // float4 group, phase (the sums of partials)
   if (static_cast<int>(blockIdx.x) < a.nb) {
     const int64_t cb = blockIdx.x % a.col_blocks, ch = blockIdx.x / a.col_blocks;
     const int g = tid & 7, p = tid >> 3;
@@ -202,9 +213,9 @@ __global__ void __launch_bounds__(kBiasThreads) mlp_bias_grads(const BiasArgs a)
     for (int i = 0; i < 8; ++i) redB[p][g * 8 + i] = s[i];
     __syncthreads();
     if (tid < kBiasCols && cb * kBiasCols + tid < a.h) {
-      float t = 0.0f;
+      float t = redB[0][tid];
 #pragma unroll 8
-      for (int k = 0; k < 32; ++k) t += redB[k][tid];
+      for (int k = 1; k < 32; ++k) t += redB[k][tid];
       a.partB[ch * a.h + cb * kBiasCols + tid] = t;
     }
     __threadfence();
@@ -213,6 +224,7 @@ __global__ void __launch_bounds__(kBiasThreads) mlp_bias_grads(const BiasArgs a)
     __syncthreads();
     if (!last) return;
     __threadfence();
+    const int g4 = tid & 15, q = tid >> 4;
     const int64_t c4 = cb * kBiasCols + g4 * 4;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     if (c4 < a.h) {
@@ -222,10 +234,11 @@ __global__ void __launch_bounds__(kBiasThreads) mlp_bias_grads(const BiasArgs a)
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
     }
-    red[q][g4] = acc;
+    red4[q * 16 + g4] = acc;
     __syncthreads();
-    if (tid < 16 && c4 < a.h) bias_finish4(red, g4, a.dbB + c4);
+    if (tid < 16 && c4 < a.h) bias_finish4<16, 16>(red4, g4, a.dbB + c4);
   } else {
+    const int g4 = tid & 15, q = tid >> 4;
     const int64_t c4 = (static_cast<int64_t>(blockIdx.x) - a.nb) * kBiasCols + g4 * 4;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     if (c4 < a.f) {
@@ -235,9 +248,9 @@ __global__ void __launch_bounds__(kBiasThreads) mlp_bias_grads(const BiasArgs a)
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
     }
-    red[q][g4] = acc;
+    red4[q * 16 + g4] = acc;
     __syncthreads();
-    if (tid < 16 && c4 < a.f) bias_finish4(red, g4, a.dbA + c4);
+    if (tid < 16 && c4 < a.f) bias_finish4<16, 16>(red4, g4, a.dbA + c4);
   }
 }
 

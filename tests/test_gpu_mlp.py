@@ -82,8 +82,8 @@ def test_mlp_fp32_shard_counts(t):
 
 
 def test_mlp_bias_grads_many_row_chunks():
-    """M = 8200 rows: the bias-gradient pass takes 256-row chunks (33 of them,
-    the last ragged) and a ragged last column block of dZ (h = 264) and of
+    """M = 8200 rows: the bias-gradient pass takes 160-row chunks (52 of them,
+    the last ragged), with a ragged last column block of dZ (h = 264) and of
     the dY partials (f = 544)."""
     wl = Workload(93, "bias chunks", b=1, s=8200, h=264, f=544, t=2, w_std=0.05,
                   bias_std=0.05)
