@@ -92,6 +92,37 @@ def test_mlp_bias_grads_many_row_chunks():
     compare_full(out, inp, "bf16")
 
 
+@pytest.mark.parametrize("which", ["dbA", "dbB"])
+@pytest.mark.parametrize("rows", [1, 3])
+def test_mlp_bias_grads_one_of_two_few_rows(rows, which):
+    """One bias gradient requested (the other pointer NULL) on 1 and 3 rows:
+    one row chunk, one partial row of dY; the other gradient is not written."""
+    wl = Workload(94, "few rows", b=1, s=rows, h=72, f=144, t=2, w_std=0.05, bias_std=0.05)
+    inp = make_mlp_inputs(wl)
+    d = {k: cuda(v) for k, v in inp.items()}
+    X, A, B = d["X"], d["A"], d["B"]
+    M, h = X.shape
+    f = A.shape[1]
+    Z = torch.empty(M, h, dtype=torch.bfloat16, device="cuda")
+    Y = torch.empty(M, f, dtype=torch.bfloat16, device="cuda")
+    L.tp_mlp_fwd(X, A, d["bA"], B, d["bB"], Z, Y, wl.t,
+                 L.workspace(L.TP_OP_MLP_FWD, M, h, f, 0, wl.t, L.TP_BF16))
+    g = {k: torch.empty_like(v) for k, v in (("dX", X), ("dA", A), ("dB", B))}
+    sentinel = 7.0
+    dbA = torch.full((f,), sentinel, dtype=torch.bfloat16, device="cuda")
+    dbB = torch.full((h,), sentinel, dtype=torch.bfloat16, device="cuda")
+    L.tp_mlp_bwd(X, A, d["bA"], B, Y, d["dZ"], g["dX"], g["dA"],
+                 dbA if which == "dbA" else None, g["dB"], dbB if which == "dbB" else None, wl.t,
+                 L.workspace(L.TP_OP_MLP_BWD, M, h, f, 0, wl.t, L.TP_BF16))
+    torch.cuda.synchronize()
+    bw = O.mlp_bwd(inp["X"], inp["A"], inp["bA"], inp["B"], inp["dZ"])
+    got, other = (dbA, dbB) if which == "dbA" else (dbB, dbA)
+    check(got, bw[which], which, "bf16")
+    assert torch.all(other.float() == sentinel), "the gradient not asked for was written"
+    for k in ("dX", "dA", "dB"):
+        check(g[k], bw[k], k, "bf16")
+
+
 def test_mlp_config2_bf16():
     wl = WORKLOADS[2]
     inp = make_mlp_inputs(wl)
