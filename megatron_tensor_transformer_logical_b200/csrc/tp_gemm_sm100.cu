@@ -72,20 +72,32 @@ struct Cfg {
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
-// Epilogues that read an operand (`aux`: Y for GeLU', the residual) fetch
-// it one 32-column chunk ahead into two more boxes per epilogue warp where
-// shared memory has room for them (BN = 192: four 40 KB stages), so the
-// fetch of the next chunk's rows overlaps the current chunk instead of
-// being waited for at the start of every chunk; elsewhere the aux rows come
-// into the output box at the start of their own chunk.
+// Shared-memory layout of a single-SM kernel: the operand ring, the epilogue
+// staging boxes, the aux boxes fetched ahead, the barriers.
+// * Epilogues that read an operand (`aux`: Y for GeLU', the residual) fetch
+//   it one 32-column chunk ahead into two more boxes per epilogue warp where
+//   shared memory has room for them (BN = 192: four 40 KB stages), so the
+//   fetch of the next chunk's rows overlaps the current chunk instead of
+//   being waited for at the start of every chunk; elsewhere the aux rows
+//   come into the output box at the start of their own chunk.
+// * Epilogues with one output and no aux need one staging box per warp; at
+//   BN = 192 the 16 KB this frees and the spare room hold a fifth 40 KB
+//   stage, so more operand bytes are in flight per SM.
 template <int BN, int EPI>
-struct AuxAhead {
-  static constexpr bool kOn = BN == 192 && (EPI == kEpiResidual || EPI == kEpiDGelu);
-  static constexpr int kBytes = kOn ? kEpiWarps * 2 * kEpiBoxBytes : 0;
-  static constexpr int kBars = kOn ? 2 * kEpiWarps : kEpiWarps;
-  static constexpr int kSmemBytes = Cfg<BN>::kSmemBytes + kBytes;
+struct Layout {
+  static constexpr bool kAux = (EPI == kEpiResidual || EPI == kEpiDGelu);
+  static constexpr bool kOut2 = (EPI == kEpiBiasGelu || EPI == kEpiDGelu);
+  static constexpr bool kAhead = BN == 192 && kAux;
+  static constexpr bool kOneBox = BN == 192 && !kAux && !kOut2;
+  static constexpr int kStages = kOneBox ? 5 : Cfg<BN>::kStages;
+  static constexpr int kBoxes = kOneBox ? 1 : 2;  // output boxes per epilogue warp
+  static constexpr int kBoxBytes = kEpiWarps * kBoxes * kEpiBoxBytes;
+  static constexpr int kAuxBytes = kAhead ? kEpiWarps * 2 * kEpiBoxBytes : 0;
+  static constexpr int kBars = kAhead ? 2 * kEpiWarps : kEpiWarps;
+  static constexpr int kSmemBytes = 1024 + kStages * (Cfg<BN>::kABytes + Cfg<BN>::kBBytes) +
+                                    kBoxBytes + kAuxBytes + kBarBytes;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-  static_assert((4 + 2 * Cfg<BN>::kStages + kBars) * 8 + 8 <= kBarBytes, "barrier area");
+  static_assert((4 + 2 * kStages + kBars) * 8 + 8 <= kBarBytes, "barrier area");
 };
 
 struct Args {
@@ -651,27 +663,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmO2,
                       const __grid_constant__ CUtensorMap tmX, const Args args) {
   using C = Cfg<BN>;
-  using AX = AuxAhead<BN, EPI>;
+  using LY = Layout<BN, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + C::kStages * C::kABytes;
-  uint8_t* sE = sB + C::kStages * C::kBBytes;  // epilogue boxes, 1024-byte aligned
-  uint8_t* sX = sE + kEpiStageBytes;           // aux boxes fetched ahead (AX::kOn)
-  uint64_t* full = reinterpret_cast<uint64_t*>(sX + AX::kBytes);
-  uint64_t* empty = full + C::kStages;
-  uint64_t* tfull = empty + C::kStages;
+  uint8_t* sB = smem + LY::kStages * C::kABytes;
+  uint8_t* sE = sB + LY::kStages * C::kBBytes;  // epilogue boxes, 1024-byte aligned
+  uint8_t* sX = sE + LY::kBoxBytes;             // aux boxes fetched ahead (LY::kAhead)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sX + LY::kAuxBytes);
+  uint64_t* empty = full + LY::kStages;
+  uint64_t* tfull = empty + LY::kStages;
   uint64_t* tempty = tfull + 2;
-  uint64_t* auxbar = tempty + 2;  // one (two with AX::kOn) per epilogue warp
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + AX::kBars);
+  uint64_t* auxbar = tempty + 2;  // one (two with LY::kAhead) per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + LY::kBars);
   int* tail_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < LY::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -679,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], kEpiWarps);
     }
-    for (int i = 0; i < AX::kBars; ++i) mbar_init(&auxbar[i], 1);
+    for (int i = 0; i < LY::kBars; ++i) mbar_init(&auxbar[i], 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -728,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < BN / 64; ++c)
               tma_load_2d(b_dst + c * (BK * 128), &tmB, &full[stage], tc.n0 + 64 * c, kc);
           }
-          if (++stage == C::kStages) {
+          if (++stage == LY::kStages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -766,7 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16(d_tmem, ad, bd, kIdesc, (kb != w.kb0 || k != 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
-          if (++stage == C::kStages) {
+          if (++stage == LY::kStages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -784,10 +796,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - kFirstEpiWarp;
     const int quarter = warp & 3;  // tensor-memory lanes this warp may read
     const int half = ew >> 2;      // which half of the tile's columns
-    uint8_t* box0 = sE + ew * (2 * kEpiBoxBytes);
-    uint8_t* box1 = box0 + kEpiBoxBytes;
+    uint8_t* box0 = sE + ew * (LY::kBoxes * kEpiBoxBytes);
+    uint8_t* box1 = box0 + (LY::kBoxes - 1) * kEpiBoxBytes;  // box0 when there is one
     uint32_t aux_phase = 0;
-    // Aux fetched ahead (AX::kOn): the chunk (unit ax_u, column offset ax_c)
+    // Aux fetched ahead (LY::kAhead): the chunk (unit ax_u, column offset ax_c)
     // whose rows are on their way into aux box ax_slot (ax_u < 0: none);
     // ax_par holds each box's wait parity.
     uint8_t* xbox = sX + ew * (2 * kEpiBoxBytes);
@@ -819,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                static_cast<uint32_t>(acc * BN + cl);
         if constexpr (OUT != kOutF32) {
           if (args.tma_out && w.part < 0 && col + 32 <= tc.n_end) {
-            if constexpr (AX::kOn) {
+            if constexpr (LY::kAhead) {
               // This chunk's aux rows: requested by the previous chunk, else now.
               const int slot = ax_slot;
               if (ax_u != u || ax_c != c) ax_fetch(slot, col, tc.m0 + quarter * 32);
@@ -883,7 +895,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // An aux fetch still in flight (only after a wait gave up): let it land
     // before the CTA's shared memory goes away.
-    if (AX::kOn && ax_u >= 0)
+    if (LY::kAhead && ax_u >= 0)
       mbar_wait(&auxbar[2 * ew + ax_slot], (ax_par >> ax_slot) & 1u, args.status,
                 kStatusEpilogueTimeout);
     if (lane == 0) bulk_wait<0>();  // this warp's TMA stores have landed
@@ -1434,7 +1446,7 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
   if (bit == 0 || !(configured.load(std::memory_order_acquire) & bit)) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             AuxAhead<BN, EPI>::kSmemBytes);
+                             Layout<BN, EPI>::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
     configured.fetch_or(bit, std::memory_order_release);
   }
@@ -1452,8 +1464,7 @@ tp_status launch_impl(const Gemm& g, cudaStream_t stream) {
                        (EPI == kEpiCE ? 8.0 * double(g.M) * g.N / 32.0 : 0.0);
   {
     LaunchScope scope(TP_KIND_GEMM_TCGEN05, flops, bytes, stream, 1, BN, g.M, g.N, g.K);
-    kern<<<grid, kThreads, AuxAhead<BN, EPI>::kSmemBytes, stream>>>(ta, tb, em.o, em.o2, em.x,
-                                                                       a);
+    kern<<<grid, kThreads, Layout<BN, EPI>::kSmemBytes, stream>>>(ta, tb, em.o, em.o2, em.x, a);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm_bf16_tcgen05 launch");

@@ -20,8 +20,11 @@ Cases (175B-shaped layer unless noted; bf16, t = 8):
   layernorm   tp_layernorm_fwd + tp_layernorm_bwd on X[8192,12288] (201 MB, larger
               than L2), gamma and beta, with a residual gradient
   mlp_bwd_bias tp_mlp_bwd with both bias gradients, M=8192, h=12288, f=1024, t=8:
-              dbB = colsum(dZ [8192,12288]) runs the two-pass column sum over 201 MB,
-              dbA the GeLU' epilogue's partials and the finishing pass
+              dbB = colsum(dZ [8192,12288], 201 MB) and dbA from the GeLU' epilogue's
+              partials, both in one launch (mlp_bias_grads)
+  mlp_small   tp_mlp_fwd + tp_mlp_bwd with biases at the GPT-2-small shape: M=8192,
+              h=768, f=3072, t=4 (K = 768 and 3072 GEMMs bound by their epilogues and
+              by L2 traffic; about 0.2 GB on the device)
   attn_bwd_big tp_attn_bwd at b=2, s=4096, h=6144 (48 heads; about 2.7 GB on the
               device): the D = rowsum(dO * O) kernel reads 2 x 100 MB
   linear_f32  tp_linear_col in fp32, X[4096,4096] @ W[4096,4096] (the CUDA-core path)
@@ -158,6 +161,21 @@ def make_case(name: str):
         dbA, dbB = torch.empty_like(bA), torch.empty_like(bB)
         wsb = L.workspace(L.TP_OP_MLP_BWD, Mb, h, fb, 0, t, L.TP_BF16)
         return lambda: L.tp_mlp_bwd(X, A, bA, B, Y, dZ, dX, dA, dbA, dB, dbB, t, wsb)
+    if name == "mlp_small":
+        Ms, hs, fs, ts = 8192, 768, 3072, 4
+        X, A, B = _t((Ms, hs), 1.0), _t((hs, fs), 0.02, seed=1), _t((fs, hs), 0.02, seed=2)
+        bA, bB = _t((fs,), 0.01, seed=5), _t((hs,), 0.01, seed=6)
+        dZ = _t((Ms, hs), 1.0, seed=3)
+        Z, Y = torch.empty(Ms, hs, dtype=bf, device="cuda"), torch.empty(Ms, fs, dtype=bf, device="cuda")
+        dX, dA, dB = torch.empty_like(X), torch.empty_like(A), torch.empty_like(B)
+        dbA, dbB = torch.empty_like(bA), torch.empty_like(bB)
+        wsf = L.workspace(L.TP_OP_MLP_FWD, Ms, hs, fs, 0, ts, L.TP_BF16)
+        wsb = L.workspace(L.TP_OP_MLP_BWD, Ms, hs, fs, 0, ts, L.TP_BF16)
+
+        def mlp_small():
+            L.tp_mlp_fwd(X, A, bA, B, bB, Z, Y, ts, wsf)
+            L.tp_mlp_bwd(X, A, bA, B, Y, dZ, dX, dA, dbA, dB, dbB, ts, wsb)
+        return mlp_small
     if name == "attn_bwd_big":
         b2, s2 = 2, 4096
         Mb = b2 * s2
