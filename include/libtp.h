@@ -25,6 +25,12 @@
  * - Each call validates its arguments on the host, synchronously, before any
  *   launch, and then enqueues its kernels on `stream` (a cudaStream_t; NULL is
  *   the legacy default stream) and returns without waiting.
+ * - Calls other than tp_device_status() and the profiling reads never
+ *   synchronise the host, so a sequence of them may be captured in a CUDA
+ *   graph and replayed (after one ordinary call of each, so one-time set-up
+ *   is done outside the capture); the graph replays the same pointers, so the
+ *   tensors and workspaces must outlive it.  Arrival counters in a workspace
+ *   are left cleared by every launch, so replays count from zero.
  * - Alignment: every pointer must be 16-byte aligned and every row length
  *   (number of columns) a multiple of 8 elements, otherwise TP_ERR_ALIGN.
  * - Shard i of a column split owns columns [i*n/t, (i+1)*n/t); shard i of a

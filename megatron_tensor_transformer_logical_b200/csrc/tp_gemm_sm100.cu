@@ -638,7 +638,9 @@ __device__ __forceinline__ void tail_finish(const Args& a, const TileCoord& tc, 
 }
 
 // After a CTA's epilogue warps stored their parts of a slice of split tile
-// ti (counter slot `slot`): the last CTA to do so for that tile finishes it.
+// ti (counter slot `slot`): the last CTA to do so for that tile finishes it
+// and clears the counter, so that a CUDA graph replaying this launch (the
+// same generation baked into its arguments) counts from zero again.
 // Called by all epilogue warps of the CTA together (named barrier 1).
 template <int TM, int TN, int EPI, int OUT>
 __device__ __forceinline__ void tail_arrive(const Args& a, const TileCoord& tc, int ti, int slot,
@@ -646,8 +648,11 @@ __device__ __forceinline__ void tail_arrive(const Args& a, const TileCoord& tc, 
                                             int* flag) {
   __threadfence();
   named_sync(1, kEpiWarps * 32);
-  if (ew == 0 && lane == 0)
-    *flag = gen_ticket(a.tail_ctr + slot, a.status.gen, a.tail_split) ? 1 : 0;
+  if (ew == 0 && lane == 0) {
+    const bool last = gen_ticket(a.tail_ctr + slot, a.status.gen, a.tail_split);
+    if (last) atomicExch(a.tail_ctr + slot, 0ull);
+    *flag = last ? 1 : 0;
+  }
   named_sync(1, kEpiWarps * 32);
   if (*reinterpret_cast<volatile int*>(flag)) {
     __threadfence();
