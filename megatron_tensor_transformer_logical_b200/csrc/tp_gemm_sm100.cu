@@ -435,25 +435,45 @@ __device__ __forceinline__ uint32_t sw64_off(int r, int j) {
   return static_cast<uint32_t>(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
 }
 
+// The bias of a warp's half tile, fetched when the tile starts (before its
+// accumulator is ready): lane l holds columns [8 l, 8 l + 8) of the half
+// (zeros past the tile's column range); a chunk takes its four groups from
+// lanes bl0 .. bl0 + 3 by shuffles, instead of four global loads whose
+// latency would open every chunk.
+template <int EPI, int HALF>
+__device__ __forceinline__ uint4 bias_half(const Args& a, int col0, int col_end, int lane) {
+  uint4 q = make_uint4(0u, 0u, 0u, 0u);
+  if (EPI != kEpiDGelu && EPI != kEpiCE && a.bias != nullptr) {
+    const int col = col0 + 8 * lane;
+    if (lane < HALF / 8 && col + 8 <= col_end)
+      q = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.bias) + col);
+  }
+  return q;
+}
+
 // The epilogue of one row's 32 consecutive columns, all inside the tile's
 // column range, written to the warp's staging boxes (row r of a box = this
 // thread's lane): abox holds the row of `aux` for the epilogues that read
-// one (it may be box0), box0 receives `out` and box1 out2.  Rows past M are
-// computed too and dropped by the TMA store.
+// one (it may be box0), box0 receives `out` and box1 out2.  The bias of the
+// columns comes from lanes bl0 .. bl0 + 3 of the warp's bias_half `bq`.
+// Rows past M are computed too and dropped by the TMA store.
 template <int EPI, int OUT>
-__device__ __forceinline__ void epilogue_box32(float (&v)[32], int r, int col0, uint8_t* box0,
+__device__ __forceinline__ void epilogue_box32(float (&v)[32], int r, uint8_t* box0,
                                                uint8_t* box1, const uint8_t* abox,
-                                               const Args& a) {
+                                               const uint4& bq, int bl0, const Args& a) {
   constexpr bool kAux = (EPI == kEpiResidual || EPI == kEpiDGelu);
   bool clamped = false;
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     float* x = v + 8 * g;
-    const int col = col0 + 8 * g;
     if (EPI != kEpiDGelu && a.bias != nullptr) {
+      uint4 b;
+      b.x = __shfl_sync(0xffffffffu, bq.x, bl0 + g);
+      b.y = __shfl_sync(0xffffffffu, bq.y, bl0 + g);
+      b.z = __shfl_sync(0xffffffffu, bq.z, bl0 + g);
+      b.w = __shfl_sync(0xffffffffu, bq.w, bl0 + g);
       float bb[8];
-      unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.bias) + col),
-              bb);
+      unpack8(b, bb);
       add8(x, bb);
     }
     float y[8];
@@ -541,7 +561,8 @@ __device__ __forceinline__ bool epilogue_chunk_boxed(uint32_t taddr, int lane, i
                                                      uint8_t* box1, uint64_t* auxbar,
                                                      uint32_t& aux_phase, const CUtensorMap* tmO,
                                                      const CUtensorMap* tmO2,
-                                                     const CUtensorMap* tmX, const Args& a) {
+                                                     const CUtensorMap* tmX, const uint4& bq,
+                                                     int bl0, const Args& a) {
   constexpr bool kAux = (EPI == kEpiResidual || EPI == kEpiDGelu);
   constexpr bool kOut2 = (EPI == kEpiBiasGelu || EPI == kEpiDGelu);
   if (lane == 0) bulk_wait_read<0>();
@@ -560,7 +581,7 @@ __device__ __forceinline__ bool epilogue_chunk_boxed(uint32_t taddr, int lane, i
   if constexpr (EPI == kEpiCE)
     epilogue_ce32(v, row, col, col_end, tg, a, box0, lane);
   else
-    epilogue_box32<EPI, OUT>(v, lane, col, box0, box1, box0, a);
+    epilogue_box32<EPI, OUT>(v, lane, box0, box1, box0, bq, bl0, a);
   epilogue_colsum<EPI>(v, row, col, col_end, lane, a);
   fence_async_smem();
   __syncwarp();
@@ -582,7 +603,8 @@ __device__ __forceinline__ bool epilogue_chunk_ahead(uint32_t taddr, int lane, i
                                                      uint8_t* box1, const uint8_t* abox,
                                                      uint64_t* abar, uint32_t aphase,
                                                      const CUtensorMap* tmO,
-                                                     const CUtensorMap* tmO2, const Args& a) {
+                                                     const CUtensorMap* tmO2, const uint4& bq,
+                                                     int bl0, const Args& a) {
   constexpr bool kOut2 = (EPI == kEpiBiasGelu || EPI == kEpiDGelu);
   if (lane == 0) bulk_wait_read<0>();
   __syncwarp();
@@ -590,7 +612,7 @@ __device__ __forceinline__ bool epilogue_chunk_ahead(uint32_t taddr, int lane, i
   tmem_ld32(taddr, v);
   const bool got = mbar_wait(abar, aphase, a.status, kStatusEpilogueTimeout);
   if (!__all_sync(0xffffffffu, got)) return false;
-  epilogue_box32<EPI, OUT>(v, lane, col, box0, box1, abox, a);
+  epilogue_box32<EPI, OUT>(v, lane, box0, box1, abox, bq, bl0, a);
   epilogue_colsum<EPI>(v, row, col, col_end, lane, a);
   fence_async_smem();
   __syncwarp();
@@ -822,6 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
       const Unit w = unit_of(u, args);
       const TileCoord tc = tile_coord<BN>(w.tile, args);
+      const uint4 bq = bias_half<EPI, BN / 2>(args, tc.n0 + half * (BN / 2), tc.n_end, lane);
       if (!mbar_wait(&tfull[acc], acc_phase, args.status, kStatusEpilogueTimeout)) break;
       tc_fence_after();
       const int lrow = quarter * 32 + lane;
@@ -864,12 +887,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = epilogue_chunk_ahead<EPI, OUT>(
                   taddr, lane, row, tc.m0 + quarter * 32, col, tc.n_end, box0, box1,
                   xbox + slot * kEpiBoxBytes, &auxbar[2 * ew + slot], (ax_par >> slot) & 1u,
-                  &tmO, &tmO2, args);
+                  &tmO, &tmO2, bq, c / 8, args);
               ax_par ^= 1u << slot;
             } else {
               ok = epilogue_chunk_boxed<EPI, OUT>(taddr, lane, row, tc.m0 + quarter * 32, col,
                                                   tc.n_end, tg, box0, box1, &auxbar[ew],
-                                                  aux_phase, &tmO, &tmO2, &tmX, args);
+                                                  aux_phase, &tmO, &tmO2, &tmX, bq, c / 8, args);
             }
             if (!ok) break;
             continue;
@@ -1108,6 +1131,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int u = cluster_id; u < args.units && ok; u += num_clusters) {
       const Unit w = unit_of(u, args);
       const TileCoord tc = tile_coord_pair(w.tile, args);
+      const uint4 bq =
+          bias_half<EPI, kPairTN / 2>(args, tc.n0 + half * (kPairTN / 2), tc.n_end, lane);
       if (!mbar_wait(&tfull[acc], acc_phase, args.status, kStatusEpilogueTimeout)) break;
       tc_fence_after();
       const int lrow = 128 * static_cast<int>(rank) + quarter * 32 + lane;
@@ -1124,7 +1149,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (args.tma_out && w.part < 0 && col + 32 <= tc.n_end) {
             ok = epilogue_chunk_boxed<EPI, OUT>(
                 taddr, lane, row, tc.m0 + 128 * static_cast<int>(rank) + quarter * 32, col,
-                tc.n_end, tg, box0, box1, &auxbar[ew], aux_phase, &tmO, &tmO2, &tmX, args);
+                tc.n_end, tg, box0, box1, &auxbar[ew], aux_phase, &tmO, &tmO2, &tmX, bq, c / 8,
+                args);
             if (!ok) break;
             continue;
           }
