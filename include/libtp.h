@@ -30,7 +30,10 @@
  *   graph and replayed (after one ordinary call of each, so one-time set-up
  *   is done outside the capture); the graph replays the same pointers, so the
  *   tensors and workspaces must outlive it.  Arrival counters in a workspace
- *   are left cleared by every launch, so replays count from zero.
+ *   are left cleared by every launch, so replays count from zero.  A replay
+ *   keeps the launch generations of its capture, so after a bounded wait of
+ *   a later launch has expired, the replays' waits give up as well until
+ *   tp_device_status() has read and cleared the record.
  * - Alignment: every pointer must be 16-byte aligned and every row length
  *   (number of columns) a multiple of 8 elements, otherwise TP_ERR_ALIGN.
  * - Shard i of a column split owns columns [i*n/t, (i+1)*n/t); shard i of a
